@@ -1,0 +1,439 @@
+#!/usr/bin/env python
+"""Benchmark of the memory-bounded KV decode step on B200.
+
+Default workload: the Qwen3-8B-shaped layer decode step (B=32, Hq=32, Hkv=8,
+d=128, budget M=4096 slots per kv head, beta = sigmoid(N(2, 1.5))). A step is
+one decode token per sequence: budget enforcement + insertion
+(kvb_evict_insert), then split-K retention-gated attention with the split
+merge fused into the same launch (kvb_decode_attn). Block compaction and the
+attention-state-memory lookup belong to other workloads (--config 5, 4).
+
+Prints ONE JSON line (rank 0). `value` is decode tokens/s of the whole job
+(one attention layer) with inputs resident in HBM; `e2e` is the same metric
+through the public API with the step's inputs copied from pinned host memory
+and the output read back every step. Every step reads > 126 MB (L2) of K/V,
+so no L2 flush is needed.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1..5] [--impl kvb|reference]
+
+For N > 1 launch with torch.distributed.run: every rank runs an independent
+replica (the path shards into independent sequences; no collective on the
+data path), timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attn tokens/s and KV-cache GB/s (% of B200 HBM peak) at budget M"
+FALLBACK_HBM_GBS = 6650.0
+
+# ncu DRAM traffic (read + write bytes per launch) of the dominant kernel, keyed by
+# (sha256 of the kernel's source file, config). Reported only while the source is
+# unchanged since the counters were taken (profiles/decode_attn_config2.md).
+MEASURED_TRAFFIC = {}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--impl", default="kvb", choices=["kvb", "reference"])
+    ap.add_argument("--splits", type=int, default=0, help="num_splits (0: the workload's default)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------------------------
+# environment
+# ----------------------------------------------------------------------------------------------
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                             device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 50 ms while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        self.device_id = None
+        try:
+            prop = torch.cuda.get_device_properties(device)
+            self.device_id = f"{prop.pci_domain_id:08X}:{prop.pci_bus_id:02X}:{prop.pci_device_id:02X}.0"
+        except Exception:
+            self.device_id = None
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu=timestamp,{self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50"]
+        if self.device_id:
+            cmd += ["-i", self.device_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.15)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 7]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def kernel_src_hash() -> str:
+    with open(os.path.join(ROOT, "memory_bounded_kv_b200", "csrc", "decode_attn.cuh"), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+# ----------------------------------------------------------------------------------------------
+# decode workloads (configs 1, 2, 3): evict+insert, then attention
+# ----------------------------------------------------------------------------------------------
+
+class DecodeBench:
+    def __init__(self, cfg: int, splits: int, rank: int):
+        from memory_bounded_kv_b200 import synth
+        from memory_bounded_kv_b200.cache import BoundedKVCache
+        import memory_bounded_kv_b200 as kvb
+        self.cfg = cfg
+        self.w = w = synth.decode_workload(cfg)
+        self.S = splits or w.splits[-1]
+        self.cache = BoundedKVCache.from_host(w.k, w.v, w.log_beta, w.pos, w.len, w.Hq, w.M, num_splits=self.S)
+        if cfg == 3:   # stream positions cap .. 131071 through budget enforcement, then draw survivors' K/V
+            blocks = (synth.CONFIG3_LOGICAL_T - w.cap) // synth.STREAM_BLOCK
+            for blk in range(blocks):
+                lbs = torch.from_numpy(synth.stream_log_beta(w, blk)).cuda()
+                base = w.cap + blk * synth.STREAM_BLOCK
+                ts = torch.arange(base, base + synth.STREAM_BLOCK, dtype=torch.int32, device="cuda")
+                ts = ts[:, None].expand(-1, w.B).contiguous()
+                for i in range(synth.STREAM_BLOCK):
+                    kvb.kvb_evict_insert(self.cache.k, self.cache.v, self.cache.log_beta, self.cache.pos,
+                                         self.cache.len, None, None, lbs[i], ts[i], w.M)
+            k, v = synth.config3_kv(w)
+            self.cache.k.copy_(torch.from_numpy(k.view(np.int16)).view(torch.bfloat16).cuda())
+            self.cache.v.copy_(torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).cuda())
+            torch.cuda.synchronize()
+        self.pool = min(w.steps, 1024)
+        inp = [w.step_inputs(s) for s in range(self.pool)]
+
+        def stack(key, dt):
+            a = np.stack([x[key] for x in inp])
+            t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
+            return t.view(dt) if a.dtype == np.uint16 else t
+
+        self.h_q = stack("q", torch.bfloat16).pin_memory()
+        self.h_kn = stack("k_new", torch.bfloat16).pin_memory()
+        self.h_vn = stack("v_new", torch.bfloat16).pin_memory()
+        self.h_lb = stack("log_beta_new", torch.float32).pin_memory()
+        self.d_q, self.d_kn, self.d_vn, self.d_lb = (x.cuda() for x in (self.h_q, self.h_kn, self.h_vn, self.h_lb))
+        self.o = torch.zeros(w.B, w.Hq, w.d, device="cuda")
+        self.lse = torch.zeros(w.B, w.Hq, device="cuda")
+        self.tokens_per_step = w.B
+        self.launches_per_step = 2
+        self.workload = f"{w.name} (config {cfg})"
+
+    def t_of(self, i: int):
+        return self.w.t0 + i
+
+    def run_device(self, first: int, count: int, events=None):
+        """Steps first .. first+count-1 with inputs resident in HBM."""
+        c, t_all = self.cache, self.t_dev
+        for i in range(first, first + count):
+            p = i % self.pool
+            t = t_all[i]
+            c.insert(self.d_kn[p], self.d_vn[p], self.d_lb[p], t)
+            if events is not None:
+                events[i - first][0].record()
+            c.attend(self.d_q[p], t, self.o, self.lse)
+            if events is not None:
+                events[i - first][1].record()
+
+    def prepare(self, total_steps: int):
+        self.t_dev = torch.tensor([[self.t_of(i)] * self.w.B for i in range(total_steps)], dtype=torch.int32,
+                                  device="cuda")
+        self.h_t = self.t_dev.cpu().pin_memory()
+        self.s_q = torch.empty_like(self.d_q[0])
+        self.s_kn = torch.empty_like(self.d_kn[0])
+        self.s_vn = torch.empty_like(self.d_vn[0])
+        self.s_lb = torch.empty_like(self.d_lb[0])
+        self.s_t = torch.empty_like(self.t_dev[0])
+        self.h_o = torch.empty(self.o.shape, dtype=torch.float32).pin_memory()
+        self.h_lse = torch.empty(self.lse.shape, dtype=torch.float32).pin_memory()
+
+    def run_e2e(self, first: int, count: int):
+        """Steps through the public API from pinned host buffers; output read back every step."""
+        c = self.cache
+        for i in range(first, first + count):
+            p = i % self.pool
+            self.s_q.copy_(self.h_q[p], non_blocking=True)
+            self.s_kn.copy_(self.h_kn[p], non_blocking=True)
+            self.s_vn.copy_(self.h_vn[p], non_blocking=True)
+            self.s_lb.copy_(self.h_lb[p], non_blocking=True)
+            self.s_t.copy_(self.h_t[i], non_blocking=True)
+            c.step(self.s_q, self.s_kn, self.s_vn, self.s_lb, self.s_t, self.o, self.lse)
+            self.h_o.copy_(self.o, non_blocking=True)
+            self.h_lse.copy_(self.lse, non_blocking=True)
+
+    def e2e_bytes(self):
+        h2d = sum(x[0].numel() * x.element_size() for x in (self.h_q, self.h_kn, self.h_vn, self.h_lb))
+        h2d += self.w.B * 4
+        d2h = self.o.numel() * 4 + self.lse.numel() * 4
+        return h2d, d2h
+
+    def attn_bytes(self):
+        """Algorithmic bytes of one attention launch: K, V (+ log beta, pos) of the cached slots,
+        q, len, t in; o (fp32), lse out."""
+        w = self.w
+        n = int(self.cache.len.sum().item())
+        per_slot = 2 * w.d * 2 + 8
+        return n * per_slot + w.B * w.Hq * w.d * 2 + w.B * w.Hkv * 4 + w.B * 4 + w.B * w.Hq * (w.d * 4 + 4)
+
+    def evict_bytes(self):
+        w = self.w
+        n = int(self.cache.len.sum().item())
+        return n * 8 + w.B * w.Hkv * (2 * w.d * 2 + 4 + 4 + 4)
+
+    def kernel_name(self):
+        return f"decode_attn_kernel<d={self.w.d},G={self.w.Hq // self.w.Hkv},bias=1> S={self.S}"
+
+    def config(self):
+        w = self.w
+        return {"workload": self.workload, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "budget_M": w.M,
+                "num_splits": self.S, "beta": "sigmoid(N(2,1.5))",
+                "l2": "no flush: every step reads > 126 MB of K/V (inputs larger than L2)",
+                "parallelism": "replicas (independent sequences per GPU)"}
+
+    def oracle_sample(self, budget_s: float = 15.0):
+        """The oracle as it stands on whole-batch decode steps from the prefill state; returns
+        (tokens/s, description)."""
+        import oracle
+        w = self.w
+        c = dict(k=w.k.copy(), v=w.v.copy(), log_beta=w.log_beta.copy(), pos=w.pos.copy(), len=w.len.copy())
+        t0 = time.perf_counter()
+        steps = 0
+        while True:
+            x = w.step_inputs(steps)
+            oracle.evict_insert(c, x["k_new"], x["v_new"], x["log_beta_new"], x["t"], w.M)
+            oracle.decode_attn(x["q"], c["k"], c["v"], c["log_beta"], c["pos"], c["len"], x["t"])
+            steps += 1
+            if time.perf_counter() - t0 > budget_s or steps >= 64:
+                break
+        dt = time.perf_counter() - t0
+        return w.B * steps / dt, f"{steps} whole-batch decode steps (B={w.B}) from the prefill state"
+
+
+# ----------------------------------------------------------------------------------------------
+# timing driver
+# ----------------------------------------------------------------------------------------------
+
+def time_region(fn, world):
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    fn()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    return e0.elapsed_time(e1)
+
+
+def run_kvb(args, world, rank, local):
+    hbm_peak, peak_kind = peaks()
+    if args.config in (1, 2, 3):
+        bench = DecodeBench(args.config, args.splits, rank)
+    elif args.config == 4:
+        from bench_extra import ASMBench
+        bench = ASMBench()
+    else:
+        from bench_extra import MementoBench
+        bench = MementoBench()
+    K, W = args.steps, args.warmup
+    if args.config == 5:
+        K, W = bench.clamp_steps(K, W)
+    bench.prepare(2 * (W + K) + 2)
+
+    # warm-up, then the device-resident timed region with per-kernel events
+    bench.run_device(0, W)
+    torch.cuda.synchronize()
+    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    ms = time_region(lambda: bench.run_device(W, K, events), world)
+    clk = clocks.stop()
+    kern_ms = [a.elapsed_time(b) for a, b in events]
+    ms = max_over_ranks(ms, world)
+    kms = max_over_ranks(statistics.mean(kern_ms), world)
+
+    tokens = bench.tokens_per_step * K * world
+    value = tokens / (ms / 1e3)
+    attn_bytes = bench.attn_bytes()
+    achieved = attn_bytes / (kms / 1e3) / 1e9
+    step_bytes = attn_bytes + bench.evict_bytes()
+    kv_gbs = step_bytes * K / (ms / 1e3) / 1e9
+
+    e2e = None
+    if not args.no_e2e and hasattr(bench, "run_e2e"):
+        bench.run_e2e(W + K, W)
+        torch.cuda.synchronize()
+        ms_e2e = max_over_ranks(time_region(lambda: bench.run_e2e(2 * W + K, K), world), world)
+        h2d, d2h = bench.e2e_bytes()
+        e2e = {"value": bench.tokens_per_step * K * world / (ms_e2e / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e / K}
+
+    src = kernel_src_hash()
+    traffic = MEASURED_TRAFFIC.get((src, args.config))
+    out = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": ms / K,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "storage_dtype": "bf16",
+        "data": "synthetic (seeded; shapes and distributions of the workload)",
+        "config": bench.config(),
+        "kv_gbs": kv_gbs,
+        "kv_frac_of_hbm_peak": kv_gbs / hbm_peak,
+        "roofline": {"bound": "hbm", "kernel": bench.kernel_name(), "achieved": achieved, "peak": hbm_peak,
+                     "unit": "GB/s", "frac": achieved / hbm_peak, "peak_source": f"{peak_kind} (hbm_gbs)",
+                     "traffic": traffic, "algorithmic_bytes_per_launch": attn_bytes,
+                     "kernel_ms_avg": kms},
+        "clocks": clk,
+        "e2e": e2e,
+        "gpu_launches": bench.launches_per_step * K,
+        "kernel_src_sha256_16": src,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and hasattr(bench, "oracle_sample"):
+        v, sample = bench.oracle_sample()
+        out["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample}
+    return out
+
+
+def run_reference(args, world, rank):
+    """The oracle as it stands, timed on the host cores, on the workload's metric (rank 0 only)."""
+    if rank != 0:
+        return None
+    import oracle
+    from memory_bounded_kv_b200 import synth
+    w = synth.decode_workload(2 if args.config not in (1, 3) else args.config)
+    nb = 1   # one sequence per step keeps --steps K --warmup W within minutes
+    c = dict(k=w.k[:nb].copy(), v=w.v[:nb].copy(), log_beta=w.log_beta[:nb].copy(), pos=w.pos[:nb].copy(),
+             len=w.len[:nb].copy())
+
+    def step(s):
+        x = w.step_inputs(s % w.steps)
+        t = np.full(nb, w.t0 + s, np.int32)
+        oracle.evict_insert(c, x["k_new"][:nb], x["v_new"][:nb], x["log_beta_new"][:nb], t, w.M)
+        oracle.decode_attn(x["q"][:nb], c["k"], c["v"], c["log_beta"], c["pos"], c["len"], t)
+
+    for s in range(args.warmup):
+        step(s)
+    t0 = time.perf_counter()
+    for s in range(args.warmup, args.warmup + args.steps):
+        step(s)
+    dt = time.perf_counter() - t0
+    value = nb * args.steps / dt
+    sample = f"{nb} of {w.B} sequences per decode step (one attention layer), steps continue from t={w.t0}"
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{w.name} (config {2 if args.config not in (1, 3) else args.config})"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        out = run_reference(args, world, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+    world, rank, local = dist_init()
+    try:
+        out = run_kvb(args, world, rank, local)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,250 @@
+/*
+ * kvb.h -- C ABI of libkvb: decode-step attention over a memory-bounded KV
+ * cache, for NVIDIA B200 (sm_100a).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every data pointer is a DEVICE pointer owned by the caller. The library
+ *   allocates nothing, keeps no pointer after a call returns and holds no
+ *   state except one device error word per GPU (see kvb_get_error).
+ * - bf16 tensors are passed as uint16_t bit patterns (IEEE bfloat16).
+ * - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *   default stream). Results are valid once the stream has reached the call.
+ * - Host-side argument checks run before any launch; a failed check returns
+ *   KVB_EINVAL and launches nothing. A launch failure returns KVB_ECUDA.
+ *   Inconsistent device data (a length above the capacity, a removal range
+ *   outside the cache, ...) cannot be seen on the host: the kernels skip the
+ *   offending row, leave it in a defined state and set a bit in the device
+ *   error word, which kvb_get_error reports as KVB_EDEVICE. No kernel traps,
+ *   asserts or spins without a bound.
+ * - "len" is the number of valid slots of a (sequence, kv head); slots
+ *   [0, len) hold the cache in slot order, slots beyond len are never read.
+ * - t[b] is the position of sequence b's current token. t[b] < 0 marks an
+ *   inactive sequence: nothing is inserted and its attention is empty.
+ *
+ * Sources (web pages) the operations follow:
+ *   [TRIM] "Cache What Lasts: Token Retention for Memory-Bounded KV Cache in
+ *          LLMs" (ICLR 2026), section 2.1.
+ *   [ASM]  "Context Memorization for Efficient Long Context Generation",
+ *          background (online-softmax identity, GQA) and core method steps 1-4.
+ *   [MEM]  "MEMENTO: Teaching LLMs to Manage Their Own Context", sections on
+ *          chunking/compression, the dual information stream and the
+ *          systems implementation.
+ */
+#ifndef KVB_H
+#define KVB_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum kvb_status {
+    KVB_OK = 0,
+    KVB_EINVAL = 1,  /* bad argument, detected on the host; nothing launched */
+    KVB_ECUDA = 2,   /* a CUDA runtime call or a launch failed */
+    KVB_EDEVICE = 3  /* a kernel met inconsistent device data (kvb_get_error) */
+} kvb_status;
+
+typedef void* kvb_stream; /* cudaStream_t */
+
+enum kvb_out_dtype { KVB_OUT_F32 = 0, KVB_OUT_BF16 = 1 };
+
+/* bits of the device error word */
+enum kvb_device_error {
+    KVB_DERR_LEN = 1u << 0,       /* len < 0 or len > cap */
+    KVB_DERR_SPLIT = 1u << 1,     /* split_len * num_splits < len */
+    KVB_DERR_RANGE = 1u << 2,     /* compaction range outside [0, len) */
+    KVB_DERR_TIMEOUT = 1u << 3    /* a bounded wait on a copy gave up */
+};
+
+/* ------------------------------------------------------------------------
+ * kvb_decode_attn -- split-K GQA decode attention with retention bias
+ *
+ * [TRIM] 2.1: the weight of cached token i in the attention of the token at
+ * position t is proportional to exp(q.k_i + (t - i) log beta_i); [ASM] step
+ * 1 adds the 1/sqrt(d_h) scale and defines the attention state (a, Z),
+ * a = softmax-weighted mean of the values, Z = sum of exp(logit). For query
+ * head h of sequence b (kv head g = h / (Hq / Hkv)) and slot s < len[b, g]:
+ *
+ *     logit_s = scale * (q . k_s) + bias_s,
+ *     bias_s  = (float)(t[b] - pos_s) * log_beta_s   (0 when log_beta == NULL)
+ *
+ * The output state is (o, lse) with o = sum_s softmax(logit)_s v_s and
+ * lse = ln sum_s exp(logit_s); an empty state is (o = 0, lse = -inf).
+ * Split j covers slots [j*C, min((j+1)*C, len)), C = split_len if
+ * split_len > 0, else ceil(len / num_splits). The splits' states are
+ * combined with the merge operator of [ASM] step 2 (see kvb_merge_states);
+ * by the online-softmax identity ([ASM] background) the result equals
+ * attention over all len slots.
+ *
+ * Layouts (element strides; the innermost dimension d is contiguous):
+ *   q        [B, Hq, d]          bf16, strides q_stride_b, q_stride_h
+ *   k, v     [B, Hkv, cap, d]    bf16, strides kv_stride_b, kv_stride_h,
+ *                                slot stride d; kv_stride_b may be 0 (one
+ *                                cache read by every row b)
+ *   log_beta [B, Hkv, cap] f32 and pos [B, Hkv, cap] int32, strides
+ *            meta_stride_b, meta_stride_h (slot stride 1); log_beta may be
+ *            NULL (beta = 1: plain attention), then pos and t may be NULL
+ *   len      [B, Hkv] int32, contiguous
+ *   t        [B] int32 (NULL: every row active, only allowed without bias)
+ *   o        [B, Hq, d] f32 or bf16 (o_dtype), contiguous
+ *   lse      [B, Hq] f32, contiguous, may be NULL
+ *   o_part   [B, Hq, num_splits, d] f32, lse_part [B, Hq, num_splits] f32:
+ *            every split's state (empty splits get (0, -inf)); required when
+ *            num_splits > 1, may be NULL when num_splits == 1
+ *   counters [B, Hkv] uint32: required when num_splits > 1. They must be
+ *            zero before the first call; every call leaves them zero. The
+ *            last split to finish for a (b, g) merges the states, so no
+ *            second launch and no waiting is needed.
+ *
+ * Requirements (else KVB_EINVAL): d in {64, 128}; Hq % Hkv == 0 and
+ * Hq / Hkv in {1, 2, 4, 8}; B, Hkv, cap >= 1; 1 <= num_splits <= 1024;
+ * split_len >= 0; q, k, v 16-byte aligned and every q/kv stride a multiple
+ * of 8 elements; scale finite (0 selects 1/sqrt(d)).
+ * Device-side checks: len in [0, cap] and len <= num_splits * split_len
+ * (when split_len > 0); a row that fails gets the empty state.
+ * Preconditions (not checked): log beta finite and <= 0, positions unique
+ * per (b, g), pos <= t.
+ * ---------------------------------------------------------------------- */
+typedef struct kvb_attn_args {
+    const uint16_t* q;
+    int64_t q_stride_b, q_stride_h;
+    const uint16_t* k;
+    const uint16_t* v;
+    int64_t kv_stride_b, kv_stride_h;
+    const float* log_beta;
+    const int32_t* pos;
+    int64_t meta_stride_b, meta_stride_h;
+    const int32_t* len;
+    const int32_t* t;
+    int32_t B, Hq, Hkv, d, cap;
+    float scale;
+    int32_t num_splits, split_len;
+    float* o_part;
+    float* lse_part;
+    uint32_t* counters;
+    void* o;
+    int32_t o_dtype;
+    float* lse;
+} kvb_attn_args;
+
+kvb_status kvb_decode_attn(const kvb_attn_args* args, kvb_stream stream);
+
+/* ------------------------------------------------------------------------
+ * kvb_merge_states -- n-way merge of attention states
+ *
+ * [ASM] step 2: merge((a_A, Z_A), (a_B, Z_B)) = ((Z_A a_A + Z_B a_B) /
+ * (Z_A + Z_B), Z_A + Z_B), applied across the n states of each row with Z
+ * carried as lse = ln Z:
+ *     m = max_j lse_j,  lse = m + ln sum_j exp(lse_j - m),
+ *     o = sum_j exp(lse_j - lse) o_j;
+ * rows whose states are all empty get (0, -inf). The identity element is
+ * (0, -inf), so external states (e.g. a stored prefix state) merge the same
+ * way.
+ *
+ * State j of row r: o_in[j*o_stride_n + r*o_stride_r + e] (e < d, f32) and
+ * lse_in[j*lse_stride_n + r*lse_stride_r]. Outputs o_out [R, d] and
+ * lse_out [R] (may be NULL), contiguous.
+ * Requirements: n >= 1, R >= 0, 1 <= d <= 1024, o_in/o_out 16-byte aligned
+ * and o strides multiples of 4 when d % 4 == 0 (else any alignment).
+ * ---------------------------------------------------------------------- */
+kvb_status kvb_merge_states(const float* o_in, const float* lse_in,
+                            int64_t o_stride_n, int64_t o_stride_r,
+                            int64_t lse_stride_n, int64_t lse_stride_r,
+                            int32_t n, int32_t R, int32_t d,
+                            float* o_out, float* lse_out, kvb_stream stream);
+
+/* ------------------------------------------------------------------------
+ * kvb_evict_insert -- budget enforcement and insertion of the new token
+ *
+ * [TRIM] 2.1, inference: when the cache exceeds the budget M the token with
+ * the lowest beta_i^(t-i) is evicted. Per (b, g), for the token at t[b]:
+ *   t[b] < 0      nothing changes, victim = -1;
+ *   len < M       the token goes to slot len, len += 1, victim = -1;
+ *   len >= M      victim = the slot with the smallest (score, pos), compared
+ *                 lexicographically, where score = (float)(t - pos) *
+ *                 log_beta as ONE float32 multiply rounded to nearest even
+ *                 (-0 counts as +0; score = 0 when log_beta is NULL, which
+ *                 makes eviction FIFO); the token overwrites that slot and
+ *                 len is unchanged.
+ * The written slot receives k_new/v_new [B, Hkv, d] (both NULL: K/V are not
+ * written, only log_beta and pos), log_beta_new [B, Hkv] (ignored when
+ * log_beta is NULL) and pos = t[b].
+ * Cache layout: k, v [B, Hkv, cap, d], log_beta, pos [B, Hkv, cap], len
+ * [B, Hkv], all contiguous. victim [B, Hkv] int32 (may be NULL).
+ * Requirements: d in [1, 1024] with d % 8 == 0 and k/v/k_new/v_new 16-byte
+ * aligned; 1 <= M <= cap. Device-side check: len in [0, cap].
+ * ---------------------------------------------------------------------- */
+kvb_status kvb_evict_insert(uint16_t* k, uint16_t* v, float* log_beta, int32_t* pos,
+                            int32_t* len, const uint16_t* k_new, const uint16_t* v_new,
+                            const float* log_beta_new, const int32_t* t,
+                            int32_t B, int32_t Hkv, int32_t d, int32_t cap, int32_t M,
+                            int32_t* victim, kvb_stream stream);
+
+/* ------------------------------------------------------------------------
+ * kvb_compact_blocks -- in-place removal of a slot range
+ *
+ * [MEM]: once a thinking block's memento is written, the block's KV entries
+ * are physically removed in place and later entries (the memento) are kept
+ * bit for bit. For every sequence b with rm_len[b] > 0 and every kv head g:
+ * slots [r0, r0 + rl) (r0 = rm_start[b], rl = rm_len[b]) are removed,
+ * slots r0 + rl .. len - 1 move to r0 .. len - rl - 1 in order with their
+ * K, V, pos (and log_beta, when not NULL) bytes unchanged, and len -= rl.
+ * Overlapping moves (more than rl slots after the range) are handled.
+ * Layout as kvb_evict_insert. A range outside [0, len) leaves that head
+ * untouched and sets KVB_DERR_RANGE.
+ * Requirements: d % 8 == 0, k/v 16-byte aligned, cap >= 1.
+ * ---------------------------------------------------------------------- */
+kvb_status kvb_compact_blocks(uint16_t* k, uint16_t* v, int32_t* pos, float* log_beta,
+                              int32_t* len, const int32_t* rm_start, const int32_t* rm_len,
+                              int32_t B, int32_t Hkv, int32_t d, int32_t cap,
+                              kvb_stream stream);
+
+/* ------------------------------------------------------------------------
+ * kvb_asm_lookup_merge -- attention-state-memory lookup and merge
+ *
+ * [ASM] steps 3-4. For query token n and head h:
+ *   c* = argmax_k cos(q[n,h], qbar[h,k]) (the lowest k among equal values;
+ *        cos = 0 when either vector has zero norm);
+ *   (o, lse) = merge((o_self, lse_self), (abar[h, c*], log_zbar[h, c*]))
+ * with the merge of kvb_merge_states; o_self/lse_self is the query's own
+ * attention state (e.g. from kvb_decode_attn).
+ * Layouts (contiguous): q [N, H, d] bf16; qbar [H, K, d] f32; abar [H, K, d]
+ * bf16; log_zbar [H, K] f32; o_self [N, H, d] f32; lse_self [N, H] f32 ->
+ * idx [N, H] int32 (may be NULL), o [N, H, d] f32, lse [N, H] f32 (may be
+ * NULL).
+ * workspace: device scratch of kvb_asm_workspace_bytes(N, H, K) bytes,
+ * 16-byte aligned, contents irrelevant on entry.
+ * Requirements: d == 128; N, H, K >= 1; all pointers 16-byte aligned.
+ * ---------------------------------------------------------------------- */
+size_t kvb_asm_workspace_bytes(int32_t N, int32_t H, int32_t K);
+
+kvb_status kvb_asm_lookup_merge(const uint16_t* q, const float* qbar, const uint16_t* abar,
+                                const float* log_zbar, const float* o_self,
+                                const float* lse_self, int32_t N, int32_t H, int32_t K,
+                                int32_t d, int32_t* idx, float* o, float* lse,
+                                void* workspace, size_t workspace_bytes, kvb_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Errors and diagnostics
+ * ---------------------------------------------------------------------- */
+
+/* Synchronizes `stream`, then reads and clears the current GPU's device
+ * error word. Returns KVB_OK, KVB_EDEVICE (with the word's bits in *bits
+ * when bits != NULL) or KVB_ECUDA. */
+kvb_status kvb_get_error(kvb_stream stream, uint32_t* bits);
+
+/* Static text for a status code. */
+const char* kvb_status_str(kvb_status s);
+
+/* Version of the ABI described by this header. */
+int32_t kvb_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVB_H */

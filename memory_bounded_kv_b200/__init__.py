@@ -1,0 +1,221 @@
+"""memory_bounded_kv_b200: decode-step attention over a memory-bounded KV cache on B200.
+
+Python binding of libkvb (include/kvb.h). Each function has the name of the C
+entry point it calls and only marshals arguments: it checks dtypes, devices
+and layouts of torch tensors, passes their device pointers and strides, and
+raises KvbError when the library returns a non-OK status. Every step of the
+path runs in the library's CUDA kernels; there is no other implementation.
+
+bf16 tensors are torch.bfloat16. Calls run on `stream` (default: torch's
+current stream) and are asynchronous.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+
+__all__ = [
+    "KvbError", "kvb_decode_attn", "kvb_merge_states", "kvb_evict_insert", "kvb_compact_blocks",
+    "kvb_asm_workspace_bytes", "kvb_asm_lookup_merge", "kvb_get_error", "kvb_abi_version",
+    "decode_workspace",
+]
+
+
+class KvbError(RuntimeError):
+    def __init__(self, status: int, where: str, bits: int = 0):
+        msg = _lib.lib().kvb_status_str(status).decode()
+        super().__init__(f"{where}: {msg} (status {status}{', device error bits %#x' % bits if bits else ''})")
+        self.status = status
+        self.bits = bits
+
+
+def _check(status: int, where: str):
+    if status != _lib.KVB_OK:
+        raise KvbError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _need(t, dtype, name, cuda=True):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if cuda and not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    return t
+
+
+def _contig(t, name):
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def kvb_abi_version() -> int:
+    return int(_lib.lib().kvb_abi_version())
+
+
+def kvb_get_error(stream=None) -> int:
+    """Synchronize `stream`, read and clear the device error word; returns its bits (0 = none)."""
+    bits = ctypes.c_uint32(0)
+    st = _lib.lib().kvb_get_error(_stream(stream), ctypes.byref(bits))
+    if st not in (_lib.KVB_OK, _lib.KVB_EDEVICE):
+        raise KvbError(st, "kvb_get_error")
+    return int(bits.value)
+
+
+def decode_workspace(B: int, Hq: int, Hkv: int, d: int, num_splits: int, device="cuda"):
+    """Zero-filled (o_part, lse_part, counters) buffers for kvb_decode_attn with num_splits > 1."""
+    o_part = torch.zeros(B, Hq, num_splits, d, dtype=torch.float32, device=device)
+    lse_part = torch.zeros(B, Hq, num_splits, dtype=torch.float32, device=device)
+    counters = torch.zeros(B, Hkv, dtype=torch.int32, device=device)
+    return o_part, lse_part, counters
+
+
+def kvb_decode_attn(q, k, v, log_beta, pos, len, t, o, lse=None, *, scale: float = 0.0,
+                    num_splits: int = 1, split_len: int = 0, o_part=None, lse_part=None, counters=None,
+                    stream=None) -> None:
+    """Split-K GQA decode attention with retention bias; see kvb_decode_attn in include/kvb.h.
+
+    q [B, Hq, d] bf16; k, v [B, Hkv, cap, d] bf16 (stride(2) == d, stride(3) == 1; an expanded
+    view with stride(0) == 0 shares one cache); log_beta [B, Hkv, cap] f32 or None; pos
+    [B, Hkv, cap] int32 (same strides as log_beta); len [B, Hkv] int32; t [B] int32 or None;
+    o [B, Hq, d] f32 or bf16; lse [B, Hq] f32 or None; o_part/lse_part/counters from
+    decode_workspace() when num_splits > 1.
+    """
+    _need(q, torch.bfloat16, "q"); _need(k, torch.bfloat16, "k"); _need(v, torch.bfloat16, "v")
+    B, Hq, d = q.shape
+    Bk, Hkv, cap, dk = k.shape
+    if dk != d or tuple(v.shape) != tuple(k.shape) or Bk != B:
+        raise ValueError("k/v must be [B, Hkv, cap, d] matching q")
+    if q.stride(2) != 1 or k.stride(3) != 1 or k.stride(2) != d or v.stride() != k.stride():
+        raise ValueError("q/k/v: innermost dim contiguous, slot stride d, k and v with equal strides")
+    _need(len, torch.int32, "len"); _contig(len, "len")
+    meta = None
+    if log_beta is not None:
+        _need(log_beta, torch.float32, "log_beta")
+        _need(pos, torch.int32, "pos")
+        if log_beta.stride() != pos.stride() or log_beta.stride(2) != 1:
+            raise ValueError("log_beta and pos need equal strides with slot stride 1")
+        _need(t, torch.int32, "t")
+        meta = log_beta
+    if t is not None:
+        _need(t, torch.int32, "t"); _contig(t, "t")
+    if o.dtype == torch.float32:
+        odt = _lib.KVB_OUT_F32
+    elif o.dtype == torch.bfloat16:
+        odt = _lib.KVB_OUT_BF16
+    else:
+        raise TypeError("o must be float32 or bfloat16")
+    _contig(o, "o")
+    if lse is not None:
+        _need(lse, torch.float32, "lse"); _contig(lse, "lse")
+    for name, x, dt in (("o_part", o_part, torch.float32), ("lse_part", lse_part, torch.float32),
+                        ("counters", counters, torch.int32)):
+        if x is not None:
+            _need(x, dt, name); _contig(x, name)
+    a = _lib.AttnArgs(
+        q=q.data_ptr(), q_stride_b=q.stride(0), q_stride_h=q.stride(1),
+        k=k.data_ptr(), v=v.data_ptr(), kv_stride_b=k.stride(0), kv_stride_h=k.stride(1),
+        log_beta=None if meta is None else log_beta.data_ptr(),
+        pos=None if pos is None else pos.data_ptr(),
+        meta_stride_b=0 if meta is None else meta.stride(0), meta_stride_h=0 if meta is None else meta.stride(1),
+        len=len.data_ptr(), t=None if t is None else t.data_ptr(),
+        B=B, Hq=Hq, Hkv=Hkv, d=d, cap=cap, scale=float(scale),
+        num_splits=int(num_splits), split_len=int(split_len),
+        o_part=None if o_part is None else o_part.data_ptr(),
+        lse_part=None if lse_part is None else lse_part.data_ptr(),
+        counters=None if counters is None else counters.data_ptr(),
+        o=o.data_ptr(), o_dtype=odt, lse=None if lse is None else lse.data_ptr())
+    _check(_lib.lib().kvb_decode_attn(ctypes.byref(a), _stream(stream)), "kvb_decode_attn")
+
+
+def kvb_merge_states(o_in, lse_in, o_out, lse_out=None, *, stream=None) -> None:
+    """Merge n attention states per row: o_in [n, R, d] f32 (d contiguous; any n/R strides),
+    lse_in [n, R] f32 -> o_out [R, d], lse_out [R]."""
+    _need(o_in, torch.float32, "o_in"); _need(lse_in, torch.float32, "lse_in")
+    _need(o_out, torch.float32, "o_out"); _contig(o_out, "o_out")
+    n, R, d = o_in.shape
+    if o_in.stride(2) != 1 or tuple(lse_in.shape) != (n, R):
+        raise ValueError("o_in [n, R, d] with d contiguous, lse_in [n, R]")
+    if lse_out is not None:
+        _need(lse_out, torch.float32, "lse_out"); _contig(lse_out, "lse_out")
+    _check(_lib.lib().kvb_merge_states(_ptr(o_in), _ptr(lse_in), o_in.stride(0), o_in.stride(1),
+                                       lse_in.stride(0), lse_in.stride(1), n, R, d, _ptr(o_out), _ptr(lse_out),
+                                       _stream(stream)), "kvb_merge_states")
+
+
+def kvb_evict_insert(k, v, log_beta, pos, len, k_new, v_new, log_beta_new, t, M: int, victim=None, *,
+                     stream=None) -> None:
+    """Budget enforcement + insertion (in place); see kvb_evict_insert in include/kvb.h.
+    k_new/v_new may both be None (only log_beta and pos are written)."""
+    for name, x in (("k", k), ("v", v)):
+        _need(x, torch.bfloat16, name); _contig(x, name)
+    _need(pos, torch.int32, "pos"); _contig(pos, "pos")
+    _need(len, torch.int32, "len"); _contig(len, "len")
+    _need(t, torch.int32, "t"); _contig(t, "t")
+    B, Hkv, cap, d = k.shape
+    if log_beta is not None:
+        _need(log_beta, torch.float32, "log_beta"); _contig(log_beta, "log_beta")
+        _need(log_beta_new, torch.float32, "log_beta_new"); _contig(log_beta_new, "log_beta_new")
+    for name, x in (("k_new", k_new), ("v_new", v_new)):
+        if x is not None:
+            _need(x, torch.bfloat16, name); _contig(x, name)
+    if victim is not None:
+        _need(victim, torch.int32, "victim"); _contig(victim, "victim")
+    _check(_lib.lib().kvb_evict_insert(_ptr(k), _ptr(v), _ptr(log_beta), _ptr(pos), _ptr(len), _ptr(k_new),
+                                       _ptr(v_new), _ptr(log_beta_new), _ptr(t), B, Hkv, d, cap, int(M),
+                                       _ptr(victim), _stream(stream)), "kvb_evict_insert")
+
+
+def kvb_compact_blocks(k, v, pos, log_beta, len, rm_start, rm_len, *, stream=None) -> None:
+    """In-place removal of slots [rm_start[b], +rm_len[b]) from every kv head of sequence b."""
+    for name, x in (("k", k), ("v", v)):
+        _need(x, torch.bfloat16, name); _contig(x, name)
+    for name, x in (("pos", pos), ("len", len), ("rm_start", rm_start), ("rm_len", rm_len)):
+        _need(x, torch.int32, name); _contig(x, name)
+    if log_beta is not None:
+        _need(log_beta, torch.float32, "log_beta"); _contig(log_beta, "log_beta")
+    B, Hkv, cap, d = k.shape
+    _check(_lib.lib().kvb_compact_blocks(_ptr(k), _ptr(v), _ptr(pos), _ptr(log_beta), _ptr(len), _ptr(rm_start),
+                                         _ptr(rm_len), B, Hkv, d, cap, _stream(stream)), "kvb_compact_blocks")
+
+
+def kvb_asm_workspace_bytes(N: int, H: int, K: int) -> int:
+    return int(_lib.lib().kvb_asm_workspace_bytes(N, H, K))
+
+
+def kvb_asm_lookup_merge(q, qbar, abar, log_zbar, o_self, lse_self, idx, o, lse, workspace, *,
+                         stream=None) -> None:
+    """Attention-state-memory lookup and merge; see kvb_asm_lookup_merge in include/kvb.h.
+    workspace: a uint8 CUDA tensor of at least kvb_asm_workspace_bytes(N, H, K) bytes."""
+    _need(q, torch.bfloat16, "q"); _need(qbar, torch.float32, "qbar"); _need(abar, torch.bfloat16, "abar")
+    _need(log_zbar, torch.float32, "log_zbar"); _need(o_self, torch.float32, "o_self")
+    _need(lse_self, torch.float32, "lse_self"); _need(o, torch.float32, "o")
+    for name, x in (("q", q), ("qbar", qbar), ("abar", abar), ("log_zbar", log_zbar), ("o_self", o_self),
+                    ("lse_self", lse_self), ("o", o), ("workspace", workspace)):
+        _contig(x, name)
+    if idx is not None:
+        _need(idx, torch.int32, "idx"); _contig(idx, "idx")
+    if lse is not None:
+        _need(lse, torch.float32, "lse"); _contig(lse, "lse")
+    N, H, d = q.shape
+    K = qbar.shape[1]
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(_lib.lib().kvb_asm_lookup_merge(_ptr(q), _ptr(qbar), _ptr(abar), _ptr(log_zbar), _ptr(o_self),
+                                           _ptr(lse_self), N, H, K, d, _ptr(idx), _ptr(o), _ptr(lse),
+                                           _ptr(workspace), nbytes, _stream(stream)), "kvb_asm_lookup_merge")

@@ -1,0 +1,72 @@
+"""ctypes declarations of the C ABI in include/kvb.h (libkvb.so, built in-tree)."""
+from __future__ import annotations
+
+import ctypes
+import os
+
+from . import _build
+
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+
+# symbols include/kvb.h declares (kept in sync by tests/test_abi.py)
+EXPORTS = (
+    "kvb_decode_attn", "kvb_merge_states", "kvb_evict_insert", "kvb_compact_blocks",
+    "kvb_asm_workspace_bytes", "kvb_asm_lookup_merge", "kvb_get_error", "kvb_status_str",
+    "kvb_abi_version",
+)
+
+KVB_OK, KVB_EINVAL, KVB_ECUDA, KVB_EDEVICE = 0, 1, 2, 3
+KVB_OUT_F32, KVB_OUT_BF16 = 0, 1
+DERR_LEN, DERR_SPLIT, DERR_RANGE, DERR_TIMEOUT = 1, 2, 4, 8
+
+
+class AttnArgs(ctypes.Structure):
+    """Mirror of struct kvb_attn_args."""
+    _fields_ = [
+        ("q", _P), ("q_stride_b", _I64), ("q_stride_h", _I64),
+        ("k", _P), ("v", _P), ("kv_stride_b", _I64), ("kv_stride_h", _I64),
+        ("log_beta", _P), ("pos", _P), ("meta_stride_b", _I64), ("meta_stride_h", _I64),
+        ("len", _P), ("t", _P),
+        ("B", _I32), ("Hq", _I32), ("Hkv", _I32), ("d", _I32), ("cap", _I32),
+        ("scale", ctypes.c_float),
+        ("num_splits", _I32), ("split_len", _I32),
+        ("o_part", _P), ("lse_part", _P), ("counters", _P),
+        ("o", _P), ("o_dtype", _I32), ("lse", _P),
+    ]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libkvb.so, building it first if it is missing or older than its sources."""
+    global _lib
+    if _lib is None:
+        path = _build.SO
+        if _build.stale():
+            try:
+                path = _build.build()
+            except Exception as e:  # no nvcc and no prebuilt library: the CUDA path is unavailable
+                raise RuntimeError(f"libkvb.so is missing and could not be built: {e}") from e
+        if not os.path.exists(path):
+            raise RuntimeError(f"libkvb.so not found at {path}")
+        L = ctypes.CDLL(path)
+        L.kvb_decode_attn.argtypes = [ctypes.POINTER(AttnArgs), _P]
+        L.kvb_merge_states.argtypes = [_P, _P, _I64, _I64, _I64, _I64, _I32, _I32, _I32, _P, _P, _P]
+        L.kvb_evict_insert.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _P, _P]
+        L.kvb_compact_blocks.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _P]
+        L.kvb_asm_workspace_bytes.argtypes = [_I32, _I32, _I32]
+        L.kvb_asm_workspace_bytes.restype = _SZ
+        L.kvb_asm_lookup_merge.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _SZ, _P]
+        L.kvb_get_error.argtypes = [_P, ctypes.POINTER(ctypes.c_uint32)]
+        L.kvb_status_str.argtypes = [_I32]
+        L.kvb_status_str.restype = ctypes.c_char_p
+        L.kvb_abi_version.argtypes = []
+        for f in ("kvb_decode_attn", "kvb_merge_states", "kvb_evict_insert", "kvb_compact_blocks",
+                  "kvb_asm_lookup_merge", "kvb_get_error", "kvb_abi_version"):
+            getattr(L, f).restype = _I32
+        _lib = L
+    return _lib

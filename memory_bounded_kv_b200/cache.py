@@ -1,0 +1,77 @@
+"""Device-resident memory-bounded KV cache of one attention layer, and its decode step.
+
+A decode step for the token at position t (per sequence) follows "Cache What
+Lasts" section 2.1 at inference time: if the cache already holds M tokens the
+token with the lowest beta_i^(t-i) is evicted and the new token takes its
+slot (kvb_evict_insert); then the token attends over the <= M cached tokens,
+itself included, with the retention-gated logits (kvb_decode_attn, split-K
+with the splits merged in the same launch).
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import kvb_compact_blocks, kvb_decode_attn, kvb_evict_insert, decode_workspace
+
+
+def _dev(a, device):
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+    return torch.from_numpy(a).to(device)
+
+
+class BoundedKVCache:
+    """K, V [B, Hkv, cap, d] bf16, log_beta [B, Hkv, cap] f32 (None: beta = 1), pos [B, Hkv, cap]
+    int32, len [B, Hkv] int32, plus the split-K workspace for `num_splits` splits."""
+
+    def __init__(self, B, Hq, Hkv, d, cap, M, num_splits=1, split_len=0, with_beta=True, device="cuda"):
+        self.B, self.Hq, self.Hkv, self.d, self.cap, self.M = B, Hq, Hkv, d, cap, M
+        self.num_splits, self.split_len = num_splits, split_len
+        self.device = device
+        self.k = torch.zeros(B, Hkv, cap, d, dtype=torch.bfloat16, device=device)
+        self.v = torch.zeros_like(self.k)
+        self.log_beta = torch.zeros(B, Hkv, cap, dtype=torch.float32, device=device) if with_beta else None
+        self.pos = torch.zeros(B, Hkv, cap, dtype=torch.int32, device=device)
+        self.len = torch.zeros(B, Hkv, dtype=torch.int32, device=device)
+        self.victim = torch.zeros(B, Hkv, dtype=torch.int32, device=device)
+        self.o_part = self.lse_part = self.counters = None
+        if num_splits > 1:
+            self.o_part, self.lse_part, self.counters = decode_workspace(B, Hq, Hkv, d, num_splits, device)
+
+    @classmethod
+    def from_host(cls, k, v, log_beta, pos, len_, Hq, M, num_splits=1, split_len=0, device="cuda"):
+        B, Hkv, cap, d = k.shape
+        c = cls(B, Hq, Hkv, d, cap, M, num_splits, split_len, log_beta is not None, device)
+        c.k.copy_(_dev(k, device))
+        c.v.copy_(_dev(v, device))
+        if log_beta is not None:
+            c.log_beta.copy_(_dev(log_beta, device))
+        c.pos.copy_(_dev(pos, device))
+        c.len.copy_(_dev(len_, device))
+        return c
+
+    def insert(self, k_new, v_new, log_beta_new, t, stream=None):
+        kvb_evict_insert(self.k, self.v, self.log_beta, self.pos, self.len, k_new, v_new,
+                         log_beta_new if self.log_beta is not None else None, t, self.M, self.victim, stream=stream)
+
+    def attend(self, q, t, o, lse=None, stream=None, use_beta=True):
+        lb = self.log_beta if use_beta else None
+        kvb_decode_attn(q, self.k, self.v, lb, self.pos, self.len, t if (lb is not None or t is not None) else None,
+                        o, lse, num_splits=self.num_splits, split_len=self.split_len, o_part=self.o_part,
+                        lse_part=self.lse_part, counters=self.counters, stream=stream)
+
+    def step(self, q, k_new, v_new, log_beta_new, t, o, lse=None, stream=None):
+        """One decode step: budget enforcement + insertion, then attention (2 launches)."""
+        self.insert(k_new, v_new, log_beta_new, t, stream)
+        self.attend(q, t, o, lse, stream)
+
+    def compact(self, rm_start, rm_len, stream=None):
+        kvb_compact_blocks(self.k, self.v, self.pos, self.log_beta, self.len, rm_start, rm_len, stream=stream)
+
+    def kv_bytes_read(self) -> int:
+        """Bytes of K, V (and log_beta, pos when the bias is on) that one attention pass reads."""
+        n = int(self.len.sum().item())
+        per_slot = 2 * self.d * 2 + (8 if self.log_beta is not None else 0)
+        return n * per_slot

@@ -1,0 +1,119 @@
+// Budget enforcement of "Cache What Lasts" section 2.1 (inference): when the
+// cache holds M tokens, the one with the lowest beta_i^(t-i) is evicted and
+// the new token takes its slot. "Lowest beta^(t-i)" is computed as the
+// lowest score (t - pos) * log beta, one float32 multiply rounded to nearest
+// even, ties to the lower position (-0 == +0), which is bit-reproducible.
+//
+// One CTA per (sequence, kv head). Each thread scans a strided share of the
+// slots keeping the best 64-bit key (order key of the score << 32 | order
+// key of the position) with its slot; a warp-shuffle argmin and a shared-
+// memory pass across warps give the victim; then the CTA writes the new row.
+#pragma once
+
+#include "common.cuh"
+
+namespace kvb {
+
+struct EvictParams {
+    uint16_t* k;
+    uint16_t* v;
+    float* lb;
+    int* pos;
+    int* len;
+    const uint16_t* k_new;
+    const uint16_t* v_new;
+    const float* lb_new;
+    const int* t;
+    int Hkv, d, cap, M;
+    int* victim;
+};
+
+__device__ __forceinline__ void argmin_merge(unsigned long long& key, int& slot, unsigned long long k2, int s2) {
+    if (k2 < key || (k2 == key && s2 < slot)) {
+        key = k2;
+        slot = s2;
+    }
+}
+
+template <int NT>
+__global__ void __launch_bounds__(NT) evict_insert_kernel(const __grid_constant__ EvictParams p) {
+    __shared__ unsigned long long s_key[NT / 32];
+    __shared__ int s_slot[NT / 32];
+    const int bg = blockIdx.x, b = bg / p.Hkv, tid = threadIdx.x;
+    const int tb = p.t[b];
+    if (tb < 0) {
+        if (tid == 0 && p.victim) p.victim[bg] = -1;
+        return;
+    }
+    const int n = p.len[bg];
+    if (n < 0 || n > p.cap) {
+        if (tid == 0) {
+            raise_error(KVB_DERR_LEN);
+            if (p.victim) p.victim[bg] = -1;
+        }
+        return;
+    }
+    int slot;
+    if (n < p.M) {
+        slot = n;
+    } else {
+        const size_t base = (size_t)bg * p.cap;
+        const int* ps = p.pos + base;
+        const float* lb = p.lb ? p.lb + base : nullptr;
+        unsigned long long best = ~0ull;
+        int best_slot = 0x7fffffff;
+#pragma unroll 4
+        for (int s = tid; s < n; s += NT) {
+            const int ps_s = ps[s];
+            const float sc = lb ? __fmul_rn(__int2float_rn(tb - ps_s), lb[s]) : 0.f;
+            const unsigned long long key =
+                ((unsigned long long)float_order_key(sc) << 32) | (unsigned)(ps_s ^ 0x80000000);
+            argmin_merge(best, best_slot, key, s);
+        }
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) {
+            const unsigned long long k2 = __shfl_xor_sync(kFull, best, m);
+            const int s2 = __shfl_xor_sync(kFull, best_slot, m);
+            argmin_merge(best, best_slot, k2, s2);
+        }
+        if ((tid & 31) == 0) {
+            s_key[tid >> 5] = best;
+            s_slot[tid >> 5] = best_slot;
+        }
+        __syncthreads();
+        if (tid < 32) {
+            best = (tid < NT / 32) ? s_key[tid] : ~0ull;
+            best_slot = (tid < NT / 32) ? s_slot[tid] : 0x7fffffff;
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) {
+                const unsigned long long k2 = __shfl_xor_sync(kFull, best, m);
+                const int s2 = __shfl_xor_sync(kFull, best_slot, m);
+                argmin_merge(best, best_slot, k2, s2);
+            }
+            if (tid == 0) s_slot[0] = best_slot;
+        }
+        __syncthreads();
+        slot = s_slot[0];
+    }
+    const size_t row = (size_t)bg * p.cap + slot;
+    if (p.k_new != nullptr) {
+        const int vecs = p.d / 8;
+        for (int i = tid; i < 2 * vecs; i += NT) {
+            if (i < vecs) {
+                reinterpret_cast<uint4*>(p.k + row * p.d)[i] =
+                    reinterpret_cast<const uint4*>(p.k_new + (size_t)bg * p.d)[i];
+            } else {
+                reinterpret_cast<uint4*>(p.v + row * p.d)[i - vecs] =
+                    reinterpret_cast<const uint4*>(p.v_new + (size_t)bg * p.d)[i - vecs];
+            }
+        }
+    }
+    if (tid == 0) {
+        if (p.lb != nullptr) p.lb[row] = p.lb_new[bg];
+        p.pos[row] = tb;
+        if (n < p.M) p.len[bg] = n + 1;
+        if (p.victim) p.victim[bg] = (n < p.M) ? -1 : slot;
+    }
+}
+
+}  // namespace kvb

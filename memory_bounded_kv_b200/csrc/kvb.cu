@@ -1,0 +1,209 @@
+// libkvb: C ABI (include/kvb.h) over the sm_100a kernels. Host code here
+// validates arguments, picks the kernel instantiation and launches it on the
+// caller's stream; it allocates nothing.
+#include <cmath>
+#include <cstdint>
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "../../include/kvb.h"
+#include "asm_lookup.cuh"
+#include "common.cuh"
+#include "compact_blocks.cuh"
+#include "decode_attn.cuh"
+#include "evict_insert.cuh"
+#include "merge_states.cuh"
+
+namespace {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline kvb_status launched() { return cudaGetLastError() == cudaSuccess ? KVB_OK : KVB_ECUDA; }
+
+// Raises a kernel's dynamic shared-memory limit once per (kernel, device):
+// later calls (e.g. inside a stream capture) make no runtime call here.
+template <typename Kern>
+kvb_status set_smem(Kern kern, size_t bytes) {
+    if (bytes <= 48 * 1024) return KVB_OK;
+    static std::mutex mu;
+    static std::map<std::pair<const void*, int>, size_t> granted;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return KVB_ECUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    size_t& g = granted[{reinterpret_cast<const void*>(kern), dev}];
+    if (g >= bytes) return KVB_OK;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
+        return KVB_ECUDA;
+    g = bytes;
+    return KVB_OK;
+}
+
+template <int D, int G, bool BIAS>
+kvb_status launch_decode(const kvb::DecodeParams& p, int B, cudaStream_t st) {
+    using SH = kvb::DecodeShape<D, G>;
+    auto kern = kvb::decode_attn_kernel<D, G, BIAS>;
+    const size_t smem = SH::smem_bytes(p.S);
+    if (set_smem(kern, smem) != KVB_OK) return KVB_ECUDA;
+    kern<<<dim3(p.S, p.Hkv, B), SH::NT, smem, st>>>(p);
+    return launched();
+}
+
+template <int D, int G>
+kvb_status dispatch_bias(const kvb::DecodeParams& p, int B, bool bias, cudaStream_t st) {
+    return bias ? launch_decode<D, G, true>(p, B, st) : launch_decode<D, G, false>(p, B, st);
+}
+
+template <int D>
+kvb_status dispatch_g(const kvb::DecodeParams& p, int B, int G, bool bias, cudaStream_t st) {
+    switch (G) {
+        case 1: return dispatch_bias<D, 1>(p, B, bias, st);
+        case 2: return dispatch_bias<D, 2>(p, B, bias, st);
+        case 4: return dispatch_bias<D, 4>(p, B, bias, st);
+        case 8: return dispatch_bias<D, 8>(p, B, bias, st);
+        default: return KVB_EINVAL;
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t kvb_abi_version(void) { return 1; }
+
+const char* kvb_status_str(kvb_status s) {
+    switch (s) {
+        case KVB_OK: return "ok";
+        case KVB_EINVAL: return "invalid argument";
+        case KVB_ECUDA: return "CUDA error";
+        case KVB_EDEVICE: return "inconsistent device data";
+        default: return "unknown status";
+    }
+}
+
+kvb_status kvb_get_error(kvb_stream stream, uint32_t* bits) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return KVB_ECUDA;
+    unsigned w = 0;
+    if (cudaMemcpyFromSymbol(&w, kvb::g_error_word, sizeof w) != cudaSuccess) return KVB_ECUDA;
+    if (bits != nullptr) *bits = w;
+    if (w == 0) return KVB_OK;
+    const unsigned zero = 0;
+    if (cudaMemcpyToSymbol(kvb::g_error_word, &zero, sizeof zero) != cudaSuccess) return KVB_ECUDA;
+    return KVB_EDEVICE;
+}
+
+kvb_status kvb_decode_attn(const kvb_attn_args* a, kvb_stream stream) {
+    if (a == nullptr) return KVB_EINVAL;
+    if (a->B < 1 || a->Hq < 1 || a->Hkv < 1 || a->cap < 1) return KVB_EINVAL;
+    if (a->d != 64 && a->d != 128) return KVB_EINVAL;
+    if (a->Hq % a->Hkv != 0) return KVB_EINVAL;
+    const int G = a->Hq / a->Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return KVB_EINVAL;
+    if (a->num_splits < 1 || a->num_splits > 1024 || a->split_len < 0) return KVB_EINVAL;
+    if (a->B > 65535 || a->Hkv > 65535) return KVB_EINVAL;
+    if (!std::isfinite(a->scale)) return KVB_EINVAL;
+    if (!a->q || !a->k || !a->v || !a->len || !a->o) return KVB_EINVAL;
+    if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v)) return KVB_EINVAL;
+    if (a->q_stride_b < 0 || a->q_stride_h < 0 || a->kv_stride_b < 0 || a->kv_stride_h < 0) return KVB_EINVAL;
+    if ((a->q_stride_b % 8) || (a->q_stride_h % 8) || (a->kv_stride_b % 8) || (a->kv_stride_h % 8)) return KVB_EINVAL;
+    const bool bias = a->log_beta != nullptr;
+    if (bias && (!a->pos || !a->t)) return KVB_EINVAL;
+    if (bias && (a->meta_stride_b < 0 || a->meta_stride_h < 0)) return KVB_EINVAL;
+    if (a->o_dtype != KVB_OUT_F32 && a->o_dtype != KVB_OUT_BF16) return KVB_EINVAL;
+    if (a->num_splits > 1 && (!a->o_part || !a->lse_part || !a->counters)) return KVB_EINVAL;
+    if ((a->o_part == nullptr) != (a->lse_part == nullptr)) return KVB_EINVAL;
+
+    kvb::DecodeParams p;
+    p.q = a->q; p.q_sb = a->q_stride_b; p.q_sh = a->q_stride_h;
+    p.k = a->k; p.v = a->v; p.kv_sb = a->kv_stride_b; p.kv_sh = a->kv_stride_h;
+    p.lb = a->log_beta; p.pos = a->pos; p.m_sb = a->meta_stride_b; p.m_sh = a->meta_stride_h;
+    p.len = a->len; p.t = a->t;
+    p.Hq = a->Hq; p.Hkv = a->Hkv; p.cap = a->cap; p.S = a->num_splits; p.split_len = a->split_len;
+    const double scale = (a->scale == 0.0f) ? 1.0 / std::sqrt((double)a->d) : (double)a->scale;
+    p.qscale = (float)(scale * 1.4426950408889634);
+    p.o_part = a->o_part; p.lse_part = a->lse_part; p.counters = a->counters;
+    p.o = a->o; p.o_bf16 = (a->o_dtype == KVB_OUT_BF16); p.lse = a->lse;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return a->d == 128 ? dispatch_g<128>(p, a->B, G, bias, st) : dispatch_g<64>(p, a->B, G, bias, st);
+}
+
+kvb_status kvb_merge_states(const float* o_in, const float* lse_in, int64_t o_stride_n, int64_t o_stride_r,
+                            int64_t lse_stride_n, int64_t lse_stride_r, int32_t n, int32_t R, int32_t d,
+                            float* o_out, float* lse_out, kvb_stream stream) {
+    if (!o_in || !lse_in || !o_out) return KVB_EINVAL;
+    if (n < 1 || R < 0 || d < 1 || d > 1024) return KVB_EINVAL;
+    if (R == 0) return KVB_OK;
+    kvb::MergeParams p{o_in, lse_in, o_stride_n, o_stride_r, lse_stride_n, lse_stride_r, n, R, d, o_out, lse_out};
+    const bool vec4 = (d % 4 == 0) && aligned16(o_in) && aligned16(o_out) && (o_stride_n % 4 == 0) &&
+                      (o_stride_r % 4 == 0);
+    const dim3 grid((R + 7) / 8);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (vec4) {
+        kvb::merge_states_kernel<true><<<grid, 256, 0, st>>>(p);
+    } else {
+        kvb::merge_states_kernel<false><<<grid, 256, 0, st>>>(p);
+    }
+    return launched();
+}
+
+kvb_status kvb_evict_insert(uint16_t* k, uint16_t* v, float* log_beta, int32_t* pos, int32_t* len,
+                            const uint16_t* k_new, const uint16_t* v_new, const float* log_beta_new,
+                            const int32_t* t, int32_t B, int32_t Hkv, int32_t d, int32_t cap, int32_t M,
+                            int32_t* victim, kvb_stream stream) {
+    if (B < 1 || Hkv < 1 || d < 8 || d > 1024 || (d % 8) || cap < 1 || M < 1 || M > cap) return KVB_EINVAL;
+    if ((long long)B * Hkv > 0x7fffffffLL) return KVB_EINVAL;
+    if (!pos || !len || !t) return KVB_EINVAL;
+    if ((k_new == nullptr) != (v_new == nullptr)) return KVB_EINVAL;
+    if (k_new && (!k || !v || !aligned16(k) || !aligned16(v) || !aligned16(k_new) || !aligned16(v_new)))
+        return KVB_EINVAL;
+    if (log_beta && !log_beta_new) return KVB_EINVAL;
+    kvb::EvictParams p{k, v, log_beta, pos, len, k_new, v_new, log_beta_new, t, Hkv, d, cap, M, victim};
+    kvb::evict_insert_kernel<256><<<B * Hkv, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    return launched();
+}
+
+kvb_status kvb_compact_blocks(uint16_t* k, uint16_t* v, int32_t* pos, float* log_beta, int32_t* len,
+                              const int32_t* rm_start, const int32_t* rm_len, int32_t B, int32_t Hkv,
+                              int32_t d, int32_t cap, kvb_stream stream) {
+    if (B < 1 || Hkv < 1 || d < 8 || d > 1024 || (d % 8) || cap < 1) return KVB_EINVAL;
+    if ((long long)B * Hkv > 0x7fffffffLL) return KVB_EINVAL;
+    if (!k || !v || !pos || !len || !rm_start || !rm_len) return KVB_EINVAL;
+    if (!aligned16(k) || !aligned16(v)) return KVB_EINVAL;
+    const int row_bytes = 2 * d * 2 + 8;
+    int W = 32768 / row_bytes;
+    W = W < 1 ? 1 : (W > 64 ? 64 : W);
+    kvb::CompactParams p{k, v, pos, log_beta, len, rm_start, rm_len, Hkv, d, cap, W};
+    const size_t smem = (size_t)W * row_bytes;
+    kvb::compact_blocks_kernel<256><<<B * Hkv, 256, smem, static_cast<cudaStream_t>(stream)>>>(p);
+    return launched();
+}
+
+size_t kvb_asm_workspace_bytes(int32_t N, int32_t H, int32_t K) {
+    if (N < 1 || H < 1 || K < 1) return 0;
+    return (size_t)kvb::asm_ksplit(K) * N * H * sizeof(unsigned long long);
+}
+
+kvb_status kvb_asm_lookup_merge(const uint16_t* q, const float* qbar, const uint16_t* abar, const float* log_zbar,
+                                const float* o_self, const float* lse_self, int32_t N, int32_t H, int32_t K,
+                                int32_t d, int32_t* idx, float* o, float* lse, void* workspace,
+                                size_t workspace_bytes, kvb_stream stream) {
+    if (d != kvb::kAsmD || N < 1 || H < 1 || K < 1 || H > 65535) return KVB_EINVAL;
+    if (!q || !qbar || !abar || !log_zbar || !o_self || !lse_self || !o || !workspace) return KVB_EINVAL;
+    if (!aligned16(q) || !aligned16(qbar) || !aligned16(abar) || !aligned16(o_self) || !aligned16(o) ||
+        !aligned16(workspace))
+        return KVB_EINVAL;
+    if (workspace_bytes < kvb_asm_workspace_bytes(N, H, K)) return KVB_EINVAL;
+    const int qtiles = (N + kvb::kAsmQT - 1) / kvb::kAsmQT;
+    if (qtiles > 65535) return KVB_EINVAL;
+    kvb::AsmParams p{q, qbar, abar, log_zbar, o_self, lse_self, N, H, K, kvb::asm_ksplit(K), kvb::asm_kchunk(K),
+                     idx, o, lse, static_cast<unsigned long long*>(workspace)};
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (set_smem(kvb::asm_score_kernel, kvb::kAsmSmem) != KVB_OK) return KVB_ECUDA;
+    kvb::asm_score_kernel<<<dim3(H, qtiles, p.ksplit), kvb::kAsmNT, kvb::kAsmSmem, st>>>(p);
+    if (launched() != KVB_OK) return KVB_ECUDA;
+    const long long rows = (long long)N * H;
+    kvb::asm_merge_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p);
+    return launched();
+}
+
+}  // extern "C"

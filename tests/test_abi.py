@@ -1,0 +1,85 @@
+"""The C-ABI library builds for sm_100a, loads, and exports every entry point
+include/kvb.h declares; host-side argument checks reject bad arguments before
+any launch (these calls need no GPU: nothing reaches the device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from memory_bounded_kv_b200 import _lib, _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kvb.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kvb_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_functions() == sorted(_lib.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    L = _lib.lib()
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    out = os.popen(f"nm -D --defined-only {_build.SO}").read()
+    for name in declared_functions():
+        assert re.search(rf"\bT {name}\b", out), name
+
+
+def test_attn_args_struct_matches_header():
+    src = open(HEADER).read()
+    body = re.search(r"typedef struct kvb_attn_args \{(.*?)\} kvb_attn_args;", src, re.S).group(1)
+    names = []
+    for decl in body.split(";"):
+        decl = decl.strip()
+        if not decl:
+            continue
+        decl = re.sub(r"^(const\s+)?\w+\s*\**\s*", "", decl)
+        names += [n.strip().lstrip("*") for n in decl.split(",")]
+    assert names == [f[0] for f in _lib.AttnArgs._fields_]
+
+
+def test_status_strings_and_version():
+    L = _lib.lib()
+    assert L.kvb_abi_version() == 1
+    assert L.kvb_status_str(0) == b"ok"
+    assert L.kvb_status_str(1) == b"invalid argument"
+
+
+def _args(**kw):
+    fake = 1 << 20  # a 16-byte aligned non-null value; the host checks never dereference it
+    a = dict(q=fake, q_stride_b=32 * 128, q_stride_h=128, k=fake, v=fake, kv_stride_b=8 * 64 * 128,
+             kv_stride_h=64 * 128, log_beta=None, pos=None, meta_stride_b=0, meta_stride_h=0, len=fake, t=None,
+             B=2, Hq=32, Hkv=8, d=128, cap=64, scale=0.0, num_splits=1, split_len=0, o_part=None, lse_part=None,
+             counters=None, o=fake, o_dtype=0, lse=None)
+    a.update(kw)
+    return _lib.AttnArgs(**a)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(d=96), dict(Hq=12), dict(Hq=48, Hkv=3), dict(num_splits=0), dict(num_splits=2),
+    dict(q=(1 << 20) + 2), dict(kv_stride_h=100), dict(log_beta=1 << 20), dict(o_dtype=5),
+    dict(scale=float("nan")), dict(B=0), dict(split_len=-1), dict(q=None),
+])
+def test_decode_attn_rejects_bad_arguments_on_the_host(bad):
+    L = _lib.lib()
+    assert L.kvb_decode_attn(ctypes.byref(_args(**bad)), None) == _lib.KVB_EINVAL
+
+
+def test_other_entry_points_reject_bad_arguments_on_the_host():
+    L = _lib.lib()
+    f = ctypes.c_void_p(1 << 20)
+    assert L.kvb_evict_insert(f, f, None, f, f, f, f, None, f, 1, 1, 128, 64, 65, None, None) == _lib.KVB_EINVAL
+    assert L.kvb_evict_insert(f, f, None, f, f, f, None, None, f, 1, 1, 128, 64, 8, None, None) == _lib.KVB_EINVAL
+    assert L.kvb_compact_blocks(f, f, f, None, f, f, f, 1, 1, 12, 64, None) == _lib.KVB_EINVAL
+    assert L.kvb_merge_states(f, f, 1, 1, 1, 1, 0, 4, 8, f, None, None) == _lib.KVB_EINVAL
+    assert L.kvb_asm_lookup_merge(f, f, f, f, f, f, 4, 2, 16, 64, None, f, None, f, 1 << 20, None) == _lib.KVB_EINVAL
+    ws = L.kvb_asm_workspace_bytes(256, 32, 4096)
+    assert ws == 8 * 256 * 32 * 8
+    assert L.kvb_asm_lookup_merge(f, f, f, f, f, f, 256, 32, 4096, 128, None, f, None, f, ws - 1, None) == _lib.KVB_EINVAL
