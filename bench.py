@@ -288,6 +288,177 @@ class DecodeBench:
 
 
 # ----------------------------------------------------------------------------------------------
+# config 4: attention-state-memory lookup (self attention + lookup/merge per step)
+# ----------------------------------------------------------------------------------------------
+
+def _dev(a):
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(a).cuda()
+
+
+class ASMBench:
+    """A step: the 256 query tokens' causal self attention over the shared 2048-token cache
+    (kvb_decode_attn, batch stride 0) and the memory lookup + merge (kvb_asm_lookup_merge)."""
+
+    FP32_PEAK_NOTE = "148 SMs x 128 FP32 FMA/clk x 2 flop x 1.965 GHz (max SM clock) = 74.4 TFLOP/s"
+
+    def __init__(self, splits: int = 0):
+        import memory_bounded_kv_b200 as kvb
+        from memory_bounded_kv_b200 import synth
+        self.kvb = kvb
+        self.w = w = synth.asm_workload()
+        self.S = splits or 4
+        N, H, Hkv, d = w.N, w.H, w.Hkv, w.d
+        self.k = _dev(w.k).expand(N, Hkv, w.L, d)
+        self.v = _dev(w.v).expand(N, Hkv, w.L, d)
+        self.pos = _dev(w.pos).expand(N, Hkv, w.L)
+        self.len, self.t = _dev(w.len), _dev(w.t)
+        self.h_q = torch.from_numpy(w.q.view(np.int16)).view(torch.bfloat16).pin_memory()
+        self.q = self.h_q.cuda()
+        self.qbar, self.abar, self.lz = _dev(w.qbar), _dev(w.abar), _dev(w.log_zbar)
+        self.o_self = torch.zeros(N, H, d, device="cuda")
+        self.l_self = torch.zeros(N, H, device="cuda")
+        self.op, self.lp, self.cnt = kvb.decode_workspace(N, H, Hkv, d, self.S)
+        self.idx = torch.zeros(N, H, dtype=torch.int32, device="cuda")
+        self.o = torch.zeros(N, H, d, device="cuda")
+        self.lse = torch.zeros(N, H, device="cuda")
+        self.ws = torch.empty(kvb.kvb_asm_workspace_bytes(N, H, w.K), dtype=torch.uint8, device="cuda")
+        self.tokens_per_step = N
+        self.launches_per_step = 3
+        self.workload = "attention-state memory H32 K4096 d128, 256 queries, self attention over 2048 (config 4)"
+
+    def prepare(self, total_steps):
+        self.s_q = torch.empty_like(self.q)
+        self.h_o = torch.empty(self.o.shape, dtype=torch.float32).pin_memory()
+        self.h_idx = torch.empty(self.idx.shape, dtype=torch.int32).pin_memory()
+
+    def _step(self, q, events=None, j=0):
+        kvb = self.kvb
+        kvb.kvb_decode_attn(q, self.k, self.v, None, self.pos, self.len, self.t, self.o_self, self.l_self,
+                            num_splits=self.S, o_part=self.op, lse_part=self.lp, counters=self.cnt)
+        if events is not None:
+            events[j][0].record()
+        kvb.kvb_asm_lookup_merge(q, self.qbar, self.abar, self.lz, self.o_self, self.l_self, self.idx, self.o,
+                                 self.lse, self.ws)
+        if events is not None:
+            events[j][1].record()
+
+    def run_device(self, first, count, events=None):
+        for j in range(count):
+            self._step(self.q, events, j)
+
+    def run_e2e(self, first, count):
+        for _ in range(count):
+            self.s_q.copy_(self.h_q, non_blocking=True)
+            self._step(self.s_q)
+            self.h_o.copy_(self.o, non_blocking=True)
+            self.h_idx.copy_(self.idx, non_blocking=True)
+
+    def e2e_bytes(self):
+        return self.h_q.numel() * 2, self.o.numel() * 4 + self.idx.numel() * 4
+
+    def attn_bytes(self):
+        return 0
+
+    def evict_bytes(self):
+        w = self.w
+        kv = int(w.len.sum()) * w.d * 2 * 2
+        return kv + w.H * w.K * w.d * 4
+
+    def flops(self):
+        w = self.w
+        return 2.0 * w.N * w.H * w.K * w.d
+
+    def kernel_name(self):
+        return "asm_score_kernel + asm_merge_kernel (kvb_asm_lookup_merge)"
+
+    def config(self):
+        w = self.w
+        return {"workload": self.workload, "N": w.N, "H": w.H, "Hkv": w.Hkv, "K": w.K, "d": w.d, "L": w.L,
+                "self_attn_splits": self.S, "l2": "qbar (64 MiB) + abar (32 MiB) per step; no flush",
+                "parallelism": "replicas"}
+
+
+# ----------------------------------------------------------------------------------------------
+# config 5: memento-style block compaction (sawtooth cache)
+# ----------------------------------------------------------------------------------------------
+
+class MementoBench:
+    """A step: every active sequence decodes one token (append, attention); after the last
+    token of a memento, the finished block's slots are removed in place (kvb_compact_blocks)."""
+
+    SPLIT_LEN = 512
+
+    def __init__(self, splits: int = 0):
+        from memory_bounded_kv_b200 import synth
+        from memory_bounded_kv_b200.cache import BoundedKVCache
+        self.w = w = synth.memento_workload()
+        self.S = -(-w.cap // self.SPLIT_LEN)
+        self.cache = BoundedKVCache(w.B, w.Hq, w.Hkv, w.d, w.cap, w.cap, num_splits=self.S,
+                                    split_len=self.SPLIT_LEN, with_beta=False)
+        pool = [w.step_inputs(s) for s in range(w.pool)]
+        self.q = [_dev(x["q"]) for x in pool]
+        self.kn = [_dev(x["k_new"]) for x in pool]
+        self.vn = [_dev(x["v_new"]) for x in pool]
+        self.o = torch.zeros(w.B, w.Hq, w.d, device="cuda")
+        self.lse = torch.zeros(w.B, w.Hq, device="cuda")
+        self.comp = {}
+        for s in w.compaction_steps().tolist():
+            rs, rl = w.compaction(s)
+            self.comp[s] = (_dev(rs), _dev(rl))
+        self.active = np.array([(s < w.total).sum() for s in range(w.steps)], np.int64)
+        self.lens = None
+        self.tokens_per_step = None
+        self.launches_per_step = None
+        self.workload = "memento compaction B64 Hq32 Hkv8 d128, 9 x (Geom(1500) block + U[120,180] memento) (config 5)"
+
+    def clamp_steps(self, K, W):
+        W = min(W, self.w.steps // 4)
+        K = min(K, self.w.steps - W) if K > 0 else self.w.steps - W
+        return K, W
+
+    def prepare(self, total_steps):
+        w = self.w
+        steps = np.arange(w.steps)
+        self.t_dev = torch.from_numpy(np.where(steps[:, None] < w.total[None, :], steps[:, None], -1)
+                                      .astype(np.int32)).cuda()
+
+    def run_device(self, first, count, events=None):
+        c, w = self.cache, self.w
+        for j, i in enumerate(range(first, min(first + count, w.steps))):
+            p = i % w.pool
+            t = self.t_dev[i]
+            c.insert(self.kn[p], self.vn[p], None, t)
+            if events is not None:
+                events[j][0].record()
+            c.attend(self.q[p], t, self.o, self.lse)
+            if events is not None:
+                events[j][1].record()
+            if i in self.comp:
+                c.compact(*self.comp[i])
+
+    def tokens(self, first, count):
+        return int(self.active[first:first + count].sum())
+
+    def launches(self, first, count):
+        return 2 * count + sum(1 for i in range(first, first + count) if i in self.comp)
+
+    def mean_kv_bytes(self, first, count):
+        w = self.w
+        tot = 0
+        for i in range(first, first + count):
+            tot += int(w.cache_len(i)[i < w.total].sum())
+        return tot * w.Hkv * (2 * w.d * 2) / count
+
+    def config(self):
+        w = self.w
+        return {"workload": self.workload, "B": w.B, "cap": w.cap, "split_len": self.SPLIT_LEN,
+                "num_splits": self.S, "schedule_steps": w.steps, "parallelism": "replicas"}
+
+
+# ----------------------------------------------------------------------------------------------
 # timing driver
 # ----------------------------------------------------------------------------------------------
 
@@ -309,17 +480,15 @@ def run_kvb(args, world, rank, local):
     if args.config in (1, 2, 3):
         bench = DecodeBench(args.config, args.splits, rank)
     elif args.config == 4:
-        from bench_extra import ASMBench
-        bench = ASMBench()
+        bench = ASMBench(args.splits)
     else:
-        from bench_extra import MementoBench
-        bench = MementoBench()
+        bench = MementoBench(args.splits)
     K, W = args.steps, args.warmup
-    if args.config == 5:
+    if hasattr(bench, "clamp_steps"):
         K, W = bench.clamp_steps(K, W)
     bench.prepare(2 * (W + K) + 2)
 
-    # warm-up, then the device-resident timed region with per-kernel events
+    # warm-up, then the device-resident timed region with events around the dominant kernel
     bench.run_device(0, W)
     torch.cuda.synchronize()
     events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
@@ -331,11 +500,26 @@ def run_kvb(args, world, rank, local):
     ms = max_over_ranks(ms, world)
     kms = max_over_ranks(statistics.mean(kern_ms), world)
 
-    tokens = bench.tokens_per_step * K * world
+    tokens = (bench.tokens(W, K) if hasattr(bench, "tokens") else bench.tokens_per_step * K) * world
+    launches = bench.launches(W, K) if hasattr(bench, "launches") else bench.launches_per_step * K
     value = tokens / (ms / 1e3)
-    attn_bytes = bench.attn_bytes()
-    achieved = attn_bytes / (kms / 1e3) / 1e9
-    step_bytes = attn_bytes + bench.evict_bytes()
+    src = kernel_src_hash()
+    if hasattr(bench, "flops"):      # attention-state-memory lookup: fp32 ALU bound
+        peak_tf = 148 * 128 * 2 * 1.965e9 / 1e12
+        achieved = bench.flops() / (kms / 1e3) / 1e12
+        roofline = {"bound": "alu", "kernel": bench.kernel_name(), "achieved": achieved, "peak": peak_tf,
+                    "unit": "TFLOP/s", "frac": achieved / peak_tf, "peak_source": ASMBench.FP32_PEAK_NOTE,
+                    "traffic": None, "algorithmic_flops_per_launch": bench.flops(), "kernel_ms_avg": kms}
+        step_bytes = bench.evict_bytes()
+    else:
+        attn_bytes = bench.mean_kv_bytes(W, K) if hasattr(bench, "mean_kv_bytes") else bench.attn_bytes()
+        achieved = attn_bytes / (kms / 1e3) / 1e9
+        name = bench.kernel_name() if hasattr(bench, "kernel_name") else "decode_attn_kernel<128,4,plain>"
+        roofline = {"bound": "hbm", "kernel": name, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": achieved / hbm_peak, "peak_source": f"{peak_kind} (hbm_gbs)",
+                    "traffic": MEASURED_TRAFFIC.get((src, args.config)),
+                    "algorithmic_bytes_per_launch": attn_bytes, "kernel_ms_avg": kms}
+        step_bytes = attn_bytes + (bench.evict_bytes() if hasattr(bench, "evict_bytes") else 0)
     kv_gbs = step_bytes * K / (ms / 1e3) / 1e9
 
     e2e = None
@@ -347,8 +531,6 @@ def run_kvb(args, world, rank, local):
         e2e = {"value": bench.tokens_per_step * K * world / (ms_e2e / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e / K}
 
-    src = kernel_src_hash()
-    traffic = MEASURED_TRAFFIC.get((src, args.config))
     out = {
         "metric": METRIC,
         "value": value,
@@ -366,13 +548,10 @@ def run_kvb(args, world, rank, local):
         "config": bench.config(),
         "kv_gbs": kv_gbs,
         "kv_frac_of_hbm_peak": kv_gbs / hbm_peak,
-        "roofline": {"bound": "hbm", "kernel": bench.kernel_name(), "achieved": achieved, "peak": hbm_peak,
-                     "unit": "GB/s", "frac": achieved / hbm_peak, "peak_source": f"{peak_kind} (hbm_gbs)",
-                     "traffic": traffic, "algorithmic_bytes_per_launch": attn_bytes,
-                     "kernel_ms_avg": kms},
+        "roofline": roofline,
         "clocks": clk,
         "e2e": e2e,
-        "gpu_launches": bench.launches_per_step * K,
+        "gpu_launches": launches,
         "kernel_src_sha256_16": src,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline and hasattr(bench, "oracle_sample"):

@@ -164,14 +164,14 @@ __global__ void __launch_bounds__(256) asm_merge_kernel(const __grid_constant__ 
     }
     const int k = (int)(0xffffffffu - (unsigned)(best & 0xffffffffull));
     if (lane == 0 && p.idx != nullptr) p.idx[nh] = k;
-    const float ls = p.lse_self[nh] * kLog2e;
-    const float lm = p.lz[(size_t)h * p.K + k] * kLog2e;
+    const float ls = p.lse_self[nh];
+    const float lm = p.lz[(size_t)h * p.K + k];
     const float mx = fmaxf(ls, lm);
     const float mu = (mx == -INFINITY) ? 0.f : mx;
-    const float ws = exp2f(ls - mu), wm = exp2f(lm - mu);
+    const float ws = exp2f((ls - mu) * kLog2e), wm = exp2f((lm - mu) * kLog2e);
     const float tot = ws + wm;
     const float inv = (tot > 0.f) ? 1.f / tot : 0.f;
-    if (lane == 0 && p.lse != nullptr) p.lse[nh] = (tot > 0.f) ? (mx + log2f(tot)) * kLn2 : -INFINITY;
+    if (lane == 0 && p.lse != nullptr) p.lse[nh] = (tot > 0.f) ? mx + log2f(tot) * kLn2 : -INFINITY;
     const float4 os = *reinterpret_cast<const float4*>(p.o_self + nh * kAsmD + lane * 4);
     const uint2 am = *reinterpret_cast<const uint2*>(p.abar + ((size_t)h * p.K + k) * kAsmD + lane * 4);
     float4 r;

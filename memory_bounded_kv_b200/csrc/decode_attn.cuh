@@ -15,7 +15,8 @@
 //    heads in registers; the LPK partial dots of KPG keys x G heads are
 //    finished with a reduce-scatter over the group (log2(LPK) shuffle
 //    steps), after which each lane holds one (key, head) logit.
-//  - Online softmax per warp and head in the exp2 domain; p goes to shared
+//  - Online softmax per warp and head (maxima in natural units, exp2 of
+//    scaled differences); p goes to shared
 //    memory and is read back as a broadcast for PV, where each lane
 //    accumulates 8 dims x G heads of the output over its group's keys.
 //  - Epilogue: warps combine through shared memory into the split's state.
@@ -37,7 +38,7 @@ struct DecodeParams {
     const int* len;
     const int* t;
     int Hq, Hkv, cap, S, split_len;
-    float qscale;  // scale * log2(e)
+    float qscale;  // the logit scale (1/sqrt(d) unless given)
     float* o_part;
     float* lse_part;
     unsigned* counters;
@@ -60,8 +61,12 @@ struct DecodeShape {
     static constexpr int STAGE_BYTES = 2 * TILE_ELEMS * 2;  // K and V tile, bf16
     static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
     static constexpr int EPI_BYTES = NW * G * (D + 2) * 4;  // epilogue reuses the ring
-    // fixed area in front of the ring: mbarriers, flag, bias [2][T], p [NW][32]
-    static constexpr int FIXED_BYTES = ((STAGES * 8 + 16 + 2 * T * 4 + NW * 32 * 4) + 127) / 128 * 128;
+    // fixed area in front of the ring: mbarriers at 0, flag at 64, bias [2][T] at 128,
+    // p [NW][32] after it (16-byte aligned: it is read back as float2/float4)
+    static constexpr int BIAS_OFF = 128;
+    static constexpr int P_OFF = BIAS_OFF + 2 * T * 4;
+    static constexpr int FIXED_BYTES = ((P_OFF + NW * 32 * 4) + 127) / 128 * 128;
+    static_assert(STAGES * 8 <= 64 && P_OFF % 16 == 0, "fixed-area layout");
     static_assert(LPK % G == 0, "G must divide d/8");
     static_assert(EPI_BYTES <= RING_BYTES, "epilogue must fit in the ring");
     // dynamic shared memory for S splits: the merge of S states needs G*(S+2) floats
@@ -113,9 +118,9 @@ __global__ void __launch_bounds__(DecodeShape<D, G>::NT)
 
     extern __shared__ __align__(128) unsigned char smem_raw[];
     uint64_t* s_bar = reinterpret_cast<uint64_t*>(smem_raw);                 // [ST]
-    int* s_flag = reinterpret_cast<int*>(smem_raw + ST * 8);
-    float* s_bias = reinterpret_cast<float*>(smem_raw + ST * 8 + 16);        // [2][T]
-    float* s_p = s_bias + 2 * T;                                            // [NW][32]
+    int* s_flag = reinterpret_cast<int*>(smem_raw + 64);
+    float* s_bias = reinterpret_cast<float*>(smem_raw + SH::BIAS_OFF);      // [2][T]
+    float* s_p = reinterpret_cast<float*>(smem_raw + SH::P_OFF);            // [NW][32]
     unsigned char* smem = smem_raw + SH::FIXED_BYTES;                        // ring / epilogue / merge
     uint16_t* s_ring = reinterpret_cast<uint16_t*>(smem);
 
@@ -147,10 +152,10 @@ __global__ void __launch_bounds__(DecodeShape<D, G>::NT)
     const float* glb = BIAS ? p.lb + m_off : nullptr;
     const int* gpos = BIAS ? p.pos + m_off : nullptr;
 
-    auto bias_of = [&](int key) -> float {  // log2-domain bias, -inf beyond the split
+    auto bias_of = [&](int key) -> float {  // (t - pos) * log beta, -inf beyond the split
         if (key >= nk) return -INFINITY;
         if constexpr (BIAS) {
-            return __fmul_rn(__int2float_rn(tb - gpos[key]), glb[key]) * kLog2e;
+            return __fmul_rn(__int2float_rn(tb - gpos[key]), glb[key]);
         } else {
             return 0.f;
         }
@@ -176,7 +181,7 @@ __global__ void __launch_bounds__(DecodeShape<D, G>::NT)
         for (int i = 0; i < min(ST, ntiles); ++i) issue(i);
     }
 
-    // q for my 8 dims, all G heads, pre-scaled into the log2 domain
+    // q for my 8 dims, all G heads, pre-multiplied by the logit scale
     float qf[G][8];
 #pragma unroll
     for (int hh = 0; hh < G; ++hh) {
@@ -246,8 +251,9 @@ __global__ void __launch_bounds__(DecodeShape<D, G>::NT)
         for (int m = G; m < 32; m <<= 1) tmax = fmaxf(tmax, __shfl_xor_sync(kFull, tmax, m));
         const float m_new = fmaxf(m_run, tmax);
         const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-        const float alpha = exp2f(m_run - m_use);
-        const float pv = exp2f(x - m_use);
+        // logits and maxima stay in natural units; only differences are scaled by log2(e)
+        const float alpha = exp2f((m_run - m_use) * kLog2e);
+        const float pv = exp2f((x - m_use) * kLog2e);
         l_run = fmaf(l_run, alpha, pv);
         m_run = m_new;
         if (__any_sync(kFull, alpha != 1.f)) {
@@ -325,12 +331,12 @@ __global__ void __launch_bounds__(DecodeShape<D, G>::NT)
         float L = 0.f, O = 0.f;
 #pragma unroll
         for (int w = 0; w < NW; ++w) {
-            const float f = exp2f(s_ml[(w * G + hh) * 2] - Mu);
+            const float f = exp2f((s_ml[(w * G + hh) * 2] - Mu) * kLog2e);
             L = fmaf(f, s_ml[(w * G + hh) * 2 + 1], L);
             O = fmaf(f, s_o[(w * G + hh) * D + e], O);
         }
         const float out = (L > 0.f) ? O / L : 0.f;
-        const float lse = (L > 0.f) ? (M + log2f(L)) * kLn2 : -INFINITY;
+        const float lse = (L > 0.f) ? M + log2f(L) * kLn2 : -INFINITY;
         const int h = g * G + hh;
         const size_t row = (size_t)b * p.Hq + h;
         if (p.o_part != nullptr) {
@@ -361,29 +367,29 @@ __global__ void __launch_bounds__(DecodeShape<D, G>::NT)
 
     // splits past the last non-empty one hold (0, -inf) and are skipped
     const int nz = (C > 0) ? (int)min((long long)S, ((long long)n + C - 1) / C) : 0;
-    float* s_w = reinterpret_cast<float*>(smem);  // [G][S] weights (log2 domain first)
+    float* s_w = reinterpret_cast<float*>(smem);  // [G][S]: lse of each split, then its weight
     float* s_hl = s_w + G * S;                    // [G][2]: lse, 1/L
     if (warp < G) {
         const size_t row = (size_t)b * p.Hq + g * G + warp;
         float mx = -INFINITY;
         for (int j = lane; j < nz; j += 32) {
-            const float l2 = __ldcg(p.lse_part + row * S + j) * kLog2e;
-            s_w[warp * S + j] = l2;
-            mx = fmaxf(mx, l2);
+            const float lj = __ldcg(p.lse_part + row * S + j);
+            s_w[warp * S + j] = lj;
+            mx = fmaxf(mx, lj);
         }
 #pragma unroll
         for (int m = 16; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
         const float mu = (mx == -INFINITY) ? 0.f : mx;
         float sum = 0.f;
         for (int j = lane; j < nz; j += 32) {
-            const float w = exp2f(s_w[warp * S + j] - mu);
+            const float w = exp2f((s_w[warp * S + j] - mu) * kLog2e);
             s_w[warp * S + j] = w;
             sum += w;
         }
 #pragma unroll
         for (int m = 16; m >= 1; m >>= 1) sum += __shfl_xor_sync(kFull, sum, m);
         if (lane == 0) {
-            s_hl[warp * 2] = (sum > 0.f) ? (mx + log2f(sum)) * kLn2 : -INFINITY;
+            s_hl[warp * 2] = (sum > 0.f) ? mx + log2f(sum) * kLn2 : -INFINITY;
             s_hl[warp * 2 + 1] = (sum > 0.f) ? 1.f / sum : 0.f;
         }
     }

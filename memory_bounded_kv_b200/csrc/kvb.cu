@@ -120,7 +120,7 @@ kvb_status kvb_decode_attn(const kvb_attn_args* a, kvb_stream stream) {
     p.len = a->len; p.t = a->t;
     p.Hq = a->Hq; p.Hkv = a->Hkv; p.cap = a->cap; p.S = a->num_splits; p.split_len = a->split_len;
     const double scale = (a->scale == 0.0f) ? 1.0 / std::sqrt((double)a->d) : (double)a->scale;
-    p.qscale = (float)(scale * 1.4426950408889634);
+    p.qscale = (float)scale;
     p.o_part = a->o_part; p.lse_part = a->lse_part; p.counters = a->counters;
     p.o = a->o; p.o_bf16 = (a->o_dtype == KVB_OUT_BF16); p.lse = a->lse;
     cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -24,23 +24,23 @@ __global__ void __launch_bounds__(256) merge_states_kernel(const __grid_constant
     const int r = blockIdx.x * 8 + warp;
     if (r >= p.R) return;
     float mx = -INFINITY;
-    for (int j = lane; j < p.n; j += 32) mx = fmaxf(mx, p.lse_in[j * p.l_sn + r * p.l_sr] * kLog2e);
+    for (int j = lane; j < p.n; j += 32) mx = fmaxf(mx, p.lse_in[j * p.l_sn + r * p.l_sr]);
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
     const float mu = (mx == -INFINITY) ? 0.f : mx;
     float sum = 0.f;
-    for (int j = lane; j < p.n; j += 32) sum += exp2f(p.lse_in[j * p.l_sn + r * p.l_sr] * kLog2e - mu);
+    for (int j = lane; j < p.n; j += 32) sum += exp2f((p.lse_in[j * p.l_sn + r * p.l_sr] - mu) * kLog2e);
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1) sum += __shfl_xor_sync(kFull, sum, m);
-    // weight of state j: exp(lse_j - lse) = exp2(lse2_j - mu) / sum
+    // weight of state j: exp(lse_j - lse) = exp(lse_j - mu) / sum; maxima stay in natural units
     const float inv = (sum > 0.f) ? 1.f / sum : 0.f;
-    if (lane == 0 && p.lse_out != nullptr) p.lse_out[r] = (sum > 0.f) ? (mx + log2f(sum)) * kLn2 : -INFINITY;
+    if (lane == 0 && p.lse_out != nullptr) p.lse_out[r] = (sum > 0.f) ? mx + log2f(sum) * kLn2 : -INFINITY;
     float* out = p.o_out + (size_t)r * p.d;
     if constexpr (VEC4) {
         for (int e = lane * 4; e < p.d; e += 128) {
             float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
             for (int j = 0; j < p.n; ++j) {
-                const float w = exp2f(p.lse_in[j * p.l_sn + r * p.l_sr] * kLog2e - mu);
+                const float w = exp2f((p.lse_in[j * p.l_sn + r * p.l_sr] - mu) * kLog2e);
                 const float4 x = *reinterpret_cast<const float4*>(p.o_in + j * p.o_sn + r * p.o_sr + e);
                 a.x = fmaf(w, x.x, a.x); a.y = fmaf(w, x.y, a.y);
                 a.z = fmaf(w, x.z, a.z); a.w = fmaf(w, x.w, a.w);
@@ -51,7 +51,7 @@ __global__ void __launch_bounds__(256) merge_states_kernel(const __grid_constant
         for (int e = lane; e < p.d; e += 32) {
             float a = 0.f;
             for (int j = 0; j < p.n; ++j) {
-                const float w = exp2f(p.lse_in[j * p.l_sn + r * p.l_sr] * kLog2e - mu);
+                const float w = exp2f((p.lse_in[j * p.l_sn + r * p.l_sr] - mu) * kLog2e);
                 a = fmaf(w, p.o_in[j * p.o_sn + r * p.o_sr + e], a);
             }
             out[e] = a * inv;

@@ -2,7 +2,10 @@
 
 Tolerances (bf16 inputs, fp32 accumulation on the GPU, float64 oracle):
   o:   max-abs <= 2e-2 and rel-L2 <= 1e-3 (over the compared tensor)
-  lse: |delta| <= 1e-4, and -inf exactly where the oracle has -inf
+  lse: |delta| <= max(1e-4, 2^-22 |lse|), and -inf exactly where the oracle has -inf.
+       1e-4 absolute is the target; a float32 lse cannot hold it when |lse| > 419
+       (its spacing there reaches 2^-23 |lse| ~ 5e-5 per rounding), so the bound
+       becomes two float32 roundings at the magnitude of lse.
 Indices, victims, lengths and cache bytes: bit-exact.
 """
 from __future__ import annotations
@@ -13,6 +16,7 @@ import torch
 O_MAXABS = 2e-2
 O_RELL2 = 1e-3
 LSE_ABS = 1e-4
+LSE_REL_F32 = 2.0 ** -22
 
 
 def dev(a: np.ndarray) -> torch.Tensor:
@@ -53,8 +57,9 @@ def assert_state_close(o, lse, o_ref, lse_ref, what: str = ""):
         inf_ref = np.isneginf(lse_ref)
         assert np.array_equal(np.isneginf(lse), inf_ref), f"{what}: -inf pattern of lse differs"
         d = np.abs(lse[~inf_ref] - lse_ref[~inf_ref])
-        dmax = float(d.max()) if d.size else 0.0
-        assert dmax <= LSE_ABS, f"{what}: lse max |delta| {dmax:.3e}"
+        tol = np.maximum(LSE_ABS, LSE_REL_F32 * np.abs(lse_ref[~inf_ref]))
+        worst = float((d / tol).max()) if d.size else 0.0
+        assert worst <= 1.0, f"{what}: lse |delta| {float(d.max()):.3e} exceeds its bound ({worst:.2f}x)"
     return maxabs, rel
 
 
