@@ -6,7 +6,8 @@
  * ---------------------------------------
  * - Every data pointer is a DEVICE pointer owned by the caller. The library
  *   allocates nothing, keeps no pointer after a call returns and holds no
- *   state except one device error word per GPU (see kvb_get_error).
+ *   state except one device error word per GPU (see kvb_get_error) and the
+ *   fixed scratch array of kvb_decode_attn_noalloc.
  * - bf16 tensors are passed as uint16_t bit patterns (IEEE bfloat16).
  * - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *   default stream). Results are valid once the stream has reached the call.
@@ -132,6 +133,38 @@ typedef struct kvb_attn_args {
 } kvb_attn_args;
 
 kvb_status kvb_decode_attn(const kvb_attn_args* args, kvb_stream stream);
+
+/* ------------------------------------------------------------------------
+ * kvb_decode_attn_noalloc -- kvb_decode_attn without caller scratch
+ *
+ * No counterpart in the pages: this is a deployment convenience. Some
+ * callers cannot hand the library temporary device memory: a plugin inside
+ * a serving process whose memory pool belongs to someone else, or code that
+ * must not call cudaMalloc on the decode path because it synchronizes the
+ * device and can stall or fail when memory is fully reserved. For them this
+ * entry point computes exactly what kvb_decode_attn computes, with the same
+ * arguments, but keeps the split states and ticket counters in one fixed
+ * array of KVB_NOALLOC_SCRATCH_BYTES in the library's own device memory
+ * (every GPU that loads the library holds it until the process exits).
+ *
+ * - o_part, lse_part and counters must be NULL (else KVB_EINVAL); o and lse
+ *   are the outputs, as for kvb_decode_attn.
+ * - A call whose split states would need more than the array, i.e.
+ *   256-rounded B*Hkv*4 + 256-rounded B*Hq*S*4 + B*Hq*S*d*4 bytes with
+ *   S = num_splits > 1, returns KVB_EINVAL and launches nothing. With
+ *   num_splits == 1 no scratch is used.
+ * - The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress with that device current); make that first call
+ *   before any stream capture.
+ * - Every call clears its counters with cudaMemsetAsync on `stream`, then
+ *   launches; it calls no cudaMalloc/cudaFree.
+ * - All calls share the one array: calls whose execution overlaps on the GPU
+ *   (different streams, or different threads with no ordering) race and
+ *   corrupt each other's results. Serialize them on one stream.
+ * ---------------------------------------------------------------------- */
+#define KVB_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+kvb_status kvb_decode_attn_noalloc(const kvb_attn_args* args, kvb_stream stream);
 
 /* ------------------------------------------------------------------------
  * kvb_merge_states -- n-way merge of attention states

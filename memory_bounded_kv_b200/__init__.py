@@ -18,7 +18,7 @@ import torch
 from . import _lib
 
 __all__ = [
-    "KvbError", "kvb_decode_attn", "kvb_merge_states", "kvb_evict_insert", "kvb_compact_blocks",
+    "KvbError", "kvb_decode_attn", "kvb_decode_attn_noalloc", "kvb_merge_states", "kvb_evict_insert", "kvb_compact_blocks",
     "kvb_asm_workspace_bytes", "kvb_asm_lookup_merge", "kvb_get_error", "kvb_abi_version",
     "decode_workspace",
 ]
@@ -142,6 +142,53 @@ def kvb_decode_attn(q, k, v, log_beta, pos, len, t, o, lse=None, *, scale: float
         counters=None if counters is None else counters.data_ptr(),
         o=o.data_ptr(), o_dtype=odt, lse=None if lse is None else lse.data_ptr())
     _check(_lib.lib().kvb_decode_attn(ctypes.byref(a), _stream(stream)), "kvb_decode_attn")
+
+
+def kvb_decode_attn_noalloc(q, k, v, log_beta, pos, len, t, o, lse=None, *, scale: float = 0.0,
+                            num_splits: int = 1, split_len: int = 0, stream=None) -> None:
+    """kvb_decode_attn for callers that cannot provide scratch device memory.
+
+    Same inputs and outputs as kvb_decode_attn, without o_part/lse_part/counters: the split
+    states live in the library's fixed device array (NOALLOC_SCRATCH_BYTES per GPU), so the
+    call allocates nothing. A problem whose split states do not fit raises KvbError (invalid
+    argument). Calls that overlap on the GPU share that array and race: keep them on one
+    stream. The first call on a device looks up the array's address; make it before any
+    stream capture.
+    """
+    _need(q, torch.bfloat16, "q"); _need(k, torch.bfloat16, "k"); _need(v, torch.bfloat16, "v")
+    B, Hq, d = q.shape
+    Bk, Hkv, cap, dk = k.shape
+    if dk != d or tuple(v.shape) != tuple(k.shape) or Bk != B:
+        raise ValueError("k/v must be [B, Hkv, cap, d] matching q")
+    if q.stride(2) != 1 or k.stride(3) != 1 or k.stride(2) != d or v.stride() != k.stride():
+        raise ValueError("q/k/v: innermost dim contiguous, slot stride d, k and v with equal strides")
+    _need(len, torch.int32, "len"); _contig(len, "len")
+    if log_beta is not None:
+        _need(log_beta, torch.float32, "log_beta")
+        _need(pos, torch.int32, "pos")
+        if log_beta.stride() != pos.stride() or log_beta.stride(2) != 1:
+            raise ValueError("log_beta and pos need equal strides with slot stride 1")
+        _need(t, torch.int32, "t")
+    if t is not None:
+        _need(t, torch.int32, "t"); _contig(t, "t")
+    if o.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("o must be float32 or bfloat16")
+    _contig(o, "o")
+    if lse is not None:
+        _need(lse, torch.float32, "lse"); _contig(lse, "lse")
+    a = _lib.AttnArgs(
+        q=q.data_ptr(), q_stride_b=q.stride(0), q_stride_h=q.stride(1),
+        k=k.data_ptr(), v=v.data_ptr(), kv_stride_b=k.stride(0), kv_stride_h=k.stride(1),
+        log_beta=None if log_beta is None else log_beta.data_ptr(),
+        pos=None if pos is None else pos.data_ptr(),
+        meta_stride_b=0 if log_beta is None else log_beta.stride(0),
+        meta_stride_h=0 if log_beta is None else log_beta.stride(1),
+        len=len.data_ptr(), t=None if t is None else t.data_ptr(),
+        B=B, Hq=Hq, Hkv=Hkv, d=d, cap=cap, scale=float(scale),
+        num_splits=int(num_splits), split_len=int(split_len), o_part=None, lse_part=None, counters=None,
+        o=o.data_ptr(), o_dtype=_lib.KVB_OUT_F32 if o.dtype == torch.float32 else _lib.KVB_OUT_BF16,
+        lse=None if lse is None else lse.data_ptr())
+    _check(_lib.lib().kvb_decode_attn_noalloc(ctypes.byref(a), _stream(stream)), "kvb_decode_attn_noalloc")
 
 
 def kvb_merge_states(o_in, lse_in, o_out, lse_out=None, *, stream=None) -> None:

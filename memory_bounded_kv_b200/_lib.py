@@ -13,7 +13,7 @@ _SZ = ctypes.c_size_t
 
 # symbols include/kvb.h declares (kept in sync by tests/test_abi.py)
 EXPORTS = (
-    "kvb_decode_attn", "kvb_merge_states", "kvb_evict_insert", "kvb_compact_blocks",
+    "kvb_decode_attn", "kvb_decode_attn_noalloc", "kvb_merge_states", "kvb_evict_insert", "kvb_compact_blocks",
     "kvb_asm_workspace_bytes", "kvb_asm_lookup_merge", "kvb_get_error", "kvb_status_str",
     "kvb_abi_version",
 )
@@ -21,6 +21,7 @@ EXPORTS = (
 KVB_OK, KVB_EINVAL, KVB_ECUDA, KVB_EDEVICE = 0, 1, 2, 3
 KVB_OUT_F32, KVB_OUT_BF16 = 0, 1
 DERR_LEN, DERR_SPLIT, DERR_RANGE, DERR_TIMEOUT = 1, 2, 4, 8
+NOALLOC_SCRATCH_BYTES = 16 << 20   # KVB_NOALLOC_SCRATCH_BYTES
 
 
 class AttnArgs(ctypes.Structure):
@@ -55,6 +56,7 @@ def lib() -> ctypes.CDLL:
             raise RuntimeError(f"libkvb.so not found at {path}")
         L = ctypes.CDLL(path)
         L.kvb_decode_attn.argtypes = [ctypes.POINTER(AttnArgs), _P]
+        L.kvb_decode_attn_noalloc.argtypes = [ctypes.POINTER(AttnArgs), _P]
         L.kvb_merge_states.argtypes = [_P, _P, _I64, _I64, _I64, _I64, _I32, _I32, _I32, _P, _P, _P]
         L.kvb_evict_insert.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _P, _P]
         L.kvb_compact_blocks.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _P]
@@ -65,7 +67,7 @@ def lib() -> ctypes.CDLL:
         L.kvb_status_str.argtypes = [_I32]
         L.kvb_status_str.restype = ctypes.c_char_p
         L.kvb_abi_version.argtypes = []
-        for f in ("kvb_decode_attn", "kvb_merge_states", "kvb_evict_insert", "kvb_compact_blocks",
+        for f in ("kvb_decode_attn", "kvb_decode_attn_noalloc", "kvb_merge_states", "kvb_evict_insert", "kvb_compact_blocks",
                   "kvb_asm_lookup_merge", "kvb_get_error", "kvb_abi_version"):
             getattr(L, f).restype = _I32
         _lib = L

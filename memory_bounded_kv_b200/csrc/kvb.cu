@@ -65,6 +65,32 @@ kvb_status dispatch_g(const kvb::DecodeParams& p, int B, int G, bool bias, cudaS
     }
 }
 
+// ---- fixed scratch of kvb_decode_attn_noalloc ------------------------------
+// The split states and ticket counters of the no-allocation entry point live
+// here instead of in caller memory. Host code must not use the symbol itself
+// as a device address: it is a host-side stand-in. The device address is
+// looked up once per device with cudaGetSymbolAddress (that device current).
+static __device__ __align__(256) unsigned char g_noalloc_scratch[KVB_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+kvb_status noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVB_ECUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_addr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return KVB_ECUDA;
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return KVB_OK;
+}
+
+inline size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
 }  // namespace
 
 extern "C" {
@@ -125,6 +151,34 @@ kvb_status kvb_decode_attn(const kvb_attn_args* a, kvb_stream stream) {
     p.o = a->o; p.o_bf16 = (a->o_dtype == KVB_OUT_BF16); p.lse = a->lse;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return a->d == 128 ? dispatch_g<128>(p, a->B, G, bias, st) : dispatch_g<64>(p, a->B, G, bias, st);
+}
+
+kvb_status kvb_decode_attn_noalloc(const kvb_attn_args* a, kvb_stream stream) {
+    if (a == nullptr) return KVB_EINVAL;
+    if (a->o_part != nullptr || a->lse_part != nullptr || a->counters != nullptr) return KVB_EINVAL;
+    kvb_attn_args b = *a;
+    if (a->num_splits > 1) {
+        if (a->B < 1 || a->Hq < 1 || a->Hkv < 1 || (a->d != 64 && a->d != 128) || a->num_splits > 1024 ||
+            a->B > 65535 || a->Hkv > 65535 || a->Hq > 65535)
+            return KVB_EINVAL;
+        const size_t rows = (size_t)a->B * a->Hq * a->num_splits;
+        const size_t cnt_bytes = (size_t)a->B * a->Hkv * sizeof(uint32_t);
+        const size_t lse_off = round256(cnt_bytes);
+        const size_t o_off = lse_off + round256(rows * sizeof(float));
+        const size_t need = o_off + rows * a->d * sizeof(float);
+        if (need > (size_t)KVB_NOALLOC_SCRATCH_BYTES) return KVB_EINVAL;
+        void* base = nullptr;
+        const kvb_status st = noalloc_scratch(&base);
+        if (st != KVB_OK) return st;
+        unsigned char* s = static_cast<unsigned char*>(base);
+        b.counters = reinterpret_cast<uint32_t*>(s);
+        b.lse_part = reinterpret_cast<float*>(s + lse_off);
+        b.o_part = reinterpret_cast<float*>(s + o_off);
+        // the array keeps the last call's contents: the ticket counters must start at zero
+        if (cudaMemsetAsync(b.counters, 0, cnt_bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+            return KVB_ECUDA;
+    }
+    return kvb_decode_attn(&b, stream);
 }
 
 kvb_status kvb_merge_states(const float* o_in, const float* lse_in, int64_t o_stride_n, int64_t o_stride_r,
