@@ -147,7 +147,7 @@ class ClockSampler:
 
 
 def kernel_src_hash() -> str:
-    with open(os.path.join(ROOT, "memory_bounded_kv_b200", "csrc", "decode_attn.cuh"), "rb") as f:
+    with open(os.path.join(ROOT, "memory_bounded_kv_b200", "csrc", "decode_attn_tc.cuh"), "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
@@ -194,7 +194,7 @@ class DecodeBench:
         self.o = torch.zeros(w.B, w.Hq, w.d, device="cuda")
         self.lse = torch.zeros(w.B, w.Hq, device="cuda")
         self.tokens_per_step = w.B
-        self.launches_per_step = 2
+        self.launches_per_step = 2 + (self.S > 1)   # evict/insert, attention (+ split merge)
         self.workload = f"{w.name} (config {cfg})"
 
     def t_of(self, i: int):
@@ -259,7 +259,9 @@ class DecodeBench:
         return n * 8 + w.B * w.Hkv * (2 * w.d * 2 + 4 + 4 + 4)
 
     def kernel_name(self):
-        return f"decode_attn_kernel<d={self.w.d},G={self.w.Hq // self.w.Hkv},bias=1> S={self.S}"
+        merge = " + merge_splits_kernel" if self.S > 1 else ""
+        return (f"kvb_decode_attn = decode_attn_tc_kernel<d={self.w.d},G={self.w.Hq // self.w.Hkv},bias=1>"
+                f"{merge}, S={self.S}")
 
     def config(self):
         w = self.w
@@ -326,7 +328,7 @@ class ASMBench:
         self.lse = torch.zeros(N, H, device="cuda")
         self.ws = torch.empty(kvb.kvb_asm_workspace_bytes(N, H, w.K), dtype=torch.uint8, device="cuda")
         self.tokens_per_step = N
-        self.launches_per_step = 3
+        self.launches_per_step = 4   # attention + split merge, lookup + state merge
         self.workload = "attention-state memory H32 K4096 d128, 256 queries, self attention over 2048 (config 4)"
 
     def prepare(self, total_steps):
@@ -443,7 +445,8 @@ class MementoBench:
         return int(self.active[first:first + count].sum())
 
     def launches(self, first, count):
-        return 2 * count + sum(1 for i in range(first, first + count) if i in self.comp)
+        per = 2 + (self.S > 1)
+        return per * count + sum(1 for i in range(first, first + count) if i in self.comp)
 
     def mean_kv_bytes(self, first, count):
         w = self.w
@@ -514,7 +517,8 @@ def run_kvb(args, world, rank, local):
     else:
         attn_bytes = bench.mean_kv_bytes(W, K) if hasattr(bench, "mean_kv_bytes") else bench.attn_bytes()
         achieved = attn_bytes / (kms / 1e3) / 1e9
-        name = bench.kernel_name() if hasattr(bench, "kernel_name") else "decode_attn_kernel<128,4,plain>"
+        name = (bench.kernel_name() if hasattr(bench, "kernel_name")
+                else "kvb_decode_attn = decode_attn_tc_kernel<128,4,plain> + merge_splits_kernel")
         roofline = {"bound": "hbm", "kernel": name, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                     "frac": achieved / hbm_peak, "peak_source": f"{peak_kind} (hbm_gbs)",
                     "traffic": MEASURED_TRAFFIC.get((src, args.config)),

@@ -95,16 +95,18 @@ enum kvb_device_error {
  *   lse      [B, Hq] f32, contiguous, may be NULL
  *   o_part   [B, Hq, num_splits, d] f32, lse_part [B, Hq, num_splits] f32:
  *            every split's state (empty splits get (0, -inf)); required when
- *            num_splits > 1, may be NULL when num_splits == 1
- *   counters [B, Hkv] uint32: required when num_splits > 1. They must be
- *            zero before the first call; every call leaves them zero. The
- *            last split to finish for a (b, g) merges the states, so no
- *            second launch and no waiting is needed.
+ *            num_splits > 1, may be NULL when num_splits == 1. With
+ *            num_splits > 1 the call launches the attention kernel, which
+ *            writes every split's state, and a merge kernel that combines
+ *            them into o and lse.
+ *   counters reserved; ignored (may be NULL).
  *
  * Requirements (else KVB_EINVAL): d in {64, 128}; Hq % Hkv == 0 and
  * Hq / Hkv in {1, 2, 4, 8}; B, Hkv, cap >= 1; 1 <= num_splits <= 1024;
  * split_len >= 0; q, k, v 16-byte aligned and every q/kv stride a multiple
- * of 8 elements; scale finite (0 selects 1/sqrt(d)).
+ * of 8 elements; kv_stride_h > 0 when Hkv > 1; scale finite (0 selects
+ * 1/sqrt(d)). K and V are read with TMA tensor copies, so a layout the
+ * tensor-map encoder refuses also returns KVB_EINVAL.
  * Device-side checks: len in [0, cap] and len <= num_splits * split_len
  * (when split_len > 0); a row that fails gets the empty state.
  * Preconditions (not checked): log beta finite and <= 0, positions unique
@@ -143,21 +145,21 @@ kvb_status kvb_decode_attn(const kvb_attn_args* args, kvb_stream stream);
  * must not call cudaMalloc on the decode path because it synchronizes the
  * device and can stall or fail when memory is fully reserved. For them this
  * entry point computes exactly what kvb_decode_attn computes, with the same
- * arguments, but keeps the split states and ticket counters in one fixed
- * array of KVB_NOALLOC_SCRATCH_BYTES in the library's own device memory
- * (every GPU that loads the library holds it until the process exits).
+ * arguments, but keeps the split states in one fixed array of
+ * KVB_NOALLOC_SCRATCH_BYTES in the library's own device memory (every GPU
+ * that loads the library holds it until the process exits).
  *
  * - o_part, lse_part and counters must be NULL (else KVB_EINVAL); o and lse
  *   are the outputs, as for kvb_decode_attn.
  * - A call whose split states would need more than the array, i.e.
- *   256-rounded B*Hkv*4 + 256-rounded B*Hq*S*4 + B*Hq*S*d*4 bytes with
- *   S = num_splits > 1, returns KVB_EINVAL and launches nothing. With
- *   num_splits == 1 no scratch is used.
+ *   256-rounded B*Hq*S*4 + B*Hq*S*d*4 bytes with S = num_splits > 1,
+ *   returns KVB_EINVAL and launches nothing. With num_splits == 1 no
+ *   scratch is used.
  * - The first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress with that device current); make that first call
  *   before any stream capture.
- * - Every call clears its counters with cudaMemsetAsync on `stream`, then
- *   launches; it calls no cudaMalloc/cudaFree.
+ * - Every call writes all the split states it reads back, so the array's
+ *   previous contents never matter; it calls no cudaMalloc/cudaFree.
  * - All calls share the one array: calls whose execution overlaps on the GPU
  *   (different streams, or different threads with no ordering) race and
  *   corrupt each other's results. Serialize them on one stream.

@@ -1,0 +1,561 @@
+// Split-K GQA decode attention with the retention bias of "Cache What Lasts"
+// section 2.1 (logit = scale * q.k_i + (t - i) log beta_i) and the (o, lse)
+// state of "Context Memorization" core method step 1. With several splits
+// the kernel writes every split's state and merge_splits_kernel (below)
+// combines them with that page's step-2 operator. (Merging in the last CTA
+// of each (sequence, kv head) to finish was measured and rejected: a CTA
+// that lags once is likely to be last again, so merges pile up on it.)
+//
+// Persistent, warp-specialised kernel:
+//  - The work is a list of units (sequence b, kv head g, split j); CTA c
+//    takes units c, c + grid, c + 2*grid, ...
+//  - One producer warp streams each unit's K/V tiles (T slots) with TMA
+//    tensor loads (128-byte swizzle) into a STAGES-deep shared-memory ring.
+//    With every tile it also stages the tile's bias ((t - pos) * log beta, or
+//    -inf past the split's end) and, with a unit's first tile, the unit's
+//    G query rows; one "full" mbarrier per stage counts the bytes and the
+//    producer lanes' arrivals, one "empty" mbarrier the consumers' release.
+//  - Four consumer warps each own 16 slots of a tile. Both products run on
+//    the tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate) with the
+//    G query heads as the M rows (padded to 16):
+//      S = Q . K^T       A = q rows (registers), B = K via ldmatrix
+//      O += P . V        A = P in the accumulator layout of S (no shuffles),
+//                        B = V via ldmatrix.trans; P is split into a bf16
+//                        high part and a bf16 residual, two mma each, which
+//                        keeps ~16 bits of P (a single bf16 P would cost
+//                        ~1e-3 relative error in o).
+//    Online softmax per warp and head (maxima in natural units, exp2 of
+//    scaled differences), O rescaled only when a maximum moved.
+//  - At the end of a unit the consumer warps combine through shared memory
+//    (a named barrier among consumers only; the producer keeps prefetching
+//    the next unit's tiles) and write the split's state.
+// Every wait is bounded (1 s); on a timeout the CTA records KVB_DERR_TIMEOUT,
+// stops, and drains the copies it issued before exiting.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace kvb {
+
+struct DecodeTcParams {
+    const uint16_t* q;
+    long long q_sb, q_sh;
+    const float* lb;
+    const int* pos;
+    long long m_sb, m_sh;
+    const int* len;
+    const int* t;
+    int Hq, Hkv, cap, S, split_len;
+    int units;      // B * Hkv * S
+    int kv_shared;  // kv_stride_b == 0: every row reads sequence 0's cache
+    float scale;
+    float* o_part;
+    float* lse_part;
+    void* o;
+    int o_bf16;
+    float* lse;
+};
+
+template <int D, int G>
+struct TcShape {
+    static constexpr int NWC = 4;                 // consumer warps
+    static constexpr int NT = (NWC + 1) * 32;     // + one producer warp
+    static constexpr int T = 16 * NWC;            // slots per tile
+    static constexpr int STAGES = 3;
+    static constexpr int HALVES = D / 64;         // 128-byte swizzle rows hold 64 bf16
+    static constexpr int HALF_BYTES = T * 128;
+    static constexpr int TILE_BYTES = HALVES * HALF_BYTES;  // one of K or V
+    static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+    static constexpr int KSTEPS = D / 16;
+    static constexpr int NTILES = D / 8;          // n-tiles of the PV product
+    static constexpr int QBYTES = G * D * 2;
+    // shared-memory layout (offsets from a 1024-aligned base)
+    static constexpr int RING_OFF = 0;
+    static constexpr int Q_OFF = RING_OFF + STAGES * STAGE_BYTES;       // [ST][G][D] bf16
+    static constexpr int BIAS_OFF = Q_OFF + STAGES * QBYTES;            // [ST][T] f32
+    static constexpr int META_OFF = BIAS_OFF + STAGES * T * 4;          // [ST][8] int
+    static constexpr int BAR_OFF = META_OFF + STAGES * 32;              // full[ST], empty[ST]
+    static constexpr int MISC_OFF = BAR_OFF + 2 * STAGES * 8;           // abort, issued
+    static constexpr int EPI_OFF = (MISC_OFF + 16 + 15) / 16 * 16;      // [NWC][G][D] f32
+    static constexpr int ML_OFF = EPI_OFF + NWC * G * D * 4;            // [NWC][G][2] f32
+    static constexpr int END_OFF = ML_OFF + NWC * G * 2 * 4;
+    static constexpr size_t SMEM = 1024 + END_OFF;
+    static_assert(D == 64 || D == 128, "d");
+    static_assert(G == 1 || G == 2 || G == 4 || G == 8, "G");
+    static_assert(STAGE_BYTES % 1024 == 0 && Q_OFF % 16 == 0, "alignment");
+};
+
+// ---- PTX wrappers -------------------------------------------------------------
+
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+// D = A . B + C, m16n8k16, bf16 inputs, fp32 accumulators; A rows 8..15 are zero.
+__device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+__device__ __forceinline__ void named_bar(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ---- unit bookkeeping shared by producer and consumers --------------------------
+
+struct UnitInfo {
+    int b, g, split, s0, nk, ntiles, n;  // n: the (b, g) length after the validity checks
+};
+
+// The two loads a unit's geometry depends on; fetched one unit ahead by the producer.
+struct UnitRaw {
+    int len, t;
+};
+
+__device__ __forceinline__ UnitRaw unit_raw(const DecodeTcParams& p, int u) {
+    UnitRaw r{0, 0};
+    if (u < p.units) {
+        const int per_b = p.Hkv * p.S;
+        const int b = u / per_b;
+        const int g = (u - b * per_b) / p.S;
+        r.len = p.len[b * p.Hkv + g];
+        r.t = (p.t == nullptr) ? 0 : p.t[b];
+    }
+    return r;
+}
+
+template <int T>
+__device__ __forceinline__ UnitInfo unit_info(const DecodeTcParams& p, int u, UnitRaw raw, bool record_errors) {
+    UnitInfo r;
+    const int per_b = p.Hkv * p.S;
+    r.b = u / per_b;
+    const int rem = u - r.b * per_b;
+    r.g = rem / p.S;
+    r.split = rem - r.g * p.S;
+    int n = raw.len;
+    const bool active = (p.t == nullptr) || (raw.t >= 0);
+    const bool bad_len = n < 0 || n > p.cap;
+    const bool bad_split = !bad_len && p.split_len > 0 && (long long)n > (long long)p.S * p.split_len;
+    if (record_errors && (bad_len || bad_split) && r.split == 0) raise_error(bad_len ? KVB_DERR_LEN : KVB_DERR_SPLIT);
+    if (bad_len || bad_split || !active) n = 0;
+    const long long C = p.split_len > 0 ? (long long)p.split_len : (long long)((n + p.S - 1) / p.S);
+    r.s0 = (int)min((long long)r.split * C, (long long)n);
+    const int s1 = (int)min((long long)r.s0 + C, (long long)n);
+    r.nk = s1 - r.s0;
+    r.ntiles = (r.nk + T - 1) / T;
+    r.n = n;
+    return r;
+}
+
+template <int D, int G, bool BIAS>
+__global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
+    decode_attn_tc_kernel(const __grid_constant__ DecodeTcParams p, const __grid_constant__ CUtensorMap tmK,
+                          const __grid_constant__ CUtensorMap tmV) {
+    using SH = TcShape<D, G>;
+    constexpr int NWC = SH::NWC, T = SH::T, ST = SH::STAGES;
+    extern __shared__ unsigned char smem_dyn[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint16_t* s_q = reinterpret_cast<uint16_t*>(smem + SH::Q_OFF);
+    float* s_bias = reinterpret_cast<float*>(smem + SH::BIAS_OFF);
+    int* s_meta = reinterpret_cast<int*>(smem + SH::META_OFF);
+    uint64_t* s_full = reinterpret_cast<uint64_t*>(smem + SH::BAR_OFF);
+    uint64_t* s_empty = s_full + ST;
+    volatile int* s_abort = reinterpret_cast<int*>(smem + SH::MISC_OFF);
+    int* s_issued = reinterpret_cast<int*>(smem + SH::MISC_OFF) + 1;
+    float* s_o = reinterpret_cast<float*>(smem + SH::EPI_OFF);
+    float* s_ml = reinterpret_cast<float*>(smem + SH::ML_OFF);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        for (int s = 0; s < ST; ++s) {
+            mbar_init(&s_full[s], 33);          // producer lane 0's expect_tx + 32 producer lanes
+            mbar_init(&s_empty[s], NWC * 32);   // every consumer lane
+        }
+        *s_abort = 0;
+        *s_issued = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == NWC) {
+        // ======================= producer warp =======================
+        int it = 0;
+        bool stop = false;
+        UnitRaw next_raw = unit_raw(p, blockIdx.x);
+        for (int u = blockIdx.x; u < p.units + gridDim.x && !stop; u += gridDim.x) {
+            const bool end = u >= p.units;  // one end record after the last unit
+            const UnitRaw raw = next_raw;
+            next_raw = unit_raw(p, u + gridDim.x);  // in flight while this unit's tiles are issued
+            UnitInfo ui{};
+            if (!end) ui = unit_info<T>(p, u, raw, lane == 0);
+            const int records = end ? 1 : max(ui.ntiles, 1);
+            const int tb = raw.t;
+            const size_t m_off = end ? 0 : (size_t)ui.b * p.m_sb + (size_t)ui.g * p.m_sh + (size_t)ui.s0;
+            for (int i = 0; i < records; ++i, ++it) {
+                const int st = it % ST;
+                // this tile's bias, loaded before waiting for the stage
+                float bias[T / 32];
+#pragma unroll
+                for (int j = 0; j < T / 32; ++j) {
+                    const int key = i * T + lane + 32 * j;
+                    float bv = -INFINITY;
+                    if (!end && key < ui.nk) {
+                        if constexpr (BIAS) {
+                            bv = __fmul_rn(__int2float_rn(tb - p.pos[m_off + key]), p.lb[m_off + key]);
+                        } else {
+                            bv = 0.f;
+                        }
+                    }
+                    bias[j] = bv;
+                }
+                if (it >= ST && !mbar_wait(&s_empty[st], (unsigned)((it / ST) - 1) & 1u)) {
+                    if (lane == 0) {
+                        raise_error(KVB_DERR_TIMEOUT);
+                        *s_abort = 1;
+                    }
+                    stop = true;
+                    break;
+                }
+                if (*s_abort) {
+                    stop = true;
+                    break;
+                }
+                const bool data = !end && ui.ntiles > 0;
+                if (lane == 0) {
+                    int* m = s_meta + st * 8;
+                    m[0] = end ? -1 : u;
+                    m[1] = i;
+                    m[2] = end ? 0 : ui.ntiles;
+                    m[3] = data ? min(T, ui.nk - i * T) : 0;
+                    m[4] = ui.b;
+                    m[5] = ui.g;
+                    m[6] = ui.split;
+                    m[7] = ui.n;
+                    unsigned tx = data ? (unsigned)SH::STAGE_BYTES : 0u;
+                    const bool with_q = data && i == 0;
+                    if (with_q) tx += SH::QBYTES;
+                    mbar_arrive_expect_tx(&s_full[st], tx);
+                    if (data) {
+                        unsigned char* kt = smem + SH::RING_OFF + st * SH::STAGE_BYTES;
+                        unsigned char* vt = kt + SH::TILE_BYTES;
+                        const int row = ui.s0 + i * T;
+                        const int bb = p.kv_shared ? 0 : ui.b;
+#pragma unroll
+                        for (int h = 0; h < SH::HALVES; ++h) {
+                            tma_load_4d(kt + h * SH::HALF_BYTES, &tmK, 64 * h, row, ui.g, bb, &s_full[st]);
+                            tma_load_4d(vt + h * SH::HALF_BYTES, &tmV, 64 * h, row, ui.g, bb, &s_full[st]);
+                        }
+                    }
+                    if (with_q) {
+                        const uint16_t* qsrc = p.q + (size_t)ui.b * p.q_sb + (size_t)(ui.g * G) * p.q_sh;
+                        uint16_t* qdst = s_q + st * G * D;
+                        if (p.q_sh == D) {
+                            bulk_g2s(qdst, qsrc, (unsigned)SH::QBYTES, &s_full[st]);
+                        } else {
+                            for (int hh = 0; hh < G; ++hh)
+                                bulk_g2s(qdst + hh * D, qsrc + (size_t)hh * p.q_sh, (unsigned)(D * 2), &s_full[st]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < T / 32; ++j) s_bias[st * T + lane + 32 * j] = bias[j];
+                __syncwarp();
+                mbar_arrive(&s_full[st]);
+            }
+        }
+        if (lane == 0) *s_issued = it;
+    } else {
+        // ======================= consumer warps =======================
+        const int r = lane >> 2;          // M row = query head within the group (rows >= G are padding)
+        const int cq = lane & 3;          // quad index: columns 2*cq, 2*cq+1 of each 8-wide n-tile
+        const int kw = 16 * warp;         // this warp's first slot in a tile
+        const uint32_t ring = smem_u32(smem + SH::RING_OFF);
+        // ldmatrix row addresses (relative to a tile half): swizzle xor = row & 7 = lane & 7
+        const int kq_row = kw + (lane & 7) + ((lane >> 4) << 3);   // QK operand rows (keys)
+        const int kq_hi = (lane >> 3) & 1;
+        const int v_row = kw + (lane & 7) + (((lane >> 3) & 1) << 3);  // PV operand rows
+        const int v_hi = lane >> 4;
+        const int sw = lane & 7;
+
+        uint32_t qa[SH::KSTEPS][2];
+        float acc[SH::NTILES][4];
+        float m_run = -INFINITY, l_run = 0.f;
+        int it = 0;
+        bool aborted = false;
+        while (true) {
+            const int st = it % ST;
+            if (!mbar_wait(&s_full[st], (unsigned)(it / ST) & 1u)) {
+                if (lane == 0) {
+                    raise_error(KVB_DERR_TIMEOUT);
+                    *s_abort = 1;
+                }
+                aborted = true;
+                break;
+            }
+            const int* m = s_meta + st * 8;
+            const int u = m[0], i = m[1], ntiles = m[2], rows = m[3];
+            if (u < 0) break;
+            const int ub = m[4], ug = m[5], usplit = m[6], un = m[7];
+            if (i == 0) {
+                m_run = -INFINITY;
+                l_run = 0.f;
+#pragma unroll
+                for (int j = 0; j < SH::NTILES; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+                if (ntiles > 0) {
+                    const uint16_t* qs = s_q + st * G * D;
+#pragma unroll
+                    for (int s = 0; s < SH::KSTEPS; ++s) {
+                        uint32_t a0 = 0u, a2 = 0u;
+                        if (r < G) {
+                            a0 = *reinterpret_cast<const uint32_t*>(qs + r * D + 16 * s + 2 * cq);
+                            a2 = *reinterpret_cast<const uint32_t*>(qs + r * D + 16 * s + 8 + 2 * cq);
+                        }
+                        qa[s][0] = a0;
+                        qa[s][1] = a2;
+                    }
+                }
+            }
+            if (ntiles > 0) {
+                const uint32_t kt = ring + st * SH::STAGE_BYTES;
+                const uint32_t vt = kt + SH::TILE_BYTES;
+                // ---- S = Q K^T for this warp's 16 slots (two n-tiles of 8)
+                float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+                for (int s = 0; s < SH::KSTEPS; ++s) {
+                    const int chunk = 2 * (s & 3) + kq_hi;
+                    const uint32_t addr =
+                        kt + (s >> 2) * SH::HALF_BYTES + kq_row * 128 + ((chunk ^ sw) << 4);
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4(addr, b0, b1, b2, b3);
+                    mma_bf16(sc[0], qa[s][0], qa[s][1], b0, b1);
+                    mma_bf16(sc[1], qa[s][0], qa[s][1], b2, b3);
+                }
+                if (rows < T && kw + 16 > rows) {
+                    // tail: zero this warp's V rows past the split end (K rows there are masked)
+                    for (int idx = lane; idx < 16 * SH::HALVES * 8; idx += 32) {
+                        const int row = kw + idx / (SH::HALVES * 8);
+                        const int c = idx % (SH::HALVES * 8);
+                        if (row >= rows) {
+                            unsigned char* vp = smem + SH::RING_OFF + st * SH::STAGE_BYTES + SH::TILE_BYTES +
+                                                (c >> 3) * SH::HALF_BYTES + row * 128 + ((c & 7) << 4);
+                            *reinterpret_cast<uint4*>(vp) = make_uint4(0u, 0u, 0u, 0u);
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
+                // ---- logits, online softmax (row r of this lane; slots 2cq, 2cq+1, 8+2cq, 8+2cq+1)
+                const float* sb = s_bias + st * T + kw;
+                const float2 bA = *reinterpret_cast<const float2*>(sb + 2 * cq);
+                const float2 bB = *reinterpret_cast<const float2*>(sb + 8 + 2 * cq);
+                float x[4];
+                x[0] = (bA.x == -INFINITY) ? -INFINITY : fmaf(sc[0][0], p.scale, bA.x);
+                x[1] = (bA.y == -INFINITY) ? -INFINITY : fmaf(sc[0][1], p.scale, bA.y);
+                x[2] = (bB.x == -INFINITY) ? -INFINITY : fmaf(sc[1][0], p.scale, bB.x);
+                x[3] = (bB.y == -INFINITY) ? -INFINITY : fmaf(sc[1][1], p.scale, bB.y);
+                float tmax = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+                tmax = fmaxf(tmax, __shfl_xor_sync(kFull, tmax, 1));
+                tmax = fmaxf(tmax, __shfl_xor_sync(kFull, tmax, 2));
+                const float m_new = fmaxf(m_run, tmax);
+                const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+                const float alpha = exp2f((m_run - m_use) * kLog2e);
+                float pr[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) pr[j] = exp2f((x[j] - m_use) * kLog2e);
+                l_run = fmaf(l_run, alpha, (pr[0] + pr[1]) + (pr[2] + pr[3]));
+                m_run = m_new;
+                if (__any_sync(kFull, alpha != 1.f)) {
+#pragma unroll
+                    for (int j = 0; j < SH::NTILES; ++j) {
+                        acc[j][0] *= alpha;
+                        acc[j][1] *= alpha;
+                    }
+                }
+                // ---- P as the A operand: high bf16 part and bf16 residual
+                const uint32_t ph0 = pack_bf16(pr[0], pr[1]);
+                const uint32_t ph2 = pack_bf16(pr[2], pr[3]);
+                const uint32_t pl0 = pack_bf16(pr[0] - __uint_as_float(ph0 << 16),
+                                               pr[1] - __uint_as_float(ph0 & 0xffff0000u));
+                const uint32_t pl2 = pack_bf16(pr[2] - __uint_as_float(ph2 << 16),
+                                               pr[3] - __uint_as_float(ph2 & 0xffff0000u));
+                // ---- O += P V (two n-tiles of 8 dims per ldmatrix)
+#pragma unroll
+                for (int j = 0; j < SH::NTILES / 2; ++j) {
+                    const int chunk = 2 * (j & 3) + v_hi;
+                    const uint32_t addr =
+                        vt + (j >> 2) * SH::HALF_BYTES + v_row * 128 + ((chunk ^ sw) << 4);
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4_t(addr, b0, b1, b2, b3);
+                    mma_bf16(acc[2 * j], ph0, ph2, b0, b1);
+                    mma_bf16(acc[2 * j], pl0, pl2, b0, b1);
+                    mma_bf16(acc[2 * j + 1], ph0, ph2, b2, b3);
+                    mma_bf16(acc[2 * j + 1], pl0, pl2, b2, b3);
+                }
+            }
+            __syncwarp();
+            mbar_arrive(&s_empty[st]);
+            ++it;
+            if (ntiles > 0 && i != ntiles - 1) continue;
+
+            // ======== end of unit: combine warps, write the split's state ========
+            l_run += __shfl_xor_sync(kFull, l_run, 1);
+            l_run += __shfl_xor_sync(kFull, l_run, 2);
+            if (r < G) {
+#pragma unroll
+                for (int j = 0; j < SH::NTILES; ++j)
+                    *reinterpret_cast<float2*>(s_o + (warp * G + r) * D + 8 * j + 2 * cq) =
+                        make_float2(acc[j][0], acc[j][1]);
+                if (cq == 0) {
+                    s_ml[(warp * G + r) * 2] = m_run;
+                    s_ml[(warp * G + r) * 2 + 1] = l_run;
+                }
+            }
+            named_bar(1, NWC * 32);
+            const int S = p.S;
+            for (int idx = tid; idx < G * D; idx += NWC * 32) {
+                const int hh = idx / D, e = idx % D;
+                float M = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < NWC; ++w) M = fmaxf(M, s_ml[(w * G + hh) * 2]);
+                const float Mu = (M == -INFINITY) ? 0.f : M;
+                float L = 0.f, O = 0.f;
+#pragma unroll
+                for (int w = 0; w < NWC; ++w) {
+                    const float f = exp2f((s_ml[(w * G + hh) * 2] - Mu) * kLog2e);
+                    L = fmaf(f, s_ml[(w * G + hh) * 2 + 1], L);
+                    O = fmaf(f, s_o[(w * G + hh) * D + e], O);
+                }
+                const float out = (L > 0.f) ? O / L : 0.f;
+                const float lse = (L > 0.f) ? M + log2f(L) * kLn2 : -INFINITY;
+                const size_t row = (size_t)ub * p.Hq + ug * G + hh;
+                if (p.o_part != nullptr) {
+                    p.o_part[(row * S + usplit) * D + e] = out;
+                    if (e == 0) p.lse_part[row * S + usplit] = lse;
+                }
+                if (S == 1) {
+                    if (p.o_bf16) {
+                        reinterpret_cast<__nv_bfloat16*>(p.o)[row * D + e] = __float2bfloat16_rn(out);
+                    } else {
+                        reinterpret_cast<float*>(p.o)[row * D + e] = out;
+                    }
+                    if (e == 0 && p.lse != nullptr) p.lse[row] = lse;
+                }
+            }
+            named_bar(1, NWC * 32);  // s_o and s_ml free for the next unit
+        }
+        (void)aborted;
+    }
+
+    // drain: copies issued into stages that no consumer waited for
+    __syncthreads();
+    if (tid == 0 && *s_abort) {
+        const int issued = *s_issued;
+        for (int k = max(0, issued - ST); k < issued; ++k) mbar_wait(&s_full[k % ST], (unsigned)(k / ST) & 1u, 100000000ull);
+    }
+}
+
+// Merge of the num_splits states of each (b, query head) row, [ASM] step 2's
+// operator with Z carried as lse: one warp per row; lane j holds split j's
+// weight exp(lse_j - max) and hands it out by shuffle while every lane
+// accumulates its D/32 dims, with eight independent L2 loads in flight.
+template <int D>
+__global__ void __launch_bounds__(256) merge_splits_kernel(const float* __restrict__ o_part,
+                                                           const float* __restrict__ lse_part, int R, int S,
+                                                           void* o, int o_bf16, float* lse) {
+    constexpr int E = D / 32;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r = blockIdx.x * 8 + warp;
+    if (r >= R) return;
+    const float* lp = lse_part + (size_t)r * S;
+    float mx = -INFINITY;
+    for (int j = lane; j < S; j += 32) mx = fmaxf(mx, lp[j]);
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
+    const float mu = (mx == -INFINITY) ? 0.f : mx;
+    float sum = 0.f;
+    for (int j = lane; j < S; j += 32) sum += exp2f((lp[j] - mu) * kLog2e);
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) sum += __shfl_xor_sync(kFull, sum, m);
+    float acc[E];
+#pragma unroll
+    for (int k = 0; k < E; ++k) acc[k] = 0.f;
+    const float* op = o_part + (size_t)r * S * D + lane * E;
+    for (int j0 = 0; j0 < S; j0 += 32) {
+        const int cnt = min(32, S - j0);
+        const float wl = (lane < cnt) ? exp2f((lp[j0 + lane] - mu) * kLog2e) : 0.f;
+        for (int k0 = 0; k0 < cnt; k0 += 8) {
+            float w[8];
+            float v[8][E];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                w[k] = __shfl_sync(kFull, wl, (k0 + k) & 31);
+                const bool use = (k0 + k < cnt) && w[k] > 0.f;
+                const float* src = op + (size_t)(j0 + k0 + k) * D;
+                if constexpr (E == 4) {
+                    const float4 x = use ? __ldcg(reinterpret_cast<const float4*>(src)) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    v[k][0] = x.x; v[k][1] = x.y; v[k][2] = x.z; v[k][3] = x.w;
+                } else {
+                    const float2 x = use ? __ldcg(reinterpret_cast<const float2*>(src)) : make_float2(0.f, 0.f);
+                    v[k][0] = x.x; v[k][1] = x.y;
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+#pragma unroll
+                for (int e = 0; e < E; ++e) acc[e] = fmaf(w[k], v[k][e], acc[e]);
+        }
+    }
+    const float inv = (sum > 0.f) ? 1.f / sum : 0.f;
+    if (o_bf16) {
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(o) + (size_t)r * D + lane * E;
+#pragma unroll
+        for (int e = 0; e < E; ++e) out[e] = __float2bfloat16_rn(acc[e] * inv);
+    } else {
+        float* out = reinterpret_cast<float*>(o) + (size_t)r * D + lane * E;
+        if constexpr (E == 4) {
+            *reinterpret_cast<float4*>(out) = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+        } else {
+            *reinterpret_cast<float2*>(out) = make_float2(acc[0] * inv, acc[1] * inv);
+        }
+    }
+    if (lane == 0 && lse != nullptr) lse[r] = (sum > 0.f) ? mx + log2f(sum) * kLn2 : -INFINITY;
+}
+
+}  // namespace kvb

@@ -26,6 +26,7 @@ struct EvictParams {
     const int* t;
     int Hkv, d, cap, M;
     int* victim;
+    int vec4;  // pos/log_beta rows start 16-byte aligned (cap % 4 == 0, aligned bases)
 };
 
 __device__ __forceinline__ void argmin_merge(unsigned long long& key, int& slot, unsigned long long k2, int s2) {
@@ -62,14 +63,41 @@ __global__ void __launch_bounds__(NT) evict_insert_kernel(const __grid_constant_
         const float* lb = p.lb ? p.lb + base : nullptr;
         unsigned long long best = ~0ull;
         int best_slot = 0x7fffffff;
-#pragma unroll 4
-        for (int s = tid; s < n; s += NT) {
-            const int ps_s = ps[s];
-            const float sc = lb ? __fmul_rn(__int2float_rn(tb - ps_s), lb[s]) : 0.f;
+        auto consider = [&](int s, int ps_s, float l) {
+            const float sc = lb ? __fmul_rn(__int2float_rn(tb - ps_s), l) : 0.f;
             const unsigned long long key =
                 ((unsigned long long)float_order_key(sc) << 32) | (unsigned)(ps_s ^ 0x80000000);
             argmin_merge(best, best_slot, key, s);
+        };
+        int s_done = 0;
+        if (p.vec4) {  // 16-byte loads: four slots per load, all issued before the compares
+            const int n4 = n / 4;
+            constexpr int U = 4;
+            for (int base = 0; base < n4; base += U * NT) {
+                int4 pv[U];
+                float4 lv[U];
+#pragma unroll
+                for (int k = 0; k < U; ++k) {
+                    const int v = base + k * NT + tid;
+                    if (v < n4) {
+                        pv[k] = reinterpret_cast<const int4*>(ps)[v];
+                        lv[k] = lb ? reinterpret_cast<const float4*>(lb)[v] : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < U; ++k) {
+                    const int v = base + k * NT + tid;
+                    if (v < n4) {
+                        consider(4 * v, pv[k].x, lv[k].x);
+                        consider(4 * v + 1, pv[k].y, lv[k].y);
+                        consider(4 * v + 2, pv[k].z, lv[k].z);
+                        consider(4 * v + 3, pv[k].w, lv[k].w);
+                    }
+                }
+            }
+            s_done = n4 * 4;
         }
+        for (int s = s_done + tid; s < n; s += NT) consider(s, ps[s], lb ? lb[s] : 0.f);
 #pragma unroll
         for (int m = 16; m >= 1; m >>= 1) {
             const unsigned long long k2 = __shfl_xor_sync(kFull, best, m);

@@ -5,13 +5,14 @@
 #include <cstdint>
 #include <map>
 #include <mutex>
+#include <tuple>
 #include <utility>
 
 #include "../../include/kvb.h"
 #include "asm_lookup.cuh"
 #include "common.cuh"
 #include "compact_blocks.cuh"
-#include "decode_attn.cuh"
+#include "decode_attn_tc.cuh"
 #include "evict_insert.cuh"
 #include "merge_states.cuh"
 
@@ -39,35 +40,104 @@ kvb_status set_smem(Kern kern, size_t bytes) {
     return KVB_OK;
 }
 
+// ---- tensor maps (driver entry point, no link against libcuda) -------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+
+// 4-D view (d, slot, kv head, sequence) of a [B, Hkv, cap, d] bf16 cache, loaded in boxes of
+// 64 dims x `rows` slots with the 128-byte swizzle.
+bool make_kv_map(CUtensorMap* map, const void* base, int d, int cap, int Hkv, int Bk, long long kv_sh,
+                 long long kv_sb, int rows) {
+    EncodeTiledFn fn = encode_tiled();
+    if (fn == nullptr) return false;
+    const cuuint64_t row_bytes = (cuuint64_t)d * 2;
+    const cuuint64_t sh = (Hkv == 1 && kv_sh == 0) ? row_bytes * cap : (cuuint64_t)kv_sh * 2;
+    const cuuint64_t sb = (Bk == 1) ? sh * Hkv : (cuuint64_t)kv_sb * 2;
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)cap, (cuuint64_t)Hkv, (cuuint64_t)Bk};
+    cuuint64_t strides[3] = {row_bytes, sh, sb};
+    cuuint32_t box[4] = {64, (cuuint32_t)rows, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Resident CTAs the device holds for a kernel (SMs x blocks per SM), once per (kernel, smem, device).
+template <typename Kern>
+int resident_ctas(Kern kern, int threads, size_t smem) {
+    static std::mutex mu;
+    static std::map<std::tuple<const void*, size_t, int>, int> cache;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    auto key = std::make_tuple(reinterpret_cast<const void*>(kern), smem, dev);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+    int sms = 0, per_sm = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess) return 0;
+    const int n = sms * (per_sm > 0 ? per_sm : 1);
+    cache[key] = n;
+    return n;
+}
+
 template <int D, int G, bool BIAS>
-kvb_status launch_decode(const kvb::DecodeParams& p, int B, cudaStream_t st) {
-    using SH = kvb::DecodeShape<D, G>;
-    auto kern = kvb::decode_attn_kernel<D, G, BIAS>;
-    const size_t smem = SH::smem_bytes(p.S);
+kvb_status launch_decode_tc(const kvb::DecodeTcParams& p, const kvb_attn_args* a, cudaStream_t st) {
+    using SH = kvb::TcShape<D, G>;
+    auto kern = kvb::decode_attn_tc_kernel<D, G, BIAS>;
+    const size_t smem = SH::SMEM;
     if (set_smem(kern, smem) != KVB_OK) return KVB_ECUDA;
-    kern<<<dim3(p.S, p.Hkv, B), SH::NT, smem, st>>>(p);
-    return launched();
+    CUtensorMap mk, mv;
+    const int Bk = p.kv_shared ? 1 : a->B;
+    if (!make_kv_map(&mk, a->k, D, a->cap, a->Hkv, Bk, a->kv_stride_h, a->kv_stride_b, SH::T) ||
+        !make_kv_map(&mv, a->v, D, a->cap, a->Hkv, Bk, a->kv_stride_h, a->kv_stride_b, SH::T))
+        return KVB_EINVAL;
+    const int slots = resident_ctas(kern, SH::NT, smem);
+    if (slots <= 0) return KVB_ECUDA;
+    const int grid = p.units < slots ? p.units : slots;
+    kern<<<grid, SH::NT, smem, st>>>(p, mk, mv);
+    if (launched() != KVB_OK) return KVB_ECUDA;
+    if (p.S > 1) {
+        const int R = a->B * a->Hq;
+        kvb::merge_splits_kernel<D><<<(R + 7) / 8, 256, 0, st>>>(p.o_part, p.lse_part, R, p.S, p.o, p.o_bf16, p.lse);
+        return launched();
+    }
+    return KVB_OK;
 }
 
 template <int D, int G>
-kvb_status dispatch_bias(const kvb::DecodeParams& p, int B, bool bias, cudaStream_t st) {
-    return bias ? launch_decode<D, G, true>(p, B, st) : launch_decode<D, G, false>(p, B, st);
+kvb_status tc_bias(const kvb::DecodeTcParams& p, const kvb_attn_args* a, bool bias, cudaStream_t st) {
+    return bias ? launch_decode_tc<D, G, true>(p, a, st) : launch_decode_tc<D, G, false>(p, a, st);
 }
 
 template <int D>
-kvb_status dispatch_g(const kvb::DecodeParams& p, int B, int G, bool bias, cudaStream_t st) {
+kvb_status tc_g(const kvb::DecodeTcParams& p, const kvb_attn_args* a, int G, bool bias, cudaStream_t st) {
     switch (G) {
-        case 1: return dispatch_bias<D, 1>(p, B, bias, st);
-        case 2: return dispatch_bias<D, 2>(p, B, bias, st);
-        case 4: return dispatch_bias<D, 4>(p, B, bias, st);
-        case 8: return dispatch_bias<D, 8>(p, B, bias, st);
+        case 1: return tc_bias<D, 1>(p, a, bias, st);
+        case 2: return tc_bias<D, 2>(p, a, bias, st);
+        case 4: return tc_bias<D, 4>(p, a, bias, st);
+        case 8: return tc_bias<D, 8>(p, a, bias, st);
         default: return KVB_EINVAL;
     }
 }
 
 // ---- fixed scratch of kvb_decode_attn_noalloc ------------------------------
-// The split states and ticket counters of the no-allocation entry point live
-// here instead of in caller memory. Host code must not use the symbol itself
+// The split states of the no-allocation entry point live here instead of in
+// caller memory. Host code must not use the symbol itself
 // as a device address: it is a host-side stand-in. The device address is
 // looked up once per device with cudaGetSymbolAddress (that device current).
 static __device__ __align__(256) unsigned char g_noalloc_scratch[KVB_NOALLOC_SCRATCH_BYTES];
@@ -136,21 +206,26 @@ kvb_status kvb_decode_attn(const kvb_attn_args* a, kvb_stream stream) {
     if (bias && (!a->pos || !a->t)) return KVB_EINVAL;
     if (bias && (a->meta_stride_b < 0 || a->meta_stride_h < 0)) return KVB_EINVAL;
     if (a->o_dtype != KVB_OUT_F32 && a->o_dtype != KVB_OUT_BF16) return KVB_EINVAL;
-    if (a->num_splits > 1 && (!a->o_part || !a->lse_part || !a->counters)) return KVB_EINVAL;
+    if (a->num_splits > 1 && (!a->o_part || !a->lse_part)) return KVB_EINVAL;
     if ((a->o_part == nullptr) != (a->lse_part == nullptr)) return KVB_EINVAL;
 
-    kvb::DecodeParams p;
+    if (a->Hkv > 1 && a->kv_stride_h == 0) return KVB_EINVAL;
+    const long long units = (long long)a->B * a->Hkv * a->num_splits;
+    if (units > 0x7fffffffLL) return KVB_EINVAL;
+
+    kvb::DecodeTcParams p;
     p.q = a->q; p.q_sb = a->q_stride_b; p.q_sh = a->q_stride_h;
-    p.k = a->k; p.v = a->v; p.kv_sb = a->kv_stride_b; p.kv_sh = a->kv_stride_h;
     p.lb = a->log_beta; p.pos = a->pos; p.m_sb = a->meta_stride_b; p.m_sh = a->meta_stride_h;
     p.len = a->len; p.t = a->t;
     p.Hq = a->Hq; p.Hkv = a->Hkv; p.cap = a->cap; p.S = a->num_splits; p.split_len = a->split_len;
+    p.units = (int)units;
+    p.kv_shared = (a->kv_stride_b == 0 && a->B > 1) ? 1 : 0;
     const double scale = (a->scale == 0.0f) ? 1.0 / std::sqrt((double)a->d) : (double)a->scale;
-    p.qscale = (float)scale;
-    p.o_part = a->o_part; p.lse_part = a->lse_part; p.counters = a->counters;
+    p.scale = (float)scale;
+    p.o_part = a->o_part; p.lse_part = a->lse_part;
     p.o = a->o; p.o_bf16 = (a->o_dtype == KVB_OUT_BF16); p.lse = a->lse;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    return a->d == 128 ? dispatch_g<128>(p, a->B, G, bias, st) : dispatch_g<64>(p, a->B, G, bias, st);
+    return a->d == 128 ? tc_g<128>(p, a, G, bias, st) : tc_g<64>(p, a, G, bias, st);
 }
 
 kvb_status kvb_decode_attn_noalloc(const kvb_attn_args* a, kvb_stream stream) {
@@ -162,21 +237,16 @@ kvb_status kvb_decode_attn_noalloc(const kvb_attn_args* a, kvb_stream stream) {
             a->B > 65535 || a->Hkv > 65535 || a->Hq > 65535)
             return KVB_EINVAL;
         const size_t rows = (size_t)a->B * a->Hq * a->num_splits;
-        const size_t cnt_bytes = (size_t)a->B * a->Hkv * sizeof(uint32_t);
-        const size_t lse_off = round256(cnt_bytes);
-        const size_t o_off = lse_off + round256(rows * sizeof(float));
+        const size_t o_off = round256(rows * sizeof(float));
         const size_t need = o_off + rows * a->d * sizeof(float);
         if (need > (size_t)KVB_NOALLOC_SCRATCH_BYTES) return KVB_EINVAL;
         void* base = nullptr;
         const kvb_status st = noalloc_scratch(&base);
         if (st != KVB_OK) return st;
+        // every call writes all the split states it reads back: nothing needs clearing
         unsigned char* s = static_cast<unsigned char*>(base);
-        b.counters = reinterpret_cast<uint32_t*>(s);
-        b.lse_part = reinterpret_cast<float*>(s + lse_off);
+        b.lse_part = reinterpret_cast<float*>(s);
         b.o_part = reinterpret_cast<float*>(s + o_off);
-        // the array keeps the last call's contents: the ticket counters must start at zero
-        if (cudaMemsetAsync(b.counters, 0, cnt_bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
-            return KVB_ECUDA;
     }
     return kvb_decode_attn(&b, stream);
 }
@@ -211,7 +281,8 @@ kvb_status kvb_evict_insert(uint16_t* k, uint16_t* v, float* log_beta, int32_t* 
     if (k_new && (!k || !v || !aligned16(k) || !aligned16(v) || !aligned16(k_new) || !aligned16(v_new)))
         return KVB_EINVAL;
     if (log_beta && !log_beta_new) return KVB_EINVAL;
-    kvb::EvictParams p{k, v, log_beta, pos, len, k_new, v_new, log_beta_new, t, Hkv, d, cap, M, victim};
+    const int vec4 = (cap % 4 == 0) && aligned16(pos) && (log_beta == nullptr || aligned16(log_beta)) ? 1 : 0;
+    kvb::EvictParams p{k, v, log_beta, pos, len, k_new, v_new, log_beta_new, t, Hkv, d, cap, M, victim, vec4};
     kvb::evict_insert_kernel<256><<<B * Hkv, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
     return launched();
 }
