@@ -100,6 +100,15 @@ enum kvb_device_error {
  *            writes every split's state, and a merge kernel that combines
  *            them into o and lse.
  *   counters reserved; ignored (may be NULL).
+ *   evict_cand  [B, Hkv, num_splits] kvb_evict_cand records, may be NULL.
+ *            When given, the kernel also writes, for every split, the slot
+ *            that budget enforcement at the NEXT position t[b] + 1 would pick
+ *            within the split (the smallest (score, pos) with score =
+ *            (float)(t[b] + 1 - pos) * log_beta, or 0 when log_beta is NULL;
+ *            slot -1 for an empty split). It reads those fields anyway, so
+ *            kvb_evict_insert can then skip its scan of the whole cache.
+ *            Needs pos and t (and meta strides describing pos), 16-byte
+ *            alignment; else KVB_EINVAL.
  *
  * Requirements (else KVB_EINVAL): d in {64, 128}; Hq % Hkv == 0 and
  * Hq / Hkv in {1, 2, 4, 8}; B, Hkv, cap >= 1; 1 <= num_splits <= 1024;
@@ -132,7 +141,15 @@ typedef struct kvb_attn_args {
     void* o;
     int32_t o_dtype;
     float* lse;
+    void* evict_cand;
 } kvb_attn_args;
+
+/* Eviction candidate of one split (see evict_cand / kvb_evict_insert). */
+typedef struct kvb_evict_cand {
+    uint64_t key;   /* order-preserving key of (score, pos) */
+    int32_t slot;   /* -1 for an empty split */
+    int32_t reserved;
+} kvb_evict_cand;
 
 kvb_status kvb_decode_attn(const kvb_attn_args* args, kvb_stream stream);
 
@@ -210,6 +227,13 @@ kvb_status kvb_merge_states(const float* o_in, const float* lse_in,
  * log_beta is NULL) and pos = t[b].
  * Cache layout: k, v [B, Hkv, cap, d], log_beta, pos [B, Hkv, cap], len
  * [B, Hkv], all contiguous. victim [B, Hkv] int32 (may be NULL).
+ * cand, cand_n: optional [B, Hkv, cand_n] kvb_evict_cand records written by
+ * the kvb_decode_attn call that immediately preceded this one on the same
+ * cache (same scoring: both with or both without log_beta), for position
+ * t[b] - 1. When len >= M the victim is then the best record -- the same
+ * slot a full scan picks, because the splits partition the slots -- and
+ * the scan is skipped; a record set with no usable slot falls back to the
+ * scan. 16-byte aligned, 1 <= cand_n <= 1024. NULL: always scan.
  * Requirements: d in [1, 1024] with d % 8 == 0 and k/v/k_new/v_new 16-byte
  * aligned; 1 <= M <= cap. Device-side check: len in [0, cap].
  * ---------------------------------------------------------------------- */
@@ -217,7 +241,7 @@ kvb_status kvb_evict_insert(uint16_t* k, uint16_t* v, float* log_beta, int32_t* 
                             int32_t* len, const uint16_t* k_new, const uint16_t* v_new,
                             const float* log_beta_new, const int32_t* t,
                             int32_t B, int32_t Hkv, int32_t d, int32_t cap, int32_t M,
-                            int32_t* victim, kvb_stream stream);
+                            int32_t* victim, const void* cand, int32_t cand_n, kvb_stream stream);
 
 /* ------------------------------------------------------------------------
  * kvb_compact_blocks -- in-place removal of a slot range

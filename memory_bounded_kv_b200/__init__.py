@@ -20,7 +20,7 @@ from . import _lib
 __all__ = [
     "KvbError", "kvb_decode_attn", "kvb_decode_attn_noalloc", "kvb_merge_states", "kvb_evict_insert", "kvb_compact_blocks",
     "kvb_asm_workspace_bytes", "kvb_asm_lookup_merge", "kvb_get_error", "kvb_abi_version",
-    "decode_workspace",
+    "decode_workspace", "evict_candidates",
 ]
 
 
@@ -78,6 +78,19 @@ def kvb_get_error(stream=None) -> int:
     return int(bits.value)
 
 
+def evict_candidates(B: int, Hkv: int, num_splits: int, device="cuda"):
+    """Buffer of B*Hkv*num_splits kvb_evict_cand records (16 bytes each) as an int64 tensor."""
+    return torch.empty(B * Hkv * num_splits * 2, dtype=torch.int64, device=device)
+
+
+def _cand_ptr(c, records):
+    if not isinstance(c, torch.Tensor) or not c.is_cuda or not c.is_contiguous():
+        raise TypeError("evict candidates must be a contiguous CUDA tensor")
+    if c.numel() * c.element_size() < records * _lib.EVICT_CAND_BYTES:
+        raise ValueError("evict candidate buffer too small")
+    return c.data_ptr()
+
+
 def decode_workspace(B: int, Hq: int, Hkv: int, d: int, num_splits: int, device="cuda"):
     """Zero-filled (o_part, lse_part, counters) buffers for kvb_decode_attn with num_splits > 1."""
     o_part = torch.zeros(B, Hq, num_splits, d, dtype=torch.float32, device=device)
@@ -88,14 +101,16 @@ def decode_workspace(B: int, Hq: int, Hkv: int, d: int, num_splits: int, device=
 
 def kvb_decode_attn(q, k, v, log_beta, pos, len, t, o, lse=None, *, scale: float = 0.0,
                     num_splits: int = 1, split_len: int = 0, o_part=None, lse_part=None, counters=None,
-                    stream=None) -> None:
+                    evict_cand=None, stream=None) -> None:
     """Split-K GQA decode attention with retention bias; see kvb_decode_attn in include/kvb.h.
 
     q [B, Hq, d] bf16; k, v [B, Hkv, cap, d] bf16 (stride(2) == d, stride(3) == 1; an expanded
     view with stride(0) == 0 shares one cache); log_beta [B, Hkv, cap] f32 or None; pos
     [B, Hkv, cap] int32 (same strides as log_beta); len [B, Hkv] int32; t [B] int32 or None;
-    o [B, Hq, d] f32 or bf16; lse [B, Hq] f32 or None; o_part/lse_part/counters from
-    decode_workspace() when num_splits > 1.
+    o [B, Hq, d] f32 or bf16; lse [B, Hq] f32 or None; o_part/lse_part from
+    decode_workspace() when num_splits > 1 (counters is accepted and ignored); evict_cand: a
+    CUDA tensor of >= B*Hkv*num_splits*16 bytes to receive the next position's eviction
+    candidates (see evict_candidates()), or None.
     """
     _need(q, torch.bfloat16, "q"); _need(k, torch.bfloat16, "k"); _need(v, torch.bfloat16, "v")
     B, Hq, d = q.shape
@@ -105,7 +120,7 @@ def kvb_decode_attn(q, k, v, log_beta, pos, len, t, o, lse=None, *, scale: float
     if q.stride(2) != 1 or k.stride(3) != 1 or k.stride(2) != d or v.stride() != k.stride():
         raise ValueError("q/k/v: innermost dim contiguous, slot stride d, k and v with equal strides")
     _need(len, torch.int32, "len"); _contig(len, "len")
-    meta = None
+    meta = None   # the tensor whose strides describe log_beta and pos
     if log_beta is not None:
         _need(log_beta, torch.float32, "log_beta")
         _need(pos, torch.int32, "pos")
@@ -113,6 +128,11 @@ def kvb_decode_attn(q, k, v, log_beta, pos, len, t, o, lse=None, *, scale: float
             raise ValueError("log_beta and pos need equal strides with slot stride 1")
         _need(t, torch.int32, "t")
         meta = log_beta
+    elif pos is not None:
+        _need(pos, torch.int32, "pos")
+        if pos.stride(2) != 1:
+            raise ValueError("pos needs slot stride 1")
+        meta = pos
     if t is not None:
         _need(t, torch.int32, "t"); _contig(t, "t")
     if o.dtype == torch.float32:
@@ -131,7 +151,7 @@ def kvb_decode_attn(q, k, v, log_beta, pos, len, t, o, lse=None, *, scale: float
     a = _lib.AttnArgs(
         q=q.data_ptr(), q_stride_b=q.stride(0), q_stride_h=q.stride(1),
         k=k.data_ptr(), v=v.data_ptr(), kv_stride_b=k.stride(0), kv_stride_h=k.stride(1),
-        log_beta=None if meta is None else log_beta.data_ptr(),
+        log_beta=None if log_beta is None else log_beta.data_ptr(),
         pos=None if pos is None else pos.data_ptr(),
         meta_stride_b=0 if meta is None else meta.stride(0), meta_stride_h=0 if meta is None else meta.stride(1),
         len=len.data_ptr(), t=None if t is None else t.data_ptr(),
@@ -140,7 +160,8 @@ def kvb_decode_attn(q, k, v, log_beta, pos, len, t, o, lse=None, *, scale: float
         o_part=None if o_part is None else o_part.data_ptr(),
         lse_part=None if lse_part is None else lse_part.data_ptr(),
         counters=None if counters is None else counters.data_ptr(),
-        o=o.data_ptr(), o_dtype=odt, lse=None if lse is None else lse.data_ptr())
+        o=o.data_ptr(), o_dtype=odt, lse=None if lse is None else lse.data_ptr(),
+        evict_cand=None if evict_cand is None else _cand_ptr(evict_cand, B * Hkv * int(num_splits)))
     _check(_lib.lib().kvb_decode_attn(ctypes.byref(a), _stream(stream)), "kvb_decode_attn")
 
 
@@ -181,8 +202,8 @@ def kvb_decode_attn_noalloc(q, k, v, log_beta, pos, len, t, o, lse=None, *, scal
         k=k.data_ptr(), v=v.data_ptr(), kv_stride_b=k.stride(0), kv_stride_h=k.stride(1),
         log_beta=None if log_beta is None else log_beta.data_ptr(),
         pos=None if pos is None else pos.data_ptr(),
-        meta_stride_b=0 if log_beta is None else log_beta.stride(0),
-        meta_stride_h=0 if log_beta is None else log_beta.stride(1),
+        meta_stride_b=0 if pos is None else pos.stride(0),
+        meta_stride_h=0 if pos is None else pos.stride(1),
         len=len.data_ptr(), t=None if t is None else t.data_ptr(),
         B=B, Hq=Hq, Hkv=Hkv, d=d, cap=cap, scale=float(scale),
         num_splits=int(num_splits), split_len=int(split_len), o_part=None, lse_part=None, counters=None,
@@ -207,9 +228,10 @@ def kvb_merge_states(o_in, lse_in, o_out, lse_out=None, *, stream=None) -> None:
 
 
 def kvb_evict_insert(k, v, log_beta, pos, len, k_new, v_new, log_beta_new, t, M: int, victim=None, *,
-                     stream=None) -> None:
+                     cand=None, cand_n: int = 0, stream=None) -> None:
     """Budget enforcement + insertion (in place); see kvb_evict_insert in include/kvb.h.
-    k_new/v_new may both be None (only log_beta and pos are written)."""
+    k_new/v_new may both be None (only log_beta and pos are written); cand/cand_n: the
+    candidates of the immediately preceding kvb_decode_attn on this cache, or None."""
     for name, x in (("k", k), ("v", v)):
         _need(x, torch.bfloat16, name); _contig(x, name)
     _need(pos, torch.int32, "pos"); _contig(pos, "pos")
@@ -224,9 +246,11 @@ def kvb_evict_insert(k, v, log_beta, pos, len, k_new, v_new, log_beta_new, t, M:
             _need(x, torch.bfloat16, name); _contig(x, name)
     if victim is not None:
         _need(victim, torch.int32, "victim"); _contig(victim, "victim")
+    cp = None if cand is None else ctypes.c_void_p(_cand_ptr(cand, B * Hkv * int(cand_n)))
     _check(_lib.lib().kvb_evict_insert(_ptr(k), _ptr(v), _ptr(log_beta), _ptr(pos), _ptr(len), _ptr(k_new),
                                        _ptr(v_new), _ptr(log_beta_new), _ptr(t), B, Hkv, d, cap, int(M),
-                                       _ptr(victim), _stream(stream)), "kvb_evict_insert")
+                                       _ptr(victim), cp, int(cand_n) if cand is not None else 0,
+                                       _stream(stream)), "kvb_evict_insert")
 
 
 def kvb_compact_blocks(k, v, pos, log_beta, len, rm_start, rm_len, *, stream=None) -> None:

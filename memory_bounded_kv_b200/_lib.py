@@ -36,7 +36,10 @@ class AttnArgs(ctypes.Structure):
         ("num_splits", _I32), ("split_len", _I32),
         ("o_part", _P), ("lse_part", _P), ("counters", _P),
         ("o", _P), ("o_dtype", _I32), ("lse", _P),
+        ("evict_cand", _P),
     ]
+
+EVICT_CAND_BYTES = 16   # sizeof(kvb_evict_cand)
 
 
 _lib = None
@@ -58,7 +61,8 @@ def lib() -> ctypes.CDLL:
         L.kvb_decode_attn.argtypes = [ctypes.POINTER(AttnArgs), _P]
         L.kvb_decode_attn_noalloc.argtypes = [ctypes.POINTER(AttnArgs), _P]
         L.kvb_merge_states.argtypes = [_P, _P, _I64, _I64, _I64, _I64, _I32, _I32, _I32, _P, _P, _P]
-        L.kvb_evict_insert.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _P, _P]
+        L.kvb_evict_insert.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _P, _P,
+                                       _I32, _P]
         L.kvb_compact_blocks.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _P]
         L.kvb_asm_workspace_bytes.argtypes = [_I32, _I32, _I32]
         L.kvb_asm_workspace_bytes.restype = _SZ

@@ -12,7 +12,7 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import kvb_compact_blocks, kvb_decode_attn, kvb_evict_insert, decode_workspace
+from . import kvb_compact_blocks, kvb_decode_attn, kvb_evict_insert, decode_workspace, evict_candidates
 
 
 def _dev(a, device):
@@ -39,6 +39,9 @@ class BoundedKVCache:
         self.o_part = self.lse_part = self.counters = None
         if num_splits > 1:
             self.o_part, self.lse_part, self.counters = decode_workspace(B, Hq, Hkv, d, num_splits, device)
+        # eviction candidates for the next position, left by each attention pass
+        self.cand = evict_candidates(B, Hkv, num_splits, device)
+        self.cand_valid = False
 
     @classmethod
     def from_host(cls, k, v, log_beta, pos, len_, Hq, M, num_splits=1, split_len=0, device="cuda"):
@@ -53,14 +56,24 @@ class BoundedKVCache:
         return c
 
     def insert(self, k_new, v_new, log_beta_new, t, stream=None):
+        """Budget enforcement + insertion at position t. Uses the candidates of the attention at
+        t - 1 when the last operation on the cache was that attention (the decode-step order)."""
         kvb_evict_insert(self.k, self.v, self.log_beta, self.pos, self.len, k_new, v_new,
-                         log_beta_new if self.log_beta is not None else None, t, self.M, self.victim, stream=stream)
+                         log_beta_new if self.log_beta is not None else None, t, self.M, self.victim,
+                         cand=self.cand if self.cand_valid else None, cand_n=self.num_splits, stream=stream)
+        self.cand_valid = False
 
     def attend(self, q, t, o, lse=None, stream=None, use_beta=True):
         lb = self.log_beta if use_beta else None
+        # candidates use the cache's own eviction score: only an attention with the same scoring
+        # (bias on a retention cache, plain on a plain cache) can leave them
+        same_scoring = (lb is not None) == (self.log_beta is not None)
+        cand = self.cand if (same_scoring and t is not None) else None
         kvb_decode_attn(q, self.k, self.v, lb, self.pos, self.len, t if (lb is not None or t is not None) else None,
                         o, lse, num_splits=self.num_splits, split_len=self.split_len, o_part=self.o_part,
-                        lse_part=self.lse_part, counters=self.counters, stream=stream)
+                        lse_part=self.lse_part, counters=self.counters, evict_cand=cand, stream=stream)
+        if cand is not None:
+            self.cand_valid = True
 
     def step(self, q, k_new, v_new, log_beta_new, t, o, lse=None, stream=None):
         """One decode step: budget enforcement + insertion, then attention (2 launches)."""
@@ -69,6 +82,7 @@ class BoundedKVCache:
 
     def compact(self, rm_start, rm_len, stream=None):
         kvb_compact_blocks(self.k, self.v, self.pos, self.log_beta, self.len, rm_start, rm_len, stream=stream)
+        self.cand_valid = False
 
     def kv_bytes_read(self) -> int:
         """Bytes of K, V (and log_beta, pos when the bias is on) that one attention pass reads."""

@@ -113,6 +113,23 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     return pol;
 }
 
+// Programmatic dependent launch: wait until the previous kernel in the stream
+// has completed and its writes are visible (a no-op when the launch did not
+// ask for programmatic serialization), and allow the next kernel to launch.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// One eviction candidate: the best (order key of the score << 32 | order key
+// of the position) of a slot range, with its slot (-1 when the range is empty).
+struct EvictCand {
+    unsigned long long key;
+    int slot;
+    int pad;
+};
+static_assert(sizeof(EvictCand) == 16, "candidate record");
+
 // Order-preserving map of a float's bits to an unsigned key (for a, b not NaN:
 // a < b  <=>  key(a) < key(b)); -0 is mapped like +0.
 __device__ __forceinline__ unsigned float_order_key(float f) {

@@ -56,6 +56,7 @@ struct DecodeTcParams {
     void* o;
     int o_bf16;
     float* lse;
+    EvictCand* cand;  // nullable: per-split eviction candidates for position t + 1
 };
 
 template <int D, int G>
@@ -75,12 +76,15 @@ struct TcShape {
     static constexpr int RING_OFF = 0;
     static constexpr int Q_OFF = RING_OFF + STAGES * STAGE_BYTES;       // [ST][G][D] bf16
     static constexpr int BIAS_OFF = Q_OFF + STAGES * QBYTES;            // [ST][T] f32
-    static constexpr int META_OFF = BIAS_OFF + STAGES * T * 4;          // [ST][8] int
-    static constexpr int BAR_OFF = META_OFF + STAGES * 32;              // full[ST], empty[ST]
+    static constexpr int CPOS_OFF = BIAS_OFF + STAGES * T * 4;          // [ST][T] int (pos, for candidates)
+    static constexpr int CLB_OFF = CPOS_OFF + STAGES * T * 4;           // [ST][T] f32 (log beta)
+    static constexpr int META_OFF = CLB_OFF + STAGES * T * 4;           // [ST][16] int
+    static constexpr int BAR_OFF = META_OFF + STAGES * 64;              // full[ST], empty[ST]
     static constexpr int MISC_OFF = BAR_OFF + 2 * STAGES * 8;           // abort, issued
     static constexpr int EPI_OFF = (MISC_OFF + 16 + 15) / 16 * 16;      // [NWC][G][D] f32
     static constexpr int ML_OFF = EPI_OFF + NWC * G * D * 4;            // [NWC][G][2] f32
-    static constexpr int END_OFF = ML_OFF + NWC * G * 2 * 4;
+    static constexpr int CAND_OFF = ML_OFF + NWC * G * 2 * 4;           // [NWC] (key, slot)
+    static constexpr int END_OFF = CAND_OFF + NWC * 16;
     static constexpr size_t SMEM = 1024 + END_OFF;
     static_assert(D == 64 || D == 128, "d");
     static_assert(G == 1 || G == 2 || G == 4 || G == 8, "G");
@@ -195,6 +199,10 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
     uint16_t* s_q = reinterpret_cast<uint16_t*>(smem + SH::Q_OFF);
     float* s_bias = reinterpret_cast<float*>(smem + SH::BIAS_OFF);
     int* s_meta = reinterpret_cast<int*>(smem + SH::META_OFF);
+    int* s_pos = reinterpret_cast<int*>(smem + SH::CPOS_OFF);
+    float* s_lb = reinterpret_cast<float*>(smem + SH::CLB_OFF);
+    unsigned long long* s_ck = reinterpret_cast<unsigned long long*>(smem + SH::CAND_OFF);
+    int* s_cs = reinterpret_cast<int*>(smem + SH::CAND_OFF + NWC * 8);
     uint64_t* s_full = reinterpret_cast<uint64_t*>(smem + SH::BAR_OFF);
     uint64_t* s_empty = s_full + ST;
     volatile int* s_abort = reinterpret_cast<int*>(smem + SH::MISC_OFF);
@@ -203,6 +211,8 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
     float* s_ml = reinterpret_cast<float*>(smem + SH::ML_OFF);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    griddep_wait();  // the previous kernel in the stream (e.g. the insertion) has finished writing
+    griddep_launch_dependents();
     if (tid == 0) {
         for (int s = 0; s < ST; ++s) {
             mbar_init(&s_full[s], 33);          // producer lane 0's expect_tx + 32 producer lanes
@@ -225,20 +235,58 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
             next_raw = unit_raw(p, u + gridDim.x);  // in flight while this unit's tiles are issued
             UnitInfo ui{};
             if (!end) ui = unit_info<T>(p, u, raw, lane == 0);
-            const int records = end ? 1 : max(ui.ntiles, 1);
+            if (!end && ui.ntiles == 0) {
+                // an empty split (ragged lengths, inactive rows): write its empty state here;
+                // no record reaches the consumers
+                const size_t row0 = (size_t)ui.b * p.Hq + ui.g * G;
+                if (p.o_part != nullptr) {
+                    for (int idx = lane; idx < G * D / 4; idx += 32) {
+                        const int hh = idx / (D / 4), e4 = idx % (D / 4);
+                        reinterpret_cast<float4*>(p.o_part + ((row0 + hh) * p.S + ui.split) * D)[e4] =
+                            make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+                    if (lane < G) p.lse_part[(row0 + lane) * p.S + ui.split] = -INFINITY;
+                }
+                if (p.S == 1) {
+                    for (int idx = lane; idx < G * D; idx += 32) {
+                        const size_t oi = row0 * D + idx;
+                        if (p.o_bf16) {
+                            reinterpret_cast<__nv_bfloat16*>(p.o)[oi] = __float2bfloat16_rn(0.f);
+                        } else {
+                            reinterpret_cast<float*>(p.o)[oi] = 0.f;
+                        }
+                    }
+                    if (lane < G && p.lse != nullptr) p.lse[row0 + lane] = -INFINITY;
+                }
+                if (lane == 0 && p.cand != nullptr) {
+                    EvictCand* c = p.cand + ((size_t)ui.b * p.Hkv + ui.g) * p.S + ui.split;
+                    c->key = ~0ull;
+                    c->slot = -1;
+                }
+                continue;
+            }
+            const int records = end ? 1 : ui.ntiles;
             const int tb = raw.t;
             const size_t m_off = end ? 0 : (size_t)ui.b * p.m_sb + (size_t)ui.g * p.m_sh + (size_t)ui.s0;
+            const bool want_cand = p.cand != nullptr;
             for (int i = 0; i < records; ++i, ++it) {
                 const int st = it % ST;
-                // this tile's bias, loaded before waiting for the stage
+                // this tile's bias (and, for the eviction candidates, its pos and log beta),
+                // loaded before waiting for the stage
                 float bias[T / 32];
+                int psv[T / 32];
+                float lbv[T / 32];
 #pragma unroll
                 for (int j = 0; j < T / 32; ++j) {
                     const int key = i * T + lane + 32 * j;
                     float bv = -INFINITY;
+                    psv[j] = 0;
+                    lbv[j] = 0.f;
                     if (!end && key < ui.nk) {
+                        if (BIAS || want_cand) psv[j] = p.pos[m_off + key];
                         if constexpr (BIAS) {
-                            bv = __fmul_rn(__int2float_rn(tb - p.pos[m_off + key]), p.lb[m_off + key]);
+                            lbv[j] = p.lb[m_off + key];
+                            bv = __fmul_rn(__int2float_rn(tb - psv[j]), lbv[j]);
                         } else {
                             bv = 0.f;
                         }
@@ -259,7 +307,7 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                 }
                 const bool data = !end && ui.ntiles > 0;
                 if (lane == 0) {
-                    int* m = s_meta + st * 8;
+                    int* m = s_meta + st * 16;
                     m[0] = end ? -1 : u;
                     m[1] = i;
                     m[2] = end ? 0 : ui.ntiles;
@@ -268,6 +316,8 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                     m[5] = ui.g;
                     m[6] = ui.split;
                     m[7] = ui.n;
+                    m[8] = tb;
+                    m[9] = ui.s0 + i * T;
                     unsigned tx = data ? (unsigned)SH::STAGE_BYTES : 0u;
                     const bool with_q = data && i == 0;
                     if (with_q) tx += SH::QBYTES;
@@ -295,7 +345,13 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                     }
                 }
 #pragma unroll
-                for (int j = 0; j < T / 32; ++j) s_bias[st * T + lane + 32 * j] = bias[j];
+                for (int j = 0; j < T / 32; ++j) {
+                    s_bias[st * T + lane + 32 * j] = bias[j];
+                    if (want_cand) {
+                        s_pos[st * T + lane + 32 * j] = psv[j];
+                        s_lb[st * T + lane + 32 * j] = lbv[j];
+                    }
+                }
                 __syncwarp();
                 mbar_arrive(&s_full[st]);
             }
@@ -317,6 +373,9 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
         uint32_t qa[SH::KSTEPS][2];
         float acc[SH::NTILES][4];
         float m_run = -INFINITY, l_run = 0.f;
+        const bool want_cand = p.cand != nullptr;
+        unsigned long long cand_key = ~0ull;  // this lane's best eviction key in the unit
+        int cand_slot = 0x7fffffff;
         int it = 0;
         bool aborted = false;
         while (true) {
@@ -329,10 +388,27 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                 aborted = true;
                 break;
             }
-            const int* m = s_meta + st * 8;
+            const int* m = s_meta + st * 16;
             const int u = m[0], i = m[1], ntiles = m[2], rows = m[3];
             if (u < 0) break;
             const int ub = m[4], ug = m[5], usplit = m[6], un = m[7];
+            if (i == 0) {
+                cand_key = ~0ull;
+                cand_slot = 0x7fffffff;
+            }
+            if (want_cand && ntiles > 0 && lane < 16 && kw + lane < rows) {
+                // eviction key of this slot for position t + 1 (one lane per slot)
+                const int kk = kw + lane;
+                const int ps = s_pos[st * T + kk];
+                const float sc = BIAS ? __fmul_rn(__int2float_rn(m[8] + 1 - ps), s_lb[st * T + kk]) : 0.f;
+                const unsigned long long k64 =
+                    ((unsigned long long)float_order_key(sc) << 32) | (unsigned)(ps ^ 0x80000000);
+                const int slot = m[9] + kk;
+                if (k64 < cand_key || (k64 == cand_key && slot < cand_slot)) {
+                    cand_key = k64;
+                    cand_slot = slot;
+                }
+            }
             if (i == 0) {
                 m_run = -INFINITY;
                 l_run = 0.f;
@@ -447,7 +523,35 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                     s_ml[(warp * G + r) * 2 + 1] = l_run;
                 }
             }
+            if (want_cand) {
+#pragma unroll
+                for (int o2 = 8; o2 >= 1; o2 >>= 1) {
+                    const unsigned long long k2 = __shfl_xor_sync(kFull, cand_key, o2);
+                    const int s2 = __shfl_xor_sync(kFull, cand_slot, o2);
+                    if (k2 < cand_key || (k2 == cand_key && s2 < cand_slot)) {
+                        cand_key = k2;
+                        cand_slot = s2;
+                    }
+                }
+                if (lane == 0) {
+                    s_ck[warp] = cand_key;
+                    s_cs[warp] = cand_slot;
+                }
+            }
             named_bar(1, NWC * 32);
+            if (want_cand && tid == 0) {
+                unsigned long long bk = s_ck[0];
+                int bs = s_cs[0];
+#pragma unroll
+                for (int w = 1; w < NWC; ++w)
+                    if (s_ck[w] < bk || (s_ck[w] == bk && s_cs[w] < bs)) {
+                        bk = s_ck[w];
+                        bs = s_cs[w];
+                    }
+                EvictCand* c = p.cand + ((size_t)ub * p.Hkv + ug) * p.S + usplit;
+                c->key = bk;
+                c->slot = (bk == ~0ull) ? -1 : bs;
+            }
             const int S = p.S;
             for (int idx = tid; idx < G * D; idx += NWC * 32) {
                 const int hh = idx / D, e = idx % D;
@@ -492,34 +596,44 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
 }
 
 // Merge of the num_splits states of each (b, query head) row, [ASM] step 2's
-// operator with Z carried as lse: one warp per row; lane j holds split j's
-// weight exp(lse_j - max) and hands it out by shuffle while every lane
-// accumulates its D/32 dims, with eight independent L2 loads in flight.
+// operator with Z carried as lse. One warp per row, one pass over chunks of
+// 32 splits: lane j loads split j's lse, the warp forms the running maximum
+// and sum, and every lane accumulates its D/32 dims from eight independent
+// L2 loads at a time (splits with zero weight are not read). Two dependent
+// memory round trips for up to 32 splits.
 template <int D>
 __global__ void __launch_bounds__(256) merge_splits_kernel(const float* __restrict__ o_part,
                                                            const float* __restrict__ lse_part, int R, int S,
                                                            void* o, int o_bf16, float* lse) {
+    griddep_wait();
+    griddep_launch_dependents();
     constexpr int E = D / 32;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = blockIdx.x * 8 + warp;
     if (r >= R) return;
     const float* lp = lse_part + (size_t)r * S;
-    float mx = -INFINITY;
-    for (int j = lane; j < S; j += 32) mx = fmaxf(mx, lp[j]);
-#pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
-    const float mu = (mx == -INFINITY) ? 0.f : mx;
-    float sum = 0.f;
-    for (int j = lane; j < S; j += 32) sum += exp2f((lp[j] - mu) * kLog2e);
-#pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) sum += __shfl_xor_sync(kFull, sum, m);
+    const float* op = o_part + (size_t)r * S * D + lane * E;
+    float m_run = -INFINITY, s_run = 0.f;
     float acc[E];
 #pragma unroll
-    for (int k = 0; k < E; ++k) acc[k] = 0.f;
-    const float* op = o_part + (size_t)r * S * D + lane * E;
+    for (int e = 0; e < E; ++e) acc[e] = 0.f;
     for (int j0 = 0; j0 < S; j0 += 32) {
         const int cnt = min(32, S - j0);
-        const float wl = (lane < cnt) ? exp2f((lp[j0 + lane] - mu) * kLog2e) : 0.f;
+        const float l = (lane < cnt) ? __ldcg(lp + j0 + lane) : -INFINITY;
+        float cm = l;
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, m));
+        const float m_new = fmaxf(m_run, cm);
+        const float mu = (m_new == -INFINITY) ? 0.f : m_new;
+        const float a = exp2f((m_run - mu) * kLog2e);
+        const float wl = exp2f((l - mu) * kLog2e);
+        float ws = wl;
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) ws += __shfl_xor_sync(kFull, ws, m);
+        s_run = fmaf(s_run, a, ws);
+        m_run = m_new;
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] *= a;
         for (int k0 = 0; k0 < cnt; k0 += 8) {
             float w[8];
             float v[8][E];
@@ -542,7 +656,7 @@ __global__ void __launch_bounds__(256) merge_splits_kernel(const float* __restri
                 for (int e = 0; e < E; ++e) acc[e] = fmaf(w[k], v[k][e], acc[e]);
         }
     }
-    const float inv = (sum > 0.f) ? 1.f / sum : 0.f;
+    const float inv = (s_run > 0.f) ? 1.f / s_run : 0.f;
     if (o_bf16) {
         __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(o) + (size_t)r * D + lane * E;
 #pragma unroll
@@ -555,7 +669,7 @@ __global__ void __launch_bounds__(256) merge_splits_kernel(const float* __restri
             *reinterpret_cast<float2*>(out) = make_float2(acc[0] * inv, acc[1] * inv);
         }
     }
-    if (lane == 0 && lse != nullptr) lse[r] = (sum > 0.f) ? mx + log2f(sum) * kLn2 : -INFINITY;
+    if (lane == 0 && lse != nullptr) lse[r] = (s_run > 0.f) ? m_run + log2f(s_run) * kLn2 : -INFINITY;
 }
 
 }  // namespace kvb

@@ -8,6 +8,10 @@
 // slots keeping the best 64-bit key (order key of the score << 32 | order
 // key of the position) with its slot; a warp-shuffle argmin and a shared-
 // memory pass across warps give the victim; then the CTA writes the new row.
+// When the preceding attention left per-split candidates (the same key for
+// position t, computed while it read every slot), the victim is the best of
+// those few records instead: the same argmin, since the splits partition
+// the slots.
 #pragma once
 
 #include "common.cuh"
@@ -27,6 +31,8 @@ struct EvictParams {
     int Hkv, d, cap, M;
     int* victim;
     int vec4;  // pos/log_beta rows start 16-byte aligned (cap % 4 == 0, aligned bases)
+    const EvictCand* cand;  // nullable: per-split candidates from the preceding attention
+    int cand_n;
 };
 
 __device__ __forceinline__ void argmin_merge(unsigned long long& key, int& slot, unsigned long long k2, int s2) {
@@ -40,6 +46,9 @@ template <int NT>
 __global__ void __launch_bounds__(NT) evict_insert_kernel(const __grid_constant__ EvictParams p) {
     __shared__ unsigned long long s_key[NT / 32];
     __shared__ int s_slot[NT / 32];
+    __shared__ int s_cand;
+    griddep_wait();  // the previous kernel in the stream (e.g. the last attention) has finished
+    griddep_launch_dependents();
     const int bg = blockIdx.x, b = bg / p.Hkv, tid = threadIdx.x;
     const int tb = p.t[b];
     if (tb < 0) {
@@ -54,10 +63,30 @@ __global__ void __launch_bounds__(NT) evict_insert_kernel(const __grid_constant_
         }
         return;
     }
-    int slot;
+    int slot = -1;
+    if (n >= p.M && p.cand != nullptr) {
+        // the attention of the previous position already reduced every split's slots
+        if (tid < 32) {
+            unsigned long long best = ~0ull;
+            int best_slot = 0x7fffffff;
+            for (int j = tid; j < p.cand_n; j += 32) {
+                const EvictCand c = p.cand[(size_t)bg * p.cand_n + j];
+                if (c.slot >= 0) argmin_merge(best, best_slot, c.key, c.slot);
+            }
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) {
+                const unsigned long long k2 = __shfl_xor_sync(kFull, best, m);
+                const int s2 = __shfl_xor_sync(kFull, best_slot, m);
+                argmin_merge(best, best_slot, k2, s2);
+            }
+            if (tid == 0) s_cand = (best != ~0ull && best_slot < n) ? best_slot : -1;
+        }
+        __syncthreads();
+        slot = s_cand;
+    }
     if (n < p.M) {
         slot = n;
-    } else {
+    } else if (slot < 0) {  // no usable candidates: scan every slot
         const size_t base = (size_t)bg * p.cap;
         const int* ps = p.pos + base;
         const float* lb = p.lb ? p.lb + base : nullptr;

@@ -95,6 +95,25 @@ int resident_ctas(Kern kern, int threads, size_t smem) {
     return n;
 }
 
+// Launch with programmatic stream serialization: the kernel may start while the
+// previous kernel in the stream drains; its first instruction waits for that
+// kernel's completion (griddepcontrol.wait), so only the launch latency overlaps.
+template <typename... KArgs, typename... Args>
+kvb_status launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                      Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...) == cudaSuccess ? KVB_OK : KVB_ECUDA;
+}
+
 template <int D, int G, bool BIAS>
 kvb_status launch_decode_tc(const kvb::DecodeTcParams& p, const kvb_attn_args* a, cudaStream_t st) {
     using SH = kvb::TcShape<D, G>;
@@ -109,12 +128,12 @@ kvb_status launch_decode_tc(const kvb::DecodeTcParams& p, const kvb_attn_args* a
     const int slots = resident_ctas(kern, SH::NT, smem);
     if (slots <= 0) return KVB_ECUDA;
     const int grid = p.units < slots ? p.units : slots;
-    kern<<<grid, SH::NT, smem, st>>>(p, mk, mv);
-    if (launched() != KVB_OK) return KVB_ECUDA;
+    if (launch_pdl(kern, dim3(grid), dim3(SH::NT), smem, st, p, mk, mv) != KVB_OK) return KVB_ECUDA;
     if (p.S > 1) {
         const int R = a->B * a->Hq;
-        kvb::merge_splits_kernel<D><<<(R + 7) / 8, 256, 0, st>>>(p.o_part, p.lse_part, R, p.S, p.o, p.o_bf16, p.lse);
-        return launched();
+        return launch_pdl(kvb::merge_splits_kernel<D>, dim3((R + 7) / 8), dim3(256), 0, st,
+                          static_cast<const float*>(p.o_part), static_cast<const float*>(p.lse_part), R, p.S,
+                          p.o, p.o_bf16, p.lse);
     }
     return KVB_OK;
 }
@@ -165,7 +184,7 @@ inline size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
 extern "C" {
 
-int32_t kvb_abi_version(void) { return 1; }
+int32_t kvb_abi_version(void) { return 2; }
 
 const char* kvb_status_str(kvb_status s) {
     switch (s) {
@@ -205,6 +224,10 @@ kvb_status kvb_decode_attn(const kvb_attn_args* a, kvb_stream stream) {
     const bool bias = a->log_beta != nullptr;
     if (bias && (!a->pos || !a->t)) return KVB_EINVAL;
     if (bias && (a->meta_stride_b < 0 || a->meta_stride_h < 0)) return KVB_EINVAL;
+    if (a->evict_cand != nullptr &&
+        (!a->pos || !a->t || a->meta_stride_b < 0 || a->meta_stride_h < 0 ||
+         (reinterpret_cast<uintptr_t>(a->evict_cand) & 15u)))
+        return KVB_EINVAL;
     if (a->o_dtype != KVB_OUT_F32 && a->o_dtype != KVB_OUT_BF16) return KVB_EINVAL;
     if (a->num_splits > 1 && (!a->o_part || !a->lse_part)) return KVB_EINVAL;
     if ((a->o_part == nullptr) != (a->lse_part == nullptr)) return KVB_EINVAL;
@@ -224,6 +247,7 @@ kvb_status kvb_decode_attn(const kvb_attn_args* a, kvb_stream stream) {
     p.scale = (float)scale;
     p.o_part = a->o_part; p.lse_part = a->lse_part;
     p.o = a->o; p.o_bf16 = (a->o_dtype == KVB_OUT_BF16); p.lse = a->lse;
+    p.cand = static_cast<kvb::EvictCand*>(a->evict_cand);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return a->d == 128 ? tc_g<128>(p, a, G, bias, st) : tc_g<64>(p, a, G, bias, st);
 }
@@ -273,7 +297,7 @@ kvb_status kvb_merge_states(const float* o_in, const float* lse_in, int64_t o_st
 kvb_status kvb_evict_insert(uint16_t* k, uint16_t* v, float* log_beta, int32_t* pos, int32_t* len,
                             const uint16_t* k_new, const uint16_t* v_new, const float* log_beta_new,
                             const int32_t* t, int32_t B, int32_t Hkv, int32_t d, int32_t cap, int32_t M,
-                            int32_t* victim, kvb_stream stream) {
+                            int32_t* victim, const void* cand, int32_t cand_n, kvb_stream stream) {
     if (B < 1 || Hkv < 1 || d < 8 || d > 1024 || (d % 8) || cap < 1 || M < 1 || M > cap) return KVB_EINVAL;
     if ((long long)B * Hkv > 0x7fffffffLL) return KVB_EINVAL;
     if (!pos || !len || !t) return KVB_EINVAL;
@@ -281,10 +305,12 @@ kvb_status kvb_evict_insert(uint16_t* k, uint16_t* v, float* log_beta, int32_t* 
     if (k_new && (!k || !v || !aligned16(k) || !aligned16(v) || !aligned16(k_new) || !aligned16(v_new)))
         return KVB_EINVAL;
     if (log_beta && !log_beta_new) return KVB_EINVAL;
+    if (cand != nullptr && (cand_n < 1 || cand_n > 1024 || (reinterpret_cast<uintptr_t>(cand) & 15u))) return KVB_EINVAL;
     const int vec4 = (cap % 4 == 0) && aligned16(pos) && (log_beta == nullptr || aligned16(log_beta)) ? 1 : 0;
-    kvb::EvictParams p{k, v, log_beta, pos, len, k_new, v_new, log_beta_new, t, Hkv, d, cap, M, victim, vec4};
-    kvb::evict_insert_kernel<256><<<B * Hkv, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
-    return launched();
+    kvb::EvictParams p{k, v, log_beta, pos, len, k_new, v_new, log_beta_new, t, Hkv, d, cap, M, victim, vec4,
+                       static_cast<const kvb::EvictCand*>(cand), cand_n};
+    return launch_pdl(kvb::evict_insert_kernel<256>, dim3(B * Hkv), dim3(256), 0, static_cast<cudaStream_t>(stream),
+                      p);
 }
 
 kvb_status kvb_compact_blocks(uint16_t* k, uint16_t* v, int32_t* pos, float* log_beta, int32_t* len,

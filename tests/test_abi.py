@@ -47,7 +47,7 @@ def test_attn_args_struct_matches_header():
 
 def test_status_strings_and_version():
     L = _lib.lib()
-    assert L.kvb_abi_version() == 1
+    assert L.kvb_abi_version() == 2
     assert L.kvb_status_str(0) == b"ok"
     assert L.kvb_status_str(1) == b"invalid argument"
 
@@ -75,8 +75,12 @@ def test_decode_attn_rejects_bad_arguments_on_the_host(bad):
 def test_other_entry_points_reject_bad_arguments_on_the_host():
     L = _lib.lib()
     f = ctypes.c_void_p(1 << 20)
-    assert L.kvb_evict_insert(f, f, None, f, f, f, f, None, f, 1, 1, 128, 64, 65, None, None) == _lib.KVB_EINVAL
-    assert L.kvb_evict_insert(f, f, None, f, f, f, None, None, f, 1, 1, 128, 64, 8, None, None) == _lib.KVB_EINVAL
+    assert L.kvb_evict_insert(f, f, None, f, f, f, f, None, f, 1, 1, 128, 64, 65, None, None, 0, None) == _lib.KVB_EINVAL
+    assert L.kvb_evict_insert(f, f, None, f, f, f, None, None, f, 1, 1, 128, 64, 8, None, None, 0, None) == _lib.KVB_EINVAL
+    # candidates: count out of range, misaligned buffer
+    assert L.kvb_evict_insert(f, f, None, f, f, f, f, None, f, 1, 1, 128, 64, 8, None, f, 0, None) == _lib.KVB_EINVAL
+    assert L.kvb_evict_insert(f, f, None, f, f, f, f, None, f, 1, 1, 128, 64, 8, None,
+                              ctypes.c_void_p((1 << 20) + 8), 2, None) == _lib.KVB_EINVAL
     assert L.kvb_compact_blocks(f, f, f, None, f, f, f, 1, 1, 12, 64, None) == _lib.KVB_EINVAL
     assert L.kvb_merge_states(f, f, 1, 1, 1, 1, 0, 4, 8, f, None, None) == _lib.KVB_EINVAL
     assert L.kvb_asm_lookup_merge(f, f, f, f, f, f, 4, 2, 16, 64, None, f, None, f, 1 << 20, None) == _lib.KVB_EINVAL

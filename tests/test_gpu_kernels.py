@@ -75,6 +75,44 @@ def test_evict_insert_large_cache_bit_exact(oracle):
     assert_cache_equal(gc, c)
 
 
+@pytest.mark.parametrize("S,with_beta", [(1, True), (3, True), (16, True), (5, False)])
+def test_attention_leaves_exact_eviction_candidates(oracle, S, with_beta):
+    """Each split's record is the slot the oracle evicts at t + 1 among that split's slots."""
+    B, Hq, Hkv, d, cap = 2, 8, 2, 128, 300
+    g = rng(25, S)
+    q = normal_bf16(g, (B, Hq, d))
+    k, v = normal_bf16(g, (B, Hkv, cap, d)), normal_bf16(g, (B, Hkv, cap, d))
+    lb = log_beta(g, (B, Hkv, cap)) if with_beta else None
+    if with_beta:
+        lb[0, 0, 10:20] = -0.125   # equal scores for equal distances: ties resolved by position
+    pos = np.stack([np.stack([g.permutation(2 * cap)[:cap] for _ in range(Hkv)]) for _ in range(B)]).astype(np.int32)
+    ln = np.array([[300, 257], [1, 64]], np.int32)
+    t = np.full(B, 2 * cap + 1, np.int32)
+    o = torch.zeros(B, Hq, d, device="cuda")
+    op, lp, _ = kvb.decode_workspace(B, Hq, Hkv, d, S)
+    cand = kvb.evict_candidates(B, Hkv, S)
+    kvb.kvb_decode_attn(dev(q), dev(k), dev(v), None if lb is None else dev(lb), dev(pos), dev(ln), dev(t), o,
+                        num_splits=S, o_part=op, lse_part=lp, evict_cand=cand)
+    rec = host(cand).reshape(B, Hkv, S, 2)
+    slots = (rec[..., 1] & 0xffffffff).astype(np.int64)
+    slots = np.where(slots >= 2**31, slots - 2**32, slots)
+    for b in range(B):
+        for gg in range(Hkv):
+            n = ln[b, gg]
+            C = -(-n // S)
+            for j in range(S):
+                s0, s1 = min(j * C, n), min((j + 1) * C, n)
+                if s1 <= s0:
+                    assert slots[b, gg, j] == -1
+                    continue
+                sub = dict(k=np.zeros((1, 1, s1 - s0, 8), np.uint16), v=np.zeros((1, 1, s1 - s0, 8), np.uint16),
+                           log_beta=None if lb is None else lb[b, gg, s0:s1][None, None].copy(),
+                           pos=pos[b, gg, s0:s1][None, None].copy(), len=np.array([[s1 - s0]], np.int32))
+                vic = oracle.evict_insert(sub, None, None, None if lb is None else np.zeros((1, 1), np.float32),
+                                          np.array([t[b] + 1], np.int32), s1 - s0)
+                assert slots[b, gg, j] == s0 + vic[0, 0], (b, gg, j)
+
+
 def test_evict_insert_bad_length_flags_error():
     c = empty_cache(1, 2, 8, 64)
     c["len"][0, 1] = 9
