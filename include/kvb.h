@@ -94,7 +94,9 @@ enum kvb_device_error {
  *   o        [B, Hq, d] f32 or bf16 (o_dtype), contiguous
  *   lse      [B, Hq] f32, contiguous, may be NULL
  *   o_part   [B, Hq, num_splits, d] f32, lse_part [B, Hq, num_splits] f32:
- *            every split's state (empty splits get (0, -inf)); required when
+ *            every split's state; an empty split gets lse = -inf and its o_part
+ *            row is left as it was (no merge reads the o of an empty state,
+ *            kvb_merge_states included); required when
  *            num_splits > 1, may be NULL when num_splits == 1. With
  *            num_splits > 1 the call launches the attention kernel, which
  *            writes every split's state, and a merge kernel that combines
@@ -195,7 +197,7 @@ kvb_status kvb_decode_attn_noalloc(const kvb_attn_args* args, kvb_stream stream)
  *     o = sum_j exp(lse_j - lse) o_j;
  * rows whose states are all empty get (0, -inf). The identity element is
  * (0, -inf), so external states (e.g. a stored prefix state) merge the same
- * way.
+ * way. The o of a state with lse = -inf is never read.
  *
  * State j of row r: o_in[j*o_stride_n + r*o_stride_r + e] (e < d, f32) and
  * lse_in[j*lse_stride_n + r*lse_stride_r]. Outputs o_out [R, d] and

@@ -239,14 +239,8 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                 // an empty split (ragged lengths, inactive rows): write its empty state here;
                 // no record reaches the consumers
                 const size_t row0 = (size_t)ui.b * p.Hq + ui.g * G;
-                if (p.o_part != nullptr) {
-                    for (int idx = lane; idx < G * D / 4; idx += 32) {
-                        const int hh = idx / (D / 4), e4 = idx % (D / 4);
-                        reinterpret_cast<float4*>(p.o_part + ((row0 + hh) * p.S + ui.split) * D)[e4] =
-                            make_float4(0.f, 0.f, 0.f, 0.f);
-                    }
-                    if (lane < G) p.lse_part[(row0 + lane) * p.S + ui.split] = -INFINITY;
-                }
+                // lse = -inf marks the empty state; its o_part row is not written (no merge reads it)
+                if (p.o_part != nullptr && lane < G) p.lse_part[(row0 + lane) * p.S + ui.split] = -INFINITY;
                 if (p.S == 1) {
                     for (int idx = lane; idx < G * D; idx += 32) {
                         const size_t oi = row0 * D + idx;
@@ -670,6 +664,103 @@ __global__ void __launch_bounds__(256) merge_splits_kernel(const float* __restri
         }
     }
     if (lane == 0 && lse != nullptr) lse[r] = (s_run > 0.f) ? m_run + log2f(s_run) * kLn2 : -INFINITY;
+}
+
+// Merge for many splits: one CTA per (b, query head) row; warp w folds a contiguous chunk of the
+// splits exactly as merge_splits_kernel does, then warp 0 combines the eight partial states
+// through shared memory. Every warp has at most ceil(S/8) splits in flight.
+template <int D>
+__global__ void __launch_bounds__(256) merge_splits_cta_kernel(const float* __restrict__ o_part,
+                                                               const float* __restrict__ lse_part, int R, int S,
+                                                               void* o, int o_bf16, float* lse) {
+    griddep_wait();
+    griddep_launch_dependents();
+    constexpr int E = D / 32, NWM = 8;
+    __shared__ float s_m[NWM], s_s[NWM];
+    __shared__ __align__(16) float s_acc[NWM][D];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r = blockIdx.x;
+    const int cs = (S + NWM - 1) / NWM;
+    const int j_beg = min(S, warp * cs), j_end = min(S, j_beg + cs);
+    const float* lp = lse_part + (size_t)r * S;
+    const float* op = o_part + (size_t)r * S * D + lane * E;
+    float m_run = -INFINITY, s_run = 0.f;
+    float acc[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = 0.f;
+    for (int j0 = j_beg; j0 < j_end; j0 += 32) {
+        const int cnt = min(32, j_end - j0);
+        const float l = (lane < cnt) ? __ldcg(lp + j0 + lane) : -INFINITY;
+        float cm = l;
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, m));
+        const float m_new = fmaxf(m_run, cm);
+        const float mu = (m_new == -INFINITY) ? 0.f : m_new;
+        const float a = exp2f((m_run - mu) * kLog2e);
+        const float wl = exp2f((l - mu) * kLog2e);
+        float ws = wl;
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) ws += __shfl_xor_sync(kFull, ws, m);
+        s_run = fmaf(s_run, a, ws);
+        m_run = m_new;
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] *= a;
+        for (int k0 = 0; k0 < cnt; k0 += 8) {
+            float w[8];
+            float v[8][E];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                w[k] = __shfl_sync(kFull, wl, (k0 + k) & 31);
+                const bool use = (k0 + k < cnt) && w[k] > 0.f;
+                const float* src = op + (size_t)(j0 + k0 + k) * D;
+                if constexpr (E == 4) {
+                    const float4 x = use ? __ldcg(reinterpret_cast<const float4*>(src)) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    v[k][0] = x.x; v[k][1] = x.y; v[k][2] = x.z; v[k][3] = x.w;
+                } else {
+                    const float2 x = use ? __ldcg(reinterpret_cast<const float2*>(src)) : make_float2(0.f, 0.f);
+                    v[k][0] = x.x; v[k][1] = x.y;
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+#pragma unroll
+                for (int e = 0; e < E; ++e) acc[e] = fmaf(w[k], v[k][e], acc[e]);
+        }
+    }
+    if (lane == 0) {
+        s_m[warp] = m_run;
+        s_s[warp] = s_run;
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) s_acc[warp][lane * E + e] = acc[e];
+    __syncthreads();
+    if (warp != 0) return;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NWM; ++w) M = fmaxf(M, s_m[w]);
+    const float Mu = (M == -INFINITY) ? 0.f : M;
+    float tot = 0.f;
+    float out[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) out[e] = 0.f;
+#pragma unroll
+    for (int w = 0; w < NWM; ++w) {
+        const float f = exp2f((s_m[w] - Mu) * kLog2e);
+        tot = fmaf(f, s_s[w], tot);
+#pragma unroll
+        for (int e = 0; e < E; ++e) out[e] = fmaf(f, s_acc[w][lane * E + e], out[e]);
+    }
+    const float inv = (tot > 0.f) ? 1.f / tot : 0.f;
+    if (o_bf16) {
+        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(o) + (size_t)r * D + lane * E;
+#pragma unroll
+        for (int e = 0; e < E; ++e) dst[e] = __float2bfloat16_rn(out[e] * inv);
+    } else {
+        float* dst = reinterpret_cast<float*>(o) + (size_t)r * D + lane * E;
+#pragma unroll
+        for (int e = 0; e < E; ++e) dst[e] = out[e] * inv;
+    }
+    if (lane == 0 && lse != nullptr) lse[r] = (tot > 0.f) ? M + log2f(tot) * kLn2 : -INFINITY;
 }
 
 }  // namespace kvb

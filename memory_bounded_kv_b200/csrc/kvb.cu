@@ -131,6 +131,11 @@ kvb_status launch_decode_tc(const kvb::DecodeTcParams& p, const kvb_attn_args* a
     if (launch_pdl(kern, dim3(grid), dim3(SH::NT), smem, st, p, mk, mv) != KVB_OK) return KVB_ECUDA;
     if (p.S > 1) {
         const int R = a->B * a->Hq;
+        // few rows with many splits: a CTA per row keeps more loads in flight per row
+        if (p.S > 16 && R < 4 * 148)
+            return launch_pdl(kvb::merge_splits_cta_kernel<D>, dim3(R), dim3(256), 0, st,
+                              static_cast<const float*>(p.o_part), static_cast<const float*>(p.lse_part), R, p.S,
+                              p.o, p.o_bf16, p.lse);
         return launch_pdl(kvb::merge_splits_kernel<D>, dim3((R + 7) / 8), dim3(256), 0, st,
                           static_cast<const float*>(p.o_part), static_cast<const float*>(p.lse_part), R, p.S,
                           p.o, p.o_bf16, p.lse);

@@ -41,6 +41,7 @@ __global__ void __launch_bounds__(256) merge_states_kernel(const __grid_constant
             float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
             for (int j = 0; j < p.n; ++j) {
                 const float w = exp2f((p.lse_in[j * p.l_sn + r * p.l_sr] - mu) * kLog2e);
+                if (w == 0.f) continue;  // an empty state: its o is not read
                 const float4 x = *reinterpret_cast<const float4*>(p.o_in + j * p.o_sn + r * p.o_sr + e);
                 a.x = fmaf(w, x.x, a.x); a.y = fmaf(w, x.y, a.y);
                 a.z = fmaf(w, x.z, a.z); a.w = fmaf(w, x.w, a.w);
@@ -52,7 +53,7 @@ __global__ void __launch_bounds__(256) merge_states_kernel(const __grid_constant
             float a = 0.f;
             for (int j = 0; j < p.n; ++j) {
                 const float w = exp2f((p.lse_in[j * p.l_sn + r * p.l_sr] - mu) * kLog2e);
-                a = fmaf(w, p.o_in[j * p.o_sn + r * p.o_sr + e], a);
+                if (w != 0.f) a = fmaf(w, p.o_in[j * p.o_sn + r * p.o_sr + e], a);
             }
             out[e] = a * inv;
         }

@@ -63,6 +63,15 @@ def assert_state_close(o, lse, o_ref, lse_ref, what: str = ""):
     return maxabs, rel
 
 
+def assert_splits_close(o_part, lse_part, o_ref, lse_ref, what: str = "splits"):
+    """Per-split states: lse everywhere; o only where the split is not empty (an empty split's
+    o row is not written by the library)."""
+    o_part = np.asarray(o_part, np.float64).copy()
+    empty = np.isneginf(np.asarray(lse_ref))
+    o_part[empty] = 0.0
+    return assert_state_close(o_part, lse_part, o_ref, lse_ref, what)
+
+
 class GpuCache:
     """Device copy of a host cache dict {k, v, log_beta, pos, len}."""
 

@@ -17,7 +17,7 @@ import torch
 import memory_bounded_kv_b200 as kvb
 from memory_bounded_kv_b200 import synth
 from memory_bounded_kv_b200.cache import BoundedKVCache
-from gpu_util import dev, host, assert_state_close
+from gpu_util import dev, host, assert_state_close, assert_splits_close
 
 pytestmark = pytest.mark.gpu
 
@@ -137,7 +137,7 @@ def test_config3_stream_and_decode(oracle):
             o_ref, l_ref, op_ref, lp_ref = oracle.decode_attn(inp["q"], c["k"], c["v"], c["log_beta"], c["pos"],
                                                               c["len"], inp["t"], num_splits=S, want_parts=True)
             assert_state_close(host(o), host(lse), o_ref, l_ref, f"step {step}")
-            assert_state_close(host(cache.o_part), host(cache.lse_part), op_ref, lp_ref, f"step {step} splits")
+            assert_splits_close(host(cache.o_part), host(cache.lse_part), op_ref, lp_ref, f"step {step} splits")
             # plain variant: beta = 1 (no log beta, no positions read)
             cache.attend(dev(inp["q"]), None, o_plain, lse_plain, use_beta=False)
             o_ref, l_ref = oracle.decode_attn(inp["q"], c["k"], c["v"], None, c["pos"], c["len"], None)
