@@ -41,9 +41,12 @@ METRIC = "decode-attn tokens/s and KV-cache GB/s (% of B200 HBM peak) at budget 
 FALLBACK_HBM_GBS = 6650.0
 
 # ncu DRAM traffic (read + write bytes per launch) of the dominant kernel, keyed by
-# (sha256 of the kernel's source file, config). Reported only while the source is
-# unchanged since the counters were taken (profiles/decode_attn_config2.md).
-MEASURED_TRAFFIC = {}
+# (sha256 of the kernel's source file, config, num_splits). Reported only while the source is
+# unchanged since the counters were taken (profiles/decode_attn_tc_config2.md).
+MEASURED_TRAFFIC = {
+    # decode_attn_tc_kernel<128,4,1>, Qwen3-8B-shaped layer, S=2: 545,583,616 read + 4,786,688 written
+    ("621484185f5a7665", 2, 2): 550370304,
+}
 
 
 def parse():
@@ -543,7 +546,7 @@ def run_kvb(args, world, rank, local):
                 else "kvb_decode_attn = decode_attn_tc_kernel<128,4,plain> + merge_splits_kernel")
         roofline = {"bound": "hbm", "kernel": name, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                     "frac": achieved / hbm_peak, "peak_source": f"{peak_kind} (hbm_gbs)",
-                    "traffic": MEASURED_TRAFFIC.get((src, args.config)),
+                    "traffic": MEASURED_TRAFFIC.get((src, args.config, getattr(bench, "S", 0))),
                     "algorithmic_bytes_per_launch": attn_bytes, "kernel_ms_avg": kms}
         step_bytes = attn_bytes + (bench.evict_bytes() if hasattr(bench, "evict_bytes") else 0)
     kv_gbs = step_bytes * K / (ms / 1e3) / 1e9
