@@ -385,7 +385,7 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
             const int* m = s_meta + st * 16;
             const int u = m[0], i = m[1], ntiles = m[2], rows = m[3];
             if (u < 0) break;
-            const int ub = m[4], ug = m[5], usplit = m[6], un = m[7];
+            const int ub = m[4], ug = m[5], usplit = m[6];
             if (i == 0) {
                 cand_key = ~0ull;
                 cand_slot = 0x7fffffff;

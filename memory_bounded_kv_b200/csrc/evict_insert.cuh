@@ -50,12 +50,21 @@ __global__ void __launch_bounds__(NT) evict_insert_kernel(const __grid_constant_
     griddep_wait();  // the previous kernel in the stream (e.g. the last attention) has finished
     griddep_launch_dependents();
     const int bg = blockIdx.x, b = bg / p.Hkv, tid = threadIdx.x;
+    // every load that does not depend on another is issued here, before any of them is used:
+    // position, length, this thread's candidate record and its 16 bytes of the new row
     const int tb = p.t[b];
+    const int n = p.len[bg];
+    EvictCand my_cand{~0ull, -1, 0};
+    if (p.cand != nullptr && tid < 32 && tid < p.cand_n) my_cand = p.cand[(size_t)bg * p.cand_n + tid];
+    const int vecs = p.d / 8;
+    uint4 row_part = make_uint4(0u, 0u, 0u, 0u);
+    if (p.k_new != nullptr && tid < 2 * vecs)
+        row_part = (tid < vecs) ? reinterpret_cast<const uint4*>(p.k_new + (size_t)bg * p.d)[tid]
+                                : reinterpret_cast<const uint4*>(p.v_new + (size_t)bg * p.d)[tid - vecs];
     if (tb < 0) {
         if (tid == 0 && p.victim) p.victim[bg] = -1;
         return;
     }
-    const int n = p.len[bg];
     if (n < 0 || n > p.cap) {
         if (tid == 0) {
             raise_error(KVB_DERR_LEN);
@@ -69,7 +78,8 @@ __global__ void __launch_bounds__(NT) evict_insert_kernel(const __grid_constant_
         if (tid < 32) {
             unsigned long long best = ~0ull;
             int best_slot = 0x7fffffff;
-            for (int j = tid; j < p.cand_n; j += 32) {
+            if (my_cand.slot >= 0) argmin_merge(best, best_slot, my_cand.key, my_cand.slot);
+            for (int j = tid + 32; j < p.cand_n; j += 32) {   // records past the first 32
                 const EvictCand c = p.cand[(size_t)bg * p.cand_n + j];
                 if (c.slot >= 0) argmin_merge(best, best_slot, c.key, c.slot);
             }
@@ -154,8 +164,14 @@ __global__ void __launch_bounds__(NT) evict_insert_kernel(const __grid_constant_
     }
     const size_t row = (size_t)bg * p.cap + slot;
     if (p.k_new != nullptr) {
-        const int vecs = p.d / 8;
-        for (int i = tid; i < 2 * vecs; i += NT) {
+        if (tid < 2 * vecs) {
+            if (tid < vecs) {
+                reinterpret_cast<uint4*>(p.k + row * p.d)[tid] = row_part;
+            } else {
+                reinterpret_cast<uint4*>(p.v + row * p.d)[tid - vecs] = row_part;
+            }
+        }
+        for (int i = tid + NT; i < 2 * vecs; i += NT) {   // rows wider than the block
             if (i < vecs) {
                 reinterpret_cast<uint4*>(p.k + row * p.d)[i] =
                     reinterpret_cast<const uint4*>(p.k_new + (size_t)bg * p.d)[i];

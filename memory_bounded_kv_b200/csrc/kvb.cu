@@ -127,7 +127,10 @@ kvb_status launch_decode_tc(const kvb::DecodeTcParams& p, const kvb_attn_args* a
         return KVB_EINVAL;
     const int slots = resident_ctas(kern, SH::NT, smem);
     if (slots <= 0) return KVB_ECUDA;
-    const int grid = p.units < slots ? p.units : slots;
+    // as many CTAs as keep every CTA's unit count equal to the busiest one's: the makespan in
+    // units is unchanged and no CTA idles while the others finish
+    const int per_cta = (p.units + slots - 1) / slots;
+    const int grid = (p.units + per_cta - 1) / per_cta;
     if (launch_pdl(kern, dim3(grid), dim3(SH::NT), smem, st, p, mk, mv) != KVB_OK) return KVB_ECUDA;
     if (p.S > 1) {
         const int R = a->B * a->Hq;

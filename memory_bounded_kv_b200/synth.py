@@ -107,7 +107,7 @@ _DECODE_CONFIGS = {
             M=256, cap=256, prefill=256, steps=512, splits=(1, 4)),
     # Qwen3-8B-shaped layer: full budget 4096, 1024 steps of evict+insert+attend
     2: dict(name="qwen3-8b-layer B32 Hq32 Hkv8 d128 M4096", seed=2, B=32, Hq=32, Hkv=8, d=128,
-            M=4096, cap=4096, prefill=4096, steps=1024, splits=(2,)),
+            M=4096, cap=4096, prefill=4096, steps=1024, splits=(1,)),
     # long context 131072 held in 8192 slots, 64 splits
     3: dict(name="long-context B4 Hq32 Hkv8 d128 M8192 ctx131072", seed=3, B=4, Hq=32, Hkv=8, d=128,
             M=8192, cap=8192, prefill=8192, steps=64, splits=(64,)),
