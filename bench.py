@@ -44,8 +44,8 @@ FALLBACK_HBM_GBS = 6650.0
 # (sha256 of the kernel's source file, config, num_splits). Reported only while the source is
 # unchanged since the counters were taken (profiles/decode_attn_tc_config2.md).
 MEASURED_TRAFFIC = {
-    # decode_attn_tc_kernel<128,4,1>, Qwen3-8B-shaped layer, S=2: 545,583,616 read + 4,786,688 written
-    ("621484185f5a7665", 2, 2): 550370304,
+    # decode_attn_tc_kernel<128,4,1>, Qwen3-8B-shaped layer, S=1: 545,628,416 read + 3,972,608 written
+    ("f9553bcebbe325aa", 2, 1): 549601024,
 }
 
 

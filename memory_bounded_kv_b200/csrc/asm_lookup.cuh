@@ -4,10 +4,11 @@
 //
 // Phase 1 (asm_score_kernel) is a dense fp32 contraction per head,
 // [N queries x d] . [d x K centroids], fused with a running argmax: a CTA
-// takes 64 queries x one range of centroids, stages both tiles in shared
-// memory (row-major, rows padded by 4 floats so the float4 reads of 8
-// threads touch 8 distinct bank quads) and each thread keeps a 4 x 4 block
-// of dot products in registers. The compared value is q.qbar_k / |qbar_k|,
+// takes 64 queries x one range of centroids, stages the queries and a
+// double-buffered pair of centroid tiles in shared memory (cp.async, the
+// next tile lands while the current one is computed; rows padded by 4
+// floats so the float4 reads of 8 threads touch 8 distinct bank quads) and
+// each thread keeps a 4 x 4 block of dot products in registers. The compared value is q.qbar_k / |qbar_k|,
 // which orders the centroids exactly as cos does for a fixed q. The best
 // (value, -k) per query is packed into one 64-bit key and written per range.
 // Phase 2 (asm_merge_kernel) reduces the ranges' keys, gathers abar_c* and
@@ -22,7 +23,17 @@ namespace kvb {
 
 constexpr int kAsmD = 128, kAsmQT = 64, kAsmKT = 64, kAsmNT = 256, kAsmPad = 4;
 constexpr int kAsmRow = kAsmD + kAsmPad;
-constexpr size_t kAsmSmem = (size_t)(kAsmQT + kAsmKT) * kAsmRow * 4 + kAsmKT * 4;
+// q tile, two centroid tiles (double buffer), two 1/|qbar| vectors
+constexpr size_t kAsmSmem = (size_t)(kAsmQT + 2 * kAsmKT) * kAsmRow * 4 + 2 * kAsmKT * 4;
+
+// 16-byte global -> shared copy; src_bytes = 0 fills the 16 bytes with zeros.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 struct AsmParams {
     const uint16_t* q;
@@ -51,13 +62,29 @@ __host__ __device__ inline int asm_kchunk(int K) {
 
 __global__ void __launch_bounds__(kAsmNT) asm_score_kernel(const __grid_constant__ AsmParams p) {
     extern __shared__ __align__(16) float s_asm[];
-    float* s_q = s_asm;                       // [QT][Row]
-    float* s_c = s_q + kAsmQT * kAsmRow;      // [KT][Row]
-    float* s_inv = s_c + kAsmKT * kAsmRow;    // [KT]
+    float* s_q = s_asm;                            // [QT][Row]
+    float* s_cbuf = s_q + kAsmQT * kAsmRow;        // [2][KT][Row]
+    float* s_invb = s_cbuf + 2 * kAsmKT * kAsmRow; // [2][KT]
     const int h = blockIdx.x, n0 = blockIdx.y * kAsmQT, ks = blockIdx.z;
     const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
     const int k_begin = ks * p.kchunk;
     const int k_end = min(p.K, k_begin + p.kchunk);
+    const int ntile = (k_end > k_begin) ? (k_end - k_begin + kAsmKT - 1) / kAsmKT : 0;
+
+    // centroid tile `it` -> buffer it & 1, 16 bytes per cp.async, rows past k_end zero-filled
+    auto prefetch = [&](int it) {
+        float* dst = s_cbuf + (it & 1) * kAsmKT * kAsmRow;
+        const int kt = k_begin + it * kAsmKT;
+        for (int i = tid; i < kAsmKT * (kAsmD / 4); i += kAsmNT) {
+            const int r = i / (kAsmD / 4), c = i % (kAsmD / 4);
+            const int k = kt + r;
+            const bool in = k < k_end;
+            const float* src = p.qbar + ((size_t)h * p.K + (in ? k : k_begin)) * kAsmD + c * 4;
+            cp_async16(dst + r * kAsmRow + c * 4, src, in ? 16 : 0);
+        }
+        cp_async_commit();
+    };
+    if (ntile > 0) prefetch(0);
 
     for (int i = tid; i < kAsmQT * (kAsmD / 8); i += kAsmNT) {
         const int r = i / (kAsmD / 8), c = i % (kAsmD / 8);
@@ -75,16 +102,17 @@ __global__ void __launch_bounds__(kAsmNT) asm_score_kernel(const __grid_constant
     }
 
     unsigned long long best[4] = {0ull, 0ull, 0ull, 0ull};
-    for (int kt = k_begin; kt < k_end; kt += kAsmKT) {
-        __syncthreads();  // previous tile consumed (and, first time, q staged)
-        for (int i = tid; i < kAsmKT * (kAsmD / 4); i += kAsmNT) {
-            const int r = i / (kAsmD / 4), c = i % (kAsmD / 4);
-            const int k = kt + r;
-            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (k < k_end) x = *reinterpret_cast<const float4*>(p.qbar + ((size_t)h * p.K + k) * kAsmD + c * 4);
-            *reinterpret_cast<float4*>(s_c + r * kAsmRow + c * 4) = x;
+    for (int it = 0; it < ntile; ++it) {
+        const int kt = k_begin + it * kAsmKT;
+        if (it + 1 < ntile) {
+            prefetch(it + 1);      // lands while this tile is computed
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
         }
-        __syncthreads();
+        __syncthreads();           // tile `it` (and, first time, q) visible to all threads
+        const float* s_c = s_cbuf + (it & 1) * kAsmKT * kAsmRow;
+        float* s_inv = s_invb + (it & 1) * kAsmKT;
         {   // 1/|qbar_k| (0 for a zero vector: its cosine is defined as 0)
             const int r = tid >> 2, part = tid & 3;
             float ss = 0.f;
@@ -134,6 +162,7 @@ __global__ void __launch_bounds__(kAsmNT) asm_score_kernel(const __grid_constant
                 }
             }
         }
+        __syncthreads();           // buffer it & 1 is refilled by the prefetch of tile it + 2
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
