@@ -39,6 +39,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "decode-attn tokens/s and KV-cache GB/s (% of B200 HBM peak) at budget M"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 # ncu DRAM traffic (read + write bytes per launch) of the dominant kernel, keyed by
 # (sha256 of the kernel's source file, config, num_splits). Reported only while the source is
@@ -108,6 +109,17 @@ def peaks():
             p = json.load(f)
         return float(p["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def bf16_peak():
+    """Dense bf16 tensor TFLOP/s for a kernel timed alone (burst figure), and where it comes from."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        if "bf16_tflops" in p:
+            return float(p["bf16_tflops"]), "measured"
+    return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 class ClockSampler:
@@ -316,7 +328,8 @@ class ASMBench:
     """A step: the 256 query tokens' causal self attention over the shared 2048-token cache
     (kvb_decode_attn, batch stride 0) and the memory lookup + merge (kvb_asm_lookup_merge)."""
 
-    FP32_PEAK_NOTE = "148 SMs x 128 FP32 FMA/clk x 2 flop x 1.965 GHz (max SM clock) = 74.4 TFLOP/s"
+    # the fp32 contraction runs as three exact bf16 products per element (q . hi + q . mid + q . lo)
+    PEAK_NOTE = "{kind} dense bf16 {bf16:.0f} TFLOP/s (bf16_tflops, burst) / 3 bf16 products per fp32 product"
 
     def __init__(self, splits: int = 0):
         import memory_bounded_kv_b200 as kvb
@@ -386,7 +399,7 @@ class ASMBench:
         return 2.0 * w.N * w.H * w.K * w.d
 
     def kernel_name(self):
-        return "asm_score_kernel + asm_merge_kernel (kvb_asm_lookup_merge)"
+        return "asm_score_tc_kernel + asm_merge_kernel (kvb_asm_lookup_merge)"
 
     def config(self):
         w = self.w
@@ -532,11 +545,13 @@ def run_kvb(args, world, rank, local):
     launches = bench.launches(W, K) if hasattr(bench, "launches") else bench.launches_per_step * K
     value = replica_value(tokens, world, ms)
     src = kernel_src_hash()
-    if hasattr(bench, "flops"):      # attention-state-memory lookup: fp32 ALU bound
-        peak_tf = 148 * 128 * 2 * 1.965e9 / 1e12
+    if hasattr(bench, "flops"):      # attention-state-memory lookup: tensor bound (bf16 x 3)
+        bf16_tf, bf16_kind = bf16_peak()
+        peak_tf = bf16_tf / 3.0
         achieved = bench.flops() / (kms / 1e3) / 1e12
-        roofline = {"bound": "alu", "kernel": bench.kernel_name(), "achieved": achieved, "peak": peak_tf,
-                    "unit": "TFLOP/s", "frac": achieved / peak_tf, "peak_source": ASMBench.FP32_PEAK_NOTE,
+        roofline = {"bound": "tensor", "kernel": bench.kernel_name(), "achieved": achieved, "peak": peak_tf,
+                    "unit": "TFLOP/s", "frac": achieved / peak_tf,
+                    "peak_source": ASMBench.PEAK_NOTE.format(kind=bf16_kind, bf16=bf16_tf),
                     "traffic": None, "algorithmic_flops_per_launch": bench.flops(), "kernel_ms_avg": kms}
         step_bytes = bench.evict_bytes()
     else:

@@ -2,29 +2,24 @@
 // steps 3-4: c* = argmax_k cos(q, qbar_k), then the retrieved state
 // (abar_c*, Zbar_c*) is merged with the query's own attention state.
 //
-// Phase 1 (asm_score_kernel) is a dense fp32 contraction per head,
-// [N queries x d] . [d x K centroids], fused with a running argmax: a CTA
-// takes 64 queries x one range of centroids, stages the queries and a
-// double-buffered pair of centroid tiles in shared memory (cp.async, the
-// next tile lands while the current one is computed; rows padded by 4
-// floats so the float4 reads of 8 threads touch 8 distinct bank quads) and
-// each thread keeps a 4 x 4 block of dot products in registers. The compared value is q.qbar_k / |qbar_k|,
-// which orders the centroids exactly as cos does for a fixed q. The best
-// (value, -k) per query is packed into one 64-bit key and written per range.
+// Phase 1 (asm_score_tc_kernel) is a dense contraction per head,
+// [N queries x d] . [d x K centroids], fused with a running argmax. The compared
+// value is q.qbar_k / |qbar_k|, which orders the centroids exactly as cos does
+// for a fixed q. The best (value, -k) per query is packed into one 64-bit key
+// and written per range of centroids.
 // Phase 2 (asm_merge_kernel) reduces the ranges' keys, gathers abar_c* and
 // merges it with the self state: one warp per (query, head).
 //
-// fp32 arithmetic throughout: tf32 tensor cores would reorder near-ties.
+// The products are fp32-exact (bf16 q times an exact three-way bf16 split of
+// the fp32 centroid) and accumulate in fp32; tf32 would round the centroids and
+// reorder near-ties.
 #pragma once
 
 #include "common.cuh"
 
 namespace kvb {
 
-constexpr int kAsmD = 128, kAsmQT = 64, kAsmKT = 64, kAsmNT = 256, kAsmPad = 4;
-constexpr int kAsmRow = kAsmD + kAsmPad;
-// q tile, two centroid tiles (double buffer), two 1/|qbar| vectors
-constexpr size_t kAsmSmem = (size_t)(kAsmQT + 2 * kAsmKT) * kAsmRow * 4 + 2 * kAsmKT * 4;
+constexpr int kAsmD = 128, kAsmKT = 64;   // head dim; centroids per tile
 
 // 16-byte global -> shared copy; src_bytes = 0 fills the 16 bytes with zeros.
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, int src_bytes) {
@@ -60,119 +55,174 @@ __host__ __device__ inline int asm_kchunk(int K) {
     return (c + kAsmKT - 1) / kAsmKT * kAsmKT;
 }
 
-__global__ void __launch_bounds__(kAsmNT) asm_score_kernel(const __grid_constant__ AsmParams p) {
-    extern __shared__ __align__(16) float s_asm[];
-    float* s_q = s_asm;                            // [QT][Row]
-    float* s_cbuf = s_q + kAsmQT * kAsmRow;        // [2][KT][Row]
-    float* s_invb = s_cbuf + 2 * kAsmKT * kAsmRow; // [2][KT]
-    const int h = blockIdx.x, n0 = blockIdx.y * kAsmQT, ks = blockIdx.z;
-    const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+// Phase 1: the contraction on the tensor cores, fp32-exact products. q is bf16, hence
+// exact in bf16; each fp32 centroid element is split exactly into three bf16 parts
+// (hi = rn(x), mid = rn(x - hi), lo = x - hi - mid), and q . qbar = q . hi + q . mid + q . lo
+// with exact products and fp32 accumulation (mma.sync m16n8k16). A CTA owns 128 queries of one
+// head (8 warps x 16 query rows, q held in registers as A fragments) and walks its range of
+// centroids in tiles of 64: the fp32 tile arrives by cp.async, the CTA splits it into three
+// padded bf16 tiles (row pitch 272 bytes: the 8 rows of an ldmatrix hit distinct bank groups) and takes the
+// 1/|qbar| of each row, then each warp multiplies its rows by all 64 centroids.
+constexpr int kAtQT = 128, kAtKT = kAsmKT, kAtNT = 256;
+constexpr int kAtPitch = kAsmD + 8;   // bf16 elements per row of a part
+constexpr int kAtSP = kAsmD + 16;     // floats per row of the fp32 stage
+constexpr size_t kAtStage = (size_t)kAtKT * kAtSP * 4;                       // fp32 tile
+constexpr size_t kAtPart = (size_t)kAtKT * kAtPitch * 2;                      // one bf16 part
+constexpr size_t kAtSmem = kAtStage + 3 * kAtPart + kAtKT * 4;
+
+__device__ __forceinline__ void mma_bf16_full(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldsm_x4_asm(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ unsigned short bf16_bits_rn(float x) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
+__global__ void __launch_bounds__(kAtNT, 2) asm_score_tc_kernel(const __grid_constant__ AsmParams p) {
+    extern __shared__ __align__(16) unsigned char s_at[];
+    float* s_stage = reinterpret_cast<float*>(s_at);                                      // [KT][D] f32
+    uint16_t* s_part = reinterpret_cast<uint16_t*>(s_at + kAtStage);                      // [3][KT][pitch]
+    float* s_inv = reinterpret_cast<float*>(s_at + kAtStage + 3 * kAtPart);               // [KT]
+    const int h = blockIdx.x, n0 = blockIdx.y * kAtQT, ks = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int k_begin = ks * p.kchunk;
     const int k_end = min(p.K, k_begin + p.kchunk);
-    const int ntile = (k_end > k_begin) ? (k_end - k_begin + kAsmKT - 1) / kAsmKT : 0;
+    const int ntile = (k_end > k_begin) ? (k_end - k_begin + kAtKT - 1) / kAtKT : 0;
 
-    // centroid tile `it` -> buffer it & 1, 16 bytes per cp.async, rows past k_end zero-filled
     auto prefetch = [&](int it) {
-        float* dst = s_cbuf + (it & 1) * kAsmKT * kAsmRow;
-        const int kt = k_begin + it * kAsmKT;
-        for (int i = tid; i < kAsmKT * (kAsmD / 4); i += kAsmNT) {
+        const int kt = k_begin + it * kAtKT;
+        for (int i = tid; i < kAtKT * (kAsmD / 4); i += kAtNT) {
             const int r = i / (kAsmD / 4), c = i % (kAsmD / 4);
             const int k = kt + r;
             const bool in = k < k_end;
             const float* src = p.qbar + ((size_t)h * p.K + (in ? k : k_begin)) * kAsmD + c * 4;
-            cp_async16(dst + r * kAsmRow + c * 4, src, in ? 16 : 0);
+            cp_async16(s_stage + r * kAtSP + c * 4, src, in ? 16 : 0);
         }
         cp_async_commit();
     };
     if (ntile > 0) prefetch(0);
 
-    for (int i = tid; i < kAsmQT * (kAsmD / 8); i += kAsmNT) {
-        const int r = i / (kAsmD / 8), c = i % (kAsmD / 8);
-        const int n = n0 + r;
-        float f[8];
-        if (n < p.N) {
-            unpack8(*reinterpret_cast<const uint4*>(p.q + ((size_t)n * p.H + h) * kAsmD + c * 8), f);
-        } else {
+    // A fragments of this warp's 16 query rows (rows past N are zero)
+    const int qr = n0 + 16 * warp + (lane >> 2);
+    uint32_t qa[kAsmD / 16][4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = 0.f;
+    for (int s = 0; s < kAsmD / 16; ++s) {
+        const int c0 = 16 * s + 2 * (lane & 3);
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {   // rows qr, qr + 8
+            const int n = qr + 8 * hf;
+            uint32_t lo = 0u, hi = 0u;
+            if (n < p.N) {
+                const uint16_t* qp = p.q + ((size_t)n * p.H + h) * kAsmD;
+                lo = *reinterpret_cast<const uint32_t*>(qp + c0);
+                hi = *reinterpret_cast<const uint32_t*>(qp + c0 + 8);
+            }
+            qa[s][hf] = lo;       // a0 (row), a1 (row + 8)
+            qa[s][2 + hf] = hi;   // a2 (row, col + 8), a3 (row + 8, col + 8)
         }
-        float4* dst = reinterpret_cast<float4*>(s_q + r * kAsmRow + c * 8);
-        dst[0] = make_float4(f[0], f[1], f[2], f[3]);
-        dst[1] = make_float4(f[4], f[5], f[6], f[7]);
     }
 
-    unsigned long long best[4] = {0ull, 0ull, 0ull, 0ull};
+    unsigned long long best[2] = {0ull, 0ull};   // rows qr and qr + 8
+    const uint32_t part_base = smem_u32(s_part);
     for (int it = 0; it < ntile; ++it) {
-        const int kt = k_begin + it * kAsmKT;
-        if (it + 1 < ntile) {
-            prefetch(it + 1);      // lands while this tile is computed
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
-        }
-        __syncthreads();           // tile `it` (and, first time, q) visible to all threads
-        const float* s_c = s_cbuf + (it & 1) * kAsmKT * kAsmRow;
-        float* s_inv = s_invb + (it & 1) * kAsmKT;
-        {   // 1/|qbar_k| (0 for a zero vector: its cosine is defined as 0)
+        const int kt = k_begin + it * kAtKT;
+        cp_async_wait<0>();
+        __syncthreads();   // fp32 tile visible; the bf16 parts of the previous tile are no longer read
+        {   // split into three bf16 parts; 1/|qbar| per row. Four threads per row, each taking
+            // 4-float chunks 16 apart (stage pitch 144 floats: a quarter warp reads 32 distinct banks)
             const int r = tid >> 2, part = tid & 3;
             float ss = 0.f;
 #pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-                const float4 x = *reinterpret_cast<const float4*>(s_c + r * kAsmRow + part * 32 + e);
+            for (int e = 0; e < kAsmD / 16; ++e) {
+                const int col = part * 4 + 16 * e;
+                const float4 x = *reinterpret_cast<const float4*>(s_stage + r * kAtSP + col);
                 ss = fmaf(x.x, x.x, fmaf(x.y, x.y, fmaf(x.z, x.z, fmaf(x.w, x.w, ss))));
+                const float xs[4] = {x.x, x.y, x.z, x.w};
+                uint32_t hw[2] = {0u, 0u}, mw[2] = {0u, 0u}, lw[2] = {0u, 0u};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const unsigned short hb = bf16_bits_rn(xs[c]);
+                    const float r1 = xs[c] - __uint_as_float((unsigned)hb << 16);   // exact
+                    const unsigned short mb = bf16_bits_rn(r1);
+                    const float r2 = r1 - __uint_as_float((unsigned)mb << 16);      // exact
+                    const unsigned short lb = bf16_bits_rn(r2);                     // exact: <= 8 bits left
+                    hw[c >> 1] |= (uint32_t)hb << (16 * (c & 1));
+                    mw[c >> 1] |= (uint32_t)mb << (16 * (c & 1));
+                    lw[c >> 1] |= (uint32_t)lb << (16 * (c & 1));
+                }
+                const int off = r * kAtPitch + col;
+                *reinterpret_cast<uint2*>(s_part + off) = make_uint2(hw[0], hw[1]);
+                *reinterpret_cast<uint2*>(s_part + kAtKT * kAtPitch + off) = make_uint2(mw[0], mw[1]);
+                *reinterpret_cast<uint2*>(s_part + 2 * kAtKT * kAtPitch + off) = make_uint2(lw[0], lw[1]);
             }
             ss += __shfl_xor_sync(kFull, ss, 1);
             ss += __shfl_xor_sync(kFull, ss, 2);
             if (part == 0) s_inv[r] = (ss > 0.f) ? 1.f / sqrtf(ss) : 0.f;
         }
-        __syncthreads();
-        float acc[4][4];
+        __syncthreads();                      // parts and norms ready; the stage buffer is free
+        if (it + 1 < ntile) prefetch(it + 1); // lands while this tile is multiplied
+
+        float acc[kAtKT / 8][4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int j = 0; j < kAtKT / 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+        // ldmatrix row of this lane: centroid (8 x matrix) and 16-byte chunk
+        const int lrow = (lane & 7) + ((lane >> 4) << 3);
+        const int lchk = (lane >> 3) & 1;
+        // k-step outermost: consecutive mma go to the 8 independent accumulators
 #pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-#pragma unroll 8
-        for (int e = 0; e < kAsmD; e += 4) {
-            float4 a[4], c[4];
+        for (int pt = 0; pt < 3; ++pt) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) a[i] = *reinterpret_cast<const float4*>(s_q + (ty * 4 + i) * kAsmRow + e);
+            for (int s = 0; s < kAsmD / 16; ++s) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) c[j] = *reinterpret_cast<const float4*>(s_c + (tx + 16 * j) * kAsmRow + e);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    acc[i][j] = fmaf(a[i].x, c[j].x, acc[i][j]);
-                    acc[i][j] = fmaf(a[i].y, c[j].y, acc[i][j]);
-                    acc[i][j] = fmaf(a[i].z, c[j].z, acc[i][j]);
-                    acc[i][j] = fmaf(a[i].w, c[j].w, acc[i][j]);
-                }
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int r = tx + 16 * j;
-            const int k = kt + r;
-            if (k < k_end) {
-                const float inv = s_inv[r];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const unsigned long long key =
-                        ((unsigned long long)float_order_key(acc[i][j] * inv) << 32) | (0xffffffffu - (unsigned)k);
-                    best[i] = best[i] > key ? best[i] : key;
+                for (int jp = 0; jp < kAtKT / 16; ++jp) {           // pairs of 8-centroid n-tiles
+                    const uint32_t addr = part_base +
+                        (uint32_t)(((pt * kAtKT + 16 * jp + lrow) * kAtPitch + 16 * s + 8 * lchk) * 2);
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4_asm(addr, b0, b1, b2, b3);
+                    mma_bf16_full(acc[2 * jp], qa[s], b0, b1);
+                    mma_bf16_full(acc[2 * jp + 1], qa[s], b2, b3);
                 }
             }
         }
-        __syncthreads();           // buffer it & 1 is refilled by the prefetch of tile it + 2
+        // running argmax of q.qbar / |qbar| per query row (lowest k among equal values)
+#pragma unroll
+        for (int j = 0; j < kAtKT / 8; ++j) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const int r = 8 * j + 2 * (lane & 3) + c;
+                const int k = kt + r;
+                if (k < k_end) {
+                    const float inv = s_inv[r];
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        const unsigned long long key =
+                            ((unsigned long long)float_order_key(acc[j][2 * hf + c] * inv) << 32) |
+                            (0xffffffffu - (unsigned)k);
+                        best[hf] = best[hf] > key ? best[hf] : key;
+                    }
+                }
+            }
+        }
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int hf = 0; hf < 2; ++hf) {
 #pragma unroll
-        for (int m = 8; m >= 1; m >>= 1) {
-            const unsigned long long o = __shfl_xor_sync(kFull, best[i], m);
-            best[i] = best[i] > o ? best[i] : o;
+        for (int m = 1; m <= 2; m <<= 1) {
+            const unsigned long long o = __shfl_xor_sync(kFull, best[hf], m);
+            best[hf] = best[hf] > o ? best[hf] : o;
         }
-        const int n = n0 + ty * 4 + i;
-        if (tx == 0 && n < p.N) p.ws[((size_t)ks * p.N + n) * p.H + h] = best[i];
+        const int n = qr + 8 * hf;
+        if ((lane & 3) == 0 && n < p.N) p.ws[((size_t)ks * p.N + n) * p.H + h] = best[hf];
     }
 }
 

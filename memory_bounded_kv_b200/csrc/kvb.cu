@@ -352,13 +352,13 @@ kvb_status kvb_asm_lookup_merge(const uint16_t* q, const float* qbar, const uint
         !aligned16(workspace))
         return KVB_EINVAL;
     if (workspace_bytes < kvb_asm_workspace_bytes(N, H, K)) return KVB_EINVAL;
-    const int qtiles = (N + kvb::kAsmQT - 1) / kvb::kAsmQT;
+    const int qtiles = (N + kvb::kAtQT - 1) / kvb::kAtQT;
     if (qtiles > 65535) return KVB_EINVAL;
     kvb::AsmParams p{q, qbar, abar, log_zbar, o_self, lse_self, N, H, K, kvb::asm_ksplit(K), kvb::asm_kchunk(K),
                      idx, o, lse, static_cast<unsigned long long*>(workspace)};
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (set_smem(kvb::asm_score_kernel, kvb::kAsmSmem) != KVB_OK) return KVB_ECUDA;
-    kvb::asm_score_kernel<<<dim3(H, qtiles, p.ksplit), kvb::kAsmNT, kvb::kAsmSmem, st>>>(p);
+    if (set_smem(kvb::asm_score_tc_kernel, kvb::kAtSmem) != KVB_OK) return KVB_ECUDA;
+    kvb::asm_score_tc_kernel<<<dim3(H, qtiles, p.ksplit), kvb::kAtNT, kvb::kAtSmem, st>>>(p);
     if (launched() != KVB_OK) return KVB_ECUDA;
     const long long rows = (long long)N * H;
     kvb::asm_merge_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p);

@@ -250,3 +250,26 @@ def test_asm_exact_match_and_zero_vectors(oracle):
     rows = np.arange(N) != 7   # centroid 7 of head 1 is the zero vector: cos 0, not the maximum
     np.testing.assert_array_equal(idx[rows, 1], expect[rows, 1])
     check_asm(oracle, q, qbar, abar, lz, o_self, l_self, idx, o, lse)
+
+
+@pytest.mark.parametrize("eps_exp", [9, 13, 16])
+def test_asm_lookup_uses_full_fp32_centroids(oracle, eps_exp):
+    """Centroids whose order is decided below bf16 precision. For q = e0, centroid
+    (c0, 0.5, 0, ...) has cos c0 / sqrt(c0^2 + 0.25), increasing in c0; c0 = 1 + 2^-e
+    beats c0 = 1 by about 0.18 * 2^-e, far above the near-tie tolerance, yet 1 + 2^-e
+    rounds to 1 in bf16 (e >= 9). The winner sits at the higher index, so a contraction
+    that loses the low bits of the centroid ties and picks the lower one."""
+    N, H, K, d = 3, 2, 130, 128
+    q, qbar, abar, lz, o_self, l_self = asm_inputs(40 + eps_exp, N, H, K)
+    q[:] = 0
+    q[:, :, 0] = 0x3F80                                    # bf16 1.0: q = e0 in every row and head
+    qbar[:, :, 0] *= 0.1                                   # fillers: cos <= 0.1
+    for h in range(H):
+        qbar[h, 5] = 0
+        qbar[h, 5, :2] = [1.0, 0.5]
+        qbar[h, 70] = 0
+        qbar[h, 70, :2] = [np.float32(1.0) + np.float32(2.0 ** -eps_exp), 0.5]
+    assert np.float32(qbar[0, 70, 0]) != np.float32(1.0)
+    idx, o, lse = run_asm(q, qbar, abar, lz, o_self, l_self)
+    np.testing.assert_array_equal(idx, np.full((N, H), 70))
+    assert check_asm(oracle, q, qbar, abar, lz, o_self, l_self, idx, o, lse) == 0
