@@ -352,13 +352,19 @@ kvb_status kvb_asm_lookup_merge(const uint16_t* q, const float* qbar, const uint
         !aligned16(workspace))
         return KVB_EINVAL;
     if (workspace_bytes < kvb_asm_workspace_bytes(N, H, K)) return KVB_EINVAL;
-    const int qtiles = (N + kvb::kAtQT - 1) / kvb::kAtQT;
-    if (qtiles > 65535) return KVB_EINVAL;
-    kvb::AsmParams p{q, qbar, abar, log_zbar, o_self, lse_self, N, H, K, kvb::asm_ksplit(K), kvb::asm_kchunk(K),
-                     idx, o, lse, static_cast<unsigned long long*>(workspace)};
+    const int qtiles = (N + kvb::kUMT * kvb::kUQ - 1) / (kvb::kUMT * kvb::kUQ);
+    const long long items = (long long)H * qtiles * kvb::asm_ksplit(K);
+    if (items > (1ll << 30)) return KVB_EINVAL;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (set_smem(kvb::asm_score_tc_kernel, kvb::kAtSmem) != KVB_OK) return KVB_ECUDA;
-    kvb::asm_score_tc_kernel<<<dim3(H, qtiles, p.ksplit), kvb::kAtNT, kvb::kAtSmem, st>>>(p);
+    if (set_smem(kvb::asm_score_umma_kernel, kvb::kUSmem) != KVB_OK) return KVB_ECUDA;
+    // persistent: one CTA per SM (the shared memory allows no second), items split evenly
+    const int slots = resident_ctas(kvb::asm_score_umma_kernel, kvb::kUThreads, kvb::kUSmem);
+    if (slots < 1) return KVB_ECUDA;
+    const int per_cta = (int)((items + slots - 1) / slots);
+    const int grid = (int)((items + per_cta - 1) / per_cta);
+    kvb::AsmParams p{q, qbar, abar, log_zbar, o_self, lse_self, N, H, K, kvb::asm_ksplit(K), kvb::asm_kchunk(K),
+                     qtiles, per_cta, idx, o, lse, static_cast<unsigned long long*>(workspace)};
+    kvb::asm_score_umma_kernel<<<grid, kvb::kUThreads, kvb::kUSmem, st>>>(p);
     if (launched() != KVB_OK) return KVB_ECUDA;
     const long long rows = (long long)N * H;
     kvb::asm_merge_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p);

@@ -85,5 +85,5 @@ def test_other_entry_points_reject_bad_arguments_on_the_host():
     assert L.kvb_merge_states(f, f, 1, 1, 1, 1, 0, 4, 8, f, None, None) == _lib.KVB_EINVAL
     assert L.kvb_asm_lookup_merge(f, f, f, f, f, f, 4, 2, 16, 64, None, f, None, f, 1 << 20, None) == _lib.KVB_EINVAL
     ws = L.kvb_asm_workspace_bytes(256, 32, 4096)
-    assert ws == 8 * 256 * 32 * 8
+    assert ws == 32 * 256 * 32 * 8   # 32 ranges of 128 centroids, one 8-byte key per (range, query, head)
     assert L.kvb_asm_lookup_merge(f, f, f, f, f, f, 256, 32, 4096, 128, None, f, None, f, ws - 1, None) == _lib.KVB_EINVAL
