@@ -169,8 +169,9 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def kernel_src_hash() -> str:
-    with open(os.path.join(ROOT, "memory_bounded_kv_b200", "csrc", "decode_attn_tc.cuh"), "rb") as f:
+def kernel_src_hash(name: str = "decode_attn_tc.cuh") -> str:
+    """Hash of the dominant kernel's source: stored ncu traffic applies only to that exact source."""
+    with open(os.path.join(ROOT, "memory_bounded_kv_b200", "csrc", name), "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
@@ -328,6 +329,8 @@ class ASMBench:
     """A step: the 256 query tokens' causal self attention over the shared 2048-token cache
     (kvb_decode_attn, batch stride 0) and the memory lookup + merge (kvb_asm_lookup_merge)."""
 
+    KERNEL_SRC = "asm_lookup.cuh"
+
     # the fp32 contraction runs as three exact bf16 products per element (q . hi + q . mid + q . lo)
     PEAK_NOTE = "{kind} dense bf16 {bf16:.0f} TFLOP/s (bf16_tflops, burst) / 3 bf16 products per fp32 product"
 
@@ -399,7 +402,7 @@ class ASMBench:
         return 2.0 * w.N * w.H * w.K * w.d
 
     def kernel_name(self):
-        return "asm_score_tc_kernel + asm_merge_kernel (kvb_asm_lookup_merge)"
+        return "asm_score_umma_kernel + asm_merge_kernel (kvb_asm_lookup_merge)"
 
     def config(self):
         w = self.w
@@ -544,7 +547,7 @@ def run_kvb(args, world, rank, local):
     tokens = bench.tokens(W, K) if hasattr(bench, "tokens") else bench.tokens_per_step * K
     launches = bench.launches(W, K) if hasattr(bench, "launches") else bench.launches_per_step * K
     value = replica_value(tokens, world, ms)
-    src = kernel_src_hash()
+    src = kernel_src_hash(getattr(bench, "KERNEL_SRC", "decode_attn_tc.cuh"))
     if hasattr(bench, "flops"):      # attention-state-memory lookup: tensor bound (bf16 x 3)
         bf16_tf, bf16_kind = bf16_peak()
         peak_tf = bf16_tf / 3.0
