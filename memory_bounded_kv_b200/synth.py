@@ -216,6 +216,67 @@ def asm_workload(N: int = 256, H: int = 32, Hkv: int = 8, K: int = 4096, d: int 
     return w
 
 
+@dataclass
+class ASMIndex:
+    """A clustered attention-state memory with its two-level index.
+
+    Per head: C cluster directions u_c (unit, float32) serve as the first-level centroids
+    qhat [H, C, d]; cluster c holds a ragged number of entries (sizes around K / C, every entry
+    in exactly one cluster, ids scattered over [0, K)), each entry qbar_k = unit(u_c + sigma g).
+    members [H, K] int32 lists the entries cluster by cluster, offsets [H, C + 1] int32 bounds
+    each cluster's run. Queries are unit(u_c' + sigma_q g) for a random cluster c', in bf16.
+    """
+    seed: int
+    N: int
+    H: int
+    K: int
+    C: int
+    d: int
+    qhat: np.ndarray = field(repr=False, default=None)
+    offsets: np.ndarray = field(repr=False, default=None)
+    members: np.ndarray = field(repr=False, default=None)
+    qbar: np.ndarray = field(repr=False, default=None)
+    abar: np.ndarray = field(repr=False, default=None)
+    log_zbar: np.ndarray = field(repr=False, default=None)
+    q: np.ndarray = field(repr=False, default=None)
+    o_self: np.ndarray = field(repr=False, default=None)
+    lse_self: np.ndarray = field(repr=False, default=None)
+
+
+def _unit(x: np.ndarray) -> np.ndarray:
+    n = np.linalg.norm(x, axis=-1, keepdims=True)
+    return x / np.where(n > 0, n, 1.0)
+
+
+def asm_index_workload(N: int = 1, H: int = 32, K: int = 4096, C: int = 64, d: int = 128,
+                       sigma: float = 2.5, sigma_q: float = 2.0, seed: int = 6) -> ASMIndex:
+    w = ASMIndex(seed=seed, N=N, H=H, K=K, C=C, d=d)
+    g = rng(seed, _S_CACHE)
+    u = _unit(g.standard_normal((H, C, d)))
+    w.qhat = u.astype(np.float32)
+    w.qbar = np.zeros((H, K, d), np.float32)
+    w.members = np.zeros((H, K), np.int32)
+    w.offsets = np.zeros((H, C + 1), np.int32)
+    for h in range(H):
+        # ragged sizes: a multinomial split of K over the C clusters
+        sizes = g.multinomial(K, np.full(C, 1.0 / C))
+        w.offsets[h, 1:] = np.cumsum(sizes)
+        ids = g.permutation(K).astype(np.int32)
+        w.members[h] = ids
+        owner = np.repeat(np.arange(C), sizes)          # cluster of the i-th listed entry
+        x = u[h, owner] + sigma * g.standard_normal((K, d)) / np.sqrt(d)
+        w.qbar[h, ids] = _unit(x).astype(np.float32)
+    w.abar = normal_bf16(g, (H, K, d))
+    w.log_zbar = g.uniform(5.0, 12.0, (H, K)).astype(np.float32)
+    gq = rng(seed, _S_STEP)
+    target = gq.integers(0, C, (N, H))
+    xq = u[np.arange(H)[None, :], target] + sigma_q * gq.standard_normal((N, H, d)) / np.sqrt(d)
+    w.q = to_bf16_bits(_unit(xq).astype(np.float32))
+    w.o_self = gq.standard_normal((N, H, d)).astype(np.float32)
+    w.lse_self = gq.uniform(3.0, 9.0, (N, H)).astype(np.float32)
+    return w
+
+
 # --------------------------------------------------------------------------
 # config 5: memento-style block compaction (sawtooth cache)
 # --------------------------------------------------------------------------

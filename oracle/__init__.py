@@ -17,6 +17,11 @@ Parity status (what pins each function, see tests/test_oracle_*.py):
                    compaction == masked SDPA over the old cache
   asm_lookup_merge pinned: sklearn cosine_similarity argmax, exact-match
                    retrieval, merged state == SDPA over prefix + self
+  asm_hier_lookup_merge
+                   pinned: m = C over a partition == sklearn cosine_similarity
+                   argmax; constructed indexes with known answers (best
+                   centroid outside the selected clusters, coarse ties,
+                   empty clusters); merge as asm_lookup_merge
 """
 from __future__ import annotations
 
@@ -60,8 +65,10 @@ def _load():
         lib.oracle_compact_blocks.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I]
         lib.oracle_asm_cosines.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _P]
         lib.oracle_asm_lookup_merge.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P]
+        lib.oracle_asm_hier_lookup_merge.argtypes = [_P] * 9 + [_I] * 6 + [_P] * 4
         for f in (lib.oracle_decode_attn, lib.oracle_merge_states, lib.oracle_evict_insert,
-                  lib.oracle_compact_blocks, lib.oracle_asm_cosines, lib.oracle_asm_lookup_merge):
+                  lib.oracle_compact_blocks, lib.oracle_asm_cosines, lib.oracle_asm_lookup_merge,
+                  lib.oracle_asm_hier_lookup_merge):
             f.restype = _I
         _lib = lib
     return _lib
@@ -193,3 +200,30 @@ def asm_lookup_merge(q, qbar, abar, log_zbar, o_self, lse_self):
                                        _ptr(lse_self), N, H, K, d, _ptr(idx), _ptr(o), _ptr(lse)),
            "oracle_asm_lookup_merge")
     return idx, o, lse
+
+
+def asm_hier_lookup_merge(q, qhat, offsets, members, qbar, abar, log_zbar, o_self, lse_self, m: int):
+    """Two-level lookup. Returns (sel [N, H, m] int32, idx [N, H] int32, o [N, H, d] float64,
+    lse [N, H] float64); idx = -1 where the selected clusters hold no member."""
+    lib = _load()
+    q = _c(q, np.uint16)
+    qhat = _c(qhat, np.float32)
+    offsets = _c(offsets, np.int32)
+    members = _c(members, np.int32)
+    qbar = _c(qbar, np.float32)
+    abar = _c(abar, np.uint16)
+    log_zbar = _c(log_zbar, np.float32)
+    o_self = _c(o_self, np.float32)
+    lse_self = _c(lse_self, np.float32)
+    N, H, d = q.shape
+    K = qbar.shape[1]
+    C = qhat.shape[1]
+    sel = np.zeros((N, H, m), np.int32)
+    idx = np.zeros((N, H), np.int32)
+    o = np.zeros((N, H, d), np.float64)
+    lse = np.zeros((N, H), np.float64)
+    _check(lib.oracle_asm_hier_lookup_merge(_ptr(q), _ptr(qhat), _ptr(offsets), _ptr(members), _ptr(qbar),
+                                            _ptr(abar), _ptr(log_zbar), _ptr(o_self), _ptr(lse_self), N, H, K,
+                                            C, int(m), d, _ptr(sel), _ptr(idx), _ptr(o), _ptr(lse)),
+           "oracle_asm_hier_lookup_merge")
+    return sel, idx, o, lse

@@ -38,6 +38,7 @@
 // Status codes: 0 = ok, 1 = invalid argument, 3 = invalid data (a length,
 // position or range that the preconditions exclude).
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -336,6 +337,60 @@ int oracle_asm_lookup_merge(const uint16_t* q, const float* qbar, const uint16_t
             double* a = o + nh * d;
             for (int e = 0; e < d; ++e) a[e] = static_cast<double>(o_self[nh * d + e]);
             lse[nh] = static_cast<double>(lse_self[nh]);
+            const int64_t hk = static_cast<int64_t>(h) * K + best;
+            for (int e = 0; e < d; ++e) mem[e] = bf16_value(abar[hk * d + e]);
+            merge_two(a, &lse[nh], mem.data(), static_cast<double>(log_zbar[hk]), d);
+        }
+    }
+    return 0;
+}
+
+// Two-level attention-state-memory lookup and merge ([ASM] hierarchical lookup index), per (n, h):
+//   s_c = cos(q, qhat_c) for the C first-level centroids of head h;
+//   S = the m clusters with the largest s_c (the lower c among equal values), m = min(m, C);
+//   c* = argmax of cos(q, qbar_k) over the members k of the clusters in S (the lowest k among
+//        equal values); no member at all: c* = -1 and the state is the self state;
+//   (o, lse) = merge((o_self, lse_self), (abar[c*], log_zbar[c*])).
+// Cluster c of head h holds members[h * K + i] for offsets[h * (C + 1) + c] <= i < offsets[... + c + 1].
+//   qhat [H, C, d] f32; offsets [H, C + 1]; members [H, K] in [0, K); the rest as oracle_asm_lookup_merge
+//   -> sel [N, H, m] (the selected clusters, best first), idx [N, H], o [N, H, d], lse [N, H].
+int oracle_asm_hier_lookup_merge(const uint16_t* q, const float* qhat, const int32_t* offsets,
+                                 const int32_t* members, const float* qbar, const uint16_t* abar,
+                                 const float* log_zbar, const float* o_self, const float* lse_self,
+                                 int N, int H, int K, int C, int m, int d,
+                                 int32_t* sel, int32_t* idx, double* o, double* lse) {
+    if (N < 0 || H <= 0 || K < 1 || C < 1 || m < 1 || d <= 0) return 1;
+    const int mm = m < C ? m : C;
+    std::vector<double> coarse(static_cast<size_t>(C)), cosk(static_cast<size_t>(K));
+    std::vector<char> taken(static_cast<size_t>(C));
+    std::vector<double> mem(static_cast<size_t>(d));
+    for (int n = 0; n < N; ++n) {
+        for (int h = 0; h < H; ++h) {
+            oracle_asm_cosines(q, qhat, N, H, C, d, n, h, coarse.data());
+            oracle_asm_cosines(q, qbar, N, H, K, d, n, h, cosk.data());
+            const int64_t nh = static_cast<int64_t>(n) * H + h;
+            std::fill(taken.begin(), taken.end(), 0);
+            int best = -1;
+            for (int j = 0; j < mm; ++j) {
+                int c_sel = -1;   // the largest cosine not taken yet, the lower c on ties
+                for (int c = 0; c < C; ++c)
+                    if (!taken[c] && (c_sel < 0 || coarse[c] > coarse[c_sel])) c_sel = c;
+                taken[c_sel] = 1;
+                sel[nh * m + j] = c_sel;
+                const int32_t* off = offsets + static_cast<int64_t>(h) * (C + 1);
+                if (off[c_sel] < 0 || off[c_sel + 1] > K) return 2;
+                for (int32_t i = off[c_sel]; i < off[c_sel + 1]; ++i) {
+                    const int32_t kk = members[static_cast<int64_t>(h) * K + i];
+                    if (kk < 0 || kk >= K) return 2;
+                    if (best < 0 || cosk[kk] > cosk[best] || (cosk[kk] == cosk[best] && kk < best)) best = kk;
+                }
+            }
+            for (int j = mm; j < m; ++j) sel[nh * m + j] = -1;
+            idx[nh] = best;
+            double* a = o + nh * d;
+            for (int e = 0; e < d; ++e) a[e] = static_cast<double>(o_self[nh * d + e]);
+            lse[nh] = static_cast<double>(lse_self[nh]);
+            if (best < 0) continue;
             const int64_t hk = static_cast<int64_t>(h) * K + best;
             for (int e = 0; e < d; ++e) mem[e] = bf16_value(abar[hk * d + e]);
             merge_two(a, &lse[nh], mem.data(), static_cast<double>(log_zbar[hk]), d);
