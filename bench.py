@@ -61,6 +61,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the timed steps one by one")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--asm-crossover", action="store_true",
+                    help="time the linear and the two-level memory lookups alone over query counts and memory "
+                         "sizes (one GPU; L2 flushed between iterations) instead of a decode step")
     return ap.parse_args()
 
 
@@ -645,6 +648,82 @@ def run_reference(args, world, rank):
     }
 
 
+def run_asm_crossover(args) -> dict:
+    """Lookup + merge alone, linear (kvb_asm_lookup_merge) against two-level
+    (kvb_asm_hier_lookup_merge, C = sqrt(K) clusters, top-16), on the clustered memory
+    of synth.asm_index_workload: 32 heads, d = 128, N query tokens per call. Every
+    timed call starts with a cold L2 (a 256 MiB buffer is written before it, outside
+    the events), as in decoding, where the other layers evict the memory between
+    lookups. Recall = share of (query, head) whose two-level entry is the linear one."""
+    import memory_bounded_kv_b200 as kvb
+    from memory_bounded_kv_b200 import synth
+    hbm_peak, peak_kind = peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    iters, warm = max(5, min(args.steps, 200)), max(3, args.warmup)
+    rows = []
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    for K in (4096, 16384):
+        C = int(round(K ** 0.5))
+        m = 16
+        w = synth.asm_index_workload(N=256, H=32, K=K, C=C)
+        g = {name: _dev(getattr(w, name)) for name in ("q", "qhat", "offsets", "members", "qbar", "abar",
+                                                      "log_zbar", "o_self", "lse_self")}
+        for N in (1, 8, 64, 256):
+            q, o_self, l_self = g["q"][:N].contiguous(), g["o_self"][:N].contiguous(), g["lse_self"][:N].contiguous()
+            H, d = w.H, w.d
+            out = {}
+            for kind in ("linear", "hier"):
+                idx = torch.zeros(N, H, dtype=torch.int32, device="cuda")
+                o = torch.zeros(N, H, d, device="cuda")
+                lse = torch.zeros(N, H, device="cuda")
+                if kind == "linear":
+                    ws = torch.empty(kvb.kvb_asm_workspace_bytes(N, H, K), dtype=torch.uint8, device="cuda")
+                    call = lambda: kvb.kvb_asm_lookup_merge(q, g["qbar"], g["abar"], g["log_zbar"], o_self, l_self,
+                                                            idx, o, lse, ws)
+                else:
+                    ws = torch.empty(kvb.kvb_asm_hier_workspace_bytes(N, H, m), dtype=torch.uint8, device="cuda")
+                    call = lambda: kvb.kvb_asm_hier_lookup_merge(q, g["qhat"], g["offsets"], g["members"], g["qbar"],
+                                                                 g["abar"], g["log_zbar"], o_self, l_self, idx, o,
+                                                                 lse, ws, m)
+                ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                      for _ in range(iters)]
+                for _ in range(warm):
+                    call()
+                torch.cuda.synchronize()
+                for a, b in ev:
+                    flush.fill_(1)
+                    a.record()
+                    call()
+                    b.record()
+                torch.cuda.synchronize()
+                ms = statistics.median(x.elapsed_time(y) for x, y in ev)
+                out[kind] = (ms, idx.cpu().numpy(), ws)
+            # algorithmic bytes of the two-level lookup: the first level, the selected clusters' rows, the merge
+            nhm = N * H * m
+            sel = out["hier"][2][nhm * 8: nhm * 12].view(torch.int32).cpu().numpy().reshape(N, H, m)
+            sizes = np.diff(w.offsets, axis=1)
+            rows_read = sum(int(sizes[h][sel[n, h][sel[n, h] >= 0]].sum()) for n in range(N) for h in range(H))
+            hier_bytes = (N * H * C + rows_read) * d * 4 + N * H * (d * 2 + d * 4 * 2 + d * 2)
+            lin_bytes = H * K * d * 4 + N * H * (d * 2 + d * 4 * 2 + d * 2)
+            rows.append({
+                "K": K, "C": C, "m": m, "N": N,
+                "linear_us": round(out["linear"][0] * 1e3, 2), "hier_us": round(out["hier"][0] * 1e3, 2),
+                "speedup": round(out["linear"][0] / out["hier"][0], 2),
+                "recall": round(float((out["linear"][1] == out["hier"][1]).mean()), 4),
+                "hier_gbs": round(hier_bytes / (out["hier"][0] / 1e3) / 1e9, 1),
+                "hier_frac": round(hier_bytes / (out["hier"][0] / 1e3) / 1e9 / hbm_peak, 3),
+                "linear_gbs": round(lin_bytes / (out["linear"][0] / 1e3) / 1e9, 1),
+            })
+    clk = clocks.stop()
+    return {"metric": "ASM lookup + merge latency, linear vs two-level (median of cold-L2 calls)",
+            "unit": "us", "higher_is_better": False, "n_gpus": 1, "steps": iters, "warmup": warm,
+            "dtype": "f32", "data": "synthetic clustered memory (synth.asm_index_workload)",
+            "config": {"workload": "attention-state memory, 32 heads, d 128, top-16 of sqrt(K) clusters",
+                       "l2": "flushed before every timed call (256 MiB write)"},
+            "peak_gbs": hbm_peak, "peak_source": f"{peak_kind} (hbm_gbs)", "rows": rows, "clocks": clk}
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -653,6 +732,9 @@ def main():
         out = run_reference(args, world, rank)
         if out is not None:
             print(json.dumps(out), flush=True)
+        return
+    if args.asm_crossover:
+        print(json.dumps(run_asm_crossover(args)), flush=True)
         return
     world, rank, local = dist_init()
     try:

@@ -280,6 +280,8 @@ kvb_status kvb_compact_blocks(uint16_t* k, uint16_t* v, int32_t* pos, float* log
  * workspace: device scratch of kvb_asm_workspace_bytes(N, H, K) bytes,
  * 16-byte aligned, contents irrelevant on entry.
  * Requirements: d == 128; N, H, K >= 1; all pointers 16-byte aligned.
+ * A (query, head) whose every cosine is NaN retrieves nothing: idx = -1 and
+ * (o, lse) = (o_self, lse_self).
  * ---------------------------------------------------------------------- */
 size_t kvb_asm_workspace_bytes(int32_t N, int32_t H, int32_t K);
 
@@ -288,6 +290,45 @@ kvb_status kvb_asm_lookup_merge(const uint16_t* q, const float* qbar, const uint
                                 const float* lse_self, int32_t N, int32_t H, int32_t K,
                                 int32_t d, int32_t* idx, float* o, float* lse,
                                 void* workspace, size_t workspace_bytes, kvb_stream stream);
+
+/* ------------------------------------------------------------------------
+ * kvb_asm_hier_lookup_merge -- two-level attention-state-memory lookup
+ *
+ * [ASM] hierarchical lookup index (technical novelty: retrieval in
+ * O(log K) instead of O(K); expanding the top-16 first-level centroids
+ * matches the linear top-1). The index is an input, like qbar: per head h,
+ * C first-level centroids qhat[h, c] and a partition of the K entries into
+ * clusters, listed cluster by cluster: cluster c holds the entries
+ * members[h, i] for offsets[h, c] <= i < offsets[h, c + 1]. For query token
+ * n and head h:
+ *   S  = the m clusters with the largest cos(q[n,h], qhat[h,c]) (the lower c
+ *        among equal values; all C when m >= C);
+ *   c* = argmax of cos(q[n,h], qbar[h,k]) over the members k of the clusters
+ *        in S (the lowest k among equal values);
+ *   (o, lse) = merge((o_self, lse_self), (abar[h, c*], log_zbar[h, c*]))
+ *        as kvb_asm_lookup_merge; when the clusters in S hold no entry,
+ *        idx = -1 and (o, lse) = (o_self, lse_self).
+ * Layouts (contiguous): q [N, H, d] bf16; qhat [H, C, d] f32; offsets
+ * [H, C + 1] int32 (0 <= offsets[h, c] <= offsets[h, c + 1] <= K); members
+ * [H, K] int32 in [0, K); qbar, abar, log_zbar, o_self, lse_self, idx, o,
+ * lse as kvb_asm_lookup_merge (idx may be NULL, lse may be NULL).
+ * workspace: device scratch of kvb_asm_hier_workspace_bytes(N, H, m) bytes,
+ * 16-byte aligned, contents irrelevant on entry. Three launches on
+ * `stream`: first-level scores and selection, member scores per selected
+ * cluster, reduction + merge.
+ * Requirements: d == 128; N, H, K >= 1; 1 <= C <= 1024; 1 <= m <= 64;
+ * q, qhat, qbar, abar, o_self, o 16-byte aligned. Offsets out of order or
+ * member ids outside [0, K) found on the device are skipped and set
+ * KVB_DERR_RANGE.
+ * ---------------------------------------------------------------------- */
+size_t kvb_asm_hier_workspace_bytes(int32_t N, int32_t H, int32_t m);
+
+kvb_status kvb_asm_hier_lookup_merge(const uint16_t* q, const float* qhat, const int32_t* offsets,
+                                     const int32_t* members, const float* qbar, const uint16_t* abar,
+                                     const float* log_zbar, const float* o_self, const float* lse_self,
+                                     int32_t N, int32_t H, int32_t K, int32_t C, int32_t m, int32_t d,
+                                     int32_t* idx, float* o, float* lse,
+                                     void* workspace, size_t workspace_bytes, kvb_stream stream);
 
 /* ------------------------------------------------------------------------
  * Errors and diagnostics

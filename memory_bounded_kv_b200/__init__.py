@@ -19,7 +19,8 @@ from . import _lib
 
 __all__ = [
     "KvbError", "kvb_decode_attn", "kvb_decode_attn_noalloc", "kvb_merge_states", "kvb_evict_insert", "kvb_compact_blocks",
-    "kvb_asm_workspace_bytes", "kvb_asm_lookup_merge", "kvb_get_error", "kvb_abi_version",
+    "kvb_asm_workspace_bytes", "kvb_asm_lookup_merge", "kvb_asm_hier_workspace_bytes",
+    "kvb_asm_hier_lookup_merge", "kvb_get_error", "kvb_abi_version",
     "decode_workspace", "evict_candidates",
 ]
 
@@ -290,3 +291,34 @@ def kvb_asm_lookup_merge(q, qbar, abar, log_zbar, o_self, lse_self, idx, o, lse,
     _check(_lib.lib().kvb_asm_lookup_merge(_ptr(q), _ptr(qbar), _ptr(abar), _ptr(log_zbar), _ptr(o_self),
                                            _ptr(lse_self), N, H, K, d, _ptr(idx), _ptr(o), _ptr(lse),
                                            _ptr(workspace), nbytes, _stream(stream)), "kvb_asm_lookup_merge")
+
+
+def kvb_asm_hier_workspace_bytes(N: int, H: int, m: int) -> int:
+    return int(_lib.lib().kvb_asm_hier_workspace_bytes(N, H, m))
+
+
+def kvb_asm_hier_lookup_merge(q, qhat, offsets, members, qbar, abar, log_zbar, o_self, lse_self, idx, o, lse,
+                              workspace, m: int, *, stream=None) -> None:
+    """Two-level attention-state-memory lookup and merge; see kvb_asm_hier_lookup_merge in
+    include/kvb.h. workspace: a uint8 CUDA tensor of at least kvb_asm_hier_workspace_bytes(N, H, m)
+    bytes."""
+    _need(q, torch.bfloat16, "q"); _need(qhat, torch.float32, "qhat"); _need(offsets, torch.int32, "offsets")
+    _need(members, torch.int32, "members"); _need(qbar, torch.float32, "qbar"); _need(abar, torch.bfloat16, "abar")
+    _need(log_zbar, torch.float32, "log_zbar"); _need(o_self, torch.float32, "o_self")
+    _need(lse_self, torch.float32, "lse_self"); _need(o, torch.float32, "o")
+    for name, x in (("q", q), ("qhat", qhat), ("offsets", offsets), ("members", members), ("qbar", qbar),
+                    ("abar", abar), ("log_zbar", log_zbar), ("o_self", o_self), ("lse_self", lse_self), ("o", o),
+                    ("workspace", workspace)):
+        _contig(x, name)
+    if idx is not None:
+        _need(idx, torch.int32, "idx"); _contig(idx, "idx")
+    if lse is not None:
+        _need(lse, torch.float32, "lse"); _contig(lse, "lse")
+    N, H, d = q.shape
+    K = qbar.shape[1]
+    C = qhat.shape[1]
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(_lib.lib().kvb_asm_hier_lookup_merge(_ptr(q), _ptr(qhat), _ptr(offsets), _ptr(members), _ptr(qbar),
+                                                _ptr(abar), _ptr(log_zbar), _ptr(o_self), _ptr(lse_self), N, H, K,
+                                                C, int(m), d, _ptr(idx), _ptr(o), _ptr(lse), _ptr(workspace),
+                                                nbytes, _stream(stream)), "kvb_asm_hier_lookup_merge")

@@ -388,6 +388,7 @@ __global__ void __launch_bounds__(256) asm_merge_kernel(const __grid_constant__ 
     const long long nh = (long long)blockIdx.x * 8 + warp;
     if (nh >= (long long)p.N * p.H) return;
     const int n = (int)(nh / p.H), h = (int)(nh % p.H);
+    griddep_wait();   // the keys come from the previous kernel (a no-op without programmatic launch)
     unsigned long long best = 0ull;
     for (int s = lane; s < p.ksplit; s += 32) {
         const unsigned long long x = p.ws[((size_t)s * p.N + n) * p.H + h];
@@ -398,8 +399,14 @@ __global__ void __launch_bounds__(256) asm_merge_kernel(const __grid_constant__ 
         const unsigned long long o = __shfl_xor_sync(kFull, best, m);
         best = best > o ? best : o;
     }
-    // no key at all (every score NaN): index 0
-    const int k = (best == 0ull) ? 0 : (int)(0xffffffffu - (unsigned)(best & 0xffffffffull));
+    if (best == 0ull) {   // nothing retrieved (no candidate, or every score NaN): the self state
+        if (lane == 0 && p.idx != nullptr) p.idx[nh] = -1;
+        if (lane == 0 && p.lse != nullptr) p.lse[nh] = p.lse_self[nh];
+        *reinterpret_cast<float4*>(p.o + nh * kAsmD + lane * 4) =
+            *reinterpret_cast<const float4*>(p.o_self + nh * kAsmD + lane * 4);
+        return;
+    }
+    const int k = (int)(0xffffffffu - (unsigned)(best & 0xffffffffull));
     if (lane == 0 && p.idx != nullptr) p.idx[nh] = k;
     const float ls = p.lse_self[nh];
     const float lm = p.lz[(size_t)h * p.K + k];

@@ -10,6 +10,7 @@
 
 #include "../../include/kvb.h"
 #include "asm_lookup.cuh"
+#include "asm_hier.cuh"
 #include "common.cuh"
 #include "compact_blocks.cuh"
 #include "decode_attn_tc.cuh"
@@ -192,7 +193,7 @@ inline size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
 extern "C" {
 
-int32_t kvb_abi_version(void) { return 2; }
+int32_t kvb_abi_version(void) { return 3; }
 
 const char* kvb_status_str(kvb_status s) {
     switch (s) {
@@ -369,6 +370,46 @@ kvb_status kvb_asm_lookup_merge(const uint16_t* q, const float* qbar, const uint
     const long long rows = (long long)N * H;
     kvb::asm_merge_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p);
     return launched();
+}
+
+size_t kvb_asm_hier_workspace_bytes(int32_t N, int32_t H, int32_t m) {
+    if (N < 1 || H < 1 || m < 1) return 0;
+    return (size_t)N * H * m * (sizeof(unsigned long long) + sizeof(int32_t));
+}
+
+kvb_status kvb_asm_hier_lookup_merge(const uint16_t* q, const float* qhat, const int32_t* offsets,
+                                     const int32_t* members, const float* qbar, const uint16_t* abar,
+                                     const float* log_zbar, const float* o_self, const float* lse_self,
+                                     int32_t N, int32_t H, int32_t K, int32_t C, int32_t m, int32_t d,
+                                     int32_t* idx, float* o, float* lse, void* workspace,
+                                     size_t workspace_bytes, kvb_stream stream) {
+    if (d != kvb::kHierD || N < 1 || H < 1 || K < 1 || C < 1 || C > kvb::kHierMaxC || m < 1 ||
+        m > kvb::kHierMaxM)
+        return KVB_EINVAL;
+    if (!q || !qhat || !offsets || !members || !qbar || !abar || !log_zbar || !o_self || !lse_self || !o ||
+        !workspace)
+        return KVB_EINVAL;
+    if (!aligned16(q) || !aligned16(qhat) || !aligned16(qbar) || !aligned16(abar) || !aligned16(o_self) ||
+        !aligned16(o) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(offsets) & 3) ||
+        (reinterpret_cast<uintptr_t>(members) & 3))
+        return KVB_EINVAL;
+    if (workspace_bytes < kvb_asm_hier_workspace_bytes(N, H, m)) return KVB_EINVAL;
+    const long long nh = (long long)N * H;
+    if (nh * m > (1ll << 31) - 1) return KVB_EINVAL;   // one CTA per (selected cluster, query, head)
+    auto* keys = static_cast<unsigned long long*>(workspace);
+    auto* sel = reinterpret_cast<int32_t*>(keys + nh * m);
+    kvb::AsmHierParams hp{q, qhat, offsets, members, qbar, N, H, K, C, m, sel, keys};
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // three launches chained by programmatic dependent launch: each waits (griddepcontrol.wait)
+    // for its predecessor's results, only the launch latency overlaps
+    const size_t smem = kvb::hier_select_smem(C);
+    if (launch_pdl(kvb::asm_hier_select_kernel, dim3((unsigned)nh), dim3(256), smem, st, hp) != KVB_OK)
+        return KVB_ECUDA;
+    if (launch_pdl(kvb::asm_hier_score_kernel, dim3((unsigned)(nh * m)), dim3(256), 0, st, hp) != KVB_OK)
+        return KVB_ECUDA;
+    // reduction over the m selected clusters' keys + merge: the linear lookup's merge kernel
+    kvb::AsmParams p{q, qbar, abar, log_zbar, o_self, lse_self, N, H, K, m, 0, 0, 0, idx, o, lse, keys};
+    return launch_pdl(kvb::asm_merge_kernel, dim3((unsigned)((nh + 7) / 8)), dim3(256), 0, st, p);
 }
 
 }  // extern "C"

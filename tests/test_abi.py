@@ -47,7 +47,7 @@ def test_attn_args_struct_matches_header():
 
 def test_status_strings_and_version():
     L = _lib.lib()
-    assert L.kvb_abi_version() == 2
+    assert L.kvb_abi_version() == 3
     assert L.kvb_status_str(0) == b"ok"
     assert L.kvb_status_str(1) == b"invalid argument"
 
@@ -84,6 +84,18 @@ def test_other_entry_points_reject_bad_arguments_on_the_host():
     assert L.kvb_compact_blocks(f, f, f, None, f, f, f, 1, 1, 12, 64, None) == _lib.KVB_EINVAL
     assert L.kvb_merge_states(f, f, 1, 1, 1, 1, 0, 4, 8, f, None, None) == _lib.KVB_EINVAL
     assert L.kvb_asm_lookup_merge(f, f, f, f, f, f, 4, 2, 16, 64, None, f, None, f, 1 << 20, None) == _lib.KVB_EINVAL
+    # two-level lookup: C, m out of range, short workspace, misaligned members
+    assert L.kvb_asm_hier_lookup_merge(f, f, f, f, f, f, f, f, f, 1, 2, 64, 0, 4, 128, None, f, None, f, 1 << 20,
+                                       None) == _lib.KVB_EINVAL
+    assert L.kvb_asm_hier_lookup_merge(f, f, f, f, f, f, f, f, f, 1, 2, 64, 1025, 4, 128, None, f, None, f, 1 << 20,
+                                       None) == _lib.KVB_EINVAL
+    assert L.kvb_asm_hier_lookup_merge(f, f, f, f, f, f, f, f, f, 1, 2, 64, 8, 65, 128, None, f, None, f, 1 << 20,
+                                       None) == _lib.KVB_EINVAL
+    assert L.kvb_asm_hier_workspace_bytes(3, 2, 16) == 3 * 2 * 16 * 12
+    assert L.kvb_asm_hier_lookup_merge(f, f, f, f, f, f, f, f, f, 3, 2, 64, 8, 16, 128, None, f, None, f,
+                                       3 * 2 * 16 * 12 - 1, None) == _lib.KVB_EINVAL
+    assert L.kvb_asm_hier_lookup_merge(f, f, f, ctypes.c_void_p((1 << 20) + 2), f, f, f, f, f, 1, 2, 64, 8, 4, 128,
+                                       None, f, None, f, 1 << 20, None) == _lib.KVB_EINVAL
     ws = L.kvb_asm_workspace_bytes(256, 32, 4096)
     assert ws == 32 * 256 * 32 * 8   # 32 ranges of 128 centroids, one 8-byte key per (range, query, head)
     assert L.kvb_asm_lookup_merge(f, f, f, f, f, f, 256, 32, 4096, 128, None, f, None, f, ws - 1, None) == _lib.KVB_EINVAL
