@@ -8,9 +8,10 @@
 // contractions: per (query, head), C + sum of the selected clusters' sizes rows
 // of 512 bytes. The win over the linear lookup is at few queries per step.
 //
-//   asm_hier_select_kernel  one CTA per (n, h): C first-level scores, then m
-//                           rounds of a warp argmax over packed (score, -c)
-//                           keys -> sel [N, H, m]
+//   asm_hier_select_kernel  one CTA per (n, h): C first-level scores as packed
+//                           (score, -c) keys; the m largest by rank (C <= 256,
+//                           every thread ranks its clusters against all C) or
+//                           by m rounds of a warp argmax -> sel [N, H, m]
 //   asm_hier_score_kernel   one CTA per (selected cluster j, n, h): the
 //                           members' scores, best (score, -k) key -> keys [m, N, H]
 // Rows are read by whole warps (one coalesced 512-byte access per row, 8 rows
@@ -38,8 +39,8 @@ struct AsmHierParams {
     unsigned long long* keys;   // [m][N][H]
 };
 
-// bytes of shared memory of the select kernel: C scores, then C taken flags
-__host__ __device__ inline size_t hier_select_smem(int C) { return (size_t)C * sizeof(float) + (size_t)C; }
+// bytes of shared memory of the select kernel: C packed (score, -c) keys, then C taken flags
+__host__ __device__ inline size_t hier_select_smem(int C) { return (size_t)C * 8 + (size_t)C; }
 
 // q[nh] (bf16, 128): lane l holds dims 4l..4l+3
 __device__ __forceinline__ float4 hier_q4(const uint16_t* q, long long nh, int lane) {
@@ -55,21 +56,46 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // Scores q . x / |x| of up to 8 fp32 rows of 128 (0 for a zero row), the warp reading each
 // row as one coalesced 512-byte access (lane l: elements 4l..4l+3), the 8 rows in flight at
-// once. rows[r] == nullptr: no row (score unused). Every lane returns all 8 scores.
-__device__ __forceinline__ void hier_score8(const float4 qv, const float* const (&rows)[8], float (&score)[8],
-                                            int lane) {
-    float dot[8], ss[8];
+// once. rows[r] == nullptr: no row. The 16 partial sums (8 dots, 8 squared norms) are reduced
+// by a butterfly that halves the values each step (16 shuffles in all): afterwards lanes 2r
+// and 2r + 1 hold the score of row r; the return value is meaningful on those lanes.
+__device__ __forceinline__ float hier_score8(const float4 qv, const float* const (&rows)[8], int lane) {
+    float v[16];
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
         const float4 x = rows[r] ? __ldg(reinterpret_cast<const float4*>(rows[r]) + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
-        dot[r] = fmaf(qv.x, x.x, fmaf(qv.y, x.y, fmaf(qv.z, x.z, qv.w * x.w)));
-        ss[r] = fmaf(x.x, x.x, fmaf(x.y, x.y, fmaf(x.z, x.z, x.w * x.w)));
+        v[r] = fmaf(qv.x, x.x, fmaf(qv.y, x.y, fmaf(qv.z, x.z, qv.w * x.w)));
+        v[8 + r] = fmaf(x.x, x.x, fmaf(x.y, x.y, fmaf(x.z, x.z, x.w * x.w)));
+    }
+    // step with lane bit b: keep the half of the values selected by the bit, add the partner's
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const bool up = lane & 16;
+        const float send = up ? v[i] : v[8 + i], keep = up ? v[8 + i] : v[i];
+        v[i] = keep + __shfl_xor_sync(kFull, send, 16);
     }
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        const float d = warp_sum(dot[r]), n = warp_sum(ss[r]);
-        score[r] = (n > 0.f) ? d * (1.f / sqrtf(n)) : 0.f;
+    for (int i = 0; i < 4; ++i) {
+        const bool up = lane & 8;
+        const float send = up ? v[i] : v[4 + i], keep = up ? v[4 + i] : v[i];
+        v[i] = keep + __shfl_xor_sync(kFull, send, 8);
     }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const bool up = lane & 4;
+        const float send = up ? v[i] : v[2 + i], keep = up ? v[2 + i] : v[i];
+        v[i] = keep + __shfl_xor_sync(kFull, send, 4);
+    }
+    {
+        const bool up = lane & 2;
+        const float send = up ? v[0] : v[1], keep = up ? v[1] : v[0];
+        v[0] = keep + __shfl_xor_sync(kFull, send, 2);
+    }
+    v[0] += __shfl_xor_sync(kFull, v[0], 1);
+    // lane l now holds value 8 (l >> 4 & 1) + 4 (l >> 3 & 1) + 2 (l >> 2 & 1) + (l >> 1 & 1):
+    // lanes 2r, 2r + 1 the dot of row r, lanes 16 + 2r, 16 + 2r + 1 its squared norm
+    const float ss = __shfl_xor_sync(kFull, v[0], 16);
+    return (ss > 0.f) ? v[0] * (1.f / sqrtf(ss)) : 0.f;
 }
 
 __device__ __forceinline__ unsigned long long hier_key(float score, int id) {
@@ -88,8 +114,8 @@ __device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v)
 // one CTA (8 warps) per (n, h): the C first-level scores, 64 rows at a time, then warp 0 takes
 // the m best clusters in m rounds of a warp argmax over packed (score, -c) keys
 __global__ void __launch_bounds__(256) asm_hier_select_kernel(const __grid_constant__ AsmHierParams p) {
-    extern __shared__ __align__(16) float s_sc[];
-    unsigned char* taken = reinterpret_cast<unsigned char*>(s_sc + p.C);
+    extern __shared__ __align__(16) unsigned long long s_key[];
+    unsigned char* taken = reinterpret_cast<unsigned char*>(s_key + p.C);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long nh = blockIdx.x;
     const int h = (int)(nh % p.H);
@@ -100,33 +126,40 @@ __global__ void __launch_bounds__(256) asm_hier_select_kernel(const __grid_const
         const float* rows[8];
 #pragma unroll
         for (int r = 0; r < 8; ++r) rows[r] = (c0 + r < p.C) ? p.qhat + ((size_t)h * p.C + c0 + r) * kHierD : nullptr;
-        float sc[8];
-        hier_score8(qv, rows, sc, lane);
-#pragma unroll
-        for (int r = 0; r < 8; ++r)
-            if (lane == r && c0 + r < p.C) {
-                s_sc[c0 + r] = sc[r];
-                taken[c0 + r] = 0;
-            }
+        const float sc = hier_score8(qv, rows, lane);
+        const int r = lane >> 1;
+        if (lane < 16 && !(lane & 1) && c0 + r < p.C) {
+            s_key[c0 + r] = hier_key(sc, c0 + r);
+            taken[c0 + r] = 0;
+        }
     }
     __syncthreads();
-    if (warp != 0) return;
     const int mm = min(p.m, p.C);
-    for (int j = 0; j < p.m; ++j) {
-        int out = -1;
-        if (j < mm) {
-            unsigned long long best = 0ull;
-            for (int c = lane; c < p.C; c += 32)
-                if (!taken[c]) {
-                    const unsigned long long k = hier_key(s_sc[c], c);
-                    best = best > k ? best : k;
-                }
-            best = warp_max_u64(best);
-            out = (int)(0xffffffffu - (unsigned)(best & 0xffffffffull));
-            if (lane == 0) taken[out] = 1;
-            __syncwarp();
+    int32_t* sel = p.sel + nh * p.m;
+    for (int j = mm + threadIdx.x; j < p.m; j += blockDim.x) sel[j] = -1;
+    if (p.C <= 256) {
+        // rank of each cluster = number of larger keys (keys are distinct: they carry c);
+        // the clusters of rank < m are kept, best first
+        for (int c = threadIdx.x; c < p.C; c += blockDim.x) {
+            const unsigned long long kc = s_key[c];
+            int rank = 0;
+            for (int i = 0; i < p.C; ++i) rank += s_key[i] > kc;
+            if (rank < mm) sel[rank] = c;
         }
-        if (lane == 0) p.sel[nh * p.m + j] = out;
+        return;
+    }
+    if (warp != 0) return;
+    for (int j = 0; j < mm; ++j) {   // many clusters: m rounds of a warp argmax
+        unsigned long long best = 0ull;
+        for (int c = lane; c < p.C; c += 32)
+            if (!taken[c]) best = best > s_key[c] ? best : s_key[c];
+        best = warp_max_u64(best);
+        const int out = (int)(0xffffffffu - (unsigned)(best & 0xffffffffull));
+        if (lane == 0) {
+            taken[out] = 1;
+            sel[j] = out;
+        }
+        __syncwarp();
     }
 }
 
@@ -164,15 +197,17 @@ __global__ void __launch_bounds__(256) asm_hier_score_kernel(const __grid_consta
                 }
                 rows[r] = (kk[r] >= 0) ? p.qbar + ((size_t)h * p.K + kk[r]) * kHierD : nullptr;
             }
-            float sc[8];
-            hier_score8(qv, rows, sc, lane);
+            const float sc = hier_score8(qv, rows, lane);
+            // lane 2r holds row r: select its entry id without indexing the array dynamically
+            int kl = -1;
 #pragma unroll
-            for (int r = 0; r < 8; ++r)
-                if (kk[r] >= 0) {
-                    const unsigned long long key = hier_key(sc[r], kk[r]);
-                    best = best > key ? best : key;
-                }
+            for (int r = 0; r < 8; ++r) kl = (lane == 2 * r) ? kk[r] : kl;
+            if (kl >= 0) {
+                const unsigned long long key = hier_key(sc, kl);
+                best = best > key ? best : key;
+            }
         }
+        best = warp_max_u64(best);
     }
     if (lane == 0) s_best[warp] = best;
     __syncthreads();
