@@ -4,8 +4,11 @@ A decode step for the token at position t (per sequence) follows "Cache What
 Lasts" section 2.1 at inference time: if the cache already holds M tokens the
 token with the lowest beta_i^(t-i) is evicted and the new token takes its
 slot (kvb_evict_insert); then the token attends over the <= M cached tokens,
-itself included, with the retention-gated logits (kvb_decode_attn, split-K
-with the splits merged in the same launch).
+itself included, with the retention-gated logits (kvb_decode_attn, split-K;
+with several splits the same call launches the merge of the split states).
+The attention also leaves, per split, the slot that the next position's
+eviction would pick, so that the next insert reads candidates instead of
+rescanning the cache.
 """
 from __future__ import annotations
 
