@@ -40,6 +40,7 @@ sys.path.insert(0, ROOT)
 METRIC = "decode-attn tokens/s and KV-cache GB/s (% of B200 HBM peak) at budget M"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+L2_BYTES = 126 * 1000 * 1000      # B200 L2 (126 MB)
 
 # ncu DRAM traffic (read + write bytes per launch) of the dominant kernel, keyed by
 # (sha256 of the kernel's source file, config, num_splits). Reported only while the source is
@@ -291,11 +292,16 @@ class DecodeBench:
         return (f"kvb_decode_attn = decode_attn_tc_kernel<d={self.w.d},G={self.w.Hq // self.w.Hkv},bias=1>"
                 f"{merge}, S={self.S}")
 
+    def flush_l2(self):
+        return self.attn_bytes() < L2_BYTES
+
     def config(self):
         w = self.w
+        l2 = (f"flushed before every timed step (256 MiB write): a step reads {self.attn_bytes() / 1e6:.2f} MB"
+              if self.flush_l2() else
+              f"no flush: every step reads {self.attn_bytes() / 1e6:.0f} MB of K/V (inputs larger than L2)")
         return {"workload": self.workload, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "budget_M": w.M,
-                "num_splits": self.S, "beta": "sigmoid(N(2,1.5))",
-                "l2": "no flush: every step reads > 126 MB of K/V (inputs larger than L2)",
+                "num_splits": self.S, "beta": "sigmoid(N(2,1.5))", "l2": l2,
                 "parallelism": "replicas (independent sequences per GPU)"}
 
     def oracle_sample(self, budget_s: float = 15.0):
@@ -333,6 +339,9 @@ class ASMBench:
     (kvb_decode_attn, batch stride 0) and the memory lookup + merge (kvb_asm_lookup_merge)."""
 
     KERNEL_SRC = "asm_lookup.cuh"
+
+    def flush_l2(self):
+        return True
 
     # the fp32 contraction runs as three exact bf16 products per element (q . hi + q . mid + q . lo)
     PEAK_NOTE = "{kind} dense bf16 {bf16:.0f} TFLOP/s (bf16_tflops, burst) / 3 bf16 products per fp32 product"
@@ -410,7 +419,8 @@ class ASMBench:
     def config(self):
         w = self.w
         return {"workload": self.workload, "N": w.N, "H": w.H, "Hkv": w.Hkv, "K": w.K, "d": w.d, "L": w.L,
-                "self_attn_splits": self.S, "l2": "qbar (64 MiB) + abar (32 MiB) per step; no flush",
+                "self_attn_splits": self.S,
+                "l2": "flushed before every timed step (256 MiB write): q̄ 64 MiB + ā 32 MiB + K/V 8 MiB fit in L2",
                 "parallelism": "replicas"}
 
 
@@ -446,6 +456,9 @@ class MementoBench:
         self.tokens_per_step = None
         self.launches_per_step = None
         self.workload = "memento compaction B64 Hq32 Hkv8 d128, 9 x (Geom(1500) block + U[120,180] memento) (config 5)"
+
+    def flush_l2(self):
+        return True
 
     def clamp_steps(self, K, W, KR):
         n = self.w.steps
@@ -491,12 +504,32 @@ class MementoBench:
     def config(self):
         w = self.w
         return {"workload": self.workload, "B": w.B, "cap": w.cap, "split_len": self.SPLIT_LEN,
-                "num_splits": self.S, "schedule_steps": w.steps, "parallelism": "replicas"}
+                "num_splits": self.S, "schedule_steps": w.steps, "parallelism": "replicas",
+                "l2": "flushed before every timed step (256 MiB write): the live caches grow from "
+                      "a few MB to ~350 MB over the timed steps"}
 
 
 # ----------------------------------------------------------------------------------------------
 # timing driver
 # ----------------------------------------------------------------------------------------------
+
+def time_flushed_steps(steps, flush, world):
+    """Device time of the steps, each started with a cold L2 (flush written before it, outside
+    its events): the sum of the per-step event times, after a barrier on both sides."""
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in steps]
+    for (a, b), step in zip(ev, steps):
+        flush.fill_(1)
+        a.record()
+        step()
+        b.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    return sum(a.elapsed_time(b) for a, b in ev)
+
 
 def time_region(fn, world):
     barrier(world)
@@ -530,20 +563,45 @@ def run_kvb(args, world, rank, local):
     # inside); then a region of KR steps with CUDA events around the dominant launch
     bench.run_device(0, W)
     torch.cuda.synchronize()
-    graph = None
+    # a workload whose step touches less than L2 holds is timed step by step with a cold L2:
+    # each step is its own CUDA graph, replayed after a 256 MiB write, with events around the
+    # replay only (the flush is not timed); otherwise the K steps are one graph
+    flush_l2 = bench.flush_l2() if hasattr(bench, "flush_l2") else False
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if flush_l2 else None
+    graph, step_graphs = None, None
     if not args.no_graph:
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            bench.run_device(W, K)
+        if flush_l2:
+            step_graphs = []
+            for i in range(K):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    bench.run_device(W + i, 1)
+                step_graphs.append(g)
+        else:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                bench.run_device(W, K)
     clocks = ClockSampler(local)
     clocks.start()
-    if graph is not None:
+    if step_graphs is not None:
+        ms = time_flushed_steps([g.replay for g in step_graphs], flush, world)
+    elif flush_l2:
+        ms = time_flushed_steps([lambda i=i: bench.run_device(W + i, 1) for i in range(K)], flush, world)
+    elif graph is not None:
         ms = time_region(graph.replay, world)
     else:
         ms = time_region(lambda: bench.run_device(W, K), world)
     events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(KR)]
-    time_region(lambda: bench.run_device(W + K, KR, events), world)
+    if flush_l2:
+        def kernel_region():
+            for j in range(KR):
+                flush.fill_(1)
+                bench.run_device(W + K + j, 1, events[j:j + 1])
+        time_region(kernel_region, world)
+    else:
+        time_region(lambda: bench.run_device(W + K, KR, events), world)
     clk = clocks.stop()
+    del step_graphs
     kern_ms = [a.elapsed_time(b) for a, b in events]
     ms = max_over_ranks(ms, world)
     kms = max_over_ranks(statistics.mean(kern_ms), world)
