@@ -17,6 +17,11 @@ Parity status (what pins each function, see tests/test_oracle_*.py):
                    compaction == masked SDPA over the old cache
   asm_lookup_merge pinned: sklearn cosine_similarity argmax, exact-match
                    retrieval, merged state == SDPA over prefix + self
+  asm_build.asm_aggregate, asm_build.asm_kmeans (numpy, float64)
+                   pinned: single members, the two-state Z-domain formula, the
+                   pinned n-way merge, chunked prefix build == SDPA over the
+                   whole prefix, closed-form means, separated groups recovered
+                   by the clustering, objective never decreasing
   asm_hier_lookup_merge
                    pinned: m = C over a partition == sklearn cosine_similarity
                    argmax; constructed indexes with known answers (best
