@@ -282,6 +282,9 @@ kvb_status kvb_compact_blocks(uint16_t* k, uint16_t* v, int32_t* pos, float* log
  * Requirements: d == 128; N, H, K >= 1; all pointers 16-byte aligned.
  * A (query, head) whose every cosine is NaN retrieves nothing: idx = -1 and
  * (o, lse) = (o_self, lse_self).
+ * o == NULL: only idx is computed (it must then be non-NULL; abar, log_zbar,
+ * o_self, lse_self and lse may be NULL) -- the assignment step of clustering
+ * the calibration queries under the cosine.
  * ---------------------------------------------------------------------- */
 size_t kvb_asm_workspace_bytes(int32_t N, int32_t H, int32_t K);
 
@@ -329,6 +332,36 @@ kvb_status kvb_asm_hier_lookup_merge(const uint16_t* q, const float* qhat, const
                                      int32_t N, int32_t H, int32_t K, int32_t C, int32_t m, int32_t d,
                                      int32_t* idx, float* o, float* lse,
                                      void* workspace, size_t workspace_bytes, kvb_stream stream);
+
+/* ------------------------------------------------------------------------
+ * kvb_asm_aggregate -- attention-aware aggregation (offline memory build)
+ *
+ * [ASM] core method step 2. For head h and cluster k, over the calibration
+ * queries i with idx[i, h] == k (idx < 0: the query is in no cluster):
+ *   qbar[h, k]     = mean of q[i, h]
+ *   abar[h, k]     = sum Z_i a[i, h] / sum Z_i, with Z_i = exp(lse[i, h])
+ *   log_zbar[h, k] = ln sum Z_i (the page's merge operator sums Z); with
+ *                    z_mean != 0, ln of the mean of the Z_i
+ *   count[h, k]    = number of members
+ * An empty cluster gets qbar = 0, abar = 0, log_zbar = -inf, count = 0.
+ * Layouts (contiguous): q [M, H, d] bf16; a [M, H, d] f32; lse [M, H] f32;
+ * idx [M, H] int32 -> qbar [H, K, d] f32; abar [H, K, d] bf16 (round to
+ * nearest even), the format kvb_asm_lookup_merge reads; log_zbar [H, K] f32;
+ * count [H, K] int32 (may be NULL). a and lse NULL together: only qbar and
+ * count are computed (abar, log_zbar may then be NULL) -- the centroid update
+ * of the clustering.
+ * workspace: device memory of kvb_asm_aggregate_workspace_bytes(H, K) bytes,
+ * 16-byte aligned, contents irrelevant on entry. The sums are fp32 atomics:
+ * their rounding order varies between runs.
+ * Requirements: d == 128; M, H, K >= 1; q, a, qbar, abar, workspace 16-byte
+ * aligned. idx >= K found on the device is skipped and sets KVB_DERR_RANGE.
+ * ---------------------------------------------------------------------- */
+size_t kvb_asm_aggregate_workspace_bytes(int32_t H, int32_t K);
+
+kvb_status kvb_asm_aggregate(const uint16_t* q, const float* a, const float* lse, const int32_t* idx,
+                             int32_t M, int32_t H, int32_t K, int32_t d, int32_t z_mean,
+                             float* qbar, uint16_t* abar, float* log_zbar, int32_t* count,
+                             void* workspace, size_t workspace_bytes, kvb_stream stream);
 
 /* ------------------------------------------------------------------------
  * Errors and diagnostics

@@ -20,7 +20,8 @@ from . import _lib
 __all__ = [
     "KvbError", "kvb_decode_attn", "kvb_decode_attn_noalloc", "kvb_merge_states", "kvb_evict_insert", "kvb_compact_blocks",
     "kvb_asm_workspace_bytes", "kvb_asm_lookup_merge", "kvb_asm_hier_workspace_bytes",
-    "kvb_asm_hier_lookup_merge", "kvb_get_error", "kvb_abi_version",
+    "kvb_asm_hier_lookup_merge", "kvb_asm_aggregate_workspace_bytes", "kvb_asm_aggregate",
+    "kvb_get_error", "kvb_abi_version",
     "decode_workspace", "evict_candidates",
 ]
 
@@ -274,13 +275,19 @@ def kvb_asm_workspace_bytes(N: int, H: int, K: int) -> int:
 def kvb_asm_lookup_merge(q, qbar, abar, log_zbar, o_self, lse_self, idx, o, lse, workspace, *,
                          stream=None) -> None:
     """Attention-state-memory lookup and merge; see kvb_asm_lookup_merge in include/kvb.h.
-    workspace: a uint8 CUDA tensor of at least kvb_asm_workspace_bytes(N, H, K) bytes."""
-    _need(q, torch.bfloat16, "q"); _need(qbar, torch.float32, "qbar"); _need(abar, torch.bfloat16, "abar")
-    _need(log_zbar, torch.float32, "log_zbar"); _need(o_self, torch.float32, "o_self")
-    _need(lse_self, torch.float32, "lse_self"); _need(o, torch.float32, "o")
+    workspace: a uint8 CUDA tensor of at least kvb_asm_workspace_bytes(N, H, K) bytes.
+    o=None: only idx is computed (abar, log_zbar, o_self, lse_self, lse may be None)."""
+    _need(q, torch.bfloat16, "q"); _need(qbar, torch.float32, "qbar")
+    if o is not None:
+        _need(abar, torch.bfloat16, "abar"); _need(log_zbar, torch.float32, "log_zbar")
+        _need(o_self, torch.float32, "o_self"); _need(lse_self, torch.float32, "lse_self")
+        _need(o, torch.float32, "o")
+    elif idx is None:
+        raise KvbError("kvb_asm_lookup_merge: o=None (assignment only) needs idx")
     for name, x in (("q", q), ("qbar", qbar), ("abar", abar), ("log_zbar", log_zbar), ("o_self", o_self),
                     ("lse_self", lse_self), ("o", o), ("workspace", workspace)):
-        _contig(x, name)
+        if x is not None:
+            _contig(x, name)
     if idx is not None:
         _need(idx, torch.int32, "idx"); _contig(idx, "idx")
     if lse is not None:
@@ -291,6 +298,35 @@ def kvb_asm_lookup_merge(q, qbar, abar, log_zbar, o_self, lse_self, idx, o, lse,
     _check(_lib.lib().kvb_asm_lookup_merge(_ptr(q), _ptr(qbar), _ptr(abar), _ptr(log_zbar), _ptr(o_self),
                                            _ptr(lse_self), N, H, K, d, _ptr(idx), _ptr(o), _ptr(lse),
                                            _ptr(workspace), nbytes, _stream(stream)), "kvb_asm_lookup_merge")
+
+
+def kvb_asm_aggregate_workspace_bytes(H: int, K: int) -> int:
+    return int(_lib.lib().kvb_asm_aggregate_workspace_bytes(H, K))
+
+
+def kvb_asm_aggregate(q, a, lse, idx, qbar, abar, log_zbar, count, workspace, *, z_mean: bool = False,
+                      stream=None) -> None:
+    """Attention-aware aggregation (offline memory build); see kvb_asm_aggregate in include/kvb.h.
+    a, lse None: only qbar (and count) are computed. workspace: a uint8 CUDA tensor of at least
+    kvb_asm_aggregate_workspace_bytes(H, K) bytes."""
+    _need(q, torch.bfloat16, "q"); _need(idx, torch.int32, "idx"); _need(qbar, torch.float32, "qbar")
+    if (a is None) != (lse is None):
+        raise KvbError("kvb_asm_aggregate: a and lse go together")
+    if a is not None:
+        _need(a, torch.float32, "a"); _need(lse, torch.float32, "lse")
+        _need(abar, torch.bfloat16, "abar"); _need(log_zbar, torch.float32, "log_zbar")
+    if count is not None:
+        _need(count, torch.int32, "count")
+    for name, x in (("q", q), ("a", a), ("lse", lse), ("idx", idx), ("qbar", qbar), ("abar", abar),
+                    ("log_zbar", log_zbar), ("count", count), ("workspace", workspace)):
+        if x is not None:
+            _contig(x, name)
+    M, H, d = q.shape
+    K = qbar.shape[1]
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(_lib.lib().kvb_asm_aggregate(_ptr(q), _ptr(a), _ptr(lse), _ptr(idx), M, H, K, d, int(bool(z_mean)),
+                                        _ptr(qbar), _ptr(abar), _ptr(log_zbar), _ptr(count), _ptr(workspace),
+                                        nbytes, _stream(stream)), "kvb_asm_aggregate")
 
 
 def kvb_asm_hier_workspace_bytes(N: int, H: int, m: int) -> int:

@@ -399,6 +399,10 @@ __global__ void __launch_bounds__(256) asm_merge_kernel(const __grid_constant__ 
         const unsigned long long o = __shfl_xor_sync(kFull, best, m);
         best = best > o ? best : o;
     }
+    if (p.o == nullptr) {   // assignment only
+        if (lane == 0) p.idx[nh] = (best == 0ull) ? -1 : (int)(0xffffffffu - (unsigned)(best & 0xffffffffull));
+        return;
+    }
     if (best == 0ull) {   // nothing retrieved (no candidate, or every score NaN): the self state
         if (lane == 0 && p.idx != nullptr) p.idx[nh] = -1;
         if (lane == 0 && p.lse != nullptr) p.lse[nh] = p.lse_self[nh];

@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstdint>
 #include <map>
+#include <algorithm>
 #include <mutex>
 #include <tuple>
 #include <utility>
@@ -11,6 +12,7 @@
 #include "../../include/kvb.h"
 #include "asm_lookup.cuh"
 #include "asm_hier.cuh"
+#include "asm_build.cuh"
 #include "common.cuh"
 #include "compact_blocks.cuh"
 #include "decode_attn_tc.cuh"
@@ -193,7 +195,7 @@ inline size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
 extern "C" {
 
-int32_t kvb_abi_version(void) { return 3; }
+int32_t kvb_abi_version(void) { return 4; }
 
 const char* kvb_status_str(kvb_status s) {
     switch (s) {
@@ -348,10 +350,14 @@ kvb_status kvb_asm_lookup_merge(const uint16_t* q, const float* qbar, const uint
                                 int32_t d, int32_t* idx, float* o, float* lse, void* workspace,
                                 size_t workspace_bytes, kvb_stream stream) {
     if (d != kvb::kAsmD || N < 1 || H < 1 || K < 1 || H > 65535) return KVB_EINVAL;
-    if (!q || !qbar || !abar || !log_zbar || !o_self || !lse_self || !o || !workspace) return KVB_EINVAL;
-    if (!aligned16(q) || !aligned16(qbar) || !aligned16(abar) || !aligned16(o_self) || !aligned16(o) ||
-        !aligned16(workspace))
+    if (!q || !qbar || !workspace) return KVB_EINVAL;
+    if (o == nullptr) {   // assignment only
+        if (idx == nullptr) return KVB_EINVAL;
+    } else if (!abar || !log_zbar || !o_self || !lse_self || !aligned16(abar) || !aligned16(o_self) ||
+               !aligned16(o)) {
         return KVB_EINVAL;
+    }
+    if (!aligned16(q) || !aligned16(qbar) || !aligned16(workspace)) return KVB_EINVAL;
     if (workspace_bytes < kvb_asm_workspace_bytes(N, H, K)) return KVB_EINVAL;
     const int qtiles = (N + kvb::kUMT * kvb::kUQ - 1) / (kvb::kUMT * kvb::kUQ);
     const long long items = (long long)H * qtiles * kvb::asm_ksplit(K);
@@ -410,6 +416,48 @@ kvb_status kvb_asm_hier_lookup_merge(const uint16_t* q, const float* qhat, const
     // reduction over the m selected clusters' keys + merge: the linear lookup's merge kernel
     kvb::AsmParams p{q, qbar, abar, log_zbar, o_self, lse_self, N, H, K, m, 0, 0, 0, idx, o, lse, keys};
     return launch_pdl(kvb::asm_merge_kernel, dim3((unsigned)((nh + 7) / 8)), dim3(256), 0, st, p);
+}
+
+size_t kvb_asm_aggregate_workspace_bytes(int32_t H, int32_t K) {
+    if (H < 1 || K < 1) return 0;
+    const size_t hk = (size_t)H * K;
+    return hk * (3 * sizeof(uint32_t)) + 2 * hk * kvb::kBuildD * sizeof(float);
+}
+
+kvb_status kvb_asm_aggregate(const uint16_t* q, const float* a, const float* lse, const int32_t* idx,
+                             int32_t M, int32_t H, int32_t K, int32_t d, int32_t z_mean,
+                             float* qbar, uint16_t* abar, float* log_zbar, int32_t* count,
+                             void* workspace, size_t workspace_bytes, kvb_stream stream) {
+    if (d != kvb::kBuildD || M < 1 || H < 1 || K < 1) return KVB_EINVAL;
+    if (!q || !idx || !qbar || !workspace) return KVB_EINVAL;
+    if ((a == nullptr) != (lse == nullptr)) return KVB_EINVAL;
+    if (a != nullptr && (!abar || !log_zbar || !aligned16(a) || !aligned16(abar))) return KVB_EINVAL;
+    if (!aligned16(q) || !aligned16(qbar) || !aligned16(workspace)) return KVB_EINVAL;
+    if (workspace_bytes < kvb_asm_aggregate_workspace_bytes(H, K)) return KVB_EINVAL;
+    const long long rows = (long long)M * H, hk = (long long)H * K;
+    if (rows > (1ll << 34) || hk * kvb::kBuildD > (1ll << 34)) return KVB_EINVAL;
+    // workspace: qsum [H, K, d], asum [H, K, d], wsum [H, K], cmax [H, K], cnt [H, K]
+    auto* base = static_cast<unsigned char*>(workspace);
+    float* qsum = reinterpret_cast<float*>(base);
+    float* asum = qsum + hk * kvb::kBuildD;
+    float* wsum = asum + hk * kvb::kBuildD;
+    auto* cmax = reinterpret_cast<unsigned*>(wsum + hk);
+    int* cnt = reinterpret_cast<int*>(cmax + hk);
+    kvb::AsmBuildParams p{q, a, lse, idx, M, H, K, z_mean ? 1 : 0, qbar, abar, log_zbar, count,
+                          cmax, cnt, wsum, qsum, asum};
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t words = kvb_asm_aggregate_workspace_bytes(H, K) / sizeof(unsigned);
+    kvb::asm_build_zero_kernel<<<(unsigned)std::min<size_t>((words + 255) / 256, 4096), 256, 0, st>>>(
+        static_cast<unsigned*>(workspace), words);
+    if (launched() != KVB_OK) return KVB_ECUDA;
+    kvb::asm_build_pass1_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p);
+    if (launched() != KVB_OK) return KVB_ECUDA;
+    if (a != nullptr) {
+        kvb::asm_build_pass2_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p);
+        if (launched() != KVB_OK) return KVB_ECUDA;
+    }
+    kvb::asm_build_final_kernel<<<(unsigned)((hk + 7) / 8), 256, 0, st>>>(p);
+    return launched();
 }
 
 }  // extern "C"

@@ -47,7 +47,7 @@ def test_attn_args_struct_matches_header():
 
 def test_status_strings_and_version():
     L = _lib.lib()
-    assert L.kvb_abi_version() == 3
+    assert L.kvb_abi_version() == 4
     assert L.kvb_status_str(0) == b"ok"
     assert L.kvb_status_str(1) == b"invalid argument"
 
@@ -96,6 +96,15 @@ def test_other_entry_points_reject_bad_arguments_on_the_host():
                                        3 * 2 * 16 * 12 - 1, None) == _lib.KVB_EINVAL
     assert L.kvb_asm_hier_lookup_merge(f, f, f, ctypes.c_void_p((1 << 20) + 2), f, f, f, f, f, 1, 2, 64, 8, 4, 128,
                                        None, f, None, f, 1 << 20, None) == _lib.KVB_EINVAL
+    # aggregation: a without lse, d != 128, short workspace; assignment-only lookup without idx
+    assert L.kvb_asm_aggregate(f, f, None, f, 10, 2, 8, 128, 0, f, f, f, None, f, 1 << 24, None) == _lib.KVB_EINVAL
+    assert L.kvb_asm_aggregate(f, None, None, f, 10, 2, 8, 64, 0, f, None, None, None, f, 1 << 24,
+                               None) == _lib.KVB_EINVAL
+    assert L.kvb_asm_aggregate_workspace_bytes(2, 8) == 2 * 8 * 12 + 2 * 2 * 8 * 128 * 4
+    assert L.kvb_asm_aggregate(f, None, None, f, 10, 2, 8, 128, 0, f, None, None, None, f,
+                               2 * 8 * 12 + 2 * 2 * 8 * 128 * 4 - 1, None) == _lib.KVB_EINVAL
+    assert L.kvb_asm_lookup_merge(f, f, None, None, None, None, 4, 2, 16, 128, None, None, None, f, 1 << 20,
+                                  None) == _lib.KVB_EINVAL
     ws = L.kvb_asm_workspace_bytes(256, 32, 4096)
     assert ws == 32 * 256 * 32 * 8   # 32 ranges of 128 centroids, one 8-byte key per (range, query, head)
     assert L.kvb_asm_lookup_merge(f, f, f, f, f, f, 256, 32, 4096, 128, None, f, None, f, ws - 1, None) == _lib.KVB_EINVAL

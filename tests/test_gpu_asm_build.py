@@ -1,0 +1,136 @@
+"""GPU parity of the attention-state-memory offline build against the oracle:
+kvb_asm_aggregate (ragged and empty clusters, unassigned queries, members with
+Z = 0, sum and mean Z, queries only), the range error, the cosine Lloyd
+clustering on separated groups, and the whole build (clusters + aggregation)."""
+import numpy as np
+import pytest
+import torch
+
+import memory_bounded_kv_b200 as kvb
+from memory_bounded_kv_b200 import asm_build
+from memory_bounded_kv_b200.synth import normal_bf16, rng, to_bf16_bits
+import oracle.asm_build as ob
+from gpu_util import dev, host, assert_state_close, bf16_round
+
+pytestmark = pytest.mark.gpu
+
+
+def run_aggregate(q, a, lse, idx, K, z_mean=False):
+    M, H, d = q.shape
+    qbar = torch.full((H, K, d), 7.0, device="cuda")
+    abar = torch.zeros(H, K, d, dtype=torch.bfloat16, device="cuda")
+    lz = torch.zeros(H, K, device="cuda")
+    cnt = torch.full((H, K), -5, dtype=torch.int32, device="cuda")
+    ws = torch.empty(kvb.kvb_asm_aggregate_workspace_bytes(H, K), dtype=torch.uint8, device="cuda")
+    with_states = a is not None
+    kvb.kvb_asm_aggregate(dev(q), dev(a) if with_states else None, dev(lse) if with_states else None, dev(idx),
+                          qbar, abar if with_states else None, lz if with_states else None, cnt, ws,
+                          z_mean=z_mean)
+    torch.cuda.synchronize()
+    return host(qbar), host(abar.float()), host(lz), host(cnt)
+
+
+def check_aggregate(got, want, with_states=True):
+    qbar, abar, lz, cnt = got
+    q_r, a_r, l_r, c_r = want
+    np.testing.assert_array_equal(cnt, c_r)
+    np.testing.assert_allclose(qbar, q_r, rtol=1e-5, atol=1e-6)
+    if with_states:
+        H, K, d = a_r.shape
+        assert_state_close(abar.reshape(H * K, d), lz.reshape(-1), bf16_round(a_r).reshape(H * K, d),
+                           l_r.reshape(-1), "aggregated state")
+
+
+def _inputs(seed, M, H, K, d=128):
+    g = rng(seed, 31)
+    q = normal_bf16(g, (M, H, d))
+    a = g.standard_normal((M, H, d)).astype(np.float32)
+    lse = g.uniform(-4, 9, (M, H)).astype(np.float32)
+    lse[g.random((M, H)) < 0.03] = -np.inf                  # members with an empty prefix
+    idx = g.integers(-1, K, (M, H)).astype(np.int32)          # -1: in no cluster
+    idx[:, 0] = np.where(idx[:, 0] == 3, 4, idx[:, 0])        # cluster 3 of head 0 stays empty
+    return q, a, lse, idx
+
+
+@pytest.mark.parametrize("M,H,K", [(500, 3, 37), (64, 1, 1), (2000, 2, 300)])
+@pytest.mark.parametrize("z_mean", [False, True])
+def test_aggregate_matches_oracle(M, H, K, z_mean):
+    q, a, lse, idx = _inputs(M + K, M, H, K)
+    got = run_aggregate(q, a, lse, idx, K, z_mean)
+    want = ob.asm_aggregate(q, a, lse, idx, K, z_mean)
+    check_aggregate(got, want)
+
+
+def test_cluster_of_empty_prefixes_is_the_merge_identity():
+    q, a, lse, idx = _inputs(5, 40, 1, 4)
+    idx[:, 0] = np.arange(40) % 4
+    lse[idx[:, 0] == 2, 0] = -np.inf
+    got = run_aggregate(q, a, lse, idx, 4)
+    assert got[2][0, 2] == -np.inf and not got[1][0, 2].any() and got[3][0, 2] == 10
+    check_aggregate(got, ob.asm_aggregate(q, a, lse, idx, 4))
+
+
+def test_queries_only():
+    q, a, lse, idx = _inputs(6, 300, 2, 11)
+    got = run_aggregate(q, None, None, idx, 11)
+    want = ob.asm_aggregate(q, None, None, idx, 11)
+    check_aggregate(got, want, with_states=False)
+
+
+def test_cluster_out_of_range_sets_the_range_error():
+    q, a, lse, idx = _inputs(7, 50, 1, 5)
+    idx[3, 0] = 5
+    kvb.kvb_get_error()
+    got = run_aggregate(q, a, lse, idx, 5)
+    assert kvb.kvb_get_error() & 4
+    idx_ok = idx.copy()
+    idx_ok[3, 0] = -1
+    check_aggregate(got, ob.asm_aggregate(q, a, lse, idx_ok, 5))
+
+
+def _separated(seed, M, H, K, d=128, spread=0.05):
+    g = rng(seed, 32)
+    u = g.standard_normal((H, K, d))
+    u /= np.linalg.norm(u, axis=-1, keepdims=True)
+    owner = np.stack([g.permutation(np.arange(M) % K) for _ in range(H)], axis=1)
+    x = u[np.arange(H)[None, :], owner] + spread * g.standard_normal((M, H, d))
+    init = np.stack([np.array([np.nonzero(owner[:, h] == k)[0][0] for k in range(K)]) for h in range(H)])
+    return to_bf16_bits(x.astype(np.float32)), owner.astype(np.int32), init
+
+
+def test_kmeans_matches_oracle_on_separated_groups():
+    q, owner, init = _separated(8, 384, 2, 12)
+    idx, cent = asm_build.asm_kmeans(dev(q), init, iters=3)
+    idx_r, cent_r = ob.asm_kmeans(q, init, iters=3)
+    np.testing.assert_array_equal(idx_r, owner)
+    np.testing.assert_array_equal(host(idx), idx_r)
+    np.testing.assert_allclose(host(cent), cent_r, rtol=1e-5, atol=1e-6)
+
+
+def test_kmeans_from_overlapping_starts_matches_oracle():
+    """Wider groups and two starting centroids in one group: the clusters move over the
+    iterations; every assignment on the way must match the oracle's (margins checked)."""
+    q, owner, init = _separated(9, 256, 1, 8, spread=0.3)
+    init[0, 1] = np.nonzero(owner[:, 0] == 0)[0][1]
+    idx, cent = asm_build.asm_kmeans(dev(q), init, iters=4)
+    idx_r, cent_r = ob.asm_kmeans(q, init, iters=4)
+    # the oracle's decisions must not sit on a near tie for the comparison to be exact
+    qf = (q.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    cn = cent_r / np.maximum(np.linalg.norm(cent_r, axis=-1, keepdims=True), 1e-300)
+    cos = np.einsum("md,kd->mk", qf[:, 0] / np.linalg.norm(qf[:, 0], axis=1, keepdims=True), cn[0])
+    top = np.sort(cos, axis=1)
+    assert (top[:, -1] - top[:, -2]).min() > 1e-4
+    np.testing.assert_array_equal(host(idx), idx_r)
+    np.testing.assert_allclose(host(cent), cent_r, rtol=1e-5, atol=1e-6)
+
+
+def test_build_matches_oracle():
+    q, owner, init = _separated(10, 320, 2, 10)
+    g = rng(10, 33)
+    a = g.standard_normal(q.shape).astype(np.float32)
+    lse = g.uniform(0, 8, q.shape[:2]).astype(np.float32)
+    qbar, abar, lz, cnt, idx = asm_build.asm_build(dev(q), dev(a), dev(lse), init, iters=2)
+    idx_r, _ = ob.asm_kmeans(q, init, iters=2)
+    np.testing.assert_array_equal(host(idx), idx_r)
+    want = ob.asm_aggregate(q, a, lse, idx_r, 10)
+    check_aggregate((host(qbar), host(abar.float()), host(lz), host(cnt)), want)
