@@ -62,6 +62,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the timed steps one by one")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--asm-build", action="store_true",
+                    help="time the offline memory build (cosine Lloyd iteration, aggregation) instead of a "
+                         "decode step")
     ap.add_argument("--asm-crossover", action="store_true",
                     help="time the linear and the two-level memory lookups alone over query counts and memory "
                          "sizes (one GPU; L2 flushed between iterations) instead of a decode step")
@@ -706,6 +709,74 @@ def run_reference(args, world, rank):
     }
 
 
+def run_asm_build(args) -> dict:
+    """The offline memory build at 16384 calibration queries per head (4 per entry), 32 heads,
+    K = 4096 entries, d = 128: one Lloyd iteration (mean update by kvb_asm_aggregate, cosine
+    assignment by kvb_asm_lookup_merge without merge) and the final aggregation of the states
+    (q 134 MB bf16, a 268 MB f32 in). Each replayed from a CUDA graph after an L2 flush."""
+    import memory_bounded_kv_b200 as kvb
+    from memory_bounded_kv_b200 import asm_build
+    from memory_bounded_kv_b200.synth import normal_bf16, rng
+    hbm_peak, peak_kind = peaks()
+    bf16_tf, bf16_kind = bf16_peak()
+    M, H, K, d = 16384, 32, 4096, 128
+    g = rng(44, 0)
+    q = _dev(normal_bf16(g, (M, H, d)))
+    a = torch.randn(M, H, d, device="cuda")
+    lse = torch.rand(M, H, device="cuda") * 8
+    init = np.tile(np.arange(K), (H, 1))
+    idx, cent = asm_build.asm_kmeans(q, init, iters=1)
+    ws_agg = torch.empty(kvb.kvb_asm_aggregate_workspace_bytes(H, K), dtype=torch.uint8, device="cuda")
+    ws_lk = torch.empty(kvb.kvb_asm_workspace_bytes(M, H, K), dtype=torch.uint8, device="cuda")
+    qbar = torch.empty(H, K, d, device="cuda")
+    abar = torch.empty(H, K, d, dtype=torch.bfloat16, device="cuda")
+    lz = torch.empty(H, K, device="cuda")
+    cnt = torch.empty(H, K, dtype=torch.int32, device="cuda")
+
+    def update():
+        kvb.kvb_asm_aggregate(q, None, None, idx, cent, None, None, None, ws_agg)
+
+    def assign():
+        kvb.kvb_asm_lookup_merge(q, cent, None, None, None, None, idx, None, None, ws_lk)
+
+    def aggregate():
+        kvb.kvb_asm_aggregate(q, a, lse, idx, qbar, abar, lz, cnt, ws_agg)
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    iters = max(3, min(args.steps, 20))
+    out = {}
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    for name, fn in (("update", update), ("assign", assign), ("aggregate", aggregate)):
+        for _ in range(max(2, args.warmup)):
+            fn()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            fn()
+        out[name] = time_flushed_steps([graph.replay] * iters, flush, 1) / iters
+        del graph
+    clk = clocks.stop()
+    flops = 2.0 * M * H * K * d
+    agg_bytes = M * H * (d * 2 + d * 4 + 4 + 4) + H * K * (d * 4 + d * 2 + 4 + 4)
+    return {"metric": "ASM offline build: Lloyd iteration and aggregation time", "unit": "ms",
+            "higher_is_better": False, "n_gpus": 1, "steps": iters, "warmup": max(2, args.warmup),
+            "dtype": "f32 (bf16 x 3 products)", "data": "synthetic (random queries and states)",
+            "config": {"workload": f"{M} calibration queries x {H} heads -> {K} entries, d {d}",
+                       "l2": "flushed before every timed call (256 MiB write)"},
+            "lloyd_iteration_ms": out["update"] + out["assign"], "update_ms": out["update"],
+            "assign_ms": out["assign"], "aggregate_ms": out["aggregate"],
+            "assign_roofline": {"bound": "tensor", "achieved": flops / (out["assign"] / 1e3) / 1e12,
+                                "peak": bf16_tf / 3.0, "unit": "TFLOP/s",
+                                "frac": flops / (out["assign"] / 1e3) / 1e12 / (bf16_tf / 3.0),
+                                "peak_source": f"{bf16_kind} bf16_tflops / 3"},
+            "aggregate_roofline": {"bound": "hbm", "achieved": agg_bytes / (out["aggregate"] / 1e3) / 1e9,
+                                   "peak": hbm_peak, "unit": "GB/s",
+                                   "frac": agg_bytes / (out["aggregate"] / 1e3) / 1e9 / hbm_peak,
+                                   "algorithmic_bytes": agg_bytes, "peak_source": f"{peak_kind} (hbm_gbs)"},
+            "clocks": clk}
+
+
 def run_asm_crossover(args) -> dict:
     """Lookup + merge alone, linear (kvb_asm_lookup_merge) against two-level
     (kvb_asm_hier_lookup_merge, C = sqrt(K) clusters, top-16), on the clustered memory
@@ -816,6 +887,9 @@ def main():
         return
     if args.asm_crossover:
         print(json.dumps(run_asm_crossover(args)), flush=True)
+        return
+    if args.asm_build:
+        print(json.dumps(run_asm_build(args)), flush=True)
         return
     world, rank, local = dist_init()
     try:
