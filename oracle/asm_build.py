@@ -85,3 +85,26 @@ def asm_kmeans(q, init_rows, iters: int):
         cent, _, _, _ = asm_aggregate(q, None, None, idx, K)
         idx = cosine_assign(q, cent)
     return idx, cent
+
+
+def asm_index(qbar, init_rows, iters: int):
+    """Two-level index of a memory ([ASM] hierarchical lookup; the index is built the way the
+    memory is, by clustering): the entries qbar [H, K, d] (fp32), rounded to bf16, are clustered
+    into C = init_rows.shape[1] groups per head by asm_kmeans (starting from the entries
+    init_rows[h]); the first-level centroids are the groups' means; each group lists its
+    entries in increasing order. Returns (qhat [H, C, d], offsets [H, C + 1], members [H, K],
+    idx [K, H])."""
+    qb = np.asarray(qbar, np.float32)
+    H, K, d = qb.shape
+    bits = qb.view(np.uint32)
+    rounded = ((bits + (((bits >> 16) & 1) + 0x7FFF)) >> 16).astype(np.uint16)   # nearest, ties even
+    q = np.ascontiguousarray(rounded.transpose(1, 0, 2))                           # [K, H, d]
+    idx, cent = asm_kmeans(q, init_rows, iters)
+    C = np.asarray(init_rows).shape[1]
+    offsets = np.zeros((H, C + 1), np.int32)
+    members = np.zeros((H, K), np.int32)
+    for h in range(H):
+        order = [np.nonzero(idx[:, h] == c)[0] for c in range(C)]
+        offsets[h, 1:] = np.cumsum([len(o) for o in order])
+        members[h] = np.concatenate(order).astype(np.int32)
+    return cent, offsets, members, idx

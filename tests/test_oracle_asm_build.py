@@ -148,3 +148,30 @@ def test_kmeans_from_a_poor_start_still_improves():
         cn = c / np.maximum(np.linalg.norm(c, axis=-1, keepdims=True), 1e-300)
         return (qf[:, 0] * cn[0, ix[:, 0]]).sum()
     assert objective(idx) >= objective(idx0)
+
+
+def test_index_of_a_clustered_memory_lists_each_group_once(oracle):
+    """Entries scattered around C directions: the index recovers the groups (entries listed in
+    increasing order), and the two-level lookup with every cluster kept equals the linear one."""
+    g = rng(21, 8)
+    H, C, per, d = 2, 5, 12, 32
+    K = C * per
+    u = g.standard_normal((H, C, d))
+    u /= np.linalg.norm(u, axis=-1, keepdims=True)
+    owner = np.stack([g.permutation(np.arange(K) % C) for _ in range(H)])          # [H, K]
+    qbar = (u[np.arange(H)[:, None], owner] + 0.05 * g.standard_normal((H, K, d))).astype(np.float32)
+    init = np.stack([np.array([np.nonzero(owner[h] == c)[0][0] for c in range(C)]) for h in range(H)])
+    qhat, offsets, members, idx = ob.asm_index(qbar, init, iters=2)
+    for h in range(H):
+        np.testing.assert_array_equal(idx[:, h], owner[h])
+        for c in range(C):
+            np.testing.assert_array_equal(members[h, offsets[h, c]:offsets[h, c + 1]], np.nonzero(owner[h] == c)[0])
+        assert offsets[h, -1] == K
+    q = normal_bf16(g, (4, H, d))
+    abar = normal_bf16(g, (H, K, d))
+    lz = g.uniform(1, 3, (H, K)).astype(np.float32)
+    o_self, l_self = g.standard_normal((4, H, d)).astype(np.float32), np.zeros((4, H), np.float32)
+    _, idx_h, _, _ = oracle.asm_hier_lookup_merge(q, qhat.astype(np.float32), offsets, members, qbar, abar, lz,
+                                                  o_self, l_self, C)
+    idx_l, _, _ = oracle.asm_lookup_merge(q, qbar, abar, lz, o_self, l_self)
+    np.testing.assert_array_equal(idx_h, idx_l)
