@@ -364,6 +364,30 @@ kvb_status kvb_asm_aggregate(const uint16_t* q, const float* a, const float* lse
                              void* workspace, size_t workspace_bytes, kvb_stream stream);
 
 /* ------------------------------------------------------------------------
+ * Two-level index of a memory (for kvb_asm_hier_lookup_merge)
+ *
+ * [ASM] hierarchical lookup index, built the way the memory is built: the
+ * entries are clustered (kvb_asm_lookup_merge with o = NULL assigns, the
+ * query part of kvb_asm_aggregate moves the centroids), which needs them as
+ * bf16 queries first:
+ * kvb_asm_entries_bf16: qbar [H, K, d] f32 -> q [K, H, d] bf16 (round to
+ *   nearest even). d == 128; both 16-byte aligned.
+ * kvb_asm_index_csr: from an assignment idx [K, H] int32 (entry k of head h
+ *   in cluster idx[k, h]; values outside [0, C) are listed nowhere), writes
+ *   offsets [H, C + 1] and members [H, K] int32 in the layout
+ *   kvb_asm_hier_lookup_merge reads, every cluster's entries in increasing
+ *   order (deterministic). workspace: kvb_asm_index_workspace_bytes(H, C)
+ *   bytes, 16-byte aligned. 1 <= C <= 65536.
+ * ---------------------------------------------------------------------- */
+kvb_status kvb_asm_entries_bf16(const float* qbar, int32_t H, int32_t K, int32_t d, uint16_t* q,
+                                kvb_stream stream);
+
+size_t kvb_asm_index_workspace_bytes(int32_t H, int32_t C);
+
+kvb_status kvb_asm_index_csr(const int32_t* idx, int32_t K, int32_t H, int32_t C, int32_t* offsets,
+                             int32_t* members, void* workspace, size_t workspace_bytes, kvb_stream stream);
+
+/* ------------------------------------------------------------------------
  * Errors and diagnostics
  * ---------------------------------------------------------------------- */
 

@@ -21,6 +21,7 @@ __all__ = [
     "KvbError", "kvb_decode_attn", "kvb_decode_attn_noalloc", "kvb_merge_states", "kvb_evict_insert", "kvb_compact_blocks",
     "kvb_asm_workspace_bytes", "kvb_asm_lookup_merge", "kvb_asm_hier_workspace_bytes",
     "kvb_asm_hier_lookup_merge", "kvb_asm_aggregate_workspace_bytes", "kvb_asm_aggregate",
+    "kvb_asm_entries_bf16", "kvb_asm_index_workspace_bytes", "kvb_asm_index_csr",
     "kvb_get_error", "kvb_abi_version",
     "decode_workspace", "evict_candidates",
 ]
@@ -327,6 +328,31 @@ def kvb_asm_aggregate(q, a, lse, idx, qbar, abar, log_zbar, count, workspace, *,
     _check(_lib.lib().kvb_asm_aggregate(_ptr(q), _ptr(a), _ptr(lse), _ptr(idx), M, H, K, d, int(bool(z_mean)),
                                         _ptr(qbar), _ptr(abar), _ptr(log_zbar), _ptr(count), _ptr(workspace),
                                         nbytes, _stream(stream)), "kvb_asm_aggregate")
+
+
+def kvb_asm_entries_bf16(qbar, q, *, stream=None) -> None:
+    """qbar [H, K, d] f32 -> q [K, H, d] bf16; see kvb_asm_entries_bf16 in include/kvb.h."""
+    _need(qbar, torch.float32, "qbar"); _need(q, torch.bfloat16, "q")
+    _contig(qbar, "qbar"); _contig(q, "q")
+    H, K, d = qbar.shape
+    _check(_lib.lib().kvb_asm_entries_bf16(_ptr(qbar), H, K, d, _ptr(q), _stream(stream)), "kvb_asm_entries_bf16")
+
+
+def kvb_asm_index_workspace_bytes(H: int, C: int) -> int:
+    return int(_lib.lib().kvb_asm_index_workspace_bytes(H, C))
+
+
+def kvb_asm_index_csr(idx, offsets, members, workspace, *, stream=None) -> None:
+    """Cluster lists from an assignment idx [K, H] into offsets [H, C + 1], members [H, K];
+    see kvb_asm_index_csr in include/kvb.h."""
+    for name, x in (("idx", idx), ("offsets", offsets), ("members", members)):
+        _need(x, torch.int32, name); _contig(x, name)
+    _contig(workspace, "workspace")
+    K, H = idx.shape
+    C = offsets.shape[1] - 1
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(_lib.lib().kvb_asm_index_csr(_ptr(idx), K, H, C, _ptr(offsets), _ptr(members), _ptr(workspace), nbytes,
+                                        _stream(stream)), "kvb_asm_index_csr")
 
 
 def kvb_asm_hier_workspace_bytes(N: int, H: int, m: int) -> int:

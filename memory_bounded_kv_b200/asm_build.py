@@ -17,8 +17,8 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (kvb_asm_aggregate, kvb_asm_aggregate_workspace_bytes, kvb_asm_lookup_merge,
-               kvb_asm_workspace_bytes)
+from . import (kvb_asm_aggregate, kvb_asm_aggregate_workspace_bytes, kvb_asm_entries_bf16, kvb_asm_index_csr,
+               kvb_asm_index_workspace_bytes, kvb_asm_lookup_merge, kvb_asm_workspace_bytes)
 
 
 def _initial_assignment(init_rows, M: int, device) -> torch.Tensor:
@@ -70,3 +70,22 @@ def asm_build(q: torch.Tensor, a: torch.Tensor, lse: torch.Tensor, init_rows, it
     ws = torch.empty(kvb_asm_aggregate_workspace_bytes(H, K), dtype=torch.uint8, device=dev)
     kvb_asm_aggregate(q, a, lse, idx, qbar, abar, log_zbar, count, ws, z_mean=z_mean, stream=stream)
     return qbar, abar, log_zbar, count, idx
+
+
+def asm_index(qbar: torch.Tensor, init_rows, iters: int, stream=None):
+    """Two-level index of a memory for kvb_asm_hier_lookup_merge: the entries qbar [H, K, d] f32,
+    as bf16 queries (kvb_asm_entries_bf16), are clustered into C = init_rows.shape[1] groups per
+    head (asm_kmeans, starting from the entries init_rows[h]); the groups' means are the
+    first-level centroids and kvb_asm_index_csr lists each group's entries in increasing order.
+    Returns (qhat [H, C, d] f32, offsets [H, C + 1] int32, members [H, K] int32, idx [K, H] int32)."""
+    H, K, d = qbar.shape
+    C = np.asarray(init_rows).shape[1]
+    dev = qbar.device
+    q = torch.empty(K, H, d, dtype=torch.bfloat16, device=dev)
+    kvb_asm_entries_bf16(qbar, q, stream=stream)
+    idx, qhat = asm_kmeans(q, init_rows, iters, stream)
+    offsets = torch.empty(H, C + 1, dtype=torch.int32, device=dev)
+    members = torch.empty(H, K, dtype=torch.int32, device=dev)
+    ws = torch.empty(kvb_asm_index_workspace_bytes(H, C), dtype=torch.uint8, device=dev)
+    kvb_asm_index_csr(idx, offsets, members, ws, stream=stream)
+    return qhat, offsets, members, idx

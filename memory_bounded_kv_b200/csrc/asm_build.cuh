@@ -115,4 +115,71 @@ __global__ void __launch_bounds__(256) asm_build_final_kernel(const __grid_const
     if (lane == 0) p.log_zbar[hk] = lz;
 }
 
+// ---- two-level index of a memory -----------------------------------------------------------
+// The entries are clustered like calibration queries (the lookup's cosine argmax + the mean
+// update), so they are first laid out as bf16 queries: qbar [H, K, d] f32 -> q [K, H, d] bf16
+// (round to nearest even); one thread per 4 elements.
+__global__ void __launch_bounds__(256) asm_entries_bf16_kernel(const float* __restrict__ qbar, int H, int K,
+                                                               uint16_t* __restrict__ q) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;   // (h, k, 4-element group)
+    const long long total = (long long)H * K * (kBuildD / 4);
+    if (i >= total) return;
+    const int e4 = (int)(i % (kBuildD / 4));
+    const long long hk = i / (kBuildD / 4);
+    const int h = (int)(hk / K), k = (int)(hk % K);
+    const float4 x = *reinterpret_cast<const float4*>(qbar + hk * kBuildD + e4 * 4);
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(x.x, x.y), hi = __floats2bfloat162_rn(x.z, x.w);
+    *reinterpret_cast<uint2*>(q + ((size_t)k * H + h) * kBuildD + e4 * 4) =
+        make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+}
+
+// Cluster lists from an assignment idx [K, H] (entry k of head h in cluster idx[k, h]; values
+// outside [0, C) are listed nowhere): counts, then offsets, then members in increasing entry
+// order, deterministic (warp ballots in entry order, no atomics).
+struct AsmCsrParams {
+    const int32_t* idx;   // [K, H]
+    int K, H, C;
+    int32_t* offsets;     // [H, C + 1]
+    int32_t* members;     // [H, K]
+    int32_t* counts;      // [H, C] workspace
+};
+
+// one warp per (h, c): pass 0 counts the members, pass 1 writes them from offsets[h, c] on
+template <int PASS>
+__global__ void __launch_bounds__(256) asm_csr_kernel(const __grid_constant__ AsmCsrParams p) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long hc = (long long)blockIdx.x * 8 + warp;
+    if (hc >= (long long)p.H * p.C) return;
+    const int h = (int)(hc / p.C), c = (int)(hc % p.C);
+    int pos = (PASS == 0) ? 0 : p.offsets[(size_t)h * (p.C + 1) + c];
+    for (int k0 = 0; k0 < p.K; k0 += 32) {
+        const int k = k0 + lane;
+        const bool in = k < p.K && p.idx[(size_t)k * p.H + h] == c;
+        const unsigned mask = __ballot_sync(kFull, in);
+        if (PASS == 1 && in) p.members[(size_t)h * p.K + pos + __popc(mask & ((1u << lane) - 1u))] = k;
+        pos += __popc(mask);
+    }
+    if (PASS == 0 && lane == 0) p.counts[hc] = pos;
+}
+
+// one warp per head: offsets[h, 0] = 0, offsets[h, c + 1] = offsets[h, c] + counts[h, c]
+__global__ void __launch_bounds__(32) asm_csr_scan_kernel(const __grid_constant__ AsmCsrParams p) {
+    const int h = blockIdx.x, lane = threadIdx.x;
+    const int32_t* cnt = p.counts + (size_t)h * p.C;
+    int32_t* off = p.offsets + (size_t)h * (p.C + 1);
+    if (lane == 0) off[0] = 0;
+    int carry = 0;
+    for (int c0 = 0; c0 < p.C; c0 += 32) {
+        const int c = c0 + lane;
+        int v = (c < p.C) ? cnt[c] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {   // inclusive warp scan
+            const int u = __shfl_up_sync(kFull, v, o);
+            if (lane >= o) v += u;
+        }
+        if (c < p.C) off[c + 1] = carry + v;
+        carry += __shfl_sync(kFull, v, 31);
+    }
+}
+
 }  // namespace kvb

@@ -460,4 +460,37 @@ kvb_status kvb_asm_aggregate(const uint16_t* q, const float* a, const float* lse
     return launched();
 }
 
+kvb_status kvb_asm_entries_bf16(const float* qbar, int32_t H, int32_t K, int32_t d, uint16_t* q,
+                                kvb_stream stream) {
+    if (d != kvb::kBuildD || H < 1 || K < 1 || !qbar || !q || !aligned16(qbar) || !aligned16(q)) return KVB_EINVAL;
+    const long long total = (long long)H * K * (kvb::kBuildD / 4);
+    if ((total + 255) / 256 > 0x7fffffffll) return KVB_EINVAL;
+    kvb::asm_entries_bf16_kernel<<<(unsigned)((total + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        qbar, H, K, q);
+    return launched();
+}
+
+size_t kvb_asm_index_workspace_bytes(int32_t H, int32_t C) {
+    if (H < 1 || C < 1) return 0;
+    return (size_t)H * C * sizeof(int32_t);
+}
+
+kvb_status kvb_asm_index_csr(const int32_t* idx, int32_t K, int32_t H, int32_t C, int32_t* offsets,
+                             int32_t* members, void* workspace, size_t workspace_bytes, kvb_stream stream) {
+    if (K < 1 || H < 1 || C < 1 || C > 65536 || !idx || !offsets || !members || !workspace) return KVB_EINVAL;
+    if (!aligned16(workspace) || workspace_bytes < kvb_asm_index_workspace_bytes(H, C)) return KVB_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(idx) | reinterpret_cast<uintptr_t>(offsets) |
+         reinterpret_cast<uintptr_t>(members)) & 3)
+        return KVB_EINVAL;
+    kvb::AsmCsrParams p{idx, K, H, C, offsets, members, static_cast<int32_t*>(workspace)};
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const unsigned grid = (unsigned)(((long long)H * C + 7) / 8);
+    kvb::asm_csr_kernel<0><<<grid, 256, 0, st>>>(p);
+    if (launched() != KVB_OK) return KVB_ECUDA;
+    kvb::asm_csr_scan_kernel<<<(unsigned)H, 32, 0, st>>>(p);
+    if (launched() != KVB_OK) return KVB_ECUDA;
+    kvb::asm_csr_kernel<1><<<grid, 256, 0, st>>>(p);
+    return launched();
+}
+
 }  // extern "C"

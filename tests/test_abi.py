@@ -105,6 +105,12 @@ def test_other_entry_points_reject_bad_arguments_on_the_host():
                                2 * 8 * 12 + 2 * 2 * 8 * 128 * 4 - 1, None) == _lib.KVB_EINVAL
     assert L.kvb_asm_lookup_merge(f, f, None, None, None, None, 4, 2, 16, 128, None, None, None, f, 1 << 20,
                                   None) == _lib.KVB_EINVAL
+    # index: d != 128, misaligned output, C out of range, short workspace
+    assert L.kvb_asm_entries_bf16(f, 2, 8, 64, f, None) == _lib.KVB_EINVAL
+    assert L.kvb_asm_entries_bf16(f, 2, 8, 128, ctypes.c_void_p((1 << 20) + 8), None) == _lib.KVB_EINVAL
+    assert L.kvb_asm_index_csr(f, 100, 2, 0, f, f, f, 1 << 20, None) == _lib.KVB_EINVAL
+    assert L.kvb_asm_index_workspace_bytes(2, 7) == 2 * 7 * 4
+    assert L.kvb_asm_index_csr(f, 100, 2, 7, f, f, f, 2 * 7 * 4 - 1, None) == _lib.KVB_EINVAL
     ws = L.kvb_asm_workspace_bytes(256, 32, 4096)
     assert ws == 32 * 256 * 32 * 8   # 32 ranges of 128 centroids, one 8-byte key per (range, query, head)
     assert L.kvb_asm_lookup_merge(f, f, f, f, f, f, 256, 32, 4096, 128, None, f, None, f, ws - 1, None) == _lib.KVB_EINVAL

@@ -134,3 +134,34 @@ def test_build_matches_oracle():
     np.testing.assert_array_equal(host(idx), idx_r)
     want = ob.asm_aggregate(q, a, lse, idx_r, 10)
     check_aggregate((host(qbar), host(abar.float()), host(lz), host(cnt)), want)
+
+
+def test_index_build_matches_oracle_and_serves_the_two_level_lookup(oracle):
+    """A memory whose entries sit in 16 groups per head: the GPU index (bf16 entries clustered
+    by the lookup + mean update, then the deterministic cluster lists) equals the oracle's, and
+    the two-level lookup through it answers as the oracle's lookup through the oracle's index."""
+    from test_gpu_asm_hier import run_hier, check_hier
+    g = rng(11, 34)
+    H, C, per, d = 3, 16, 40, 128
+    K = C * per
+    u = g.standard_normal((H, C, d))
+    u /= np.linalg.norm(u, axis=-1, keepdims=True)
+    owner = np.stack([g.permutation(np.arange(K) % C) for _ in range(H)])             # [H, K]
+    qbar = (u[np.arange(H)[:, None], owner] + 0.05 * g.standard_normal((H, K, d))).astype(np.float32)
+    init = np.stack([np.array([np.nonzero(owner[h] == c)[0][0] for c in range(C)]) for h in range(H)])
+    qhat, offsets, members, idx = asm_build.asm_index(dev(qbar), init, iters=2)
+    qhat_r, off_r, mem_r, idx_r = ob.asm_index(qbar, init, 2)
+    np.testing.assert_array_equal(idx_r, owner.T)
+    np.testing.assert_array_equal(host(idx), idx_r)
+    np.testing.assert_array_equal(host(offsets), off_r)
+    np.testing.assert_array_equal(host(members), mem_r)
+    np.testing.assert_allclose(host(qhat), qhat_r, rtol=1e-5, atol=1e-6)
+    N, m = 24, 4
+    q = normal_bf16(g, (N, H, d))
+    abar = normal_bf16(g, (H, K, d))
+    lz = g.uniform(2, 9, (H, K)).astype(np.float32)
+    o_self = g.standard_normal((N, H, d)).astype(np.float32)
+    l_self = g.uniform(1, 5, (N, H)).astype(np.float32)
+    sel, hidx, o, lse = run_hier(q, host(qhat), host(offsets), host(members), qbar, abar, lz, o_self, l_self, m)
+    check_hier(oracle, q, qhat_r.astype(np.float32), off_r, mem_r, qbar, abar, lz, o_self, l_self, m,
+               sel, hidx, o, lse)
