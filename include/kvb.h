@@ -388,6 +388,31 @@ kvb_status kvb_asm_index_csr(const int32_t* idx, int32_t K, int32_t H, int32_t C
                              int32_t* members, void* workspace, size_t workspace_bytes, kvb_stream stream);
 
 /* ------------------------------------------------------------------------
+ * GQA-grouped memory tables ([ASM] GQA extension: a group's queries are
+ * aggregated and the centroids stored per KV head)
+ *
+ * kvb_asm_lookup_merge_grouped / kvb_asm_aggregate_grouped: as
+ * kvb_asm_lookup_merge / kvb_asm_aggregate with H_tables tables shared by
+ * the H query heads: head h reads (lookup) or feeds (aggregation) table
+ * h / (H / H_tables); qbar, abar, log_zbar, count have H_tables rows instead
+ * of H. The aggregation folds the calibration rows of all heads of a table
+ * together; its workspace is kvb_asm_aggregate_workspace_bytes(H_tables, K).
+ * H_tables must divide H. kvb_asm_lookup_merge and kvb_asm_aggregate are the
+ * case H_tables == H.
+ * ---------------------------------------------------------------------- */
+kvb_status kvb_asm_lookup_merge_grouped(const uint16_t* q, const float* qbar, const uint16_t* abar,
+                                        const float* log_zbar, const float* o_self, const float* lse_self,
+                                        int32_t N, int32_t H, int32_t H_tables, int32_t K, int32_t d,
+                                        int32_t* idx, float* o, float* lse, void* workspace,
+                                        size_t workspace_bytes, kvb_stream stream);
+
+kvb_status kvb_asm_aggregate_grouped(const uint16_t* q, const float* a, const float* lse, const int32_t* idx,
+                                     int32_t M, int32_t H, int32_t H_tables, int32_t K, int32_t d,
+                                     int32_t z_mean, float* qbar, uint16_t* abar, float* log_zbar,
+                                     int32_t* count, void* workspace, size_t workspace_bytes,
+                                     kvb_stream stream);
+
+/* ------------------------------------------------------------------------
  * Errors and diagnostics
  * ---------------------------------------------------------------------- */
 

@@ -22,6 +22,7 @@ __all__ = [
     "kvb_asm_workspace_bytes", "kvb_asm_lookup_merge", "kvb_asm_hier_workspace_bytes",
     "kvb_asm_hier_lookup_merge", "kvb_asm_aggregate_workspace_bytes", "kvb_asm_aggregate",
     "kvb_asm_entries_bf16", "kvb_asm_index_workspace_bytes", "kvb_asm_index_csr",
+    "kvb_asm_lookup_merge_grouped", "kvb_asm_aggregate_grouped",
     "kvb_get_error", "kvb_abi_version",
     "decode_workspace", "evict_candidates",
 ]
@@ -275,9 +276,10 @@ def kvb_asm_workspace_bytes(N: int, H: int, K: int) -> int:
 
 def kvb_asm_lookup_merge(q, qbar, abar, log_zbar, o_self, lse_self, idx, o, lse, workspace, *,
                          stream=None) -> None:
-    """Attention-state-memory lookup and merge; see kvb_asm_lookup_merge in include/kvb.h.
+    """Attention-state-memory lookup and merge; see kvb_asm_lookup_merge(_grouped) in include/kvb.h.
     workspace: a uint8 CUDA tensor of at least kvb_asm_workspace_bytes(N, H, K) bytes.
-    o=None: only idx is computed (abar, log_zbar, o_self, lse_self, lse may be None)."""
+    o=None: only idx is computed (abar, log_zbar, o_self, lse_self, lse may be None).
+    qbar [H_tables, K, d] with H_tables dividing H: head h reads table h // (H // H_tables)."""
     _need(q, torch.bfloat16, "q"); _need(qbar, torch.float32, "qbar")
     if o is not None:
         _need(abar, torch.bfloat16, "abar"); _need(log_zbar, torch.float32, "log_zbar")
@@ -294,11 +296,15 @@ def kvb_asm_lookup_merge(q, qbar, abar, log_zbar, o_self, lse_self, idx, o, lse,
     if lse is not None:
         _need(lse, torch.float32, "lse"); _contig(lse, "lse")
     N, H, d = q.shape
-    K = qbar.shape[1]
+    Ht, K = qbar.shape[0], qbar.shape[1]
     nbytes = workspace.numel() * workspace.element_size()
-    _check(_lib.lib().kvb_asm_lookup_merge(_ptr(q), _ptr(qbar), _ptr(abar), _ptr(log_zbar), _ptr(o_self),
-                                           _ptr(lse_self), N, H, K, d, _ptr(idx), _ptr(o), _ptr(lse),
-                                           _ptr(workspace), nbytes, _stream(stream)), "kvb_asm_lookup_merge")
+    _check(_lib.lib().kvb_asm_lookup_merge_grouped(_ptr(q), _ptr(qbar), _ptr(abar), _ptr(log_zbar), _ptr(o_self),
+                                                   _ptr(lse_self), N, H, Ht, K, d, _ptr(idx), _ptr(o), _ptr(lse),
+                                                   _ptr(workspace), nbytes, _stream(stream)),
+           "kvb_asm_lookup_merge_grouped")
+
+
+kvb_asm_lookup_merge_grouped = kvb_asm_lookup_merge   # the table count is qbar's first dimension
 
 
 def kvb_asm_aggregate_workspace_bytes(H: int, K: int) -> int:
@@ -307,9 +313,10 @@ def kvb_asm_aggregate_workspace_bytes(H: int, K: int) -> int:
 
 def kvb_asm_aggregate(q, a, lse, idx, qbar, abar, log_zbar, count, workspace, *, z_mean: bool = False,
                       stream=None) -> None:
-    """Attention-aware aggregation (offline memory build); see kvb_asm_aggregate in include/kvb.h.
-    a, lse None: only qbar (and count) are computed. workspace: a uint8 CUDA tensor of at least
-    kvb_asm_aggregate_workspace_bytes(H, K) bytes."""
+    """Attention-aware aggregation (offline memory build); see kvb_asm_aggregate(_grouped) in
+    include/kvb.h. a, lse None: only qbar (and count) are computed. qbar [H_tables, K, d]: the
+    rows of head h feed table h // (H // H_tables). workspace: a uint8 CUDA tensor of at least
+    kvb_asm_aggregate_workspace_bytes(H_tables, K) bytes."""
     _need(q, torch.bfloat16, "q"); _need(idx, torch.int32, "idx"); _need(qbar, torch.float32, "qbar")
     if (a is None) != (lse is None):
         raise KvbError("kvb_asm_aggregate: a and lse go together")
@@ -323,11 +330,15 @@ def kvb_asm_aggregate(q, a, lse, idx, qbar, abar, log_zbar, count, workspace, *,
         if x is not None:
             _contig(x, name)
     M, H, d = q.shape
-    K = qbar.shape[1]
+    Ht, K = qbar.shape[0], qbar.shape[1]
     nbytes = workspace.numel() * workspace.element_size()
-    _check(_lib.lib().kvb_asm_aggregate(_ptr(q), _ptr(a), _ptr(lse), _ptr(idx), M, H, K, d, int(bool(z_mean)),
-                                        _ptr(qbar), _ptr(abar), _ptr(log_zbar), _ptr(count), _ptr(workspace),
-                                        nbytes, _stream(stream)), "kvb_asm_aggregate")
+    _check(_lib.lib().kvb_asm_aggregate_grouped(_ptr(q), _ptr(a), _ptr(lse), _ptr(idx), M, H, Ht, K, d,
+                                                int(bool(z_mean)), _ptr(qbar), _ptr(abar), _ptr(log_zbar),
+                                                _ptr(count), _ptr(workspace), nbytes, _stream(stream)),
+           "kvb_asm_aggregate_grouped")
+
+
+kvb_asm_aggregate_grouped = kvb_asm_aggregate   # the table count is qbar's first dimension
 
 
 def kvb_asm_entries_bf16(qbar, q, *, stream=None) -> None:

@@ -17,6 +17,7 @@ EXPORTS = (
     "kvb_asm_workspace_bytes", "kvb_asm_lookup_merge", "kvb_asm_hier_workspace_bytes",
     "kvb_asm_hier_lookup_merge", "kvb_asm_aggregate_workspace_bytes", "kvb_asm_aggregate",
     "kvb_asm_entries_bf16", "kvb_asm_index_workspace_bytes", "kvb_asm_index_csr",
+    "kvb_asm_lookup_merge_grouped", "kvb_asm_aggregate_grouped",
     "kvb_get_error", "kvb_status_str",
     "kvb_abi_version",
 )
@@ -80,13 +81,16 @@ def lib() -> ctypes.CDLL:
         L.kvb_asm_index_workspace_bytes.argtypes = [_I32, _I32]
         L.kvb_asm_index_workspace_bytes.restype = _SZ
         L.kvb_asm_index_csr.argtypes = [_P, _I32, _I32, _I32, _P, _P, _P, _SZ, _P]
+        L.kvb_asm_lookup_merge_grouped.argtypes = [_P] * 6 + [_I32] * 5 + [_P] * 4 + [_SZ, _P]
+        L.kvb_asm_aggregate_grouped.argtypes = [_P] * 4 + [_I32] * 6 + [_P] * 5 + [_SZ, _P]
         L.kvb_get_error.argtypes = [_P, ctypes.POINTER(ctypes.c_uint32)]
         L.kvb_status_str.argtypes = [_I32]
         L.kvb_status_str.restype = ctypes.c_char_p
         L.kvb_abi_version.argtypes = []
         for f in ("kvb_decode_attn", "kvb_decode_attn_noalloc", "kvb_merge_states", "kvb_evict_insert", "kvb_compact_blocks",
                   "kvb_asm_lookup_merge", "kvb_asm_hier_lookup_merge", "kvb_asm_aggregate",
-                  "kvb_asm_entries_bf16", "kvb_asm_index_csr", "kvb_get_error",
+                  "kvb_asm_entries_bf16", "kvb_asm_index_csr", "kvb_asm_lookup_merge_grouped",
+                  "kvb_asm_aggregate_grouped", "kvb_get_error",
                   "kvb_abi_version"):
             getattr(L, f).restype = _I32
         _lib = L

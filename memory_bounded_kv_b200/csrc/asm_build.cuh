@@ -1,7 +1,7 @@
 // Attention-state-memory offline build, "Context Memorization" core method
-// step 2 (attention-aware aggregation): per head h and cluster k, over the
-// calibration queries i assigned to k,
-//   qbar[h, k]     = mean of q[i, h]
+// step 2 (attention-aware aggregation): per table t and cluster k, over the
+// calibration rows (i, h) of the table's heads (h / G == t) assigned to k,
+//   qbar[t, k]     = mean of q[i, h]
 //   (abar, Zbar)   = merge-fold of (a[i, h], Z[i, h]): Zbar = sum Z_i (the page's merge
 //                    operator sums Z; z_mean divides by the member count),
 //                    abar = sum Z_i a_i / Zbar, computed in the log domain:
@@ -34,6 +34,7 @@ struct AsmBuildParams {
     float* wsum;            // [H, K]
     float* qsum;            // [H, K, d]
     float* asum;            // [H, K, d]
+    int G;                  // query heads per table: row (i, h) goes to table h / G
 };
 
 __device__ __forceinline__ float float_from_order_key(unsigned k) {
@@ -56,7 +57,7 @@ __global__ void __launch_bounds__(256) asm_build_pass1_kernel(const __grid_const
         if (lane == 0) raise_error(KVB_DERR_RANGE);
         return;
     }
-    const size_t hk = (size_t)h * p.K + k;
+    const size_t hk = (size_t)(h / p.G) * p.K + k;
     if (lane == 0) {
         atomicAdd(p.cnt + hk, 1);
         if (p.lse != nullptr) atomicMax(p.cmax + hk, float_order_key(p.lse[r]));
@@ -73,7 +74,7 @@ __global__ void __launch_bounds__(256) asm_build_pass2_kernel(const __grid_const
     if (r >= (long long)p.M * p.H) return;
     const int h = (int)(r % p.H), k = p.idx[r];
     if (k < 0 || k >= p.K) return;
-    const size_t hk = (size_t)h * p.K + k;
+    const size_t hk = (size_t)(h / p.G) * p.K + k;
     const float m = float_from_order_key(p.cmax[hk]);
     const float l = p.lse[r];
     if (l == -INFINITY || m == -INFINITY) return;   // Z_i = 0 contributes nothing
@@ -87,8 +88,8 @@ __global__ void __launch_bounds__(256) asm_build_pass2_kernel(const __grid_const
 // finalise: one warp per (h, k)
 __global__ void __launch_bounds__(256) asm_build_final_kernel(const __grid_constant__ AsmBuildParams p) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long hk = (long long)blockIdx.x * 8 + warp;
-    if (hk >= (long long)p.H * p.K) return;
+    const long long hk = (long long)blockIdx.x * 8 + warp;   // table * K + cluster
+    if (hk >= (long long)(p.H / p.G) * p.K) return;
     const int n = p.cnt[hk];
     if (lane == 0 && p.count != nullptr) p.count[hk] = n;
     float4 qm = make_float4(0.f, 0.f, 0.f, 0.f);

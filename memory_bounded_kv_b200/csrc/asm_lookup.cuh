@@ -37,6 +37,7 @@ struct AsmParams {
     float* o;
     float* lse;
     unsigned long long* ws;  // [ksplit][N][H]
+    int G;                   // query heads per table: head h reads table h / G
 };
 
 // Centroid ranges per head: ranges of 128 centroids (two tiles) or more, at most 64 of them,
@@ -243,7 +244,7 @@ __global__ void __launch_bounds__(kUThreads, 1) asm_score_umma_kernel(const __gr
         auto load_tile = [&](const AsmTile& c) {
             const int k = c.kt + cr;
             const bool in = k < c.k_end;
-            const float* src = p.qbar + ((size_t)c.h * p.K + (in ? k : 0)) * kAsmD;
+            const float* src = p.qbar + ((size_t)(c.h / p.G) * p.K + (in ? k : 0)) * kAsmD;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int j = 8 * (i >> 1) + ca + 4 * ((i + cr) & 1);
@@ -413,7 +414,8 @@ __global__ void __launch_bounds__(256) asm_merge_kernel(const __grid_constant__ 
     const int k = (int)(0xffffffffu - (unsigned)(best & 0xffffffffull));
     if (lane == 0 && p.idx != nullptr) p.idx[nh] = k;
     const float ls = p.lse_self[nh];
-    const float lm = p.lz[(size_t)h * p.K + k];
+    const int t = h / p.G;   // the head's table
+    const float lm = p.lz[(size_t)t * p.K + k];
     const float mx = fmaxf(ls, lm);
     const float mu = (mx == -INFINITY) ? 0.f : mx;
     const float ws = exp2f((ls - mu) * kLog2e), wm = exp2f((lm - mu) * kLog2e);
@@ -421,7 +423,7 @@ __global__ void __launch_bounds__(256) asm_merge_kernel(const __grid_constant__ 
     const float inv = (tot > 0.f) ? 1.f / tot : 0.f;
     if (lane == 0 && p.lse != nullptr) p.lse[nh] = (tot > 0.f) ? mx + log2f(tot) * kLn2 : -INFINITY;
     const float4 os = *reinterpret_cast<const float4*>(p.o_self + nh * kAsmD + lane * 4);
-    const uint2 am = *reinterpret_cast<const uint2*>(p.abar + ((size_t)h * p.K + k) * kAsmD + lane * 4);
+    const uint2 am = *reinterpret_cast<const uint2*>(p.abar + ((size_t)t * p.K + k) * kAsmD + lane * 4);
     float4 r;
     r.x = (ws * os.x + wm * bf16_lo(am.x)) * inv;
     r.y = (ws * os.y + wm * bf16_hi(am.x)) * inv;

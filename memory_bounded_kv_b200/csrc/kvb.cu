@@ -195,7 +195,7 @@ inline size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
 extern "C" {
 
-int32_t kvb_abi_version(void) { return 4; }
+int32_t kvb_abi_version(void) { return 5; }
 
 const char* kvb_status_str(kvb_status s) {
     switch (s) {
@@ -345,11 +345,13 @@ size_t kvb_asm_workspace_bytes(int32_t N, int32_t H, int32_t K) {
     return (size_t)kvb::asm_ksplit(K) * N * H * sizeof(unsigned long long);
 }
 
-kvb_status kvb_asm_lookup_merge(const uint16_t* q, const float* qbar, const uint16_t* abar, const float* log_zbar,
-                                const float* o_self, const float* lse_self, int32_t N, int32_t H, int32_t K,
-                                int32_t d, int32_t* idx, float* o, float* lse, void* workspace,
-                                size_t workspace_bytes, kvb_stream stream) {
+kvb_status kvb_asm_lookup_merge_grouped(const uint16_t* q, const float* qbar, const uint16_t* abar,
+                                        const float* log_zbar, const float* o_self, const float* lse_self,
+                                        int32_t N, int32_t H, int32_t H_tables, int32_t K, int32_t d, int32_t* idx,
+                                        float* o, float* lse, void* workspace, size_t workspace_bytes,
+                                        kvb_stream stream) {
     if (d != kvb::kAsmD || N < 1 || H < 1 || K < 1 || H > 65535) return KVB_EINVAL;
+    if (H_tables < 1 || H % H_tables != 0) return KVB_EINVAL;
     if (!q || !qbar || !workspace) return KVB_EINVAL;
     if (o == nullptr) {   // assignment only
         if (idx == nullptr) return KVB_EINVAL;
@@ -370,12 +372,20 @@ kvb_status kvb_asm_lookup_merge(const uint16_t* q, const float* qbar, const uint
     const int per_cta = (int)((items + slots - 1) / slots);
     const int grid = (int)((items + per_cta - 1) / per_cta);
     kvb::AsmParams p{q, qbar, abar, log_zbar, o_self, lse_self, N, H, K, kvb::asm_ksplit(K), kvb::asm_kchunk(K),
-                     qtiles, per_cta, idx, o, lse, static_cast<unsigned long long*>(workspace)};
+                     qtiles, per_cta, idx, o, lse, static_cast<unsigned long long*>(workspace), H / H_tables};
     kvb::asm_score_umma_kernel<<<grid, kvb::kUThreads, kvb::kUSmem, st>>>(p);
     if (launched() != KVB_OK) return KVB_ECUDA;
     const long long rows = (long long)N * H;
     kvb::asm_merge_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p);
     return launched();
+}
+
+kvb_status kvb_asm_lookup_merge(const uint16_t* q, const float* qbar, const uint16_t* abar, const float* log_zbar,
+                                const float* o_self, const float* lse_self, int32_t N, int32_t H, int32_t K,
+                                int32_t d, int32_t* idx, float* o, float* lse, void* workspace,
+                                size_t workspace_bytes, kvb_stream stream) {
+    return kvb_asm_lookup_merge_grouped(q, qbar, abar, log_zbar, o_self, lse_self, N, H, H, K, d, idx, o, lse,
+                                        workspace, workspace_bytes, stream);
 }
 
 size_t kvb_asm_hier_workspace_bytes(int32_t N, int32_t H, int32_t m) {
@@ -414,7 +424,7 @@ kvb_status kvb_asm_hier_lookup_merge(const uint16_t* q, const float* qhat, const
     if (launch_pdl(kvb::asm_hier_score_kernel, dim3((unsigned)(nh * m)), dim3(256), 0, st, hp) != KVB_OK)
         return KVB_ECUDA;
     // reduction over the m selected clusters' keys + merge: the linear lookup's merge kernel
-    kvb::AsmParams p{q, qbar, abar, log_zbar, o_self, lse_self, N, H, K, m, 0, 0, 0, idx, o, lse, keys};
+    kvb::AsmParams p{q, qbar, abar, log_zbar, o_self, lse_self, N, H, K, m, 0, 0, 0, idx, o, lse, keys, 1};
     return launch_pdl(kvb::asm_merge_kernel, dim3((unsigned)((nh + 7) / 8)), dim3(256), 0, st, p);
 }
 
@@ -424,17 +434,18 @@ size_t kvb_asm_aggregate_workspace_bytes(int32_t H, int32_t K) {
     return hk * (3 * sizeof(uint32_t)) + 2 * hk * kvb::kBuildD * sizeof(float);
 }
 
-kvb_status kvb_asm_aggregate(const uint16_t* q, const float* a, const float* lse, const int32_t* idx,
-                             int32_t M, int32_t H, int32_t K, int32_t d, int32_t z_mean,
-                             float* qbar, uint16_t* abar, float* log_zbar, int32_t* count,
-                             void* workspace, size_t workspace_bytes, kvb_stream stream) {
+kvb_status kvb_asm_aggregate_grouped(const uint16_t* q, const float* a, const float* lse, const int32_t* idx,
+                                     int32_t M, int32_t H, int32_t H_tables, int32_t K, int32_t d, int32_t z_mean,
+                                     float* qbar, uint16_t* abar, float* log_zbar, int32_t* count,
+                                     void* workspace, size_t workspace_bytes, kvb_stream stream) {
     if (d != kvb::kBuildD || M < 1 || H < 1 || K < 1) return KVB_EINVAL;
+    if (H_tables < 1 || H % H_tables != 0) return KVB_EINVAL;
     if (!q || !idx || !qbar || !workspace) return KVB_EINVAL;
     if ((a == nullptr) != (lse == nullptr)) return KVB_EINVAL;
     if (a != nullptr && (!abar || !log_zbar || !aligned16(a) || !aligned16(abar))) return KVB_EINVAL;
     if (!aligned16(q) || !aligned16(qbar) || !aligned16(workspace)) return KVB_EINVAL;
-    if (workspace_bytes < kvb_asm_aggregate_workspace_bytes(H, K)) return KVB_EINVAL;
-    const long long rows = (long long)M * H, hk = (long long)H * K;
+    if (workspace_bytes < kvb_asm_aggregate_workspace_bytes(H_tables, K)) return KVB_EINVAL;
+    const long long rows = (long long)M * H, hk = (long long)H_tables * K;
     if (rows > (1ll << 34) || hk * kvb::kBuildD > (1ll << 34)) return KVB_EINVAL;
     // workspace: qsum [H, K, d], asum [H, K, d], wsum [H, K], cmax [H, K], cnt [H, K]
     auto* base = static_cast<unsigned char*>(workspace);
@@ -444,9 +455,9 @@ kvb_status kvb_asm_aggregate(const uint16_t* q, const float* a, const float* lse
     auto* cmax = reinterpret_cast<unsigned*>(wsum + hk);
     int* cnt = reinterpret_cast<int*>(cmax + hk);
     kvb::AsmBuildParams p{q, a, lse, idx, M, H, K, z_mean ? 1 : 0, qbar, abar, log_zbar, count,
-                          cmax, cnt, wsum, qsum, asum};
+                          cmax, cnt, wsum, qsum, asum, H / H_tables};
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const size_t words = kvb_asm_aggregate_workspace_bytes(H, K) / sizeof(unsigned);
+    const size_t words = kvb_asm_aggregate_workspace_bytes(H_tables, K) / sizeof(unsigned);
     kvb::asm_build_zero_kernel<<<(unsigned)std::min<size_t>((words + 255) / 256, 4096), 256, 0, st>>>(
         static_cast<unsigned*>(workspace), words);
     if (launched() != KVB_OK) return KVB_ECUDA;
@@ -458,6 +469,14 @@ kvb_status kvb_asm_aggregate(const uint16_t* q, const float* a, const float* lse
     }
     kvb::asm_build_final_kernel<<<(unsigned)((hk + 7) / 8), 256, 0, st>>>(p);
     return launched();
+}
+
+kvb_status kvb_asm_aggregate(const uint16_t* q, const float* a, const float* lse, const int32_t* idx,
+                             int32_t M, int32_t H, int32_t K, int32_t d, int32_t z_mean,
+                             float* qbar, uint16_t* abar, float* log_zbar, int32_t* count,
+                             void* workspace, size_t workspace_bytes, kvb_stream stream) {
+    return kvb_asm_aggregate_grouped(q, a, lse, idx, M, H, H, K, d, z_mean, qbar, abar, log_zbar, count, workspace,
+                                     workspace_bytes, stream);
 }
 
 kvb_status kvb_asm_entries_bf16(const float* qbar, int32_t H, int32_t K, int32_t d, uint16_t* q,

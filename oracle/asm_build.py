@@ -108,3 +108,18 @@ def asm_index(qbar, init_rows, iters: int):
         offsets[h, 1:] = np.cumsum([len(o) for o in order])
         members[h] = np.concatenate(order).astype(np.int32)
     return cent, offsets, members, idx
+
+
+def group_rows(x, G: int):
+    """Calibration rows of a grouped table: x [M, H, ...] -> [M * G, H // G, ...], row (i, h)
+    going to table h // G ([ASM] GQA extension: the group's queries are aggregated)."""
+    x = np.asarray(x)
+    M, H = x.shape[:2]
+    y = x.reshape((M, H // G, G) + x.shape[2:])
+    y = np.moveaxis(y, 2, 1)                       # [M, G, H // G, ...]
+    return np.ascontiguousarray(y.reshape((M * G, H // G) + x.shape[2:]))
+
+
+def expand_tables(t, G: int):
+    """Per-head view of grouped tables: t [H // G, ...] -> [H, ...], head h reading table h // G."""
+    return np.repeat(np.asarray(t), G, axis=0)

@@ -47,7 +47,7 @@ def test_attn_args_struct_matches_header():
 
 def test_status_strings_and_version():
     L = _lib.lib()
-    assert L.kvb_abi_version() == 4
+    assert L.kvb_abi_version() == 5
     assert L.kvb_status_str(0) == b"ok"
     assert L.kvb_status_str(1) == b"invalid argument"
 
@@ -111,6 +111,11 @@ def test_other_entry_points_reject_bad_arguments_on_the_host():
     assert L.kvb_asm_index_csr(f, 100, 2, 0, f, f, f, 1 << 20, None) == _lib.KVB_EINVAL
     assert L.kvb_asm_index_workspace_bytes(2, 7) == 2 * 7 * 4
     assert L.kvb_asm_index_csr(f, 100, 2, 7, f, f, f, 2 * 7 * 4 - 1, None) == _lib.KVB_EINVAL
+    # grouped tables must divide the heads
+    assert L.kvb_asm_lookup_merge_grouped(f, f, f, f, f, f, 4, 6, 4, 16, 128, None, f, None, f, 1 << 20,
+                                          None) == _lib.KVB_EINVAL
+    assert L.kvb_asm_aggregate_grouped(f, None, None, f, 10, 6, 0, 8, 128, 0, f, None, None, None, f, 1 << 24,
+                                       None) == _lib.KVB_EINVAL
     ws = L.kvb_asm_workspace_bytes(256, 32, 4096)
     assert ws == 32 * 256 * 32 * 8   # 32 ranges of 128 centroids, one 8-byte key per (range, query, head)
     assert L.kvb_asm_lookup_merge(f, f, f, f, f, f, 256, 32, 4096, 128, None, f, None, f, ws - 1, None) == _lib.KVB_EINVAL

@@ -165,3 +165,41 @@ def test_index_build_matches_oracle_and_serves_the_two_level_lookup(oracle):
     sel, hidx, o, lse = run_hier(q, host(qhat), host(offsets), host(members), qbar, abar, lz, o_self, l_self, m)
     check_hier(oracle, q, qhat_r.astype(np.float32), off_r, mem_r, qbar, abar, lz, o_self, l_self, m,
                sel, hidx, o, lse)
+
+
+def test_grouped_lookup_reads_the_group_table(oracle):
+    """8 query heads sharing 2 tables (GQA groups of 4): equal to the per-head lookup with each
+    head given its group's table."""
+    from test_gpu_kernels import check_asm
+    g = rng(12, 35)
+    N, H, Ht, K, d = 50, 8, 2, 300, 128
+    q = normal_bf16(g, (N, H, d))
+    x = g.standard_normal((Ht, K, d))
+    qbar = (x / np.linalg.norm(x, axis=-1, keepdims=True)).astype(np.float32)
+    abar = normal_bf16(g, (Ht, K, d))
+    lz = g.uniform(5, 12, (Ht, K)).astype(np.float32)
+    o_self = g.standard_normal((N, H, d)).astype(np.float32)
+    l_self = g.uniform(3, 9, (N, H)).astype(np.float32)
+    idx = torch.zeros(N, H, dtype=torch.int32, device="cuda")
+    o = torch.zeros(N, H, d, device="cuda")
+    lse = torch.zeros(N, H, device="cuda")
+    ws = torch.empty(kvb.kvb_asm_workspace_bytes(N, H, K), dtype=torch.uint8, device="cuda")
+    kvb.kvb_asm_lookup_merge_grouped(dev(q), dev(qbar), dev(abar), dev(lz), dev(o_self), dev(l_self), idx, o, lse, ws)
+    torch.cuda.synchronize()
+    G = H // Ht
+    check_asm(oracle, q, ob.expand_tables(qbar, G), ob.expand_tables(abar, G), ob.expand_tables(lz, G), o_self,
+              l_self, host(idx), host(o), host(lse))
+
+
+def test_grouped_aggregate_folds_the_group_rows():
+    q, a, lse, idx = _inputs(13, 200, 8, 23)
+    Ht, G, K = 2, 4, 23
+    qbar = torch.zeros(Ht, K, 128, device="cuda")
+    abar = torch.zeros(Ht, K, 128, dtype=torch.bfloat16, device="cuda")
+    lz = torch.zeros(Ht, K, device="cuda")
+    cnt = torch.zeros(Ht, K, dtype=torch.int32, device="cuda")
+    ws = torch.empty(kvb.kvb_asm_aggregate_workspace_bytes(Ht, K), dtype=torch.uint8, device="cuda")
+    kvb.kvb_asm_aggregate_grouped(dev(q), dev(a), dev(lse), dev(idx), qbar, abar, lz, cnt, ws)
+    torch.cuda.synchronize()
+    want = ob.asm_aggregate(ob.group_rows(q, G), ob.group_rows(a, G), ob.group_rows(lse, G), ob.group_rows(idx, G), K)
+    check_aggregate((host(qbar), host(abar.float()), host(lz), host(cnt)), want)

@@ -175,3 +175,15 @@ def test_index_of_a_clustered_memory_lists_each_group_once(oracle):
                                                   o_self, l_self, C)
     idx_l, _, _ = oracle.asm_lookup_merge(q, qbar, abar, lz, o_self, l_self)
     np.testing.assert_array_equal(idx_h, idx_l)
+
+
+def test_group_helpers_route_rows_and_tables():
+    x = np.arange(3 * 4 * 2).reshape(3, 4, 2)           # M = 3, H = 4 heads
+    y = ob.group_rows(x, 2)                              # 2 tables of 2 heads
+    assert y.shape == (6, 2, 2)
+    for i in range(3):
+        for h in range(4):
+            hits = [r for r in range(6) if (y[r, h // 2] == x[i, h]).all()]
+            assert len(hits) == 1 and hits[0] // 2 == i
+    t = np.arange(2 * 3).reshape(2, 3)
+    np.testing.assert_array_equal(ob.expand_tables(t, 2), t[[0, 0, 1, 1]])
