@@ -187,3 +187,29 @@ def test_group_helpers_route_rows_and_tables():
             assert len(hits) == 1 and hits[0] // 2 == i
     t = np.arange(2 * 3).reshape(2, 3)
     np.testing.assert_array_equal(ob.expand_tables(t, 2), t[[0, 0, 1, 1]])
+
+
+def test_assignment_ties_and_zero_vectors_take_the_lower_index():
+    d = 8
+    v = np.linspace(0.5, 1.5, d).astype(np.float32)
+    q = to_bf16_bits(np.stack([v, np.zeros(d, np.float32)])[:, None, :])   # a query, a zero query
+    cent = np.stack([-v, v, v, 2 * v])[None].astype(np.float64)            # entries 1, 2, 3 tie at cos 1
+    idx = ob.cosine_assign(q, cent)
+    assert idx[0, 0] == 1 and idx[1, 0] == 0
+
+
+def test_one_lloyd_step_moves_a_centroid_by_hand():
+    """Unit vectors at 0, 10, 80 and 90 degrees; centroids start at the first two. Assignment:
+    [0, 1, 1, 1] (80 and 90 are nearer 10 than 0). Update: centroid 1 = mean of 10, 80, 90 degrees
+    (about 60 degrees). Reassignment: 10 degrees is now nearer 0 -> [0, 0, 1, 1]."""
+    ang = np.deg2rad([0.0, 10.0, 80.0, 90.0])
+    x = np.zeros((4, 1, 16), np.float32)
+    x[:, 0, 0], x[:, 0, 1] = np.cos(ang), np.sin(ang)
+    q = to_bf16_bits(x)
+    init = np.array([[0, 1]])
+    idx0, _ = ob.asm_kmeans(q, init, iters=0)
+    idx1, cent = ob.asm_kmeans(q, init, iters=1)
+    np.testing.assert_array_equal(idx0[:, 0], [0, 1, 1, 1])
+    np.testing.assert_array_equal(idx1[:, 0], [0, 0, 1, 1])
+    c1 = cent[0, 1, :2]
+    assert 55 < np.rad2deg(np.arctan2(c1[1], c1[0])) < 65
