@@ -1,10 +1,16 @@
 """memory_bounded_kv_b200: decode-step attention over a memory-bounded KV cache on B200.
 
-Python binding of libkvb (include/kvb.h). Each function has the name of the C
-entry point it calls and only marshals arguments: it checks dtypes, devices
-and layouts of torch tensors, passes their device pointers and strides, and
-raises KvbError when the library returns a non-OK status. Every step of the
-path runs in the library's CUDA kernels; there is no other implementation.
+Python binding of libkvb (include/kvb.h). Each function has the name of a C
+entry point and only marshals arguments: it checks dtypes, devices and layouts
+of torch tensors, passes their device pointers and strides, and raises
+KvbError when the library returns a non-OK status (kvb_asm_lookup_merge and
+kvb_asm_aggregate call the _grouped entry points, with the table count taken
+from qbar's first dimension). Every step of the path runs in the library's
+CUDA kernels; there is no other implementation.
+
+Modules: cache (BoundedKVCache: the decode step of one layer), asm_build (the
+memory's offline build: clustering, aggregation, two-level index), synth
+(seeded synthetic workloads).
 
 bf16 tensors are torch.bfloat16. Calls run on `stream` (default: torch's
 current stream) and are asynchronous.
