@@ -4,17 +4,25 @@
 Default workload: the Qwen3-8B-shaped layer decode step (B=32, Hq=32, Hkv=8,
 d=128, budget M=4096 slots per kv head, beta = sigmoid(N(2, 1.5))). A step is
 one decode token per sequence: budget enforcement + insertion
-(kvb_evict_insert), then split-K retention-gated attention with the split
-merge fused into the same launch (kvb_decode_attn). Block compaction and the
-attention-state-memory lookup belong to other workloads (--config 5, 4).
+(kvb_evict_insert), then split-K retention-gated attention, with the merge of
+the split states launched by the same call when there are several
+(kvb_decode_attn). --config selects the workload:
+  1  tiny decode step (B=1, Hq=8, Hkv=2, d=64, M=256)
+  2  the Qwen3-8B-shaped layer above (default)
+  3  long context: B=4, Hq=32, Hkv=8, d=128, 131072 positions kept in 8192 slots, 64 splits
+  4  attention-state memory: 256 query tokens x 32 heads, self attention over a shared
+     2048-token cache, then the lookup + merge against 4096 entries per head
+  5  memento compaction: B=64 sawtooth caches, 9 x (Geom(1500) block + U[120,180] memento)
 
-Prints ONE JSON line (rank 0). `value` is decode tokens/s of the whole job
-(one attention layer) with inputs resident in HBM; `e2e` is the same metric
-through the public API with the step's inputs copied from pinned host memory
-and the output read back every step. Every step reads > 126 MB (L2) of K/V,
-so no L2 flush is needed.
+Prints ONE JSON line (rank 0). `value` is tokens/s of the whole job (one
+attention layer) with inputs resident in HBM; `e2e` is the same metric through
+the public API with the step's inputs copied from pinned host memory and the
+output read back every step. The default workload reads > 126 MB (L2) of K/V
+per step, so no L2 flush is needed; workloads that fit in L2 are timed step by
+step after a flush (the JSON line's config says which).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1..5] [--impl kvb|reference]
+  python bench.py --asm-crossover | --asm-build     (lookup and build measurements, 1 GPU)
 
 For N > 1 launch with torch.distributed.run: every rank runs an independent
 replica (the path shards into independent sequences; no collective on the
@@ -183,7 +191,7 @@ def kernel_src_hash(name: str = "decode_attn_tc.cuh") -> str:
 
 
 # ----------------------------------------------------------------------------------------------
-# decode workloads (configs 1, 2, 3): evict+insert, then attention
+# decode workloads (tiny, Qwen3-8B-shaped, long context): evict+insert, then attention
 # ----------------------------------------------------------------------------------------------
 
 class DecodeBench:
@@ -226,7 +234,7 @@ class DecodeBench:
         self.lse = torch.zeros(w.B, w.Hq, device="cuda")
         self.tokens_per_step = w.B
         self.launches_per_step = 2 + (self.S > 1)   # evict/insert, attention (+ split merge)
-        self.workload = f"{w.name} (config {cfg})"
+        self.workload = w.name
 
     def t_of(self, i: int):
         return self.w.t0 + i
@@ -327,7 +335,7 @@ class DecodeBench:
 
 
 # ----------------------------------------------------------------------------------------------
-# config 4: attention-state-memory lookup (self attention + lookup/merge per step)
+# attention-state-memory workload: self attention + lookup/merge per step
 # ----------------------------------------------------------------------------------------------
 
 def _dev(a):
@@ -372,7 +380,7 @@ class ASMBench:
         self.ws = torch.empty(kvb.kvb_asm_workspace_bytes(N, H, w.K), dtype=torch.uint8, device="cuda")
         self.tokens_per_step = N
         self.launches_per_step = 4   # attention + split merge, lookup + state merge
-        self.workload = "attention-state memory H32 K4096 d128, 256 queries, self attention over 2048 (config 4)"
+        self.workload = "attention-state memory H32 K4096 d128, 256 queries, self attention over 2048"
 
     def prepare(self, total_steps):
         self.s_q = torch.empty_like(self.q)
@@ -428,7 +436,7 @@ class ASMBench:
 
 
 # ----------------------------------------------------------------------------------------------
-# config 5: memento-style block compaction (sawtooth cache)
+# memento-style block compaction (sawtooth cache)
 # ----------------------------------------------------------------------------------------------
 
 class MementoBench:
@@ -458,7 +466,7 @@ class MementoBench:
         self.lens = None
         self.tokens_per_step = None
         self.launches_per_step = None
-        self.workload = "memento compaction B64 Hq32 Hkv8 d128, 9 x (Geom(1500) block + U[120,180] memento) (config 5)"
+        self.workload = "memento compaction B64 Hq32 Hkv8 d128, 9 x (Geom(1500) block + U[120,180] memento)"
 
     def flush_l2(self):
         return True
@@ -703,7 +711,7 @@ def run_reference(args, world, rank):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{w.name} (config {2 if args.config not in (1, 3) else args.config})"},
+        "config": {"workload": w.name},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }

@@ -63,7 +63,7 @@ def log_beta(g: np.random.Generator, shape, mu: float = 2.0, sigma: float = 1.5)
 
 
 # --------------------------------------------------------------------------
-# decode workloads (configs 1-3)
+# decode workloads: tiny (1), Qwen3-8B-shaped layer (2), long context (3)
 # --------------------------------------------------------------------------
 
 @dataclass
@@ -117,14 +117,14 @@ CONFIG3_LOGICAL_T = 131072
 
 
 def decode_workload(cfg: int, B: int | None = None, prefill: int | None = None) -> DecodeWorkload:
-    """Prefilled cache for config 1, 2 or 3.
+    """Prefilled cache of decode workload 1 (tiny), 2 (Qwen3-8B-shaped) or 3 (long context).
 
     Prefill writes positions 0..prefill-1 into slots 0..prefill-1 (no eviction
     while the cache is within budget). `B` may shrink the batch (the first B
     sequences of the full draw are not reproduced; a smaller B is a different,
     smaller workload of the same shape).
 
-    For config 3 the returned cache is the starting point of the streaming
+    For the long-context workload the returned cache is the starting point of the streaming
     build (positions 0..8191); the caller streams positions 8192..131071
     through budget enforcement with ``stream_log_beta`` (30 blocks of 4096
     positions) and then redraws the surviving slots' K/V with ``config3_kv``.
@@ -169,7 +169,7 @@ def config3_kv(w: DecodeWorkload) -> tuple[np.ndarray, np.ndarray]:
 
 
 # --------------------------------------------------------------------------
-# config 4: attention-state memory lookup
+# attention-state memory lookup workload
 # --------------------------------------------------------------------------
 
 @dataclass
@@ -278,7 +278,7 @@ def asm_index_workload(N: int = 1, H: int = 32, K: int = 4096, C: int = 64, d: i
 
 
 # --------------------------------------------------------------------------
-# config 5: memento-style block compaction (sawtooth cache)
+# memento-style block compaction (sawtooth cache)
 # --------------------------------------------------------------------------
 
 @dataclass
