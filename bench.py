@@ -52,7 +52,7 @@ L2_BYTES = 126 * 1000 * 1000      # B200 L2 (126 MB)
 
 # ncu DRAM traffic (read + write bytes per launch) of the dominant kernel, keyed by
 # (sha256 of the kernel's source file, config, num_splits). Reported only while the source is
-# unchanged since the counters were taken (profiles/decode_attn_tc_config2.md).
+# unchanged since the counters were taken (profiles/decode_attn_tc_qwen3_layer.md).
 MEASURED_TRAFFIC = {
     # decode_attn_tc_kernel<128,4,1>, Qwen3-8B-shaped layer, S=1: 545,628,416 read + 3,972,608 written
     ("f9553bcebbe325aa", 2, 1): 549601024,
@@ -213,7 +213,7 @@ class DecodeBench:
                 for i in range(synth.STREAM_BLOCK):
                     kvb.kvb_evict_insert(self.cache.k, self.cache.v, self.cache.log_beta, self.cache.pos,
                                          self.cache.len, None, None, lbs[i], ts[i], w.M)
-            k, v = synth.config3_kv(w)
+            k, v = synth.long_context_kv(w)
             self.cache.k.copy_(torch.from_numpy(k.view(np.int16)).view(torch.bfloat16).cuda())
             self.cache.v.copy_(torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).cuda())
             torch.cuda.synchronize()

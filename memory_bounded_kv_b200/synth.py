@@ -127,7 +127,7 @@ def decode_workload(cfg: int, B: int | None = None, prefill: int | None = None) 
     For the long-context workload the returned cache is the starting point of the streaming
     build (positions 0..8191); the caller streams positions 8192..131071
     through budget enforcement with ``stream_log_beta`` (30 blocks of 4096
-    positions) and then redraws the surviving slots' K/V with ``config3_kv``.
+    positions) and then redraws the surviving slots' K/V with ``long_context_kv``.
     """
     c = dict(_DECODE_CONFIGS[cfg])
     if B is not None:
@@ -161,7 +161,7 @@ def stream_log_beta(w: DecodeWorkload, block: int) -> np.ndarray:
     return log_beta(g, (STREAM_BLOCK, w.B, w.Hkv))
 
 
-def config3_kv(w: DecodeWorkload) -> tuple[np.ndarray, np.ndarray]:
+def long_context_kv(w: DecodeWorkload) -> tuple[np.ndarray, np.ndarray]:
     """K/V of the slots that survive the config-3 streaming build (drawn after the build)."""
     g = rng(w.seed, _S_CACHE, 1)
     shape = (w.B, w.Hkv, w.cap, w.d)

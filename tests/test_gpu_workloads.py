@@ -45,7 +45,7 @@ def compare_cache(cache, c, what, b_max=None):
 
 
 @pytest.mark.parametrize("S", [1, 4])
-def test_config1_every_step(oracle, S):
+def test_tiny_decode_every_step(oracle, S):
     w = synth.decode_workload(1)
     cache = BoundedKVCache.from_host(w.k, w.v, w.log_beta, w.pos, w.len, w.Hq, w.M, num_splits=S)
     c = host_cache(w)
@@ -62,7 +62,7 @@ def test_config1_every_step(oracle, S):
             compare_cache(cache, c, f"step {step}")
 
 
-def test_config2_sampled_steps(oracle):
+def test_qwen3_layer_sampled_steps(oracle):
     w = synth.decode_workload(2)
     S = w.splits[0]
     cache = BoundedKVCache.from_host(w.k, w.v, w.log_beta, w.pos, w.len, w.Hq, w.M, num_splits=S)
@@ -81,7 +81,7 @@ def test_config2_sampled_steps(oracle):
             compare_cache(cache, c, f"step {step}")
 
 
-def config3_build(w, cache):
+def long_context_build(w, cache):
     """Stream positions cap .. 131071 through budget enforcement (log beta and pos only)."""
     blocks = (synth.CONFIG3_LOGICAL_T - w.cap) // synth.STREAM_BLOCK
     for blk in range(blocks):
@@ -94,11 +94,11 @@ def config3_build(w, cache):
     return blocks
 
 
-def test_config3_stream_and_decode(oracle):
+def test_long_context_stream_and_decode(oracle):
     w = synth.decode_workload(3)
     S = w.splits[0]
     cache = BoundedKVCache.from_host(w.k, w.v, w.log_beta, w.pos, w.len, w.Hq, w.M, num_splits=S)
-    blocks = config3_build(w, cache)
+    blocks = long_context_build(w, cache)
     torch.cuda.synchronize()
     # the oracle replays the stream for kv heads 0 and 5 of sequence 2
     sel = [(2, 0), (2, 5)]
@@ -120,7 +120,7 @@ def test_config3_stream_and_decode(oracle):
     assert np.all(gpos < synth.CONFIG3_LOGICAL_T) and all(
         len(np.unique(gpos[b, g])) == w.M for b in range(w.B) for g in range(w.Hkv))
     # survivors get their K/V, then 64 decode steps with 64 splits
-    k, v = synth.config3_kv(w)
+    k, v = synth.long_context_kv(w)
     cache.k.copy_(dev(k))
     cache.v.copy_(dev(v))
     c = dict(k=k, v=v, log_beta=glb.copy(), pos=gpos.copy(), len=host(cache.len))
@@ -144,7 +144,7 @@ def test_config3_stream_and_decode(oracle):
             assert_state_close(host(o_plain), host(lse_plain), o_ref, l_ref, f"plain step {step}")
 
 
-def test_config4_full(oracle):
+def test_memory_lookup_workload_full(oracle):
     w = synth.asm_workload()
     N, H, Hkv, d = w.N, w.H, w.Hkv, w.d
     # self attention of each query over its causal prefix of the shared cache (batch stride 0)
@@ -169,7 +169,7 @@ def test_config4_full(oracle):
     check_asm(oracle, w.q, w.qbar, w.abar, w.log_zbar, host(o_self), host(l_self), host(idx), host(o), host(lse))
 
 
-def test_config5_memento_compaction(oracle):
+def test_memento_compaction_workload(oracle):
     w = synth.memento_workload()
     SPLIT_LEN = 512
     S = -(-w.cap // SPLIT_LEN)
