@@ -52,7 +52,7 @@ L2_BYTES = 126 * 1000 * 1000      # B200 L2 (126 MB)
 
 # ncu DRAM traffic (read + write bytes per launch) of the dominant kernel, keyed by
 # (sha256 of the kernel's source file, config, num_splits). Reported only while the source is
-# unchanged since the counters were taken (profiles/decode_attn_tc_qwen3_layer.md).
+# unchanged since the counters were taken.
 MEASURED_TRAFFIC = {
     # decode_attn_tc_kernel<128,4,1>, Qwen3-8B-shaped layer, S=1: 545,628,416 read + 3,972,608 written
     ("f9553bcebbe325aa", 2, 1): 549601024,
@@ -373,7 +373,7 @@ class ASMBench:
         self.qbar, self.abar, self.lz = _dev(w.qbar), _dev(w.abar), _dev(w.log_zbar)
         self.o_self = torch.zeros(N, H, d, device="cuda")
         self.l_self = torch.zeros(N, H, device="cuda")
-        self.op, self.lp, self.cnt = kvb.decode_workspace(N, H, Hkv, d, self.S)
+        self.op, self.lp = kvb.decode_workspace(N, H, d, self.S)
         self.idx = torch.zeros(N, H, dtype=torch.int32, device="cuda")
         self.o = torch.zeros(N, H, d, device="cuda")
         self.lse = torch.zeros(N, H, device="cuda")
@@ -390,7 +390,7 @@ class ASMBench:
     def _step(self, q, events=None, j=0):
         kvb = self.kvb
         kvb.kvb_decode_attn(q, self.k, self.v, None, self.pos, self.len, self.t, self.o_self, self.l_self,
-                            num_splits=self.S, o_part=self.op, lse_part=self.lp, counters=self.cnt)
+                            num_splits=self.S, o_part=self.op, lse_part=self.lp)
         if events is not None:
             events[j][0].record()
         kvb.kvb_asm_lookup_merge(q, self.qbar, self.abar, self.lz, self.o_self, self.l_self, self.idx, self.o,

@@ -101,25 +101,31 @@ enum kvb_device_error {
  *            num_splits > 1 the call launches the attention kernel, which
  *            writes every split's state, and a merge kernel that combines
  *            them into o and lse.
- *   counters reserved; ignored (may be NULL).
+ *   counters reserved: no longer read; pass NULL (kept so that the
+ *            struct layout does not change).
  *   evict_cand  [B, Hkv, num_splits] kvb_evict_cand records, may be NULL.
  *            When given, the kernel also writes, for every split, the slot
  *            that budget enforcement at the NEXT position t[b] + 1 would pick
  *            within the split (the smallest (score, pos) with score =
  *            (float)(t[b] + 1 - pos) * log_beta, or 0 when log_beta is NULL;
- *            slot -1 for an empty split). It reads those fields anyway, so
- *            kvb_evict_insert can then skip its scan of the whole cache.
- *            Needs pos and t (and meta strides describing pos), 16-byte
- *            alignment; else KVB_EINVAL.
+ *            slot -1 for an empty split), stamped with that position t[b] + 1.
+ *            It reads those fields anyway, so kvb_evict_insert can then skip
+ *            its scan of the whole cache. Needs pos and t (and meta strides
+ *            describing pos), 16-byte alignment; else KVB_EINVAL.
  *
  * Requirements (else KVB_EINVAL): d in {64, 128}; Hq % Hkv == 0 and
- * Hq / Hkv in {1, 2, 4, 8}; B, Hkv, cap >= 1; 1 <= num_splits <= 1024;
+ * Hq / Hkv in {1, 2, 4, 8}; B, Hkv, cap >= 1; B * Hq < 2^31;
+ * 1 <= num_splits <= 1024;
  * split_len >= 0; q, k, v 16-byte aligned and every q/kv stride a multiple
  * of 8 elements; kv_stride_h > 0 when Hkv > 1; scale finite (0 selects
  * 1/sqrt(d)). K and V are read with TMA tensor copies, so a layout the
  * tensor-map encoder refuses also returns KVB_EINVAL.
  * Device-side checks: len in [0, cap] and len <= num_splits * split_len
- * (when split_len > 0); a row that fails gets the empty state.
+ * (when split_len > 0); a row that fails gets the empty state. Every wait
+ * of a CTA on its copies is bounded (1 s); a CTA that gives up sets
+ * KVB_DERR_TIMEOUT, waits (bounded) for the copies it issued and writes the
+ * empty state for every split it owns (lse_part = -inf, and with
+ * num_splits == 1 o = 0, lse = -inf; its candidate records get slot -1).
  * Preconditions (not checked): log beta finite and <= 0, positions unique
  * per (b, g), pos <= t.
  * ---------------------------------------------------------------------- */
@@ -150,7 +156,7 @@ typedef struct kvb_attn_args {
 typedef struct kvb_evict_cand {
     uint64_t key;   /* order-preserving key of (score, pos) */
     int32_t slot;   /* -1 for an empty split */
-    int32_t reserved;
+    int32_t t;      /* the position the record was scored for (t[b] + 1 of the attention) */
 } kvb_evict_cand;
 
 kvb_status kvb_decode_attn(const kvb_attn_args* args, kvb_stream stream);
@@ -231,11 +237,14 @@ kvb_status kvb_merge_states(const float* o_in, const float* lse_in,
  * [B, Hkv], all contiguous. victim [B, Hkv] int32 (may be NULL).
  * cand, cand_n: optional [B, Hkv, cand_n] kvb_evict_cand records written by
  * the kvb_decode_attn call that immediately preceded this one on the same
- * cache (same scoring: both with or both without log_beta), for position
- * t[b] - 1. When len >= M the victim is then the best record -- the same
- * slot a full scan picks, because the splits partition the slots -- and
- * the scan is skipped; a record set with no usable slot falls back to the
- * scan. 16-byte aligned, 1 <= cand_n <= 1024. NULL: always scan.
+ * cache (same scoring: both with or both without log_beta). A (b, g) uses
+ * its records only when every one of them is stamped with t[b] (the
+ * attention ran at t[b] - 1); when len >= M the victim is then the best
+ * record -- the same slot a full scan picks, because the splits partition
+ * the slots -- and the scan is skipped. Records stamped for another
+ * position (the caller skipped a position, or attended elsewhere in
+ * between) or with no usable slot fall back to the scan. 16-byte aligned,
+ * 1 <= cand_n <= 1024. NULL: always scan.
  * Requirements: d in [1, 1024] with d % 8 == 0 and k/v/k_new/v_new 16-byte
  * aligned; 1 <= M <= cap. Device-side check: len in [0, cap].
  * ---------------------------------------------------------------------- */
@@ -426,6 +435,21 @@ const char* kvb_status_str(kvb_status s);
 
 /* Version of the ABI described by this header. */
 int32_t kvb_abi_version(void);
+
+/* ------------------------------------------------------------------------
+ * Testing hook (failure detection without faulting a GPU)
+ *
+ * kvb_test_withhold_next_decode: the next kvb_decode_attn (or
+ * kvb_decode_attn_noalloc) call in this process launches its attention
+ * kernel with every producer warp withholding its copies: no copy is issued
+ * and no tile is ever signalled, so each CTA's first bounded wait runs out
+ * after wait_limit_ns nanoseconds. The kernel then takes its timeout path:
+ * KVB_DERR_TIMEOUT in the device error word and the empty state for every
+ * split (see kvb_decode_attn). The call returns normally and the context
+ * stays usable. One call arms one launch; 1000 <= wait_limit_ns <= 1e9, else
+ * KVB_EINVAL. Not for production use.
+ * ---------------------------------------------------------------------- */
+kvb_status kvb_test_withhold_next_decode(uint64_t wait_limit_ns);
 
 #ifdef __cplusplus
 }

@@ -29,7 +29,7 @@ __all__ = [
     "kvb_asm_hier_lookup_merge", "kvb_asm_aggregate_workspace_bytes", "kvb_asm_aggregate",
     "kvb_asm_entries_bf16", "kvb_asm_index_workspace_bytes", "kvb_asm_index_csr",
     "kvb_asm_lookup_merge_grouped", "kvb_asm_aggregate_grouped",
-    "kvb_get_error", "kvb_abi_version",
+    "kvb_get_error", "kvb_abi_version", "kvb_test_withhold_next_decode",
     "decode_workspace", "evict_candidates",
 ]
 
@@ -75,8 +75,46 @@ def _contig(t, name):
     return t
 
 
+def _shape(t, shape, name):
+    """Raise ValueError unless tensor t (skipped when None) has exactly `shape`. The library
+    cannot see buffer sizes, so every tensor is checked here before anything is launched."""
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if tuple(t.shape) != tuple(int(x) for x in shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _decode_shapes(q, k, v, log_beta, pos, len, t, o, lse, num_splits, o_part=None, lse_part=None):
+    """Shapes of every kvb_decode_attn(_noalloc) argument, from q [B, Hq, d] and k [B, Hkv, cap, d]."""
+    if q.dim() != 3 or k.dim() != 4:
+        raise ValueError("q must be [B, Hq, d] and k, v [B, Hkv, cap, d]")
+    B, Hq, d = q.shape
+    _, Hkv, cap, _ = k.shape
+    _shape(k, (B, Hkv, cap, d), "k")
+    _shape(v, (B, Hkv, cap, d), "v")
+    _shape(log_beta, (B, Hkv, cap), "log_beta")
+    _shape(pos, (B, Hkv, cap), "pos")
+    _shape(len, (B, Hkv), "len")
+    _shape(t, (B,), "t")
+    _shape(o, (B, Hq, d), "o")
+    _shape(lse, (B, Hq), "lse")
+    if int(num_splits) < 1:
+        raise ValueError("num_splits must be >= 1")
+    _shape(o_part, (B, Hq, num_splits, d), "o_part")
+    _shape(lse_part, (B, Hq, num_splits), "lse_part")
+    return B, Hq, Hkv, d, cap
+
+
 def kvb_abi_version() -> int:
     return int(_lib.lib().kvb_abi_version())
+
+
+def kvb_test_withhold_next_decode(wait_limit_ns: int) -> None:
+    """Testing hook: the next decode-attention call's producers withhold their copies, so its
+    bounded waits run out after wait_limit_ns (see kvb_test_withhold_next_decode in kvb.h)."""
+    _check(_lib.lib().kvb_test_withhold_next_decode(int(wait_limit_ns)), "kvb_test_withhold_next_decode")
 
 
 def kvb_get_error(stream=None) -> int:
@@ -101,32 +139,30 @@ def _cand_ptr(c, records):
     return c.data_ptr()
 
 
-def decode_workspace(B: int, Hq: int, Hkv: int, d: int, num_splits: int, device="cuda"):
-    """Zero-filled (o_part, lse_part, counters) buffers for kvb_decode_attn with num_splits > 1."""
+def decode_workspace(B: int, Hq: int, d: int, num_splits: int, device="cuda"):
+    """(o_part [B, Hq, S, d], lse_part [B, Hq, S]) f32 buffers for kvb_decode_attn with num_splits > 1."""
     o_part = torch.zeros(B, Hq, num_splits, d, dtype=torch.float32, device=device)
     lse_part = torch.zeros(B, Hq, num_splits, dtype=torch.float32, device=device)
-    counters = torch.zeros(B, Hkv, dtype=torch.int32, device=device)
-    return o_part, lse_part, counters
+    return o_part, lse_part
 
 
 def kvb_decode_attn(q, k, v, log_beta, pos, len, t, o, lse=None, *, scale: float = 0.0,
-                    num_splits: int = 1, split_len: int = 0, o_part=None, lse_part=None, counters=None,
+                    num_splits: int = 1, split_len: int = 0, o_part=None, lse_part=None,
                     evict_cand=None, stream=None) -> None:
     """Split-K GQA decode attention with retention bias; see kvb_decode_attn in include/kvb.h.
 
     q [B, Hq, d] bf16; k, v [B, Hkv, cap, d] bf16 (stride(2) == d, stride(3) == 1; an expanded
     view with stride(0) == 0 shares one cache); log_beta [B, Hkv, cap] f32 or None; pos
     [B, Hkv, cap] int32 (same strides as log_beta); len [B, Hkv] int32; t [B] int32 or None;
-    o [B, Hq, d] f32 or bf16; lse [B, Hq] f32 or None; o_part/lse_part from
-    decode_workspace() when num_splits > 1 (counters is accepted and ignored); evict_cand: a
-    CUDA tensor of >= B*Hkv*num_splits*16 bytes to receive the next position's eviction
-    candidates (see evict_candidates()), or None.
+    o [B, Hq, d] f32 or bf16; lse [B, Hq] f32 or None; o_part [B, Hq, S, d] / lse_part
+    [B, Hq, S] from decode_workspace() when num_splits = S > 1; evict_cand: a CUDA tensor of
+    >= B*Hkv*num_splits*16 bytes to receive the next position's eviction candidates (see
+    evict_candidates()), or None. Every shape is checked before anything is launched.
     """
+    B, Hq, Hkv, d, cap = _decode_shapes(q, k, v, log_beta, pos, len, t, o, lse, num_splits, o_part, lse_part)
+    if num_splits > 1 and (o_part is None or lse_part is None):
+        raise ValueError("num_splits > 1 needs o_part and lse_part (decode_workspace())")
     _need(q, torch.bfloat16, "q"); _need(k, torch.bfloat16, "k"); _need(v, torch.bfloat16, "v")
-    B, Hq, d = q.shape
-    Bk, Hkv, cap, dk = k.shape
-    if dk != d or tuple(v.shape) != tuple(k.shape) or Bk != B:
-        raise ValueError("k/v must be [B, Hkv, cap, d] matching q")
     if q.stride(2) != 1 or k.stride(3) != 1 or k.stride(2) != d or v.stride() != k.stride():
         raise ValueError("q/k/v: innermost dim contiguous, slot stride d, k and v with equal strides")
     _need(len, torch.int32, "len"); _contig(len, "len")
@@ -154,10 +190,9 @@ def kvb_decode_attn(q, k, v, log_beta, pos, len, t, o, lse=None, *, scale: float
     _contig(o, "o")
     if lse is not None:
         _need(lse, torch.float32, "lse"); _contig(lse, "lse")
-    for name, x, dt in (("o_part", o_part, torch.float32), ("lse_part", lse_part, torch.float32),
-                        ("counters", counters, torch.int32)):
+    for name, x in (("o_part", o_part), ("lse_part", lse_part)):
         if x is not None:
-            _need(x, dt, name); _contig(x, name)
+            _need(x, torch.float32, name); _contig(x, name)
     a = _lib.AttnArgs(
         q=q.data_ptr(), q_stride_b=q.stride(0), q_stride_h=q.stride(1),
         k=k.data_ptr(), v=v.data_ptr(), kv_stride_b=k.stride(0), kv_stride_h=k.stride(1),
@@ -168,8 +203,7 @@ def kvb_decode_attn(q, k, v, log_beta, pos, len, t, o, lse=None, *, scale: float
         B=B, Hq=Hq, Hkv=Hkv, d=d, cap=cap, scale=float(scale),
         num_splits=int(num_splits), split_len=int(split_len),
         o_part=None if o_part is None else o_part.data_ptr(),
-        lse_part=None if lse_part is None else lse_part.data_ptr(),
-        counters=None if counters is None else counters.data_ptr(),
+        lse_part=None if lse_part is None else lse_part.data_ptr(), counters=None,
         o=o.data_ptr(), o_dtype=odt, lse=None if lse is None else lse.data_ptr(),
         evict_cand=None if evict_cand is None else _cand_ptr(evict_cand, B * Hkv * int(num_splits)))
     _check(_lib.lib().kvb_decode_attn(ctypes.byref(a), _stream(stream)), "kvb_decode_attn")
@@ -179,18 +213,15 @@ def kvb_decode_attn_noalloc(q, k, v, log_beta, pos, len, t, o, lse=None, *, scal
                             num_splits: int = 1, split_len: int = 0, stream=None) -> None:
     """kvb_decode_attn for callers that cannot provide scratch device memory.
 
-    Same inputs and outputs as kvb_decode_attn, without o_part/lse_part/counters: the split
+    Same inputs and outputs as kvb_decode_attn, without o_part/lse_part: the split
     states live in the library's fixed device array (NOALLOC_SCRATCH_BYTES per GPU), so the
     call allocates nothing. A problem whose split states do not fit raises KvbError (invalid
     argument). Calls that overlap on the GPU share that array and race: keep them on one
     stream. The first call on a device looks up the array's address; make it before any
     stream capture.
     """
+    B, Hq, Hkv, d, cap = _decode_shapes(q, k, v, log_beta, pos, len, t, o, lse, num_splits)
     _need(q, torch.bfloat16, "q"); _need(k, torch.bfloat16, "k"); _need(v, torch.bfloat16, "v")
-    B, Hq, d = q.shape
-    Bk, Hkv, cap, dk = k.shape
-    if dk != d or tuple(v.shape) != tuple(k.shape) or Bk != B:
-        raise ValueError("k/v must be [B, Hkv, cap, d] matching q")
     if q.stride(2) != 1 or k.stride(3) != 1 or k.stride(2) != d or v.stride() != k.stride():
         raise ValueError("q/k/v: innermost dim contiguous, slot stride d, k and v with equal strides")
     _need(len, torch.int32, "len"); _contig(len, "len")
@@ -242,12 +273,19 @@ def kvb_evict_insert(k, v, log_beta, pos, len, k_new, v_new, log_beta_new, t, M:
     """Budget enforcement + insertion (in place); see kvb_evict_insert in include/kvb.h.
     k_new/v_new may both be None (only log_beta and pos are written); cand/cand_n: the
     candidates of the immediately preceding kvb_decode_attn on this cache, or None."""
+    if k.dim() != 4:
+        raise ValueError("k must be [B, Hkv, cap, d]")
+    B, Hkv, cap, d = k.shape
+    for name, x, shp in (("v", v, (B, Hkv, cap, d)), ("log_beta", log_beta, (B, Hkv, cap)),
+                         ("pos", pos, (B, Hkv, cap)), ("len", len, (B, Hkv)), ("k_new", k_new, (B, Hkv, d)),
+                         ("v_new", v_new, (B, Hkv, d)), ("log_beta_new", log_beta_new, (B, Hkv)),
+                         ("t", t, (B,)), ("victim", victim, (B, Hkv))):
+        _shape(x, shp, name)
     for name, x in (("k", k), ("v", v)):
         _need(x, torch.bfloat16, name); _contig(x, name)
     _need(pos, torch.int32, "pos"); _contig(pos, "pos")
     _need(len, torch.int32, "len"); _contig(len, "len")
     _need(t, torch.int32, "t"); _contig(t, "t")
-    B, Hkv, cap, d = k.shape
     if log_beta is not None:
         _need(log_beta, torch.float32, "log_beta"); _contig(log_beta, "log_beta")
         _need(log_beta_new, torch.float32, "log_beta_new"); _contig(log_beta_new, "log_beta_new")
@@ -265,13 +303,18 @@ def kvb_evict_insert(k, v, log_beta, pos, len, k_new, v_new, log_beta_new, t, M:
 
 def kvb_compact_blocks(k, v, pos, log_beta, len, rm_start, rm_len, *, stream=None) -> None:
     """In-place removal of slots [rm_start[b], +rm_len[b]) from every kv head of sequence b."""
+    if k.dim() != 4:
+        raise ValueError("k must be [B, Hkv, cap, d]")
+    B, Hkv, cap, d = k.shape
+    for name, x, shp in (("v", v, (B, Hkv, cap, d)), ("pos", pos, (B, Hkv, cap)), ("log_beta", log_beta, (B, Hkv, cap)),
+                         ("len", len, (B, Hkv)), ("rm_start", rm_start, (B,)), ("rm_len", rm_len, (B,))):
+        _shape(x, shp, name)
     for name, x in (("k", k), ("v", v)):
         _need(x, torch.bfloat16, name); _contig(x, name)
     for name, x in (("pos", pos), ("len", len), ("rm_start", rm_start), ("rm_len", rm_len)):
         _need(x, torch.int32, name); _contig(x, name)
     if log_beta is not None:
         _need(log_beta, torch.float32, "log_beta"); _contig(log_beta, "log_beta")
-    B, Hkv, cap, d = k.shape
     _check(_lib.lib().kvb_compact_blocks(_ptr(k), _ptr(v), _ptr(pos), _ptr(log_beta), _ptr(len), _ptr(rm_start),
                                          _ptr(rm_len), B, Hkv, d, cap, _stream(stream)), "kvb_compact_blocks")
 

@@ -19,7 +19,7 @@ EXPORTS = (
     "kvb_asm_entries_bf16", "kvb_asm_index_workspace_bytes", "kvb_asm_index_csr",
     "kvb_asm_lookup_merge_grouped", "kvb_asm_aggregate_grouped",
     "kvb_get_error", "kvb_status_str",
-    "kvb_abi_version",
+    "kvb_abi_version", "kvb_test_withhold_next_decode",
 )
 
 KVB_OK, KVB_EINVAL, KVB_ECUDA, KVB_EDEVICE = 0, 1, 2, 3
@@ -87,11 +87,12 @@ def lib() -> ctypes.CDLL:
         L.kvb_status_str.argtypes = [_I32]
         L.kvb_status_str.restype = ctypes.c_char_p
         L.kvb_abi_version.argtypes = []
+        L.kvb_test_withhold_next_decode.argtypes = [ctypes.c_uint64]
         for f in ("kvb_decode_attn", "kvb_decode_attn_noalloc", "kvb_merge_states", "kvb_evict_insert", "kvb_compact_blocks",
                   "kvb_asm_lookup_merge", "kvb_asm_hier_lookup_merge", "kvb_asm_aggregate",
                   "kvb_asm_entries_bf16", "kvb_asm_index_csr", "kvb_asm_lookup_merge_grouped",
                   "kvb_asm_aggregate_grouped", "kvb_get_error",
-                  "kvb_abi_version"):
+                  "kvb_abi_version", "kvb_test_withhold_next_decode"):
             getattr(L, f).restype = _I32
         _lib = L
     return _lib

@@ -39,9 +39,9 @@ class BoundedKVCache:
         self.pos = torch.zeros(B, Hkv, cap, dtype=torch.int32, device=device)
         self.len = torch.zeros(B, Hkv, dtype=torch.int32, device=device)
         self.victim = torch.zeros(B, Hkv, dtype=torch.int32, device=device)
-        self.o_part = self.lse_part = self.counters = None
+        self.o_part = self.lse_part = None
         if num_splits > 1:
-            self.o_part, self.lse_part, self.counters = decode_workspace(B, Hq, Hkv, d, num_splits, device)
+            self.o_part, self.lse_part = decode_workspace(B, Hq, d, num_splits, device)
         # eviction candidates for the next position, left by each attention pass
         self.cand = evict_candidates(B, Hkv, num_splits, device)
         self.cand_valid = False
@@ -74,9 +74,10 @@ class BoundedKVCache:
         cand = self.cand if (same_scoring and t is not None) else None
         kvb_decode_attn(q, self.k, self.v, lb, self.pos, self.len, t if (lb is not None or t is not None) else None,
                         o, lse, num_splits=self.num_splits, split_len=self.split_len, o_part=self.o_part,
-                        lse_part=self.lse_part, counters=self.counters, evict_cand=cand, stream=stream)
-        if cand is not None:
-            self.cand_valid = True
+                        lse_part=self.lse_part, evict_cand=cand, stream=stream)
+        # the records describe this attention's cache state only: an attention that leaves none
+        # makes earlier records stale for the next insertion
+        self.cand_valid = cand is not None
 
     def step(self, q, k_new, v_new, log_beta_new, t, o, lse=None, stream=None):
         """One decode step: budget enforcement + insertion, then attention (2 launches)."""

@@ -126,7 +126,7 @@ __device__ __forceinline__ void griddep_launch_dependents() {
 struct EvictCand {
     unsigned long long key;
     int slot;
-    int pad;
+    int t;  // the position the key was scored for
 };
 static_assert(sizeof(EvictCand) == 16, "candidate record");
 

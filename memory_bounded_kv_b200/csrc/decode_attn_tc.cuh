@@ -29,8 +29,9 @@
 //  - At the end of a unit the consumer warps combine through shared memory
 //    (a named barrier among consumers only; the producer keeps prefetching
 //    the next unit's tiles) and write the split's state.
-// Every wait is bounded (1 s); on a timeout the CTA records KVB_DERR_TIMEOUT,
-// stops, and drains the copies it issued before exiting.
+// Every wait is bounded (wait_ns, 1 s by default); on a timeout the CTA
+// records KVB_DERR_TIMEOUT, stops, drains the copies it issued (bounded) and
+// writes the empty state for every unit it owns.
 #pragma once
 
 #include <cuda.h>
@@ -57,6 +58,8 @@ struct DecodeTcParams {
     int o_bf16;
     float* lse;
     EvictCand* cand;  // nullable: per-split eviction candidates for position t + 1
+    unsigned long long wait_ns;  // limit of every mbarrier wait
+    int withhold;     // test hook: the producer issues nothing, so the consumers' first wait runs out
 };
 
 template <int D, int G>
@@ -256,6 +259,7 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                     EvictCand* c = p.cand + ((size_t)ui.b * p.Hkv + ui.g) * p.S + ui.split;
                     c->key = ~0ull;
                     c->slot = -1;
+                    c->t = raw.t + 1;
                 }
                 continue;
             }
@@ -263,6 +267,10 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
             const int tb = raw.t;
             const size_t m_off = end ? 0 : (size_t)ui.b * p.m_sb + (size_t)ui.g * p.m_sh + (size_t)ui.s0;
             const bool want_cand = p.cand != nullptr;
+            if (p.withhold) {   // test hook: no copy, no arrival; the consumers' wait runs out
+                stop = true;
+                break;
+            }
             for (int i = 0; i < records; ++i, ++it) {
                 const int st = it % ST;
                 // this tile's bias (and, for the eviction candidates, its pos and log beta),
@@ -287,7 +295,7 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                     }
                     bias[j] = bv;
                 }
-                if (it >= ST && !mbar_wait(&s_empty[st], (unsigned)((it / ST) - 1) & 1u)) {
+                if (it >= ST && !mbar_wait(&s_empty[st], (unsigned)((it / ST) - 1) & 1u, p.wait_ns)) {
                     if (lane == 0) {
                         raise_error(KVB_DERR_TIMEOUT);
                         *s_abort = 1;
@@ -374,7 +382,7 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
         bool aborted = false;
         while (true) {
             const int st = it % ST;
-            if (!mbar_wait(&s_full[st], (unsigned)(it / ST) & 1u)) {
+            if (!mbar_wait(&s_full[st], (unsigned)(it / ST) & 1u, p.wait_ns)) {
                 if (lane == 0) {
                     raise_error(KVB_DERR_TIMEOUT);
                     *s_abort = 1;
@@ -545,6 +553,7 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                 EvictCand* c = p.cand + ((size_t)ub * p.Hkv + ug) * p.S + usplit;
                 c->key = bk;
                 c->slot = (bk == ~0ull) ? -1 : bs;
+                c->t = m[8] + 1;
             }
             const int S = p.S;
             for (int idx = tid; idx < G * D; idx += NWC * 32) {
@@ -583,9 +592,36 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
 
     // drain: copies issued into stages that no consumer waited for
     __syncthreads();
-    if (tid == 0 && *s_abort) {
+    if (!*s_abort) return;
+    if (tid == 0) {
         const int issued = *s_issued;
         for (int k = max(0, issued - ST); k < issued; ++k) mbar_wait(&s_full[k % ST], (unsigned)(k / ST) & 1u, 100000000ull);
+    }
+    __syncthreads();
+    // a CTA that gave up leaves every unit it owns in the empty state (and no eviction candidate)
+    for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
+        const int per_b = p.Hkv * p.S;
+        const int b = u / per_b;
+        const int g = (u - b * per_b) / p.S;
+        const int split = u - b * per_b - g * p.S;
+        const size_t row0 = (size_t)b * p.Hq + g * G;
+        if (p.o_part != nullptr && tid < G) p.lse_part[(row0 + tid) * p.S + split] = -INFINITY;
+        if (p.S == 1) {
+            for (int idx = tid; idx < G * D; idx += SH::NT) {
+                if (p.o_bf16) {
+                    reinterpret_cast<__nv_bfloat16*>(p.o)[row0 * D + idx] = __float2bfloat16_rn(0.f);
+                } else {
+                    reinterpret_cast<float*>(p.o)[row0 * D + idx] = 0.f;
+                }
+            }
+            if (tid < G && p.lse != nullptr) p.lse[row0 + tid] = -INFINITY;
+        }
+        if (tid == 0 && p.cand != nullptr) {
+            EvictCand* c = p.cand + ((size_t)b * p.Hkv + g) * p.S + split;
+            c->key = ~0ull;
+            c->slot = -1;
+            c->t = (p.t == nullptr) ? 0 : p.t[b] + 1;
+        }
     }
 }
 

@@ -11,7 +11,8 @@
 // When the preceding attention left per-split candidates (the same key for
 // position t, computed while it read every slot), the victim is the best of
 // those few records instead: the same argmin, since the splits partition
-// the slots.
+// the slots. The records carry the position they were scored for; a set in
+// which any record was scored for another position is ignored (full scan).
 #pragma once
 
 #include "common.cuh"
@@ -78,9 +79,11 @@ __global__ void __launch_bounds__(NT) evict_insert_kernel(const __grid_constant_
         if (tid < 32) {
             unsigned long long best = ~0ull;
             int best_slot = 0x7fffffff;
+            bool stale = tid < p.cand_n && my_cand.t != tb;
             if (my_cand.slot >= 0) argmin_merge(best, best_slot, my_cand.key, my_cand.slot);
             for (int j = tid + 32; j < p.cand_n; j += 32) {   // records past the first 32
                 const EvictCand c = p.cand[(size_t)bg * p.cand_n + j];
+                stale = stale || c.t != tb;
                 if (c.slot >= 0) argmin_merge(best, best_slot, c.key, c.slot);
             }
 #pragma unroll
@@ -89,7 +92,9 @@ __global__ void __launch_bounds__(NT) evict_insert_kernel(const __grid_constant_
                 const int s2 = __shfl_xor_sync(kFull, best_slot, m);
                 argmin_merge(best, best_slot, k2, s2);
             }
-            if (tid == 0) s_cand = (best != ~0ull && best_slot < n) ? best_slot : -1;
+            // records scored for another position rank the slots differently: scan instead
+            stale = __any_sync(kFull, stale);
+            if (tid == 0) s_cand = (!stale && best != ~0ull && best_slot < n) ? best_slot : -1;
         }
         __syncthreads();
         slot = s_cand;

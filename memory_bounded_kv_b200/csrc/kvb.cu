@@ -5,6 +5,7 @@
 #include <cstdint>
 #include <map>
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <tuple>
 #include <utility>
@@ -191,11 +192,21 @@ kvb_status noalloc_scratch(void** out) {
 
 inline size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
+// Test hook of kvb_test_withhold_next_decode: the wait limit (ns) the next decode launch uses
+// with its producers withholding their copies; 0 = off. Taken (and cleared) by one call.
+std::atomic<unsigned long long> g_withhold_next{0};
+
 }  // namespace
 
 extern "C" {
 
-int32_t kvb_abi_version(void) { return 5; }
+int32_t kvb_abi_version(void) { return 6; }
+
+kvb_status kvb_test_withhold_next_decode(uint64_t wait_limit_ns) {
+    if (wait_limit_ns < 1000ull || wait_limit_ns > 1000000000ull) return KVB_EINVAL;
+    g_withhold_next.store(wait_limit_ns);
+    return KVB_OK;
+}
 
 const char* kvb_status_str(kvb_status s) {
     switch (s) {
@@ -227,6 +238,7 @@ kvb_status kvb_decode_attn(const kvb_attn_args* a, kvb_stream stream) {
     if (G != 1 && G != 2 && G != 4 && G != 8) return KVB_EINVAL;
     if (a->num_splits < 1 || a->num_splits > 1024 || a->split_len < 0) return KVB_EINVAL;
     if (a->B > 65535 || a->Hkv > 65535) return KVB_EINVAL;
+    if ((long long)a->B * a->Hq > 0x7fffffffLL) return KVB_EINVAL;   // rows of the merge and the outputs
     if (!std::isfinite(a->scale)) return KVB_EINVAL;
     if (!a->q || !a->k || !a->v || !a->len || !a->o) return KVB_EINVAL;
     if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v)) return KVB_EINVAL;
@@ -259,6 +271,15 @@ kvb_status kvb_decode_attn(const kvb_attn_args* a, kvb_stream stream) {
     p.o_part = a->o_part; p.lse_part = a->lse_part;
     p.o = a->o; p.o_bf16 = (a->o_dtype == KVB_OUT_BF16); p.lse = a->lse;
     p.cand = static_cast<kvb::EvictCand*>(a->evict_cand);
+    p.wait_ns = 1000000000ull;
+    p.withhold = 0;
+    if (g_withhold_next.load(std::memory_order_relaxed) != 0) {
+        const unsigned long long lim = g_withhold_next.exchange(0);
+        if (lim != 0) {
+            p.wait_ns = lim;
+            p.withhold = 1;
+        }
+    }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return a->d == 128 ? tc_g<128>(p, a, G, bias, st) : tc_g<64>(p, a, G, bias, st);
 }

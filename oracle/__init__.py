@@ -22,6 +22,9 @@ Parity status (what pins each function, see tests/test_oracle_*.py):
                    pinned n-way merge, chunked prefix build == SDPA over the
                    whole prefix, closed-form means, separated groups recovered
                    by the clustering, objective never decreasing
+  decode_steps_threads (parallel driver of evict_insert + decode_attn)
+                   pinned: bit-identical to the serial functions called step by
+                   step over the whole batch (victims, cache bytes, o, lse)
   asm_hier_lookup_merge
                    pinned: m = C over a partition == sklearn cosine_similarity
                    argmax; constructed indexes with known answers (best
@@ -51,7 +54,7 @@ def build(force: bool = False) -> str:
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + f".{os.getpid()}.tmp"
         subprocess.check_call(["g++", "-O2", "-std=c++17", "-fPIC", "-shared", "-ffp-contract=off",
-                               "-fno-fast-math", "-o", tmp, _SRC])
+                               "-fno-fast-math", "-pthread", "-o", tmp, _SRC])
         os.replace(tmp, _LIB)
     return _LIB
 
@@ -71,9 +74,10 @@ def _load():
         lib.oracle_asm_cosines.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _P]
         lib.oracle_asm_lookup_merge.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P]
         lib.oracle_asm_hier_lookup_merge.argtypes = [_P] * 9 + [_I] * 6 + [_P] * 4
+        lib.oracle_decode_steps_threads.argtypes = [_P] * 10 + [_I] * 8 + [_P] * 3
         for f in (lib.oracle_decode_attn, lib.oracle_merge_states, lib.oracle_evict_insert,
                   lib.oracle_compact_blocks, lib.oracle_asm_cosines, lib.oracle_asm_lookup_merge,
-                  lib.oracle_asm_hier_lookup_merge):
+                  lib.oracle_asm_hier_lookup_merge, lib.oracle_decode_steps_threads):
             f.restype = _I
         _lib = lib
     return _lib
@@ -162,6 +166,37 @@ def evict_insert(cache: dict, k_new, v_new, log_beta_new, t, M: int):
                                    _ptr(v_new), _ptr(log_beta_new), _ptr(t), B, Hkv, d, cap, int(M),
                                    _ptr(victim)), "oracle_evict_insert")
     return victim
+
+
+def decode_steps_threads(cache: dict, q, k_new, v_new, log_beta_new, t, M: int, nthreads: int = 0):
+    """`steps` decode steps (evict_insert, then decode_attn with one split) on a host cache dict,
+    in place, with the (sequence, kv head) units spread over `nthreads` threads (0 = all cores).
+
+    q [steps, B, Hq, d] or None (no attention); k_new, v_new [steps, B, Hkv, d] or None;
+    log_beta_new [steps, B, Hkv]; t [steps, B]. Each thread runs the serial functions on one
+    unit's slice, so the results equal evict_insert + decode_attn called step by step.
+    Returns (victim [steps, B, Hkv], o [B, Hq, d], lse [B, Hq]) -- o, lse of the last step,
+    None when q is None."""
+    lib = _load()
+    k, v, lb, pos, ln = cache["k"], cache["v"], cache.get("log_beta"), cache["pos"], cache["len"]
+    for a in (k, v, pos, ln) + ((lb,) if lb is not None else ()):
+        assert a.flags.c_contiguous
+    B, Hkv, cap, d = k.shape
+    t = _c(t, np.int32)
+    steps = t.shape[0]
+    q = _c(q, np.uint16)
+    Hq = q.shape[2] if q is not None else Hkv
+    k_new = _c(k_new, np.uint16)
+    v_new = _c(v_new, np.uint16)
+    log_beta_new = _c(log_beta_new, np.float32)
+    victim = np.zeros((steps, B, Hkv), np.int32)
+    o = np.zeros((B, Hq, d), np.float64) if q is not None else None
+    lse = np.zeros((B, Hq), np.float64) if q is not None else None
+    _check(lib.oracle_decode_steps_threads(_ptr(k), _ptr(v), _ptr(lb), _ptr(pos), _ptr(ln), _ptr(q), _ptr(k_new),
+                                           _ptr(v_new), _ptr(log_beta_new), _ptr(t), steps, B, Hq, Hkv, d, cap,
+                                           int(M), int(nthreads), _ptr(victim), _ptr(o), _ptr(lse)),
+           "oracle_decode_steps_threads")
+    return victim, o, lse
 
 
 def compact_blocks(cache: dict, rm_start, rm_len):

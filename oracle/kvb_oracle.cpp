@@ -43,6 +43,7 @@
 #include <cstdint>
 #include <cstring>
 #include <limits>
+#include <thread>
 #include <vector>
 
 namespace {
@@ -396,6 +397,73 @@ int oracle_asm_hier_lookup_merge(const uint16_t* q, const float* qhat, const int
             merge_two(a, &lse[nh], mem.data(), static_cast<double>(log_zbar[hk]), d);
         }
     }
+    return 0;
+}
+
+// ---- parallel driver ------------------------------------------------------
+// Runs `steps` decode steps -- budget enforcement + insertion
+// (oracle_evict_insert), then attention (oracle_decode_attn, one split) -- for
+// every (sequence b, kv head g) unit, spreading the units over `nthreads`
+// threads (0 = every host core). Units are independent: each thread calls the
+// single-threaded functions above, unchanged, on one unit's slice (B = 1,
+// Hkv = 1, the unit's G query heads), so the results are the ones a serial
+// call over the whole batch gives. Only the bench's CPU baseline and the
+// tests use it, to spread long replays over the host's cores.
+//   cache: k, v [B, Hkv, cap, d], log_beta (nullable), pos [B, Hkv, cap],
+//          len [B, Hkv], contiguous, updated in place
+//   per step s: q [steps, B, Hq, d] (null: no attention), k_new, v_new
+//          [steps, B, Hkv, d] (both null: only log_beta and pos are written),
+//          log_beta_new [steps, B, Hkv] (ignored when log_beta is null),
+//          t [steps, B]
+//   victim [steps, B, Hkv] (nullable); o [B, Hq, d], lse [B, Hq] (nullable):
+//          the last step's attention state
+// Returns the first nonzero status of any call (0 = ok).
+int oracle_decode_steps_threads(uint16_t* k, uint16_t* v, float* log_beta, int32_t* pos, int32_t* len,
+                                const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                                const float* log_beta_new, const int32_t* t, int steps, int B, int Hq,
+                                int Hkv, int d, int cap, int M, int nthreads, int32_t* victim, double* o,
+                                double* lse) {
+    if (steps < 0 || B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || cap <= 0) return 1;
+    if (q != nullptr && (o == nullptr || lse == nullptr)) return 1;
+    const int G = Hq / Hkv;
+    const int64_t units = static_cast<int64_t>(B) * Hkv;
+    int nt = nthreads > 0 ? nthreads : static_cast<int>(std::thread::hardware_concurrency());
+    if (nt < 1) nt = 1;
+    if (nt > units) nt = static_cast<int>(units > 0 ? units : 1);
+    std::vector<int> status(static_cast<size_t>(nt), 0);
+    auto work = [&](int w) {
+        for (int64_t u = w; u < units; u += nt) {
+            const int64_t b = u / Hkv, g = u % Hkv;
+            uint16_t* ku = k + u * cap * d;
+            uint16_t* vu = v + u * cap * d;
+            float* lbu = log_beta ? log_beta + u * cap : nullptr;
+            int32_t* pu = pos + u * cap;
+            int32_t* lu = len + u;
+            for (int s = 0; s < steps; ++s) {
+                const int64_t sb = static_cast<int64_t>(s) * B + b;   // (step, sequence)
+                const int64_t su = static_cast<int64_t>(s) * units + u;  // (step, unit)
+                int32_t vic = -1;
+                int st = oracle_evict_insert(ku, vu, lbu, pu, lu, k_new ? k_new + su * d : nullptr,
+                                             v_new ? v_new + su * d : nullptr,
+                                             log_beta_new ? log_beta_new + su : nullptr, t + sb, 1, 1, d, cap, M,
+                                             &vic);
+                if (victim != nullptr) victim[su] = vic;
+                if (st != 0 && status[w] == 0) status[w] = st;
+                if (q == nullptr) continue;
+                const uint16_t* qu = q + (sb * Hq + g * G) * d;
+                st = oracle_decode_attn(qu, static_cast<int64_t>(Hq) * d, d, ku, vu, static_cast<int64_t>(cap) * d,
+                                        static_cast<int64_t>(cap) * d, lbu, pu, cap, cap, lu, t + sb, 1, G, 1, d, cap,
+                                        0.0, 1, 0, o + (b * Hq + g * G) * d, lse + b * Hq + g * G, nullptr, nullptr);
+                if (st != 0 && status[w] == 0) status[w] = st;
+            }
+        }
+    };
+    std::vector<std::thread> pool;
+    for (int w = 1; w < nt; ++w) pool.emplace_back(work, w);
+    work(0);
+    for (auto& th : pool) th.join();
+    for (int st : status)
+        if (st != 0) return st;
     return 0;
 }
 

@@ -40,14 +40,12 @@ def run_gpu(q, k, v, lb, pos, ln, t, S=1, split_len=0, out_bf16=False, kv_shared
             lbd = lbd.expand(B, *lbd.shape[1:])
     o = torch.zeros(B, Hq, d, dtype=torch.bfloat16 if out_bf16 else torch.float32, device="cuda")
     lse = torch.zeros(B, Hq, dtype=torch.float32, device="cuda")
-    op = lp = cnt = None
+    op = lp = None
     if S > 1:
-        op, lp, cnt = kvb.decode_workspace(B, Hq, Hkv, d, S)
+        op, lp = kvb.decode_workspace(B, Hq, d, S)
     kvb.kvb_decode_attn(qd, kd, vd, lbd, posd, dev(ln), None if t is None else dev(t), o, lse, num_splits=S,
-                        split_len=split_len, o_part=op, lse_part=lp, counters=cnt)
+                        split_len=split_len, o_part=op, lse_part=lp)
     torch.cuda.synchronize()
-    if cnt is not None:
-        assert int(cnt.abs().sum()) == 0, "counters must be left at zero"
     res = dict(o=host(o.float()) if out_bf16 else host(o), lse=host(lse))
     if op is not None:
         res["o_part"], res["lse_part"] = host(op), host(lp)
@@ -126,17 +124,16 @@ def test_split_len_overflow_sets_device_error():
     assert np.all(res["lse"] == -np.inf)
 
 
-def test_repeated_calls_reuse_counters(oracle):
+def test_repeated_calls_reuse_workspace(oracle):
     q, k, v, lb, pos, ln, t = make_case(13, 2, 32, 8, 128, 256, [[256] * 8, [100] * 8])
     B, Hq, d = q.shape
     qd, kd, vd, lbd, posd, lnd, td = map(dev, (q, k, v, lb, pos, ln, t))
-    op, lp, cnt = kvb.decode_workspace(B, Hq, 8, d, 7)
+    op, lp = kvb.decode_workspace(B, Hq, d, 7)
     outs = []
     for _ in range(5):
         o = torch.empty(B, Hq, d, device="cuda")
         lse = torch.empty(B, Hq, device="cuda")
-        kvb.kvb_decode_attn(qd, kd, vd, lbd, posd, lnd, td, o, lse, num_splits=7, o_part=op, lse_part=lp,
-                            counters=cnt)
+        kvb.kvb_decode_attn(qd, kd, vd, lbd, posd, lnd, td, o, lse, num_splits=7, o_part=op, lse_part=lp)
         outs.append((host(o), host(lse)))
     for o, lse in outs[1:]:
         np.testing.assert_array_equal(o, outs[0][0])
@@ -158,5 +155,8 @@ def test_explicit_scale(oracle):
 def test_host_rejects_bad_layout():
     q, k, v, lb, pos, ln, t = make_case(15, 1, 4, 1, 64, 16, [[16]])
     o = torch.zeros(1, 4, 64, device="cuda")
-    with pytest.raises(kvb.KvbError):
+    with pytest.raises(ValueError):   # num_splits > 1 without split-state buffers
         kvb.kvb_decode_attn(dev(q), dev(k), dev(v), dev(lb), dev(pos), dev(ln), dev(t), o, num_splits=2)
+    with pytest.raises(kvb.KvbError):   # q not 16-byte aligned: refused by the library
+        qd = torch.empty(q.size + 8, dtype=torch.bfloat16, device="cuda")[1:1 + q.size].view(q.shape)
+        kvb.kvb_decode_attn(qd, dev(k), dev(v), dev(lb), dev(pos), dev(ln), dev(t), o)

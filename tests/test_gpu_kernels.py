@@ -7,6 +7,7 @@ import torch
 
 import memory_bounded_kv_b200 as kvb
 from memory_bounded_kv_b200.synth import normal_bf16, log_beta, rng
+from memory_bounded_kv_b200 import _lib
 from gpu_util import dev, host, GpuCache, assert_state_close
 
 pytestmark = pytest.mark.gpu
@@ -89,13 +90,16 @@ def test_attention_leaves_exact_eviction_candidates(oracle, S, with_beta):
     ln = np.array([[300, 257], [1, 64]], np.int32)
     t = np.full(B, 2 * cap + 1, np.int32)
     o = torch.zeros(B, Hq, d, device="cuda")
-    op, lp, _ = kvb.decode_workspace(B, Hq, Hkv, d, S)
+    op, lp = kvb.decode_workspace(B, Hq, d, S)
     cand = kvb.evict_candidates(B, Hkv, S)
     kvb.kvb_decode_attn(dev(q), dev(k), dev(v), None if lb is None else dev(lb), dev(pos), dev(ln), dev(t), o,
                         num_splits=S, o_part=op, lse_part=lp, evict_cand=cand)
     rec = host(cand).reshape(B, Hkv, S, 2)
     slots = (rec[..., 1] & 0xffffffff).astype(np.int64)
     slots = np.where(slots >= 2**31, slots - 2**32, slots)
+    # every record carries the position it was scored for
+    stamps = (rec[..., 1] >> 32).astype(np.int64)
+    assert np.all(stamps == (t + 1)[:, None, None])
     for b in range(B):
         for gg in range(Hkv):
             n = ln[b, gg]
@@ -111,6 +115,81 @@ def test_attention_leaves_exact_eviction_candidates(oracle, S, with_beta):
                 vic = oracle.evict_insert(sub, None, None, None if lb is None else np.zeros((1, 1), np.float32),
                                           np.array([t[b] + 1], np.int32), s1 - s0)
                 assert slots[b, gg, j] == s0 + vic[0, 0], (b, gg, j)
+
+
+def _crossing_cache(M, T0):
+    """A full cache whose victim at T0 + 1 is slot 3 and at T0 + 2 is slot 7: slot 3 (pos T0 - 10,
+    log beta -0.2) scores (T - pos) log beta = -2.2 then -2.4, slot 7 (pos T0 - 1, log beta -1)
+    -2.0 then -3.0; every other slot keeps log beta -1e-4."""
+    Hkv, d = 1, 64
+    g = rng(31, 0)
+    k, v = normal_bf16(g, (1, Hkv, M, d)), normal_bf16(g, (1, Hkv, M, d))
+    lb = np.full((1, Hkv, M), -1e-4, np.float32)
+    pos = np.arange(T0 - 2 * M, T0 - M, dtype=np.int32).reshape(1, 1, M).copy()
+    lb[0, 0, 3], pos[0, 0, 3] = -0.2, T0 - 10
+    lb[0, 0, 7], pos[0, 0, 7] = -1.0, T0 - 1
+    return dict(k=k, v=v, log_beta=lb, pos=pos, len=np.full((1, Hkv), M, np.int32))
+
+
+@pytest.mark.parametrize("skip", [1, 2])
+def test_evict_candidates_only_for_the_position_they_were_scored_for(oracle, skip):
+    """Attention at T0 leaves candidates for T0 + 1. Inserting at T0 + 1 uses them; inserting at
+    T0 + 2 (a skipped position) must not: the ranking changed, and the victim is the scan's."""
+    M, T0, S = 64, 1000, 4
+    c = _crossing_cache(M, T0)
+    gc = GpuCache(c["k"], c["v"], c["log_beta"], c["pos"], c["len"])
+    g = rng(32, skip)
+    q = normal_bf16(g, (1, 4, 64))
+    o = torch.zeros(1, 4, 64, device="cuda")
+    op, lp = kvb.decode_workspace(1, 4, 64, S)
+    cand = kvb.evict_candidates(1, 1, S)
+    kvb.kvb_decode_attn(dev(q), gc.k, gc.v, gc.log_beta, gc.pos, gc.len, dev(np.array([T0], np.int32)), o,
+                        num_splits=S, o_part=op, lse_part=lp, evict_cand=cand)
+    kn, vn, lbn = normal_bf16(g, (1, 1, 64)), normal_bf16(g, (1, 1, 64)), np.full((1, 1), -0.5, np.float32)
+    t_ins = np.array([T0 + skip], np.int32)
+    victim = torch.zeros(1, 1, dtype=torch.int32, device="cuda")
+    kvb.kvb_evict_insert(gc.k, gc.v, gc.log_beta, gc.pos, gc.len, dev(kn), dev(vn), dev(lbn), dev(t_ins), M,
+                         victim, cand=cand, cand_n=S)
+    want = oracle.evict_insert(c, kn, vn, lbn, t_ins, M)
+    assert int(want[0, 0]) == (3 if skip == 1 else 7)
+    np.testing.assert_array_equal(host(victim), want)
+    assert_cache_equal(gc, c)
+    assert kvb.kvb_get_error() == 0
+
+
+@pytest.mark.parametrize("S", [1, 3])
+def test_bounded_wait_runs_out_and_leaves_the_empty_state(oracle, S):
+    """The testing hook makes every producer withhold its copies, so each CTA's first bounded
+    wait on a tile runs out (after 20 us). The call returns, the device error word reports
+    KVB_DERR_TIMEOUT, every row is the empty state, the candidates name no slot, and the next
+    call on the same context is correct again."""
+    B, Hq, Hkv, d, cap = 2, 8, 2, 128, 200
+    g = rng(33, S)
+    q, k, v = normal_bf16(g, (B, Hq, d)), normal_bf16(g, (B, Hkv, cap, d)), normal_bf16(g, (B, Hkv, cap, d))
+    lb = log_beta(g, (B, Hkv, cap))
+    pos = np.tile(np.arange(cap, dtype=np.int32), (B, Hkv, 1))
+    ln = np.array([[200, 130], [77, 1]], np.int32)
+    t = np.full(B, cap + 2, np.int32)
+    args = [dev(x) for x in (q, k, v, lb, pos, ln, t)]
+    op = lp = None
+    if S > 1:
+        op, lp = kvb.decode_workspace(B, Hq, d, S)
+    cand = kvb.evict_candidates(B, Hkv, S)
+    kvb.kvb_get_error()
+    o = torch.full((B, Hq, d), 7.0, device="cuda")
+    lse = torch.full((B, Hq), 7.0, device="cuda")
+    kvb.kvb_test_withhold_next_decode(20_000)
+    kvb.kvb_decode_attn(*args, o, lse, num_splits=S, o_part=op, lse_part=lp, evict_cand=cand)
+    bits = kvb.kvb_get_error()
+    assert bits & _lib.DERR_TIMEOUT, bits
+    assert np.all(host(lse) == -np.inf) and not host(o).any()
+    rec = host(cand).reshape(B, Hkv, S, 2)
+    assert np.all((rec[..., 1] & 0xffffffff) == 0xffffffff)   # slot -1 everywhere
+    # the hook armed one launch only: the same call now matches the oracle
+    kvb.kvb_decode_attn(*args, o, lse, num_splits=S, o_part=op, lse_part=lp, evict_cand=cand)
+    assert kvb.kvb_get_error() == 0
+    o_ref, l_ref = oracle.decode_attn(q, k, v, lb, pos, ln, t)
+    assert_state_close(host(o), host(lse), o_ref, l_ref, "after the timeout")
 
 
 def test_evict_insert_bad_length_flags_error():

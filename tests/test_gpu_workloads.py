@@ -4,11 +4,13 @@ merge fused), against the oracle on the same seeded inputs.
 
 1 tiny retention decode      every one of 512 steps, S = 1 and S = 4: victims, whole cache, o, lse
 2 Qwen3-8B-shaped layer      victims + len every step; o, lse, whole cache at sampled steps
-3 long context (131072/8192) streaming build of log beta/pos (two kv heads replayed by the oracle),
-                             then 64 steps with 64 splits: victims every step, final and per-split
-                             states at sampled steps; plain (beta = 1) variant
+3 long context (131072/8192) streaming build of log beta/pos (every kv head of every sequence
+                             replayed by the oracle: pos and log beta bit-exact), then 64 steps with
+                             64 splits: victims every step, final and per-split states at sampled
+                             steps; plain (beta = 1) variant
 4 attention-state memory     all 256 x 32 indices (near-tie rule) and merged states
-5 memento compaction         the full batch of 64 on the GPU; sequences 0-3 replayed by the oracle
+5 memento compaction         all 64 sequences replayed by the oracle: every compaction's lengths
+                             and bytes exact; attention states on a sample
 """
 import numpy as np
 import pytest
@@ -100,22 +102,20 @@ def test_long_context_stream_and_decode(oracle):
     cache = BoundedKVCache.from_host(w.k, w.v, w.log_beta, w.pos, w.len, w.Hq, w.M, num_splits=S)
     blocks = long_context_build(w, cache)
     torch.cuda.synchronize()
-    # the oracle replays the stream for kv heads 0 and 5 of sequence 2
-    sel = [(2, 0), (2, 5)]
-    sub = dict(k=np.zeros((1, 2, w.cap, 8), np.uint16), v=np.zeros((1, 2, w.cap, 8), np.uint16),
-               log_beta=np.stack([w.log_beta[b, g] for b, g in sel])[None].copy(),
-               pos=np.stack([w.pos[b, g] for b, g in sel])[None].copy(), len=np.full((1, 2), w.cap, np.int32))
+    # the oracle replays the stream for every (sequence, kv head), the heads spread over the host's
+    # cores by its parallel driver (the serial functions on each head's slice)
+    sub = dict(k=np.zeros((w.B, w.Hkv, w.cap, 8), np.uint16), v=np.zeros((w.B, w.Hkv, w.cap, 8), np.uint16),
+               log_beta=w.log_beta.copy(), pos=w.pos.copy(), len=np.full((w.B, w.Hkv), w.cap, np.int32))
     for blk in range(blocks):
         lbs = synth.stream_log_beta(w, blk)
         base = w.cap + blk * synth.STREAM_BLOCK
-        for i in range(synth.STREAM_BLOCK):
-            lb = np.array([[lbs[i, b, g] for b, g in sel]], np.float32)
-            oracle.evict_insert(sub, None, None, lb, np.array([base + i], np.int32), w.M)
+        ts = np.repeat((base + np.arange(synth.STREAM_BLOCK, dtype=np.int32))[:, None], w.B, axis=1)
+        oracle.decode_steps_threads(sub, None, None, None, lbs, ts, w.M)
     gpos, glb = host(cache.pos), host(cache.log_beta)
-    for j, (b, g) in enumerate(sel):
-        np.testing.assert_array_equal(gpos[b, g], sub["pos"][0, j])
-        np.testing.assert_array_equal(glb[b, g], sub["log_beta"][0, j])
-    # every head: full, unique positions below the logical length
+    np.testing.assert_array_equal(host(cache.len), sub["len"])
+    np.testing.assert_array_equal(gpos, sub["pos"])
+    np.testing.assert_array_equal(glb, sub["log_beta"])
+    # and the invariants: every head full, unique positions below the logical length
     assert np.all(host(cache.len) == w.M)
     assert np.all(gpos < synth.CONFIG3_LOGICAL_T) and all(
         len(np.unique(gpos[b, g])) == w.M for b in range(w.B) for g in range(w.Hkv))
@@ -153,9 +153,9 @@ def test_memory_lookup_workload_full(oracle):
     posd = dev(w.pos).expand(N, Hkv, w.L)
     o_self = torch.zeros(N, H, d, device="cuda")
     l_self = torch.zeros(N, H, device="cuda")
-    op, lp, cnt = kvb.decode_workspace(N, H, Hkv, d, 4)
+    op, lp = kvb.decode_workspace(N, H, d, 4)
     kvb.kvb_decode_attn(dev(w.q), kd, vd, None, posd, dev(w.len), dev(w.t), o_self, l_self, num_splits=4,
-                        o_part=op, lse_part=lp, counters=cnt)
+                        o_part=op, lse_part=lp)
     os_ref, ls_ref = oracle.decode_attn(w.q, w.k, w.v, None, w.pos, w.len, w.t, kv_batch_stride=0,
                                         meta_batch_stride=0)
     assert_state_close(host(o_self), host(l_self), os_ref, ls_ref, "self attention")
@@ -170,25 +170,44 @@ def test_memory_lookup_workload_full(oracle):
 
 
 def test_memento_compaction_workload(oracle):
+    """Scope: the oracle replays every one of the 64 sequences (append at every step, removal at
+    every memento end). At every compaction step the lengths of all 64 sequences are compared,
+    and the K, V and pos bytes of every sequence compacted at that step, over its whole length;
+    the whole batch's bytes at eight spread compaction steps and at the end. Attention states
+    are compared on a sample: sequences 0, 1, 31, 63 around their compactions and at 20 random
+    steps, plus every sequence at 4 of those steps."""
     w = synth.memento_workload()
     SPLIT_LEN = 512
     S = -(-w.cap // SPLIT_LEN)
     cache = BoundedKVCache(w.B, w.Hq, w.Hkv, w.d, w.cap, w.cap, num_splits=S, split_len=SPLIT_LEN, with_beta=False)
-    nsub = 4
-    c = dict(k=np.zeros((nsub, w.Hkv, w.cap, w.d), np.uint16), v=np.zeros((nsub, w.Hkv, w.cap, w.d), np.uint16),
-             log_beta=None, pos=np.zeros((nsub, w.Hkv, w.cap), np.int32), len=np.zeros((nsub, w.Hkv), np.int32))
+    c = dict(k=np.zeros((w.B, w.Hkv, w.cap, w.d), np.uint16), v=np.zeros((w.B, w.Hkv, w.cap, w.d), np.uint16),
+             log_beta=None, pos=np.zeros((w.B, w.Hkv, w.cap), np.int32), len=np.zeros((w.B, w.Hkv), np.int32))
     o = torch.zeros(w.B, w.Hq, w.d, device="cuda")
     lse = torch.zeros(w.B, w.Hq, device="cuda")
     ends = np.cumsum(w.blk + w.mem, axis=1) - 1
+    watch = [0, 1, 31, 63]
     check_steps = set()
-    for b in range(2):
+    for b in watch:
         for e in ends[b]:
             check_steps.update({int(e) - 1, int(e), int(e) + 1})
-    check_steps.update(np.random.default_rng(5).integers(0, w.steps, 20).tolist())
-    comp_steps = set(w.compaction_steps().tolist())
+    rand_steps = np.random.default_rng(5).integers(0, w.steps, 20).tolist()
+    check_steps.update(rand_steps)
+    full_attn_steps = set(rand_steps[:4])
+    comp_list = w.compaction_steps().tolist()
+    comp_steps = set(comp_list)
+    full_cache_steps = set(comp_list[:: max(1, len(comp_list) // 8)])
     pool = [w.step_inputs(s) for s in range(w.pool)]
     pool_dev = [{key: dev(val) for key, val in inp.items() if key != "t"} for inp in pool]
-    n_checked = 0
+
+    def compare_seq(b, what):
+        n = int(c["len"][b].max())
+        for key, t in (("k", cache.k), ("v", cache.v), ("pos", cache.pos)):
+            h = host(t[b, :, :n])
+            for g in range(w.Hkv):
+                m = c["len"][b, g]
+                np.testing.assert_array_equal(h[g, :m], c[key][b, g, :m], err_msg=f"{what} {key} b{b} g{g}")
+
+    n_checked = n_compared = 0
     for step in range(w.steps):
         inp = pool[step % w.pool]
         t = np.where(step < w.total, step, -1).astype(np.int32)
@@ -196,18 +215,27 @@ def test_memento_compaction_workload(oracle):
         pd = pool_dev[step % w.pool]
         cache.insert(pd["k_new"], pd["v_new"], None, td)
         cache.attend(pd["q"], td, o, lse)
-        oracle.evict_insert(c, inp["k_new"][:nsub], inp["v_new"][:nsub], None, t[:nsub], w.cap)
+        oracle.evict_insert(c, inp["k_new"], inp["v_new"], None, t, w.cap)
         if step in check_steps:
-            o_ref, l_ref = oracle.decode_attn(inp["q"][:nsub], c["k"], c["v"], None, c["pos"], c["len"], t[:nsub])
-            assert_state_close(host(o[:nsub]), host(lse[:nsub]), o_ref, l_ref, f"step {step}")
+            sel = slice(None) if step in full_attn_steps else watch   # a slice: no copy of the whole cache
+            o_ref, l_ref = oracle.decode_attn(inp["q"][sel], c["k"][sel], c["v"][sel], None, c["pos"][sel],
+                                              c["len"][sel], t[sel])
+            assert_state_close(host(o[sel]), host(lse[sel]), o_ref, l_ref, f"step {step}")
             n_checked += 1
         if step in comp_steps:
             rs, rl = w.compaction(step)
             cache.compact(dev(rs), dev(rl))
-            oracle.compact_blocks(c, rs[:nsub], rl[:nsub])
-            if rl[:2].any():
-                compare_cache(cache, c, f"compaction at {step}", b_max=2)
+            oracle.compact_blocks(c, rs, rl)
+            np.testing.assert_array_equal(host(cache.len), c["len"], err_msg=f"len after compaction at {step}")
+            for b in np.nonzero(rl)[0]:
+                compare_seq(int(b), f"compaction at {step}")
+                n_compared += 1
+            if step in full_cache_steps:
+                for b in range(w.B):
+                    compare_seq(b, f"whole batch at {step}")
     assert n_checked >= 40
-    np.testing.assert_array_equal(host(cache.len)[:nsub], c["len"])
+    assert n_compared == int((w.blk > 0).sum())   # every block removal was compared
+    for b in range(w.B):
+        compare_seq(b, "end")
     # finished sequences hold exactly their mementos
     np.testing.assert_array_equal(host(cache.len)[:, 0], w.mem.sum(axis=1))
