@@ -1,27 +1,37 @@
 #!/usr/bin/env python
 """Benchmark of the memory-bounded KV decode step on B200.
 
-Default workload: the Qwen3-8B-shaped layer decode step (B=32, Hq=32, Hkv=8,
+Headline workload: the Qwen3-8B-shaped layer decode step (B=32, Hq=32, Hkv=8,
 d=128, budget M=4096 slots per kv head, beta = sigmoid(N(2, 1.5))). A step is
 one decode token per sequence: budget enforcement + insertion
 (kvb_evict_insert), then split-K retention-gated attention, with the merge of
 the split states launched by the same call when there are several
-(kvb_decode_attn). --config selects the workload:
-  1  tiny decode step (B=1, Hq=8, Hkv=2, d=64, M=256)
-  2  the Qwen3-8B-shaped layer above (default)
-  3  long context: B=4, Hq=32, Hkv=8, d=128, 131072 positions kept in 8192 slots, 64 splits
-  4  attention-state memory: 256 query tokens x 32 heads, self attention over a shared
-     2048-token cache, then the lookup + merge against 4096 entries per head
-  5  memento compaction: B=64 sawtooth caches, 9 x (Geom(1500) block + U[120,180] memento)
+(kvb_decode_attn). The other workloads are measured in the same run and
+reported under "configs" on the same JSON line:
+  1   tiny decode step (B=1, Hq=8, Hkv=2, d=64, M=256)
+  2   the Qwen3-8B-shaped layer above (the headline)
+  3   long context: B=4, Hq=32, Hkv=8, d=128, 131072 positions kept in 8192 slots, 64 splits
+  3p  the same with beta = 1 (no log beta; eviction is first-in first-out)
+  4   attention-state memory: 256 query tokens x 32 heads, self attention over a shared
+      2048-token cache, then the lookup + merge against 4096 entries per head
+  5   memento compaction: B=64 sawtooth caches, 9 x (Geom(1500) block + U[120,180] memento)
+  5p  the same on the paged cache (pages of 64 slots from one pool sized to the schedule's peak)
 
 Prints ONE JSON line (rank 0). `value` is tokens/s of the whole job (one
 attention layer) with inputs resident in HBM; `e2e` is the same metric through
-the public API with the step's inputs copied from pinned host memory and the
-output read back every step. The default workload reads > 126 MB (L2) of K/V
-per step, so no L2 flush is needed; workloads that fit in L2 are timed step by
-step after a flush (the JSON line's config says which).
+the public API with every step's inputs copied from pinned host memory (one
+packed copy) and its outputs read back (one copy), each step replayed from a
+CUDA graph. Workloads whose step reads more than the 126 MB L2 are timed as
+graphs of many steps; the others step by step, each step after a 256 MiB
+write that flushes L2 (outside the events). The roofline of the dominant
+launch comes from events around that launch's own graph in a second region.
+After timing, one more step is computed two ways on the GPU (the timed path and
+an independent one: full eviction scan, other split counts, the per-row kernel)
+and compared ("consistency"); parity with the CPU oracle is the tests' job.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1..5] [--impl kvb|reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1|2|3|4|5] [--plain] [--paged]
+                  [--configs all|none|LIST] [--seed S] [--check sampled|full|off]
+                  [--impl kvb|reference]
   python bench.py --asm-crossover | --asm-build     (lookup and build measurements, 1 GPU)
 
 For N > 1 launch with torch.distributed.run: every rank runs an independent
@@ -34,6 +44,7 @@ import argparse
 import hashlib
 import json
 import os
+import platform
 import statistics
 import subprocess
 import sys
@@ -49,26 +60,33 @@ METRIC = "decode-attn tokens/s and KV-cache GB/s (% of B200 HBM peak) at budget 
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 L2_BYTES = 126 * 1000 * 1000      # B200 L2 (126 MB)
+WORKLOADS = ("1", "2", "3", "3p", "4", "5", "5p")
 
 # ncu DRAM traffic (read + write bytes per launch) of the dominant kernel, keyed by
-# (sha256 of the kernel's source file, config, num_splits). Reported only while the source is
+# (sha256 of the kernel's source file, workload, num_splits). Reported only while the source is
 # unchanged since the counters were taken.
 MEASURED_TRAFFIC = {
-    # decode_attn_tc_kernel<128,4,1>, Qwen3-8B-shaped layer, S=1: 545,628,416 read + 3,972,608 written
-    ("f9553bcebbe325aa", 2, 1): 549601024,
 }
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--plain", action="store_true", help="beta = 1 variant of the long-context workload")
+    ap.add_argument("--configs", default="all",
+                    help="other workloads measured in the same run and reported under 'configs': 'all', "
+                         "'none' or a comma list of " + ",".join(WORKLOADS))
+    ap.add_argument("--seed", type=int, default=None, help="replace the workloads' own seeds")
+    ap.add_argument("--paged", action="store_true", help="paged-cache variant of the memento workload")
+    ap.add_argument("--check", default="sampled", choices=["sampled", "full", "off"],
+                    help="after timing, one more step computed two ways on the GPU (the timed path and an "
+                         "independent one) and compared (sampled: cache bytes of a few sequences; full: all)")
     ap.add_argument("--impl", default="kvb", choices=["kvb", "reference"])
-    ap.add_argument("--splits", type=int, default=0, help="num_splits (0: the workload's default)")
+    ap.add_argument("--splits", type=int, default=0, help="num_splits of the headline workload (0: its default)")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-graph", action="store_true", help="launch the timed steps one by one")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--asm-build", action="store_true",
                     help="time the offline memory build (cosine Lloyd iteration, aggregation) instead of a "
@@ -76,7 +94,7 @@ def parse():
     ap.add_argument("--asm-crossover", action="store_true",
                     help="time the linear and the two-level memory lookups alone over query counts and memory "
                          "sizes (one GPU; L2 flushed between iterations) instead of a decode step")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 # ----------------------------------------------------------------------------------------------
@@ -117,24 +135,45 @@ def replica_value(units_per_rank: float, world: int, ms_max: float) -> float:
     return units_per_rank * world / (ms_max / 1e3)
 
 
-def peaks():
+def _peaks_file():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         with open(path) as f:
-            p = json.load(f)
+            return json.load(f)
+    return None
+
+
+def peaks():
+    p = _peaks_file()
+    if p is not None and "hbm_gbs" in p:
         return float(p["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
 
 
 def bf16_peak():
     """Dense bf16 tensor TFLOP/s for a kernel timed alone (burst figure), and where it comes from."""
-    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(path):
-        with open(path) as f:
-            p = json.load(f)
-        if "bf16_tflops" in p:
-            return float(p["bf16_tflops"]), "measured"
+    p = _peaks_file()
+    if p is not None and "bf16_tflops" in p:
+        return float(p["bf16_tflops"]), "measured"
     return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
 
 
 class ClockSampler:
@@ -190,153 +229,13 @@ def kernel_src_hash(name: str = "decode_attn_tc.cuh") -> str:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-# ----------------------------------------------------------------------------------------------
-# decode workloads (tiny, Qwen3-8B-shaped, long context): evict+insert, then attention
-# ----------------------------------------------------------------------------------------------
-
-class DecodeBench:
-    def __init__(self, cfg: int, splits: int, rank: int):
-        from memory_bounded_kv_b200 import synth
-        from memory_bounded_kv_b200.cache import BoundedKVCache
-        import memory_bounded_kv_b200 as kvb
-        self.cfg = cfg
-        self.w = w = synth.decode_workload(cfg)
-        self.S = splits or w.splits[-1]
-        self.cache = BoundedKVCache.from_host(w.k, w.v, w.log_beta, w.pos, w.len, w.Hq, w.M, num_splits=self.S)
-        if cfg == 3:   # stream positions cap .. 131071 through budget enforcement, then draw survivors' K/V
-            blocks = (synth.CONFIG3_LOGICAL_T - w.cap) // synth.STREAM_BLOCK
-            for blk in range(blocks):
-                lbs = torch.from_numpy(synth.stream_log_beta(w, blk)).cuda()
-                base = w.cap + blk * synth.STREAM_BLOCK
-                ts = torch.arange(base, base + synth.STREAM_BLOCK, dtype=torch.int32, device="cuda")
-                ts = ts[:, None].expand(-1, w.B).contiguous()
-                for i in range(synth.STREAM_BLOCK):
-                    kvb.kvb_evict_insert(self.cache.k, self.cache.v, self.cache.log_beta, self.cache.pos,
-                                         self.cache.len, None, None, lbs[i], ts[i], w.M)
-            k, v = synth.long_context_kv(w)
-            self.cache.k.copy_(torch.from_numpy(k.view(np.int16)).view(torch.bfloat16).cuda())
-            self.cache.v.copy_(torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).cuda())
-            torch.cuda.synchronize()
-        self.pool = min(w.steps, 1024)
-        inp = [w.step_inputs(s) for s in range(self.pool)]
-
-        def stack(key, dt):
-            a = np.stack([x[key] for x in inp])
-            t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
-            return t.view(dt) if a.dtype == np.uint16 else t
-
-        self.h_q = stack("q", torch.bfloat16).pin_memory()
-        self.h_kn = stack("k_new", torch.bfloat16).pin_memory()
-        self.h_vn = stack("v_new", torch.bfloat16).pin_memory()
-        self.h_lb = stack("log_beta_new", torch.float32).pin_memory()
-        self.d_q, self.d_kn, self.d_vn, self.d_lb = (x.cuda() for x in (self.h_q, self.h_kn, self.h_vn, self.h_lb))
-        self.o = torch.zeros(w.B, w.Hq, w.d, device="cuda")
-        self.lse = torch.zeros(w.B, w.Hq, device="cuda")
-        self.tokens_per_step = w.B
-        self.launches_per_step = 2 + (self.S > 1)   # evict/insert, attention (+ split merge)
-        self.workload = w.name
-
-    def t_of(self, i: int):
-        return self.w.t0 + i
-
-    def run_device(self, first: int, count: int, events=None):
-        """Steps first .. first+count-1 with inputs resident in HBM."""
-        c, t_all = self.cache, self.t_dev
-        for i in range(first, first + count):
-            p = i % self.pool
-            t = t_all[i]
-            c.insert(self.d_kn[p], self.d_vn[p], self.d_lb[p], t)
-            if events is not None:
-                events[i - first][0].record()
-            c.attend(self.d_q[p], t, self.o, self.lse)
-            if events is not None:
-                events[i - first][1].record()
-
-    def prepare(self, total_steps: int):
-        self.t_dev = torch.tensor([[self.t_of(i)] * self.w.B for i in range(total_steps)], dtype=torch.int32,
-                                  device="cuda")
-        self.h_t = self.t_dev.cpu().pin_memory()
-        self.s_q = torch.empty_like(self.d_q[0])
-        self.s_kn = torch.empty_like(self.d_kn[0])
-        self.s_vn = torch.empty_like(self.d_vn[0])
-        self.s_lb = torch.empty_like(self.d_lb[0])
-        self.s_t = torch.empty_like(self.t_dev[0])
-        self.h_o = torch.empty(self.o.shape, dtype=torch.float32).pin_memory()
-        self.h_lse = torch.empty(self.lse.shape, dtype=torch.float32).pin_memory()
-
-    def run_e2e(self, first: int, count: int):
-        """Steps through the public API from pinned host buffers; output read back every step."""
-        c = self.cache
-        for i in range(first, first + count):
-            p = i % self.pool
-            self.s_q.copy_(self.h_q[p], non_blocking=True)
-            self.s_kn.copy_(self.h_kn[p], non_blocking=True)
-            self.s_vn.copy_(self.h_vn[p], non_blocking=True)
-            self.s_lb.copy_(self.h_lb[p], non_blocking=True)
-            self.s_t.copy_(self.h_t[i], non_blocking=True)
-            c.step(self.s_q, self.s_kn, self.s_vn, self.s_lb, self.s_t, self.o, self.lse)
-            self.h_o.copy_(self.o, non_blocking=True)
-            self.h_lse.copy_(self.lse, non_blocking=True)
-
-    def e2e_bytes(self):
-        h2d = sum(x[0].numel() * x.element_size() for x in (self.h_q, self.h_kn, self.h_vn, self.h_lb))
-        h2d += self.w.B * 4
-        d2h = self.o.numel() * 4 + self.lse.numel() * 4
-        return h2d, d2h
-
-    def attn_bytes(self):
-        """Algorithmic bytes of one attention launch: K, V (+ log beta, pos) of the cached slots,
-        q, len, t in; o (fp32), lse out."""
-        w = self.w
-        n = int(self.cache.len.sum().item())
-        per_slot = 2 * w.d * 2 + 8
-        return n * per_slot + w.B * w.Hq * w.d * 2 + w.B * w.Hkv * 4 + w.B * 4 + w.B * w.Hq * (w.d * 4 + 4)
-
-    def evict_bytes(self):
-        """Budget enforcement reads the attention's per-split candidates (16 B each) and writes the
-        new row; the scan of log beta/pos happens inside the attention pass."""
-        w = self.w
-        return w.B * w.Hkv * (self.S * 16 + 2 * w.d * 2 + 4 + 4 + 4)
-
-    def kernel_name(self):
-        merge = " + merge_splits_kernel" if self.S > 1 else ""
-        return (f"kvb_decode_attn = decode_attn_tc_kernel<d={self.w.d},G={self.w.Hq // self.w.Hkv},bias=1>"
-                f"{merge}, S={self.S}")
-
-    def flush_l2(self):
-        return self.attn_bytes() < L2_BYTES
-
-    def config(self):
-        w = self.w
-        l2 = (f"flushed before every timed step (256 MiB write): a step reads {self.attn_bytes() / 1e6:.2f} MB"
-              if self.flush_l2() else
-              f"no flush: every step reads {self.attn_bytes() / 1e6:.0f} MB of K/V (inputs larger than L2)")
-        return {"workload": self.workload, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "budget_M": w.M,
-                "num_splits": self.S, "beta": "sigmoid(N(2,1.5))", "l2": l2,
-                "parallelism": "replicas (independent sequences per GPU)"}
-
-    def oracle_sample(self, budget_s: float = 15.0):
-        """The oracle as it stands on whole-batch decode steps from the prefill state; returns
-        (tokens/s, description)."""
-        import oracle
-        w = self.w
-        c = dict(k=w.k.copy(), v=w.v.copy(), log_beta=w.log_beta.copy(), pos=w.pos.copy(), len=w.len.copy())
-        t0 = time.perf_counter()
-        steps = 0
-        while True:
-            x = w.step_inputs(steps)
-            oracle.evict_insert(c, x["k_new"], x["v_new"], x["log_beta_new"], x["t"], w.M)
-            oracle.decode_attn(x["q"], c["k"], c["v"], c["log_beta"], c["pos"], c["len"], x["t"])
-            steps += 1
-            if time.perf_counter() - t0 > budget_s or steps >= 64:
-                break
-        dt = time.perf_counter() - t0
-        return w.B * steps / dt, f"{steps} whole-batch decode steps (B={w.B}) from the prefill state"
+_T0 = time.perf_counter()
 
 
-# ----------------------------------------------------------------------------------------------
-# attention-state-memory workload: self attention + lookup/merge per step
-# ----------------------------------------------------------------------------------------------
+def log(msg: str):
+    """Progress on stderr (the JSON line alone goes to stdout)."""
+    print(f"[bench {time.perf_counter() - _T0:7.1f}s] {msg}", file=sys.stderr, flush=True)
+
 
 def _dev(a):
     a = np.ascontiguousarray(a)
@@ -345,201 +244,565 @@ def _dev(a):
     return torch.from_numpy(a).cuda()
 
 
+def _np(t: torch.Tensor) -> np.ndarray:
+    t = t.detach().cpu()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16).copy()
+    return t.numpy().copy()
+
+
+class Packed:
+    """One device buffer holding several tensors (each at a 256-byte aligned offset), so that a
+    step's inputs arrive with one host-to-device copy and its outputs leave with one copy."""
+
+    def __init__(self, layout):
+        self.offsets, off = {}, 0
+        for name, shape, dt in layout:
+            n = int(np.prod(shape)) * torch.empty((), dtype=dt).element_size()
+            self.offsets[name] = (off, n, tuple(shape), dt)
+            off = (off + n + 255) // 256 * 256
+        self.nbytes = off
+        self.payload = sum(v[1] for v in self.offsets.values())
+        self.dev = torch.zeros(self.nbytes, dtype=torch.uint8, device="cuda")
+        self.views = {k: self.dev[o:o + n].view(dt).view(shape) for k, (o, n, shape, dt) in self.offsets.items()}
+
+    def fill_host(self, row: torch.Tensor, arrays: dict):
+        """Write numpy arrays into a host uint8 row laid out like the device buffer."""
+        for k, a in arrays.items():
+            o, n, _, _ = self.offsets[k]
+            row[o:o + n] = torch.from_numpy(np.ascontiguousarray(a).view(np.uint8).reshape(-1))
+
+
+def capture(fn):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
+def _consistency(exact: dict, o, lse, o_ref, l_ref, what: str, dev_err: int) -> dict:
+    """Two GPU computations of the same step: fields in `exact` compared bit for bit; o within
+    max-abs 2e-2 and rel-L2 1e-3; lse within max(1e-4, 2^-22 |lse|) (the tolerances of the parity
+    tests, which compare with the CPU oracle)."""
+    ok = dev_err == 0
+    res = {"checked": what, "device_error_bits": int(dev_err)}
+    for k, (a, b) in exact.items():
+        same = bool(np.array_equal(a, b))
+        res[f"{k}_exact"] = same
+        ok &= same
+    o = np.asarray(o, np.float64)
+    err = np.abs(o - o_ref)
+    nref = float(np.linalg.norm(o_ref))
+    rel = float(np.linalg.norm(o - o_ref) / nref) if nref > 0 else float(np.linalg.norm(o))
+    fin = ~np.isneginf(l_ref)
+    same_inf = bool(np.array_equal(np.isneginf(lse), ~fin))
+    dl = np.abs(np.asarray(lse, np.float64)[fin] - l_ref[fin])
+    tol = np.maximum(1e-4, 2.0 ** -22 * np.abs(l_ref[fin]))
+    res.update(max_abs=float(err.max()) if err.size else 0.0, rel_l2=rel,
+               lse_max_abs=float(dl.max()) if dl.size else 0.0)
+    ok &= res["max_abs"] <= 2e-2 and rel <= 1e-3 and same_inf and bool(np.all(dl <= tol))
+    res["ok"] = bool(ok)
+    return res
+
+
+# ----------------------------------------------------------------------------------------------
+# workloads. Each one enqueues step i on the current stream in three parts: pre (budget
+# enforcement + insertion, or the self attention), attn (the dominant launch), post (compaction)
+# ----------------------------------------------------------------------------------------------
+
+class DecodeBench:
+    """Decode workloads 1 (tiny), 2 (Qwen3-8B-shaped) and 3 (long context), and 3's beta = 1 variant."""
+
+    bound = "hbm"
+    KERNEL_SRC = "decode_attn_tc.cuh"
+
+    def __init__(self, cfg: int, splits: int, seed=None, plain: bool = False):
+        import memory_bounded_kv_b200 as kvb
+        from memory_bounded_kv_b200 import synth
+        from memory_bounded_kv_b200.cache import BoundedKVCache
+        self.cfg, self.plain = cfg, plain
+        self.key = f"{cfg}{'p' if plain else ''}"
+        self.w = w = synth.decode_workload(cfg, seed=seed)
+        self.S = splits or w.splits[-1]
+        if cfg == 3:
+            self.cache = BoundedKVCache(w.B, w.Hq, w.Hkv, w.d, w.cap, w.M, num_splits=self.S, with_beta=not plain)
+            if plain:   # first-in first-out keeps exactly the last M positions of the stream
+                pos = np.broadcast_to(np.arange(synth.CONFIG3_LOGICAL_T - w.M, synth.CONFIG3_LOGICAL_T,
+                                                dtype=np.int32), (w.B, w.Hkv, w.M))
+                self.cache.pos.copy_(_dev(pos.copy()))
+                self.cache.len.fill_(w.M)
+            else:
+                self.cache.log_beta.copy_(_dev(w.log_beta))
+                self.cache.pos.copy_(_dev(w.pos))
+                self.cache.len.copy_(_dev(w.len))
+                self._stream_build(kvb, synth)
+            k, v = synth.long_context_kv(w)
+            self.cache.k.copy_(_dev(k))
+            self.cache.v.copy_(_dev(v))
+            torch.cuda.synchronize()
+        else:
+            self.cache = BoundedKVCache.from_host(w.k, w.v, None if plain else w.log_beta, w.pos, w.len, w.Hq, w.M,
+                                                  num_splits=self.S)
+        self.pool = min(w.steps, 1024)
+        self.inp = [w.step_inputs(s) for s in range(self.pool)]
+
+        def stack(key):
+            return _dev(np.stack([x[key] for x in self.inp]))
+
+        self.d_q, self.d_kn, self.d_vn, self.d_lb = stack("q"), stack("k_new"), stack("v_new"), stack("log_beta_new")
+        layout = [("q", (w.B, w.Hq, w.d), torch.bfloat16), ("k_new", (w.B, w.Hkv, w.d), torch.bfloat16),
+                  ("v_new", (w.B, w.Hkv, w.d), torch.bfloat16), ("t", (w.B,), torch.int32)]
+        if not plain:
+            layout.append(("log_beta_new", (w.B, w.Hkv), torch.float32))
+        self.stage = Packed(layout)
+        self.out = Packed([("o", (w.B, w.Hq, w.d), torch.float32), ("lse", (w.B, w.Hq), torch.float32)])
+        self.o, self.lse = self.out.views["o"], self.out.views["lse"]
+        self.workload = w.name + (" beta=1" if plain else "")
+        self.flush_l2 = self.attn_bytes() < L2_BYTES
+
+    def _stream_build(self, kvb, synth):
+        """Stream positions cap .. 131071 through budget enforcement (log beta and pos only): one
+        block of 4096 insertions captured as a CUDA graph, replayed per block with its log beta."""
+        w, c = self.w, self.cache
+        lbs = torch.empty(synth.STREAM_BLOCK, w.B, w.Hkv, device="cuda")
+        ts = torch.empty(synth.STREAM_BLOCK, w.B, dtype=torch.int32, device="cuda")
+
+        def block():
+            for i in range(synth.STREAM_BLOCK):
+                kvb.kvb_evict_insert(c.k, c.v, c.log_beta, c.pos, c.len, None, None, lbs[i], ts[i], w.M)
+
+        blocks = (synth.CONFIG3_LOGICAL_T - w.cap) // synth.STREAM_BLOCK
+        g = None
+        for blk in range(blocks):
+            lbs.copy_(torch.from_numpy(synth.stream_log_beta(w, blk)))
+            base = w.cap + blk * synth.STREAM_BLOCK
+            ts.copy_(torch.arange(base, base + synth.STREAM_BLOCK, dtype=torch.int32)[:, None].expand(-1, w.B))
+            if g is None:
+                torch.cuda.synchronize()
+                g = capture(block)
+            g.replay()
+        torch.cuda.synchronize()
+        del g
+
+    def prepare(self, total_steps: int):
+        self.t_dev = (self.w.t0 + torch.arange(total_steps, dtype=torch.int32, device="cuda"))[:, None].expand(
+            -1, self.w.B).contiguous()
+
+    def n_steps(self):
+        return None   # positions continue past the workload's own step count
+
+    def _in(self, i, x):
+        if x is not None:
+            return x["q"], x["k_new"], x["v_new"], x.get("log_beta_new"), x["t"]
+        p = i % self.pool
+        return self.d_q[p], self.d_kn[p], self.d_vn[p], None if self.plain else self.d_lb[p], self.t_dev[i]
+
+    def pre(self, i, x=None):
+        _, kn, vn, lb, t = self._in(i, x)
+        self.cache.insert(kn, vn, lb, t)
+
+    def attn(self, i, x=None):
+        q, _, _, _, t = self._in(i, x)
+        self.cache.attend(q, t, self.o, self.lse)
+
+    def post(self, i, x=None):
+        pass
+
+    def host_inputs(self, i):
+        x = self.inp[i % self.pool]
+        out = dict(q=x["q"], k_new=x["k_new"], v_new=x["v_new"], t=np.full(self.w.B, self.w.t0 + i, np.int32))
+        if not self.plain:
+            out["log_beta_new"] = x["log_beta_new"]
+        return out
+
+    def tokens(self, i):
+        return self.w.B
+
+    def launches(self, i):
+        return 2 + (self.S > 1)   # evict/insert, attention (+ split merge)
+
+    def attn_bytes(self, i=None):
+        """Algorithmic bytes of one attention launch: K, V (+ log beta) and pos of the cached slots
+        (pos feeds the eviction candidates), q, len, t in; o (fp32), lse out."""
+        w = self.w
+        n = w.B * w.Hkv * w.M        # every (b, g) holds M slots in these workloads
+        per_slot = 2 * w.d * 2 + 4 + (0 if self.plain else 4)
+        return n * per_slot + w.B * w.Hq * w.d * 2 + w.B * w.Hkv * 4 + w.B * 4 + w.B * w.Hq * (w.d * 4 + 4)
+
+    def other_bytes(self, i=None):
+        """Budget enforcement reads the attention's per-split candidates (16 B each) and writes the
+        new row; the scan of log beta/pos happens inside the attention pass."""
+        w = self.w
+        return w.B * w.Hkv * (self.S * 16 + 2 * w.d * 2 + 4 + 4 + 4)
+
+    def kernel_name(self):
+        merge = " + merge_splits_kernel" if self.S > 1 else ""
+        return (f"kvb_decode_attn = decode_attn_tc_kernel<d={self.w.d},G={self.w.Hq // self.w.Hkv},"
+                f"bias={0 if self.plain else 1}>{merge}, S={self.S}")
+
+    def config(self):
+        w = self.w
+        l2 = (f"flushed before every timed step (256 MiB write): a step reads {self.attn_bytes() / 1e6:.2f} MB"
+              if self.flush_l2 else
+              f"no flush: every step reads {self.attn_bytes() / 1e6:.0f} MB of K/V (inputs larger than L2)")
+        return {"workload": self.workload, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "budget_M": w.M,
+                "num_splits": self.S, "beta": "1" if self.plain else "sigmoid(N(2,1.5))", "seed": w.seed,
+                "l2": l2, "parallelism": "replicas (independent sequences per GPU)"}
+
+    def check(self, i, full: bool):
+        """Consistency of one more step (position t0 + i) computed two ways on the GPU from the same
+        cache: the timed path (eviction from the attention's candidates, the workload's splits) and
+        a copy of the cache stepped through the full eviction scan and another split count."""
+        from memory_bounded_kv_b200 import kvb_get_error
+        from memory_bounded_kv_b200.cache import BoundedKVCache
+        w, c = self.w, self.cache
+        torch.cuda.synchronize()
+        S2 = 4 if self.S == 1 else 1
+        c2 = BoundedKVCache(w.B, w.Hq, w.Hkv, w.d, w.cap, w.M, num_splits=S2, with_beta=not self.plain)
+        for name in ("k", "v", "pos", "len") + (() if self.plain else ("log_beta",)):
+            getattr(c2, name).copy_(getattr(c, name))
+        o2, l2 = torch.zeros_like(self.o), torch.zeros_like(self.lse)
+        q, kn, vn, lb, t = self._in(i, None)
+        self.pre(i)
+        self.attn(i)
+        c2.insert(kn, vn, lb, t)          # no candidates: the scan
+        c2.attend(q, t, o2, l2)
+        torch.cuda.synchronize()
+        sel = list(range(w.B)) if full else sorted({0, w.B - 1})
+        exact = dict(victims=(_np(c.victim), _np(c2.victim)), len=(_np(c.len), _np(c2.len)),
+                     pos=(_np(c.pos[sel]), _np(c2.pos[sel])), k=(_np(c.k[sel]), _np(c2.k[sel])))
+        return _consistency(exact, _np(self.o), _np(self.lse), _np(o2), _np(l2),
+                            f"one step at t={w.t0 + i}: candidates + {self.S} split(s) against the full scan + "
+                            f"{S2} split(s); cache bytes of sequences {'all' if full else sel}", kvb_get_error())
+
+    def oracle_sample(self, oracle, nthreads: int, budget_s: float):
+        """The oracle as it stands on whole-batch decode steps from the prefill state, the
+        (sequence, kv head) units spread over `nthreads` threads; returns (tokens/s, steps)."""
+        w = self.w
+        c = dict(k=w.k.copy(), v=w.v.copy(), log_beta=None if self.plain else w.log_beta.copy(), pos=w.pos.copy(),
+                 len=w.len.copy())
+        t0 = time.perf_counter()
+        steps = 0
+        while True:
+            x = w.step_inputs(steps)
+            oracle.decode_steps_threads(c, x["q"][None], x["k_new"][None], x["v_new"][None],
+                                        None if self.plain else x["log_beta_new"][None], x["t"][None], w.M, nthreads)
+            steps += 1
+            if time.perf_counter() - t0 > budget_s or steps >= 64:
+                break
+        return w.B * steps / (time.perf_counter() - t0), steps
+
+
 class ASMBench:
     """A step: the 256 query tokens' causal self attention over the shared 2048-token cache
-    (kvb_decode_attn, batch stride 0) and the memory lookup + merge (kvb_asm_lookup_merge)."""
+    (kvb_decode_attn, batch stride 0: the query-batched kernel) and the memory lookup + merge over
+    the memory prepared once at set-up (kvb_asm_prepare, then kvb_asm_lookup_merge_planes)."""
 
-    KERNEL_SRC = "asm_lookup.cuh"
-
-    def flush_l2(self):
-        return True
-
+    bound = "tensor"
+    KERNEL_SRC = "asm_planes.cuh"
+    flush_l2 = True
     # the fp32 contraction runs as three exact bf16 products per element (q . hi + q . mid + q . lo)
     PEAK_NOTE = "{kind} dense bf16 {bf16:.0f} TFLOP/s (bf16_tflops, burst) / 3 bf16 products per fp32 product"
 
-    def __init__(self, splits: int = 0):
+    SPLIT_LEN = 512   # the self attention's splits: a fixed length shared by every query row
+
+    def __init__(self, splits: int = 0, seed=None):
         import memory_bounded_kv_b200 as kvb
         from memory_bounded_kv_b200 import synth
         self.kvb = kvb
-        self.w = w = synth.asm_workload()
+        self.key = "4"
+        self.w = w = synth.asm_workload(seed=4 if seed is None else seed)
         self.S = splits or 4
         N, H, Hkv, d = w.N, w.H, w.Hkv, w.d
         self.k = _dev(w.k).expand(N, Hkv, w.L, d)
         self.v = _dev(w.v).expand(N, Hkv, w.L, d)
         self.pos = _dev(w.pos).expand(N, Hkv, w.L)
         self.len, self.t = _dev(w.len), _dev(w.t)
-        self.h_q = torch.from_numpy(w.q.view(np.int16)).view(torch.bfloat16).pin_memory()
-        self.q = self.h_q.cuda()
+        self.q = _dev(w.q)
         self.qbar, self.abar, self.lz = _dev(w.qbar), _dev(w.abar), _dev(w.log_zbar)
         self.o_self = torch.zeros(N, H, d, device="cuda")
         self.l_self = torch.zeros(N, H, device="cuda")
         self.op, self.lp = kvb.decode_workspace(N, H, d, self.S)
-        self.idx = torch.zeros(N, H, dtype=torch.int32, device="cuda")
-        self.o = torch.zeros(N, H, d, device="cuda")
-        self.lse = torch.zeros(N, H, device="cuda")
+        self.out = Packed([("o", (N, H, d), torch.float32), ("lse", (N, H), torch.float32),
+                           ("idx", (N, H), torch.int32)])
+        self.o, self.lse, self.idx = self.out.views["o"], self.out.views["lse"], self.out.views["idx"]
+        self.stage = Packed([("q", (N, H, d), torch.bfloat16)])
         self.ws = torch.empty(kvb.kvb_asm_workspace_bytes(N, H, w.K), dtype=torch.uint8, device="cuda")
-        self.tokens_per_step = N
-        self.launches_per_step = 4   # attention + split merge, lookup + state merge
-        self.workload = "attention-state memory H32 K4096 d128, 256 queries, self attention over 2048"
+        self.planes = kvb.kvb_asm_prepare(self.qbar)   # the memory is static: prepared once, untimed
+        self.workload = f"attention-state memory H{H} K{w.K} d{d}, {N} queries, self attention over {w.L}"
 
     def prepare(self, total_steps):
-        self.s_q = torch.empty_like(self.q)
-        self.h_o = torch.empty(self.o.shape, dtype=torch.float32).pin_memory()
-        self.h_idx = torch.empty(self.idx.shape, dtype=torch.int32).pin_memory()
+        pass
 
-    def _step(self, q, events=None, j=0):
-        kvb = self.kvb
-        kvb.kvb_decode_attn(q, self.k, self.v, None, self.pos, self.len, self.t, self.o_self, self.l_self,
-                            num_splits=self.S, o_part=self.op, lse_part=self.lp)
-        if events is not None:
-            events[j][0].record()
-        kvb.kvb_asm_lookup_merge(q, self.qbar, self.abar, self.lz, self.o_self, self.l_self, self.idx, self.o,
-                                 self.lse, self.ws)
-        if events is not None:
-            events[j][1].record()
+    def n_steps(self):
+        return None
 
-    def run_device(self, first, count, events=None):
-        for j in range(count):
-            self._step(self.q, events, j)
+    def pre(self, i, x=None):
+        q = self.q if x is None else x["q"]
+        self.kvb.kvb_decode_attn(q, self.k, self.v, None, self.pos, self.len, self.t, self.o_self, self.l_self,
+                                 num_splits=self.S, split_len=self.SPLIT_LEN, o_part=self.op, lse_part=self.lp)
 
-    def run_e2e(self, first, count):
-        for _ in range(count):
-            self.s_q.copy_(self.h_q, non_blocking=True)
-            self._step(self.s_q)
-            self.h_o.copy_(self.o, non_blocking=True)
-            self.h_idx.copy_(self.idx, non_blocking=True)
-
-    def e2e_bytes(self):
-        return self.h_q.numel() * 2, self.o.numel() * 4 + self.idx.numel() * 4
-
-    def attn_bytes(self):
-        return 0
-
-    def evict_bytes(self):
+    def attn(self, i, x=None):   # the dominant launch: the lookup + merge
+        q = self.q if x is None else x["q"]
         w = self.w
-        kv = int(w.len.sum()) * w.d * 2 * 2
-        return kv + w.H * w.K * w.d * 4
+        self.kvb.kvb_asm_lookup_merge_planes(q, self.planes, w.H, w.K, self.abar, self.lz, self.o_self, self.l_self,
+                                             self.idx, self.o, self.lse, self.ws)
+
+    def post(self, i, x=None):
+        pass
+
+    def host_inputs(self, i):
+        return {"q": self.w.q}
+
+    def tokens(self, i):
+        return self.w.N
+
+    def launches(self, i):
+        return 4   # attention + split merge, lookup + state merge
+
+    def attn_bytes(self, i=None):
+        """The lookup reads every prepared centroid (three bf16 parts) once and per query its q,
+        o_self and ā, and writes o."""
+        w = self.w
+        return w.H * w.K * w.d * 6 + w.N * w.H * (w.d * 2 + w.d * 4 * 2 + w.d * 2)
+
+    def other_bytes(self, i=None):
+        """The self attention reads the shared cache's K and V once, and q."""
+        w = self.w
+        return w.L * w.Hkv * w.d * 2 * 2 + w.N * w.H * w.d * 2
 
     def flops(self):
         w = self.w
         return 2.0 * w.N * w.H * w.K * w.d
 
     def kernel_name(self):
-        return "asm_score_umma_kernel + asm_merge_kernel (kvb_asm_lookup_merge)"
+        return "asm_score_planes_kernel + asm_merge_kernel (kvb_asm_lookup_merge_planes)"
 
     def config(self):
         w = self.w
         return {"workload": self.workload, "N": w.N, "H": w.H, "Hkv": w.Hkv, "K": w.K, "d": w.d, "L": w.L,
-                "self_attn_splits": self.S,
+                "self_attn_splits": self.S, "seed": w.seed,
                 "l2": "flushed before every timed step (256 MiB write): q̄ 64 MiB + ā 32 MiB + K/V 8 MiB fit in L2",
                 "parallelism": "replicas"}
 
+    def check(self, i, full: bool):
+        """Consistency of the step computed two ways on the GPU: the self attention through the
+        query-batched kernel (the timed path) and through the per-row kernel (splits of
+        ceil(len / 4) slots); the lookup over the prepared memory (the timed path) and over the
+        fp32 centroids (indices compared exactly)."""
+        from memory_bounded_kv_b200 import kvb_get_error
+        w = self.w
+        self.pre(i)
+        self.attn(i)
+        o_self2, l_self2 = torch.zeros_like(self.o_self), torch.zeros_like(self.l_self)
+        self.kvb.kvb_decode_attn(self.q, self.k, self.v, None, self.pos, self.len, self.t, o_self2, l_self2,
+                                 num_splits=self.S, split_len=0, o_part=self.op, lse_part=self.lp)
+        idx2 = torch.zeros_like(self.idx)
+        o2, l2 = torch.zeros_like(self.o), torch.zeros_like(self.lse)
+        # the lookup over the fp32 centroids (normalised and split on the fly)
+        self.kvb.kvb_asm_lookup_merge(self.q, self.qbar, self.abar, self.lz, o_self2, l_self2, idx2, o2, l2, self.ws)
+        torch.cuda.synchronize()
+        self_par = _consistency({}, _np(self.o_self), _np(self.l_self), _np(o_self2), _np(l_self2), "self attention", 0)
+        res = _consistency(dict(idx=(_np(self.idx), _np(idx2))), _np(self.o), _np(self.lse), _np(o2), _np(l2),
+                           "query-batched self attention against the per-row kernel, then the lookup + merge of "
+                           "each", kvb_get_error())
+        res["self_attention"] = {k: self_par[k] for k in ("max_abs", "rel_l2", "lse_max_abs", "ok")}
+        res["ok"] = res["ok"] and self_par["ok"]
+        return res
 
-# ----------------------------------------------------------------------------------------------
-# memento-style block compaction (sawtooth cache)
-# ----------------------------------------------------------------------------------------------
 
 class MementoBench:
-    """A step: every active sequence decodes one token (append, attention); after the last
-    token of a memento, the finished block's slots are removed in place (kvb_compact_blocks)."""
+    """A step: every active sequence decodes one token (append, attention); after the last token
+    of a memento, the finished block's slots are removed in place (kvb_compact_blocks). The
+    schedule is finite: timed steps are a spread sample of it, the others run untimed."""
 
+    bound = "hbm"
+    KERNEL_SRC = "decode_attn_tc.cuh"
+    flush_l2 = True
     SPLIT_LEN = 512
 
-    def __init__(self, splits: int = 0):
-        from memory_bounded_kv_b200 import synth
-        from memory_bounded_kv_b200.cache import BoundedKVCache
-        self.w = w = synth.memento_workload()
+    def __init__(self, splits: int = 0, seed=None, paged: bool = False):
+        from memory_bounded_kv_b200 import synth, _lib
+        from memory_bounded_kv_b200.cache import BoundedKVCache, PagedKVCache
+        self.paged = paged
+        self.key = "5p" if paged else "5"
+        self.w = w = synth.memento_workload(seed=5 if seed is None else seed)
         self.S = -(-w.cap // self.SPLIT_LEN)
-        self.cache = BoundedKVCache(w.B, w.Hq, w.Hkv, w.d, w.cap, w.cap, num_splits=self.S,
-                                    split_len=self.SPLIT_LEN, with_beta=False)
-        pool = [w.step_inputs(s) for s in range(w.pool)]
-        self.q = [_dev(x["q"]) for x in pool]
-        self.kn = [_dev(x["k_new"]) for x in pool]
-        self.vn = [_dev(x["v_new"]) for x in pool]
-        self.o = torch.zeros(w.B, w.Hq, w.d, device="cuda")
-        self.lse = torch.zeros(w.B, w.Hq, device="cuda")
+        if paged:
+            self.page = _lib.PAGE_SLOTS
+            self.num_pages = w.peak_pages(self.page)
+            self.cache = PagedKVCache(w.B, w.Hq, w.Hkv, w.d, max_pages=-(-w.cap // self.page),
+                                      num_pages=self.num_pages, M=w.cap, num_splits=self.S,
+                                      split_len=self.SPLIT_LEN, with_beta=False)
+        else:
+            self.cache = BoundedKVCache(w.B, w.Hq, w.Hkv, w.d, w.cap, w.cap, num_splits=self.S,
+                                        split_len=self.SPLIT_LEN, with_beta=False)
+        self.pool_in = [w.step_inputs(s) for s in range(w.pool)]
+        self.q = [_dev(x["q"]) for x in self.pool_in]
+        self.kn = [_dev(x["k_new"]) for x in self.pool_in]
+        self.vn = [_dev(x["v_new"]) for x in self.pool_in]
+        self.out = Packed([("o", (w.B, w.Hq, w.d), torch.float32), ("lse", (w.B, w.Hq), torch.float32)])
+        self.o, self.lse = self.out.views["o"], self.out.views["lse"]
+        self.stage = Packed([("q", (w.B, w.Hq, w.d), torch.bfloat16), ("k_new", (w.B, w.Hkv, w.d), torch.bfloat16),
+                             ("v_new", (w.B, w.Hkv, w.d), torch.bfloat16), ("t", (w.B,), torch.int32),
+                             ("rm_start", (w.B,), torch.int32), ("rm_len", (w.B,), torch.int32)])
         self.comp = {}
         for s in w.compaction_steps().tolist():
-            rs, rl = w.compaction(s)
-            self.comp[s] = (_dev(rs), _dev(rl))
+            self.comp[s] = tuple(_dev(a) for a in w.compaction(s))
         self.active = np.array([(s < w.total).sum() for s in range(w.steps)], np.int64)
-        self.lens = None
-        self.tokens_per_step = None
-        self.launches_per_step = None
-        self.workload = "memento compaction B64 Hq32 Hkv8 d128, 9 x (Geom(1500) block + U[120,180] memento)"
-
-    def flush_l2(self):
-        return True
-
-    def clamp_steps(self, K, W, KR):
-        n = self.w.steps
-        W = min(W, n // 8)
-        KR = min(KR, n // 8)
-        K = min(K, n - W - KR) if K > 0 else n - W - KR
-        return K, W, KR
+        steps = np.arange(w.steps)
+        self.t_np = np.where(steps[:, None] < w.total[None, :], steps[:, None], -1).astype(np.int32)
+        self.t_dev = torch.from_numpy(self.t_np).cuda()
+        self._lens = {}
+        self.workload = (f"memento compaction B{w.B} Hq{w.Hq} Hkv{w.Hkv} d{w.d}, 9 x (Geom(1500) block + "
+                         f"U[120,180] memento){', paged cache' if paged else ''}")
 
     def prepare(self, total_steps):
+        pass
+
+    def n_steps(self):
+        return self.w.steps
+
+    def reset(self):
+        if self.paged:
+            self.cache.reset()
+        else:
+            self.cache.len.zero_()
+        self.cache.cand_valid = False
+
+    def pre(self, i, x=None):
+        p = i % self.w.pool
+        kn, vn, t = (self.kn[p], self.vn[p], self.t_dev[i]) if x is None else (x["k_new"], x["v_new"], x["t"])
+        self.cache.cand_valid = False   # the cache never reaches its budget: insertion appends
+        self.cache.insert(kn, vn, None, t)
+
+    def attn(self, i, x=None):
+        p = i % self.w.pool
+        q, t = (self.q[p], self.t_dev[i]) if x is None else (x["q"], x["t"])
+        self.cache.attend(q, t, self.o, self.lse)
+
+    def post(self, i, x=None):
+        if i in self.comp:
+            rs, rl = self.comp[i] if x is None else (x["rm_start"], x["rm_len"])
+            self.cache.compact(rs, rl)
+
+    def host_inputs(self, i):
+        x = self.pool_in[i % self.w.pool]
+        rs, rl = self.w.compaction(i) if i in self.comp else (np.zeros(self.w.B, np.int32),) * 2
+        return dict(q=x["q"], k_new=x["k_new"], v_new=x["v_new"], t=self.t_np[i], rm_start=rs, rm_len=rl)
+
+    def tokens(self, i):
+        return int(self.active[i])
+
+    def launches(self, i):
+        return 2 + (self.S > 1) + (1 if i in self.comp else 0)
+
+    def _len(self, i):
+        if i not in self._lens:
+            self._lens[i] = self.w.cache_len(i)
+        return self._lens[i]
+
+    def attn_bytes(self, i=None):
+        """K, V and pos of the live slots of step i (pos feeds the eviction candidates), q in,
+        o and lse out for the active sequences."""
         w = self.w
-        steps = np.arange(w.steps)
-        self.t_dev = torch.from_numpy(np.where(steps[:, None] < w.total[None, :], steps[:, None], -1)
-                                      .astype(np.int32)).cuda()
+        n = int(self._len(i)[i < w.total].sum())
+        act = int(self.active[i])
+        return n * w.Hkv * (2 * w.d * 2 + 4) + act * w.Hq * w.d * 2 + act * w.Hq * (w.d * 4 + 4)
 
-    def run_device(self, first, count, events=None):
-        c, w = self.cache, self.w
-        for j, i in enumerate(range(first, min(first + count, w.steps))):
-            p = i % w.pool
-            t = self.t_dev[i]
-            c.insert(self.kn[p], self.vn[p], None, t)
-            if events is not None:
-                events[j][0].record()
-            c.attend(self.q[p], t, self.o, self.lse)
-            if events is not None:
-                events[j][1].record()
-            if i in self.comp:
-                c.compact(*self.comp[i])
-
-    def tokens(self, first, count):
-        return int(self.active[first:first + count].sum())
-
-    def launches(self, first, count):
-        per = 2 + (self.S > 1)
-        return per * count + sum(1 for i in range(first, first + count) if i in self.comp)
-
-    def mean_kv_bytes(self, first, count):
+    def other_bytes(self, i=None):
+        """The appended rows, and at a compaction step the moved rows (read and written)."""
         w = self.w
-        tot = 0
-        for i in range(first, first + count):
-            tot += int(w.cache_len(i)[i < w.total].sum())
-        return tot * w.Hkv * (2 * w.d * 2) / count
+        moved = 0
+        if i in self.comp:
+            rs, rl = w.compaction(i)
+            ln = self._len(i)
+            for b in np.nonzero(rl)[0]:
+                moved += int(ln[b]) - int(rs[b]) - int(rl[b])
+        return int(self.active[i]) * w.Hkv * (2 * w.d * 2 + 4) + moved * w.Hkv * 2 * (2 * w.d * 2 + 4)
+
+    def kernel_name(self):
+        entry, paged = ("kvb_paged_decode_attn", ",paged") if self.paged else ("kvb_decode_attn", "")
+        return (f"{entry} = decode_attn_tc_kernel<d={self.w.d},G={self.w.Hq // self.w.Hkv},bias=0{paged}> + "
+                f"merge_splits_kernel, split_len={self.SPLIT_LEN}")
+
+    def peak_kv_ratio(self):
+        """Peak KV slots of a cache that keeps every token over the compacted cache's peak."""
+        w = self.w
+        prev = np.concatenate([np.zeros((w.B, 1), np.int64), np.cumsum(w.mem, axis=1)[:, :-1]], axis=1)
+        return int(w.total.max()) / int((prev + w.blk + w.mem).max())
+
+    def memory(self):
+        """Device bytes of K, V and pos: the flat cache reserves cap slots per (sequence, kv head); the
+        paged pool holds the schedule's peak page count."""
+        w = self.w
+        row = 2 * w.d * 2 + 4
+        flat = w.B * w.Hkv * w.cap * row
+        out = {"flat_reserved_bytes": flat}
+        if self.paged:
+            out.update(pool_pages=self.num_pages, pool_bytes=self.num_pages * self.page * row,
+                       flat_over_paged=round(flat / (self.num_pages * self.page * row), 3))
+        return out
 
     def config(self):
         w = self.w
         return {"workload": self.workload, "B": w.B, "cap": w.cap, "split_len": self.SPLIT_LEN,
-                "num_splits": self.S, "schedule_steps": w.steps, "parallelism": "replicas",
+                "num_splits": self.S, "schedule_steps": w.steps, "seed": w.seed, "parallelism": "replicas",
+                "timed_steps": "a spread sample of the schedule (every other step runs untimed, in order)",
+                "peak_kv_full_over_compacted": round(self.peak_kv_ratio(), 3), "memory": self.memory(),
                 "l2": "flushed before every timed step (256 MiB write): the live caches grow from "
-                      "a few MB to ~350 MB over the timed steps"}
+                      "a few MB to ~350 MB over the schedule"}
+
+    def check(self, i, full: bool):
+        """Consistency of schedule step i: the timed path (eviction candidates, splits of 512
+        slots) against the same step on a copy of the cache with one split."""
+        from memory_bounded_kv_b200 import kvb_get_error
+        c = self.cache
+        torch.cuda.synchronize()
+        o2, l2 = torch.zeros_like(self.o), torch.zeros_like(self.lse)
+        p = i % self.w.pool
+        self.pre(i)
+        self.attn(i)
+        if self.paged:
+            from memory_bounded_kv_b200 import kvb_paged_decode_attn
+            kvb_paged_decode_attn(c.pool, self.q[p], self.t_dev[i], o2, l2, num_splits=1)
+        else:
+            from memory_bounded_kv_b200 import kvb_decode_attn
+            kvb_decode_attn(self.q[p], c.k, c.v, None, c.pos, c.len, self.t_dev[i], o2, l2, num_splits=1)
+        self.post(i)
+        torch.cuda.synchronize()
+        return _consistency({}, _np(self.o), _np(self.lse), _np(o2), _np(l2),
+                            f"schedule step {i}: {self.S} splits of {self.SPLIT_LEN} slots against one split",
+                            kvb_get_error())
+
+
+def make_bench(key: str, splits: int, seed):
+    if key in ("1", "2", "3", "3p"):
+        return DecodeBench(int(key[0]), splits, seed, plain=key.endswith("p"))
+    if key == "4":
+        return ASMBench(splits, seed)
+    return MementoBench(splits, seed, paged=key.endswith("p"))
 
 
 # ----------------------------------------------------------------------------------------------
 # timing driver
 # ----------------------------------------------------------------------------------------------
 
-def time_flushed_steps(steps, flush, world):
-    """Device time of the steps, each started with a cold L2 (flush written before it, outside
-    its events): the sum of the per-step event times, after a barrier on both sides."""
-    if world > 1:
-        torch.distributed.barrier()
+def time_graphs(graphs, flush, world):
+    """Per-graph device times (ms): each replay bracketed by events, after a 256 MiB write that
+    flushes L2 (outside the events) when `flush` is given."""
+    barrier(world)
     torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in steps]
-    for (a, b), step in zip(ev, steps):
-        flush.fill_(1)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in graphs]
+    for (a, b), g in zip(ev, graphs):
+        if flush is not None:
+            flush.fill_(1)
         a.record()
-        step()
+        g.replay()
         b.record()
     torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    return sum(a.elapsed_time(b) for a, b in ev)
+    barrier(world)
+    return [a.elapsed_time(b) for a, b in ev]
 
 
 def time_region(fn, world):
@@ -555,130 +818,272 @@ def time_region(fn, world):
     return e0.elapsed_time(e1)
 
 
-def run_kvb(args, world, rank, local):
-    hbm_peak, peak_kind = peaks()
-    if args.config in (1, 2, 3):
-        bench = DecodeBench(args.config, args.splits, rank)
-    elif args.config == 4:
-        bench = ASMBench(args.splits)
-    else:
-        bench = MementoBench(args.splits)
-    K, W = args.steps, args.warmup
-    KR = min(K, 500)                               # steps of the kernel-timing region
-    if hasattr(bench, "clamp_steps"):              # the memento schedule is finite
-        K, W, KR = bench.clamp_steps(K, W, KR)
-    bench.prepare(2 * (W + K) + KR + 2)
+def pct(xs):
+    a = np.asarray(xs, np.float64)
+    return {"p10": float(np.percentile(a, 10)), "p50": float(np.percentile(a, 50)),
+            "p90": float(np.percentile(a, 90)), "n": int(a.size)}
 
-    # warm-up; the timed region (the K steps captured once as a CUDA graph -- every launch of
-    # every step with the programmatic dependencies between them -- and replayed; no events
-    # inside); then a region of KR steps with CUDA events around the dominant launch
-    bench.run_device(0, W)
-    torch.cuda.synchronize()
-    # a workload whose step touches less than L2 holds is timed step by step with a cold L2:
-    # each step is its own CUDA graph, replayed after a 256 MiB write, with events around the
-    # replay only (the flush is not timed); otherwise the K steps are one graph
-    flush_l2 = bench.flush_l2() if hasattr(bench, "flush_l2") else False
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if flush_l2 else None
-    graph, step_graphs = None, None
-    if not args.no_graph:
-        if flush_l2:
-            step_graphs = []
-            for i in range(K):
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g):
-                    bench.run_device(W + i, 1)
-                step_graphs.append(g)
+
+def measure(bench, K, W, world, e2e: bool):
+    """Times one workload: the main region (inputs resident in HBM), a region with events around
+    the dominant launch's own graph, per-step times, and the e2e region (inputs from pinned host
+    memory, outputs read back). Returns the times and which steps each region ran."""
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if bench.flush_l2 else None
+    n = bench.n_steps()
+    KR = min(K, 200)
+    E = min(K, 200)
+    P = 0 if bench.flush_l2 else min(K, 200)
+
+    def full_step(i, x=None):
+        bench.pre(i, x)
+        bench.attn(i, x)
+        bench.post(i, x)
+
+    if n is None:
+        # positions continue: warm-up, main, kernel, per-step, e2e warm-up and e2e regions follow
+        # one another; `nxt` is the first position no region used
+        bounds = np.cumsum([0, W, K, KR, P, E, E])
+        main, kern, per_step, warm_e2e, e2e_steps = (list(range(bounds[j], bounds[j + 1])) for j in range(1, 6))
+        nxt = int(bounds[-1])
+        bench.prepare(nxt + 1)
+        for i in range(W):
+            full_step(i)
+        torch.cuda.synchronize()
+    else:
+        # a finite schedule: a spread sample of its steps is timed in each pass, the rest run untimed
+        stride = max(1, n // K)
+        main = list(range(stride // 2, n, stride))[:K]
+        kern, e2e_steps, warm_e2e, per_step = main[:KR], main[:E], [], []
+        nxt = main[len(main) // 2]
+
+    def schedule_pass(timed: dict):
+        """Runs the whole schedule from an empty cache; at the steps in `timed` calls their timer."""
+        log(f"{bench.key}: schedule pass of {n} steps")
+        bench.reset()
+        torch.cuda.synchronize()
+        for i in range(n):
+            if i in timed:
+                timed[i]()
+            else:
+                full_step(i)
+        torch.cuda.synchronize()
+
+    # ---- main region: device-resident inputs
+    log(f"{bench.key}: main region ({len(main)} steps)")
+    step_ms = None
+    if n is None:
+        if bench.flush_l2:
+            graphs = [capture(lambda i=i: full_step(i)) for i in main]
+            step_ms = time_graphs(graphs, flush, world)
+            ms = sum(step_ms)
         else:
-            graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(graph):
-                bench.run_device(W, K)
-    clocks = ClockSampler(local)
-    clocks.start()
-    if step_graphs is not None:
-        ms = time_flushed_steps([g.replay for g in step_graphs], flush, world)
-    elif flush_l2:
-        ms = time_flushed_steps([lambda i=i: bench.run_device(W + i, 1) for i in range(K)], flush, world)
-    elif graph is not None:
-        ms = time_region(graph.replay, world)
+            chunk = 500
+            graphs = [capture(lambda c=main[j:j + chunk]: [full_step(i) for i in c])
+                      for j in range(0, len(main), chunk)]
+            ms = time_region(lambda: [g.replay() for g in graphs], world)
+        del graphs
     else:
-        ms = time_region(lambda: bench.run_device(W, K), world)
-    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(KR)]
-    if flush_l2:
-        def kernel_region():
-            for j in range(KR):
-                flush.fill_(1)
-                bench.run_device(W + K + j, 1, events[j:j + 1])
-        time_region(kernel_region, world)
+        graphs = {i: capture(lambda i=i: full_step(i)) for i in main}
+        step_ms = []
+        barrier(world)
+        schedule_pass({i: (lambda g=graphs[i]: step_ms.extend(time_graphs([g], flush, 1))) for i in main})
+        barrier(world)
+        ms = sum(step_ms)
+        del graphs
+
+    # ---- kernel region: the dominant launch in its own graph, events around it
+    log(f"{bench.key}: kernel region ({len(kern)} launches)")
+    parts = {}
+    for i in kern:   # captured in step order, so each step sees the cache bookkeeping of the one before
+        parts[i] = (capture(lambda i=i: bench.pre(i)), capture(lambda i=i: bench.attn(i)),
+                    capture(lambda i=i: bench.post(i)))
+    kern_ms = []
+
+    def kernel_step(i):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if flush is not None:
+            flush.fill_(1)
+        parts[i][0].replay()
+        a.record()
+        parts[i][1].replay()
+        b.record()
+        parts[i][2].replay()
+        kern_ev.append((a, b))
+
+    kern_ev = []
+    barrier(world)
+    if n is None:
+        torch.cuda.synchronize()
+        for i in kern:
+            kernel_step(i)
+        torch.cuda.synchronize()
     else:
-        time_region(lambda: bench.run_device(W + K, KR, events), world)
-    clk = clocks.stop()
-    del step_graphs
-    kern_ms = [a.elapsed_time(b) for a, b in events]
-    ms = max_over_ranks(ms, world)
-    kms = max_over_ranks(statistics.mean(kern_ms), world)
-    tokens = bench.tokens(W, K) if hasattr(bench, "tokens") else bench.tokens_per_step * K
-    launches = bench.launches(W, K) if hasattr(bench, "launches") else bench.launches_per_step * K
-    value = replica_value(tokens, world, ms)
-    src = kernel_src_hash(getattr(bench, "KERNEL_SRC", "decode_attn_tc.cuh"))
-    if hasattr(bench, "flops"):      # attention-state-memory lookup: tensor bound (bf16 x 3)
+        schedule_pass({i: (lambda i=i: kernel_step(i)) for i in kern})
+    barrier(world)
+    kern_ms = [a.elapsed_time(b) for a, b in kern_ev]
+    del parts
+
+    # ---- per-step times of a workload timed as one graph: each step its own graph
+    if step_ms is None:
+        graphs = [capture(lambda i=i: full_step(i)) for i in per_step]
+        step_ms = time_graphs(graphs, None, world)
+        del graphs
+
+    # ---- e2e region: each step's inputs from pinned host memory (one packed copy), its outputs
+    # read back (one copy), the step in between; every step one CUDA graph
+    e2e_ms = None
+    if e2e:
+        log(f"{bench.key}: e2e region ({len(e2e_steps)} steps)")
+        rows = warm_e2e + e2e_steps
+        h_in = torch.empty(len(rows), bench.stage.nbytes, dtype=torch.uint8).pin_memory()
+        for j, i in enumerate(rows):
+            bench.stage.fill_host(h_in[j], bench.host_inputs(i))
+        h_out = torch.empty(bench.out.nbytes, dtype=torch.uint8).pin_memory()
+        row_of = {i: j for j, i in enumerate(rows)}
+
+        def e2e_step(i):
+            bench.stage.dev.copy_(h_in[row_of[i]], non_blocking=True)
+            full_step(i, bench.stage.views)
+            h_out.copy_(bench.out.dev, non_blocking=True)
+
+        for i in warm_e2e:   # warm-up through the same path
+            e2e_step(i)
+        torch.cuda.synchronize()
+        graphs = {i: capture(lambda i=i: e2e_step(i)) for i in e2e_steps}
+        if n is None:
+            if bench.flush_l2:
+                e2e_ms = sum(time_graphs([graphs[i] for i in e2e_steps], flush, world))
+            else:
+                e2e_ms = time_region(lambda: [graphs[i].replay() for i in e2e_steps], world)
+        else:
+            acc = []
+            barrier(world)
+            schedule_pass({i: (lambda g=graphs[i]: acc.extend(time_graphs([g], flush, 1))) for i in e2e_steps})
+            barrier(world)
+            e2e_ms = sum(acc)
+        del graphs
+    if n is not None:   # leave the cache as it was just before `nxt`, for the parity check
+        bench.reset()
+        for i in range(nxt):
+            full_step(i)
+        torch.cuda.synchronize()
+    return dict(main=main, ms=ms, step_ms=step_ms, kern=kern, kern_ms=kern_ms, e2e_steps=e2e_steps,
+                e2e_ms=e2e_ms, next=nxt)
+
+
+def report(bench, m, world, hbm_peak, peak_kind):
+    """The JSON fields of one workload from its measurement."""
+    main, K = m["main"], len(m["main"])
+    ms = max_over_ranks(m["ms"], world)
+    kms = max_over_ranks(statistics.mean(m["kern_ms"]), world)
+    value = replica_value(sum(bench.tokens(i) for i in main), world, ms)
+    src = kernel_src_hash(bench.KERNEL_SRC)
+    if bench.bound == "tensor":
         bf16_tf, bf16_kind = bf16_peak()
         peak_tf = bf16_tf / 3.0
         achieved = bench.flops() / (kms / 1e3) / 1e12
         roofline = {"bound": "tensor", "kernel": bench.kernel_name(), "achieved": achieved, "peak": peak_tf,
                     "unit": "TFLOP/s", "frac": achieved / peak_tf,
                     "peak_source": ASMBench.PEAK_NOTE.format(kind=bf16_kind, bf16=bf16_tf),
-                    "traffic": None, "algorithmic_flops_per_launch": bench.flops(), "kernel_ms_avg": kms}
-        step_bytes = bench.evict_bytes()
+                    "traffic": None, "algorithmic_flops_per_launch": bench.flops(), "kernel_ms_avg": kms,
+                    "launches_timed": len(m["kern_ms"])}
     else:
-        attn_bytes = bench.mean_kv_bytes(W + K, KR) if hasattr(bench, "mean_kv_bytes") else bench.attn_bytes()
-        achieved = attn_bytes / (kms / 1e3) / 1e9
-        name = (bench.kernel_name() if hasattr(bench, "kernel_name")
-                else "kvb_decode_attn = decode_attn_tc_kernel<128,4,plain> + merge_splits_kernel")
-        roofline = {"bound": "hbm", "kernel": name, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                    "frac": achieved / hbm_peak, "peak_source": f"{peak_kind} (hbm_gbs)",
-                    "traffic": MEASURED_TRAFFIC.get((src, args.config, getattr(bench, "S", 0))),
-                    "algorithmic_bytes_per_launch": attn_bytes, "kernel_ms_avg": kms}
-        step_bytes = attn_bytes + (bench.evict_bytes() if hasattr(bench, "evict_bytes") else 0)
-    kv_gbs = step_bytes * K / (ms / 1e3) / 1e9
+        # launches of a finite schedule differ in size: bytes over time summed over the same launches
+        kb = [bench.attn_bytes(i) for i in m["kern"]]
+        achieved = sum(kb) / (max_over_ranks(sum(m["kern_ms"]), world) / 1e3) / 1e9
+        roofline = {"bound": "hbm", "kernel": bench.kernel_name(), "achieved": achieved, "peak": hbm_peak,
+                    "unit": "GB/s", "frac": achieved / hbm_peak, "peak_source": f"{peak_kind} (hbm_gbs)",
+                    "traffic": MEASURED_TRAFFIC.get((src, bench.key, getattr(bench, "S", 0))),
+                    "algorithmic_bytes_per_launch": statistics.mean(kb), "kernel_ms_avg": kms,
+                    "launches_timed": len(m["kern_ms"])}
+    step_bytes = sum(bench.attn_bytes(i) + bench.other_bytes(i) for i in main)
+    kv_gbs = step_bytes / (ms / 1e3) / 1e9
+    out = {"value": value, "unit": "tokens/s", "steps": K, "ms_per_step": ms / K, "kv_gbs": kv_gbs,
+           "kv_frac_of_hbm_peak": kv_gbs / hbm_peak, "roofline": roofline,
+           "step_ms_percentiles": pct(m["step_ms"]) if m["step_ms"] else None,
+           "gpu_launches": sum(bench.launches(i) for i in main), "kernel_src_sha256_16": src}
+    if m["e2e_ms"] is not None:
+        E = len(m["e2e_steps"])
+        e2e_ms = max_over_ranks(m["e2e_ms"], world)
+        out["e2e"] = {"value": replica_value(sum(bench.tokens(i) for i in m["e2e_steps"]), world, e2e_ms),
+                      "unit": "tokens/s", "h2d_bytes_per_step": bench.stage.payload,
+                      "d2h_bytes_per_step": bench.out.payload, "ms_per_step": e2e_ms / E, "steps": E,
+                      "copies": "one packed host-to-device copy of the step's inputs and one device-to-host "
+                                "copy of its outputs per step, inside each step's CUDA graph"}
+    return out
 
-    e2e = None
-    if not args.no_e2e and hasattr(bench, "run_e2e"):
-        first = W + K + KR
-        bench.run_e2e(first, W)
-        torch.cuda.synchronize()
-        ms_e2e = max_over_ranks(time_region(lambda: bench.run_e2e(first + W, K), world), world)
-        h2d, d2h = bench.e2e_bytes()
-        e2e = {"value": bench.tokens_per_step * K * world / (ms_e2e / 1e3), "unit": "tokens/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e / K}
 
-    cfg = bench.config()
-    cfg["timed_launches"] = "cuda graph replay" if graph is not None else "stream launches"
+def oracle_baseline(bench, budget_s: float):
+    """The oracle as it stands on a bounded sample of the workload: on every host core (its
+    parallel driver over independent (sequence, kv head) units) and on one core."""
+    import oracle
+    oracle.build()
+    cores = host_cores()
+    v_all, n_all = bench.oracle_sample(oracle, cores, budget_s)
+    v_one, n_one = bench.oracle_sample(oracle, 1, budget_s / 3)
+    w = bench.w
+    return {"value": v_all, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n_all} whole-batch decode steps (B={w.B}) from the prefill state, the (sequence, kv head) "
+                      f"units spread over {cores} threads",
+            "cpu_model": cpu_model(),
+            "single_core": {"value": v_one, "unit": "tokens/s", "cores": 1,
+                            "sample": f"{n_one} whole-batch decode steps from the prefill state"}}
+
+
+def run_workload(key, splits, args, world, local, K, W, hbm_peak, peak_kind, cpu_baseline: bool):
+    clocks = ClockSampler(local)
+    clocks.start()
+    log(f"{key}: set-up")
+    bench = make_bench(key, splits, args.seed)
+    m = measure(bench, K, W, world, not args.no_e2e)
+    clk = clocks.stop()
+    r = report(bench, m, world, hbm_peak, peak_kind)
+    r["config"] = bench.config()
+    r["config"]["timed_launches"] = "cuda graph replay"
+    r["clocks"] = clk
+    if args.check != "off":
+        log(f"{key}: consistency check")
+        r["consistency"] = bench.check(m["next"], args.check == "full")
+    if cpu_baseline and hasattr(bench, "oracle_sample"):
+        log(f"{key}: oracle baseline")
+        r["cpu_baseline"] = oracle_baseline(bench, 12.0)
+    log(f"{key}: done")
+    del bench
+    torch.cuda.empty_cache()
+    return r
+
+
+def run_kvb(args, world, rank, local):
+    hbm_peak, peak_kind = peaks()
+    key = f"{args.config}{'p' if (args.plain and args.config == 3) or (args.paged and args.config == 5) else ''}"
+    W = max(3, args.warmup)
+    head = run_workload(key, args.splits, args, world, local, args.steps, W, hbm_peak, peak_kind,
+                        rank == 0 and world == 1 and not args.no_cpu_baseline)
     out = {
         "metric": METRIC,
-        "value": value,
-        "unit": "tokens/s",
+        "value": head.pop("value"),
+        "unit": head.pop("unit"),
         "n_gpus": world,
-        "steps": K,
+        "steps": head.pop("steps"),
         "warmup": W,
-        "ms_per_step": ms / K,
+        "ms_per_step": head.pop("ms_per_step"),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "f32",
         "storage_dtype": "bf16",
         "data": "synthetic (seeded; shapes and distributions of the workload)",
-        "config": cfg,
-        "kv_gbs": kv_gbs,
-        "kv_frac_of_hbm_peak": kv_gbs / hbm_peak,
-        "roofline": roofline,
-        "clocks": clk,
-        "e2e": e2e,
-        "gpu_launches": launches,
-        "kernel_src_sha256_16": src,
+        "config": head.pop("config"),
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and hasattr(bench, "oracle_sample"):
-        v, sample = bench.oracle_sample()
-        out["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample}
+    out.update(head)
+    spec = args.configs.strip().lower()
+    subs = [] if spec == "none" else (list(WORKLOADS) if spec == "all" else [s.strip() for s in spec.split(",")])
+    subs = [s for s in subs if s and s != key]
+    if subs:
+        out["configs"] = {}
+        for sk in subs:
+            out["configs"][sk] = run_workload(sk, 0, args, world, local, min(args.steps, 48), min(W, 8),
+                                              hbm_peak, peak_kind, False)
     return out
 
 
@@ -688,7 +1093,7 @@ def run_reference(args, world, rank):
         return None
     import oracle
     from memory_bounded_kv_b200 import synth
-    w = synth.decode_workload(2 if args.config not in (1, 3) else args.config)
+    w = synth.decode_workload(2 if args.config not in (1, 3) else args.config, seed=args.seed)
     nb = 1   # one sequence per step keeps --steps K --warmup W within minutes
     c = dict(k=w.k[:nb].copy(), v=w.v[:nb].copy(), log_beta=w.log_beta[:nb].copy(), pos=w.pos[:nb].copy(),
              len=w.len[:nb].copy())
@@ -712,7 +1117,8 @@ def run_reference(args, world, rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample,
+                         "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -762,7 +1168,7 @@ def run_asm_build(args) -> dict:
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
             fn()
-        out[name] = time_flushed_steps([graph.replay] * iters, flush, 1) / iters
+        out[name] = sum(time_graphs([graph] * iters, flush, 1)) / iters
         del graph
     clk = clocks.stop()
     flops = 2.0 * M * H * K * d
@@ -882,6 +1288,7 @@ def run_asm_crossover(args) -> dict:
             "config": {"workload": "attention-state memory, 32 heads, d 128, top-16 of sqrt(K) clusters",
                        "l2": "flushed before every timed call (256 MiB write)"},
             "peak_gbs": hbm_peak, "peak_source": f"{peak_kind} (hbm_gbs)", "rows": rows, "clocks": clk}
+
 
 
 def main():

@@ -58,7 +58,8 @@ enum kvb_device_error {
     KVB_DERR_LEN = 1u << 0,       /* len < 0 or len > cap */
     KVB_DERR_SPLIT = 1u << 1,     /* split_len * num_splits < len */
     KVB_DERR_RANGE = 1u << 2,     /* compaction range outside [0, len) */
-    KVB_DERR_TIMEOUT = 1u << 3    /* a bounded wait on a copy gave up */
+    KVB_DERR_TIMEOUT = 1u << 3,   /* a bounded wait on a copy gave up */
+    KVB_DERR_PAGES = 1u << 4      /* a paged cache needed a page and its free stack was empty */
 };
 
 /* ------------------------------------------------------------------------
@@ -274,6 +275,73 @@ kvb_status kvb_compact_blocks(uint16_t* k, uint16_t* v, int32_t* pos, float* log
                               kvb_stream stream);
 
 /* ------------------------------------------------------------------------
+ * Paged cache: kvb_paged_reset, kvb_paged_evict_insert,
+ * kvb_paged_decode_attn, kvb_paged_compact_blocks
+ *
+ * [MEM] systems: the engine removes KV entries physically inside generation,
+ * and the cache is a sawtooth (chunking and compression) -- a flat cache must
+ * reserve the peak length for every sequence, a paged one holds the pages in
+ * use. The logical cache of each (sequence b, kv head g) is the flat cache of
+ * the calls above (slots [0, len) in slot order); its slots live in pages of
+ * KVB_PAGE_SLOTS slots taken from one pool: logical slot s is row
+ * s % KVB_PAGE_SLOTS of page table[b, g, s / KVB_PAGE_SLOTS], and pages
+ * 0 .. ceil(len / KVB_PAGE_SLOTS) - 1 of the table are set (the last one
+ * partly used). Free pages are a stack on the device: free_pages[0 ..
+ * *free_count). Each operation computes exactly what its flat counterpart
+ * computes on the logical cache:
+ *   kvb_paged_evict_insert   = kvb_evict_insert; an append at a page
+ *       boundary pops a page from the free stack (none left: the token is not
+ *       inserted, victim = -1, KVB_DERR_PAGES);
+ *   kvb_paged_decode_attn    = kvb_decode_attn over the logical cache (bias
+ *       when log_beta_pages != NULL); every split starts on a page: one split,
+ *       or split_len a multiple of KVB_PAGE_SLOTS (else KVB_EINVAL); q is
+ *       [B, Hq, d] contiguous, the outputs and evict_cand as kvb_decode_attn;
+ *   kvb_paged_compact_blocks = kvb_compact_blocks; the slots after the range
+ *       move down through the table (their bytes unchanged) and the pages past
+ *       the new length go back on the free stack (their table entries -1);
+ *   kvb_paged_reset: every page free (free_pages = 0 .. num_pages - 1 in
+ *       order, *free_count = num_pages), every table entry -1, len = 0.
+ * Which physical page a logical page gets depends on the order in which
+ * CTAs pop the stack; only the logical cache is deterministic.
+ * Layouts (contiguous): k_pages, v_pages [num_pages, KVB_PAGE_SLOTS, d] bf16;
+ * log_beta_pages (nullable), pos_pages [num_pages, KVB_PAGE_SLOTS]; table
+ * [B, Hkv, max_pages] int32; len [B, Hkv]; free_pages [num_pages];
+ * free_count [1]. Capacity per (b, g): max_pages * KVB_PAGE_SLOTS slots.
+ * Requirements: B, Hkv, max_pages, num_pages >= 1; d % 8 == 0 (d in {64,
+ * 128} for the attention); k_pages, v_pages, pos_pages, log_beta_pages
+ * 16-byte aligned. A table entry outside [0, num_pages) met on the device
+ * sets KVB_DERR_RANGE (the insertion or removal of that head is skipped; the
+ * attention reads page 0 in its place).
+ * ---------------------------------------------------------------------- */
+#define KVB_PAGE_SLOTS 64
+
+typedef struct kvb_paged_cache {
+    uint16_t* k_pages;
+    uint16_t* v_pages;
+    float* log_beta_pages;
+    int32_t* pos_pages;
+    int32_t* table;
+    int32_t* len;
+    int32_t* free_pages;
+    int32_t* free_count;
+    int32_t B, Hkv, d, max_pages, num_pages;
+} kvb_paged_cache;
+
+kvb_status kvb_paged_reset(const kvb_paged_cache* cache, kvb_stream stream);
+
+kvb_status kvb_paged_evict_insert(const kvb_paged_cache* cache, const uint16_t* k_new, const uint16_t* v_new,
+                                  const float* log_beta_new, const int32_t* t, int32_t M, int32_t* victim,
+                                  const void* cand, int32_t cand_n, kvb_stream stream);
+
+kvb_status kvb_paged_decode_attn(const kvb_paged_cache* cache, const uint16_t* q, const int32_t* t, int32_t Hq,
+                                 float scale, int32_t num_splits, int32_t split_len, float* o_part,
+                                 float* lse_part, void* o, int32_t o_dtype, float* lse, void* evict_cand,
+                                 kvb_stream stream);
+
+kvb_status kvb_paged_compact_blocks(const kvb_paged_cache* cache, const int32_t* rm_start, const int32_t* rm_len,
+                                    kvb_stream stream);
+
+/* ------------------------------------------------------------------------
  * kvb_asm_lookup_merge -- attention-state-memory lookup and merge
  *
  * [ASM] steps 3-4. For query token n and head h:
@@ -302,6 +370,34 @@ kvb_status kvb_asm_lookup_merge(const uint16_t* q, const float* qbar, const uint
                                 const float* lse_self, int32_t N, int32_t H, int32_t K,
                                 int32_t d, int32_t* idx, float* o, float* lse,
                                 void* workspace, size_t workspace_bytes, kvb_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Prepared memory: kvb_asm_prepare, kvb_asm_lookup_merge_planes
+ *
+ * [ASM] steps 3-4 over a memory built once offline. kvb_asm_prepare does the
+ * per-centroid work of the lookup once: every centroid row qbar[t, k] is
+ * normalised in f32 (x / sqrt(sum x^2); a zero row stays zero) and split
+ * exactly into three bf16 parts (hi = rn(x), mid = rn(x - hi), lo = x - hi -
+ * mid), written as `planes`, an opaque device buffer of
+ * kvb_asm_planes_bytes(H_tables, K) bytes (16-byte aligned) laid out for the
+ * lookup's tensor-core tiles (64 centroids per tile, K rounded up to a
+ * multiple of 64 with zero rows). qbar [H_tables, K, d] f32, d == 128.
+ * kvb_asm_lookup_merge_planes computes exactly what kvb_asm_lookup_merge_grouped
+ * computes (same arguments, with planes in place of qbar: the index, the
+ * merged state, the assignment-only form with o == NULL, the same workspace).
+ * The planes must have been prepared from the same qbar, H_tables and K; they
+ * stay valid while qbar is unchanged.
+ * ---------------------------------------------------------------------- */
+size_t kvb_asm_planes_bytes(int32_t H_tables, int32_t K);
+
+kvb_status kvb_asm_prepare(const float* qbar, int32_t H_tables, int32_t K, int32_t d, void* planes,
+                           size_t planes_bytes, kvb_stream stream);
+
+kvb_status kvb_asm_lookup_merge_planes(const uint16_t* q, const void* planes, size_t planes_bytes,
+                                       const uint16_t* abar, const float* log_zbar, const float* o_self,
+                                       const float* lse_self, int32_t N, int32_t H, int32_t H_tables, int32_t K,
+                                       int32_t d, int32_t* idx, float* o, float* lse, void* workspace,
+                                       size_t workspace_bytes, kvb_stream stream);
 
 /* ------------------------------------------------------------------------
  * kvb_asm_hier_lookup_merge -- two-level attention-state-memory lookup

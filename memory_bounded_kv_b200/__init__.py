@@ -31,6 +31,8 @@ __all__ = [
     "kvb_asm_lookup_merge_grouped", "kvb_asm_aggregate_grouped",
     "kvb_get_error", "kvb_abi_version", "kvb_test_withhold_next_decode",
     "decode_workspace", "evict_candidates",
+    "PagedPool", "kvb_paged_reset", "kvb_paged_evict_insert", "kvb_paged_decode_attn", "kvb_paged_compact_blocks",
+    "kvb_asm_planes_bytes", "kvb_asm_prepare", "kvb_asm_lookup_merge_planes",
 ]
 
 
@@ -356,6 +358,54 @@ def kvb_asm_lookup_merge(q, qbar, abar, log_zbar, o_self, lse_self, idx, o, lse,
 kvb_asm_lookup_merge_grouped = kvb_asm_lookup_merge   # the table count is qbar's first dimension
 
 
+def kvb_asm_planes_bytes(H_tables: int, K: int) -> int:
+    return int(_lib.lib().kvb_asm_planes_bytes(H_tables, K))
+
+
+def kvb_asm_prepare(qbar, planes=None, *, stream=None):
+    """Prepare a memory for kvb_asm_lookup_merge_planes: qbar [H_tables, K, d] f32 -> planes (a uint8
+    CUDA tensor of kvb_asm_planes_bytes(H_tables, K) bytes; allocated when None). Returns planes."""
+    _need(qbar, torch.float32, "qbar"); _contig(qbar, "qbar")
+    Ht, K, d = qbar.shape
+    nbytes = kvb_asm_planes_bytes(Ht, K)
+    if planes is None:
+        planes = torch.empty(nbytes, dtype=torch.uint8, device=qbar.device)
+    _contig(planes, "planes")
+    if planes.numel() * planes.element_size() < nbytes:
+        raise ValueError("planes buffer too small")
+    _check(_lib.lib().kvb_asm_prepare(_ptr(qbar), Ht, K, d, _ptr(planes), planes.numel() * planes.element_size(),
+                                      _stream(stream)), "kvb_asm_prepare")
+    return planes
+
+
+def kvb_asm_lookup_merge_planes(q, planes, H_tables: int, K: int, abar, log_zbar, o_self, lse_self, idx, o, lse,
+                                workspace, *, stream=None) -> None:
+    """kvb_asm_lookup_merge over a memory prepared by kvb_asm_prepare (H_tables tables of K entries)."""
+    _need(q, torch.bfloat16, "q"); _contig(q, "q"); _contig(planes, "planes")
+    N, H, d = q.shape
+    if o is not None:
+        _need(abar, torch.bfloat16, "abar"); _need(log_zbar, torch.float32, "log_zbar")
+        _need(o_self, torch.float32, "o_self"); _need(lse_self, torch.float32, "lse_self")
+        _need(o, torch.float32, "o")
+        for name, x, shp in (("abar", abar, (H_tables, K, d)), ("log_zbar", log_zbar, (H_tables, K)),
+                             ("o_self", o_self, (N, H, d)), ("lse_self", lse_self, (N, H)), ("o", o, (N, H, d))):
+            _shape(x, shp, name)
+            _contig(x, name)
+    elif idx is None:
+        raise ValueError("o=None (assignment only) needs idx")
+    _shape(idx, (N, H), "idx")
+    _shape(lse, (N, H), "lse")
+    if idx is not None:
+        _need(idx, torch.int32, "idx"); _contig(idx, "idx")
+    if lse is not None:
+        _need(lse, torch.float32, "lse"); _contig(lse, "lse")
+    _contig(workspace, "workspace")
+    _check(_lib.lib().kvb_asm_lookup_merge_planes(
+        _ptr(q), _ptr(planes), planes.numel() * planes.element_size(), _ptr(abar), _ptr(log_zbar), _ptr(o_self),
+        _ptr(lse_self), N, H, int(H_tables), int(K), d, _ptr(idx), _ptr(o), _ptr(lse), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)), "kvb_asm_lookup_merge_planes")
+
+
 def kvb_asm_aggregate_workspace_bytes(H: int, K: int) -> int:
     return int(_lib.lib().kvb_asm_aggregate_workspace_bytes(H, K))
 
@@ -444,3 +494,107 @@ def kvb_asm_hier_lookup_merge(q, qhat, offsets, members, qbar, abar, log_zbar, o
                                                 _ptr(abar), _ptr(log_zbar), _ptr(o_self), _ptr(lse_self), N, H, K,
                                                 C, int(m), d, _ptr(idx), _ptr(o), _ptr(lse), _ptr(workspace),
                                                 nbytes, _stream(stream)), "kvb_asm_hier_lookup_merge")
+
+
+# ----------------------------------------------------------------------------------------------
+# paged cache (see "Paged cache" in include/kvb.h)
+# ----------------------------------------------------------------------------------------------
+
+class PagedPool:
+    """The device tensors of a paged cache: k_pages, v_pages [P, PAGE_SLOTS, d] bf16, log_beta_pages
+    (None: beta = 1) and pos_pages [P, PAGE_SLOTS], table [B, Hkv, max_pages] int32, len [B, Hkv],
+    free_pages [P], free_count [1]. Freshly made, call kvb_paged_reset() before use."""
+
+    def __init__(self, B, Hkv, d, max_pages, num_pages, with_beta=True, device="cuda"):
+        S = _lib.PAGE_SLOTS
+        self.B, self.Hkv, self.d, self.max_pages, self.num_pages = B, Hkv, d, max_pages, num_pages
+        self.k_pages = torch.zeros(num_pages, S, d, dtype=torch.bfloat16, device=device)
+        self.v_pages = torch.zeros_like(self.k_pages)
+        self.log_beta_pages = torch.zeros(num_pages, S, dtype=torch.float32, device=device) if with_beta else None
+        self.pos_pages = torch.zeros(num_pages, S, dtype=torch.int32, device=device)
+        self.table = torch.full((B, Hkv, max_pages), -1, dtype=torch.int32, device=device)
+        self.len = torch.zeros(B, Hkv, dtype=torch.int32, device=device)
+        self.free_pages = torch.zeros(num_pages, dtype=torch.int32, device=device)
+        self.free_count = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def args(self, use_beta=True) -> "_lib.PagedCacheArgs":
+        lb = self.log_beta_pages if use_beta else None
+        return _lib.PagedCacheArgs(
+            k_pages=self.k_pages.data_ptr(), v_pages=self.v_pages.data_ptr(),
+            log_beta_pages=None if lb is None else lb.data_ptr(), pos_pages=self.pos_pages.data_ptr(),
+            table=self.table.data_ptr(), len=self.len.data_ptr(), free_pages=self.free_pages.data_ptr(),
+            free_count=self.free_count.data_ptr(), B=self.B, Hkv=self.Hkv, d=self.d, max_pages=self.max_pages,
+            num_pages=self.num_pages)
+
+
+def _pool(pool, use_beta=True):
+    if not isinstance(pool, PagedPool):
+        raise TypeError("pool must be a PagedPool")
+    return ctypes.byref(pool.args(use_beta))
+
+
+def kvb_paged_reset(pool, *, stream=None) -> None:
+    """Every page free, every table entry -1, len 0."""
+    _check(_lib.lib().kvb_paged_reset(_pool(pool), _stream(stream)), "kvb_paged_reset")
+
+
+def kvb_paged_evict_insert(pool, k_new, v_new, log_beta_new, t, M: int, victim=None, *, cand=None, cand_n: int = 0,
+                           stream=None) -> None:
+    """Budget enforcement + insertion on a paged cache (kvb_evict_insert on the logical cache)."""
+    B, Hkv, d = pool.B, pool.Hkv, pool.d
+    for name, x, shp in (("k_new", k_new, (B, Hkv, d)), ("v_new", v_new, (B, Hkv, d)),
+                         ("log_beta_new", log_beta_new, (B, Hkv)), ("t", t, (B,)), ("victim", victim, (B, Hkv))):
+        _shape(x, shp, name)
+    for name, x in (("k_new", k_new), ("v_new", v_new)):
+        if x is not None:
+            _need(x, torch.bfloat16, name); _contig(x, name)
+    _need(t, torch.int32, "t"); _contig(t, "t")
+    if pool.log_beta_pages is not None:
+        _need(log_beta_new, torch.float32, "log_beta_new"); _contig(log_beta_new, "log_beta_new")
+    if victim is not None:
+        _need(victim, torch.int32, "victim"); _contig(victim, "victim")
+    cp = None if cand is None else ctypes.c_void_p(_cand_ptr(cand, B * Hkv * int(cand_n)))
+    _check(_lib.lib().kvb_paged_evict_insert(_pool(pool), _ptr(k_new), _ptr(v_new),
+                                             _ptr(log_beta_new) if pool.log_beta_pages is not None else None,
+                                             _ptr(t), int(M), _ptr(victim), cp, int(cand_n) if cand is not None else 0,
+                                             _stream(stream)), "kvb_paged_evict_insert")
+
+
+def kvb_paged_decode_attn(pool, q, t, o, lse=None, *, use_beta=True, scale: float = 0.0, num_splits: int = 1,
+                          split_len: int = 0, o_part=None, lse_part=None, evict_cand=None, stream=None) -> None:
+    """Decode attention over a paged cache (kvb_decode_attn on the logical cache). q [B, Hq, d] bf16
+    contiguous; one split, or split_len a multiple of PAGE_SLOTS; the rest as kvb_decode_attn."""
+    if q.dim() != 3:
+        raise ValueError("q must be [B, Hq, d]")
+    B, Hq, d = q.shape
+    if B != pool.B or d != pool.d:
+        raise ValueError("q must be [B, Hq, d] of the pool's B and d")
+    for name, x, shp in (("t", t, (B,)), ("o", o, (B, Hq, d)), ("lse", lse, (B, Hq)),
+                         ("o_part", o_part, (B, Hq, num_splits, d)), ("lse_part", lse_part, (B, Hq, num_splits))):
+        _shape(x, shp, name)
+    if num_splits > 1 and (o_part is None or lse_part is None):
+        raise ValueError("num_splits > 1 needs o_part and lse_part (decode_workspace())")
+    _need(q, torch.bfloat16, "q"); _contig(q, "q")
+    if t is not None:
+        _need(t, torch.int32, "t"); _contig(t, "t")
+    if o.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("o must be float32 or bfloat16")
+    _contig(o, "o")
+    for name, x in (("lse", lse), ("o_part", o_part), ("lse_part", lse_part)):
+        if x is not None:
+            _need(x, torch.float32, name); _contig(x, name)
+    cand = None if evict_cand is None else ctypes.c_void_p(_cand_ptr(evict_cand, B * pool.Hkv * int(num_splits)))
+    _check(_lib.lib().kvb_paged_decode_attn(_pool(pool, use_beta), _ptr(q), _ptr(t), Hq, float(scale),
+                                            int(num_splits), int(split_len), _ptr(o_part), _ptr(lse_part), _ptr(o),
+                                            _lib.KVB_OUT_F32 if o.dtype == torch.float32 else _lib.KVB_OUT_BF16,
+                                            _ptr(lse), cand, _stream(stream)), "kvb_paged_decode_attn")
+
+
+def kvb_paged_compact_blocks(pool, rm_start, rm_len, *, stream=None) -> None:
+    """In-place removal of slots [rm_start[b], +rm_len[b]) from every kv head of sequence b of a paged
+    cache; pages past the new lengths return to the free stack."""
+    for name, x in (("rm_start", rm_start), ("rm_len", rm_len)):
+        _shape(x, (pool.B,), name)
+        _need(x, torch.int32, name); _contig(x, name)
+    _check(_lib.lib().kvb_paged_compact_blocks(_pool(pool), _ptr(rm_start), _ptr(rm_len), _stream(stream)),
+           "kvb_paged_compact_blocks")

@@ -20,11 +20,13 @@ EXPORTS = (
     "kvb_asm_lookup_merge_grouped", "kvb_asm_aggregate_grouped",
     "kvb_get_error", "kvb_status_str",
     "kvb_abi_version", "kvb_test_withhold_next_decode",
+    "kvb_paged_reset", "kvb_paged_evict_insert", "kvb_paged_decode_attn", "kvb_paged_compact_blocks",
+    "kvb_asm_planes_bytes", "kvb_asm_prepare", "kvb_asm_lookup_merge_planes",
 )
 
 KVB_OK, KVB_EINVAL, KVB_ECUDA, KVB_EDEVICE = 0, 1, 2, 3
 KVB_OUT_F32, KVB_OUT_BF16 = 0, 1
-DERR_LEN, DERR_SPLIT, DERR_RANGE, DERR_TIMEOUT = 1, 2, 4, 8
+DERR_LEN, DERR_SPLIT, DERR_RANGE, DERR_TIMEOUT, DERR_PAGES = 1, 2, 4, 8, 16
 NOALLOC_SCRATCH_BYTES = 16 << 20   # KVB_NOALLOC_SCRATCH_BYTES
 
 
@@ -44,6 +46,16 @@ class AttnArgs(ctypes.Structure):
     ]
 
 EVICT_CAND_BYTES = 16   # sizeof(kvb_evict_cand)
+PAGE_SLOTS = 64         # KVB_PAGE_SLOTS
+
+
+class PagedCacheArgs(ctypes.Structure):
+    """Mirror of struct kvb_paged_cache."""
+    _fields_ = [
+        ("k_pages", _P), ("v_pages", _P), ("log_beta_pages", _P), ("pos_pages", _P),
+        ("table", _P), ("len", _P), ("free_pages", _P), ("free_count", _P),
+        ("B", _I32), ("Hkv", _I32), ("d", _I32), ("max_pages", _I32), ("num_pages", _I32),
+    ]
 
 
 _lib = None
@@ -88,11 +100,23 @@ def lib() -> ctypes.CDLL:
         L.kvb_status_str.restype = ctypes.c_char_p
         L.kvb_abi_version.argtypes = []
         L.kvb_test_withhold_next_decode.argtypes = [ctypes.c_uint64]
+        _PC = ctypes.POINTER(PagedCacheArgs)
+        L.kvb_paged_reset.argtypes = [_PC, _P]
+        L.kvb_paged_evict_insert.argtypes = [_PC, _P, _P, _P, _P, _I32, _P, _P, _I32, _P]
+        L.kvb_paged_decode_attn.argtypes = [_PC, _P, _P, _I32, ctypes.c_float, _I32, _I32, _P, _P, _P, _I32, _P, _P,
+                                            _P]
+        L.kvb_paged_compact_blocks.argtypes = [_PC, _P, _P, _P]
+        L.kvb_asm_planes_bytes.argtypes = [_I32, _I32]
+        L.kvb_asm_planes_bytes.restype = _SZ
+        L.kvb_asm_prepare.argtypes = [_P, _I32, _I32, _I32, _P, _SZ, _P]
+        L.kvb_asm_lookup_merge_planes.argtypes = [_P, _P, _SZ, _P, _P, _P, _P] + [_I32] * 5 + [_P] * 4 + [_SZ, _P]
         for f in ("kvb_decode_attn", "kvb_decode_attn_noalloc", "kvb_merge_states", "kvb_evict_insert", "kvb_compact_blocks",
                   "kvb_asm_lookup_merge", "kvb_asm_hier_lookup_merge", "kvb_asm_aggregate",
                   "kvb_asm_entries_bf16", "kvb_asm_index_csr", "kvb_asm_lookup_merge_grouped",
                   "kvb_asm_aggregate_grouped", "kvb_get_error",
-                  "kvb_abi_version", "kvb_test_withhold_next_decode"):
+                  "kvb_abi_version", "kvb_test_withhold_next_decode", "kvb_paged_reset",
+                  "kvb_paged_evict_insert", "kvb_paged_decode_attn", "kvb_paged_compact_blocks",
+                  "kvb_asm_prepare", "kvb_asm_lookup_merge_planes"):
             getattr(L, f).restype = _I32
         _lib = L
     return _lib

@@ -93,3 +93,61 @@ class BoundedKVCache:
         n = int(self.len.sum().item())
         per_slot = 2 * self.d * 2 + (8 if self.log_beta is not None else 0)
         return n * per_slot
+
+
+class PagedKVCache:
+    """The cache of BoundedKVCache kept in pages of PAGE_SLOTS slots from one pool (kvb_paged_*):
+    the same decode step on the same logical cache, with memory for the pages in use instead of
+    `cap` slots per (sequence, kv head). Splits start on pages: num_splits == 1 or split_len a
+    multiple of PAGE_SLOTS."""
+
+    def __init__(self, B, Hq, Hkv, d, max_pages, num_pages, M, num_splits=1, split_len=0, with_beta=True,
+                 device="cuda"):
+        from . import PagedPool, kvb_paged_reset
+        self.B, self.Hq, self.Hkv, self.d, self.M = B, Hq, Hkv, d, M
+        self.num_splits, self.split_len = num_splits, split_len
+        self.pool = PagedPool(B, Hkv, d, max_pages, num_pages, with_beta, device)
+        kvb_paged_reset(self.pool)
+        self.victim = torch.zeros(B, Hkv, dtype=torch.int32, device=device)
+        self.o_part = self.lse_part = None
+        if num_splits > 1:
+            self.o_part, self.lse_part = decode_workspace(B, Hq, d, num_splits, device)
+        self.cand = evict_candidates(B, Hkv, num_splits, device)
+        self.cand_valid = False
+
+    @property
+    def len(self):
+        return self.pool.len
+
+    def reset(self):
+        from . import kvb_paged_reset
+        kvb_paged_reset(self.pool)
+        self.cand_valid = False
+
+    def insert(self, k_new, v_new, log_beta_new, t, stream=None):
+        from . import kvb_paged_evict_insert
+        kvb_paged_evict_insert(self.pool, k_new, v_new, log_beta_new, t, self.M, self.victim,
+                               cand=self.cand if self.cand_valid else None, cand_n=self.num_splits, stream=stream)
+        self.cand_valid = False
+
+    def attend(self, q, t, o, lse=None, stream=None, use_beta=True):
+        from . import kvb_paged_decode_attn
+        with_beta = self.pool.log_beta_pages is not None
+        same_scoring = use_beta or not with_beta
+        cand = self.cand if (same_scoring and t is not None) else None
+        kvb_paged_decode_attn(self.pool, q, t, o, lse, use_beta=use_beta, num_splits=self.num_splits,
+                              split_len=self.split_len, o_part=self.o_part, lse_part=self.lse_part,
+                              evict_cand=cand, stream=stream)
+        self.cand_valid = cand is not None
+
+    def step(self, q, k_new, v_new, log_beta_new, t, o, lse=None, stream=None):
+        self.insert(k_new, v_new, log_beta_new, t, stream)
+        self.attend(q, t, o, lse, stream)
+
+    def compact(self, rm_start, rm_len, stream=None):
+        from . import kvb_paged_compact_blocks
+        kvb_paged_compact_blocks(self.pool, rm_start, rm_len, stream=stream)
+        self.cand_valid = False
+
+    def pages_in_use(self) -> int:
+        return self.pool.num_pages - int(self.pool.free_count.item())

@@ -1,0 +1,300 @@
+// Attention-state-memory lookup over a prepared memory ("Context Memorization"
+// core method step 3: c* = argmax_k cos(q, qbar_k)). The memory is static once
+// built, so the normalisation of every centroid and its exact split into three
+// bf16 parts (hi = rn(x), mid = rn(x - hi), lo = x - hi - mid) are done once by
+// asm_prepare_kernel, which writes each tile of 64 centroids as the exact
+// shared-memory image the tensor-core MMA reads: [part][K half][64 rows][128 B],
+// 16-byte chunk c of row r at chunk c ^ (r & 7) (the 128-byte swizzle).
+//
+// asm_score_planes_kernel then streams those images with one bulk copy per
+// tile into a 3-stage ring and keeps the queries in tensor memory as the A
+// operand of tcgen05.mma (so each MMA reads only its 2 KB B slice from shared
+// memory), with three accumulator buffers:
+//   warp 9 (one lane)  bulk copies of the tile images           -> b_full[s]
+//   warp 8 (one lane)  48 MMAs per tile (2 M tiles x 3 parts x 8 K steps),
+//                      committed to b_empty[s] and acc_full[b]
+//   warps 0-7          the queries into tensor memory (tcgen05.st) at each new
+//                      block of 256 queries (-> a_ready), then per tile: read
+//                      their query row's 64 scores back (tcgen05.ld), release
+//                      the buffer (-> acc_empty[b]) and keep the running best.
+// The per-range best keys go to the same workspace as asm_score_umma_kernel's,
+// reduced and merged by asm_merge_kernel.
+#pragma once
+
+#include "asm_lookup.cuh"
+
+namespace kvb {
+
+constexpr int kPStages = 3;                                    // B ring stages == accumulator buffers
+constexpr size_t kPImg = 3 * kUPart;                           // one tile image: 48 KB
+constexpr int kPThreads = kUNT + 64;                           // 8 read-back warps + MMA warp + copy warp
+constexpr int kPACols = kUMT * (kAsmD / 2);                    // queries: 2 M tiles x 64 columns
+constexpr int kPAccCols = kUMT * kUKT;                         // one accumulator buffer: 2 x 64 columns
+constexpr int kPCols = 512;                                    // kPACols + kPStages * kPAccCols
+constexpr size_t kPBar = (size_t)kPStages * kPImg;             // after the ring
+constexpr size_t kPSmem = kPBar + 128 + 1024;                  // barriers + slot, + alignment slack
+static_assert(kPACols + kPStages * kPAccCols == kPCols, "tensor memory budget");
+
+__host__ __device__ inline size_t asm_plane_tiles(int K) { return (size_t)(K + kUKT - 1) / kUKT; }
+
+// ---- preparation: one warp per centroid row --------------------------------------------------
+__global__ void __launch_bounds__(256) asm_prepare_kernel(const float* __restrict__ qbar, int H, int K,
+                                                          unsigned char* __restrict__ planes) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const size_t tiles = asm_plane_tiles(K);
+    const long long row = (long long)blockIdx.x * 8 + warp;         // (table, tile row) over padded K
+    if (row >= (long long)H * tiles * kUKT) return;
+    const int h = (int)(row / ((long long)tiles * kUKT));
+    const int kk = (int)(row % ((long long)tiles * kUKT));          // centroid index (maybe >= K: zeros)
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (kk < K) x = reinterpret_cast<const float4*>(qbar + ((size_t)h * K + kk) * kAsmD)[lane];
+    float ss = fmaf(x.x, x.x, fmaf(x.y, x.y, fmaf(x.z, x.z, x.w * x.w)));
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) ss += __shfl_xor_sync(kFull, ss, m);
+    const float inv = (ss > 0.f) ? 1.f / sqrtf(ss) : 0.f;   // a zero centroid has cos 0
+    uint32_t hw[2], mw[2], lw[2];
+    split3_bf16x2(x.x * inv, x.y * inv, hw[0], mw[0], lw[0]);
+    split3_bf16x2(x.z * inv, x.w * inv, hw[1], mw[1], lw[1]);
+    // lane l holds elements 4l .. 4l + 3: K half l / 16, chunk (l % 16) / 2, bytes 8 (l % 2) .. + 7
+    const int r = kk % kUKT;
+    const int kh = lane >> 4, c = (lane & 15) >> 1;
+    unsigned char* img = planes + ((size_t)h * tiles + kk / kUKT) * kPImg;
+    const size_t off = kh * kUPartHalf + r * 128 + ((c ^ (r & 7)) << 4) + 8 * (lane & 1);
+    *reinterpret_cast<uint2*>(img + off) = make_uint2(hw[0], hw[1]);
+    *reinterpret_cast<uint2*>(img + kUPart + off) = make_uint2(mw[0], mw[1]);
+    *reinterpret_cast<uint2*>(img + 2 * kUPart + off) = make_uint2(lw[0], lw[1]);
+}
+
+// ---- tensor-memory helpers of the lookup ------------------------------------------------------
+// D (tensor memory) (+)= A (tensor memory) . B (shared memory descriptor)
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                             uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+// 32 lanes x 32 consecutive columns from registers (lane i of the warp writes lane base + i)
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+          "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+          "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+struct AsmPlanesParams {
+    AsmParams a;                   // queries, sizes, items, outputs (a.qbar unused)
+    const unsigned char* planes;   // [H_tables][tiles][kPImg]
+    unsigned long long wait_ns;
+};
+
+__global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __grid_constant__ AsmPlanesParams pp) {
+    const AsmParams& p = pp.a;
+    extern __shared__ unsigned char s_raw[];
+    unsigned char* sm = s_raw + ((1024u - (smem_u32(s_raw) & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t* b_full = reinterpret_cast<uint64_t*>(sm + kPBar);
+    uint64_t* b_empty = b_full + kPStages;
+    uint64_t* acc_full = b_empty + kPStages;
+    uint64_t* acc_empty = acc_full + kPStages;
+    uint64_t* a_ready = acc_empty + kPStages;
+    uint32_t* slot = reinterpret_cast<uint32_t*>(a_ready + 1);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int items = p.H * p.qtiles * p.ksplit;
+    const int i0 = blockIdx.x * p.per_cta, i1 = min(items, i0 + p.per_cta);
+    if (i0 >= i1) return;   // uniform over the CTA, before any allocation
+    int G = 0;              // tiles in this CTA's stream
+    for (int it = i0; it < i1; ++it) {
+        const int kb = (it % p.ksplit) * p.kchunk;
+        G += (min(p.K, kb + p.kchunk) - kb + kUKT - 1) / kUKT;
+    }
+    const size_t tiles_per_table = asm_plane_tiles(p.K);
+
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
+                     "r"(kPCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (tid == 0) {
+        for (int s = 0; s < kPStages; ++s) {
+            mbar_init(&b_full[s], 1);
+            mbar_init(&b_empty[s], 1);
+            mbar_init(&acc_full[s], 1);
+            mbar_init(&acc_empty[s], kUNT / 32);
+        }
+        mbar_init(a_ready, kUNT / 32);
+        fence_mbar_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *slot;
+    bool ok = true;
+
+    if (warp == kUNT / 32 + 1) {
+        // ---- copy warp: tile images into the ring
+        if (lane == 0) {
+            AsmTile c;
+            asm_tile_start(p, c, i0);
+            for (int g = 0; g < G && ok; ++g) {
+                const int s = g % kPStages;
+                if (g >= kPStages && !mbar_wait(&b_empty[s], (unsigned)((g / kPStages) - 1) & 1u, pp.wait_ns)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(&b_full[s], (unsigned)kPImg);
+                const unsigned char* src = pp.planes + ((size_t)(c.h / p.G) * tiles_per_table + c.kt / kUKT) * kPImg;
+                bulk_g2s(sm + (size_t)s * kPImg, src, (unsigned)kPImg, &b_full[s]);
+                asm_tile_next(p, c);
+            }
+        }
+    } else if (warp == kUNT / 32) {
+        // ---- MMA warp
+        if (lane == 0) {
+            AsmTile cm;
+            asm_tile_start(p, cm, i0);
+            constexpr uint32_t idesc = umma_idesc_bf16(kUQ, kUKT);
+            const uint64_t b0 = umma_desc_sw128(sbase);
+            int a_block = -1, a_phase = 0;
+            for (int g = 0; g < G; ++g) {
+                const int s = g % kPStages;
+                if (!mbar_wait(&b_full[s], (unsigned)(g / kPStages) & 1u, pp.wait_ns)) { ok = false; break; }
+                if (g >= kPStages && !mbar_wait(&acc_empty[s], (unsigned)((g / kPStages) - 1) & 1u, pp.wait_ns)) {
+                    ok = false;
+                    break;
+                }
+                const int blk = cm.h * p.qtiles + cm.qt;
+                if (blk != a_block) {   // the read-back warps have put this block's queries in tensor memory
+                    if (!mbar_wait(a_ready, (unsigned)a_phase & 1u, pp.wait_ns)) { ok = false; break; }
+                    ++a_phase;
+                    a_block = blk;
+                }
+                tc_fence_after();
+                const int mts = min(kUMT, (p.N - cm.qt * (kUMT * kUQ) + kUQ - 1) / kUQ);
+                for (int mt = 0; mt < mts; ++mt) {
+                    const uint32_t d = tmem + (uint32_t)(kPACols + s * kPAccCols + mt * kUKT);
+#pragma unroll
+                    for (int pt = 0; pt < 3; ++pt)
+#pragma unroll
+                        for (int kk = 0; kk < kAsmD / 16; ++kk) {
+                            const uint32_t a = tmem + (uint32_t)(mt * (kAsmD / 2) + kk * 8);
+                            const uint32_t boff =
+                                (uint32_t)(s * kPImg + pt * kUPart + (kk >> 2) * kUPartHalf + (kk & 3) * 32);
+                            umma_bf16_ts(d, a, b0 + (boff >> 4), idesc, (pt | kk) != 0);
+                        }
+                }
+                umma_commit(&b_empty[s]);
+                umma_commit(&acc_full[s]);
+                asm_tile_next(p, cm);
+            }
+        }
+    } else {
+        // ---- warps 0-7: queries into tensor memory, read-back and argmax
+        AsmTile ce;
+        asm_tile_start(p, ce, i0);
+        const int emt = warp >> 2, elane = 32 * (warp & 3);
+        float bmax = -INFINITY;
+        int bidx = -1;
+        int a_block = -1;
+        for (int g = 0; g < G; ++g) {
+            const int s = g % kPStages;
+            const int blk = ce.h * p.qtiles + ce.qt;
+            const int n0 = ce.qt * (kUMT * kUQ);
+            if (blk != a_block) {
+                // every MMA that read the previous queries is complete: this warp has read back the
+                // tile before (its acc_full arrives after all earlier MMAs)
+                const int n = n0 + emt * kUQ + elane + lane;
+                uint32_t r[kAsmD / 2];
+                if (n < p.N) {
+                    const uint4* src = reinterpret_cast<const uint4*>(p.q + ((size_t)n * p.H + ce.h) * kAsmD);
+#pragma unroll
+                    for (int j = 0; j < kAsmD / 8; ++j) {
+                        const uint4 v = src[j];
+                        r[4 * j] = v.x; r[4 * j + 1] = v.y; r[4 * j + 2] = v.z; r[4 * j + 3] = v.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < kAsmD / 2; ++j) r[j] = 0u;
+                }
+                const uint32_t ta = tmem + ((uint32_t)elane << 16) + (uint32_t)(emt * (kAsmD / 2));
+                tmem_st32(ta, r);
+                tmem_st32(ta + 32, r + 32);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(a_ready);
+                a_block = blk;
+            }
+            if (!mbar_wait(&acc_full[s], (unsigned)(g / kPStages) & 1u, pp.wait_ns)) ok = false;
+            tc_fence_after();
+            const int mts = min(kUMT, (p.N - n0 + kUQ - 1) / kUQ);
+            float v[kUKT];
+            if (ok && emt < mts) {
+                const uint32_t ta = tmem + ((uint32_t)elane << 16) + (uint32_t)(kPACols + s * kPAccCols + emt * kUKT);
+                tmem_ld32(ta, v);
+                tmem_ld32(ta + 32, v + 32);
+                tmem_ld_wait();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[s]);   // the buffer may take tile g + 3
+            if (ok && emt < mts) {
+                if (ce.kt + kUKT > ce.k_end) {   // ragged last tile of a range
+#pragma unroll
+                    for (int c = 0; c < kUKT; ++c)
+                        if (ce.kt + c >= ce.k_end) v[c] = -INFINITY;
+                }
+                float m[kUKT / 2];
+#pragma unroll
+                for (int c = 0; c < kUKT / 2; ++c) m[c] = fmaxf(v[c], v[c + kUKT / 2]);
+#pragma unroll
+                for (int w = kUKT / 4; w >= 1; w >>= 1)
+#pragma unroll
+                    for (int c = 0; c < w; ++c) m[c] = fmaxf(m[c], m[c + w]);
+                if (m[0] > bmax) {   // strictly greater: an equal value in a later tile has a larger k
+                    int first = kUKT - 1;
+#pragma unroll
+                    for (int c = kUKT - 1; c >= 0; --c) first = (v[c] == m[0]) ? c : first;
+                    bmax = m[0];
+                    bidx = ce.kt + first;
+                }
+            }
+            if (ce.kt + kUKT >= ce.k_end) {   // end of the item: write this row's best, start afresh
+                const int n = n0 + emt * kUQ + elane + lane;
+                if (emt < mts && n < p.N) {
+                    const unsigned long long key =
+                        (bidx < 0 || !ok) ? 0ull
+                                          : ((unsigned long long)float_order_key(bmax + 0.f) << 32) |
+                                                (0xffffffffu - (unsigned)bidx);
+                    p.ws[((size_t)ce.ks * p.N + n) * p.H + ce.h] = key;
+                }
+                bmax = -INFINITY;
+                bidx = -1;
+            }
+            asm_tile_next(p, ce);
+        }
+    }
+    if (!ok) raise_error(KVB_DERR_TIMEOUT);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kUNT / 32 && lane == 0 && G > 0) {
+        // the last tile's MMAs complete before the tensor memory is released (bounded)
+        mbar_wait(&acc_full[(G - 1) % kPStages], (unsigned)((G - 1) / kPStages) & 1u, pp.wait_ns);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kPCols) : "memory");
+    }
+}
+
+}  // namespace kvb

@@ -57,6 +57,10 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, unsigned by
                  : "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
     unsigned ok;
     asm volatile(
@@ -129,6 +133,14 @@ struct EvictCand {
     int t;  // the position the key was scored for
 };
 static_assert(sizeof(EvictCand) == 16, "candidate record");
+
+// Keeps the smaller of two (key, slot) pairs: the lower key, on equal keys the lower slot.
+__device__ __forceinline__ void argmin_merge(unsigned long long& key, int& slot, unsigned long long k2, int s2) {
+    if (k2 < key || (k2 == key && s2 < slot)) {
+        key = k2;
+        slot = s2;
+    }
+}
 
 // Order-preserving map of a float's bits to an unsigned key (for a, b not NaN:
 // a < b  <=>  key(a) < key(b)); -0 is mapped like +0.

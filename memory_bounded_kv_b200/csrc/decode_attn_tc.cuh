@@ -60,6 +60,10 @@ struct DecodeTcParams {
     EvictCand* cand;  // nullable: per-split eviction candidates for position t + 1
     unsigned long long wait_ns;  // limit of every mbarrier wait
     int withhold;     // test hook: the producer issues nothing, so the consumers' first wait runs out
+    // paged cache (PAGED kernels): K, V, pos, log beta in pages of T slots from one pool;
+    // logical slot s of (b, g) is row s % T of page table[(b * Hkv + g) * max_pages + s / T]
+    const int* table;
+    int max_pages, num_pages;
 };
 
 template <int D, int G>
@@ -103,10 +107,6 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, i
             smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
         : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -190,7 +190,7 @@ __device__ __forceinline__ UnitInfo unit_info(const DecodeTcParams& p, int u, Un
     return r;
 }
 
-template <int D, int G, bool BIAS>
+template <int D, int G, bool BIAS, bool PAGED = false>
 __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
     decode_attn_tc_kernel(const __grid_constant__ DecodeTcParams p, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV) {
@@ -271,10 +271,29 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                 stop = true;
                 break;
             }
+            // paged: lane l holds the page of the unit's tile 32 * (i / 32) + l (units start on a page)
+            int lane_page = 0;
+            const size_t trow = PAGED && !end ? ((size_t)ui.b * p.Hkv + ui.g) * p.max_pages + ui.s0 / T : 0;
             for (int i = 0; i < records; ++i, ++it) {
                 const int st = it % ST;
+                int page = 0;
+                if constexpr (PAGED) {
+                    if (!end && (i & 31) == 0) {
+                        int pg = 0;
+                        if (i + lane < ui.ntiles) {
+                            pg = p.table[trow + i + lane];
+                            if (pg < 0 || pg >= p.num_pages) {   // not a page of the pool: read page 0
+                                raise_error(KVB_DERR_RANGE);
+                                pg = 0;
+                            }
+                        }
+                        lane_page = pg;
+                    }
+                    page = __shfl_sync(kFull, lane_page, i & 31);
+                }
                 // this tile's bias (and, for the eviction candidates, its pos and log beta),
                 // loaded before waiting for the stage
+                const size_t mt = PAGED ? (size_t)page * T : m_off + (size_t)i * T;
                 float bias[T / 32];
                 int psv[T / 32];
                 float lbv[T / 32];
@@ -285,9 +304,9 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                     psv[j] = 0;
                     lbv[j] = 0.f;
                     if (!end && key < ui.nk) {
-                        if (BIAS || want_cand) psv[j] = p.pos[m_off + key];
+                        if (BIAS || want_cand) psv[j] = p.pos[mt + lane + 32 * j];
                         if constexpr (BIAS) {
-                            lbv[j] = p.lb[m_off + key];
+                            lbv[j] = p.lb[mt + lane + 32 * j];
                             bv = __fmul_rn(__int2float_rn(tb - psv[j]), lbv[j]);
                         } else {
                             bv = 0.f;
@@ -327,12 +346,14 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                     if (data) {
                         unsigned char* kt = smem + SH::RING_OFF + st * SH::STAGE_BYTES;
                         unsigned char* vt = kt + SH::TILE_BYTES;
-                        const int row = ui.s0 + i * T;
-                        const int bb = p.kv_shared ? 0 : ui.b;
+                        // paged: the page's rows in the pool (one kv head, one "sequence" in the map)
+                        const int row = PAGED ? page * T : ui.s0 + i * T;
+                        const int gg = PAGED ? 0 : ui.g;
+                        const int bb = (PAGED || p.kv_shared) ? 0 : ui.b;
 #pragma unroll
                         for (int h = 0; h < SH::HALVES; ++h) {
-                            tma_load_4d(kt + h * SH::HALF_BYTES, &tmK, 64 * h, row, ui.g, bb, &s_full[st]);
-                            tma_load_4d(vt + h * SH::HALF_BYTES, &tmV, 64 * h, row, ui.g, bb, &s_full[st]);
+                            tma_load_4d(kt + h * SH::HALF_BYTES, &tmK, 64 * h, row, gg, bb, &s_full[st]);
+                            tma_load_4d(vt + h * SH::HALF_BYTES, &tmV, 64 * h, row, gg, bb, &s_full[st]);
                         }
                     }
                     if (with_q) {

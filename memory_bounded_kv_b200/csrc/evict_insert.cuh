@@ -36,13 +36,6 @@ struct EvictParams {
     int cand_n;
 };
 
-__device__ __forceinline__ void argmin_merge(unsigned long long& key, int& slot, unsigned long long k2, int s2) {
-    if (k2 < key || (k2 == key && s2 < slot)) {
-        key = k2;
-        slot = s2;
-    }
-}
-
 template <int NT>
 __global__ void __launch_bounds__(NT) evict_insert_kernel(const __grid_constant__ EvictParams p) {
     __shared__ unsigned long long s_key[NT / 32];

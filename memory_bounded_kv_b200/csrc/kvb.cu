@@ -12,13 +12,16 @@
 
 #include "../../include/kvb.h"
 #include "asm_lookup.cuh"
+#include "asm_planes.cuh"
 #include "asm_hier.cuh"
 #include "asm_build.cuh"
 #include "common.cuh"
 #include "compact_blocks.cuh"
 #include "decode_attn_tc.cuh"
+#include "decode_attn_qb.cuh"
 #include "evict_insert.cuh"
 #include "merge_states.cuh"
+#include "paged.cuh"
 
 namespace {
 
@@ -118,6 +121,18 @@ kvb_status launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem
     return cudaLaunchKernelEx(&cfg, kern, args...) == cudaSuccess ? KVB_OK : KVB_ECUDA;
 }
 
+// The merge of the split states, after either attention kernel.
+template <int D>
+kvb_status launch_merge(const float* o_part, const float* lse_part, int R, int S, void* o, int o_bf16, float* lse,
+                        cudaStream_t st) {
+    // few rows with many splits: a CTA per row keeps more loads in flight per row
+    if (S > 16 && R < 4 * 148)
+        return launch_pdl(kvb::merge_splits_cta_kernel<D>, dim3(R), dim3(256), 0, st, o_part, lse_part, R, S, o,
+                          o_bf16, lse);
+    return launch_pdl(kvb::merge_splits_kernel<D>, dim3((R + 7) / 8), dim3(256), 0, st, o_part, lse_part, R, S, o,
+                      o_bf16, lse);
+}
+
 template <int D, int G, bool BIAS>
 kvb_status launch_decode_tc(const kvb::DecodeTcParams& p, const kvb_attn_args* a, cudaStream_t st) {
     using SH = kvb::TcShape<D, G>;
@@ -136,17 +151,91 @@ kvb_status launch_decode_tc(const kvb::DecodeTcParams& p, const kvb_attn_args* a
     const int per_cta = (p.units + slots - 1) / slots;
     const int grid = (p.units + per_cta - 1) / per_cta;
     if (launch_pdl(kern, dim3(grid), dim3(SH::NT), smem, st, p, mk, mv) != KVB_OK) return KVB_ECUDA;
-    if (p.S > 1) {
-        const int R = a->B * a->Hq;
-        // few rows with many splits: a CTA per row keeps more loads in flight per row
-        if (p.S > 16 && R < 4 * 148)
-            return launch_pdl(kvb::merge_splits_cta_kernel<D>, dim3(R), dim3(256), 0, st,
-                              static_cast<const float*>(p.o_part), static_cast<const float*>(p.lse_part), R, p.S,
-                              p.o, p.o_bf16, p.lse);
-        return launch_pdl(kvb::merge_splits_kernel<D>, dim3((R + 7) / 8), dim3(256), 0, st,
-                          static_cast<const float*>(p.o_part), static_cast<const float*>(p.lse_part), R, p.S,
-                          p.o, p.o_bf16, p.lse);
+    if (p.S > 1)
+        return launch_merge<D>(p.o_part, p.lse_part, a->B * a->Hq, p.S, p.o, p.o_bf16, p.lse, st);
+    return KVB_OK;
+}
+
+template <int D, int G, bool BIAS>
+kvb_status launch_decode_qb(const kvb::DecodeQbParams& p, const kvb_attn_args* a, cudaStream_t st) {
+    using SH = kvb::QbShape<D, G>;
+    auto kern = kvb::decode_attn_qb_kernel<D, G, BIAS>;
+    const size_t smem = SH::SMEM;
+    if (set_smem(kern, smem) != KVB_OK) return KVB_ECUDA;
+    CUtensorMap mk, mv;
+    if (!make_kv_map(&mk, a->k, D, a->cap, a->Hkv, 1, a->kv_stride_h, 0, SH::T) ||
+        !make_kv_map(&mv, a->v, D, a->cap, a->Hkv, 1, a->kv_stride_h, 0, SH::T))
+        return KVB_EINVAL;
+    const int slots = resident_ctas(kern, SH::NT, smem);
+    if (slots <= 0) return KVB_ECUDA;
+    const int per_cta = (p.units + slots - 1) / slots;
+    const int grid = (p.units + per_cta - 1) / per_cta;
+    if (launch_pdl(kern, dim3(grid), dim3(SH::NT), smem, st, p, mk, mv) != KVB_OK) return KVB_ECUDA;
+    if (p.S > 1)
+        return launch_merge<D>(p.o_part, p.lse_part, a->B * a->Hq, p.S, p.o, p.o_bf16, p.lse, st);
+    return KVB_OK;
+}
+
+template <int D>
+kvb_status qb_dispatch(const kvb::DecodeQbParams& p, const kvb_attn_args* a, int G, bool bias, cudaStream_t st) {
+    switch (G) {
+        case 1: return bias ? launch_decode_qb<D, 1, true>(p, a, st) : launch_decode_qb<D, 1, false>(p, a, st);
+        case 2: return bias ? launch_decode_qb<D, 2, true>(p, a, st) : launch_decode_qb<D, 2, false>(p, a, st);
+        case 4: return bias ? launch_decode_qb<D, 4, true>(p, a, st) : launch_decode_qb<D, 4, false>(p, a, st);
+        case 8: return bias ? launch_decode_qb<D, 8, true>(p, a, st) : launch_decode_qb<D, 8, false>(p, a, st);
+        default: return KVB_EINVAL;
     }
+}
+
+// Attention over a paged cache: the tensor maps cover the page pool ([pages * T rows, d]).
+template <int D, int G, bool BIAS>
+kvb_status launch_decode_paged(const kvb::DecodeTcParams& p, const kvb_paged_cache* c, int Hq, cudaStream_t st) {
+    using SH = kvb::TcShape<D, G>;
+    static_assert(SH::T == kvb::kPageSlots, "a tile is a page");
+    auto kern = kvb::decode_attn_tc_kernel<D, G, BIAS, true>;
+    const size_t smem = SH::SMEM;
+    if (set_smem(kern, smem) != KVB_OK) return KVB_ECUDA;
+    CUtensorMap mk, mv;
+    const int rows = c->num_pages * kvb::kPageSlots;
+    if (!make_kv_map(&mk, c->k_pages, D, rows, 1, 1, 0, 0, SH::T) ||
+        !make_kv_map(&mv, c->v_pages, D, rows, 1, 1, 0, 0, SH::T))
+        return KVB_EINVAL;
+    const int slots = resident_ctas(kern, SH::NT, smem);
+    if (slots <= 0) return KVB_ECUDA;
+    const int per_cta = (p.units + slots - 1) / slots;
+    const int grid = (p.units + per_cta - 1) / per_cta;
+    if (launch_pdl(kern, dim3(grid), dim3(SH::NT), smem, st, p, mk, mv) != KVB_OK) return KVB_ECUDA;
+    if (p.S > 1) return launch_merge<D>(p.o_part, p.lse_part, c->B * Hq, p.S, p.o, p.o_bf16, p.lse, st);
+    return KVB_OK;
+}
+
+template <int D>
+kvb_status paged_dispatch(const kvb::DecodeTcParams& p, const kvb_paged_cache* c, int Hq, int G, bool bias,
+                          cudaStream_t st) {
+    switch (G) {
+        case 1: return bias ? launch_decode_paged<D, 1, true>(p, c, Hq, st) : launch_decode_paged<D, 1, false>(p, c, Hq, st);
+        case 2: return bias ? launch_decode_paged<D, 2, true>(p, c, Hq, st) : launch_decode_paged<D, 2, false>(p, c, Hq, st);
+        case 4: return bias ? launch_decode_paged<D, 4, true>(p, c, Hq, st) : launch_decode_paged<D, 4, false>(p, c, Hq, st);
+        case 8: return bias ? launch_decode_paged<D, 8, true>(p, c, Hq, st) : launch_decode_paged<D, 8, false>(p, c, Hq, st);
+        default: return KVB_EINVAL;
+    }
+}
+
+// Host checks shared by the paged entry points; fills the kernels' view of the cache.
+kvb_status paged_view(const kvb_paged_cache* c, kvb::PagedCache* out) {
+    if (c == nullptr) return KVB_EINVAL;
+    if (c->B < 1 || c->Hkv < 1 || c->d < 8 || c->d > 1024 || (c->d % 8) || c->max_pages < 1 || c->num_pages < 1)
+        return KVB_EINVAL;
+    if ((long long)c->B * c->Hkv > 0x7fffffffLL || (long long)c->max_pages * kvb::kPageSlots > 0x7fffffffLL ||
+        (long long)c->num_pages * kvb::kPageSlots > 0x7fffffffLL)
+        return KVB_EINVAL;
+    if (!c->k_pages || !c->v_pages || !c->pos_pages || !c->table || !c->len || !c->free_pages || !c->free_count)
+        return KVB_EINVAL;
+    if (!aligned16(c->k_pages) || !aligned16(c->v_pages) || !aligned16(c->pos_pages) ||
+        (c->log_beta_pages && !aligned16(c->log_beta_pages)))
+        return KVB_EINVAL;
+    *out = kvb::PagedCache{c->k_pages, c->v_pages, c->log_beta_pages, c->pos_pages, c->table, c->len,
+                           c->free_pages, c->free_count, c->Hkv, c->d, c->max_pages, c->num_pages};
     return KVB_OK;
 }
 
@@ -281,6 +370,27 @@ kvb_status kvb_decode_attn(const kvb_attn_args* a, kvb_stream stream) {
         }
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // many rows over one shared cache (and shared log beta / pos): the query-batched kernel reads
+    // every K/V tile once per block of rows. Needs split boundaries common to all rows (a fixed
+    // split length, or one split) and no eviction candidates (they are per row).
+    const bool meta_shared = (a->log_beta == nullptr && a->pos == nullptr) || a->meta_stride_b == 0;
+    if (p.kv_shared && meta_shared && a->evict_cand == nullptr && (a->num_splits == 1 || a->split_len > 0)) {
+        kvb::DecodeQbParams q;
+        q.q = a->q; q.q_sb = a->q_stride_b; q.q_sh = a->q_stride_h;
+        q.lb = a->log_beta; q.pos = a->pos; q.m_sh = a->meta_stride_h;
+        q.len = a->len; q.t = a->t;
+        q.B = a->B; q.Hq = a->Hq; q.Hkv = a->Hkv; q.cap = a->cap; q.S = a->num_splits; q.split_len = a->split_len;
+        const int BQ = 16 / G;
+        q.blocks = (a->B + BQ - 1) / BQ;
+        const long long qunits = (long long)q.blocks * a->Hkv * a->num_splits;
+        if (qunits > 0x7fffffffLL) return KVB_EINVAL;
+        q.units = (int)qunits;
+        q.scale = p.scale;
+        q.o_part = a->o_part; q.lse_part = a->lse_part;
+        q.o = a->o; q.o_bf16 = p.o_bf16; q.lse = a->lse;
+        q.wait_ns = p.wait_ns; q.withhold = p.withhold;
+        return a->d == 128 ? qb_dispatch<128>(q, a, G, bias, st) : qb_dispatch<64>(q, a, G, bias, st);
+    }
     return a->d == 128 ? tc_g<128>(p, a, G, bias, st) : tc_g<64>(p, a, G, bias, st);
 }
 
@@ -361,6 +471,86 @@ kvb_status kvb_compact_blocks(uint16_t* k, uint16_t* v, int32_t* pos, float* log
     return launched();
 }
 
+kvb_status kvb_paged_reset(const kvb_paged_cache* c, kvb_stream stream) {
+    kvb::PagedCache pc;
+    if (paged_view(c, &pc) != KVB_OK) return KVB_EINVAL;
+    const long long rows = (long long)c->B * c->Hkv;
+    const long long n = std::max((long long)c->num_pages, rows * c->max_pages);
+    kvb::paged_reset_kernel<<<(unsigned)std::min<long long>((n + 255) / 256, 65535), 256, 0,
+                              static_cast<cudaStream_t>(stream)>>>(pc, c->B);
+    return launched();
+}
+
+kvb_status kvb_paged_evict_insert(const kvb_paged_cache* c, const uint16_t* k_new, const uint16_t* v_new,
+                                  const float* log_beta_new, const int32_t* t, int32_t M, int32_t* victim,
+                                  const void* cand, int32_t cand_n, kvb_stream stream) {
+    kvb::PagedCache pc;
+    if (paged_view(c, &pc) != KVB_OK) return KVB_EINVAL;
+    if (!t || M < 1 || (long long)M > (long long)c->max_pages * kvb::kPageSlots) return KVB_EINVAL;
+    if ((k_new == nullptr) != (v_new == nullptr)) return KVB_EINVAL;
+    if (k_new && (!aligned16(k_new) || !aligned16(v_new))) return KVB_EINVAL;
+    if (c->log_beta_pages && !log_beta_new) return KVB_EINVAL;
+    if (cand != nullptr && (cand_n < 1 || cand_n > 1024 || (reinterpret_cast<uintptr_t>(cand) & 15u))) return KVB_EINVAL;
+    kvb::PagedEvictParams p{pc, k_new, v_new, log_beta_new, t, M, victim, static_cast<const kvb::EvictCand*>(cand),
+                            cand_n};
+    return launch_pdl(kvb::paged_evict_insert_kernel<256>, dim3(c->B * c->Hkv), dim3(256), 0,
+                      static_cast<cudaStream_t>(stream), p);
+}
+
+kvb_status kvb_paged_compact_blocks(const kvb_paged_cache* c, const int32_t* rm_start, const int32_t* rm_len,
+                                    kvb_stream stream) {
+    kvb::PagedCache pc;
+    if (paged_view(c, &pc) != KVB_OK) return KVB_EINVAL;
+    if (!rm_start || !rm_len) return KVB_EINVAL;
+    const int row_bytes = 2 * c->d * 2 + 8;
+    int W = 32768 / row_bytes;
+    W = W < 1 ? 1 : (W > 64 ? 64 : W);
+    kvb::PagedCompactParams p{pc, rm_start, rm_len, W};
+    const size_t smem = (size_t)W * row_bytes;
+    return launch_pdl(kvb::paged_compact_kernel<256>, dim3(c->B * c->Hkv), dim3(256), smem,
+                      static_cast<cudaStream_t>(stream), p);
+}
+
+kvb_status kvb_paged_decode_attn(const kvb_paged_cache* c, const uint16_t* q, const int32_t* t, int32_t Hq,
+                                 float scale, int32_t num_splits, int32_t split_len, float* o_part, float* lse_part,
+                                 void* o, int32_t o_dtype, float* lse, void* evict_cand, kvb_stream stream) {
+    kvb::PagedCache pc;
+    if (paged_view(c, &pc) != KVB_OK) return KVB_EINVAL;
+    if (c->d != 64 && c->d != 128) return KVB_EINVAL;
+    if (Hq < 1 || Hq % c->Hkv != 0) return KVB_EINVAL;
+    const int G = Hq / c->Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return KVB_EINVAL;
+    if (c->B > 65535 || c->Hkv > 65535 || (long long)c->B * Hq > 0x7fffffffLL) return KVB_EINVAL;
+    if (num_splits < 1 || num_splits > 1024 || split_len < 0) return KVB_EINVAL;
+    // every split starts on a page: one split, or a split length that is a multiple of a page
+    if (num_splits > 1 && (split_len == 0 || split_len % kvb::kPageSlots != 0)) return KVB_EINVAL;
+    if (!std::isfinite(scale) || !q || !o || !aligned16(q)) return KVB_EINVAL;
+    const bool bias = c->log_beta_pages != nullptr;
+    if ((bias || evict_cand) && !t) return KVB_EINVAL;
+    if (evict_cand && (reinterpret_cast<uintptr_t>(evict_cand) & 15u)) return KVB_EINVAL;
+    if (o_dtype != KVB_OUT_F32 && o_dtype != KVB_OUT_BF16) return KVB_EINVAL;
+    if (num_splits > 1 && (!o_part || !lse_part)) return KVB_EINVAL;
+    if ((o_part == nullptr) != (lse_part == nullptr)) return KVB_EINVAL;
+    const long long units = (long long)c->B * c->Hkv * num_splits;
+    if (units > 0x7fffffffLL) return KVB_EINVAL;
+    kvb::DecodeTcParams p{};
+    p.q = q; p.q_sb = (long long)Hq * c->d; p.q_sh = c->d;
+    p.lb = c->log_beta_pages; p.pos = c->pos_pages; p.m_sb = 0; p.m_sh = 0;
+    p.len = c->len; p.t = t;
+    p.Hq = Hq; p.Hkv = c->Hkv; p.cap = c->max_pages * kvb::kPageSlots; p.S = num_splits; p.split_len = split_len;
+    p.units = (int)units;
+    p.kv_shared = 0;
+    p.scale = (scale == 0.0f) ? (float)(1.0 / std::sqrt((double)c->d)) : scale;
+    p.o_part = o_part; p.lse_part = lse_part;
+    p.o = o; p.o_bf16 = (o_dtype == KVB_OUT_BF16); p.lse = lse;
+    p.cand = static_cast<kvb::EvictCand*>(evict_cand);
+    p.wait_ns = 1000000000ull;
+    p.withhold = 0;
+    p.table = c->table; p.max_pages = c->max_pages; p.num_pages = c->num_pages;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return c->d == 128 ? paged_dispatch<128>(p, c, Hq, G, bias, st) : paged_dispatch<64>(p, c, Hq, G, bias, st);
+}
+
 size_t kvb_asm_workspace_bytes(int32_t N, int32_t H, int32_t K) {
     if (N < 1 || H < 1 || K < 1) return 0;
     return (size_t)kvb::asm_ksplit(K) * N * H * sizeof(unsigned long long);
@@ -398,6 +588,61 @@ kvb_status kvb_asm_lookup_merge_grouped(const uint16_t* q, const float* qbar, co
     if (launched() != KVB_OK) return KVB_ECUDA;
     const long long rows = (long long)N * H;
     kvb::asm_merge_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p);
+    return launched();
+}
+
+size_t kvb_asm_planes_bytes(int32_t H_tables, int32_t K) {
+    if (H_tables < 1 || K < 1) return 0;
+    return (size_t)H_tables * kvb::asm_plane_tiles(K) * kvb::kPImg;
+}
+
+kvb_status kvb_asm_prepare(const float* qbar, int32_t H_tables, int32_t K, int32_t d, void* planes,
+                           size_t planes_bytes, kvb_stream stream) {
+    if (d != kvb::kAsmD || H_tables < 1 || K < 1 || !qbar || !planes) return KVB_EINVAL;
+    if (!aligned16(qbar) || !aligned16(planes) || planes_bytes < kvb_asm_planes_bytes(H_tables, K)) return KVB_EINVAL;
+    const long long rows = (long long)H_tables * (long long)kvb::asm_plane_tiles(K) * kvb::kUKT;
+    if ((rows + 7) / 8 > 0x7fffffffLL) return KVB_EINVAL;
+    kvb::asm_prepare_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        qbar, H_tables, K, static_cast<unsigned char*>(planes));
+    return launched();
+}
+
+kvb_status kvb_asm_lookup_merge_planes(const uint16_t* q, const void* planes, size_t planes_bytes,
+                                       const uint16_t* abar, const float* log_zbar, const float* o_self,
+                                       const float* lse_self, int32_t N, int32_t H, int32_t H_tables, int32_t K,
+                                       int32_t d, int32_t* idx, float* o, float* lse, void* workspace,
+                                       size_t workspace_bytes, kvb_stream stream) {
+    if (d != kvb::kAsmD || N < 1 || H < 1 || K < 1 || H > 65535) return KVB_EINVAL;
+    if (H_tables < 1 || H % H_tables != 0) return KVB_EINVAL;
+    if (!q || !planes || !workspace) return KVB_EINVAL;
+    if (planes_bytes < kvb_asm_planes_bytes(H_tables, K)) return KVB_EINVAL;
+    if (o == nullptr) {   // assignment only
+        if (idx == nullptr) return KVB_EINVAL;
+    } else if (!abar || !log_zbar || !o_self || !lse_self || !aligned16(abar) || !aligned16(o_self) ||
+               !aligned16(o)) {
+        return KVB_EINVAL;
+    }
+    if (!aligned16(q) || !aligned16(planes) || !aligned16(workspace)) return KVB_EINVAL;
+    if (workspace_bytes < kvb_asm_workspace_bytes(N, H, K)) return KVB_EINVAL;
+    const int qtiles = (N + kvb::kUMT * kvb::kUQ - 1) / (kvb::kUMT * kvb::kUQ);
+    const long long items = (long long)H * qtiles * kvb::asm_ksplit(K);
+    if (items > (1ll << 30)) return KVB_EINVAL;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (set_smem(kvb::asm_score_planes_kernel, kvb::kPSmem) != KVB_OK) return KVB_ECUDA;
+    const int slots = resident_ctas(kvb::asm_score_planes_kernel, kvb::kPThreads, kvb::kPSmem);
+    if (slots < 1) return KVB_ECUDA;
+    const int per_cta = (int)((items + slots - 1) / slots);
+    const int grid = (int)((items + per_cta - 1) / per_cta);
+    kvb::AsmPlanesParams pp;
+    pp.a = kvb::AsmParams{q, nullptr, abar, log_zbar, o_self, lse_self, N, H, K, kvb::asm_ksplit(K),
+                          kvb::asm_kchunk(K), qtiles, per_cta, idx, o, lse, static_cast<unsigned long long*>(workspace),
+                          H / H_tables};
+    pp.planes = static_cast<const unsigned char*>(planes);
+    pp.wait_ns = 1000000000ull;
+    kvb::asm_score_planes_kernel<<<grid, kvb::kPThreads, kvb::kPSmem, st>>>(pp);
+    if (launched() != KVB_OK) return KVB_ECUDA;
+    const long long rows = (long long)N * H;
+    kvb::asm_merge_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(pp.a);
     return launched();
 }
 

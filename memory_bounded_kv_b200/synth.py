@@ -116,13 +116,14 @@ _DECODE_CONFIGS = {
 CONFIG3_LOGICAL_T = 131072
 
 
-def decode_workload(cfg: int, B: int | None = None, prefill: int | None = None) -> DecodeWorkload:
+def decode_workload(cfg: int, B: int | None = None, prefill: int | None = None,
+                    seed: int | None = None) -> DecodeWorkload:
     """Prefilled cache of decode workload 1 (tiny), 2 (Qwen3-8B-shaped) or 3 (long context).
 
     Prefill writes positions 0..prefill-1 into slots 0..prefill-1 (no eviction
     while the cache is within budget). `B` may shrink the batch (the first B
     sequences of the full draw are not reproduced; a smaller B is a different,
-    smaller workload of the same shape).
+    smaller workload of the same shape). `seed` replaces the workload's own seed.
 
     For the long-context workload the returned cache is the starting point of the streaming
     build (positions 0..8191); the caller streams positions 8192..131071
@@ -132,6 +133,8 @@ def decode_workload(cfg: int, B: int | None = None, prefill: int | None = None) 
     c = dict(_DECODE_CONFIGS[cfg])
     if B is not None:
         c["B"] = B
+    if seed is not None:
+        c["seed"] = int(seed)
     P = c.pop("prefill")
     if prefill is not None:
         P = prefill
@@ -327,6 +330,25 @@ class MementoWorkload:
 
     def compaction_steps(self) -> np.ndarray:
         return np.unique(np.cumsum(self.blk + self.mem, axis=1) - 1)
+
+    def len_trajectory(self) -> np.ndarray:
+        """[steps, B] int64: every sequence's length after the insertion of each step (before that
+        step's compaction); finished sequences keep their mementos."""
+        steps = np.arange(self.steps)
+        ends = np.cumsum(self.blk + self.mem, axis=1) - 1                  # [B, nblk] compaction steps
+        out = np.zeros((self.steps, self.B), np.int64)
+        for b in range(self.B):
+            # blocks removed before step i: compactions at steps < i
+            removed = np.zeros(self.steps + 1, np.int64)
+            np.add.at(removed, ends[b] + 1, self.blk[b])
+            removed = np.cumsum(removed)[: self.steps]
+            out[:, b] = np.where(steps < self.total[b], steps + 1 - removed, self.mem[b].sum())
+        return out
+
+    def peak_pages(self, page: int = 64) -> int:
+        """The most pages of `page` slots a paged cache of this schedule holds at once (all kv heads)."""
+        n = self.len_trajectory()
+        return int((self.Hkv * (-(-n // page))).sum(axis=1).max())
 
     def cache_len(self, step: int) -> np.ndarray:
         """len of every sequence after the insertion of step `step` and before its compaction."""

@@ -119,3 +119,27 @@ def test_other_entry_points_reject_bad_arguments_on_the_host():
     ws = L.kvb_asm_workspace_bytes(256, 32, 4096)
     assert ws == 32 * 256 * 32 * 8   # 32 ranges of 128 centroids, one 8-byte key per (range, query, head)
     assert L.kvb_asm_lookup_merge(f, f, f, f, f, f, 256, 32, 4096, 128, None, f, None, f, ws - 1, None) == _lib.KVB_EINVAL
+
+
+def test_paged_and_planes_entry_points_reject_bad_arguments_on_the_host():
+    L = _lib.lib()
+    f = 1 << 20
+    pc = _lib.PagedCacheArgs(k_pages=f, v_pages=f, log_beta_pages=None, pos_pages=f, table=f, len=f, free_pages=f,
+                             free_count=f, B=2, Hkv=2, d=128, max_pages=4, num_pages=16)
+    p = ctypes.c_void_p(f)
+    # several splits must start on pages: split_len a positive multiple of 64
+    assert L.kvb_paged_decode_attn(ctypes.byref(pc), p, p, 8, 0.0, 2, 0, p, p, p, 0, None, None, None) == _lib.KVB_EINVAL
+    assert L.kvb_paged_decode_attn(ctypes.byref(pc), p, p, 8, 0.0, 2, 100, p, p, p, 0, None, None, None) == _lib.KVB_EINVAL
+    assert L.kvb_paged_decode_attn(ctypes.byref(pc), p, p, 12, 0.0, 1, 0, None, None, p, 0, None, None, None) == _lib.KVB_EINVAL
+    # budget above the capacity of the table
+    assert L.kvb_paged_evict_insert(ctypes.byref(pc), p, p, None, p, 4 * 64 + 1, None, None, 0, None) == _lib.KVB_EINVAL
+    bad = _lib.PagedCacheArgs(k_pages=f + 8, v_pages=f, log_beta_pages=None, pos_pages=f, table=f, len=f,
+                              free_pages=f, free_count=f, B=2, Hkv=2, d=128, max_pages=4, num_pages=16)
+    assert L.kvb_paged_reset(ctypes.byref(bad), None) == _lib.KVB_EINVAL
+    assert L.kvb_paged_compact_blocks(ctypes.byref(pc), None, p, None) == _lib.KVB_EINVAL
+    # prepared memory: size of the planes, and refusals
+    assert L.kvb_asm_planes_bytes(2, 100) == 2 * 2 * 3 * 2 * 64 * 128
+    assert L.kvb_asm_prepare(p, 2, 100, 64, p, 1 << 30, None) == _lib.KVB_EINVAL
+    assert L.kvb_asm_prepare(p, 2, 100, 128, p, 1000, None) == _lib.KVB_EINVAL
+    assert L.kvb_asm_lookup_merge_planes(p, p, 1000, p, p, p, p, 4, 2, 2, 100, 128, None, p, None, p, 1 << 20,
+                                         None) == _lib.KVB_EINVAL

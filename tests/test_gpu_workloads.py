@@ -155,7 +155,7 @@ def test_memory_lookup_workload_full(oracle):
     l_self = torch.zeros(N, H, device="cuda")
     op, lp = kvb.decode_workspace(N, H, d, 4)
     kvb.kvb_decode_attn(dev(w.q), kd, vd, None, posd, dev(w.len), dev(w.t), o_self, l_self, num_splits=4,
-                        o_part=op, lse_part=lp)
+                        split_len=512, o_part=op, lse_part=lp)
     os_ref, ls_ref = oracle.decode_attn(w.q, w.k, w.v, None, w.pos, w.len, w.t, kv_batch_stride=0,
                                         meta_batch_stride=0)
     assert_state_close(host(o_self), host(l_self), os_ref, ls_ref, "self attention")
