@@ -54,7 +54,7 @@ struct QbShape {
     static constexpr int NWC = 4;
     static constexpr int NT = (NWC + 1) * 32;
     static constexpr int T = 16 * NWC;
-    static constexpr int STAGES = 3;
+    static constexpr int STAGES = 2;              // two CTAs per SM: 8 consumer warps hide the MMA latency
     static constexpr int HALVES = D / 64;
     static constexpr int HALF_BYTES = T * 128;
     static constexpr int TILE_BYTES = HALVES * HALF_BYTES;
@@ -112,7 +112,7 @@ __device__ __forceinline__ void qb_empty_row(const DecodeQbParams& p, int blk, i
 }
 
 template <int D, int G, bool BIAS>
-__global__ void __launch_bounds__(QbShape<D, G>::NT, 1)
+__global__ void __launch_bounds__(QbShape<D, G>::NT, 2)
     decode_attn_qb_kernel(const __grid_constant__ DecodeQbParams p, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV) {
     using SH = QbShape<D, G>;
@@ -332,16 +332,25 @@ __global__ void __launch_bounds__(QbShape<D, G>::NT, 1)
             }
             const uint32_t kt = ring + st * SH::STAGE_BYTES;
             const uint32_t vt = kt + SH::TILE_BYTES;
-            // ---- S = Q K^T for this warp's 16 slots (two n-tiles of 8), all 16 query rows
+            // ---- S = Q K^T for this warp's 16 slots (two n-tiles of 8), all 16 query rows; even and
+            // odd K steps accumulate separately (two independent chains), then add
             float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            float sd[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
             for (int s = 0; s < SH::KSTEPS; ++s) {
                 const int chunk = 2 * (s & 3) + kq_hi;
                 const uint32_t addr = kt + (s >> 2) * SH::HALF_BYTES + kq_row * 128 + ((chunk ^ sw) << 4);
                 uint32_t b0, b1, b2, b3;
                 ldsm_x4(addr, b0, b1, b2, b3);
-                mma_bf16_16(sc[0], qa[s][0], qa[s][1], qa[s][2], qa[s][3], b0, b1);
-                mma_bf16_16(sc[1], qa[s][0], qa[s][1], qa[s][2], qa[s][3], b2, b3);
+                float (&c0)[4] = (s & 1) ? sd[0] : sc[0];
+                float (&c1)[4] = (s & 1) ? sd[1] : sc[1];
+                mma_bf16_16(c0, qa[s][0], qa[s][1], qa[s][2], qa[s][3], b0, b1);
+                mma_bf16_16(c1, qa[s][0], qa[s][1], qa[s][2], qa[s][3], b2, b3);
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                sc[0][j] += sd[0][j];
+                sc[1][j] += sd[1][j];
             }
             if (rows < T && kw + 16 > rows) {
                 // tail: zero this warp's V rows past the unit's last slot (K there is masked)

@@ -155,9 +155,10 @@ struct UnitRaw {
     int len, t;
 };
 
-__device__ __forceinline__ UnitRaw unit_raw(const DecodeTcParams& p, int u) {
+__device__ __forceinline__ UnitRaw unit_raw(const DecodeTcParams& p, long long ul) {
     UnitRaw r{0, 0};
-    if (u < p.units) {
+    if (ul < p.units) {
+        const int u = (int)ul;
         const int per_b = p.Hkv * p.S;
         const int b = u / per_b;
         const int g = (u - b * per_b) / p.S;
@@ -231,11 +232,13 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
         // ======================= producer warp =======================
         int it = 0;
         bool stop = false;
-        UnitRaw next_raw = unit_raw(p, blockIdx.x);
-        for (int u = blockIdx.x; u < p.units + gridDim.x && !stop; u += gridDim.x) {
+        // lane l holds the length and position of this CTA's unit 32 * (k / 32) + l: one round trip
+        // per 32 units, so that empty units (ragged lengths) cost no load latency each
+        UnitRaw lane_raw{0, 0};
+        for (int u = blockIdx.x, k = 0; u < p.units + gridDim.x && !stop; u += gridDim.x, ++k) {
             const bool end = u >= p.units;  // one end record after the last unit
-            const UnitRaw raw = next_raw;
-            next_raw = unit_raw(p, u + gridDim.x);  // in flight while this unit's tiles are issued
+            if ((k & 31) == 0) lane_raw = unit_raw(p, (long long)u + (long long)lane * gridDim.x);
+            const UnitRaw raw{__shfl_sync(kFull, lane_raw.len, k & 31), __shfl_sync(kFull, lane_raw.t, k & 31)};
             UnitInfo ui{};
             if (!end) ui = unit_info<T>(p, u, raw, lane == 0);
             if (!end && ui.ntiles == 0) {
