@@ -84,6 +84,12 @@ def parse(argv=None):
     ap.add_argument("--check", default="sampled", choices=["sampled", "full", "off"],
                     help="after timing, one more step computed two ways on the GPU (the timed path and an "
                          "independent one) and compared (sampled: cache bytes of a few sequences; full: all)")
+    ap.add_argument("--dump-state", default=None, metavar="DIR",
+                    help="write the cache state before the checked step and that step's inputs as raw files "
+                         "under DIR/<workload> (decode and memento workloads)")
+    ap.add_argument("--replay", default=None, metavar="DIR",
+                    help="instead of timing, run the step dumped under DIR once and write its outputs and "
+                         "the cache after it under DIR/replayed")
     ap.add_argument("--impl", default="kvb", choices=["kvb", "reference"])
     ap.add_argument("--splits", type=int, default=0, help="num_splits of the headline workload (0: its default)")
     ap.add_argument("--no-e2e", action="store_true")
@@ -450,6 +456,11 @@ class DecodeBench:
                 "num_splits": self.S, "beta": "1" if self.plain else "sigmoid(N(2,1.5))", "seed": w.seed,
                 "l2": l2, "parallelism": "replicas (independent sequences per GPU)"}
 
+    def dump_step(self, i, path):
+        """The cache before the step at position t0 + i and that step's inputs."""
+        from memory_bounded_kv_b200.state import dump_step
+        dump_step(path, self.cache, self.host_inputs(i), extra_meta={"workload": self.workload, "step": int(i)})
+
     def check(self, i, full: bool):
         """Consistency of one more step (position t0 + i) computed two ways on the GPU from the same
         cache: the timed path (eviction from the attention's candidates, the workload's splits) and
@@ -753,6 +764,14 @@ class MementoBench:
                 "peak_kv_full_over_compacted": round(self.peak_kv_ratio(), 3), "memory": self.memory(),
                 "l2": "flushed before every timed step (256 MiB write): the live caches grow from "
                       "a few MB to ~350 MB over the schedule"}
+
+    def dump_step(self, i, path):
+        """The cache before schedule step i and its inputs (the compaction only at a compaction step)."""
+        from memory_bounded_kv_b200.state import dump_step
+        x = self.host_inputs(i)
+        if i not in self.comp:
+            x.pop("rm_start"), x.pop("rm_len")
+        dump_step(path, self.cache, x, extra_meta={"workload": self.workload, "step": int(i)})
 
     def check(self, i, full: bool):
         """Consistency of schedule step i: the timed path (eviction candidates, splits of 512
@@ -1109,6 +1128,10 @@ def run_workload(key, splits, args, world, local, K, W, hbm_peak, peak_kind, cpu
     r["config"] = bench.config()
     r["config"]["timed_launches"] = "cuda graph replay"
     r["clocks"] = clk
+    if args.dump_state and hasattr(bench, "dump_step"):
+        path = os.path.join(args.dump_state, key)
+        log(f"{key}: dumping the state before step {m['next']} to {path}")
+        bench.dump_step(m["next"], path)
     if args.check != "off":
         log(f"{key}: consistency check")
         r["consistency"] = bench.check(m["next"], args.check == "full")
@@ -1119,6 +1142,23 @@ def run_workload(key, splits, args, world, local, K, W, hbm_peak, peak_kind, cpu
     del bench
     torch.cuda.empty_cache()
     return r
+
+
+def run_replay(path):
+    """One dumped step through the library: its outputs and the cache after it go to
+    path/replayed (same format), with the device error word."""
+    from memory_bounded_kv_b200 import kvb_get_error
+    from memory_bounded_kv_b200 import state
+    cache, inputs, meta = state.load_step(path)
+    o, lse = state.replay_step(cache, inputs)
+    torch.cuda.synchronize()
+    err = kvb_get_error()
+    tensors, _ = state.cache_state(cache)
+    tensors = dict(tensors, out_o=o, out_lse=lse)
+    out = os.path.join(path, "replayed")
+    state.save(out, tensors, dict(meta, device_error=err))
+    return {"replay": path, "written": out, "device_error": err, "workload": meta.get("extra", {}).get("workload"),
+            "o_finite": bool(torch.isfinite(o).all().item()), "lse_finite": bool(torch.isfinite(lse).all().item())}
 
 
 def run_kvb(args, world, rank, local):
@@ -1373,6 +1413,9 @@ def main():
         return
     if args.asm_build:
         print(json.dumps(run_asm_build(args)), flush=True)
+        return
+    if args.replay:
+        print(json.dumps(run_replay(args.replay)), flush=True)
         return
     world, rank, local = dist_init()
     try:
