@@ -217,19 +217,22 @@ __global__ void __launch_bounds__(kUThreads, 1) asm_score_umma_kernel(const __gr
             tc_fence_after();
             const int mts = min(kUMT, (p.N - cm.qt * (kUMT * kUQ) + kUQ - 1) / kUQ);
             if (lane == 0) {
-                for (int mt = 0; mt < mts; ++mt) {
-                    const uint32_t d = tmem + (uint32_t)((b * kUMT + mt) * kUKT);
+                // the M tiles' products alternate (independent accumulators back to back)
 #pragma unroll
-                    for (int pt = 0; pt < 3; ++pt)
+                for (int pt = 0; pt < 3; ++pt)
 #pragma unroll
-                        for (int kk = 0; kk < kAsmD / 16; ++kk) {
-                            // descriptors advance in 16-byte units of the start address
+                    for (int kk = 0; kk < kAsmD / 16; ++kk) {
+                        // descriptors advance in 16-byte units of the start address
+                        const uint32_t boff =
+                            (uint32_t)(b * kUBuf + pt * kUPart + (kk >> 2) * kUPartHalf + (kk & 3) * 32);
+#pragma unroll
+                        for (int mt = 0; mt < kUMT; ++mt) {
+                            if (mt >= mts) break;
+                            const uint32_t d = tmem + (uint32_t)((b * kUMT + mt) * kUKT);
                             const uint32_t aoff = (uint32_t)(mt * 2 * kUAHalf + (kk >> 2) * kUAHalf + (kk & 3) * 32);
-                            const uint32_t boff =
-                                (uint32_t)(b * kUBuf + pt * kUPart + (kk >> 2) * kUPartHalf + (kk & 3) * 32);
                             umma_bf16(d, a0 + (aoff >> 4), b0 + (boff >> 4), idesc, (pt | kk) != 0);
                         }
-                }
+                    }
                 umma_commit(&bar[b]);
             }
             __syncwarp();
@@ -266,7 +269,8 @@ __global__ void __launch_bounds__(kUThreads, 1) asm_score_umma_kernel(const __gr
 
         auto readback = [&](int g) {
             const int b = g & 1;
-            if (!mbar_wait(&bar[b], (unsigned)(g >> 1) & 1u)) ok = false;
+            // warp-uniform outcome: the tensor-memory loads below are warp-collective
+            if (!__all_sync(kFull, mbar_wait(&bar[b], (unsigned)(g >> 1) & 1u))) ok = false;
             tc_fence_after();
             const int n0 = ce.qt * (kUMT * kUQ);
             const int mts = min(kUMT, (p.N - n0 + kUQ - 1) / kUQ);

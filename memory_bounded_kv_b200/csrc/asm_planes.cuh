@@ -6,13 +6,14 @@
 // shared-memory image the tensor-core MMA reads: [part][K half][64 rows][128 B],
 // 16-byte chunk c of row r at chunk c ^ (r & 7) (the 128-byte swizzle).
 //
-// asm_score_planes_kernel then streams those images with one bulk copy per
-// tile into a 3-stage ring and keeps the queries in tensor memory as the A
-// operand of tcgen05.mma (so each MMA reads only its 2 KB B slice from shared
+// asm_score_planes_kernel then streams those images with bulk copies into a
+// ring of shared-memory stages and keeps the queries in tensor memory as the
+// A operand of tcgen05.mma (so each MMA reads only its 2 KB B slice from shared
 // memory), with three accumulator buffers:
-//   warp 9 (one lane)  bulk copies of the tile images           -> b_full[s]
+//   warp 9 (one lane)  bulk copies of the tile images (six 8 KB pieces)  -> b_full[s]
 //   warp 8 (one lane)  48 MMAs per tile (2 M tiles x 3 parts x 8 K steps),
 //                      committed to b_empty[s] and acc_full[b]
+// The ring has four stages, the accumulators three buffers (s = g % 4, b = g % 3).
 //   warps 0-7          the queries into tensor memory (tcgen05.st) at each new
 //                      block of 256 queries (-> a_ready), then per tile: read
 //                      their query row's 64 scores back (tcgen05.ld), release
@@ -25,15 +26,18 @@
 
 namespace kvb {
 
-constexpr int kPStages = 3;                                    // B ring stages == accumulator buffers
+constexpr int kPStages = 4;                                    // B ring stages
+constexpr int kPAcc = 3;                                       // accumulator buffers
 constexpr size_t kPImg = 3 * kUPart;                           // one tile image: 48 KB
+constexpr int kPPieces = 6;                                    // copies per tile: one per (part, K half)
 constexpr int kPThreads = kUNT + 64;                           // 8 read-back warps + MMA warp + copy warp
 constexpr int kPACols = kUMT * (kAsmD / 2);                    // queries: 2 M tiles x 64 columns
 constexpr int kPAccCols = kUMT * kUKT;                         // one accumulator buffer: 2 x 64 columns
-constexpr int kPCols = 512;                                    // kPACols + kPStages * kPAccCols
+constexpr int kPCols = 512;                                    // kPACols + kPAcc * kPAccCols
 constexpr size_t kPBar = (size_t)kPStages * kPImg;             // after the ring
-constexpr size_t kPSmem = kPBar + 128 + 1024;                  // barriers + slot, + alignment slack
-static_assert(kPACols + kPStages * kPAccCols == kPCols, "tensor memory budget");
+constexpr size_t kPSmem = kPBar + 192 + 1024;                  // barriers + slot, + alignment slack
+static_assert(kPACols + kPAcc * kPAccCols == kPCols, "tensor memory budget");
+static_assert(kPImg % kPPieces == 0 && (kPImg / kPPieces) % 1024 == 0, "pieces");
 
 __host__ __device__ inline size_t asm_plane_tiles(int K) { return (size_t)(K + kUKT - 1) / kUKT; }
 
@@ -104,8 +108,8 @@ __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __
     uint64_t* b_full = reinterpret_cast<uint64_t*>(sm + kPBar);
     uint64_t* b_empty = b_full + kPStages;
     uint64_t* acc_full = b_empty + kPStages;
-    uint64_t* acc_empty = acc_full + kPStages;
-    uint64_t* a_ready = acc_empty + kPStages;
+    uint64_t* acc_empty = acc_full + kPAcc;
+    uint64_t* a_ready = acc_empty + kPAcc;
     uint32_t* slot = reinterpret_cast<uint32_t*>(a_ready + 1);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int items = p.H * p.qtiles * p.ksplit;
@@ -128,8 +132,10 @@ __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __
         for (int s = 0; s < kPStages; ++s) {
             mbar_init(&b_full[s], 1);
             mbar_init(&b_empty[s], 1);
-            mbar_init(&acc_full[s], 1);
-            mbar_init(&acc_empty[s], kUNT / 32);
+        }
+        for (int b = 0; b < kPAcc; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], kUNT / 32);
         }
         mbar_init(a_ready, kUNT / 32);
         fence_mbar_init();
@@ -153,7 +159,10 @@ __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __
                 }
                 mbar_arrive_expect_tx(&b_full[s], (unsigned)kPImg);
                 const unsigned char* src = pp.planes + ((size_t)(c.h / p.G) * tiles_per_table + c.kt / kUKT) * kPImg;
-                bulk_g2s(sm + (size_t)s * kPImg, src, (unsigned)kPImg, &b_full[s]);
+#pragma unroll
+                for (int pc = 0; pc < kPPieces; ++pc)
+                    bulk_g2s(sm + (size_t)s * kPImg + pc * (kPImg / kPPieces), src + pc * (kPImg / kPPieces),
+                             (unsigned)(kPImg / kPPieces), &b_full[s]);
                 asm_tile_next(p, c);
             }
         }
@@ -166,9 +175,9 @@ __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __
             const uint64_t b0 = umma_desc_sw128(sbase);
             int a_block = -1, a_phase = 0;
             for (int g = 0; g < G; ++g) {
-                const int s = g % kPStages;
+                const int s = g % kPStages, ab = g % kPAcc;
                 if (!mbar_wait(&b_full[s], (unsigned)(g / kPStages) & 1u, pp.wait_ns)) { ok = false; break; }
-                if (g >= kPStages && !mbar_wait(&acc_empty[s], (unsigned)((g / kPStages) - 1) & 1u, pp.wait_ns)) {
+                if (g >= kPAcc && !mbar_wait(&acc_empty[ab], (unsigned)((g / kPAcc) - 1) & 1u, pp.wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -179,21 +188,25 @@ __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __
                     a_block = blk;
                 }
                 tc_fence_after();
+                // the two M tiles' products alternate: consecutive MMAs go to independent
+                // accumulators, so each one's accumulation does not wait for the one before
                 const int mts = min(kUMT, (p.N - cm.qt * (kUMT * kUQ) + kUQ - 1) / kUQ);
-                for (int mt = 0; mt < mts; ++mt) {
-                    const uint32_t d = tmem + (uint32_t)(kPACols + s * kPAccCols + mt * kUKT);
 #pragma unroll
-                    for (int pt = 0; pt < 3; ++pt)
+                for (int pt = 0; pt < 3; ++pt)
 #pragma unroll
-                        for (int kk = 0; kk < kAsmD / 16; ++kk) {
+                    for (int kk = 0; kk < kAsmD / 16; ++kk) {
+                        const uint32_t boff =
+                            (uint32_t)(s * kPImg + pt * kUPart + (kk >> 2) * kUPartHalf + (kk & 3) * 32);
+#pragma unroll
+                        for (int mt = 0; mt < kUMT; ++mt) {
+                            if (mt >= mts) break;
+                            const uint32_t d = tmem + (uint32_t)(kPACols + ab * kPAccCols + mt * kUKT);
                             const uint32_t a = tmem + (uint32_t)(mt * (kAsmD / 2) + kk * 8);
-                            const uint32_t boff =
-                                (uint32_t)(s * kPImg + pt * kUPart + (kk >> 2) * kUPartHalf + (kk & 3) * 32);
                             umma_bf16_ts(d, a, b0 + (boff >> 4), idesc, (pt | kk) != 0);
                         }
-                }
+                    }
                 umma_commit(&b_empty[s]);
-                umma_commit(&acc_full[s]);
+                umma_commit(&acc_full[ab]);
                 asm_tile_next(p, cm);
             }
         }
@@ -206,7 +219,7 @@ __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __
         int bidx = -1;
         int a_block = -1;
         for (int g = 0; g < G; ++g) {
-            const int s = g % kPStages;
+            const int s = g % kPAcc;   // the accumulator buffer of tile g
             const int blk = ce.h * p.qtiles + ce.qt;
             const int n0 = ce.qt * (kUMT * kUQ);
             if (blk != a_block) {
@@ -234,7 +247,7 @@ __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __
                 if (lane == 0) mbar_arrive(a_ready);
                 a_block = blk;
             }
-            if (!mbar_wait(&acc_full[s], (unsigned)(g / kPStages) & 1u, pp.wait_ns)) ok = false;
+            if (!__all_sync(kFull, mbar_wait(&acc_full[s], (unsigned)(g / kPAcc) & 1u, pp.wait_ns))) ok = false;
             tc_fence_after();
             const int mts = min(kUMT, (p.N - n0 + kUQ - 1) / kUQ);
             float v[kUKT];
@@ -246,7 +259,7 @@ __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[s]);   // the buffer may take tile g + 3
+            if (lane == 0) mbar_arrive(&acc_empty[s]);   // the buffer may take tile g + kPAcc
             if (ok && emt < mts) {
                 if (ce.kt + kUKT > ce.k_end) {   // ragged last tile of a range
 #pragma unroll
@@ -288,7 +301,7 @@ __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __
     __syncthreads();
     if (warp == kUNT / 32 && lane == 0 && G > 0) {
         // the last tile's MMAs complete before the tensor memory is released (bounded)
-        mbar_wait(&acc_full[(G - 1) % kPStages], (unsigned)((G - 1) / kPStages) & 1u, pp.wait_ns);
+        mbar_wait(&acc_full[(G - 1) % kPAcc], (unsigned)((G - 1) / kPAcc) & 1u, pp.wait_ns);
     }
     __syncthreads();
     if (warp == 0) {

@@ -1,0 +1,568 @@
+// Query-batched decode attention over one shared cache on the 5th-generation
+// tensor cores: the same computation as decode_attn_qb_kernel (many rows b
+// over one cache with batch stride 0, each with its own length and position;
+// "Cache What Lasts" section 2.1 logits, "Context Memorization" core method
+// step 1 state, splits of a fixed length), with 128 query rows per unit:
+// a unit is (block of 128 / G rows b, kv head g, split j), so every K/V tile
+// is read once per 128 query rows and both products run as tcgen05.mma with
+// the accumulators in tensor memory.
+//
+// Roles (192 threads, one CTA per SM):
+//   warp 0     producer: the unit's 128 query rows by TMA (a 3-D box of 64
+//              dims x G heads x 128 / G rows b, K-major with the 128-byte
+//              swizzle, two buffers), K/V tiles by TMA into a 3-stage ring with
+//              their pos / log beta (bias) and the tile's record;
+//   warp 1     MMA issuer (one lane): S = Q K^T (M = 128, N = 64, K = 128)
+//              into one of two S buffers, and O += P V (M = 128, N = 128,
+//              K = 64) with P read from tensor memory (A operand) and V from
+//              shared memory as an MN-major B operand; S(i + 1) is issued
+//              before P V(i), so the softmax of tile i overlaps the next QK;
+//   warps 2-5  softmax, one query row per thread (tensor-memory lane = row):
+//              read S, mask by the row's length, add the row's bias, keep the
+//              running maximum and sum, write P as a bf16 high part and a
+//              bf16 residual (two products each, ~16 bits of P) into tensor
+//              memory; at the end of the unit read O and write the state.
+// The running maximum is updated lazily: P is formed against a reference
+// maximum and O is rescaled (read, scaled, written back in tensor memory)
+// only when a row's maximum exceeds the reference by more than 2^8 in the
+// exponent, so P <= 256; the result is the same softmax.
+// Every wait is bounded (wait_ns); a CTA that gives up records
+// KVB_DERR_TIMEOUT, lets its copies and MMAs finish (bounded) and writes the
+// empty state for every unit it owns.
+#pragma once
+
+#include <cuda.h>
+
+#include "asm_planes.cuh"
+#include "decode_attn_qb.cuh"
+
+namespace kvb {
+
+template <int G>
+struct QbtShape {
+    static constexpr int D = 128;
+    static constexpr int R = 128;             // query rows per unit = tensor-memory lanes
+    static constexpr int BQ = R / G;          // rows b per unit
+    static constexpr int T = 64;              // slots per tile
+    static constexpr int ST = 3;              // K/V ring stages
+    static constexpr int NT = 6 * 32;
+    static constexpr int QHALF = R * 128;     // 128 rows x 64 dims of bf16
+    static constexpr int QBUF = 2 * QHALF;
+    static constexpr int KVHALF = T * 128;
+    static constexpr int KVTILE = 2 * KVHALF;
+    static constexpr int STAGE = 2 * KVTILE;  // K tile, V tile
+    static constexpr int META = 16 + 2 * 64;  // tile record + (first tile) the rows' lengths, positions
+    static constexpr int Q_OFF = 0;
+    static constexpr int RING_OFF = Q_OFF + 2 * QBUF;
+    static constexpr int POS_OFF = RING_OFF + ST * STAGE;
+    static constexpr int LB_OFF = POS_OFF + ST * T * 4;
+    static constexpr int META_OFF = LB_OFF + ST * T * 4;
+    static constexpr int BAR_OFF = (META_OFF + ST * META * 4 + 7) / 8 * 8;
+    static constexpr int NBAR = 2 * ST + 14;  // kv full/empty; q, s, p full/empty, pv_done x 2; o_free; fin
+    static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+    static constexpr int END = MISC_OFF + 32;
+    static constexpr size_t SMEM = 1024 + END;
+    static constexpr int TM_O = 0, TM_S = 128, TM_P = 256, TM_COLS = 512;
+    static_assert(G == 2 || G == 4 || G == 8, "G");
+    static_assert(BQ <= 64, "rows per unit");
+    static_assert(RING_OFF % 1024 == 0 && STAGE % 1024 == 0, "alignment");
+};
+
+// kind::f16 instruction descriptor with an MN-major B operand (bit 16)
+__host__ __device__ constexpr uint32_t umma_idesc_bf16_bmn(int M, int N) { return umma_idesc_bf16(M, N) | (1u << 16); }
+
+// A bounded wait whose outcome is the same for the whole warp (the warp then runs warp-collective
+// tensor-memory instructions or leaves together).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, unsigned parity, unsigned long long ns) {
+    return __all_sync(kFull, mbar_wait(bar, parity, ns));
+}
+
+// Shared-memory descriptor of an MN-major operand in the 128-byte swizzle: 64-element MN groups
+// `lbo` bytes apart, 8-row K groups `sbo` bytes apart.
+__device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+template <int G, bool BIAS>
+__global__ void __launch_bounds__(QbtShape<G>::NT, 1)
+    decode_attn_qbt_kernel(const __grid_constant__ DecodeQbParams p, const __grid_constant__ CUtensorMap tmK,
+                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQ) {
+    using SH = QbtShape<G>;
+    constexpr int D = SH::D, R = SH::R, BQ = SH::BQ, T = SH::T, ST = SH::ST;
+    extern __shared__ unsigned char smem_dyn[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_u32(smem);
+    int* s_pos = reinterpret_cast<int*>(smem + SH::POS_OFF);
+    float* s_lb = reinterpret_cast<float*>(smem + SH::LB_OFF);
+    int* s_meta = reinterpret_cast<int*>(smem + SH::META_OFF);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SH::BAR_OFF);
+    uint64_t* kv_full = bars;
+    uint64_t* kv_empty = bars + ST;
+    uint64_t* q_full = bars + 2 * ST;
+    uint64_t* q_empty = q_full + 2;
+    uint64_t* s_full = q_empty + 2;
+    uint64_t* s_empty = s_full + 2;
+    uint64_t* p_full = s_empty + 2;
+    uint64_t* p_empty = p_full + 2;
+    // P V of tile i is committed to pv_done[i & 1]: a tile's softmax knows that P V(i - 2) is done
+    // (it follows S(i)) and P V(i + 1) not issued, so a parity wait for P V(i - 1) or P V(i) on its
+    // own barrier can never be two phases behind
+    uint64_t* pv_done = p_empty + 2;
+    uint64_t* o_free = pv_done + 2;
+    uint64_t* fin = o_free + 1;   // the MMA warp's last commit: every tensor-core operation done
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + SH::MISC_OFF);
+    volatile int* s_abort = reinterpret_cast<int*>(smem + SH::MISC_OFF) + 1;
+    int* s_issued = reinterpret_cast<int*>(smem + SH::MISC_OFF) + 2;   // tiles the producer issued
+    int* s_mma = reinterpret_cast<int*>(smem + SH::MISC_OFF) + 3;      // PV products the MMA warp committed
+    int* s_qloads = reinterpret_cast<int*>(smem + SH::MISC_OFF) + 4;   // query blocks the producer loaded
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    griddep_wait();
+    griddep_launch_dependents();
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tslot)),
+                     "r"(SH::TM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (tid == 0) {
+        for (int s = 0; s < ST; ++s) {
+            mbar_init(&kv_full[s], 33);   // the copy's expect_tx + 32 producer lanes
+            mbar_init(&kv_empty[s], 1);   // the MMA warp's commit after P V
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&q_full[b], 1);     // the producer's expect_tx; the copy's bytes
+            mbar_init(&q_empty[b], 1);
+            mbar_init(&s_full[b], 1);
+            mbar_init(&s_empty[b], 4);    // the 4 softmax warps
+            mbar_init(&p_full[b], 4);
+            mbar_init(&p_empty[b], 1);
+        }
+        mbar_init(&pv_done[0], 1);
+        mbar_init(&pv_done[1], 1);
+        mbar_init(o_free, 4);
+        mbar_init(fin, 1);
+        *s_abort = 0;
+        *s_issued = 0;
+        *s_mma = 0;
+        *s_qloads = 0;
+        fence_mbar_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
+    const int per_blk = p.Hkv * p.S;
+
+    if (warp == 0) {
+        // ======================= producer =======================
+        int it = 0, ucount = 0;
+        bool stop = false;
+        for (int u = blockIdx.x; u < p.units + gridDim.x && !stop; u += gridDim.x) {
+            const bool end = u >= p.units;
+            int blk = 0, g = 0, split = 0, s0 = 0, nk = 0, ntiles = 0;
+            int len_r[2] = {0, 0}, t_r[2] = {0, 0};   // rows lane, lane + 32 of the block
+            if (!end) {
+                blk = u / per_blk;
+                g = (u - blk * per_blk) / p.S;
+                split = u - blk * per_blk - g * p.S;
+                int maxlen = 0;
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    const int bq = lane + 32 * k, b = blk * BQ + bq;
+                    if (bq < BQ && b < p.B) {
+                        const int n = p.len[(size_t)b * p.Hkv + g];
+                        const int tt = (p.t == nullptr) ? 0 : p.t[b];
+                        const bool active = (p.t == nullptr) || tt >= 0;
+                        const bool bad_len = n < 0 || n > p.cap;
+                        const bool bad_split =
+                            !bad_len && p.split_len > 0 && (long long)n > (long long)p.S * p.split_len;
+                        if ((bad_len || bad_split) && split == 0) raise_error(bad_len ? KVB_DERR_LEN : KVB_DERR_SPLIT);
+                        len_r[k] = (bad_len || bad_split || !active) ? 0 : n;
+                        t_r[k] = tt;
+                    }
+                    maxlen = max(maxlen, len_r[k]);
+                }
+#pragma unroll
+                for (int m = 16; m >= 1; m >>= 1) maxlen = max(maxlen, __shfl_xor_sync(kFull, maxlen, m));
+                const long long C = p.split_len > 0 ? (long long)p.split_len : (long long)maxlen;
+                s0 = (int)min((long long)split * C, (long long)maxlen);
+                const int s1 = (int)min((long long)s0 + C, (long long)maxlen);
+                nk = s1 - s0;
+                ntiles = (nk + T - 1) / T;
+                if (ntiles == 0) {
+                    for (int r = 0; r < R; ++r) {
+                        const int b = blk * BQ + r / G;
+                        if (b >= p.B) continue;
+                        const size_t row = (size_t)b * p.Hq + g * G + r % G;
+                        if (lane == 0 && p.o_part != nullptr) p.lse_part[row * p.S + split] = -INFINITY;
+                        if (p.S == 1) {
+                            for (int e = lane; e < D; e += 32) {
+                                if (p.o_bf16) {
+                                    reinterpret_cast<__nv_bfloat16*>(p.o)[row * D + e] = __float2bfloat16_rn(0.f);
+                                } else {
+                                    reinterpret_cast<float*>(p.o)[row * D + e] = 0.f;
+                                }
+                            }
+                            if (lane == 0 && p.lse != nullptr) p.lse[row] = -INFINITY;
+                        }
+                    }
+                    continue;
+                }
+            }
+            if (p.withhold) {   // test hook: no copy, no arrival; the other roles' waits run out
+                stop = true;
+                break;
+            }
+            int qb = 0;
+            if (!end) {
+                // the unit's queries into buffer qb (free once the MMAs of the unit two back are done):
+                // rows b = blk * BQ .. (zeros past B), heads g * G .., both 64-dim halves
+                qb = ucount & 1;
+                if (ucount >= 2 && !warp_wait(&q_empty[qb], (unsigned)((ucount >> 1) - 1) & 1u, p.wait_ns)) {
+                    if (lane == 0) {
+                        raise_error(KVB_DERR_TIMEOUT);
+                        *s_abort = 1;
+                    }
+                    break;
+                }
+                if (lane == 0) {
+                    unsigned char* qbuf = smem + SH::Q_OFF + qb * SH::QBUF;
+                    mbar_arrive_expect_tx(&q_full[qb], (unsigned)SH::QBUF);
+                    tma_load_4d(qbuf, &tmQ, 0, g * G, blk * BQ, 0, &q_full[qb]);
+                    tma_load_4d(qbuf + SH::QHALF, &tmQ, 64, g * G, blk * BQ, 0, &q_full[qb]);
+                }
+                ++ucount;
+            }
+            const int records = end ? 1 : ntiles;
+            const size_t m_off = end ? 0 : (size_t)g * p.m_sh + (size_t)s0;
+            for (int i = 0; i < records; ++i, ++it) {
+                const int st = it % ST;
+                int psv[2];
+                float lbv[2];
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int key = i * T + lane + 32 * j;
+                    psv[j] = 0;
+                    lbv[j] = 0.f;
+                    if (BIAS && !end && key < nk) {
+                        psv[j] = p.pos[m_off + key];
+                        lbv[j] = p.lb[m_off + key];
+                    }
+                }
+                if (it >= ST && !warp_wait(&kv_empty[st], (unsigned)((it / ST) - 1) & 1u, p.wait_ns)) {
+                    if (lane == 0) {
+                        raise_error(KVB_DERR_TIMEOUT);
+                        *s_abort = 1;
+                    }
+                    stop = true;
+                    break;
+                }
+                if (__any_sync(kFull, *s_abort != 0)) {
+                    stop = true;
+                    break;
+                }
+                int* m = s_meta + st * SH::META;
+                if (lane == 0) {
+                    m[0] = end ? -1 : u;
+                    m[1] = i;
+                    m[2] = end ? 0 : ntiles;
+                    m[3] = end ? 0 : min(T, nk - i * T);
+                    m[4] = blk;
+                    m[5] = g;
+                    m[6] = split;
+                    m[7] = s0 + i * T;
+                    m[8] = s0 + nk;
+                    m[9] = qb;
+                    mbar_arrive_expect_tx(&kv_full[st], end ? 0u : (unsigned)SH::STAGE);
+                    if (!end) {
+                        unsigned char* kt = smem + SH::RING_OFF + st * SH::STAGE;
+                        unsigned char* vt = kt + SH::KVTILE;
+                        const int row = s0 + i * T;
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            tma_load_4d(kt + h * SH::KVHALF, &tmK, 64 * h, row, g, 0, &kv_full[st]);
+                            tma_load_4d(vt + h * SH::KVHALF, &tmV, 64 * h, row, g, 0, &kv_full[st]);
+                        }
+                    }
+                }
+                if (!end && i == 0) {
+#pragma unroll
+                    for (int k = 0; k < 2; ++k)
+                        if (lane + 32 * k < BQ) {
+                            m[16 + lane + 32 * k] = len_r[k];
+                            m[16 + 64 + lane + 32 * k] = t_r[k];
+                        }
+                }
+                if (BIAS) {
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        s_pos[st * T + lane + 32 * j] = psv[j];
+                        s_lb[st * T + lane + 32 * j] = lbv[j];
+                    }
+                }
+                __syncwarp();
+                mbar_arrive(&kv_full[st]);
+            }
+        }
+        if (lane == 0) {
+            *s_issued = it;
+            *s_qloads = ucount;
+        }
+    } else if (warp == 1) {
+        // ======================= MMA issuer =======================
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = umma_idesc_bf16(R, T);          // S: 128 x 64
+            constexpr uint32_t idesc_o = umma_idesc_bf16_bmn(R, D);      // O: 128 x 128, V MN-major
+            int i = 0, units_pv = 0, pv = 0, units_qk = 0;
+            bool pending = false;
+            int pend_st = 0, pend_first = 0, pend_i = 0;
+            auto fail = [&]() {
+                raise_error(KVB_DERR_TIMEOUT);
+                *s_abort = 1;
+            };
+            auto issue_pv = [&](int st, int pi, int first) -> bool {
+                const int pb = pi & 1;
+                if (!mbar_wait(&p_full[pb], (unsigned)(pi >> 1) & 1u, p.wait_ns)) return false;
+                if (first && units_pv > 0 && !mbar_wait(o_free, (unsigned)(units_pv - 1) & 1u, p.wait_ns)) return false;
+                if (first) ++units_pv;
+                tc_fence_after();
+                const uint32_t vt = sbase + SH::RING_OFF + st * SH::STAGE + SH::KVTILE;
+#pragma unroll
+                for (int part = 0; part < 2; ++part)
+#pragma unroll
+                    for (int kk = 0; kk < T / 16; ++kk) {
+                        const uint32_t a = tmem + SH::TM_P + pb * 64 + part * 32 + kk * 8;
+                        const uint64_t bd = umma_desc_sw128_mn(vt + kk * 2048, SH::KVHALF, 1024);
+                        umma_bf16_ts(tmem + SH::TM_O, a, bd, idesc_o, (first && part == 0 && kk == 0) ? 0u : 1u);
+                    }
+                umma_commit(&kv_empty[st]);
+                umma_commit(&p_empty[pb]);
+                umma_commit(&pv_done[pb]);
+                ++pv;
+                return true;
+            };
+            while (true) {
+                const int st = i % ST;
+                if (!mbar_wait(&kv_full[st], (unsigned)(i / ST) & 1u, p.wait_ns)) { fail(); break; }
+                const int* m = s_meta + st * SH::META;
+                const int u = m[0];
+                if (u < 0) {   // the end: the last P V
+                    if (pending && !issue_pv(pend_st, pend_i, pend_first)) fail();
+                    break;
+                }
+                const int ti = m[1], ntiles = m[2], qb = m[9];
+                const int sb = i & 1;
+                // S(i) = Q K^T into buffer sb; a unit's first tile waits for its queries (the k-th unit
+                // uses query buffer k % 2 for the (k / 2)-th time)
+                if (ti == 0) {
+                    if (!mbar_wait(&q_full[qb], (unsigned)(units_qk >> 1) & 1u, p.wait_ns)) { fail(); break; }
+                    ++units_qk;
+                }
+                if (i >= 2 && !mbar_wait(&s_empty[sb], (unsigned)((i >> 1) - 1) & 1u, p.wait_ns)) { fail(); break; }
+                tc_fence_after();
+                const uint32_t qa = sbase + SH::Q_OFF + qb * SH::QBUF;
+                const uint32_t kt = sbase + SH::RING_OFF + st * SH::STAGE;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t aoff = (kk >> 2) * SH::QHALF + (kk & 3) * 32;
+                    const uint32_t boff = (kk >> 2) * SH::KVHALF + (kk & 3) * 32;
+                    umma_bf16(tmem + SH::TM_S + sb * 64, umma_desc_sw128(qa + aoff), umma_desc_sw128(kt + boff),
+                              idesc_s, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&s_full[sb]);
+                if (ti == ntiles - 1) umma_commit(&q_empty[qb]);
+                // P V of the previous tile, now that the tensor cores have the next S queued
+                if (pending && !issue_pv(pend_st, pend_i, pend_first)) { fail(); break; }
+                pending = true;
+                pend_st = st;
+                pend_i = i;
+                pend_first = (ti == 0);
+                ++i;
+            }
+            *s_mma = pv;
+        }
+    } else {
+        // ======================= softmax warps =======================
+        const int quarter = warp & 3;             // tensor-memory lanes 32 * quarter ..
+        const int r = 32 * quarter + lane;        // this thread's query row
+        const uint32_t tl = tmem + ((uint32_t)(32 * quarter) << 16);
+        const float L2E = kLog2e;
+        float m_ref = -INFINITY, l_sum = 0.f;
+        int lim = 0, trow = 0;
+        for (int i = 0;; ++i) {
+            const int st = i % ST;
+            if (!warp_wait(&kv_full[st], (unsigned)(i / ST) & 1u, p.wait_ns)) break;
+            const int* m = s_meta + st * SH::META;
+            const int u = m[0];
+            if (u < 0) break;
+            const int ti = m[1], ntiles = m[2], rows = m[3], ublk = m[4], ug = m[5], usplit = m[6], base = m[7],
+                      s1 = m[8];
+            if (rows < T) {
+                // V rows past the unit's last slot may hold any bytes: zero them (their P is 0, and
+                // 0 times a NaN would not be); the tensor cores read them only in P V(i), after p_full
+                unsigned char* vt = smem + SH::RING_OFF + st * SH::STAGE + SH::KVTILE;
+                for (int idx = r; idx < (T - rows) * 16; idx += R) {
+                    const int row = rows + (idx >> 4), c = idx & 15;
+                    *reinterpret_cast<uint4*>(vt + (c >> 3) * SH::KVHALF + row * 128 + (((c & 7) ^ (row & 7)) << 4)) =
+                        make_uint4(0u, 0u, 0u, 0u);
+                }
+                fence_proxy_async_smem();
+            }
+            if (ti == 0) {
+                lim = min(m[16 + r / G], s1);
+                trow = m[16 + 64 + r / G];
+                m_ref = -INFINITY;
+                l_sum = 0.f;
+            }
+            const int sb = i & 1;
+            if (!warp_wait(&s_full[sb], (unsigned)(i >> 1) & 1u, p.wait_ns)) break;
+            tc_fence_after();
+            float x[T];
+            tmem_ld32(tl + SH::TM_S + sb * 64, x);
+            tmem_ld32(tl + SH::TM_S + sb * 64 + 32, x + 32);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_empty[sb]);
+            float mt = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < T; ++j) {
+                float bj = 0.f;
+                if constexpr (BIAS) bj = __fmul_rn(__int2float_rn(trow - s_pos[st * T + j]), s_lb[st * T + j]);
+                x[j] = (base + j < lim) ? fmaf(x[j], p.scale, bj) : -INFINITY;
+                mt = fmaxf(mt, x[j]);
+            }
+            // the reference moves when the row's maximum passes it by more than 2^8; the rows that
+            // had one already rescale O. Tensor-memory loads and stores are warp-collective, so the
+            // whole warp takes the rescale when any of its rows needs it (the others scale by 1).
+            const bool grow = mt > m_ref && (m_ref == -INFINITY || (mt - m_ref) * L2E > 8.f);
+            const bool resc = grow && m_ref != -INFINITY;
+            if (__any_sync(kFull, resc)) {
+                // every earlier P V product of this unit first (P V(i - 1); i > 0 here)
+                if (!warp_wait(&pv_done[(i - 1) & 1], (unsigned)((i - 1) >> 1) & 1u, p.wait_ns)) break;
+                tc_fence_after();
+                const float alpha = resc ? exp2f((m_ref - mt) * L2E) : 1.f;
+#pragma unroll
+                for (int c = 0; c < D; c += 32) {
+                    float o[32];
+                    tmem_ld32(tl + SH::TM_O + c, o);
+                    tmem_ld_wait();
+                    uint32_t w[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) w[e] = __float_as_uint(o[e] * alpha);
+                    tmem_st32(tl + SH::TM_O + c, w);
+                }
+                tmem_st_wait();
+                l_sum *= alpha;
+            }
+            if (grow) m_ref = mt;
+            const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+            uint32_t hi[T / 2], lo[T / 2];
+            float ssum = 0.f;
+#pragma unroll
+            for (int j = 0; j < T; j += 2) {
+                const float p0 = exp2f((x[j] - m_use) * L2E), p1 = exp2f((x[j + 1] - m_use) * L2E);
+                ssum += p0 + p1;
+                hi[j / 2] = pack_bf16(p0, p1);
+                lo[j / 2] = pack_bf16(p0 - __uint_as_float(hi[j / 2] << 16), p1 - __uint_as_float(hi[j / 2] & 0xffff0000u));
+            }
+            l_sum += ssum;
+            const int pb = i & 1;
+            if (i >= 2 && !warp_wait(&p_empty[pb], (unsigned)((i >> 1) - 1) & 1u, p.wait_ns)) break;
+            tc_fence_after();
+            tmem_st32(tl + SH::TM_P + pb * 64, hi);
+            tmem_st32(tl + SH::TM_P + pb * 64 + 32, lo);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[pb]);
+            if (ti != ntiles - 1) continue;
+
+            // ---- end of unit: O of this row, divided by the sum; the split's state
+            if (!warp_wait(&pv_done[i & 1], (unsigned)(i >> 1) & 1u, p.wait_ns)) break;
+            tc_fence_after();
+            float o[D];
+#pragma unroll
+            for (int c = 0; c < D; c += 32) tmem_ld32(tl + SH::TM_O + c, o + c);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(o_free);
+            const int b = ublk * BQ + r / G;
+            if (b < p.B) {
+                const size_t row = (size_t)b * p.Hq + ug * G + r % G;
+                const float inv = (l_sum > 0.f) ? 1.f / l_sum : 0.f;
+                const float lse = (l_sum > 0.f) ? m_ref + log2f(l_sum) * kLn2 : -INFINITY;
+                if (p.o_part != nullptr) {
+                    float4* dst = reinterpret_cast<float4*>(p.o_part + (row * p.S + usplit) * D);
+#pragma unroll
+                    for (int e = 0; e < D; e += 4)
+                        dst[e / 4] = make_float4(o[e] * inv, o[e + 1] * inv, o[e + 2] * inv, o[e + 3] * inv);
+                    p.lse_part[row * p.S + usplit] = lse;
+                }
+                if (p.S == 1) {
+                    if (p.o_bf16) {
+                        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.o) + row * D;
+#pragma unroll
+                        for (int e = 0; e < D; ++e) dst[e] = __float2bfloat16_rn(o[e] * inv);
+                    } else {
+                        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.o) + row * D);
+#pragma unroll
+                        for (int e = 0; e < D; e += 4)
+                            dst[e / 4] = make_float4(o[e] * inv, o[e + 1] * inv, o[e + 2] * inv, o[e + 3] * inv);
+                    }
+                    if (p.lse != nullptr) p.lse[row] = lse;
+                }
+            }
+        }
+    }
+
+    // ---- teardown: copies and MMAs in flight finish (bounded) before the tensor memory goes
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1 && lane == 0) {
+        umma_commit(fin);   // arrives when every tensor-core operation this thread issued is done
+        mbar_wait(fin, 0u, p.wait_ns);
+    }
+    if (tid == 0 && *s_abort) {
+        const int issued = *s_issued;
+        for (int k = max(0, issued - ST); k < issued; ++k)
+            mbar_wait(&kv_full[k % ST], (unsigned)(k / ST) & 1u, 100000000ull);
+        // query copies: at most one in flight per buffer (the one before it was consumed)
+        const int ql = *s_qloads;
+        for (int k = max(0, ql - 2); k < ql; ++k) mbar_wait(&q_full[k & 1], (unsigned)(k >> 1) & 1u, 100000000ull);
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(SH::TM_COLS) : "memory");
+    }
+    if (!*s_abort) return;
+    // a CTA that gave up leaves every unit it owns in the empty state
+    for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
+        const int blk = u / per_blk;
+        const int g = (u - blk * per_blk) / p.S;
+        const int split = u - blk * per_blk - g * p.S;
+        for (int r = warp; r < R; r += 6) {
+            const int b = blk * BQ + r / G;
+            if (b >= p.B) continue;
+            const size_t row = (size_t)b * p.Hq + g * G + r % G;
+            if (lane == 0 && p.o_part != nullptr) p.lse_part[row * p.S + split] = -INFINITY;
+            if (p.S == 1) {
+                for (int e = lane; e < D; e += 32) {
+                    if (p.o_bf16) {
+                        reinterpret_cast<__nv_bfloat16*>(p.o)[row * D + e] = __float2bfloat16_rn(0.f);
+                    } else {
+                        reinterpret_cast<float*>(p.o)[row * D + e] = 0.f;
+                    }
+                }
+                if (lane == 0 && p.lse != nullptr) p.lse[row] = -INFINITY;
+            }
+        }
+    }
+}
+
+}  // namespace kvb

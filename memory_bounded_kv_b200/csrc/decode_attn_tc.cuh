@@ -232,12 +232,14 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
         // ======================= producer warp =======================
         int it = 0;
         bool stop = false;
+        // this CTA's units: blockIdx.x, blockIdx.x + gridDim.x, ... (round robin)
+        const int u_lo = blockIdx.x, u_hi = p.units, u_step = gridDim.x;
         // lane l holds the length and position of this CTA's unit 32 * (k / 32) + l: one round trip
         // per 32 units, so that empty units (ragged lengths) cost no load latency each
         UnitRaw lane_raw{0, 0};
-        for (int u = blockIdx.x, k = 0; u < p.units + gridDim.x && !stop; u += gridDim.x, ++k) {
-            const bool end = u >= p.units;  // one end record after the last unit
-            if ((k & 31) == 0) lane_raw = unit_raw(p, (long long)u + (long long)lane * gridDim.x);
+        for (int u = u_lo, k = 0; !stop; u += u_step, ++k) {
+            const bool end = u >= u_hi;  // one end record after the last unit
+            if ((k & 31) == 0) lane_raw = unit_raw(p, (long long)u + (long long)lane * u_step);
             const UnitRaw raw{__shfl_sync(kFull, lane_raw.len, k & 31), __shfl_sync(kFull, lane_raw.t, k & 31)};
             UnitInfo ui{};
             if (!end) ui = unit_info<T>(p, u, raw, lane == 0);
@@ -381,6 +383,7 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                 __syncwarp();
                 mbar_arrive(&s_full[st]);
             }
+            if (end) break;
         }
         if (lane == 0) *s_issued = it;
     } else {
@@ -417,7 +420,7 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
             const int* m = s_meta + st * 16;
             const int u = m[0], i = m[1], ntiles = m[2], rows = m[3];
             if (u < 0) break;
-            const int ub = m[4], ug = m[5], usplit = m[6];
+            const int ub = m[4], ug = m[5], usplit = m[6], ut = m[8];   // (read before the stage is released)
             if (i == 0) {
                 cand_key = ~0ull;
                 cand_slot = 0x7fffffff;
@@ -577,7 +580,7 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                 EvictCand* c = p.cand + ((size_t)ub * p.Hkv + ug) * p.S + usplit;
                 c->key = bk;
                 c->slot = (bk == ~0ull) ? -1 : bs;
-                c->t = m[8] + 1;
+                c->t = ut + 1;
             }
             const int S = p.S;
             for (int idx = tid; idx < G * D; idx += NWC * 32) {

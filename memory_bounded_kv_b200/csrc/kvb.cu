@@ -19,6 +19,7 @@
 #include "compact_blocks.cuh"
 #include "decode_attn_tc.cuh"
 #include "decode_attn_qb.cuh"
+#include "decode_attn_qbt.cuh"
 #include "evict_insert.cuh"
 #include "merge_states.cuh"
 #include "paged.cuh"
@@ -79,6 +80,21 @@ bool make_kv_map(CUtensorMap* map, const void* base, int d, int cap, int Hkv, in
     cuuint32_t box[4] = {64, (cuuint32_t)rows, 1, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The query rows of the query-batched tensor-core kernel: q [B][Hq][d] with strides q_sb, q_sh
+// (elements), boxes of 64 dims x G heads x BQ rows b (128-byte swizzle; rows past B read zeros).
+bool make_q_map(CUtensorMap* map, const void* q, int d, int Hq, int B, long long q_sh, long long q_sb, int G,
+                int BQ) {
+    EncodeTiledFn fn = encode_tiled();
+    if (fn == nullptr || q_sh <= 0 || q_sb <= 0) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)Hq, (cuuint64_t)B, 1};
+    cuuint64_t strides[3] = {(cuuint64_t)q_sh * 2, (cuuint64_t)q_sb * 2, (cuuint64_t)q_sb * 2 * (cuuint64_t)B};
+    cuuint32_t box[4] = {64, (cuuint32_t)G, (cuuint32_t)BQ, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(q), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -146,8 +162,8 @@ kvb_status launch_decode_tc(const kvb::DecodeTcParams& p, const kvb_attn_args* a
         return KVB_EINVAL;
     const int slots = resident_ctas(kern, SH::NT, smem);
     if (slots <= 0) return KVB_ECUDA;
-    // as many CTAs as keep every CTA's unit count equal to the busiest one's: the makespan in
-    // units is unchanged and no CTA idles while the others finish
+    // round robin: as many CTAs as keep every CTA's unit count equal to the busiest one's (the
+    // makespan in units is unchanged and no CTA idles while the others finish)
     const int per_cta = (p.units + slots - 1) / slots;
     const int grid = (p.units + per_cta - 1) / per_cta;
     if (launch_pdl(kern, dim3(grid), dim3(SH::NT), smem, st, p, mk, mv) != KVB_OK) return KVB_ECUDA;
@@ -176,8 +192,45 @@ kvb_status launch_decode_qb(const kvb::DecodeQbParams& p, const kvb_attn_args* a
     return KVB_OK;
 }
 
+// The tensor-core (tcgen05) shared-prefix kernel: 128 query rows per unit.
+template <int G, bool BIAS>
+kvb_status launch_decode_qbt(kvb::DecodeQbParams p, const kvb_attn_args* a, const CUtensorMap& mq,
+                             cudaStream_t st) {
+    using SH = kvb::QbtShape<G>;
+    auto kern = kvb::decode_attn_qbt_kernel<G, BIAS>;
+    const size_t smem = SH::SMEM;
+    if (set_smem(kern, smem) != KVB_OK) return KVB_ECUDA;
+    CUtensorMap mk, mv;
+    if (!make_kv_map(&mk, a->k, SH::D, a->cap, a->Hkv, 1, a->kv_stride_h, 0, SH::T) ||
+        !make_kv_map(&mv, a->v, SH::D, a->cap, a->Hkv, 1, a->kv_stride_h, 0, SH::T))
+        return KVB_EINVAL;
+    p.blocks = (a->B + SH::BQ - 1) / SH::BQ;
+    const long long units = (long long)p.blocks * a->Hkv * a->num_splits;
+    if (units > 0x7fffffffLL) return KVB_EINVAL;
+    p.units = (int)units;
+    const int slots = resident_ctas(kern, SH::NT, smem);
+    if (slots <= 0) return KVB_ECUDA;
+    const int per_cta = (p.units + slots - 1) / slots;
+    const int grid = (p.units + per_cta - 1) / per_cta;
+    if (launch_pdl(kern, dim3(grid), dim3(SH::NT), smem, st, p, mk, mv, mq) != KVB_OK) return KVB_ECUDA;
+    if (p.S > 1)
+        return launch_merge<128>(p.o_part, p.lse_part, a->B * a->Hq, p.S, p.o, p.o_bf16, p.lse, st);
+    return KVB_OK;
+}
+
 template <int D>
 kvb_status qb_dispatch(const kvb::DecodeQbParams& p, const kvb_attn_args* a, int G, bool bias, cudaStream_t st) {
+    // enough query rows to fill the 128 rows of a tcgen05 tile (and queries a tensor map can
+    // describe): the tensor-core kernel
+    CUtensorMap mq;
+    if (D == 128 && (G == 2 || G == 4 || G == 8) && (long long)a->B * G >= 64 &&
+        make_q_map(&mq, a->q, D, a->Hq, a->B, a->q_stride_h, a->q_stride_b, G, 128 / G)) {
+        switch (G) {
+            case 2: return bias ? launch_decode_qbt<2, true>(p, a, mq, st) : launch_decode_qbt<2, false>(p, a, mq, st);
+            case 4: return bias ? launch_decode_qbt<4, true>(p, a, mq, st) : launch_decode_qbt<4, false>(p, a, mq, st);
+            default: return bias ? launch_decode_qbt<8, true>(p, a, mq, st) : launch_decode_qbt<8, false>(p, a, mq, st);
+        }
+    }
     switch (G) {
         case 1: return bias ? launch_decode_qb<D, 1, true>(p, a, st) : launch_decode_qb<D, 1, false>(p, a, st);
         case 2: return bias ? launch_decode_qb<D, 2, true>(p, a, st) : launch_decode_qb<D, 2, false>(p, a, st);

@@ -68,6 +68,46 @@ def test_shared_prefix_matches_oracle(oracle, d, G, bias, S, split_len):
     assert kvb.kvb_get_error() == 0
 
 
+@pytest.mark.parametrize("G", [2, 4, 8])
+@pytest.mark.parametrize("bias", [True, False])
+@pytest.mark.parametrize("S,split_len", [(1, 0), (3, 96)])
+def test_shared_prefix_tensor_core_blocks_match_oracle(oracle, G, bias, S, split_len):
+    """At d = 128 with at least 64 query rows the tcgen05 kernel runs (128 rows per unit): two
+    full blocks and a ragged third, inactive and empty rows, partial last tiles."""
+    BQ = 128 // G
+    B = 2 * BQ + 5
+    q, k, v, lb, pos, ln, t = shared_case(200 + G, B, G, 2, 128, 280, bias)
+    o, lse, op, lp = run_shared(q, k, v, lb, pos, ln, t, S, split_len)
+    o_ref, l_ref, op_ref, lp_ref = oracle.decode_attn(q, k, v, lb, pos, ln, t, kv_batch_stride=0,
+                                                      meta_batch_stride=0, num_splits=S, split_len=split_len,
+                                                      want_parts=True)
+    assert_state_close(o, lse, o_ref, l_ref, f"tcgen05 G{G} bias{bias} S{S}")
+    assert np.all(lse[B - 2] == -np.inf) and not o[B - 2].any()
+    if S > 1:
+        assert_splits_close(op, lp, op_ref, lp_ref, "splits")
+    assert kvb.kvb_get_error() == 0
+
+
+def test_shared_prefix_large_logit_spread(oracle):
+    """Keys whose logits grow along the cache (so the running maximum moves by far more than 2^8
+    in the exponent, tile after tile): the tcgen05 kernel's lazy rescaling of O must give the
+    same softmax."""
+    B, G, Hkv, d, cap = 70, 4, 2, 128, 300
+    q, k, v, lb, pos, ln, t = shared_case(9, B, G, Hkv, d, cap, True)
+    lb[:] = -0.0   # no decay
+    from memory_bounded_kv_b200.synth import to_bf16_bits, bf16_bits_to_f32
+    kf = bf16_bits_to_f32(k).copy()
+    qf = bf16_bits_to_f32(q)
+    ramp = np.linspace(0.0, 30.0, cap, dtype=np.float32)   # scale 1/sqrt(d): logit grows ~ 30 * |q0|
+    kf[..., 0] = ramp[None, None, :]
+    q2 = qf.copy()
+    q2[..., 0] = 8.0   # logits span ~21 (30 in log2 units) across the cache
+    k, q = to_bf16_bits(kf), to_bf16_bits(q2)
+    o, lse, _, _ = run_shared(q, k, v, lb, pos, ln, t, 1, 0)
+    o_ref, l_ref = oracle.decode_attn(q, k, v, lb, pos, ln, t, kv_batch_stride=0, meta_batch_stride=0)
+    assert_state_close(o, lse, o_ref, l_ref, "large spread")
+
+
 def test_attention_state_memory_shape(oracle):
     """The self attention of the attention-state-memory workload in the launch configuration the
     bench times: 256 queries at positions 1792..2047 over one 2048-token cache, Hkv 8, G 4, d 128,
@@ -92,10 +132,16 @@ def test_shared_prefix_bad_length_flags_error_and_empties_the_row():
     assert np.all(np.isfinite(lse[3, :4]))
 
 
-def test_shared_prefix_bounded_wait_runs_out():
-    q, k, v, lb, pos, ln, t = shared_case(8, 11, 4, 2, 128, 200, False)
+@pytest.mark.parametrize("B", [11, 40])   # the mma.sync kernel (44 rows) and the tcgen05 kernel (160 rows)
+def test_shared_prefix_bounded_wait_runs_out(oracle, B):
+    q, k, v, lb, pos, ln, t = shared_case(8, B, 4, 2, 128, 200, False)
     kvb.kvb_get_error()
     kvb.kvb_test_withhold_next_decode(20_000)
     o, lse, _, lp = run_shared(q, k, v, lb, pos, ln, t, 2, 128)
     assert kvb.kvb_get_error() & _lib.DERR_TIMEOUT
     assert np.all(lse == -np.inf) and not o.any() and np.all(lp == -np.inf)
+    # one launch only: the same call now matches the oracle
+    o, lse, _, _ = run_shared(q, k, v, lb, pos, ln, t, 2, 128)
+    assert kvb.kvb_get_error() == 0
+    o_ref, l_ref = oracle.decode_attn(q, k, v, lb, pos, ln, t, kv_batch_stride=0, meta_batch_stride=0)
+    assert_state_close(o, lse, o_ref, l_ref, "after the timeout")
