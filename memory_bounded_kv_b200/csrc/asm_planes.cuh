@@ -2,22 +2,26 @@
 // core method step 3: c* = argmax_k cos(q, qbar_k)). The memory is static once
 // built, so the normalisation of every centroid and its exact split into three
 // bf16 parts (hi = rn(x), mid = rn(x - hi), lo = x - hi - mid) are done once by
-// asm_prepare_kernel, which writes each tile of 64 centroids as the exact
-// shared-memory image the tensor-core MMA reads: [part][K half][64 rows][128 B],
+// asm_prepare_kernel, which writes each tile of 128 centroids as the exact
+// shared-memory image the tensor-core MMA reads: [part][K half][128 rows][128 B],
 // 16-byte chunk c of row r at chunk c ^ (r & 7) (the 128-byte swizzle).
 //
-// asm_score_planes_kernel then streams those images with bulk copies into a
-// ring of shared-memory stages and keeps the queries in tensor memory as the
-// A operand of tcgen05.mma (so each MMA reads only its 2 KB B slice from shared
-// memory), with three accumulator buffers:
-//   warp 9 (one lane)  bulk copies of the tile images (six 8 KB pieces)  -> b_full[s]
-//   warp 8 (one lane)  48 MMAs per tile (2 M tiles x 3 parts x 8 K steps),
-//                      committed to b_empty[s] and acc_full[b]
-// The ring has four stages, the accumulators three buffers (s = g % 4, b = g % 3).
+// asm_score_planes_kernel streams those images with bulk copies, one part of a
+// tile (32 KB) per stage of a 6-stage ring, and keeps the queries in tensor
+// memory as the A operand of tcgen05.mma (M = 128 queries, N = 128 centroids,
+// K = 16: the shape the tensor cores run at full rate; N = 64 ran at ~70 %).
+// A tile is two units, one per block of 128 queries (M tile); each unit's
+// accumulator takes one of three 128-column buffers in turn (unit u -> buffer
+// u % 3), so the MMAs of a tile proceed while the previous units are read back:
+//   warp 9 (one lane)  bulk copies of the parts                       -> b_full[s]
+//   warp 8 (one lane)  per part 16 MMAs (8 K steps x 2 M tiles, the M tiles
+//                      alternating), committed to b_empty[s]; per tile the
+//                      two units' buffers, committed to acc_full[b]
 //   warps 0-7          the queries into tensor memory (tcgen05.st) at each new
-//                      block of 256 queries (-> a_ready), then per tile: read
-//                      their query row's 64 scores back (tcgen05.ld), release
-//                      the buffer (-> acc_empty[b]) and keep the running best.
+//                      block of 256 queries (-> a_ready), then per tile: warps
+//                      4 m .. 4 m + 3 read back unit m's 128 scores of their
+//                      query row (tcgen05.ld), release the buffer
+//                      (-> acc_empty[b]) and keep the running best.
 // The per-range best keys go to the same workspace as asm_score_umma_kernel's,
 // reduced and merged by asm_merge_kernel.
 #pragma once
@@ -26,20 +30,31 @@
 
 namespace kvb {
 
-constexpr int kPStages = 4;                                    // B ring stages
-constexpr int kPAcc = 3;                                       // accumulator buffers
-constexpr size_t kPImg = 3 * kUPart;                           // one tile image: 48 KB
-constexpr int kPPieces = 6;                                    // copies per tile: one per (part, K half)
-constexpr int kPThreads = kUNT + 64;                           // 8 read-back warps + MMA warp + copy warp
-constexpr int kPACols = kUMT * (kAsmD / 2);                    // queries: 2 M tiles x 64 columns
-constexpr int kPAccCols = kUMT * kUKT;                         // one accumulator buffer: 2 x 64 columns
-constexpr int kPCols = 512;                                    // kPACols + kPAcc * kPAccCols
-constexpr size_t kPBar = (size_t)kPStages * kPImg;             // after the ring
-constexpr size_t kPSmem = kPBar + 192 + 1024;                  // barriers + slot, + alignment slack
-static_assert(kPACols + kPAcc * kPAccCols == kPCols, "tensor memory budget");
-static_assert(kPImg % kPPieces == 0 && (kPImg / kPPieces) % 1024 == 0, "pieces");
+constexpr int kPT = 128;                                        // centroids per tile (the MMA's N)
+constexpr size_t kPHalf = (size_t)kPT * 128;                    // one K half of one part: 16 KB
+constexpr size_t kPPart = 2 * kPHalf;                           // one part: 32 KB (a ring stage)
+constexpr size_t kPImg = 3 * kPPart;                            // one tile image: 96 KB
+constexpr int kPStages = 6;                                     // ring stages (two tiles)
+constexpr int kPAcc = 3;                                        // accumulator buffers (units)
+constexpr int kPThreads = kUNT + 64;                            // 8 read-back warps + MMA warp + copy warp
+constexpr int kPACols = kUMT * (kAsmD / 2);                     // queries: 2 M tiles x 64 columns
+constexpr int kPCols = 512;                                     // kPACols + kPAcc * kPT
+constexpr size_t kPBar = (size_t)kPStages * kPPart;             // after the ring
+constexpr size_t kPSmem = kPBar + 256 + 1024;                   // barriers + slot, + alignment slack
+static_assert(kPACols + kPAcc * kPT == kPCols, "tensor memory budget");
 
-__host__ __device__ inline size_t asm_plane_tiles(int K) { return (size_t)(K + kUKT - 1) / kUKT; }
+__host__ __device__ inline size_t asm_plane_tiles(int K) { return (size_t)(K + kPT - 1) / kPT; }
+
+// Centroid ranges of the lookup over a prepared memory: whole tiles, as many ranges per (head,
+// query block) as there are CTAs for it (so that a CTA's items seldom span two blocks), at most
+// asm_ksplit(K) of them (the workspace holds that many).
+__host__ inline int asm_planes_kchunk(int K, int blocks, int slots) {
+    const int cpb = blocks >= slots ? 1 : slots / blocks;                  // CTAs per (head, query block)
+    int c = (K + cpb - 1) / cpb;
+    const int c_min = (K + asm_ksplit(K) - 1) / asm_ksplit(K);
+    c = c < c_min ? c_min : c;
+    return (c + kPT - 1) / kPT * kPT;
+}
 
 // ---- preparation: one warp per centroid row --------------------------------------------------
 __global__ void __launch_bounds__(256) asm_prepare_kernel(const float* __restrict__ qbar, int H, int K,
@@ -47,9 +62,9 @@ __global__ void __launch_bounds__(256) asm_prepare_kernel(const float* __restric
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t tiles = asm_plane_tiles(K);
     const long long row = (long long)blockIdx.x * 8 + warp;         // (table, tile row) over padded K
-    if (row >= (long long)H * tiles * kUKT) return;
-    const int h = (int)(row / ((long long)tiles * kUKT));
-    const int kk = (int)(row % ((long long)tiles * kUKT));          // centroid index (maybe >= K: zeros)
+    if (row >= (long long)H * tiles * kPT) return;
+    const int h = (int)(row / ((long long)tiles * kPT));
+    const int kk = (int)(row % ((long long)tiles * kPT));           // centroid index (maybe >= K: zeros)
     float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
     if (kk < K) x = reinterpret_cast<const float4*>(qbar + ((size_t)h * K + kk) * kAsmD)[lane];
     float ss = fmaf(x.x, x.x, fmaf(x.y, x.y, fmaf(x.z, x.z, x.w * x.w)));
@@ -60,13 +75,13 @@ __global__ void __launch_bounds__(256) asm_prepare_kernel(const float* __restric
     split3_bf16x2(x.x * inv, x.y * inv, hw[0], mw[0], lw[0]);
     split3_bf16x2(x.z * inv, x.w * inv, hw[1], mw[1], lw[1]);
     // lane l holds elements 4l .. 4l + 3: K half l / 16, chunk (l % 16) / 2, bytes 8 (l % 2) .. + 7
-    const int r = kk % kUKT;
+    const int r = kk % kPT;
     const int kh = lane >> 4, c = (lane & 15) >> 1;
-    unsigned char* img = planes + ((size_t)h * tiles + kk / kUKT) * kPImg;
-    const size_t off = kh * kUPartHalf + r * 128 + ((c ^ (r & 7)) << 4) + 8 * (lane & 1);
+    unsigned char* img = planes + ((size_t)h * tiles + kk / kPT) * kPImg;
+    const size_t off = kh * kPHalf + r * 128 + ((c ^ (r & 7)) << 4) + 8 * (lane & 1);
     *reinterpret_cast<uint2*>(img + off) = make_uint2(hw[0], hw[1]);
-    *reinterpret_cast<uint2*>(img + kUPart + off) = make_uint2(mw[0], mw[1]);
-    *reinterpret_cast<uint2*>(img + 2 * kUPart + off) = make_uint2(lw[0], lw[1]);
+    *reinterpret_cast<uint2*>(img + kPPart + off) = make_uint2(mw[0], mw[1]);
+    *reinterpret_cast<uint2*>(img + 2 * kPPart + off) = make_uint2(lw[0], lw[1]);
 }
 
 // ---- tensor-memory helpers of the lookup ------------------------------------------------------
@@ -100,6 +115,33 @@ struct AsmPlanesParams {
     unsigned long long wait_ns;
 };
 
+// The tile stream of a CTA: its run of items (head, query block, centroid range), each range
+// walked in tiles of kPT centroids (items are head-major, so the queries change rarely).
+struct PTile {
+    int h, qt, ks, kt, k_end;
+};
+__device__ __forceinline__ void ptile_start(const AsmParams& p, PTile& c, int item) {
+    c.h = item / (p.qtiles * p.ksplit);
+    const int r = item % (p.qtiles * p.ksplit);
+    c.qt = r / p.ksplit;
+    c.ks = r % p.ksplit;
+    c.kt = c.ks * p.kchunk;
+    c.k_end = min(p.K, c.kt + p.kchunk);
+}
+__device__ __forceinline__ void ptile_next(const AsmParams& p, PTile& c) {
+    c.kt += kPT;
+    if (c.kt < c.k_end) return;
+    if (++c.ks == p.ksplit) {
+        c.ks = 0;
+        if (++c.qt == p.qtiles) {
+            c.qt = 0;
+            ++c.h;
+        }
+    }
+    c.kt = c.ks * p.kchunk;
+    c.k_end = min(p.K, c.kt + p.kchunk);
+}
+
 __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __grid_constant__ AsmPlanesParams pp) {
     const AsmParams& p = pp.a;
     extern __shared__ unsigned char s_raw[];
@@ -118,7 +160,7 @@ __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __
     int G = 0;              // tiles in this CTA's stream
     for (int it = i0; it < i1; ++it) {
         const int kb = (it % p.ksplit) * p.kchunk;
-        G += (min(p.K, kb + p.kchunk) - kb + kUKT - 1) / kUKT;
+        G += (min(p.K, kb + p.kchunk) - kb + kPT - 1) / kPT;
     }
     const size_t tiles_per_table = asm_plane_tiles(p.K);
 
@@ -135,7 +177,7 @@ __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __
         }
         for (int b = 0; b < kPAcc; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], kUNT / 32);
+            mbar_init(&acc_empty[b], 4);   // the four warps of the unit's M tile
         }
         mbar_init(a_ready, kUNT / 32);
         fence_mbar_init();
@@ -147,84 +189,92 @@ __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __
     bool ok = true;
 
     if (warp == kUNT / 32 + 1) {
-        // ---- copy warp: tile images into the ring
+        // ---- copy warp: the parts of each tile into the ring, one stage each
         if (lane == 0) {
-            AsmTile c;
-            asm_tile_start(p, c, i0);
+            PTile c;
+            ptile_start(p, c, i0);
+            int issued = 0;   // stages whose copies were issued
             for (int g = 0; g < G && ok; ++g) {
-                const int s = g % kPStages;
-                if (g >= kPStages && !mbar_wait(&b_empty[s], (unsigned)((g / kPStages) - 1) & 1u, pp.wait_ns)) {
-                    ok = false;
-                    break;
+                const unsigned char* src = pp.planes + ((size_t)(c.h / p.G) * tiles_per_table + c.kt / kPT) * kPImg;
+                for (int pt = 0; pt < 3; ++pt) {
+                    const int j = 3 * g + pt, s = j % kPStages;
+                    if (j >= kPStages && !mbar_wait(&b_empty[s], (unsigned)((j / kPStages) - 1) & 1u, pp.wait_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&b_full[s], (unsigned)kPPart);
+                    bulk_g2s(sm + (size_t)s * kPPart, src + pt * kPPart, (unsigned)kPHalf, &b_full[s]);
+                    bulk_g2s(sm + (size_t)s * kPPart + kPHalf, src + pt * kPPart + kPHalf, (unsigned)kPHalf, &b_full[s]);
+                    issued = j + 1;
                 }
-                mbar_arrive_expect_tx(&b_full[s], (unsigned)kPImg);
-                const unsigned char* src = pp.planes + ((size_t)(c.h / p.G) * tiles_per_table + c.kt / kUKT) * kPImg;
-#pragma unroll
-                for (int pc = 0; pc < kPPieces; ++pc)
-                    bulk_g2s(sm + (size_t)s * kPImg + pc * (kPImg / kPPieces), src + pc * (kPImg / kPPieces),
-                             (unsigned)(kPImg / kPPieces), &b_full[s]);
-                asm_tile_next(p, c);
+                ptile_next(p, c);
             }
+            // every copy lands before the CTA can exit (bounded): the last stage issued on each slot
+            for (int j = max(0, issued - kPStages); j < issued; ++j)
+                mbar_wait(&b_full[j % kPStages], (unsigned)(j / kPStages) & 1u, 100000000ull);
         }
     } else if (warp == kUNT / 32) {
         // ---- MMA warp
         if (lane == 0) {
-            AsmTile cm;
-            asm_tile_start(p, cm, i0);
-            constexpr uint32_t idesc = umma_idesc_bf16(kUQ, kUKT);
+            PTile cm;
+            ptile_start(p, cm, i0);
+            constexpr uint32_t idesc = umma_idesc_bf16(kUQ, kPT);
             const uint64_t b0 = umma_desc_sw128(sbase);
             int a_block = -1, a_phase = 0;
-            for (int g = 0; g < G; ++g) {
-                const int s = g % kPStages, ab = g % kPAcc;
-                if (!mbar_wait(&b_full[s], (unsigned)(g / kPStages) & 1u, pp.wait_ns)) { ok = false; break; }
-                if (g >= kPAcc && !mbar_wait(&acc_empty[ab], (unsigned)((g / kPAcc) - 1) & 1u, pp.wait_ns)) {
-                    ok = false;
-                    break;
+            for (int g = 0; g < G && ok; ++g) {
+                // the two units of tile g take buffers (2g) % 3 and (2g + 1) % 3, free once the units three
+                // before them are read back
+                uint32_t dacc[kUMT];
+#pragma unroll
+                for (int mt = 0; mt < kUMT; ++mt) {
+                    const int u = 2 * g + mt, b = u % kPAcc;
+                    dacc[mt] = tmem + (uint32_t)(kPACols + b * kPT);
+                    if (u >= kPAcc && !mbar_wait(&acc_empty[b], (unsigned)((u / kPAcc) - 1) & 1u, pp.wait_ns)) ok = false;
                 }
+                if (!ok) break;
                 const int blk = cm.h * p.qtiles + cm.qt;
                 if (blk != a_block) {   // the read-back warps have put this block's queries in tensor memory
                     if (!mbar_wait(a_ready, (unsigned)a_phase & 1u, pp.wait_ns)) { ok = false; break; }
                     ++a_phase;
                     a_block = blk;
                 }
-                tc_fence_after();
-                // the two M tiles' products alternate: consecutive MMAs go to independent
-                // accumulators, so each one's accumulation does not wait for the one before
                 const int mts = min(kUMT, (p.N - cm.qt * (kUMT * kUQ) + kUQ - 1) / kUQ);
-#pragma unroll
-                for (int pt = 0; pt < 3; ++pt)
+                for (int pt = 0; pt < 3 && ok; ++pt) {
+                    const int j = 3 * g + pt, s = j % kPStages;
+                    if (!mbar_wait(&b_full[s], (unsigned)(j / kPStages) & 1u, pp.wait_ns)) { ok = false; break; }
+                    tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < kAsmD / 16; ++kk) {
-                        const uint32_t boff =
-                            (uint32_t)(s * kPImg + pt * kUPart + (kk >> 2) * kUPartHalf + (kk & 3) * 32);
+                        const uint32_t boff = (uint32_t)(s * kPPart + (kk >> 2) * kPHalf + (kk & 3) * 32);
 #pragma unroll
-                        for (int mt = 0; mt < kUMT; ++mt) {
+                        for (int mt = 0; mt < kUMT; ++mt) {   // the M tiles alternate (independent accumulators)
                             if (mt >= mts) break;
-                            const uint32_t d = tmem + (uint32_t)(kPACols + ab * kPAccCols + mt * kUKT);
                             const uint32_t a = tmem + (uint32_t)(mt * (kAsmD / 2) + kk * 8);
-                            umma_bf16_ts(d, a, b0 + (boff >> 4), idesc, (pt | kk) != 0);
+                            umma_bf16_ts(dacc[mt], a, b0 + (boff >> 4), idesc, (pt | kk) != 0);
                         }
                     }
-                umma_commit(&b_empty[s]);
-                umma_commit(&acc_full[ab]);
-                asm_tile_next(p, cm);
+                    umma_commit(&b_empty[s]);
+                }
+                if (!ok) break;
+#pragma unroll
+                for (int mt = 0; mt < kUMT; ++mt) umma_commit(&acc_full[(2 * g + mt) % kPAcc]);
+                ptile_next(p, cm);
             }
         }
     } else {
         // ---- warps 0-7: queries into tensor memory, read-back and argmax
-        AsmTile ce;
-        asm_tile_start(p, ce, i0);
+        PTile ce;
+        ptile_start(p, ce, i0);
         const int emt = warp >> 2, elane = 32 * (warp & 3);
         float bmax = -INFINITY;
         int bidx = -1;
         int a_block = -1;
         for (int g = 0; g < G; ++g) {
-            const int s = g % kPAcc;   // the accumulator buffer of tile g
             const int blk = ce.h * p.qtiles + ce.qt;
             const int n0 = ce.qt * (kUMT * kUQ);
             if (blk != a_block) {
-                // every MMA that read the previous queries is complete: this warp has read back the
-                // tile before (its acc_full arrives after all earlier MMAs)
+                // every MMA that read the previous queries is complete: this warp has read back its unit
+                // of the tile before (its acc_full arrives after all earlier MMAs)
                 const int n = n0 + emt * kUQ + elane + lane;
                 uint32_t r[kAsmD / 2];
                 if (n < p.N) {
@@ -247,41 +297,59 @@ __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __
                 if (lane == 0) mbar_arrive(a_ready);
                 a_block = blk;
             }
-            if (!__all_sync(kFull, mbar_wait(&acc_full[s], (unsigned)(g / kPAcc) & 1u, pp.wait_ns))) ok = false;
+            const int u = 2 * g + emt, b = u % kPAcc;
+            // warp-uniform outcome: the tensor-memory loads below are warp-collective
+            if (!__all_sync(kFull, mbar_wait(&acc_full[b], (unsigned)(u / kPAcc) & 1u, pp.wait_ns))) ok = false;
             tc_fence_after();
             const int mts = min(kUMT, (p.N - n0 + kUQ - 1) / kUQ);
-            float v[kUKT];
-            if (ok && emt < mts) {
-                const uint32_t ta = tmem + ((uint32_t)elane << 16) + (uint32_t)(kPACols + s * kPAccCols + emt * kUKT);
-                tmem_ld32(ta, v);
-                tmem_ld32(ta + 32, v + 32);
-                tmem_ld_wait();
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[s]);   // the buffer may take tile g + kPAcc
-            if (ok && emt < mts) {
-                if (ce.kt + kUKT > ce.k_end) {   // ragged last tile of a range
+            const bool mine = ok && emt < mts;
+            // the unit's 128 scores of this row, in two halves of 64: the best value and its first column
+            float best = -INFINITY;
+            int first = -1;
+            if (mine) {
+                const uint32_t ta = tmem + ((uint32_t)elane << 16) + (uint32_t)(kPACols + b * kPT);
 #pragma unroll
-                    for (int c = 0; c < kUKT; ++c)
-                        if (ce.kt + c >= ce.k_end) v[c] = -INFINITY;
+                for (int hf = 0; hf < 2; ++hf) {
+                    float v[64];
+                    tmem_ld32(ta + 64 * hf, v);
+                    tmem_ld32(ta + 64 * hf + 32, v + 32);
+                    tmem_ld_wait();
+                    if (hf == 1) {   // the last read of the buffer: release it before the arithmetic
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&acc_empty[b]);
+                    }
+                    const int c0 = ce.kt + 64 * hf;
+                    if (c0 + 64 > ce.k_end) {   // ragged last tile of a range
+#pragma unroll
+                        for (int c = 0; c < 64; ++c)
+                            if (c0 + c >= ce.k_end) v[c] = -INFINITY;
+                    }
+                    float m[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) m[c] = fmaxf(v[c], v[c + 32]);
+#pragma unroll
+                    for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+                        for (int c = 0; c < w; ++c) m[c] = fmaxf(m[c], m[c + w]);
+                    if (m[0] > best) {   // strictly greater: the earlier half keeps a tie
+                        int f = 63;
+#pragma unroll
+                        for (int c = 63; c >= 0; --c) f = (v[c] == m[0]) ? c : f;
+                        best = m[0];
+                        first = 64 * hf + f;
+                    }
                 }
-                float m[kUKT / 2];
-#pragma unroll
-                for (int c = 0; c < kUKT / 2; ++c) m[c] = fmaxf(v[c], v[c + kUKT / 2]);
-#pragma unroll
-                for (int w = kUKT / 4; w >= 1; w >>= 1)
-#pragma unroll
-                    for (int c = 0; c < w; ++c) m[c] = fmaxf(m[c], m[c + w]);
-                if (m[0] > bmax) {   // strictly greater: an equal value in a later tile has a larger k
-                    int first = kUKT - 1;
-#pragma unroll
-                    for (int c = kUKT - 1; c >= 0; --c) first = (v[c] == m[0]) ? c : first;
-                    bmax = m[0];
-                    bidx = ce.kt + first;
-                }
+            } else {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[b]);
             }
-            if (ce.kt + kUKT >= ce.k_end) {   // end of the item: write this row's best, start afresh
+            if (mine && best > bmax) {   // strictly greater: an equal value in a later tile has a larger k
+                bmax = best;
+                bidx = ce.kt + first;
+            }
+            if (ce.kt + kPT >= ce.k_end) {   // end of the item: write this row's best, start afresh
                 const int n = n0 + emt * kUQ + elane + lane;
                 if (emt < mts && n < p.N) {
                     const unsigned long long key =
@@ -293,7 +361,7 @@ __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __
                 bmax = -INFINITY;
                 bidx = -1;
             }
-            asm_tile_next(p, ce);
+            ptile_next(p, ce);
         }
     }
     if (!ok) raise_error(KVB_DERR_TIMEOUT);
@@ -301,7 +369,8 @@ __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __
     __syncthreads();
     if (warp == kUNT / 32 && lane == 0 && G > 0) {
         // the last tile's MMAs complete before the tensor memory is released (bounded)
-        mbar_wait(&acc_full[(G - 1) % kPAcc], (unsigned)((G - 1) / kPAcc) & 1u, pp.wait_ns);
+        const int u = 2 * (G - 1) + 1;
+        mbar_wait(&acc_full[u % kPAcc], (unsigned)(u / kPAcc) & 1u, pp.wait_ns);
     }
     __syncthreads();
     if (warp == 0) {

@@ -7,7 +7,7 @@
 // is read once per 128 query rows and both products run as tcgen05.mma with
 // the accumulators in tensor memory.
 //
-// Roles (192 threads, one CTA per SM):
+// Roles (320 threads, one CTA per SM):
 //   warp 0     producer: the unit's 128 query rows by TMA (a 3-D box of 64
 //              dims x G heads x 128 / G rows b, K-major with the 128-byte
 //              swizzle, two buffers), K/V tiles by TMA into a 3-stage ring with
@@ -17,11 +17,14 @@
 //              K = 64) with P read from tensor memory (A operand) and V from
 //              shared memory as an MN-major B operand; S(i + 1) is issued
 //              before P V(i), so the softmax of tile i overlaps the next QK;
-//   warps 2-5  softmax, one query row per thread (tensor-memory lane = row):
-//              read S, mask by the row's length, add the row's bias, keep the
-//              running maximum and sum, write P as a bf16 high part and a
-//              bf16 residual (two products each, ~16 bits of P) into tensor
-//              memory; at the end of the unit read O and write the state.
+//   warps 2-9  softmax, two threads per query row (tensor-memory lane = row;
+//              warps w and w + 4 share a lane quarter, each takes 32 of the
+//              tile's 64 scores and 64 of O's 128 columns): read S, mask by the
+//              row's length, add the row's bias, exchange the half-row maxima
+//              (an mbarrier per lane quarter), keep the running maximum and
+//              sum, write P as a bf16 high part and a bf16 residual (two
+//              products each, ~16 bits of P) into tensor memory; at the end of
+//              the unit exchange the half-row sums, read O and write the state.
 // The running maximum is updated lazily: P is formed against a reference
 // maximum and O is rescaled (read, scaled, written back in tensor memory)
 // only when a row's maximum exceeds the reference by more than 2^8 in the
@@ -45,7 +48,7 @@ struct QbtShape {
     static constexpr int BQ = R / G;          // rows b per unit
     static constexpr int T = 64;              // slots per tile
     static constexpr int ST = 3;              // K/V ring stages
-    static constexpr int NT = 6 * 32;
+    static constexpr int NT = 10 * 32;        // producer, MMA issuer, 8 softmax warps
     static constexpr int QHALF = R * 128;     // 128 rows x 64 dims of bf16
     static constexpr int QBUF = 2 * QHALF;
     static constexpr int KVHALF = T * 128;
@@ -57,8 +60,11 @@ struct QbtShape {
     static constexpr int POS_OFF = RING_OFF + ST * STAGE;
     static constexpr int LB_OFF = POS_OFF + ST * T * 4;
     static constexpr int META_OFF = LB_OFF + ST * T * 4;
-    static constexpr int BAR_OFF = (META_OFF + ST * META * 4 + 7) / 8 * 8;
-    static constexpr int NBAR = 2 * ST + 14;  // kv full/empty; q, s, p full/empty, pv_done x 2; o_free; fin
+    static constexpr int XCH_OFF = (META_OFF + ST * META * 4 + 15) / 16 * 16;   // half-row maxima [2][2][R], sums [2][R]
+    static constexpr int BAR_OFF = XCH_OFF + 6 * R * 4;
+    // kv full/empty [ST] each; q, s, p full/empty [2] each; pv_done [2]; o_free; fin; the maxima
+    // exchange [4 quarters][2]; the sums exchange [4]
+    static constexpr int NBAR = 2 * ST + 6 * 2 + 2 + 1 + 1 + 8 + 4;
     static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
     static constexpr int END = MISC_OFF + 32;
     static constexpr size_t SMEM = 1024 + END;
@@ -66,10 +72,27 @@ struct QbtShape {
     static_assert(G == 2 || G == 4 || G == 8, "G");
     static_assert(BQ <= 64, "rows per unit");
     static_assert(RING_OFF % 1024 == 0 && STAGE % 1024 == 0, "alignment");
+    static_assert(MISC_OFF >= BAR_OFF + NBAR * 8 && BAR_OFF % 8 == 0, "barriers before the misc words");
 };
 
 // kind::f16 instruction descriptor with an MN-major B operand (bit 16)
 __host__ __device__ constexpr uint32_t umma_idesc_bf16_bmn(int M, int N) { return umma_idesc_bf16(M, N) | (1u << 16); }
+
+// 32 lanes x 16 consecutive columns from registers (lane i of the warp writes lane base + i)
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16};" ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+        "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
+// 2^x by the hardware's approximate base-2 exponential (PTX ex2.approx.ftz; 2^-inf = 0)
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 // A bounded wait whose outcome is the same for the whole warp (the warp then runs warp-collective
 // tensor-memory instructions or leaves together).
@@ -112,6 +135,9 @@ __global__ void __launch_bounds__(QbtShape<G>::NT, 1)
     uint64_t* pv_done = p_empty + 2;
     uint64_t* o_free = pv_done + 2;
     uint64_t* fin = o_free + 1;   // the MMA warp's last commit: every tensor-core operation done
+    uint64_t* xm_bar = fin + 1;   // [quarter][tile parity]: both warps of a lane quarter posted their maxima
+    uint64_t* xl_bar = xm_bar + 8;   // [quarter]: both posted their sums (once per unit)
+    // (xl_bar + 4 == bars + NBAR: the last barrier)
     uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + SH::MISC_OFF);
     volatile int* s_abort = reinterpret_cast<int*>(smem + SH::MISC_OFF) + 1;
     int* s_issued = reinterpret_cast<int*>(smem + SH::MISC_OFF) + 2;   // tiles the producer issued
@@ -136,14 +162,16 @@ __global__ void __launch_bounds__(QbtShape<G>::NT, 1)
             mbar_init(&q_full[b], 1);     // the producer's expect_tx; the copy's bytes
             mbar_init(&q_empty[b], 1);
             mbar_init(&s_full[b], 1);
-            mbar_init(&s_empty[b], 4);    // the 4 softmax warps
-            mbar_init(&p_full[b], 4);
+            mbar_init(&s_empty[b], 8);    // the 8 softmax warps
+            mbar_init(&p_full[b], 8);
             mbar_init(&p_empty[b], 1);
         }
         mbar_init(&pv_done[0], 1);
         mbar_init(&pv_done[1], 1);
-        mbar_init(o_free, 4);
+        mbar_init(o_free, 8);
         mbar_init(fin, 1);
+        for (int k = 0; k < 8; ++k) mbar_init(&xm_bar[k], 2);
+        for (int k = 0; k < 4; ++k) mbar_init(&xl_bar[k], 2);
         *s_abort = 0;
         *s_issued = 0;
         *s_mma = 0;
@@ -387,14 +415,24 @@ __global__ void __launch_bounds__(QbtShape<G>::NT, 1)
     } else {
         // ======================= softmax warps =======================
         const int quarter = warp & 3;             // tensor-memory lanes 32 * quarter ..
+        const int half = (warp - 2) >> 2;         // scores 32 half .. of a tile, O columns 64 half ..
         const int r = 32 * quarter + lane;        // this thread's query row
+        const int sidx = (warp - 2) * 32 + lane;  // 0 .. 255
         const uint32_t tl = tmem + ((uint32_t)(32 * quarter) << 16);
-        const float L2E = kLog2e;
+        float* xm = reinterpret_cast<float*>(smem + SH::XCH_OFF);   // [tile parity][half][R]
+        float* xl = xm + 4 * R;                                      // [half][R]
+        const float C = p.scale * kLog2e;         // scores in log2 units: the maxima and P below are too
         float m_ref = -INFINITY, l_sum = 0.f;
-        int lim = 0, trow = 0;
+        int lim = 0, trow = 0, units_done = 0;
+        auto fail = [&]() {
+            if (lane == 0) {
+                raise_error(KVB_DERR_TIMEOUT);
+                *s_abort = 1;
+            }
+        };
         for (int i = 0;; ++i) {
             const int st = i % ST;
-            if (!warp_wait(&kv_full[st], (unsigned)(i / ST) & 1u, p.wait_ns)) break;
+            if (!warp_wait(&kv_full[st], (unsigned)(i / ST) & 1u, p.wait_ns)) { fail(); break; }
             const int* m = s_meta + st * SH::META;
             const int u = m[0];
             if (u < 0) break;
@@ -404,7 +442,7 @@ __global__ void __launch_bounds__(QbtShape<G>::NT, 1)
                 // V rows past the unit's last slot may hold any bytes: zero them (their P is 0, and
                 // 0 times a NaN would not be); the tensor cores read them only in P V(i), after p_full
                 unsigned char* vt = smem + SH::RING_OFF + st * SH::STAGE + SH::KVTILE;
-                for (int idx = r; idx < (T - rows) * 16; idx += R) {
+                for (int idx = sidx; idx < (T - rows) * 16; idx += 256) {
                     const int row = rows + (idx >> 4), c = idx & 15;
                     *reinterpret_cast<uint4*>(vt + (c >> 3) * SH::KVHALF + row * 128 + (((c & 7) ^ (row & 7)) << 4)) =
                         make_uint4(0u, 0u, 0u, 0u);
@@ -418,103 +456,120 @@ __global__ void __launch_bounds__(QbtShape<G>::NT, 1)
                 l_sum = 0.f;
             }
             const int sb = i & 1;
-            if (!warp_wait(&s_full[sb], (unsigned)(i >> 1) & 1u, p.wait_ns)) break;
+            if (!warp_wait(&s_full[sb], (unsigned)(i >> 1) & 1u, p.wait_ns)) { fail(); break; }
             tc_fence_after();
-            float x[T];
-            tmem_ld32(tl + SH::TM_S + sb * 64, x);
-            tmem_ld32(tl + SH::TM_S + sb * 64 + 32, x + 32);
+            float x[32];
+            tmem_ld32(tl + SH::TM_S + sb * 64 + 32 * half, x);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s_empty[sb]);
-            float mt = -INFINITY;
+            const int c0 = base + 32 * half;
+            float mh = -INFINITY;
 #pragma unroll
-            for (int j = 0; j < T; ++j) {
+            for (int j = 0; j < 32; ++j) {
                 float bj = 0.f;
-                if constexpr (BIAS) bj = __fmul_rn(__int2float_rn(trow - s_pos[st * T + j]), s_lb[st * T + j]);
-                x[j] = (base + j < lim) ? fmaf(x[j], p.scale, bj) : -INFINITY;
-                mt = fmaxf(mt, x[j]);
+                if constexpr (BIAS)
+                    bj = __fmul_rn(__int2float_rn(trow - s_pos[st * T + 32 * half + j]), s_lb[st * T + 32 * half + j]) *
+                         kLog2e;
+                x[j] = (c0 + j < lim) ? fmaf(x[j], C, bj) : -INFINITY;
+                mh = fmaxf(mh, x[j]);
             }
+            // the row's maximum over both halves (slot i % 2: the partner reads slot i % 2 before it can
+            // post tile i + 2's maximum there, since that needs this thread's post of tile i + 1)
+            xm[(sb * 2 + half) * R + r] = mh;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&xm_bar[quarter * 2 + sb]);
+            if (!warp_wait(&xm_bar[quarter * 2 + sb], (unsigned)(i >> 1) & 1u, p.wait_ns)) { fail(); break; }
+            const float mt = fmaxf(mh, xm[(sb * 2 + 1 - half) * R + r]);
             // the reference moves when the row's maximum passes it by more than 2^8; the rows that
-            // had one already rescale O. Tensor-memory loads and stores are warp-collective, so the
-            // whole warp takes the rescale when any of its rows needs it (the others scale by 1).
-            const bool grow = mt > m_ref && (m_ref == -INFINITY || (mt - m_ref) * L2E > 8.f);
+            // had one already rescale their half of O. Tensor-memory loads and stores are
+            // warp-collective, so the whole warp takes the rescale when any of its rows needs it.
+            const bool grow = mt > m_ref && (m_ref == -INFINITY || mt - m_ref > 8.f);
             const bool resc = grow && m_ref != -INFINITY;
             if (__any_sync(kFull, resc)) {
                 // every earlier P V product of this unit first (P V(i - 1); i > 0 here)
-                if (!warp_wait(&pv_done[(i - 1) & 1], (unsigned)((i - 1) >> 1) & 1u, p.wait_ns)) break;
+                if (!warp_wait(&pv_done[(i - 1) & 1], (unsigned)((i - 1) >> 1) & 1u, p.wait_ns)) { fail(); break; }
                 tc_fence_after();
-                const float alpha = resc ? exp2f((m_ref - mt) * L2E) : 1.f;
+                const float alpha = resc ? ex2_approx(m_ref - mt) : 1.f;
 #pragma unroll
-                for (int c = 0; c < D; c += 32) {
+                for (int c = 0; c < 64; c += 32) {
                     float o[32];
-                    tmem_ld32(tl + SH::TM_O + c, o);
+                    tmem_ld32(tl + SH::TM_O + 64 * half + c, o);
                     tmem_ld_wait();
                     uint32_t w[32];
 #pragma unroll
                     for (int e = 0; e < 32; ++e) w[e] = __float_as_uint(o[e] * alpha);
-                    tmem_st32(tl + SH::TM_O + c, w);
+                    tmem_st32(tl + SH::TM_O + 64 * half + c, w);
                 }
                 tmem_st_wait();
                 l_sum *= alpha;
             }
             if (grow) m_ref = mt;
             const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-            uint32_t hi[T / 2], lo[T / 2];
+            uint32_t hi[16], lo[16];
             float ssum = 0.f;
 #pragma unroll
-            for (int j = 0; j < T; j += 2) {
-                const float p0 = exp2f((x[j] - m_use) * L2E), p1 = exp2f((x[j + 1] - m_use) * L2E);
+            for (int j = 0; j < 32; j += 2) {
+                const float p0 = ex2_approx(x[j] - m_use), p1 = ex2_approx(x[j + 1] - m_use);
                 ssum += p0 + p1;
                 hi[j / 2] = pack_bf16(p0, p1);
                 lo[j / 2] = pack_bf16(p0 - __uint_as_float(hi[j / 2] << 16), p1 - __uint_as_float(hi[j / 2] & 0xffff0000u));
             }
             l_sum += ssum;
             const int pb = i & 1;
-            if (i >= 2 && !warp_wait(&p_empty[pb], (unsigned)((i >> 1) - 1) & 1u, p.wait_ns)) break;
+            if (i >= 2 && !warp_wait(&p_empty[pb], (unsigned)((i >> 1) - 1) & 1u, p.wait_ns)) { fail(); break; }
             tc_fence_after();
-            tmem_st32(tl + SH::TM_P + pb * 64, hi);
-            tmem_st32(tl + SH::TM_P + pb * 64 + 32, lo);
+            tmem_st16(tl + SH::TM_P + pb * 64 + 16 * half, hi);
+            tmem_st16(tl + SH::TM_P + pb * 64 + 32 + 16 * half, lo);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[pb]);
             if (ti != ntiles - 1) continue;
 
-            // ---- end of unit: O of this row, divided by the sum; the split's state
-            if (!warp_wait(&pv_done[i & 1], (unsigned)(i >> 1) & 1u, p.wait_ns)) break;
+            // ---- end of unit: the row's sum over both halves; this thread's half of O, divided by it
+            if (!warp_wait(&pv_done[i & 1], (unsigned)(i >> 1) & 1u, p.wait_ns)) { fail(); break; }
             tc_fence_after();
-            float o[D];
-#pragma unroll
-            for (int c = 0; c < D; c += 32) tmem_ld32(tl + SH::TM_O + c, o + c);
+            float o[64];
+            tmem_ld32(tl + SH::TM_O + 64 * half, o);
+            tmem_ld32(tl + SH::TM_O + 64 * half + 32, o + 32);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(o_free);
+            xl[half * R + r] = l_sum;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&xl_bar[quarter]);
+            if (!warp_wait(&xl_bar[quarter], (unsigned)units_done & 1u, p.wait_ns)) { fail(); break; }
+            const float lt = l_sum + xl[(1 - half) * R + r];
+            // the partner has read this thread's sum before it can post the next unit's (that needs
+            // this thread's maxima of the next unit's first tile)
+            ++units_done;
             const int b = ublk * BQ + r / G;
             if (b < p.B) {
                 const size_t row = (size_t)b * p.Hq + ug * G + r % G;
-                const float inv = (l_sum > 0.f) ? 1.f / l_sum : 0.f;
-                const float lse = (l_sum > 0.f) ? m_ref + log2f(l_sum) * kLn2 : -INFINITY;
+                const float inv = (lt > 0.f) ? 1.f / lt : 0.f;
+                const float lse = (lt > 0.f) ? (m_ref + log2f(lt)) * kLn2 : -INFINITY;
                 if (p.o_part != nullptr) {
-                    float4* dst = reinterpret_cast<float4*>(p.o_part + (row * p.S + usplit) * D);
+                    float4* dst = reinterpret_cast<float4*>(p.o_part + (row * p.S + usplit) * D + 64 * half);
 #pragma unroll
-                    for (int e = 0; e < D; e += 4)
+                    for (int e = 0; e < 64; e += 4)
                         dst[e / 4] = make_float4(o[e] * inv, o[e + 1] * inv, o[e + 2] * inv, o[e + 3] * inv);
-                    p.lse_part[row * p.S + usplit] = lse;
+                    if (half == 0) p.lse_part[row * p.S + usplit] = lse;
                 }
                 if (p.S == 1) {
                     if (p.o_bf16) {
-                        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.o) + row * D;
+                        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.o) + row * D + 64 * half;
 #pragma unroll
-                        for (int e = 0; e < D; ++e) dst[e] = __float2bfloat16_rn(o[e] * inv);
+                        for (int e = 0; e < 64; ++e) dst[e] = __float2bfloat16_rn(o[e] * inv);
                     } else {
-                        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.o) + row * D);
+                        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.o) + row * D + 64 * half);
 #pragma unroll
-                        for (int e = 0; e < D; e += 4)
+                        for (int e = 0; e < 64; e += 4)
                             dst[e / 4] = make_float4(o[e] * inv, o[e + 1] * inv, o[e + 2] * inv, o[e + 3] * inv);
                     }
-                    if (p.lse != nullptr) p.lse[row] = lse;
+                    if (half == 0 && p.lse != nullptr) p.lse[row] = lse;
                 }
             }
         }
@@ -546,7 +601,7 @@ __global__ void __launch_bounds__(QbtShape<G>::NT, 1)
         const int blk = u / per_blk;
         const int g = (u - blk * per_blk) / p.S;
         const int split = u - blk * per_blk - g * p.S;
-        for (int r = warp; r < R; r += 6) {
+        for (int r = warp; r < R; r += SH::NT / 32) {
             const int b = blk * BQ + r / G;
             if (b >= p.B) continue;
             const size_t row = (size_t)b * p.Hq + g * G + r % G;

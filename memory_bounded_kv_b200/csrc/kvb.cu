@@ -653,7 +653,7 @@ kvb_status kvb_asm_prepare(const float* qbar, int32_t H_tables, int32_t K, int32
                            size_t planes_bytes, kvb_stream stream) {
     if (d != kvb::kAsmD || H_tables < 1 || K < 1 || !qbar || !planes) return KVB_EINVAL;
     if (!aligned16(qbar) || !aligned16(planes) || planes_bytes < kvb_asm_planes_bytes(H_tables, K)) return KVB_EINVAL;
-    const long long rows = (long long)H_tables * (long long)kvb::asm_plane_tiles(K) * kvb::kUKT;
+    const long long rows = (long long)H_tables * (long long)kvb::asm_plane_tiles(K) * kvb::kPT;
     if ((rows + 7) / 8 > 0x7fffffffLL) return KVB_EINVAL;
     kvb::asm_prepare_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, static_cast<cudaStream_t>(stream)>>>(
         qbar, H_tables, K, static_cast<unsigned char*>(planes));
@@ -678,18 +678,21 @@ kvb_status kvb_asm_lookup_merge_planes(const uint16_t* q, const void* planes, si
     if (!aligned16(q) || !aligned16(planes) || !aligned16(workspace)) return KVB_EINVAL;
     if (workspace_bytes < kvb_asm_workspace_bytes(N, H, K)) return KVB_EINVAL;
     const int qtiles = (N + kvb::kUMT * kvb::kUQ - 1) / (kvb::kUMT * kvb::kUQ);
-    const long long items = (long long)H * qtiles * kvb::asm_ksplit(K);
-    if (items > (1ll << 30)) return KVB_EINVAL;
+    if ((long long)H * qtiles > (1ll << 30)) return KVB_EINVAL;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (set_smem(kvb::asm_score_planes_kernel, kvb::kPSmem) != KVB_OK) return KVB_ECUDA;
     const int slots = resident_ctas(kvb::asm_score_planes_kernel, kvb::kPThreads, kvb::kPSmem);
     if (slots < 1) return KVB_ECUDA;
+    // ranges of whole 128-centroid tiles, as many per (head, query block) as there are CTAs for it
+    const int kchunk = kvb::asm_planes_kchunk(K, H * qtiles, slots);
+    const int ksplit = (K + kchunk - 1) / kchunk;   // <= asm_ksplit(K): the workspace holds it
+    const long long items = (long long)H * qtiles * ksplit;
+    if (items > (1ll << 30)) return KVB_EINVAL;
     const int per_cta = (int)((items + slots - 1) / slots);
     const int grid = (int)((items + per_cta - 1) / per_cta);
     kvb::AsmPlanesParams pp;
-    pp.a = kvb::AsmParams{q, nullptr, abar, log_zbar, o_self, lse_self, N, H, K, kvb::asm_ksplit(K),
-                          kvb::asm_kchunk(K), qtiles, per_cta, idx, o, lse, static_cast<unsigned long long*>(workspace),
-                          H / H_tables};
+    pp.a = kvb::AsmParams{q, nullptr, abar, log_zbar, o_self, lse_self, N, H, K, ksplit, kchunk, qtiles, per_cta, idx,
+                          o, lse, static_cast<unsigned long long*>(workspace), H / H_tables};
     pp.planes = static_cast<const unsigned char*>(planes);
     pp.wait_ns = 1000000000ull;
     kvb::asm_score_planes_kernel<<<grid, kvb::kPThreads, kvb::kPSmem, st>>>(pp);

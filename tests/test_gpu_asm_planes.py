@@ -19,7 +19,8 @@ def run_planes(q, qbar, abar, lz, o_self, l_self, assign_only=False):
     N, H, d = q.shape
     Ht, K = qbar.shape[0], qbar.shape[1]
     planes = kvb.kvb_asm_prepare(dev(qbar))
-    assert planes.numel() == kvb.kvb_asm_planes_bytes(Ht, K) == Ht * (-(-K // 64)) * 3 * 2 * 64 * 128
+    # tiles of 128 centroids: three bf16 parts x two K halves x 128 rows x 128 bytes
+    assert planes.numel() == kvb.kvb_asm_planes_bytes(Ht, K) == Ht * (-(-K // 128)) * 3 * 2 * 128 * 128
     idx = torch.full((N, H), -7, dtype=torch.int32, device="cuda")
     o = None if assign_only else torch.zeros(N, H, d, device="cuda")
     lse = None if assign_only else torch.zeros(N, H, device="cuda")
@@ -104,3 +105,13 @@ def test_planes_attention_state_memory_shape(oracle):
     l_self = np.random.default_rng(4).uniform(3, 9, (w.N, w.H)).astype(np.float32)
     idx, o, lse = run_planes(w.q, w.qbar, w.abar, w.log_zbar, o_self, l_self)
     check_asm(oracle, w.q, w.qbar, w.abar, w.log_zbar, o_self, l_self, idx, o, lse)
+
+
+def test_planes_more_query_blocks_than_ctas(oracle):
+    """More (head, 256-query block) pairs than resident CTAs: a CTA walks two blocks, reloading the
+    queries between them; a ragged last block of 32 queries and a ragged last tile of 72 centroids."""
+    N, H, K = 800, 50, 200
+    args = asm_inputs(77, N, H, K)
+    idx, o, lse = run_planes(*args)
+    check_asm(oracle, *args, idx, o, lse)
+    assert kvb.kvb_get_error() == 0
