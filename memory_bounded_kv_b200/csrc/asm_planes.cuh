@@ -243,21 +243,36 @@ __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __
                     const int j = 3 * g + pt, s = j % kPStages;
                     if (!mbar_wait(&b_full[s], (unsigned)(j / kPStages) & 1u, pp.wait_ns)) { ok = false; break; }
                     tc_fence_after();
+                    if (pt < 2) {
 #pragma unroll
-                    for (int kk = 0; kk < kAsmD / 16; ++kk) {
-                        const uint32_t boff = (uint32_t)(s * kPPart + (kk >> 2) * kPHalf + (kk & 3) * 32);
+                        for (int kk = 0; kk < kAsmD / 16; ++kk) {
+                            const uint32_t boff = (uint32_t)(s * kPPart + (kk >> 2) * kPHalf + (kk & 3) * 32);
 #pragma unroll
-                        for (int mt = 0; mt < kUMT; ++mt) {   // the M tiles alternate (independent accumulators)
-                            if (mt >= mts) break;
-                            const uint32_t a = tmem + (uint32_t)(mt * (kAsmD / 2) + kk * 8);
-                            umma_bf16_ts(dacc[mt], a, b0 + (boff >> 4), idesc, (pt | kk) != 0);
+                            for (int mt = 0; mt < kUMT; ++mt) {   // the M tiles alternate (independent accumulators)
+                                if (mt >= mts) break;
+                                const uint32_t a = tmem + (uint32_t)(mt * (kAsmD / 2) + kk * 8);
+                                umma_bf16_ts(dacc[mt], a, b0 + (boff >> 4), idesc, (pt | kk) != 0);
+                            }
+                        }
+                    } else {
+                        // the last part one M tile after the other, each unit committed as soon as its
+                        // products are issued: the first unit's read-back starts a part's work earlier
+#pragma unroll
+                        for (int mt = 0; mt < kUMT; ++mt) {
+                            if (mt < mts) {
+#pragma unroll
+                                for (int kk = 0; kk < kAsmD / 16; ++kk) {
+                                    const uint32_t boff = (uint32_t)(s * kPPart + (kk >> 2) * kPHalf + (kk & 3) * 32);
+                                    const uint32_t a = tmem + (uint32_t)(mt * (kAsmD / 2) + kk * 8);
+                                    umma_bf16_ts(dacc[mt], a, b0 + (boff >> 4), idesc, 1u);
+                                }
+                            }
+                            umma_commit(&acc_full[(2 * g + mt) % kPAcc]);
                         }
                     }
                     umma_commit(&b_empty[s]);
                 }
                 if (!ok) break;
-#pragma unroll
-                for (int mt = 0; mt < kUMT; ++mt) umma_commit(&acc_full[(2 * g + mt) % kPAcc]);
                 ptile_next(p, cm);
             }
         }
@@ -307,39 +322,32 @@ __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __
             float best = -INFINITY;
             int first = -1;
             if (mine) {
+                // all four loads, one wait, release the buffer, then the arithmetic
                 const uint32_t ta = tmem + ((uint32_t)elane << 16) + (uint32_t)(kPACols + b * kPT);
+                float v[kPT];
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    float v[64];
-                    tmem_ld32(ta + 64 * hf, v);
-                    tmem_ld32(ta + 64 * hf + 32, v + 32);
-                    tmem_ld_wait();
-                    if (hf == 1) {   // the last read of the buffer: release it before the arithmetic
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&acc_empty[b]);
-                    }
-                    const int c0 = ce.kt + 64 * hf;
-                    if (c0 + 64 > ce.k_end) {   // ragged last tile of a range
+                for (int c = 0; c < kPT; c += 32) tmem_ld32(ta + c, v + c);
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[b]);
+                if (ce.kt + kPT > ce.k_end) {   // ragged last tile of a range
 #pragma unroll
-                        for (int c = 0; c < 64; ++c)
-                            if (c0 + c >= ce.k_end) v[c] = -INFINITY;
-                    }
-                    float m[32];
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) m[c] = fmaxf(v[c], v[c + 32]);
-#pragma unroll
-                    for (int w = 16; w >= 1; w >>= 1)
-#pragma unroll
-                        for (int c = 0; c < w; ++c) m[c] = fmaxf(m[c], m[c + w]);
-                    if (m[0] > best) {   // strictly greater: the earlier half keeps a tie
-                        int f = 63;
-#pragma unroll
-                        for (int c = 63; c >= 0; --c) f = (v[c] == m[0]) ? c : f;
-                        best = m[0];
-                        first = 64 * hf + f;
-                    }
+                    for (int c = 0; c < kPT; ++c)
+                        if (ce.kt + c >= ce.k_end) v[c] = -INFINITY;
                 }
+                float m[kPT / 2];
+#pragma unroll
+                for (int c = 0; c < kPT / 2; ++c) m[c] = fmaxf(v[c], v[c + kPT / 2]);
+#pragma unroll
+                for (int w = kPT / 4; w >= 1; w >>= 1)
+#pragma unroll
+                    for (int c = 0; c < w; ++c) m[c] = fmaxf(m[c], m[c + w]);
+                int f = kPT - 1;
+#pragma unroll
+                for (int c = kPT - 1; c >= 0; --c) f = (v[c] == m[0]) ? c : f;   // the first column of the max
+                best = m[0];
+                first = f;
             } else {
                 tc_fence_before();
                 __syncwarp();

@@ -7,16 +7,17 @@
 // is read once per 128 query rows and both products run as tcgen05.mma with
 // the accumulators in tensor memory.
 //
-// Roles (320 threads, one CTA per SM):
+// Roles (352 threads, one CTA per SM):
 //   warp 0     producer: the unit's 128 query rows by TMA (a 3-D box of 64
 //              dims x G heads x 128 / G rows b, K-major with the 128-byte
 //              swizzle, two buffers), K/V tiles by TMA into a 3-stage ring with
 //              their pos / log beta (bias) and the tile's record;
-//   warp 1     MMA issuer (one lane): S = Q K^T (M = 128, N = 64, K = 128)
-//              into one of two S buffers, and O += P V (M = 128, N = 128,
-//              K = 64) with P read from tensor memory (A operand) and V from
-//              shared memory as an MN-major B operand; S(i + 1) is issued
-//              before P V(i), so the softmax of tile i overlaps the next QK;
+//   warp 1     S issuer (one lane): S = Q K^T (M = 128, N = 64, K = 128) into
+//              one of two S buffers, so the softmax of tile i overlaps S(i + 1);
+//   warp 10    P V issuer (one lane): O += P V (M = 128, N = 128, K = 64) with
+//              P read from tensor memory (A operand) and V from shared memory
+//              as an MN-major B operand (two issuing threads: one thread
+//              issuing both products spent most of a tile waiting to issue);
 //   warps 2-9  softmax, two threads per query row (tensor-memory lane = row;
 //              warps w and w + 4 share a lane quarter, each takes 32 of the
 //              tile's 64 scores and 64 of O's 128 columns): read S, mask by the
@@ -48,7 +49,7 @@ struct QbtShape {
     static constexpr int BQ = R / G;          // rows b per unit
     static constexpr int T = 64;              // slots per tile
     static constexpr int ST = 3;              // K/V ring stages
-    static constexpr int NT = 10 * 32;        // producer, MMA issuer, 8 softmax warps
+    static constexpr int NT = 11 * 32;        // producer, S issuer, 8 softmax warps, P V issuer
     static constexpr int QHALF = R * 128;     // 128 rows x 64 dims of bf16
     static constexpr int QBUF = 2 * QHALF;
     static constexpr int KVHALF = T * 128;
@@ -62,9 +63,9 @@ struct QbtShape {
     static constexpr int META_OFF = LB_OFF + ST * T * 4;
     static constexpr int XCH_OFF = (META_OFF + ST * META * 4 + 15) / 16 * 16;   // half-row maxima [2][2][R], sums [2][R]
     static constexpr int BAR_OFF = XCH_OFF + 6 * R * 4;
-    // kv full/empty [ST] each; q, s, p full/empty [2] each; pv_done [2]; o_free; fin; the maxima
+    // kv full/empty [ST] each; q, s, p full/empty [2] each; pv_done [2]; o_free; fin [2]; the maxima
     // exchange [4 quarters][2]; the sums exchange [4]
-    static constexpr int NBAR = 2 * ST + 6 * 2 + 2 + 1 + 1 + 8 + 4;
+    static constexpr int NBAR = 2 * ST + 6 * 2 + 2 + 1 + 2 + 8 + 4;
     static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
     static constexpr int END = MISC_OFF + 32;
     static constexpr size_t SMEM = 1024 + END;
@@ -134,14 +135,13 @@ __global__ void __launch_bounds__(QbtShape<G>::NT, 1)
     // own barrier can never be two phases behind
     uint64_t* pv_done = p_empty + 2;
     uint64_t* o_free = pv_done + 2;
-    uint64_t* fin = o_free + 1;   // the MMA warp's last commit: every tensor-core operation done
-    uint64_t* xm_bar = fin + 1;   // [quarter][tile parity]: both warps of a lane quarter posted their maxima
+    uint64_t* fin = o_free + 1;   // [2] each MMA issuer's last commit: every operation it issued is done
+    uint64_t* xm_bar = fin + 2;   // [quarter][tile parity]: both warps of a lane quarter posted their maxima
     uint64_t* xl_bar = xm_bar + 8;   // [quarter]: both posted their sums (once per unit)
     // (xl_bar + 4 == bars + NBAR: the last barrier)
     uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + SH::MISC_OFF);
     volatile int* s_abort = reinterpret_cast<int*>(smem + SH::MISC_OFF) + 1;
     int* s_issued = reinterpret_cast<int*>(smem + SH::MISC_OFF) + 2;   // tiles the producer issued
-    int* s_mma = reinterpret_cast<int*>(smem + SH::MISC_OFF) + 3;      // PV products the MMA warp committed
     int* s_qloads = reinterpret_cast<int*>(smem + SH::MISC_OFF) + 4;   // query blocks the producer loaded
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -169,12 +169,12 @@ __global__ void __launch_bounds__(QbtShape<G>::NT, 1)
         mbar_init(&pv_done[0], 1);
         mbar_init(&pv_done[1], 1);
         mbar_init(o_free, 8);
-        mbar_init(fin, 1);
+        mbar_init(&fin[0], 1);
+        mbar_init(&fin[1], 1);
         for (int k = 0; k < 8; ++k) mbar_init(&xm_bar[k], 2);
         for (int k = 0; k < 4; ++k) mbar_init(&xl_bar[k], 2);
         *s_abort = 0;
         *s_issued = 0;
-        *s_mma = 0;
         *s_qloads = 0;
         fence_mbar_init();
     }
@@ -339,81 +339,74 @@ __global__ void __launch_bounds__(QbtShape<G>::NT, 1)
             *s_issued = it;
             *s_qloads = ucount;
         }
-    } else if (warp == 1) {
-        // ======================= MMA issuer =======================
+    } else if (warp == 1 || warp == SH::NT / 32 - 1) {
+        // ============ MMA issuers: S = Q K^T (warp 1), O += P V (the last warp) ============
+        // Two threads, so that neither product's issue waits behind the other's: tile i's P V
+        // needs P(i), hence S(i), hence Q K^T(i) done, so the stage it frees (kv_empty, committed
+        // after P V) is no longer read by either.
         if (lane == 0) {
+            const bool qk = warp == 1;
             constexpr uint32_t idesc_s = umma_idesc_bf16(R, T);          // S: 128 x 64
             constexpr uint32_t idesc_o = umma_idesc_bf16_bmn(R, D);      // O: 128 x 128, V MN-major
-            int i = 0, units_pv = 0, pv = 0, units_qk = 0;
-            bool pending = false;
-            int pend_st = 0, pend_first = 0, pend_i = 0;
+            int units = 0;
             auto fail = [&]() {
                 raise_error(KVB_DERR_TIMEOUT);
                 *s_abort = 1;
             };
-            auto issue_pv = [&](int st, int pi, int first) -> bool {
-                const int pb = pi & 1;
-                if (!mbar_wait(&p_full[pb], (unsigned)(pi >> 1) & 1u, p.wait_ns)) return false;
-                if (first && units_pv > 0 && !mbar_wait(o_free, (unsigned)(units_pv - 1) & 1u, p.wait_ns)) return false;
-                if (first) ++units_pv;
-                tc_fence_after();
-                const uint32_t vt = sbase + SH::RING_OFF + st * SH::STAGE + SH::KVTILE;
-#pragma unroll
-                for (int part = 0; part < 2; ++part)
-#pragma unroll
-                    for (int kk = 0; kk < T / 16; ++kk) {
-                        const uint32_t a = tmem + SH::TM_P + pb * 64 + part * 32 + kk * 8;
-                        const uint64_t bd = umma_desc_sw128_mn(vt + kk * 2048, SH::KVHALF, 1024);
-                        umma_bf16_ts(tmem + SH::TM_O, a, bd, idesc_o, (first && part == 0 && kk == 0) ? 0u : 1u);
-                    }
-                umma_commit(&kv_empty[st]);
-                umma_commit(&p_empty[pb]);
-                umma_commit(&pv_done[pb]);
-                ++pv;
-                return true;
-            };
-            while (true) {
+            for (int i = 0;; ++i) {
                 const int st = i % ST;
                 if (!mbar_wait(&kv_full[st], (unsigned)(i / ST) & 1u, p.wait_ns)) { fail(); break; }
                 const int* m = s_meta + st * SH::META;
                 const int u = m[0];
-                if (u < 0) {   // the end: the last P V
-                    if (pending && !issue_pv(pend_st, pend_i, pend_first)) fail();
-                    break;
-                }
+                if (u < 0) break;   // the end record
                 const int ti = m[1], ntiles = m[2], qb = m[9];
                 const int sb = i & 1;
-                // S(i) = Q K^T into buffer sb; a unit's first tile waits for its queries (the k-th unit
-                // uses query buffer k % 2 for the (k / 2)-th time)
-                if (ti == 0) {
-                    if (!mbar_wait(&q_full[qb], (unsigned)(units_qk >> 1) & 1u, p.wait_ns)) { fail(); break; }
-                    ++units_qk;
-                }
-                if (i >= 2 && !mbar_wait(&s_empty[sb], (unsigned)((i >> 1) - 1) & 1u, p.wait_ns)) { fail(); break; }
-                tc_fence_after();
-                const uint32_t qa = sbase + SH::Q_OFF + qb * SH::QBUF;
-                const uint32_t kt = sbase + SH::RING_OFF + st * SH::STAGE;
+                if (qk) {
+                    // S(i) into buffer i % 2; a unit's first tile waits for its queries (the k-th unit
+                    // uses query buffer k % 2 for the (k / 2)-th time)
+                    if (ti == 0) {
+                        if (!mbar_wait(&q_full[qb], (unsigned)(units >> 1) & 1u, p.wait_ns)) { fail(); break; }
+                        ++units;
+                    }
+                    if (i >= 2 && !mbar_wait(&s_empty[sb], (unsigned)((i >> 1) - 1) & 1u, p.wait_ns)) { fail(); break; }
+                    tc_fence_after();
+                    const uint32_t qa = sbase + SH::Q_OFF + qb * SH::QBUF;
+                    const uint32_t kt = sbase + SH::RING_OFF + st * SH::STAGE;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t aoff = (kk >> 2) * SH::QHALF + (kk & 3) * 32;
-                    const uint32_t boff = (kk >> 2) * SH::KVHALF + (kk & 3) * 32;
-                    umma_bf16(tmem + SH::TM_S + sb * 64, umma_desc_sw128(qa + aoff), umma_desc_sw128(kt + boff),
-                              idesc_s, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t aoff = (kk >> 2) * SH::QHALF + (kk & 3) * 32;
+                        const uint32_t boff = (kk >> 2) * SH::KVHALF + (kk & 3) * 32;
+                        umma_bf16(tmem + SH::TM_S + sb * 64, umma_desc_sw128(qa + aoff), umma_desc_sw128(kt + boff),
+                                  idesc_s, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(&s_full[sb]);
+                    if (ti == ntiles - 1) umma_commit(&q_empty[qb]);
+                } else {
+                    // O += P(i) V(i); a unit's first tile waits until the previous unit's O was read
+                    const int pb = sb;
+                    if (!mbar_wait(&p_full[pb], (unsigned)(i >> 1) & 1u, p.wait_ns)) { fail(); break; }
+                    if (ti == 0) {
+                        if (units > 0 && !mbar_wait(o_free, (unsigned)(units - 1) & 1u, p.wait_ns)) { fail(); break; }
+                        ++units;
+                    }
+                    tc_fence_after();
+                    const uint32_t vt = sbase + SH::RING_OFF + st * SH::STAGE + SH::KVTILE;
+#pragma unroll
+                    for (int part = 0; part < 2; ++part)
+#pragma unroll
+                        for (int kk = 0; kk < T / 16; ++kk) {
+                            const uint32_t a = tmem + SH::TM_P + pb * 64 + part * 32 + kk * 8;
+                            const uint64_t bd = umma_desc_sw128_mn(vt + kk * 2048, SH::KVHALF, 1024);
+                            umma_bf16_ts(tmem + SH::TM_O, a, bd, idesc_o, (ti == 0 && part == 0 && kk == 0) ? 0u : 1u);
+                        }
+                    umma_commit(&kv_empty[st]);
+                    umma_commit(&p_empty[pb]);
+                    umma_commit(&pv_done[pb]);
                 }
-                umma_commit(&s_full[sb]);
-                if (ti == ntiles - 1) umma_commit(&q_empty[qb]);
-                // P V of the previous tile, now that the tensor cores have the next S queued
-                if (pending && !issue_pv(pend_st, pend_i, pend_first)) { fail(); break; }
-                pending = true;
-                pend_st = st;
-                pend_i = i;
-                pend_first = (ti == 0);
-                ++i;
             }
-            *s_mma = pv;
         }
     } else {
-        // ======================= softmax warps =======================
+        // ======================= softmax warps (2 .. 9) =======================
         const int quarter = warp & 3;             // tensor-memory lanes 32 * quarter ..
         const int half = (warp - 2) >> 2;         // scores 32 half .. of a tile, O columns 64 half ..
         const int r = 32 * quarter + lane;        // this thread's query row
@@ -578,9 +571,10 @@ __global__ void __launch_bounds__(QbtShape<G>::NT, 1)
     // ---- teardown: copies and MMAs in flight finish (bounded) before the tensor memory goes
     tc_fence_before();
     __syncthreads();
-    if (warp == 1 && lane == 0) {
-        umma_commit(fin);   // arrives when every tensor-core operation this thread issued is done
-        mbar_wait(fin, 0u, p.wait_ns);
+    if ((warp == 1 || warp == SH::NT / 32 - 1) && lane == 0) {
+        uint64_t* f = &fin[warp == 1 ? 0 : 1];
+        umma_commit(f);   // arrives when every tensor-core operation this thread issued is done
+        mbar_wait(f, 0u, p.wait_ns);
     }
     if (tid == 0 && *s_abort) {
         const int issued = *s_issued;

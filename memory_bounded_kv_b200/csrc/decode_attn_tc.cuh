@@ -155,13 +155,22 @@ struct UnitRaw {
     int len, t;
 };
 
+// Unit u is split u mod S of row u / S, rows (b, g) in order. (A split-major order, meant to mix
+// the split indices of a CTA's round-robin units on ragged rows, measured slower on the memento
+// workload: 106.4 against 98.8 us per step.)
+__device__ __forceinline__ void unit_coords(const DecodeTcParams& p, int u, int& b, int& g, int& split) {
+    const int per_b = p.Hkv * p.S;
+    b = u / per_b;
+    const int rem = u - b * per_b;
+    g = rem / p.S;
+    split = rem - g * p.S;
+}
+
 __device__ __forceinline__ UnitRaw unit_raw(const DecodeTcParams& p, long long ul) {
     UnitRaw r{0, 0};
     if (ul < p.units) {
-        const int u = (int)ul;
-        const int per_b = p.Hkv * p.S;
-        const int b = u / per_b;
-        const int g = (u - b * per_b) / p.S;
+        int b, g, split;
+        unit_coords(p, (int)ul, b, g, split);
         r.len = p.len[b * p.Hkv + g];
         r.t = (p.t == nullptr) ? 0 : p.t[b];
     }
@@ -171,11 +180,7 @@ __device__ __forceinline__ UnitRaw unit_raw(const DecodeTcParams& p, long long u
 template <int T>
 __device__ __forceinline__ UnitInfo unit_info(const DecodeTcParams& p, int u, UnitRaw raw, bool record_errors) {
     UnitInfo r;
-    const int per_b = p.Hkv * p.S;
-    r.b = u / per_b;
-    const int rem = u - r.b * per_b;
-    r.g = rem / p.S;
-    r.split = rem - r.g * p.S;
+    unit_coords(p, u, r.b, r.g, r.split);
     int n = raw.len;
     const bool active = (p.t == nullptr) || (raw.t >= 0);
     const bool bad_len = n < 0 || n > p.cap;
@@ -296,8 +301,55 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                     }
                     page = __shfl_sync(kFull, lane_page, i & 31);
                 }
-                // this tile's bias (and, for the eviction candidates, its pos and log beta),
-                // loaded before waiting for the stage
+                // the stage's record and copies (lane 0); the first ST tiles need no stage to free, so
+                // their copies go out before this tile's pos / log beta loads, later ones after the
+                // wait (those loads are issued before it, so their latency hides behind the wait)
+                const bool data = !end && ui.ntiles > 0;
+                auto issue = [&]() {
+                    if (lane == 0) {
+                        int* m = s_meta + st * 16;
+                        m[0] = end ? -1 : u;
+                        m[1] = i;
+                        m[2] = end ? 0 : ui.ntiles;
+                        m[3] = data ? min(T, ui.nk - i * T) : 0;
+                        m[4] = ui.b;
+                        m[5] = ui.g;
+                        m[6] = ui.split;
+                        m[7] = ui.n;
+                        m[8] = tb;
+                        m[9] = ui.s0 + i * T;
+                        unsigned tx = data ? (unsigned)SH::STAGE_BYTES : 0u;
+                        const bool with_q = data && i == 0;
+                        if (with_q) tx += SH::QBYTES;
+                        mbar_arrive_expect_tx(&s_full[st], tx);
+                        if (data) {
+                            unsigned char* kt = smem + SH::RING_OFF + st * SH::STAGE_BYTES;
+                            unsigned char* vt = kt + SH::TILE_BYTES;
+                            // paged: the page's rows in the pool (one kv head, one "sequence" in the map)
+                            const int row = PAGED ? page * T : ui.s0 + i * T;
+                            const int gg = PAGED ? 0 : ui.g;
+                            const int bb = (PAGED || p.kv_shared) ? 0 : ui.b;
+#pragma unroll
+                            for (int h = 0; h < SH::HALVES; ++h) {
+                                tma_load_4d(kt + h * SH::HALF_BYTES, &tmK, 64 * h, row, gg, bb, &s_full[st]);
+                                tma_load_4d(vt + h * SH::HALF_BYTES, &tmV, 64 * h, row, gg, bb, &s_full[st]);
+                            }
+                        }
+                        if (with_q) {
+                            const uint16_t* qsrc = p.q + (size_t)ui.b * p.q_sb + (size_t)(ui.g * G) * p.q_sh;
+                            uint16_t* qdst = s_q + st * G * D;
+                            if (p.q_sh == D) {
+                                bulk_g2s(qdst, qsrc, (unsigned)SH::QBYTES, &s_full[st]);
+                            } else {
+                                for (int hh = 0; hh < G; ++hh)
+                                    bulk_g2s(qdst + hh * D, qsrc + (size_t)hh * p.q_sh, (unsigned)(D * 2), &s_full[st]);
+                            }
+                        }
+                    }
+                };
+                const bool early = it < ST;
+                if (early) issue();
+                // this tile's bias (and, for the eviction candidates, its pos and log beta)
                 const size_t mt = PAGED ? (size_t)page * T : m_off + (size_t)i * T;
                 float bias[T / 32];
                 int psv[T / 32];
@@ -327,51 +379,11 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                     stop = true;
                     break;
                 }
-                if (*s_abort) {
+                if (!early && *s_abort) {   // (an early tile's copies are out: it is arrived and counted)
                     stop = true;
                     break;
                 }
-                const bool data = !end && ui.ntiles > 0;
-                if (lane == 0) {
-                    int* m = s_meta + st * 16;
-                    m[0] = end ? -1 : u;
-                    m[1] = i;
-                    m[2] = end ? 0 : ui.ntiles;
-                    m[3] = data ? min(T, ui.nk - i * T) : 0;
-                    m[4] = ui.b;
-                    m[5] = ui.g;
-                    m[6] = ui.split;
-                    m[7] = ui.n;
-                    m[8] = tb;
-                    m[9] = ui.s0 + i * T;
-                    unsigned tx = data ? (unsigned)SH::STAGE_BYTES : 0u;
-                    const bool with_q = data && i == 0;
-                    if (with_q) tx += SH::QBYTES;
-                    mbar_arrive_expect_tx(&s_full[st], tx);
-                    if (data) {
-                        unsigned char* kt = smem + SH::RING_OFF + st * SH::STAGE_BYTES;
-                        unsigned char* vt = kt + SH::TILE_BYTES;
-                        // paged: the page's rows in the pool (one kv head, one "sequence" in the map)
-                        const int row = PAGED ? page * T : ui.s0 + i * T;
-                        const int gg = PAGED ? 0 : ui.g;
-                        const int bb = (PAGED || p.kv_shared) ? 0 : ui.b;
-#pragma unroll
-                        for (int h = 0; h < SH::HALVES; ++h) {
-                            tma_load_4d(kt + h * SH::HALF_BYTES, &tmK, 64 * h, row, gg, bb, &s_full[st]);
-                            tma_load_4d(vt + h * SH::HALF_BYTES, &tmV, 64 * h, row, gg, bb, &s_full[st]);
-                        }
-                    }
-                    if (with_q) {
-                        const uint16_t* qsrc = p.q + (size_t)ui.b * p.q_sb + (size_t)(ui.g * G) * p.q_sh;
-                        uint16_t* qdst = s_q + st * G * D;
-                        if (p.q_sh == D) {
-                            bulk_g2s(qdst, qsrc, (unsigned)SH::QBYTES, &s_full[st]);
-                        } else {
-                            for (int hh = 0; hh < G; ++hh)
-                                bulk_g2s(qdst + hh * D, qsrc + (size_t)hh * p.q_sh, (unsigned)(D * 2), &s_full[st]);
-                        }
-                    }
-                }
+                if (!early) issue();
 #pragma unroll
                 for (int j = 0; j < T / 32; ++j) {
                     s_bias[st * T + lane + 32 * j] = bias[j];
@@ -540,17 +552,13 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
             if (ntiles > 0 && i != ntiles - 1) continue;
 
             // ======== end of unit: combine warps, write the split's state ========
+            // each warp's share of a row is exp2(m_w - M) / L (M, L over the four warps); every warp
+            // folds its own share into its O before the sum, so the final pass only adds
             l_run += __shfl_xor_sync(kFull, l_run, 1);
             l_run += __shfl_xor_sync(kFull, l_run, 2);
-            if (r < G) {
-#pragma unroll
-                for (int j = 0; j < SH::NTILES; ++j)
-                    *reinterpret_cast<float2*>(s_o + (warp * G + r) * D + 8 * j + 2 * cq) =
-                        make_float2(acc[j][0], acc[j][1]);
-                if (cq == 0) {
-                    s_ml[(warp * G + r) * 2] = m_run;
-                    s_ml[(warp * G + r) * 2 + 1] = l_run;
-                }
+            if (r < G && cq == 0) {
+                s_ml[(warp * G + r) * 2] = m_run;
+                s_ml[(warp * G + r) * 2 + 1] = l_run;
             }
             if (want_cand) {
 #pragma unroll
@@ -567,7 +575,29 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                     s_cs[warp] = cand_slot;
                 }
             }
-            named_bar(1, NWC * 32);
+            named_bar(1, NWC * 32);   // every warp's (m, l) and candidate posted
+            const int S = p.S;
+            if (r < G) {
+                float M = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < NWC; ++w) M = fmaxf(M, s_ml[(w * G + r) * 2]);
+                const float Mu = (M == -INFINITY) ? 0.f : M;
+                float L = 0.f;
+#pragma unroll
+                for (int w = 0; w < NWC; ++w)
+                    L = fmaf(exp2f((s_ml[(w * G + r) * 2] - Mu) * kLog2e), s_ml[(w * G + r) * 2 + 1], L);
+                const float f = (L > 0.f) ? exp2f((m_run - Mu) * kLog2e) / L : 0.f;
+#pragma unroll
+                for (int j = 0; j < SH::NTILES; ++j)
+                    *reinterpret_cast<float2*>(s_o + (warp * G + r) * D + 8 * j + 2 * cq) =
+                        make_float2(acc[j][0] * f, acc[j][1] * f);
+                if (warp == 0 && cq == 0) {
+                    const float lse = (L > 0.f) ? M + log2f(L) * kLn2 : -INFINITY;
+                    const size_t row = (size_t)ub * p.Hq + ug * G + r;
+                    if (p.o_part != nullptr) p.lse_part[row * S + usplit] = lse;
+                    if (S == 1 && p.lse != nullptr) p.lse[row] = lse;
+                }
+            }
             if (want_cand && tid == 0) {
                 unsigned long long bk = s_ck[0];
                 int bs = s_cs[0];
@@ -582,37 +612,25 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                 c->slot = (bk == ~0ull) ? -1 : bs;
                 c->t = ut + 1;
             }
-            const int S = p.S;
+            named_bar(1, NWC * 32);   // every warp's scaled O posted
             for (int idx = tid; idx < G * D; idx += NWC * 32) {
                 const int hh = idx / D, e = idx % D;
-                float M = -INFINITY;
+                float out = 0.f;
 #pragma unroll
-                for (int w = 0; w < NWC; ++w) M = fmaxf(M, s_ml[(w * G + hh) * 2]);
-                const float Mu = (M == -INFINITY) ? 0.f : M;
-                float L = 0.f, O = 0.f;
-#pragma unroll
-                for (int w = 0; w < NWC; ++w) {
-                    const float f = exp2f((s_ml[(w * G + hh) * 2] - Mu) * kLog2e);
-                    L = fmaf(f, s_ml[(w * G + hh) * 2 + 1], L);
-                    O = fmaf(f, s_o[(w * G + hh) * D + e], O);
-                }
-                const float out = (L > 0.f) ? O / L : 0.f;
-                const float lse = (L > 0.f) ? M + log2f(L) * kLn2 : -INFINITY;
+                for (int w = 0; w < NWC; ++w) out += s_o[(w * G + hh) * D + e];
                 const size_t row = (size_t)ub * p.Hq + ug * G + hh;
-                if (p.o_part != nullptr) {
-                    p.o_part[(row * S + usplit) * D + e] = out;
-                    if (e == 0) p.lse_part[row * S + usplit] = lse;
-                }
+                if (p.o_part != nullptr) p.o_part[(row * S + usplit) * D + e] = out;
                 if (S == 1) {
                     if (p.o_bf16) {
                         reinterpret_cast<__nv_bfloat16*>(p.o)[row * D + e] = __float2bfloat16_rn(out);
                     } else {
                         reinterpret_cast<float*>(p.o)[row * D + e] = out;
                     }
-                    if (e == 0 && p.lse != nullptr) p.lse[row] = lse;
                 }
             }
-            named_bar(1, NWC * 32);  // s_o and s_ml free for the next unit
+            // no third barrier: the next unit writes s_ml and the candidates only after passing the
+            // second barrier above (so every read of them is done), and s_o only after its own first
+            // barrier, which every thread reaches after this loop
         }
         (void)aborted;
     }
@@ -627,10 +645,8 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
     __syncthreads();
     // a CTA that gave up leaves every unit it owns in the empty state (and no eviction candidate)
     for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
-        const int per_b = p.Hkv * p.S;
-        const int b = u / per_b;
-        const int g = (u - b * per_b) / p.S;
-        const int split = u - b * per_b - g * p.S;
+        int b, g, split;
+        unit_coords(p, u, b, g, split);
         const size_t row0 = (size_t)b * p.Hq + g * G;
         if (p.o_part != nullptr && tid < G) p.lse_part[(row0 + tid) * p.S + split] = -INFINITY;
         if (p.S == 1) {
