@@ -10,7 +10,7 @@
 // Roles (352 threads, one CTA per SM):
 //   warp 0     producer: the unit's 128 query rows by TMA (a 3-D box of 64
 //              dims x G heads x 128 / G rows b, K-major with the 128-byte
-//              swizzle, two buffers), K/V tiles by TMA into a 3-stage ring with
+//              swizzle, two buffers), K/V tiles by TMA into a 4-stage ring with
 //              their pos / log beta (bias) and the tile's record;
 //   warp 1     S issuer (one lane): S = Q K^T (M = 128, N = 64, K = 128) into
 //              one of two S buffers, so the softmax of tile i overlaps S(i + 1);
@@ -48,7 +48,7 @@ struct QbtShape {
     static constexpr int R = 128;             // query rows per unit = tensor-memory lanes
     static constexpr int BQ = R / G;          // rows b per unit
     static constexpr int T = 64;              // slots per tile
-    static constexpr int ST = 3;              // K/V ring stages
+    static constexpr int ST = 4;              // K/V ring stages (3 left the copies of a stage freed by P V late)
     static constexpr int NT = 11 * 32;        // producer, S issuer, 8 softmax warps, P V issuer
     static constexpr int QHALF = R * 128;     // 128 rows x 64 dims of bf16
     static constexpr int QBUF = 2 * QHALF;
