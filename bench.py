@@ -90,6 +90,9 @@ def parse(argv=None):
     ap.add_argument("--replay", default=None, metavar="DIR",
                     help="instead of timing, run the step dumped under DIR once and write its outputs and "
                          "the cache after it under DIR/replayed")
+    ap.add_argument("--profile", default=None, choices=list(PROFILE_CASES),
+                    help="instead of timing, run a few launches of one workload's dominant kernel at its shape "
+                         "(for ncu captures: small device footprint, no schedule walk)")
     ap.add_argument("--impl", default="kvb", choices=["kvb", "reference"])
     ap.add_argument("--splits", type=int, default=0, help="num_splits of the headline workload (0: its default)")
     ap.add_argument("--no-e2e", action="store_true")
@@ -1144,6 +1147,83 @@ def run_workload(key, splits, args, world, local, K, W, hbm_peak, peak_kind, cpu
     return r
 
 
+# ----------------------------------------------------------------------------------------------
+# profiling cases: the dominant launches of each workload at its shape, a few times
+# ----------------------------------------------------------------------------------------------
+
+def _profile_decode(B, Hq, Hkv, d, cap, lens, S, split_len, bias, reps=4):
+    """kvb_decode_attn over a filled cache (K, V ~ N(0, 1), log beta ~ U(-3, -0.01), positions 0..cap-1)
+    with the given lengths, `reps` times."""
+    import memory_bounded_kv_b200 as kvb
+    from memory_bounded_kv_b200.cache import BoundedKVCache
+    g = torch.Generator(device="cuda").manual_seed(0)
+    c = BoundedKVCache(B, Hq, Hkv, d, cap, cap, num_splits=S, split_len=split_len, with_beta=bias)
+    c.k.normal_(generator=g)
+    c.v.normal_(generator=g)
+    if bias:
+        c.log_beta.uniform_(-3, -0.01, generator=g)
+    c.pos.copy_(torch.arange(cap, dtype=torch.int32, device="cuda").expand(B, Hkv, cap))
+    c.len.copy_(torch.as_tensor(lens, dtype=torch.int32, device="cuda"))
+    q = torch.randn(B, Hq, d, device="cuda", generator=g).to(torch.bfloat16)
+    t = torch.full((B,), cap + 1, dtype=torch.int32, device="cuda")
+    o = torch.zeros(B, Hq, d, device="cuda")
+    lse = torch.zeros(B, Hq, device="cuda")
+    for _ in range(reps):
+        c.attend(q, t, o, lse)
+    torch.cuda.synchronize()
+    return kvb.kvb_get_error()
+
+
+def _profile_c2():
+    """The Qwen3-8B-shaped layer: 32 x 8 rows of 4096 slots, one split."""
+    return _profile_decode(32, 32, 8, 128, 4096, np.full((32, 8), 4096), 1, 0, True)
+
+
+def _profile_c3():
+    """The long-context workload's attention: 4 x 8 rows of 8192 slots, 64 splits."""
+    return _profile_decode(4, 32, 8, 128, 8192, np.full((4, 8), 8192), 64, 0, True)
+
+
+def _profile_c5():
+    """A mid-schedule memento cache: 64 x 8 rows, ragged lengths U[300, 3000), splits of 512 slots."""
+    lens = np.repeat(np.random.default_rng(0).integers(300, 3000, 64)[:, None], 8, axis=1)
+    return _profile_decode(64, 32, 8, 128, 3072, lens, 34, 512, False)
+
+
+def _profile_c4():
+    """The attention-state-memory step: shared-prefix self attention (4 splits of 512) and the lookup
+    over the prepared memory, four times."""
+    import memory_bounded_kv_b200 as kvb
+    from memory_bounded_kv_b200 import synth
+    w = synth.asm_workload()
+    N, H, Hkv, d = w.N, w.H, w.Hkv, w.d
+    k, v, pos = _dev(w.k).expand(N, Hkv, w.L, d), _dev(w.v).expand(N, Hkv, w.L, d), _dev(w.pos).expand(N, Hkv, w.L)
+    q, ln, t = _dev(w.q), _dev(w.len), _dev(w.t)
+    o_self = torch.zeros(N, H, d, device="cuda")
+    l_self = torch.zeros(N, H, device="cuda")
+    op, lp = kvb.decode_workspace(N, H, d, 4)
+    planes = kvb.kvb_asm_prepare(_dev(w.qbar))
+    abar, lz = _dev(w.abar), _dev(w.log_zbar)
+    idx = torch.zeros(N, H, dtype=torch.int32, device="cuda")
+    o = torch.zeros(N, H, d, device="cuda")
+    lse = torch.zeros(N, H, device="cuda")
+    ws = torch.empty(kvb.kvb_asm_workspace_bytes(N, H, w.K), dtype=torch.uint8, device="cuda")
+    for _ in range(4):
+        kvb.kvb_decode_attn(q, k, v, None, pos, ln, t, o_self, l_self, num_splits=4, split_len=512, o_part=op,
+                            lse_part=lp)
+        kvb.kvb_asm_lookup_merge_planes(q, planes, H, w.K, abar, lz, o_self, l_self, idx, o, lse, ws)
+    torch.cuda.synchronize()
+    return kvb.kvb_get_error()
+
+
+PROFILE_CASES = {"c2": _profile_c2, "c3": _profile_c3, "c4": _profile_c4, "c5": _profile_c5}
+
+
+def run_profile(case):
+    err = PROFILE_CASES[case]()
+    return {"profile": case, "device_error": err}
+
+
 def run_replay(path):
     """One dumped step through the library: its outputs and the cache after it go to
     path/replayed (same format), with the device error word."""
@@ -1416,6 +1496,12 @@ def main():
         return
     if args.replay:
         print(json.dumps(run_replay(args.replay)), flush=True)
+        return
+    if args.profile:
+        out = run_profile(args.profile)
+        print(json.dumps(out), flush=True)
+        if out["device_error"]:
+            sys.exit(1)
         return
     world, rank, local = dist_init()
     try:

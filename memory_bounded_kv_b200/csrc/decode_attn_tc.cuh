@@ -690,6 +690,23 @@ __global__ void __launch_bounds__(256) merge_splits_kernel(const float* __restri
     float acc[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] = 0.f;
+    // the o rows of splits j + k, k < min(8, n), whose weight w (lane j + k of the chunk, or any
+    // split when `spec`) is positive: empty splits are not read
+    float v[8][E];
+    auto load_batch = [&](int j, int n, float w, bool spec) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const float* src = op + (size_t)(j + k) * D;
+            const bool use = k < n && (spec || __shfl_sync(kFull, w, (j + k) & 31) > 0.f);
+            if constexpr (E == 4) {
+                const float4 x = use ? __ldcg(reinterpret_cast<const float4*>(src)) : make_float4(0.f, 0.f, 0.f, 0.f);
+                v[k][0] = x.x; v[k][1] = x.y; v[k][2] = x.z; v[k][3] = x.w;
+            } else {
+                const float2 x = use ? __ldcg(reinterpret_cast<const float2*>(src)) : make_float2(0.f, 0.f);
+                v[k][0] = x.x; v[k][1] = x.y;
+            }
+        }
+    };
     for (int j0 = 0; j0 < S; j0 += 32) {
         const int cnt = min(32, S - j0);
         const float l = (lane < cnt) ? __ldcg(lp + j0 + lane) : -INFINITY;
@@ -708,25 +725,18 @@ __global__ void __launch_bounds__(256) merge_splits_kernel(const float* __restri
 #pragma unroll
         for (int e = 0; e < E; ++e) acc[e] *= a;
         for (int k0 = 0; k0 < cnt; k0 += 8) {
+            load_batch(j0 + k0, cnt - k0, wl, false);
             float w[8];
-            float v[8][E];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                w[k] = __shfl_sync(kFull, wl, (k0 + k) & 31);
-                const bool use = (k0 + k < cnt) && w[k] > 0.f;
-                const float* src = op + (size_t)(j0 + k0 + k) * D;
-                if constexpr (E == 4) {
-                    const float4 x = use ? __ldcg(reinterpret_cast<const float4*>(src)) : make_float4(0.f, 0.f, 0.f, 0.f);
-                    v[k][0] = x.x; v[k][1] = x.y; v[k][2] = x.z; v[k][3] = x.w;
-                } else {
-                    const float2 x = use ? __ldcg(reinterpret_cast<const float2*>(src)) : make_float2(0.f, 0.f);
-                    v[k][0] = x.x; v[k][1] = x.y;
-                }
-            }
+            for (int k = 0; k < 8; ++k) w[k] = __shfl_sync(kFull, wl, (k0 + k) & 31);
+            // an empty split (weight 0) contributes nothing; its o rows were never written, so they are
+            // skipped rather than multiplied by 0
 #pragma unroll
             for (int k = 0; k < 8; ++k)
+                if (k0 + k < cnt && w[k] > 0.f) {
 #pragma unroll
-                for (int e = 0; e < E; ++e) acc[e] = fmaf(w[k], v[k][e], acc[e]);
+                    for (int e = 0; e < E; ++e) acc[e] = fmaf(w[k], v[k][e], acc[e]);
+                }
         }
     }
     const float inv = (s_run > 0.f) ? 1.f / s_run : 0.f;
@@ -767,8 +777,26 @@ __global__ void __launch_bounds__(256) merge_splits_cta_kernel(const float* __re
     float acc[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] = 0.f;
+    // the o rows of splits j + k, k < min(8, n), whose weight w (lane j + k of the chunk, or any
+    // split when `spec`) is positive: empty splits are not read
+    float v[8][E];
+    auto load_batch = [&](int j, int n, float w, bool spec) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const float* src = op + (size_t)(j + k) * D;
+            const bool use = k < n && (spec || __shfl_sync(kFull, w, (j + k) & 31) > 0.f);
+            if constexpr (E == 4) {
+                const float4 x = use ? __ldcg(reinterpret_cast<const float4*>(src)) : make_float4(0.f, 0.f, 0.f, 0.f);
+                v[k][0] = x.x; v[k][1] = x.y; v[k][2] = x.z; v[k][3] = x.w;
+            } else {
+                const float2 x = use ? __ldcg(reinterpret_cast<const float2*>(src)) : make_float2(0.f, 0.f);
+                v[k][0] = x.x; v[k][1] = x.y;
+            }
+        }
+    };
     for (int j0 = j_beg; j0 < j_end; j0 += 32) {
         const int cnt = min(32, j_end - j0);
+        load_batch(j0, cnt, 0.f, true);   // (rows here are few and their splits mostly full)
         const float l = (lane < cnt) ? __ldcg(lp + j0 + lane) : -INFINITY;
         float cm = l;
 #pragma unroll
@@ -785,25 +813,18 @@ __global__ void __launch_bounds__(256) merge_splits_cta_kernel(const float* __re
 #pragma unroll
         for (int e = 0; e < E; ++e) acc[e] *= a;
         for (int k0 = 0; k0 < cnt; k0 += 8) {
+            if (k0 > 0) load_batch(j0 + k0, cnt - k0, wl, false);
             float w[8];
-            float v[8][E];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                w[k] = __shfl_sync(kFull, wl, (k0 + k) & 31);
-                const bool use = (k0 + k < cnt) && w[k] > 0.f;
-                const float* src = op + (size_t)(j0 + k0 + k) * D;
-                if constexpr (E == 4) {
-                    const float4 x = use ? __ldcg(reinterpret_cast<const float4*>(src)) : make_float4(0.f, 0.f, 0.f, 0.f);
-                    v[k][0] = x.x; v[k][1] = x.y; v[k][2] = x.z; v[k][3] = x.w;
-                } else {
-                    const float2 x = use ? __ldcg(reinterpret_cast<const float2*>(src)) : make_float2(0.f, 0.f);
-                    v[k][0] = x.x; v[k][1] = x.y;
-                }
-            }
+            for (int k = 0; k < 8; ++k) w[k] = __shfl_sync(kFull, wl, (k0 + k) & 31);
+            // an empty split (weight 0) contributes nothing; its o rows were never written, so they are
+            // skipped rather than multiplied by 0
 #pragma unroll
             for (int k = 0; k < 8; ++k)
+                if (k0 + k < cnt && w[k] > 0.f) {
 #pragma unroll
-                for (int e = 0; e < E; ++e) acc[e] = fmaf(w[k], v[k][e], acc[e]);
+                    for (int e = 0; e < E; ++e) acc[e] = fmaf(w[k], v[k][e], acc[e]);
+                }
         }
     }
     if (lane == 0) {
