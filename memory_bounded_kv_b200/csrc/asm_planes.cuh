@@ -7,24 +7,28 @@
 // 16-byte chunk c of row r at chunk c ^ (r & 7) (the 128-byte swizzle).
 //
 // asm_score_planes_kernel streams those images with bulk copies, one part of a
-// tile (32 KB) per stage of a 6-stage ring, and keeps the queries in tensor
-// memory as the A operand of tcgen05.mma (M = 128 queries, N = 128 centroids,
-// K = 16: the shape the tensor cores run at full rate; N = 64 ran at ~70 %).
-// A tile is two units, one per block of 128 queries (M tile); each unit's
-// accumulator takes one of three 128-column buffers in turn (unit u -> buffer
-// u % 3), so the MMAs of a tile proceed while the previous units are read back:
-//   warp 9 (one lane)  bulk copies of the parts                       -> b_full[s]
+// tile (32 KB) per stage of a 5-stage ring, and keeps the block's 256 queries in
+// shared memory (one TMA box per M tile and K half, K-major, 128-byte swizzle):
+// every tcgen05.mma is M = 128 queries, N = 128 centroids, K = 16, the shape the
+// tensor cores run at full rate (N = 64 ran at ~70 %). A tile is two units, one
+// per M tile; unit (g, m) accumulates in buffer 2 (g % 2) + m of four 128-column
+// tensor-memory buffers, so tile g + 1's products never wait for tile g's
+// read-back:
+//   warp 9 (one lane)  the block's queries (-> a_full; a new block waits for
+//                      a_empty), then the parts of each tile    -> b_full[s]
 //   warp 8 (one lane)  per part 16 MMAs (8 K steps x 2 M tiles, the M tiles
-//                      alternating), committed to b_empty[s]; per tile the
-//                      two units' buffers, committed to acc_full[b]
-//   warps 0-7          the queries into tensor memory (tcgen05.st) at each new
-//                      block of 256 queries (-> a_ready), then per tile: warps
-//                      4 m .. 4 m + 3 read back unit m's 128 scores of their
-//                      query row (tcgen05.ld), release the buffer
+//                      alternating), committed to b_empty[s]; each unit's
+//                      buffer committed to acc_full[b] (the last part is issued
+//                      one M tile after the other, so the first unit is ready a
+//                      part's work earlier); a block's last tile -> a_empty
+//   warps 0-7          warps 4 m .. 4 m + 3 read back unit m's 128 scores of
+//                      their query row (tcgen05.ld), release the buffer
 //                      (-> acc_empty[b]) and keep the running best.
 // The per-range best keys go to the same workspace as asm_score_umma_kernel's,
 // reduced and merged by asm_merge_kernel.
 #pragma once
+
+#include <cuda.h>
 
 #include "asm_lookup.cuh"
 
@@ -34,14 +38,17 @@ constexpr int kPT = 128;                                        // centroids per
 constexpr size_t kPHalf = (size_t)kPT * 128;                    // one K half of one part: 16 KB
 constexpr size_t kPPart = 2 * kPHalf;                           // one part: 32 KB (a ring stage)
 constexpr size_t kPImg = 3 * kPPart;                            // one tile image: 96 KB
-constexpr int kPStages = 6;                                     // ring stages (two tiles)
-constexpr int kPAcc = 3;                                        // accumulator buffers (units)
+constexpr int kPStages = 5;                                     // ring stages (one part each)
+constexpr int kPAcc = 4;                                        // accumulator buffers: two per M tile
 constexpr int kPThreads = kUNT + 64;                            // 8 read-back warps + MMA warp + copy warp
-constexpr int kPACols = kUMT * (kAsmD / 2);                     // queries: 2 M tiles x 64 columns
-constexpr int kPCols = 512;                                     // kPACols + kPAcc * kPT
-constexpr size_t kPBar = (size_t)kPStages * kPPart;             // after the ring
+constexpr int kPCols = 512;                                     // kPAcc * kPT
+constexpr size_t kPAHalf = (size_t)kUQ * 128;                   // queries: one M tile, one K half: 16 KB
+constexpr size_t kPA = (size_t)kUMT * 2 * kPAHalf;              // queries [M tile][K half][128 rows][128 B]
+constexpr size_t kPRing = kPA;                                  // the ring after the queries
+constexpr size_t kPBar = kPRing + (size_t)kPStages * kPPart;    // after the ring
 constexpr size_t kPSmem = kPBar + 256 + 1024;                   // barriers + slot, + alignment slack
-static_assert(kPACols + kPAcc * kPT == kPCols, "tensor memory budget");
+static_assert(kPAcc * kPT == kPCols, "tensor memory budget");
+static_assert(kPSmem <= 227 * 1024, "shared memory budget");
 
 __host__ __device__ inline size_t asm_plane_tiles(int K) { return (size_t)(K + kPT - 1) / kPT; }
 
@@ -115,6 +122,15 @@ struct AsmPlanesParams {
     unsigned long long wait_ns;
 };
 
+// 3-D box copy (x = dims, y = head, z = query) of the queries' tensor map into shared memory
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int c0, int c1, int c2, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+        : "memory");
+}
+
 // The tile stream of a CTA: its run of items (head, query block, centroid range), each range
 // walked in tiles of kPT centroids (items are head-major, so the queries change rarely).
 struct PTile {
@@ -142,7 +158,8 @@ __device__ __forceinline__ void ptile_next(const AsmParams& p, PTile& c) {
     c.k_end = min(p.K, c.kt + p.kchunk);
 }
 
-__global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __grid_constant__ AsmPlanesParams pp) {
+__global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __grid_constant__ AsmPlanesParams pp,
+                                                                        const __grid_constant__ CUtensorMap tmQ) {
     const AsmParams& p = pp.a;
     extern __shared__ unsigned char s_raw[];
     unsigned char* sm = s_raw + ((1024u - (smem_u32(s_raw) & 1023u)) & 1023u);
@@ -151,8 +168,9 @@ __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __
     uint64_t* b_empty = b_full + kPStages;
     uint64_t* acc_full = b_empty + kPStages;
     uint64_t* acc_empty = acc_full + kPAcc;
-    uint64_t* a_ready = acc_empty + kPAcc;
-    uint32_t* slot = reinterpret_cast<uint32_t*>(a_ready + 1);
+    uint64_t* a_full = acc_empty + kPAcc;   // the block's queries landed
+    uint64_t* a_empty = a_full + 1;         // every MMA that read them is done
+    uint32_t* slot = reinterpret_cast<uint32_t*>(a_empty + 1);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int items = p.H * p.qtiles * p.ksplit;
     const int i0 = blockIdx.x * p.per_cta, i1 = min(items, i0 + p.per_cta);
@@ -179,7 +197,8 @@ __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __
             mbar_init(&acc_full[b], 1);
             mbar_init(&acc_empty[b], 4);   // the four warps of the unit's M tile
         }
-        mbar_init(a_ready, kUNT / 32);
+        mbar_init(a_full, 1);
+        mbar_init(a_empty, 1);
         fence_mbar_init();
     }
     tc_fence_before();
@@ -189,12 +208,29 @@ __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __
     bool ok = true;
 
     if (warp == kUNT / 32 + 1) {
-        // ---- copy warp: the parts of each tile into the ring, one stage each
+        // ---- copy warp: each block's queries, then the parts of each tile into the ring
         if (lane == 0) {
             PTile c;
             ptile_start(p, c, i0);
-            int issued = 0;   // stages whose copies were issued
+            int issued = 0, blocks = 0, a_block = -1;
             for (int g = 0; g < G && ok; ++g) {
+                const int blk = c.h * p.qtiles + c.qt;
+                if (blk != a_block) {
+                    // the previous block's MMAs are done before its queries are replaced
+                    if (blocks > 0 && !mbar_wait(a_empty, (unsigned)(blocks - 1) & 1u, pp.wait_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(a_full, (unsigned)kPA);
+#pragma unroll
+                    for (int mt = 0; mt < kUMT; ++mt)
+#pragma unroll
+                        for (int kh = 0; kh < 2; ++kh)   // rows past N read zeros
+                            tma_load_3d(sm + (size_t)(mt * 2 + kh) * kPAHalf, &tmQ, 64 * kh, c.h,
+                                        c.qt * (kUMT * kUQ) + mt * kUQ, a_full);
+                    ++blocks;
+                    a_block = blk;
+                }
                 const unsigned char* src = pp.planes + ((size_t)(c.h / p.G) * tiles_per_table + c.kt / kPT) * kPImg;
                 for (int pt = 0; pt < 3; ++pt) {
                     const int j = 3 * g + pt, s = j % kPStages;
@@ -202,16 +238,19 @@ __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __
                         ok = false;
                         break;
                     }
+                    unsigned char* dst = sm + kPRing + (size_t)s * kPPart;
                     mbar_arrive_expect_tx(&b_full[s], (unsigned)kPPart);
-                    bulk_g2s(sm + (size_t)s * kPPart, src + pt * kPPart, (unsigned)kPHalf, &b_full[s]);
-                    bulk_g2s(sm + (size_t)s * kPPart + kPHalf, src + pt * kPPart + kPHalf, (unsigned)kPHalf, &b_full[s]);
+                    bulk_g2s(dst, src + pt * kPPart, (unsigned)kPHalf, &b_full[s]);
+                    bulk_g2s(dst + kPHalf, src + pt * kPPart + kPHalf, (unsigned)kPHalf, &b_full[s]);
                     issued = j + 1;
                 }
                 ptile_next(p, c);
             }
-            // every copy lands before the CTA can exit (bounded): the last stage issued on each slot
+            // every copy lands before the CTA can exit (bounded): the last stage issued on each slot,
+            // and the last block's queries
             for (int j = max(0, issued - kPStages); j < issued; ++j)
                 mbar_wait(&b_full[j % kPStages], (unsigned)(j / kPStages) & 1u, 100000000ull);
+            if (blocks > 0) mbar_wait(a_full, (unsigned)(blocks - 1) & 1u, 100000000ull);
         }
     } else if (warp == kUNT / 32) {
         // ---- MMA warp
@@ -219,23 +258,23 @@ __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __
             PTile cm;
             ptile_start(p, cm, i0);
             constexpr uint32_t idesc = umma_idesc_bf16(kUQ, kPT);
-            const uint64_t b0 = umma_desc_sw128(sbase);
-            int a_block = -1, a_phase = 0;
+            const uint64_t a0 = umma_desc_sw128(sbase);
+            const uint64_t b0 = umma_desc_sw128(sbase + (uint32_t)kPRing);
+            int a_block = -1, blocks = 0;
             for (int g = 0; g < G && ok; ++g) {
-                // the two units of tile g take buffers (2g) % 3 and (2g + 1) % 3, free once the units three
-                // before them are read back
+                // unit (g, m) takes buffer 2 (g % 2) + m, free once tile g - 2's unit m is read back
                 uint32_t dacc[kUMT];
 #pragma unroll
                 for (int mt = 0; mt < kUMT; ++mt) {
-                    const int u = 2 * g + mt, b = u % kPAcc;
-                    dacc[mt] = tmem + (uint32_t)(kPACols + b * kPT);
-                    if (u >= kPAcc && !mbar_wait(&acc_empty[b], (unsigned)((u / kPAcc) - 1) & 1u, pp.wait_ns)) ok = false;
+                    const int b = 2 * (g & 1) + mt;
+                    dacc[mt] = tmem + (uint32_t)(b * kPT);
+                    if (g >= 2 && !mbar_wait(&acc_empty[b], (unsigned)((g >> 1) - 1) & 1u, pp.wait_ns)) ok = false;
                 }
                 if (!ok) break;
                 const int blk = cm.h * p.qtiles + cm.qt;
-                if (blk != a_block) {   // the read-back warps have put this block's queries in tensor memory
-                    if (!mbar_wait(a_ready, (unsigned)a_phase & 1u, pp.wait_ns)) { ok = false; break; }
-                    ++a_phase;
+                if (blk != a_block) {
+                    if (!mbar_wait(a_full, (unsigned)blocks & 1u, pp.wait_ns)) { ok = false; break; }
+                    ++blocks;
                     a_block = blk;
                 }
                 const int mts = min(kUMT, (p.N - cm.qt * (kUMT * kUQ) + kUQ - 1) / kUQ);
@@ -250,8 +289,8 @@ __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __
 #pragma unroll
                             for (int mt = 0; mt < kUMT; ++mt) {   // the M tiles alternate (independent accumulators)
                                 if (mt >= mts) break;
-                                const uint32_t a = tmem + (uint32_t)(mt * (kAsmD / 2) + kk * 8);
-                                umma_bf16_ts(dacc[mt], a, b0 + (boff >> 4), idesc, (pt | kk) != 0);
+                                const uint32_t aoff = (uint32_t)((mt * 2 + (kk >> 2)) * kPAHalf + (kk & 3) * 32);
+                                umma_bf16(dacc[mt], a0 + (aoff >> 4), b0 + (boff >> 4), idesc, (pt | kk) != 0);
                             }
                         }
                     } else {
@@ -263,67 +302,44 @@ __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __
 #pragma unroll
                                 for (int kk = 0; kk < kAsmD / 16; ++kk) {
                                     const uint32_t boff = (uint32_t)(s * kPPart + (kk >> 2) * kPHalf + (kk & 3) * 32);
-                                    const uint32_t a = tmem + (uint32_t)(mt * (kAsmD / 2) + kk * 8);
-                                    umma_bf16_ts(dacc[mt], a, b0 + (boff >> 4), idesc, 1u);
+                                    const uint32_t aoff = (uint32_t)((mt * 2 + (kk >> 2)) * kPAHalf + (kk & 3) * 32);
+                                    umma_bf16(dacc[mt], a0 + (aoff >> 4), b0 + (boff >> 4), idesc, 1u);
                                 }
                             }
-                            umma_commit(&acc_full[(2 * g + mt) % kPAcc]);
+                            umma_commit(&acc_full[2 * (g & 1) + mt]);
                         }
                     }
                     umma_commit(&b_empty[s]);
                 }
                 if (!ok) break;
-                ptile_next(p, cm);
+                PTile nx = cm;
+                ptile_next(p, nx);
+                // the block's last tile: its queries may be replaced once these products are done
+                if (g == G - 1 || nx.h * p.qtiles + nx.qt != blk) umma_commit(a_empty);
+                cm = nx;
             }
         }
     } else {
-        // ---- warps 0-7: queries into tensor memory, read-back and argmax
+        // ---- warps 0-7: read-back and argmax (warps 4 m .. 4 m + 3 read M tile m's units)
         PTile ce;
         ptile_start(p, ce, i0);
         const int emt = warp >> 2, elane = 32 * (warp & 3);
         float bmax = -INFINITY;
         int bidx = -1;
-        int a_block = -1;
         for (int g = 0; g < G; ++g) {
-            const int blk = ce.h * p.qtiles + ce.qt;
             const int n0 = ce.qt * (kUMT * kUQ);
-            if (blk != a_block) {
-                // every MMA that read the previous queries is complete: this warp has read back its unit
-                // of the tile before (its acc_full arrives after all earlier MMAs)
-                const int n = n0 + emt * kUQ + elane + lane;
-                uint32_t r[kAsmD / 2];
-                if (n < p.N) {
-                    const uint4* src = reinterpret_cast<const uint4*>(p.q + ((size_t)n * p.H + ce.h) * kAsmD);
-#pragma unroll
-                    for (int j = 0; j < kAsmD / 8; ++j) {
-                        const uint4 v = src[j];
-                        r[4 * j] = v.x; r[4 * j + 1] = v.y; r[4 * j + 2] = v.z; r[4 * j + 3] = v.w;
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < kAsmD / 2; ++j) r[j] = 0u;
-                }
-                const uint32_t ta = tmem + ((uint32_t)elane << 16) + (uint32_t)(emt * (kAsmD / 2));
-                tmem_st32(ta, r);
-                tmem_st32(ta + 32, r + 32);
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(a_ready);
-                a_block = blk;
-            }
-            const int u = 2 * g + emt, b = u % kPAcc;
+            const int b = 2 * (g & 1) + emt;
             // warp-uniform outcome: the tensor-memory loads below are warp-collective
-            if (!__all_sync(kFull, mbar_wait(&acc_full[b], (unsigned)(u / kPAcc) & 1u, pp.wait_ns))) ok = false;
+            if (!__all_sync(kFull, mbar_wait(&acc_full[b], (unsigned)(g >> 1) & 1u, pp.wait_ns))) ok = false;
             tc_fence_after();
             const int mts = min(kUMT, (p.N - n0 + kUQ - 1) / kUQ);
             const bool mine = ok && emt < mts;
-            // the unit's 128 scores of this row, in two halves of 64: the best value and its first column
+            // the unit's 128 scores of this row: the best value and its first column
             float best = -INFINITY;
             int first = -1;
             if (mine) {
                 // all four loads, one wait, release the buffer, then the arithmetic
-                const uint32_t ta = tmem + ((uint32_t)elane << 16) + (uint32_t)(kPACols + b * kPT);
+                const uint32_t ta = tmem + ((uint32_t)elane << 16) + (uint32_t)(b * kPT);
                 float v[kPT];
 #pragma unroll
                 for (int c = 0; c < kPT; c += 32) tmem_ld32(ta + c, v + c);
@@ -377,8 +393,7 @@ __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __
     __syncthreads();
     if (warp == kUNT / 32 && lane == 0 && G > 0) {
         // the last tile's MMAs complete before the tensor memory is released (bounded)
-        const int u = 2 * (G - 1) + 1;
-        mbar_wait(&acc_full[u % kPAcc], (unsigned)(u / kPAcc) & 1u, pp.wait_ns);
+        mbar_wait(&acc_full[2 * ((G - 1) & 1) + 1], (unsigned)((G - 1) >> 1) & 1u, pp.wait_ns);
     }
     __syncthreads();
     if (warp == 0) {

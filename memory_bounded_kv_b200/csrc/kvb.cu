@@ -99,6 +99,21 @@ bool make_q_map(CUtensorMap* map, const void* q, int d, int Hq, int B, long long
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The queries of the prepared-memory lookup: q [N][H][d] bf16 (d = 128, rows contiguous), boxes of
+// 64 dims x 1 head x 128 queries (128-byte swizzle; queries past N read zeros).
+bool make_asm_q_map(CUtensorMap* map, const void* q, int N, int H) {
+    EncodeTiledFn fn = encode_tiled();
+    if (fn == nullptr) return false;
+    const int d = kvb::kAsmD;
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2};
+    cuuint32_t box[3] = {64, 1, (cuuint32_t)kvb::kUQ};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Resident CTAs the device holds for a kernel (SMs x blocks per SM), once per (kernel, smem, device).
 template <typename Kern>
 int resident_ctas(Kern kern, int threads, size_t smem) {
@@ -695,7 +710,9 @@ kvb_status kvb_asm_lookup_merge_planes(const uint16_t* q, const void* planes, si
                           o, lse, static_cast<unsigned long long*>(workspace), H / H_tables};
     pp.planes = static_cast<const unsigned char*>(planes);
     pp.wait_ns = 1000000000ull;
-    kvb::asm_score_planes_kernel<<<grid, kvb::kPThreads, kvb::kPSmem, st>>>(pp);
+    CUtensorMap mq;
+    if (!make_asm_q_map(&mq, q, N, H)) return KVB_EINVAL;
+    kvb::asm_score_planes_kernel<<<grid, kvb::kPThreads, kvb::kPSmem, st>>>(pp, mq);
     if (launched() != KVB_OK) return KVB_ECUDA;
     const long long rows = (long long)N * H;
     kvb::asm_merge_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(pp.a);
