@@ -66,6 +66,15 @@ WORKLOADS = ("1", "2", "3", "3p", "4", "5", "5p")
 # (sha256 of the kernel's source file, workload, num_splits). Reported only while the source is
 # unchanged since the counters were taken.
 MEASURED_TRAFFIC = {
+    # decode_attn_tc_kernel at the Qwen3-8B-shaped layer, one split: 545,651,200 read + 3,240,192 written
+    # (bench.py --profile c2 under ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum)
+    ("f459f4592a23d661", "2", 1): 548891392,
+    # the long-context attention (136,395,776 + 4,231,424) and its 64-way merge (4,242,688 + 0)
+    # (bench.py --profile c3, the same metrics over both launches)
+    ("f459f4592a23d661", "3", 64): 144869888,
+    # the lookup over the prepared memory (102,808,576 + 3,712,000) and its merge (6,998,528 + 0)
+    # (bench.py --profile c4, the same metrics over both launches)
+    ("173295e61443b3b8", "4", 0): 113519104,
 }
 
 
@@ -1071,7 +1080,8 @@ def report(bench, m, world, hbm_peak, peak_kind):
         roofline = {"bound": "tensor", "kernel": bench.kernel_name(), "achieved": achieved, "peak": peak_tf,
                     "unit": "TFLOP/s", "frac": achieved / peak_tf,
                     "peak_source": ASMBench.PEAK_NOTE.format(kind=bf16_kind, bf16=bf16_tf),
-                    "traffic": None, "algorithmic_flops_per_launch": bench.flops(), "kernel_ms_avg": kms,
+                    "traffic": MEASURED_TRAFFIC.get((src, bench.key, getattr(bench, "S", 0))),
+                    "algorithmic_flops_per_launch": bench.flops(), "kernel_ms_avg": kms,
                     "launches_timed": len(m["kern_ms"])}
     else:
         # launches of a finite schedule differ in size: bytes over time summed over the same launches

@@ -173,6 +173,7 @@ __device__ __forceinline__ void named_bar_arrive(int id, int n) {
 }
 
 __global__ void __launch_bounds__(kUThreads, 1) asm_score_umma_kernel(const __grid_constant__ AsmParams p) {
+    griddep_launch_dependents();   // the merge may be scheduled now; it waits for this grid before reading keys
     extern __shared__ unsigned char s_raw[];
     unsigned char* sm = s_raw + ((1024u - (smem_u32(s_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(sm);
@@ -393,6 +394,13 @@ __global__ void __launch_bounds__(256) asm_merge_kernel(const __grid_constant__ 
     const long long nh = (long long)blockIdx.x * 8 + warp;
     if (nh >= (long long)p.N * p.H) return;
     const int n = (int)(nh / p.H), h = (int)(nh % p.H);
+    // the self state does not depend on the lookup: its loads go out before the keys'
+    float4 os = make_float4(0.f, 0.f, 0.f, 0.f);
+    float ls = 0.f;
+    if (p.o != nullptr) {
+        os = *reinterpret_cast<const float4*>(p.o_self + nh * kAsmD + lane * 4);
+        ls = p.lse_self[nh];
+    }
     griddep_wait();   // the keys come from the previous kernel (a no-op without programmatic launch)
     unsigned long long best = 0ull;
     for (int s = lane; s < p.ksplit; s += 32) {
@@ -410,14 +418,12 @@ __global__ void __launch_bounds__(256) asm_merge_kernel(const __grid_constant__ 
     }
     if (best == 0ull) {   // nothing retrieved (no candidate, or every score NaN): the self state
         if (lane == 0 && p.idx != nullptr) p.idx[nh] = -1;
-        if (lane == 0 && p.lse != nullptr) p.lse[nh] = p.lse_self[nh];
-        *reinterpret_cast<float4*>(p.o + nh * kAsmD + lane * 4) =
-            *reinterpret_cast<const float4*>(p.o_self + nh * kAsmD + lane * 4);
+        if (lane == 0 && p.lse != nullptr) p.lse[nh] = ls;
+        *reinterpret_cast<float4*>(p.o + nh * kAsmD + lane * 4) = os;
         return;
     }
     const int k = (int)(0xffffffffu - (unsigned)(best & 0xffffffffull));
     if (lane == 0 && p.idx != nullptr) p.idx[nh] = k;
-    const float ls = p.lse_self[nh];
     const int t = h / p.G;   // the head's table
     const float lm = p.lz[(size_t)t * p.K + k];
     const float mx = fmaxf(ls, lm);
@@ -426,7 +432,6 @@ __global__ void __launch_bounds__(256) asm_merge_kernel(const __grid_constant__ 
     const float tot = ws + wm;
     const float inv = (tot > 0.f) ? 1.f / tot : 0.f;
     if (lane == 0 && p.lse != nullptr) p.lse[nh] = (tot > 0.f) ? mx + log2f(tot) * kLn2 : -INFINITY;
-    const float4 os = *reinterpret_cast<const float4*>(p.o_self + nh * kAsmD + lane * 4);
     const uint2 am = *reinterpret_cast<const uint2*>(p.abar + ((size_t)t * p.K + k) * kAsmD + lane * 4);
     float4 r;
     r.x = (ws * os.x + wm * bf16_lo(am.x)) * inv;

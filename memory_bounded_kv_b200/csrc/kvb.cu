@@ -655,8 +655,8 @@ kvb_status kvb_asm_lookup_merge_grouped(const uint16_t* q, const float* qbar, co
     kvb::asm_score_umma_kernel<<<grid, kvb::kUThreads, kvb::kUSmem, st>>>(p);
     if (launched() != KVB_OK) return KVB_ECUDA;
     const long long rows = (long long)N * H;
-    kvb::asm_merge_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p);
-    return launched();
+    // programmatic launch: the merge's CTAs wait on the device for the lookup instead of being launched after it
+    return launch_pdl(kvb::asm_merge_kernel, dim3((unsigned)((rows + 7) / 8)), dim3(256), 0, st, p);
 }
 
 size_t kvb_asm_planes_bytes(int32_t H_tables, int32_t K) {
@@ -715,8 +715,7 @@ kvb_status kvb_asm_lookup_merge_planes(const uint16_t* q, const void* planes, si
     kvb::asm_score_planes_kernel<<<grid, kvb::kPThreads, kvb::kPSmem, st>>>(pp, mq);
     if (launched() != KVB_OK) return KVB_ECUDA;
     const long long rows = (long long)N * H;
-    kvb::asm_merge_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(pp.a);
-    return launched();
+    return launch_pdl(kvb::asm_merge_kernel, dim3((unsigned)((rows + 7) / 8)), dim3(256), 0, st, pp.a);
 }
 
 kvb_status kvb_asm_lookup_merge(const uint16_t* q, const float* qbar, const uint16_t* abar, const float* log_zbar,
