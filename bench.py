@@ -74,7 +74,7 @@ MEASURED_TRAFFIC = {
     ("f459f4592a23d661", "3", 64): 144869888,
     # the lookup over the prepared memory (102,808,576 + 3,712,000) and its merge (6,998,528 + 0)
     # (bench.py --profile c4, the same metrics over both launches)
-    ("173295e61443b3b8", "4", 0): 113519104,
+    ("173295e61443b3b8", "4", 4): 113519104,
 }
 
 

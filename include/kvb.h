@@ -117,7 +117,8 @@ enum kvb_device_error {
  * Requirements (else KVB_EINVAL): d in {64, 128}; Hq % Hkv == 0 and
  * Hq / Hkv in {1, 2, 4, 8}; B, Hkv, cap >= 1; B * Hq < 2^31;
  * 1 <= num_splits <= 1024;
- * split_len >= 0; q, k, v 16-byte aligned and every q/kv stride a multiple
+ * split_len >= 0; q, k, v, o and o_part 16-byte aligned (the outputs are
+ * written 16 bytes at a time) and every q/kv stride a multiple
  * of 8 elements; kv_stride_h > 0 when Hkv > 1; scale finite (0 selects
  * 1/sqrt(d)). K and V are read with TMA tensor copies, so a layout the
  * tensor-map encoder refuses also returns KVB_EINVAL.

@@ -136,6 +136,13 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return r;
 }
 
+// 2^x by the hardware's approximate base-2 exponential (PTX ex2.approx.ftz; 2^-inf = 0)
+__device__ __forceinline__ float ex2_fast(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ void named_bar(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
@@ -578,15 +585,23 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
             named_bar(1, NWC * 32);   // every warp's (m, l) and candidate posted
             const int S = p.S;
             if (r < G) {
+                // (the hardware's base-2 exponential and a rounded reciprocal: this block is one
+                // dependent chain per unit, and the library exp2f / IEEE division doubled it)
+                float mw[NWC], lw[NWC];
+#pragma unroll
+                for (int w = 0; w < NWC; ++w) {
+                    const float2 x = *reinterpret_cast<const float2*>(s_ml + (w * G + r) * 2);
+                    mw[w] = x.x;
+                    lw[w] = x.y;
+                }
                 float M = -INFINITY;
 #pragma unroll
-                for (int w = 0; w < NWC; ++w) M = fmaxf(M, s_ml[(w * G + r) * 2]);
+                for (int w = 0; w < NWC; ++w) M = fmaxf(M, mw[w]);
                 const float Mu = (M == -INFINITY) ? 0.f : M;
                 float L = 0.f;
 #pragma unroll
-                for (int w = 0; w < NWC; ++w)
-                    L = fmaf(exp2f((s_ml[(w * G + r) * 2] - Mu) * kLog2e), s_ml[(w * G + r) * 2 + 1], L);
-                const float f = (L > 0.f) ? exp2f((m_run - Mu) * kLog2e) / L : 0.f;
+                for (int w = 0; w < NWC; ++w) L = fmaf(ex2_fast((mw[w] - Mu) * kLog2e), lw[w], L);
+                const float f = (L > 0.f) ? ex2_fast((m_run - Mu) * kLog2e) * __frcp_rn(L) : 0.f;
 #pragma unroll
                 for (int j = 0; j < SH::NTILES; ++j)
                     *reinterpret_cast<float2*>(s_o + (warp * G + r) * D + 8 * j + 2 * cq) =
@@ -613,18 +628,26 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                 c->t = ut + 1;
             }
             named_bar(1, NWC * 32);   // every warp's scaled O posted
-            for (int idx = tid; idx < G * D; idx += NWC * 32) {
-                const int hh = idx / D, e = idx % D;
-                float out = 0.f;
+            // four consecutive outputs per thread: one 16-byte load per warp's posted O, one store
+            for (int idx = tid; idx < G * D / 4; idx += NWC * 32) {
+                const int hh = (4 * idx) / D, e = (4 * idx) % D;
+                float4 out = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-                for (int w = 0; w < NWC; ++w) out += s_o[(w * G + hh) * D + e];
+                for (int w = 0; w < NWC; ++w) {
+                    const float4 x = *reinterpret_cast<const float4*>(s_o + (w * G + hh) * D + e);
+                    out.x += x.x;
+                    out.y += x.y;
+                    out.z += x.z;
+                    out.w += x.w;
+                }
                 const size_t row = (size_t)ub * p.Hq + ug * G + hh;
-                if (p.o_part != nullptr) p.o_part[(row * S + usplit) * D + e] = out;
+                if (p.o_part != nullptr) *reinterpret_cast<float4*>(p.o_part + (row * S + usplit) * D + e) = out;
                 if (S == 1) {
                     if (p.o_bf16) {
-                        reinterpret_cast<__nv_bfloat16*>(p.o)[row * D + e] = __float2bfloat16_rn(out);
+                        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.o) + row * D + e;
+                        *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16(out.x, out.y), pack_bf16(out.z, out.w));
                     } else {
-                        reinterpret_cast<float*>(p.o)[row * D + e] = out;
+                        *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.o) + row * D + e) = out;
                     }
                 }
             }

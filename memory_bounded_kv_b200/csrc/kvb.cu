@@ -399,6 +399,7 @@ kvb_status kvb_decode_attn(const kvb_attn_args* a, kvb_stream stream) {
     if (!std::isfinite(a->scale)) return KVB_EINVAL;
     if (!a->q || !a->k || !a->v || !a->len || !a->o) return KVB_EINVAL;
     if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v)) return KVB_EINVAL;
+    if (!aligned16(a->o) || (a->o_part != nullptr && !aligned16(a->o_part))) return KVB_EINVAL;
     if (a->q_stride_b < 0 || a->q_stride_h < 0 || a->kv_stride_b < 0 || a->kv_stride_h < 0) return KVB_EINVAL;
     if ((a->q_stride_b % 8) || (a->q_stride_h % 8) || (a->kv_stride_b % 8) || (a->kv_stride_h % 8)) return KVB_EINVAL;
     const bool bias = a->log_beta != nullptr;
@@ -592,7 +593,8 @@ kvb_status kvb_paged_decode_attn(const kvb_paged_cache* c, const uint16_t* q, co
     if (num_splits < 1 || num_splits > 1024 || split_len < 0) return KVB_EINVAL;
     // every split starts on a page: one split, or a split length that is a multiple of a page
     if (num_splits > 1 && (split_len == 0 || split_len % kvb::kPageSlots != 0)) return KVB_EINVAL;
-    if (!std::isfinite(scale) || !q || !o || !aligned16(q)) return KVB_EINVAL;
+    if (!std::isfinite(scale) || !q || !o || !aligned16(q) || !aligned16(o)) return KVB_EINVAL;
+    if (o_part != nullptr && !aligned16(o_part)) return KVB_EINVAL;
     const bool bias = c->log_beta_pages != nullptr;
     if ((bias || evict_cand) && !t) return KVB_EINVAL;
     if (evict_cand && (reinterpret_cast<uintptr_t>(evict_cand) & 15u)) return KVB_EINVAL;

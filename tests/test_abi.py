@@ -66,6 +66,8 @@ def _args(**kw):
     dict(d=96), dict(Hq=12), dict(Hq=48, Hkv=3), dict(num_splits=0), dict(num_splits=2),
     dict(q=(1 << 20) + 2), dict(kv_stride_h=100), dict(log_beta=1 << 20), dict(o_dtype=5),
     dict(scale=float("nan")), dict(B=0), dict(split_len=-1), dict(q=None),
+    dict(o=(1 << 20) + 4),                                                         # outputs 16-byte aligned
+    dict(num_splits=2, split_len=32, o_part=(1 << 20) + 8, lse_part=1 << 20),
 ])
 def test_decode_attn_rejects_bad_arguments_on_the_host(bad):
     L = _lib.lib()
