@@ -11,10 +11,14 @@
 //    takes units c, c + grid, c + 2*grid, ...
 //  - One producer warp streams each unit's K/V tiles (T slots) with TMA
 //    tensor loads (128-byte swizzle) into a STAGES-deep shared-memory ring.
-//    With every tile it also stages the tile's bias ((t - pos) * log beta, or
-//    -inf past the split's end) and, with a unit's first tile, the unit's
-//    G query rows; one "full" mbarrier per stage counts the bytes and the
-//    producer lanes' arrivals, one "empty" mbarrier the consumers' release.
+//    With every tile it also copies the tile's pos and log beta into the
+//    stage (4-byte cp.async; the consumers form the bias (t - pos) * log beta
+//    and mask the slots past the split's end) and, with a unit's first tile,
+//    the unit's G query rows (bulk copy); one "full" mbarrier per stage counts
+//    the bytes and the producer lanes' cp.async arrivals, one "empty" mbarrier
+//    the consumers' release. The producer itself waits for no load: staging
+//    the bias through its registers put a DRAM round trip on every tile's
+//    path, which set the pace of short units.
 //  - Four consumer warps each own 16 slots of a tile. Both products run on
 //    the tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate) with the
 //    G query heads as the M rows (padded to 16):
@@ -82,8 +86,7 @@ struct TcShape {
     // shared-memory layout (offsets from a 1024-aligned base)
     static constexpr int RING_OFF = 0;
     static constexpr int Q_OFF = RING_OFF + STAGES * STAGE_BYTES;       // [ST][G][D] bf16
-    static constexpr int BIAS_OFF = Q_OFF + STAGES * QBYTES;            // [ST][T] f32
-    static constexpr int CPOS_OFF = BIAS_OFF + STAGES * T * 4;          // [ST][T] int (pos, for candidates)
+    static constexpr int CPOS_OFF = Q_OFF + STAGES * QBYTES;            // [ST][T] int (pos: bias, candidates)
     static constexpr int CLB_OFF = CPOS_OFF + STAGES * T * 4;           // [ST][T] f32 (log beta)
     static constexpr int META_OFF = CLB_OFF + STAGES * T * 4;           // [ST][16] int
     static constexpr int BAR_OFF = META_OFF + STAGES * 64;              // full[ST], empty[ST]
@@ -134,6 +137,15 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
+}
+
+// 4-byte asynchronous global -> shared copy (cp.async), and the arrival on an mbarrier that happens
+// once every cp.async this thread issued has landed (it counts as one of the barrier's arrivals)
+__device__ __forceinline__ void cp_async4(void* dst_smem, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst_smem)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 // 2^x by the hardware's approximate base-2 exponential (PTX ex2.approx.ftz; 2^-inf = 0)
@@ -213,7 +225,6 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~static_cast<uintptr_t>(1023));
     uint16_t* s_q = reinterpret_cast<uint16_t*>(smem + SH::Q_OFF);
-    float* s_bias = reinterpret_cast<float*>(smem + SH::BIAS_OFF);
     int* s_meta = reinterpret_cast<int*>(smem + SH::META_OFF);
     int* s_pos = reinterpret_cast<int*>(smem + SH::CPOS_OFF);
     float* s_lb = reinterpret_cast<float*>(smem + SH::CLB_OFF);
@@ -308,9 +319,7 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                     }
                     page = __shfl_sync(kFull, lane_page, i & 31);
                 }
-                // the stage's record and copies (lane 0); the first ST tiles need no stage to free, so
-                // their copies go out before this tile's pos / log beta loads, later ones after the
-                // wait (those loads are issued before it, so their latency hides behind the wait)
+                // the stage's record and copies (lane 0)
                 const bool data = !end && ui.ntiles > 0;
                 auto issue = [&]() {
                     if (lane == 0) {
@@ -354,30 +363,6 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                         }
                     }
                 };
-                const bool early = it < ST;
-                if (early) issue();
-                // this tile's bias (and, for the eviction candidates, its pos and log beta)
-                const size_t mt = PAGED ? (size_t)page * T : m_off + (size_t)i * T;
-                float bias[T / 32];
-                int psv[T / 32];
-                float lbv[T / 32];
-#pragma unroll
-                for (int j = 0; j < T / 32; ++j) {
-                    const int key = i * T + lane + 32 * j;
-                    float bv = -INFINITY;
-                    psv[j] = 0;
-                    lbv[j] = 0.f;
-                    if (!end && key < ui.nk) {
-                        if (BIAS || want_cand) psv[j] = p.pos[mt + lane + 32 * j];
-                        if constexpr (BIAS) {
-                            lbv[j] = p.lb[mt + lane + 32 * j];
-                            bv = __fmul_rn(__int2float_rn(tb - psv[j]), lbv[j]);
-                        } else {
-                            bv = 0.f;
-                        }
-                    }
-                    bias[j] = bv;
-                }
                 if (it >= ST && !mbar_wait(&s_empty[st], (unsigned)((it / ST) - 1) & 1u, p.wait_ns)) {
                     if (lane == 0) {
                         raise_error(KVB_DERR_TIMEOUT);
@@ -386,21 +371,27 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                     stop = true;
                     break;
                 }
-                if (!early && *s_abort) {   // (an early tile's copies are out: it is arrived and counted)
+                if (*s_abort) {
                     stop = true;
                     break;
                 }
-                if (!early) issue();
+                issue();
+                // this tile's pos (for the bias and the eviction candidates) and log beta go into the
+                // stage by asynchronous 4-byte copies that the stage's full barrier counts: no load
+                // round trip on this warp's path (the consumers form the bias); slots past the
+                // split's end are not copied (the consumers mask them)
+                if (BIAS || want_cand) {
+                    const size_t mt = PAGED ? (size_t)page * T : m_off + (size_t)i * T;
 #pragma unroll
-                for (int j = 0; j < T / 32; ++j) {
-                    s_bias[st * T + lane + 32 * j] = bias[j];
-                    if (want_cand) {
-                        s_pos[st * T + lane + 32 * j] = psv[j];
-                        s_lb[st * T + lane + 32 * j] = lbv[j];
+                    for (int j = 0; j < T / 32; ++j) {
+                        const int key = i * T + lane + 32 * j;
+                        if (!end && key < ui.nk) {
+                            cp_async4(s_pos + st * T + lane + 32 * j, p.pos + mt + lane + 32 * j);
+                            if constexpr (BIAS) cp_async4(s_lb + st * T + lane + 32 * j, p.lb + mt + lane + 32 * j);
+                        }
                     }
                 }
-                __syncwarp();
-                mbar_arrive(&s_full[st]);
+                cp_async_mbar_arrive(&s_full[st]);   // one arrival per lane once its copies have landed
             }
             if (end) break;
         }
@@ -505,15 +496,25 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                     fence_proxy_async_smem();
                     __syncwarp();
                 }
-                // ---- logits, online softmax (row r of this lane; slots 2cq, 2cq+1, 8+2cq, 8+2cq+1)
-                const float* sb = s_bias + st * T + kw;
-                const float2 bA = *reinterpret_cast<const float2*>(sb + 2 * cq);
-                const float2 bB = *reinterpret_cast<const float2*>(sb + 8 + 2 * cq);
+                // ---- logits, online softmax (row r of this lane; slots 2cq, 2cq+1, 8+2cq, 8+2cq+1):
+                // scale q.k + (t - pos) log beta (one float32 product), -inf past the split's end
+                const int sa = kw + 2 * cq, sbb = sa + 8;
+                float bv[4] = {0.f, 0.f, 0.f, 0.f};
+                if constexpr (BIAS) {
+                    const int2 pA = *reinterpret_cast<const int2*>(s_pos + st * T + sa);
+                    const int2 pB = *reinterpret_cast<const int2*>(s_pos + st * T + sbb);
+                    const float2 lA = *reinterpret_cast<const float2*>(s_lb + st * T + sa);
+                    const float2 lB = *reinterpret_cast<const float2*>(s_lb + st * T + sbb);
+                    bv[0] = __fmul_rn(__int2float_rn(ut - pA.x), lA.x);
+                    bv[1] = __fmul_rn(__int2float_rn(ut - pA.y), lA.y);
+                    bv[2] = __fmul_rn(__int2float_rn(ut - pB.x), lB.x);
+                    bv[3] = __fmul_rn(__int2float_rn(ut - pB.y), lB.y);
+                }
                 float x[4];
-                x[0] = (bA.x == -INFINITY) ? -INFINITY : fmaf(sc[0][0], p.scale, bA.x);
-                x[1] = (bA.y == -INFINITY) ? -INFINITY : fmaf(sc[0][1], p.scale, bA.y);
-                x[2] = (bB.x == -INFINITY) ? -INFINITY : fmaf(sc[1][0], p.scale, bB.x);
-                x[3] = (bB.y == -INFINITY) ? -INFINITY : fmaf(sc[1][1], p.scale, bB.y);
+                x[0] = (sa < rows) ? fmaf(sc[0][0], p.scale, bv[0]) : -INFINITY;
+                x[1] = (sa + 1 < rows) ? fmaf(sc[0][1], p.scale, bv[1]) : -INFINITY;
+                x[2] = (sbb < rows) ? fmaf(sc[1][0], p.scale, bv[2]) : -INFINITY;
+                x[3] = (sbb + 1 < rows) ? fmaf(sc[1][1], p.scale, bv[3]) : -INFINITY;
                 float tmax = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
                 tmax = fmaxf(tmax, __shfl_xor_sync(kFull, tmax, 1));
                 tmax = fmaxf(tmax, __shfl_xor_sync(kFull, tmax, 2));
