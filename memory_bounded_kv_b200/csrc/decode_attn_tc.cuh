@@ -30,9 +30,11 @@
 //                        ~1e-3 relative error in o).
 //    Online softmax per warp and head (maxima in natural units, exp2 of
 //    scaled differences), O rescaled only when a maximum moved.
-//  - At the end of a unit the consumer warps combine through shared memory
-//    (a named barrier among consumers only; the producer keeps prefetching
-//    the next unit's tiles) and write the split's state.
+//  - At the end of a unit each consumer warp posts its unscaled O, its
+//    (m, l) per row and its eviction candidate to shared memory (mbarrier
+//    epi_full) and goes on with the next unit; one epilogue warp combines the
+//    four states, writes the split's state and frees the buffer (epi_empty).
+//    The epilogue of one unit thus overlaps the next unit's tiles.
 // Every wait is bounded (wait_ns, 1 s by default); on a timeout the CTA
 // records KVB_DERR_TIMEOUT, stops, drains the copies it issued (bounded) and
 // writes the empty state for every unit it owns.
@@ -73,7 +75,7 @@ struct DecodeTcParams {
 template <int D, int G>
 struct TcShape {
     static constexpr int NWC = 4;                 // consumer warps
-    static constexpr int NT = (NWC + 1) * 32;     // + one producer warp
+    static constexpr int NT = (NWC + 2) * 32;     // + one producer warp, one epilogue warp
     static constexpr int T = 16 * NWC;            // slots per tile
     static constexpr int STAGES = 3;
     static constexpr int HALVES = D / 64;         // 128-byte swizzle rows hold 64 bf16
@@ -89,9 +91,9 @@ struct TcShape {
     static constexpr int CPOS_OFF = Q_OFF + STAGES * QBYTES;            // [ST][T] int (pos: bias, candidates)
     static constexpr int CLB_OFF = CPOS_OFF + STAGES * T * 4;           // [ST][T] f32 (log beta)
     static constexpr int META_OFF = CLB_OFF + STAGES * T * 4;           // [ST][16] int
-    static constexpr int BAR_OFF = META_OFF + STAGES * 64;              // full[ST], empty[ST]
-    static constexpr int MISC_OFF = BAR_OFF + 2 * STAGES * 8;           // abort, issued
-    static constexpr int EPI_OFF = (MISC_OFF + 16 + 15) / 16 * 16;      // [NWC][G][D] f32
+    static constexpr int BAR_OFF = META_OFF + STAGES * 64;              // full[ST], empty[ST], epi full/empty
+    static constexpr int MISC_OFF = BAR_OFF + (2 * STAGES + 2) * 8;     // abort, issued, -, -, unit record [5]
+    static constexpr int EPI_OFF = (MISC_OFF + 64 + 15) / 16 * 16;      // [NWC][G][D] f32
     static constexpr int ML_OFF = EPI_OFF + NWC * G * D * 4;            // [NWC][G][2] f32
     static constexpr int CAND_OFF = ML_OFF + NWC * G * 2 * 4;           // [NWC] (key, slot)
     static constexpr int END_OFF = CAND_OFF + NWC * 16;
@@ -146,6 +148,18 @@ __device__ __forceinline__ void cp_async4(void* dst_smem, const void* src) {
 }
 __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// A bounded wait that sleeps between its checks (for a warp whose waits are long and off the
+// critical path: it leaves the issue slots to the warps that compute)
+__device__ __forceinline__ bool mbar_wait_backoff(uint64_t* bar, unsigned parity, uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        __nanosleep(256);
+        if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
 }
 
 // 2^x by the hardware's approximate base-2 exponential (PTX ex2.approx.ftz; 2^-inf = 0)
@@ -232,8 +246,11 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
     int* s_cs = reinterpret_cast<int*>(smem + SH::CAND_OFF + NWC * 8);
     uint64_t* s_full = reinterpret_cast<uint64_t*>(smem + SH::BAR_OFF);
     uint64_t* s_empty = s_full + ST;
+    uint64_t* epi_full = s_empty + ST;    // the four consumer warps posted a unit's partial states
+    uint64_t* epi_empty = epi_full + 1;   // the epilogue warp has read them
     volatile int* s_abort = reinterpret_cast<int*>(smem + SH::MISC_OFF);
     int* s_issued = reinterpret_cast<int*>(smem + SH::MISC_OFF) + 1;
+    volatile int* s_epi = reinterpret_cast<int*>(smem + SH::MISC_OFF) + 4;   // b, g, split, t, stop
     float* s_o = reinterpret_cast<float*>(smem + SH::EPI_OFF);
     float* s_ml = reinterpret_cast<float*>(smem + SH::ML_OFF);
 
@@ -245,6 +262,8 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
             mbar_init(&s_full[s], 33);          // producer lane 0's expect_tx + 32 producer lanes
             mbar_init(&s_empty[s], NWC * 32);   // every consumer lane
         }
+        mbar_init(epi_full, NWC);
+        mbar_init(epi_empty, 1);
         *s_abort = 0;
         *s_issued = 0;
         fence_mbar_init();
@@ -396,7 +415,7 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
             if (end) break;
         }
         if (lane == 0) *s_issued = it;
-    } else {
+    } else if (warp < NWC) {
         // ======================= consumer warps =======================
         const int r = lane >> 2;          // M row = query head within the group (rows >= G are padding)
         const int cq = lane & 3;          // quad index: columns 2*cq, 2*cq+1 of each 8-wide n-tile
@@ -417,6 +436,7 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
         int cand_slot = 0x7fffffff;
         int it = 0;
         bool aborted = false;
+        int units_posted = 0;   // units whose partial states went to the epilogue warp
         while (true) {
             const int st = it % ST;
             if (!mbar_wait(&s_full[st], (unsigned)(it / ST) & 1u, p.wait_ns)) {
@@ -559,15 +579,9 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
             ++it;
             if (ntiles > 0 && i != ntiles - 1) continue;
 
-            // ======== end of unit: combine warps, write the split's state ========
-            // each warp's share of a row is exp2(m_w - M) / L (M, L over the four warps); every warp
-            // folds its own share into its O before the sum, so the final pass only adds
+            // ======== end of unit: post this warp's partial state to the epilogue warp ========
             l_run += __shfl_xor_sync(kFull, l_run, 1);
             l_run += __shfl_xor_sync(kFull, l_run, 2);
-            if (r < G && cq == 0) {
-                s_ml[(warp * G + r) * 2] = m_run;
-                s_ml[(warp * G + r) * 2 + 1] = l_run;
-            }
             if (want_cand) {
 #pragma unroll
                 for (int o2 = 8; o2 >= 1; o2 >>= 1) {
@@ -578,43 +592,133 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                         cand_slot = s2;
                     }
                 }
-                if (lane == 0) {
-                    s_ck[warp] = cand_key;
-                    s_cs[warp] = cand_slot;
-                }
             }
-            named_bar(1, NWC * 32);   // every warp's (m, l) and candidate posted
-            const int S = p.S;
-            if (r < G) {
-                // (the hardware's base-2 exponential and a rounded reciprocal: this block is one
-                // dependent chain per unit, and the library exp2f / IEEE division doubled it)
-                float mw[NWC], lw[NWC];
-#pragma unroll
-                for (int w = 0; w < NWC; ++w) {
-                    const float2 x = *reinterpret_cast<const float2*>(s_ml + (w * G + r) * 2);
-                    mw[w] = x.x;
-                    lw[w] = x.y;
+            // the buffer holds the previous unit until the epilogue warp has read it
+            if (units_posted > 0 &&
+                !__all_sync(kFull, mbar_wait(epi_empty, (unsigned)(units_posted - 1) & 1u, p.wait_ns))) {
+                if (lane == 0) {
+                    raise_error(KVB_DERR_TIMEOUT);
+                    *s_abort = 1;
                 }
-                float M = -INFINITY;
-#pragma unroll
-                for (int w = 0; w < NWC; ++w) M = fmaxf(M, mw[w]);
-                const float Mu = (M == -INFINITY) ? 0.f : M;
-                float L = 0.f;
-#pragma unroll
-                for (int w = 0; w < NWC; ++w) L = fmaf(ex2_fast((mw[w] - Mu) * kLog2e), lw[w], L);
-                const float f = (L > 0.f) ? ex2_fast((m_run - Mu) * kLog2e) * __frcp_rn(L) : 0.f;
+                aborted = true;
+                break;
+            }
+            if (r < G) {
 #pragma unroll
                 for (int j = 0; j < SH::NTILES; ++j)
                     *reinterpret_cast<float2*>(s_o + (warp * G + r) * D + 8 * j + 2 * cq) =
-                        make_float2(acc[j][0] * f, acc[j][1] * f);
-                if (warp == 0 && cq == 0) {
+                        make_float2(acc[j][0], acc[j][1]);
+                if (cq == 0) {
+                    s_ml[(warp * G + r) * 2] = m_run;
+                    s_ml[(warp * G + r) * 2 + 1] = l_run;
+                }
+            }
+            if (lane == 0) {
+                s_ck[warp] = cand_key;
+                s_cs[warp] = cand_slot;
+                if (warp == 0) {
+                    s_epi[0] = ub;
+                    s_epi[1] = ug;
+                    s_epi[2] = usplit;
+                    s_epi[3] = ut;
+                    s_epi[4] = 0;
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(epi_full);
+            ++units_posted;
+        }
+        if (!aborted) {
+            // the end: once the epilogue warp has read the last unit, tell it to stop
+            if (units_posted > 0 &&
+                !__all_sync(kFull, mbar_wait(epi_empty, (unsigned)(units_posted - 1) & 1u, p.wait_ns))) {
+                if (lane == 0) {
+                    raise_error(KVB_DERR_TIMEOUT);
+                    *s_abort = 1;
+                }
+            } else {
+                if (warp == 0 && lane == 0) s_epi[4] = 1;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(epi_full);
+            }
+        }
+        (void)aborted;
+    } else {
+        // ======================= epilogue warp =======================
+        // Combines a unit's four partial states while the consumers go on with the next unit: each
+        // warp's share of a row is exp2(m_w - M) / L (M, L over the four warps); lane w G + r holds
+        // the share of warp w for row r, and every output is the shares' sum of the four posted O.
+        // Its waits back off (nanosleep) so that it takes no issue slots from the consumers.
+        const bool want_cand = p.cand != nullptr;
+        const int S = p.S;
+        constexpr int NV = G * D / 4;   // float4 outputs of a unit
+        for (int k = 0;; ++k) {
+            if (!__all_sync(kFull, mbar_wait_backoff(epi_full, (unsigned)k & 1u, p.wait_ns))) {
+                if (lane == 0) {
+                    raise_error(KVB_DERR_TIMEOUT);
+                    *s_abort = 1;
+                }
+                break;
+            }
+            if (s_epi[4] != 0) break;   // the consumers' stop
+            const int ub = s_epi[0], ug = s_epi[1], usplit = s_epi[2], ut = s_epi[3];
+            float fsh = 0.f;
+            if (lane < NWC * G) {
+                const int r = lane % G, w = lane / G;
+                float mw[NWC], lw[NWC];
+#pragma unroll
+                for (int v = 0; v < NWC; ++v) {
+                    const float2 x = *reinterpret_cast<const float2*>(s_ml + (v * G + r) * 2);
+                    mw[v] = x.x;
+                    lw[v] = x.y;
+                }
+                float M = -INFINITY;
+#pragma unroll
+                for (int v = 0; v < NWC; ++v) M = fmaxf(M, mw[v]);
+                const float Mu = (M == -INFINITY) ? 0.f : M;
+                float L = 0.f;
+#pragma unroll
+                for (int v = 0; v < NWC; ++v) L = fmaf(ex2_fast((mw[v] - Mu) * kLog2e), lw[v], L);
+                float mine = mw[0];
+#pragma unroll
+                for (int v = 1; v < NWC; ++v) mine = (v == w) ? mw[v] : mine;
+                fsh = (L > 0.f) ? ex2_fast((mine - Mu) * kLog2e) * __frcp_rn(L) : 0.f;
+                if (w == 0) {
                     const float lse = (L > 0.f) ? M + log2f(L) * kLn2 : -INFINITY;
                     const size_t row = (size_t)ub * p.Hq + ug * G + r;
                     if (p.o_part != nullptr) p.lse_part[row * S + usplit] = lse;
                     if (S == 1 && p.lse != nullptr) p.lse[row] = lse;
                 }
             }
-            if (want_cand && tid == 0) {
+#pragma unroll
+            for (int v0 = 0; v0 < NV; v0 += 32) {   // every lane runs every round (the shuffles)
+                const int idx = v0 + lane;
+                const int hh = (4 * min(idx, NV - 1)) / D, e = (4 * min(idx, NV - 1)) % D;
+                float4 out = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int w = 0; w < NWC; ++w) {
+                    const float f = __shfl_sync(kFull, fsh, w * G + hh);
+                    const float4 x = *reinterpret_cast<const float4*>(s_o + (w * G + hh) * D + e);
+                    out.x = fmaf(f, x.x, out.x);
+                    out.y = fmaf(f, x.y, out.y);
+                    out.z = fmaf(f, x.z, out.z);
+                    out.w = fmaf(f, x.w, out.w);
+                }
+                if (idx < NV) {
+                    const size_t row = (size_t)ub * p.Hq + ug * G + hh;
+                    if (p.o_part != nullptr) *reinterpret_cast<float4*>(p.o_part + (row * S + usplit) * D + e) = out;
+                    if (S == 1) {
+                        if (p.o_bf16) {
+                            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.o) + row * D + e;
+                            *reinterpret_cast<uint2*>(dst) =
+                                make_uint2(pack_bf16(out.x, out.y), pack_bf16(out.z, out.w));
+                        } else {
+                            *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.o) + row * D + e) = out;
+                        }
+                    }
+                }
+            }
+            if (want_cand && lane == 0) {
                 unsigned long long bk = s_ck[0];
                 int bs = s_cs[0];
 #pragma unroll
@@ -628,35 +732,9 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                 c->slot = (bk == ~0ull) ? -1 : bs;
                 c->t = ut + 1;
             }
-            named_bar(1, NWC * 32);   // every warp's scaled O posted
-            // four consecutive outputs per thread: one 16-byte load per warp's posted O, one store
-            for (int idx = tid; idx < G * D / 4; idx += NWC * 32) {
-                const int hh = (4 * idx) / D, e = (4 * idx) % D;
-                float4 out = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                for (int w = 0; w < NWC; ++w) {
-                    const float4 x = *reinterpret_cast<const float4*>(s_o + (w * G + hh) * D + e);
-                    out.x += x.x;
-                    out.y += x.y;
-                    out.z += x.z;
-                    out.w += x.w;
-                }
-                const size_t row = (size_t)ub * p.Hq + ug * G + hh;
-                if (p.o_part != nullptr) *reinterpret_cast<float4*>(p.o_part + (row * S + usplit) * D + e) = out;
-                if (S == 1) {
-                    if (p.o_bf16) {
-                        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.o) + row * D + e;
-                        *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16(out.x, out.y), pack_bf16(out.z, out.w));
-                    } else {
-                        *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.o) + row * D + e) = out;
-                    }
-                }
-            }
-            // no third barrier: the next unit writes s_ml and the candidates only after passing the
-            // second barrier above (so every read of them is done), and s_o only after its own first
-            // barrier, which every thread reaches after this loop
+            __syncwarp();
+            if (lane == 0) mbar_arrive(epi_empty);
         }
-        (void)aborted;
     }
 
     // drain: copies issued into stages that no consumer waited for
