@@ -160,3 +160,23 @@ def test_host_rejects_bad_layout():
     with pytest.raises(kvb.KvbError):   # q not 16-byte aligned: refused by the library
         qd = torch.empty(q.size + 8, dtype=torch.bfloat16, device="cuda")[1:1 + q.size].view(q.shape)
         kvb.kvb_decode_attn(qd, dev(k), dev(v), dev(lb), dev(pos), dev(ln), dev(t), o)
+
+
+@pytest.mark.parametrize("d,G,S", [(128, 4, 8), (128, 4, 5), (64, 8, 2), (128, 8, 16), (64, 1, 3)])
+def test_equal_splits_many_rows(oracle, d, G, S):
+    """Equal splits (split_len 0) over many (b, g) rows (up to 4096 units: the persistent CTAs
+    take several in turn); lengths below S leave empty splits, length 0 empty rows. Final states
+    and every split's state against the oracle."""
+    Hkv = 2 if G == 8 else 8
+    B, Hq, cap = 64, Hkv * G, 130
+    g = rng(77, d + G + S)
+    lens = g.integers(0, cap + 1, (B, Hkv))
+    lens[0, :] = [0, 1] + [2] * (Hkv - 2)
+    lens[1, 0], lens[2, 0] = S - 1, cap
+    q, k, v, lb, pos, ln, t = make_case(d + 3 * G + 7 * S, B, Hq, Hkv, d, cap, lens)
+    kvb.kvb_get_error()   # clear
+    res = run_gpu(q, k, v, lb, pos, ln, t, S=S)
+    o_ref, l_ref, op_ref, lp_ref = oracle.decode_attn(q, k, v, lb, pos, ln, t, num_splits=S, want_parts=True)
+    assert_state_close(res["o"], res["lse"], o_ref, l_ref, "final")
+    assert_splits_close(res["o_part"], res["lse_part"], op_ref, lp_ref, "splits")
+    assert kvb.kvb_get_error() == 0
