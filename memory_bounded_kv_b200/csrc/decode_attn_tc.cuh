@@ -173,6 +173,11 @@ __device__ __forceinline__ void named_bar(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// fetch a tensor map (a __grid_constant__ kernel parameter) into the TMA unit's descriptor cache
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -255,8 +260,8 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
     float* s_ml = reinterpret_cast<float*>(smem + SH::ML_OFF);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    griddep_wait();  // the previous kernel in the stream (e.g. the insertion) has finished writing
-    griddep_launch_dependents();
+    // set-up that reads nothing the previous kernel in the stream writes runs before the wait
+    // for it: the barriers, and the tensor maps (kernel parameters) into the TMA unit's cache
     if (tid == 0) {
         for (int s = 0; s < ST; ++s) {
             mbar_init(&s_full[s], 33);          // producer lane 0's expect_tx + 32 producer lanes
@@ -268,6 +273,15 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
         *s_issued = 0;
         fence_mbar_init();
     }
+    if (warp == NWC && lane == 0) {
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+    }
+    griddep_wait();  // the previous kernel in the stream (e.g. the insertion) has finished writing
+    griddep_launch_dependents();
+    // the producer's first lengths and positions are in flight during the barrier below
+    UnitRaw first_raw{0, 0};
+    if (warp == NWC) first_raw = unit_raw(p, (long long)blockIdx.x + (long long)lane * gridDim.x);
     __syncthreads();
 
     if (warp == NWC) {
@@ -281,7 +295,11 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
         UnitRaw lane_raw{0, 0};
         for (int u = u_lo, k = 0; !stop; u += u_step, ++k) {
             const bool end = u >= u_hi;  // one end record after the last unit
-            if ((k & 31) == 0) lane_raw = unit_raw(p, (long long)u + (long long)lane * u_step);
+            if (k == 0) {
+                lane_raw = first_raw;
+            } else if ((k & 31) == 0) {
+                lane_raw = unit_raw(p, (long long)u + (long long)lane * u_step);
+            }
             const UnitRaw raw{__shfl_sync(kFull, lane_raw.len, k & 31), __shfl_sync(kFull, lane_raw.t, k & 31)};
             UnitInfo ui{};
             if (!end) ui = unit_info<T>(p, u, raw, lane == 0);
