@@ -161,6 +161,7 @@ __device__ __forceinline__ void ptile_next(const AsmParams& p, PTile& c) {
 __global__ void __launch_bounds__(kPThreads, 1) asm_score_planes_kernel(const __grid_constant__ AsmPlanesParams pp,
                                                                         const __grid_constant__ CUtensorMap tmQ) {
     griddep_launch_dependents();   // the merge may be scheduled now; it waits for this grid before reading keys
+    if (threadIdx.x == 0) prefetch_tensormap(&tmQ);
     const AsmParams& p = pp.a;
     extern __shared__ unsigned char s_raw[];
     unsigned char* sm = s_raw + ((1024u - (smem_u32(s_raw) & 1023u)) & 1023u);

@@ -120,6 +120,11 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
 // Programmatic dependent launch: wait until the previous kernel in the stream
 // has completed and its writes are visible (a no-op when the launch did not
 // ask for programmatic serialization), and allow the next kernel to launch.
+// fetch a tensor map (a __grid_constant__ kernel parameter) into the TMA unit's descriptor cache
+__device__ __forceinline__ void prefetch_tensormap(const void* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");

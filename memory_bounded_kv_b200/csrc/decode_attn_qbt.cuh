@@ -145,14 +145,8 @@ __global__ void __launch_bounds__(QbtShape<G>::NT, 1)
     int* s_qloads = reinterpret_cast<int*>(smem + SH::MISC_OFF) + 4;   // query blocks the producer loaded
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    griddep_wait();
-    griddep_launch_dependents();
-    if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tslot)),
-                     "r"(SH::TM_COLS)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-    }
+    // set-up that reads nothing the previous kernel in the stream writes runs before the wait
+    // for it: the barriers, and the tensor maps (kernel parameters) into the TMA unit's cache
     if (tid == 0) {
         for (int s = 0; s < ST; ++s) {
             mbar_init(&kv_full[s], 33);   // the copy's expect_tx + 32 producer lanes
@@ -177,6 +171,19 @@ __global__ void __launch_bounds__(QbtShape<G>::NT, 1)
         *s_issued = 0;
         *s_qloads = 0;
         fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+        prefetch_tensormap(&tmQ);
+    }
+    griddep_wait();
+    griddep_launch_dependents();
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tslot)),
+                     "r"(SH::TM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     tc_fence_before();
     __syncthreads();
