@@ -66,15 +66,15 @@ WORKLOADS = ("1", "2", "3", "3p", "4", "5", "5p")
 # (sha256 of the kernel's source file, workload, num_splits). Reported only while the source is
 # unchanged since the counters were taken.
 MEASURED_TRAFFIC = {
-    # decode_attn_tc_kernel at the Qwen3-8B-shaped layer, one split: 545,588,736 read + 3,245,824 written
+    # decode_attn_tc_kernel at the Qwen3-8B-shaped layer, one split: 545,578,752 read + 3,253,760 written
     # (bench.py --profile c2 under ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum)
-    ("ee137a975fba5d61", "2", 1): 548834560,
-    # the long-context attention (136,398,848 + 3,578,624) and its 64-way merge (4,242,688 + 0)
+    ("e062dfe96c96cf78", "2", 1): 548832512,
+    # the long-context attention (136,400,384 + 3,825,408) and its 64-way merge (4,242,688 + 0)
     # (bench.py --profile c3, the same metrics over both launches)
-    ("ee137a975fba5d61", "3", 64): 144220160,
-    # the lookup over the prepared memory (102,808,576 + 3,712,000) and its merge (6,998,528 + 0)
+    ("e062dfe96c96cf78", "3", 64): 144468480,
+    # the lookup over the prepared memory (102,811,136 + 3,112,704) and its merge (6,999,808 + 0)
     # (bench.py --profile c4, the same metrics over both launches)
-    ("173295e61443b3b8", "4", 4): 113519104,
+    ("efd6765f5e1aeb11", "4", 4): 112923648,
 }
 
 
