@@ -357,6 +357,7 @@ class DecodeBench:
             k, v = synth.long_context_kv(w)
             self.cache.k.copy_(_dev(k))
             self.cache.v.copy_(_dev(v))
+            self.cache.full = True   # every row holds its budget M after the stream
             torch.cuda.synchronize()
         else:
             self.cache = BoundedKVCache.from_host(w.k, w.v, None if plain else w.log_beta, w.pos, w.len, w.Hq, w.M,
@@ -416,13 +417,20 @@ class DecodeBench:
         return self.d_q[p], self.d_kn[p], self.d_vn[p], None if self.plain else self.d_lb[p], self.t_dev[i]
 
     def pre(self, i, x=None):
+        if self.cache.full:   # the step's one launch does the insertion (attn)
+            return
         _, kn, vn, lb, t = self._in(i, x)
         self.cache.insert(kn, vn, lb, t)
 
     def attn(self, i, x=None):
-        q, _, _, _, t = self._in(i, x)
+        q, kn, vn, lb, t = self._in(i, x)
         o, lse = (x["o"], x["lse"]) if x is not None and "o" in x else (self.o, self.lse)
-        self.cache.attend(q, t, o, lse)
+        if self.cache.full:
+            # budget enforcement from the previous step's records, insertion and attention in one
+            # launch (the first step after a set-up, with no records yet, runs as two)
+            self.cache.step(q, kn, vn, lb, t, o, lse)
+        else:
+            self.cache.attend(q, t, o, lse)
 
     def post(self, i, x=None):
         pass
@@ -438,24 +446,37 @@ class DecodeBench:
         return self.w.B
 
     def launches(self, i):
+        if self.cache.full:
+            return 1 + (self.S > 1)   # the fused step (+ split merge)
         return 2 + (self.S > 1)   # evict/insert, attention (+ split merge)
 
     def attn_bytes(self, i=None):
         """Algorithmic bytes of one attention launch: K, V (+ log beta) and pos of the cached slots
-        (pos feeds the eviction candidates), q, len, t in; o (fp32), lse out."""
+        (pos feeds the eviction candidates), q, len, t in; o (fp32), lse out. With the insertion
+        fused into it, also the step's records in, the new rows in and the victims' rows out."""
         w = self.w
         n = w.B * w.Hkv * w.M        # every (b, g) holds M slots in these workloads
         per_slot = 2 * w.d * 2 + 4 + (0 if self.plain else 4)
-        return n * per_slot + w.B * w.Hq * w.d * 2 + w.B * w.Hkv * 4 + w.B * 4 + w.B * w.Hq * (w.d * 4 + 4)
+        b = n * per_slot + w.B * w.Hq * w.d * 2 + w.B * w.Hkv * 4 + w.B * 4 + w.B * w.Hq * (w.d * 4 + 4)
+        if self.cache.full:
+            meta = 4 + (0 if self.plain else 4)
+            b += w.B * w.Hkv * (self.S * 16 + 2 * (2 * w.d * 2 + meta))
+        return b
 
     def other_bytes(self, i=None):
         """Budget enforcement reads the attention's per-split candidates (16 B each) and writes the
-        new row; the scan of log beta/pos happens inside the attention pass."""
+        new row; the scan of log beta/pos happens inside the attention pass. None when the step's
+        one launch does the insertion."""
         w = self.w
+        if self.cache.full:
+            return 0
         return w.B * w.Hkv * (self.S * 16 + 2 * w.d * 2 + 4 + 4 + 4)
 
     def kernel_name(self):
         merge = " + merge_splits_kernel" if self.S > 1 else ""
+        if self.cache.full:
+            return (f"kvb_decode_step = decode_attn_tc_kernel<d={self.w.d},G={self.w.Hq // self.w.Hkv},"
+                    f"bias={0 if self.plain else 1},insertion>{merge}, S={self.S}")
         return (f"kvb_decode_attn = decode_attn_tc_kernel<d={self.w.d},G={self.w.Hq // self.w.Hkv},"
                 f"bias={0 if self.plain else 1}>{merge}, S={self.S}")
 

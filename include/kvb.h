@@ -59,7 +59,8 @@ enum kvb_device_error {
     KVB_DERR_SPLIT = 1u << 1,     /* split_len * num_splits < len */
     KVB_DERR_RANGE = 1u << 2,     /* compaction range outside [0, len) */
     KVB_DERR_TIMEOUT = 1u << 3,   /* a bounded wait on a copy gave up */
-    KVB_DERR_PAGES = 1u << 4      /* a paged cache needed a page and its free stack was empty */
+    KVB_DERR_PAGES = 1u << 4,     /* a paged cache needed a page and its free stack was empty */
+    KVB_DERR_STEP = 1u << 5       /* kvb_decode_step: a row not full, or records not scored for t */
 };
 
 /* ------------------------------------------------------------------------
@@ -162,6 +163,41 @@ typedef struct kvb_evict_cand {
 } kvb_evict_cand;
 
 kvb_status kvb_decode_attn(const kvb_attn_args* args, kvb_stream stream);
+
+/* ------------------------------------------------------------------------
+ * kvb_decode_step -- budget enforcement, insertion and attention in one launch
+ *
+ * [TRIM] 2.1 at inference: a decode step of a cache that holds its budget
+ * evicts the slot with the lowest beta_i^(t-i) (kvb_evict_insert), writes the
+ * new token there, then attends (kvb_decode_attn). This call does both in the
+ * attention's launch, for caches that are full: the previous step's attention
+ * already scored every slot for this position and left per-split records
+ * (evict_cand), so the victim of row (b, g) is the best of its records; the
+ * CTA that reads the victim's tile replaces the staged row with the new token
+ * and writes it to the cache. Results equal kvb_evict_insert followed by
+ * kvb_decode_attn on the same arguments.
+ *
+ * - args: as kvb_decode_attn. k, v, log_beta and pos are WRITTEN at the
+ *   victim slots (the const qualifiers of kvb_attn_args do not apply here).
+ *   args->evict_cand is required: the records for position t[b] + 1 that this
+ *   step leaves for the next one.
+ * - k_new, v_new [B, Hkv, d] bf16 contiguous, 16-byte aligned; log_beta_new
+ *   [B, Hkv] f32, required exactly when args->log_beta is (else KVB_EINVAL).
+ * - M: the budget, 1 <= M <= cap. Every active row must hold M slots.
+ * - cand_in [B, Hkv, num_splits] kvb_evict_cand: the records the previous
+ *   attention left (stamped t[b]); a different array from args->evict_cand
+ *   (callers alternate two), 16-byte aligned.
+ * - victim [B, Hkv] int32, may be NULL: the slot each row's new token took,
+ *   -1 for an inactive row (t < 0).
+ * - Rows with t < 0 are inactive (nothing inserted, empty state). A row that
+ *   is not full (len != M), or whose records were not all scored for t[b], or
+ *   name no slot, is not changed: it gets the empty state, victim -1, and the
+ *   device error word KVB_DERR_STEP (use kvb_evict_insert + kvb_decode_attn
+ *   for such a step). Needs pos and t; no batch stride 0 (kv or meta).
+ * ---------------------------------------------------------------------- */
+kvb_status kvb_decode_step(const kvb_attn_args* args, const uint16_t* k_new, const uint16_t* v_new,
+                           const float* log_beta_new, int32_t M, const kvb_evict_cand* cand_in, int32_t* victim,
+                           kvb_stream stream);
 
 /* ------------------------------------------------------------------------
  * kvb_decode_attn_noalloc -- kvb_decode_attn without caller scratch

@@ -24,7 +24,7 @@ import torch
 from . import _lib
 
 __all__ = [
-    "KvbError", "kvb_decode_attn", "kvb_decode_attn_noalloc", "kvb_merge_states", "kvb_evict_insert", "kvb_compact_blocks",
+    "KvbError", "kvb_decode_attn", "kvb_decode_attn_noalloc", "kvb_decode_step", "kvb_merge_states", "kvb_evict_insert", "kvb_compact_blocks",
     "kvb_asm_workspace_bytes", "kvb_asm_lookup_merge", "kvb_asm_hier_workspace_bytes",
     "kvb_asm_hier_lookup_merge", "kvb_asm_aggregate_workspace_bytes", "kvb_asm_aggregate",
     "kvb_asm_entries_bf16", "kvb_asm_index_workspace_bytes", "kvb_asm_index_csr",
@@ -161,6 +161,49 @@ def kvb_decode_attn(q, k, v, log_beta, pos, len, t, o, lse=None, *, scale: float
     >= B*Hkv*num_splits*16 bytes to receive the next position's eviction candidates (see
     evict_candidates()), or None. Every shape is checked before anything is launched.
     """
+    a = _attn_args(q, k, v, log_beta, pos, len, t, o, lse, scale, num_splits, split_len, o_part, lse_part,
+                   evict_cand)
+    _check(_lib.lib().kvb_decode_attn(ctypes.byref(a), _stream(stream)), "kvb_decode_attn")
+
+
+def kvb_decode_step(q, k, v, log_beta, pos, len, t, o, lse, k_new, v_new, log_beta_new, M: int, cand_in,
+                    cand_out, *, victim=None, scale: float = 0.0, num_splits: int = 1, split_len: int = 0,
+                    o_part=None, lse_part=None, stream=None) -> None:
+    """Budget enforcement, insertion and attention of a full cache in one launch; see
+    kvb_decode_step in include/kvb.h. The arguments of kvb_decode_attn, plus k_new, v_new
+    [B, Hkv, d] bf16, log_beta_new [B, Hkv] f32 (exactly when log_beta is given), the budget M,
+    cand_in (the records the previous attention left, stamped t) and cand_out (the records for
+    t + 1; a different buffer), victim [B, Hkv] int32 or None. k, v, log_beta and pos are written.
+    """
+    if cand_out is None or cand_in is None:
+        raise ValueError("cand_in and cand_out are required")
+    a = _attn_args(q, k, v, log_beta, pos, len, t, o, lse, scale, num_splits, split_len, o_part, lse_part,
+                   cand_out)
+    B, Hkv, d = int(q.shape[0]), int(k.shape[1]), int(q.shape[2])
+    for name, x in (("k_new", k_new), ("v_new", v_new)):
+        _need(x, torch.bfloat16, name); _contig(x, name)
+        if tuple(x.shape) != (B, Hkv, d):
+            raise ValueError(f"{name} must be [B, Hkv, d]")
+    if (log_beta is None) != (log_beta_new is None):
+        raise ValueError("log_beta_new is needed exactly when log_beta is given")
+    if log_beta_new is not None:
+        _need(log_beta_new, torch.float32, "log_beta_new"); _contig(log_beta_new, "log_beta_new")
+        if tuple(log_beta_new.shape) != (B, Hkv):
+            raise ValueError("log_beta_new must be [B, Hkv]")
+    if victim is not None:
+        _need(victim, torch.int32, "victim"); _contig(victim, "victim")
+        if victim.numel() < B * Hkv:
+            raise ValueError("victim must hold B * Hkv entries")
+    cin = _cand_ptr(cand_in, B * Hkv * int(num_splits))
+    _check(_lib.lib().kvb_decode_step(ctypes.byref(a), k_new.data_ptr(), v_new.data_ptr(),
+                                      None if log_beta_new is None else log_beta_new.data_ptr(), int(M), cin,
+                                      None if victim is None else victim.data_ptr(), _stream(stream)),
+           "kvb_decode_step")
+
+
+def _attn_args(q, k, v, log_beta, pos, len, t, o, lse, scale, num_splits, split_len, o_part, lse_part,
+               evict_cand):
+    """Checks and marshals the arguments of kvb_decode_attn (and kvb_decode_step) into AttnArgs."""
     B, Hq, Hkv, d, cap = _decode_shapes(q, k, v, log_beta, pos, len, t, o, lse, num_splits, o_part, lse_part)
     if num_splits > 1 and (o_part is None or lse_part is None):
         raise ValueError("num_splits > 1 needs o_part and lse_part (decode_workspace())")
@@ -208,7 +251,7 @@ def kvb_decode_attn(q, k, v, log_beta, pos, len, t, o, lse=None, *, scale: float
         lse_part=None if lse_part is None else lse_part.data_ptr(), counters=None,
         o=o.data_ptr(), o_dtype=odt, lse=None if lse is None else lse.data_ptr(),
         evict_cand=None if evict_cand is None else _cand_ptr(evict_cand, B * Hkv * int(num_splits)))
-    _check(_lib.lib().kvb_decode_attn(ctypes.byref(a), _stream(stream)), "kvb_decode_attn")
+    return a
 
 
 def kvb_decode_attn_noalloc(q, k, v, log_beta, pos, len, t, o, lse=None, *, scale: float = 0.0,

@@ -13,8 +13,8 @@ _SZ = ctypes.c_size_t
 
 # symbols include/kvb.h declares (kept in sync by tests/test_abi.py)
 EXPORTS = (
-    "kvb_decode_attn", "kvb_decode_attn_noalloc", "kvb_merge_states", "kvb_evict_insert", "kvb_compact_blocks",
-    "kvb_asm_workspace_bytes", "kvb_asm_lookup_merge", "kvb_asm_hier_workspace_bytes",
+    "kvb_decode_attn", "kvb_decode_attn_noalloc", "kvb_decode_step", "kvb_merge_states", "kvb_evict_insert",
+    "kvb_compact_blocks", "kvb_asm_workspace_bytes", "kvb_asm_lookup_merge", "kvb_asm_hier_workspace_bytes",
     "kvb_asm_hier_lookup_merge", "kvb_asm_aggregate_workspace_bytes", "kvb_asm_aggregate",
     "kvb_asm_entries_bf16", "kvb_asm_index_workspace_bytes", "kvb_asm_index_csr",
     "kvb_asm_lookup_merge_grouped", "kvb_asm_aggregate_grouped",
@@ -26,7 +26,7 @@ EXPORTS = (
 
 KVB_OK, KVB_EINVAL, KVB_ECUDA, KVB_EDEVICE = 0, 1, 2, 3
 KVB_OUT_F32, KVB_OUT_BF16 = 0, 1
-DERR_LEN, DERR_SPLIT, DERR_RANGE, DERR_TIMEOUT, DERR_PAGES = 1, 2, 4, 8, 16
+DERR_LEN, DERR_SPLIT, DERR_RANGE, DERR_TIMEOUT, DERR_PAGES, DERR_STEP = 1, 2, 4, 8, 16, 32
 NOALLOC_SCRATCH_BYTES = 16 << 20   # KVB_NOALLOC_SCRATCH_BYTES
 
 
@@ -76,6 +76,7 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(path)
         L.kvb_decode_attn.argtypes = [ctypes.POINTER(AttnArgs), _P]
         L.kvb_decode_attn_noalloc.argtypes = [ctypes.POINTER(AttnArgs), _P]
+        L.kvb_decode_step.argtypes = [ctypes.POINTER(AttnArgs), _P, _P, _P, _I32, _P, _P, _P]
         L.kvb_merge_states.argtypes = [_P, _P, _I64, _I64, _I64, _I64, _I32, _I32, _I32, _P, _P, _P]
         L.kvb_evict_insert.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _P, _P,
                                        _I32, _P]
@@ -110,7 +111,7 @@ def lib() -> ctypes.CDLL:
         L.kvb_asm_planes_bytes.restype = _SZ
         L.kvb_asm_prepare.argtypes = [_P, _I32, _I32, _I32, _P, _SZ, _P]
         L.kvb_asm_lookup_merge_planes.argtypes = [_P, _P, _SZ, _P, _P, _P, _P] + [_I32] * 5 + [_P] * 4 + [_SZ, _P]
-        for f in ("kvb_decode_attn", "kvb_decode_attn_noalloc", "kvb_merge_states", "kvb_evict_insert", "kvb_compact_blocks",
+        for f in ("kvb_decode_attn", "kvb_decode_attn_noalloc", "kvb_decode_step", "kvb_merge_states", "kvb_evict_insert", "kvb_compact_blocks",
                   "kvb_asm_lookup_merge", "kvb_asm_hier_lookup_merge", "kvb_asm_aggregate",
                   "kvb_asm_entries_bf16", "kvb_asm_index_csr", "kvb_asm_lookup_merge_grouped",
                   "kvb_asm_aggregate_grouped", "kvb_get_error",

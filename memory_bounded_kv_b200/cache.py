@@ -15,7 +15,8 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import kvb_compact_blocks, kvb_decode_attn, kvb_evict_insert, decode_workspace, evict_candidates
+from . import (kvb_compact_blocks, kvb_decode_attn, kvb_decode_step, kvb_evict_insert, decode_workspace,
+               evict_candidates)
 
 
 def _dev(a, device):
@@ -42,9 +43,14 @@ class BoundedKVCache:
         self.o_part = self.lse_part = None
         if num_splits > 1:
             self.o_part, self.lse_part = decode_workspace(B, Hq, d, num_splits, device)
-        # eviction candidates for the next position, left by each attention pass
+        # eviction candidates for the next position, left by each attention pass; a fused step
+        # reads one buffer and writes the other
         self.cand = evict_candidates(B, Hkv, num_splits, device)
+        self.cand_next = evict_candidates(B, Hkv, num_splits, device)
         self.cand_valid = False
+        # the caller's statement that every row holds M slots (set by from_host when the lengths
+        # say so): then a step whose records are valid runs as one launch (kvb_decode_step)
+        self.full = False
 
     @classmethod
     def from_host(cls, k, v, log_beta, pos, len_, Hq, M, num_splits=1, split_len=0, device="cuda"):
@@ -56,6 +62,7 @@ class BoundedKVCache:
             c.log_beta.copy_(_dev(log_beta, device))
         c.pos.copy_(_dev(pos, device))
         c.len.copy_(_dev(len_, device))
+        c.full = bool(np.all(np.asarray(len_) == M))
         return c
 
     def insert(self, k_new, v_new, log_beta_new, t, stream=None):
@@ -80,13 +87,23 @@ class BoundedKVCache:
         self.cand_valid = cand is not None
 
     def step(self, q, k_new, v_new, log_beta_new, t, o, lse=None, stream=None):
-        """One decode step: budget enforcement + insertion, then attention (2 launches)."""
+        """One decode step: budget enforcement + insertion, then attention. One launch
+        (kvb_decode_step) when the cache is full and the last attention left the records for
+        this position; else two (kvb_evict_insert, kvb_decode_attn)."""
+        if self.full and self.cand_valid and t is not None:
+            kvb_decode_step(q, self.k, self.v, self.log_beta, self.pos, self.len, t, o, lse, k_new, v_new,
+                            log_beta_new if self.log_beta is not None else None, self.M, self.cand,
+                            self.cand_next, victim=self.victim, num_splits=self.num_splits,
+                            split_len=self.split_len, o_part=self.o_part, lse_part=self.lse_part, stream=stream)
+            self.cand, self.cand_next = self.cand_next, self.cand
+            return
         self.insert(k_new, v_new, log_beta_new, t, stream)
         self.attend(q, t, o, lse, stream)
 
     def compact(self, rm_start, rm_len, stream=None):
         kvb_compact_blocks(self.k, self.v, self.pos, self.log_beta, self.len, rm_start, rm_len, stream=stream)
         self.cand_valid = False
+        self.full = False
 
     def kv_bytes_read(self) -> int:
         """Bytes of K, V (and log_beta, pos when the bias is on) that one attention pass reads."""

@@ -70,6 +70,20 @@ struct DecodeTcParams {
     // logical slot s of (b, g) is row s % T of page table[(b * Hkv + g) * max_pages + s / T]
     const int* table;
     int max_pages, num_pages;
+    // fused insertion (INS kernels, a decode step in one launch): in every full row (len == M) the
+    // new token replaces the victim named by the previous attention's records cand_in (stamped
+    // t); the unit holding the victim patches its staged tile and writes the new row to the cache
+    uint16_t* k_w;
+    uint16_t* v_w;
+    long long kv_sb, kv_sh;   // element strides of the cache (slot stride D)
+    float* lb_w;              // log beta and pos of the cache, writable (meta strides m_sb, m_sh)
+    int* pos_w;
+    const uint16_t* k_new;    // [B, Hkv, D] bf16
+    const uint16_t* v_new;
+    const float* lb_new;      // [B, Hkv]; nullptr with lb == nullptr
+    const EvictCand* cand_in; // [B, Hkv, S]
+    int* victim;              // nullable [B, Hkv]: the slot replaced, -1 if none
+    int M;
 };
 
 template <int D, int G>
@@ -96,12 +110,17 @@ struct TcShape {
     static constexpr int EPI_OFF = (MISC_OFF + 64 + 15) / 16 * 16;      // [NWC][G][D] f32
     static constexpr int ML_OFF = EPI_OFF + NWC * G * D * 4;            // [NWC][G][2] f32
     static constexpr int CAND_OFF = ML_OFF + NWC * G * 2 * 4;           // [NWC] (key, slot)
-    static constexpr int END_OFF = CAND_OFF + NWC * 16;
+    // fused insertion: per stage the new token's K and V rows and its log beta
+    static constexpr int PATCH_BYTES = 4 * D + 16;
+    static constexpr int PATCH_OFF = (CAND_OFF + NWC * 16 + 15) / 16 * 16;  // [ST][PATCH_BYTES]
+    static constexpr int END_OFF = PATCH_OFF + STAGES * PATCH_BYTES;
     static constexpr size_t SMEM = 1024 + END_OFF;
     static_assert(D == 64 || D == 128, "d");
     static_assert(G == 1 || G == 2 || G == 4 || G == 8, "G");
-    static_assert(STAGE_BYTES % 1024 == 0 && Q_OFF % 16 == 0, "alignment");
+    static_assert(STAGE_BYTES % 1024 == 0 && Q_OFF % 16 == 0 && PATCH_BYTES % 16 == 0, "alignment");
 };
+// two CTAs per SM at the Qwen3-8B-like shape (228 KB of shared memory per SM, 1 KB reserved per CTA)
+static_assert(2 * (TcShape<128, 4>::SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
 
 // ---- PTX wrappers -------------------------------------------------------------
 
@@ -229,7 +248,62 @@ __device__ __forceinline__ UnitInfo unit_info(const DecodeTcParams& p, int u, Un
     return r;
 }
 
-template <int D, int G, bool BIAS, bool PAGED = false>
+// Fused insertion ("Cache What Lasts" section 2.1 at inference, as kvb_evict_insert): the slot of
+// row (b, g) that the new token takes. The victim is the smallest (score, pos) key among the row's
+// S records of the previous attention, which scored every slot for this position t.
+// RowRecords holds a lane's share of one row's records (records lane and lane + 32), loaded a unit
+// ahead of their use; rows of more than 64 splits read the rest when they are used.
+struct RowRecords {
+    EvictCand r[2];
+};
+
+__device__ __forceinline__ RowRecords load_row_records(const DecodeTcParams& p, int u, int lane) {
+    RowRecords x;
+    x.r[0] = x.r[1] = EvictCand{~0ull, -1, 0};
+    if (u < p.units) {
+        int b, g, split;
+        unit_coords(p, u, b, g, split);
+        const EvictCand* rec = p.cand_in + ((size_t)b * p.Hkv + g) * p.S;
+        if (lane < p.S) x.r[0] = rec[lane];
+        if (lane + 32 < p.S) x.r[1] = rec[lane + 32];
+    }
+    return x;
+}
+
+// Warp-collective (every lane of the producer warp). Returns -1 for an inactive row (t < 0:
+// nothing is inserted) and -2 for a row the fused step cannot update: not full (len != M), or a
+// record scored for another position, or no record naming a slot.
+__device__ __forceinline__ int row_victim(const DecodeTcParams& p, const RowRecords& x, int b, int g, int tb, int n,
+                                          int lane) {
+    unsigned long long best = ~0ull;
+    int best_slot = 0x7fffffff;
+    bool stale = false;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        if (lane + 32 * k < p.S) {
+            stale = stale || x.r[k].t != tb;
+            if (x.r[k].slot >= 0) argmin_merge(best, best_slot, x.r[k].key, x.r[k].slot);
+        }
+    }
+    const EvictCand* rec = p.cand_in + ((size_t)b * p.Hkv + g) * p.S;
+    for (int j = lane + 64; j < p.S; j += 32) {
+        const EvictCand c = rec[j];
+        stale = stale || c.t != tb;
+        if (c.slot >= 0) argmin_merge(best, best_slot, c.key, c.slot);
+    }
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) {
+        const unsigned long long k2 = __shfl_xor_sync(kFull, best, m);
+        const int s2 = __shfl_xor_sync(kFull, best_slot, m);
+        argmin_merge(best, best_slot, k2, s2);
+    }
+    stale = __any_sync(kFull, stale);
+    if (tb < 0) return -1;
+    if (n != p.M || stale || best == ~0ull || best_slot >= n) return -2;
+    return best_slot;
+}
+
+template <int D, int G, bool BIAS, bool PAGED = false, bool INS = false>
 __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
     decode_attn_tc_kernel(const __grid_constant__ DecodeTcParams p, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV) {
@@ -276,7 +350,11 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
     griddep_launch_dependents();
     // the producer's first lengths and positions are in flight during the barrier below
     UnitRaw first_raw{0, 0};
-    if (warp == NWC) first_raw = unit_raw(p, (long long)blockIdx.x + (long long)lane * gridDim.x);
+    RowRecords next_rec;   // fused insertion: the records of the producer's next unit's row
+    if (warp == NWC) {
+        first_raw = unit_raw(p, (long long)blockIdx.x + (long long)lane * gridDim.x);
+        if constexpr (INS) next_rec = load_row_records(p, blockIdx.x, lane);
+    }
     __syncthreads();
 
     if (warp == NWC) {
@@ -298,6 +376,19 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
             const UnitRaw raw{__shfl_sync(kFull, lane_raw.len, k & 31), __shfl_sync(kFull, lane_raw.t, k & 31)};
             UnitInfo ui{};
             if (!end) ui = unit_info<T>(p, u, raw, lane == 0);
+            int victim = -1;   // fused insertion: the slot (of the row) the new token takes, -1: none
+            if constexpr (INS) {
+                const RowRecords cur = next_rec;
+                next_rec = load_row_records(p, end ? p.units : u + u_step, lane);
+                if (!end) {
+                    victim = row_victim(p, cur, ui.b, ui.g, raw.t, raw.len, lane);
+                    if (ui.split == 0 && lane == 0) {
+                        if (victim == -2) raise_error(KVB_DERR_STEP);
+                        if (p.victim != nullptr) p.victim[ui.b * p.Hkv + ui.g] = max(victim, -1);
+                    }
+                    if (victim == -2) ui.ntiles = 0;   // a row the step cannot update: the empty state
+                }
+            }
             if (!end && ui.ntiles == 0) {
                 // an empty split (ragged lengths, inactive rows): write its empty state here;
                 // no record reaches the consumers
@@ -366,9 +457,13 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                         m[7] = ui.n;
                         m[8] = tb;
                         m[9] = ui.s0 + i * T;
+                        // fused insertion: the victim's row in this tile (or -1), and the new row
+                        const int vrow = (INS && data && victim >= m[9] && victim < m[9] + m[3]) ? victim - m[9] : -1;
+                        m[10] = vrow;
                         unsigned tx = data ? (unsigned)SH::STAGE_BYTES : 0u;
                         const bool with_q = data && i == 0;
                         if (with_q) tx += SH::QBYTES;
+                        if (vrow >= 0) tx += 4 * D;
                         mbar_arrive_expect_tx(&s_full[st], tx);
                         if (data) {
                             unsigned char* kt = smem + SH::RING_OFF + st * SH::STAGE_BYTES;
@@ -382,6 +477,13 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                                 tma_load_4d(kt + h * SH::HALF_BYTES, &tmK, 64 * h, row, gg, bb, &s_full[st]);
                                 tma_load_4d(vt + h * SH::HALF_BYTES, &tmV, 64 * h, row, gg, bb, &s_full[st]);
                             }
+                        }
+                        if (vrow >= 0) {
+                            unsigned char* pt = smem + SH::PATCH_OFF + st * SH::PATCH_BYTES;
+                            const size_t nrow = ((size_t)ui.b * p.Hkv + ui.g) * D;
+                            bulk_g2s(pt, p.k_new + nrow, (unsigned)(2 * D), &s_full[st]);
+                            bulk_g2s(pt + 2 * D, p.v_new + nrow, (unsigned)(2 * D), &s_full[st]);
+                            if (BIAS) cp_async4(pt + 4 * D, p.lb_new + (size_t)ui.b * p.Hkv + ui.g);
                         }
                         if (with_q) {
                             const uint16_t* qsrc = p.q + (size_t)ui.b * p.q_sb + (size_t)(ui.g * G) * p.q_sh;
@@ -464,6 +566,37 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
             const int u = m[0], i = m[1], ntiles = m[2], rows = m[3];
             if (u < 0) break;
             const int ub = m[4], ug = m[5], usplit = m[6], ut = m[8];   // (read before the stage is released)
+            if constexpr (INS) {
+                const int vrow = m[10];
+                if (vrow >= kw && vrow < kw + 16) {
+                    // fused insertion, the victim among this warp's slots: the new token's K and V
+                    // rows replace the staged ones (same 128-byte swizzle as the copy) and go to the
+                    // cache; its pos is t and its log beta the new one. No other CTA reads this slot.
+                    const unsigned char* pt = smem + SH::PATCH_OFF + st * SH::PATCH_BYTES;
+                    unsigned char* tile = smem + SH::RING_OFF + st * SH::STAGE_BYTES;
+                    const int slot = m[9] + vrow;
+                    const size_t crow = (size_t)ub * p.kv_sb + (size_t)ug * p.kv_sh + (size_t)slot * D;
+                    for (int c = lane; c < D / 4; c += 32) {   // 16-byte chunks: D/8 of K, then D/8 of V
+                        const int kv = c / (D / 8), cc = c % (D / 8);
+                        const uint4 x = *reinterpret_cast<const uint4*>(pt + kv * 2 * D + cc * 16);
+                        *reinterpret_cast<uint4*>(tile + kv * SH::TILE_BYTES + (cc >> 3) * SH::HALF_BYTES + vrow * 128 +
+                                                  (((cc & 7) ^ (vrow & 7)) << 4)) = x;
+                        *reinterpret_cast<uint4*>((kv ? p.v_w : p.k_w) + crow + cc * 8) = x;
+                    }
+                    if (lane == 0) {
+                        const size_t mrow = (size_t)ub * p.m_sb + (size_t)ug * p.m_sh + slot;
+                        s_pos[st * T + vrow] = ut;
+                        p.pos_w[mrow] = ut;
+                        if constexpr (BIAS) {
+                            const float lbn = *reinterpret_cast<const float*>(pt + 4 * D);
+                            s_lb[st * T + vrow] = lbn;
+                            p.lb_w[mrow] = lbn;
+                        }
+                    }
+                    fence_proxy_async_smem();   // the stage's next copy (async proxy) follows these writes
+                    __syncwarp();
+                }
+            }
             if (i == 0) {
                 cand_key = ~0ull;
                 cand_slot = 0x7fffffff;

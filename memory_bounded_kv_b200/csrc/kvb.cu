@@ -164,10 +164,10 @@ kvb_status launch_merge(const float* o_part, const float* lse_part, int R, int S
                       o_bf16, lse);
 }
 
-template <int D, int G, bool BIAS>
+template <int D, int G, bool BIAS, bool INS = false>
 kvb_status launch_decode_tc(const kvb::DecodeTcParams& p, const kvb_attn_args* a, cudaStream_t st) {
     using SH = kvb::TcShape<D, G>;
-    auto kern = kvb::decode_attn_tc_kernel<D, G, BIAS>;
+    auto kern = kvb::decode_attn_tc_kernel<D, G, BIAS, false, INS>;
     const size_t smem = SH::SMEM;
     if (set_smem(kern, smem) != KVB_OK) return KVB_ECUDA;
     CUtensorMap mk, mv;
@@ -307,18 +307,18 @@ kvb_status paged_view(const kvb_paged_cache* c, kvb::PagedCache* out) {
     return KVB_OK;
 }
 
-template <int D, int G>
+template <int D, int G, bool INS>
 kvb_status tc_bias(const kvb::DecodeTcParams& p, const kvb_attn_args* a, bool bias, cudaStream_t st) {
-    return bias ? launch_decode_tc<D, G, true>(p, a, st) : launch_decode_tc<D, G, false>(p, a, st);
+    return bias ? launch_decode_tc<D, G, true, INS>(p, a, st) : launch_decode_tc<D, G, false, INS>(p, a, st);
 }
 
-template <int D>
+template <int D, bool INS = false>
 kvb_status tc_g(const kvb::DecodeTcParams& p, const kvb_attn_args* a, int G, bool bias, cudaStream_t st) {
     switch (G) {
-        case 1: return tc_bias<D, 1>(p, a, bias, st);
-        case 2: return tc_bias<D, 2>(p, a, bias, st);
-        case 4: return tc_bias<D, 4>(p, a, bias, st);
-        case 8: return tc_bias<D, 8>(p, a, bias, st);
+        case 1: return tc_bias<D, 1, INS>(p, a, bias, st);
+        case 2: return tc_bias<D, 2, INS>(p, a, bias, st);
+        case 4: return tc_bias<D, 4, INS>(p, a, bias, st);
+        case 8: return tc_bias<D, 8, INS>(p, a, bias, st);
         default: return KVB_EINVAL;
     }
 }
@@ -357,7 +357,7 @@ std::atomic<unsigned long long> g_withhold_next{0};
 
 extern "C" {
 
-int32_t kvb_abi_version(void) { return 6; }
+int32_t kvb_abi_version(void) { return 7; }
 
 kvb_status kvb_test_withhold_next_decode(uint64_t wait_limit_ns) {
     if (wait_limit_ns < 1000ull || wait_limit_ns > 1000000000ull) return KVB_EINVAL;
@@ -386,7 +386,12 @@ kvb_status kvb_get_error(kvb_stream stream, uint32_t* bits) {
     return KVB_EDEVICE;
 }
 
-kvb_status kvb_decode_attn(const kvb_attn_args* a, kvb_stream stream) {
+}  // extern "C"
+
+namespace {
+
+// The host checks of kvb_decode_attn (and kvb_decode_step), and the kernel parameters.
+kvb_status attn_params(const kvb_attn_args* a, kvb::DecodeTcParams* out, int* G_out) {
     if (a == nullptr) return KVB_EINVAL;
     if (a->B < 1 || a->Hq < 1 || a->Hkv < 1 || a->cap < 1) return KVB_EINVAL;
     if (a->d != 64 && a->d != 128) return KVB_EINVAL;
@@ -417,7 +422,8 @@ kvb_status kvb_decode_attn(const kvb_attn_args* a, kvb_stream stream) {
     const long long units = (long long)a->B * a->Hkv * a->num_splits;
     if (units > 0x7fffffffLL) return KVB_EINVAL;
 
-    kvb::DecodeTcParams p;
+    kvb::DecodeTcParams& p = *out;
+    p = kvb::DecodeTcParams{};
     p.q = a->q; p.q_sb = a->q_stride_b; p.q_sh = a->q_stride_h;
     p.lb = a->log_beta; p.pos = a->pos; p.m_sb = a->meta_stride_b; p.m_sh = a->meta_stride_h;
     p.len = a->len; p.t = a->t;
@@ -431,6 +437,20 @@ kvb_status kvb_decode_attn(const kvb_attn_args* a, kvb_stream stream) {
     p.cand = static_cast<kvb::EvictCand*>(a->evict_cand);
     p.wait_ns = 1000000000ull;
     p.withhold = 0;
+    *G_out = G;
+    return KVB_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+kvb_status kvb_decode_attn(const kvb_attn_args* a, kvb_stream stream) {
+    kvb::DecodeTcParams p;
+    int G = 0;
+    const kvb_status chk = attn_params(a, &p, &G);
+    if (chk != KVB_OK) return chk;
+    const bool bias = a->log_beta != nullptr;
     if (g_withhold_next.load(std::memory_order_relaxed) != 0) {
         const unsigned long long lim = g_withhold_next.exchange(0);
         if (lim != 0) {
@@ -461,6 +481,36 @@ kvb_status kvb_decode_attn(const kvb_attn_args* a, kvb_stream stream) {
         return a->d == 128 ? qb_dispatch<128>(q, a, G, bias, st) : qb_dispatch<64>(q, a, G, bias, st);
     }
     return a->d == 128 ? tc_g<128>(p, a, G, bias, st) : tc_g<64>(p, a, G, bias, st);
+}
+
+kvb_status kvb_decode_step(const kvb_attn_args* a, const uint16_t* k_new, const uint16_t* v_new,
+                           const float* log_beta_new, int32_t M, const kvb_evict_cand* cand_in, int32_t* victim,
+                           kvb_stream stream) {
+    kvb::DecodeTcParams p;
+    int G = 0;
+    const kvb_status chk = attn_params(a, &p, &G);
+    if (chk != KVB_OK) return chk;
+    const bool bias = a->log_beta != nullptr;
+    // one cache row per (b, g): no batch stride 0; the records in and out are different arrays
+    if (a->kv_stride_b == 0 || a->meta_stride_b == 0 || !a->pos || !a->t || !a->evict_cand || !cand_in) return KVB_EINVAL;
+    if (cand_in == a->evict_cand || (reinterpret_cast<uintptr_t>(cand_in) & 15u)) return KVB_EINVAL;
+    if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return KVB_EINVAL;
+    if (bias != (log_beta_new != nullptr)) return KVB_EINVAL;
+    if (M < 1 || M > a->cap) return KVB_EINVAL;
+    p.k_w = const_cast<uint16_t*>(a->k);
+    p.v_w = const_cast<uint16_t*>(a->v);
+    p.kv_sb = a->kv_stride_b;
+    p.kv_sh = a->kv_stride_h;
+    p.lb_w = const_cast<float*>(a->log_beta);
+    p.pos_w = const_cast<int32_t*>(a->pos);
+    p.k_new = k_new;
+    p.v_new = v_new;
+    p.lb_new = log_beta_new;
+    p.cand_in = reinterpret_cast<const kvb::EvictCand*>(cand_in);
+    p.victim = victim;
+    p.M = M;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return a->d == 128 ? tc_g<128, true>(p, a, G, bias, st) : tc_g<64, true>(p, a, G, bias, st);
 }
 
 kvb_status kvb_decode_attn_noalloc(const kvb_attn_args* a, kvb_stream stream) {

@@ -47,7 +47,7 @@ def test_attn_args_struct_matches_header():
 
 def test_status_strings_and_version():
     L = _lib.lib()
-    assert L.kvb_abi_version() == 6
+    assert L.kvb_abi_version() == 7
     assert L.kvb_status_str(0) == b"ok"
     assert L.kvb_status_str(1) == b"invalid argument"
 
