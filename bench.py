@@ -1182,9 +1182,10 @@ def run_workload(key, splits, args, world, local, K, W, hbm_peak, peak_kind, cpu
 # profiling cases: the dominant launches of each workload at its shape, a few times
 # ----------------------------------------------------------------------------------------------
 
-def _profile_decode(B, Hq, Hkv, d, cap, lens, S, split_len, bias, reps=4):
+def _profile_decode(B, Hq, Hkv, d, cap, lens, S, split_len, bias, reps=4, fused=False):
     """kvb_decode_attn over a filled cache (K, V ~ N(0, 1), log beta ~ U(-3, -0.01), positions 0..cap-1)
-    with the given lengths, `reps` times."""
+    with the given lengths, `reps` times. `fused` (a full cache): one attention that leaves the
+    eviction records, then `reps` decode steps of kvb_decode_step (insertion inside the launch)."""
     import memory_bounded_kv_b200 as kvb
     from memory_bounded_kv_b200.cache import BoundedKVCache
     g = torch.Generator(device="cuda").manual_seed(0)
@@ -1199,20 +1200,31 @@ def _profile_decode(B, Hq, Hkv, d, cap, lens, S, split_len, bias, reps=4):
     t = torch.full((B,), cap + 1, dtype=torch.int32, device="cuda")
     o = torch.zeros(B, Hq, d, device="cuda")
     lse = torch.zeros(B, Hq, device="cuda")
-    for _ in range(reps):
+    if fused:
+        c.full = True
+        kn = torch.randn(B, Hkv, d, device="cuda", generator=g).to(torch.bfloat16)
+        vn = torch.randn(B, Hkv, d, device="cuda", generator=g).to(torch.bfloat16)
+        lbn = torch.full((B, Hkv), -0.5, device="cuda") if bias else None
         c.attend(q, t, o, lse)
+        for r in range(reps):
+            c.step(q, kn, vn, lbn, t + 1 + r, o, lse)
+    else:
+        for _ in range(reps):
+            c.attend(q, t, o, lse)
     torch.cuda.synchronize()
     return kvb.kvb_get_error()
 
 
 def _profile_c2():
-    """The Qwen3-8B-shaped layer: 32 x 8 rows of 4096 slots, one split."""
-    return _profile_decode(32, 32, 8, 128, 4096, np.full((32, 8), 4096), 1, 0, True)
+    """The Qwen3-8B-shaped layer: 32 x 8 rows of 4096 slots, one split; an attention, then fused
+    decode steps (the bench's steady state)."""
+    return _profile_decode(32, 32, 8, 128, 4096, np.full((32, 8), 4096), 1, 0, True, fused=True)
 
 
 def _profile_c3():
-    """The long-context workload's attention: 4 x 8 rows of 8192 slots, 64 splits."""
-    return _profile_decode(4, 32, 8, 128, 8192, np.full((4, 8), 8192), 64, 0, True)
+    """The long-context workload: 4 x 8 rows of 8192 slots, 64 splits; an attention, then fused
+    decode steps."""
+    return _profile_decode(4, 32, 8, 128, 8192, np.full((4, 8), 8192), 64, 0, True, fused=True)
 
 
 def _profile_c5():
