@@ -66,15 +66,16 @@ WORKLOADS = ("1", "2", "3", "3p", "4", "5", "5p")
 # (sha256 of the kernel's source file, workload, num_splits). Reported only while the source is
 # unchanged since the counters were taken.
 MEASURED_TRAFFIC = {
-    # decode_attn_tc_kernel at the Qwen3-8B-shaped layer, one split: 545,578,752 read + 3,253,760 written
+    # the fused decode step (decode_attn_tc_kernel with the insertion) at the Qwen3-8B-shaped layer,
+    # one split: 545,752,576 read + 3,388,416 written
     # (bench.py --profile c2 under ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum)
-    ("e062dfe96c96cf78", "2", 1): 548832512,
-    # the long-context attention (136,400,384 + 3,825,408) and its 64-way merge (4,242,688 + 0)
+    ("bebded481a40d706", "2", 1): 549140992,
+    # the long-context fused step (136,461,824 + 5,333,248) and its 64-way merge (4,242,688 + 0)
     # (bench.py --profile c3, the same metrics over both launches)
-    ("e062dfe96c96cf78", "3", 64): 144468480,
-    # the lookup over the prepared memory (102,811,136 + 3,112,704) and its merge (6,999,808 + 0)
+    ("bebded481a40d706", "3", 64): 146037760,
+    # the lookup over the prepared memory (102,807,552 + 3,361,792) and its merge (7,000,576 + 0)
     # (bench.py --profile c4, the same metrics over both launches)
-    ("efd6765f5e1aeb11", "4", 4): 112923648,
+    ("efd6765f5e1aeb11", "4", 4): 113169920,
 }
 
 
