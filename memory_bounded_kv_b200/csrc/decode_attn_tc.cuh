@@ -154,6 +154,24 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a2
         : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
 }
 
+// D = A . B + C, m16n8k16, bf16 inputs, fp32 accumulators, all 16 rows of A.
+__device__ __forceinline__ void mma_bf16_a(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// the transpose of an 8x8 b16 matrix held as the warp's standard fragment (lane l: row l / 4,
+// columns 2 (l % 4) and 2 (l % 4) + 1)
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -532,20 +550,27 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
         if (lane == 0) *s_issued = it;
     } else if (warp < NWC) {
         // ======================= consumer warps =======================
-        const int r = lane >> 2;          // M row = query head within the group (rows >= G are padding)
-        const int cq = lane & 3;          // quad index: columns 2*cq, 2*cq+1 of each 8-wide n-tile
+        // Both products keep the G query heads in the N dimension (8 columns, heads >= G zero):
+        //   S^T = K Q^T     A = this warp's 16 slots of K (ldmatrix), B = Q^T (registers)
+        //   O^T += V^T P^T  A = V^T (ldmatrix.trans), B = P^T, the accumulator of S^T with each
+        //                   8x8 block transposed in registers (movmatrix)
+        // so a warp issues D/16 + 2 D/16 mma per tile, and the fragments a lane holds are slots
+        // kw + r and kw + r + 8 of heads 2 cq and 2 cq + 1 (S), dims 16 m + r and 16 m + r + 8 of
+        // the same heads (O).
+        const int r = lane >> 2;          // fragment row; also the head whose Q column this lane loads
+        const int cq = lane & 3;          // fragment column pair: heads 2 cq, 2 cq + 1
         const int kw = 16 * warp;         // this warp's first slot in a tile
         const uint32_t ring = smem_u32(smem + SH::RING_OFF);
         // ldmatrix row addresses (relative to a tile half): swizzle xor = row & 7 = lane & 7
-        const int kq_row = kw + (lane & 7) + ((lane >> 4) << 3);   // QK operand rows (keys)
-        const int kq_hi = (lane >> 3) & 1;
-        const int v_row = kw + (lane & 7) + (((lane >> 3) & 1) << 3);  // PV operand rows
-        const int v_hi = lane >> 4;
+        const int ka_row = kw + (lane & 7) + (((lane >> 3) & 1) << 3);   // K as A: slots 0-7, 8-15
+        const int ka_hi = lane >> 4;                                     // then dims 8-15 of the step
+        const int va_row = kw + (lane & 7) + ((lane >> 4) << 3);         // V^T as A (transposed copy)
+        const int va_hi = (lane >> 3) & 1;
         const int sw = lane & 7;
 
-        uint32_t qa[SH::KSTEPS][2];
-        float acc[SH::NTILES][4];
-        float m_run = -INFINITY, l_run = 0.f;
+        uint32_t qa[SH::KSTEPS][2];       // Q^T fragments (B operand of S^T)
+        float acc[D / 16][4];             // O^T fragments
+        float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};   // heads 2 cq, 2 cq + 1
         const bool want_cand = p.cand != nullptr;
         unsigned long long cand_key = ~0ull;  // this lane's best eviction key in the unit
         int cand_slot = 0x7fffffff;
@@ -615,10 +640,10 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                 }
             }
             if (i == 0) {
-                m_run = -INFINITY;
-                l_run = 0.f;
+                m_run[0] = m_run[1] = -INFINITY;
+                l_run[0] = l_run[1] = 0.f;
 #pragma unroll
-                for (int j = 0; j < SH::NTILES; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+                for (int j = 0; j < D / 16; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
                 if (ntiles > 0) {
                     const uint16_t* qs = s_q + st * G * D;
 #pragma unroll
@@ -636,17 +661,16 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
             if (ntiles > 0) {
                 const uint32_t kt = ring + st * SH::STAGE_BYTES;
                 const uint32_t vt = kt + SH::TILE_BYTES;
-                // ---- S = Q K^T for this warp's 16 slots (two n-tiles of 8)
-                float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                // ---- S^T = K Q^T for this warp's 16 slots
+                float sc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int s = 0; s < SH::KSTEPS; ++s) {
-                    const int chunk = 2 * (s & 3) + kq_hi;
+                    const int chunk = 2 * (s & 3) + ka_hi;
                     const uint32_t addr =
-                        kt + (s >> 2) * SH::HALF_BYTES + kq_row * 128 + ((chunk ^ sw) << 4);
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4(addr, b0, b1, b2, b3);
-                    mma_bf16(sc[0], qa[s][0], qa[s][1], b0, b1);
-                    mma_bf16(sc[1], qa[s][0], qa[s][1], b2, b3);
+                        kt + (s >> 2) * SH::HALF_BYTES + ka_row * 128 + ((chunk ^ sw) << 4);
+                    uint32_t a0, a1, a2, a3;
+                    ldsm_x4(addr, a0, a1, a2, a3);
+                    mma_bf16_a(sc, a0, a1, a2, a3, qa[s][0], qa[s][1]);
                 }
                 if (rows < T && kw + 16 > rows) {
                     // tail: zero this warp's V rows past the split end (K rows there are masked)
@@ -662,62 +686,67 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                     fence_proxy_async_smem();
                     __syncwarp();
                 }
-                // ---- logits, online softmax (row r of this lane; slots 2cq, 2cq+1, 8+2cq, 8+2cq+1):
-                // scale q.k + (t - pos) log beta (one float32 product), -inf past the split's end
-                const int sa = kw + 2 * cq, sbb = sa + 8;
-                float bv[4] = {0.f, 0.f, 0.f, 0.f};
+                // ---- logits, online softmax (slots sa = kw + r and sb = sa + 8 of this lane, heads 2 cq and
+                // 2 cq + 1): scale q.k + (t - pos) log beta (one float32 product), -inf past the split's end
+                const int sa = kw + r, sb = sa + 8;
+                float ba = 0.f, bb = 0.f;
                 if constexpr (BIAS) {
-                    const int2 pA = *reinterpret_cast<const int2*>(s_pos + st * T + sa);
-                    const int2 pB = *reinterpret_cast<const int2*>(s_pos + st * T + sbb);
-                    const float2 lA = *reinterpret_cast<const float2*>(s_lb + st * T + sa);
-                    const float2 lB = *reinterpret_cast<const float2*>(s_lb + st * T + sbb);
-                    bv[0] = __fmul_rn(__int2float_rn(ut - pA.x), lA.x);
-                    bv[1] = __fmul_rn(__int2float_rn(ut - pA.y), lA.y);
-                    bv[2] = __fmul_rn(__int2float_rn(ut - pB.x), lB.x);
-                    bv[3] = __fmul_rn(__int2float_rn(ut - pB.y), lB.y);
+                    ba = __fmul_rn(__int2float_rn(ut - s_pos[st * T + sa]), s_lb[st * T + sa]);
+                    bb = __fmul_rn(__int2float_rn(ut - s_pos[st * T + sb]), s_lb[st * T + sb]);
                 }
                 float x[4];
-                x[0] = (sa < rows) ? fmaf(sc[0][0], p.scale, bv[0]) : -INFINITY;
-                x[1] = (sa + 1 < rows) ? fmaf(sc[0][1], p.scale, bv[1]) : -INFINITY;
-                x[2] = (sbb < rows) ? fmaf(sc[1][0], p.scale, bv[2]) : -INFINITY;
-                x[3] = (sbb + 1 < rows) ? fmaf(sc[1][1], p.scale, bv[3]) : -INFINITY;
-                float tmax = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-                tmax = fmaxf(tmax, __shfl_xor_sync(kFull, tmax, 1));
-                tmax = fmaxf(tmax, __shfl_xor_sync(kFull, tmax, 2));
-                const float m_new = fmaxf(m_run, tmax);
-                const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-                const float alpha = exp2f((m_run - m_use) * kLog2e);
+                x[0] = (sa < rows) ? fmaf(sc[0], p.scale, ba) : -INFINITY;   // slot sa, head 2 cq
+                x[1] = (sa < rows) ? fmaf(sc[1], p.scale, ba) : -INFINITY;   // slot sa, head 2 cq + 1
+                x[2] = (sb < rows) ? fmaf(sc[2], p.scale, bb) : -INFINITY;   // slot sb, head 2 cq
+                x[3] = (sb < rows) ? fmaf(sc[3], p.scale, bb) : -INFINITY;   // slot sb, head 2 cq + 1
+                // each head's maximum over the warp's 16 slots: the lanes with the same cq hold them
+                float t0 = fmaxf(x[0], x[2]), t1 = fmaxf(x[1], x[3]);
+#pragma unroll
+                for (int o2 = 4; o2 <= 16; o2 <<= 1) {
+                    t0 = fmaxf(t0, __shfl_xor_sync(kFull, t0, o2));
+                    t1 = fmaxf(t1, __shfl_xor_sync(kFull, t1, o2));
+                }
+                const float mn0 = fmaxf(m_run[0], t0), mn1 = fmaxf(m_run[1], t1);
+                const float mu0 = (mn0 == -INFINITY) ? 0.f : mn0, mu1 = (mn1 == -INFINITY) ? 0.f : mn1;
+                const float al0 = exp2f((m_run[0] - mu0) * kLog2e), al1 = exp2f((m_run[1] - mu1) * kLog2e);
                 float pr[4];
+                pr[0] = exp2f((x[0] - mu0) * kLog2e);
+                pr[1] = exp2f((x[1] - mu1) * kLog2e);
+                pr[2] = exp2f((x[2] - mu0) * kLog2e);
+                pr[3] = exp2f((x[3] - mu1) * kLog2e);
+                l_run[0] = fmaf(l_run[0], al0, pr[0] + pr[2]);   // this lane's slots; summed over lanes at the end
+                l_run[1] = fmaf(l_run[1], al1, pr[1] + pr[3]);
+                m_run[0] = mn0;
+                m_run[1] = mn1;
+                if (__any_sync(kFull, al0 != 1.f || al1 != 1.f)) {
 #pragma unroll
-                for (int j = 0; j < 4; ++j) pr[j] = exp2f((x[j] - m_use) * kLog2e);
-                l_run = fmaf(l_run, alpha, (pr[0] + pr[1]) + (pr[2] + pr[3]));
-                m_run = m_new;
-                if (__any_sync(kFull, alpha != 1.f)) {
-#pragma unroll
-                    for (int j = 0; j < SH::NTILES; ++j) {
-                        acc[j][0] *= alpha;
-                        acc[j][1] *= alpha;
+                    for (int j = 0; j < D / 16; ++j) {
+                        acc[j][0] *= al0;
+                        acc[j][1] *= al1;
+                        acc[j][2] *= al0;
+                        acc[j][3] *= al1;
                     }
                 }
-                // ---- P as the A operand: high bf16 part and bf16 residual
-                const uint32_t ph0 = pack_bf16(pr[0], pr[1]);
-                const uint32_t ph2 = pack_bf16(pr[2], pr[3]);
-                const uint32_t pl0 = pack_bf16(pr[0] - __uint_as_float(ph0 << 16),
-                                               pr[1] - __uint_as_float(ph0 & 0xffff0000u));
-                const uint32_t pl2 = pack_bf16(pr[2] - __uint_as_float(ph2 << 16),
-                                               pr[3] - __uint_as_float(ph2 & 0xffff0000u));
-                // ---- O += P V (two n-tiles of 8 dims per ldmatrix)
+                // ---- P^T as the B operand: high bf16 part and bf16 residual; the accumulator of S^T holds
+                // (slot, head) blocks, the B fragment wants (head, slot): one movmatrix per 8x8 block
+                const uint32_t h0 = pack_bf16(pr[0], pr[1]);
+                const uint32_t h1 = pack_bf16(pr[2], pr[3]);
+                const uint32_t l0 = pack_bf16(pr[0] - __uint_as_float(h0 << 16),
+                                              pr[1] - __uint_as_float(h0 & 0xffff0000u));
+                const uint32_t l1 = pack_bf16(pr[2] - __uint_as_float(h1 << 16),
+                                              pr[3] - __uint_as_float(h1 & 0xffff0000u));
+                const uint32_t bh0 = movmatrix_t(h0), bh1 = movmatrix_t(h1);
+                const uint32_t bl0 = movmatrix_t(l0), bl1 = movmatrix_t(l1);
+                // ---- O^T += V^T P^T, D / 16 tiles of 16 dims
 #pragma unroll
-                for (int j = 0; j < SH::NTILES / 2; ++j) {
-                    const int chunk = 2 * (j & 3) + v_hi;
+                for (int j = 0; j < D / 16; ++j) {
+                    const int chunk = 2 * (j & 3) + va_hi;
                     const uint32_t addr =
-                        vt + (j >> 2) * SH::HALF_BYTES + v_row * 128 + ((chunk ^ sw) << 4);
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4_t(addr, b0, b1, b2, b3);
-                    mma_bf16(acc[2 * j], ph0, ph2, b0, b1);
-                    mma_bf16(acc[2 * j], pl0, pl2, b0, b1);
-                    mma_bf16(acc[2 * j + 1], ph0, ph2, b2, b3);
-                    mma_bf16(acc[2 * j + 1], pl0, pl2, b2, b3);
+                        vt + (j >> 2) * SH::HALF_BYTES + va_row * 128 + ((chunk ^ sw) << 4);
+                    uint32_t a0, a1, a2, a3;
+                    ldsm_x4_t(addr, a0, a1, a2, a3);
+                    mma_bf16_a(acc[j], a0, a1, a2, a3, bh0, bh1);
+                    mma_bf16_a(acc[j], a0, a1, a2, a3, bl0, bl1);
                 }
             }
             __syncwarp();
@@ -726,8 +755,11 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
             if (ntiles > 0 && i != ntiles - 1) continue;
 
             // ======== end of unit: post this warp's partial state to the epilogue warp ========
-            l_run += __shfl_xor_sync(kFull, l_run, 1);
-            l_run += __shfl_xor_sync(kFull, l_run, 2);
+#pragma unroll
+            for (int o2 = 4; o2 <= 16; o2 <<= 1) {
+                l_run[0] += __shfl_xor_sync(kFull, l_run[0], o2);
+                l_run[1] += __shfl_xor_sync(kFull, l_run[1], o2);
+            }
             if (want_cand) {
 #pragma unroll
                 for (int o2 = 8; o2 >= 1; o2 >>= 1) {
@@ -749,14 +781,20 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                 aborted = true;
                 break;
             }
-            if (r < G) {
 #pragma unroll
-                for (int j = 0; j < SH::NTILES; ++j)
-                    *reinterpret_cast<float2*>(s_o + (warp * G + r) * D + 8 * j + 2 * cq) =
-                        make_float2(acc[j][0], acc[j][1]);
-                if (cq == 0) {
-                    s_ml[(warp * G + r) * 2] = m_run;
-                    s_ml[(warp * G + r) * 2 + 1] = l_run;
+            for (int jh = 0; jh < 2; ++jh) {
+                const int h = 2 * cq + jh;
+                if (h < G) {
+                    float* dst = s_o + (warp * G + h) * D + r;
+#pragma unroll
+                    for (int j = 0; j < D / 16; ++j) {
+                        dst[16 * j] = acc[j][jh];
+                        dst[16 * j + 8] = acc[j][2 + jh];
+                    }
+                    if (r == 0) {
+                        s_ml[(warp * G + h) * 2] = m_run[jh];
+                        s_ml[(warp * G + h) * 2 + 1] = l_run[jh];
+                    }
                 }
             }
             if (lane == 0) {
