@@ -107,12 +107,13 @@ struct TcShape {
     static constexpr int META_OFF = CLB_OFF + STAGES * T * 4;           // [ST][16] int
     static constexpr int BAR_OFF = META_OFF + STAGES * 64;              // full[ST], empty[ST], epi full/empty
     static constexpr int MISC_OFF = BAR_OFF + (2 * STAGES + 2) * 8;     // abort, issued, -, -, unit record [5]
-    static constexpr int EPI_OFF = (MISC_OFF + 64 + 15) / 16 * 16;      // [NWC][G][D] f32
-    static constexpr int ML_OFF = EPI_OFF + NWC * G * D * 4;            // [NWC][G][2] f32
-    static constexpr int CAND_OFF = ML_OFF + NWC * G * 2 * 4;           // [NWC] (key, slot)
+    static constexpr int EPI_LD = D + 4;   // row stride (floats): the posting lanes' rows fall in distinct banks
+    static constexpr int EPI_OFF = (MISC_OFF + 64 + 15) / 16 * 16;      // [NWC][G][EPI_LD] f32
+    static constexpr int ML_OFF = EPI_OFF + NWC * G * EPI_LD * 4;       // [NWC][G][2] f32
+    static constexpr int CAND_OFF = ML_OFF + NWC * G * 2 * 4;           // [NWC][16] keys, then [NWC][16] slots
     // fused insertion: per stage the new token's K and V rows and its log beta
     static constexpr int PATCH_BYTES = 4 * D + 16;
-    static constexpr int PATCH_OFF = (CAND_OFF + NWC * 16 + 15) / 16 * 16;  // [ST][PATCH_BYTES]
+    static constexpr int PATCH_OFF = (CAND_OFF + NWC * 16 * 12 + 15) / 16 * 16;  // [ST][PATCH_BYTES]
     static constexpr int END_OFF = PATCH_OFF + STAGES * PATCH_BYTES;
     static constexpr size_t SMEM = 1024 + END_OFF;
     static_assert(D == 64 || D == 128, "d");
@@ -335,7 +336,7 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
     int* s_pos = reinterpret_cast<int*>(smem + SH::CPOS_OFF);
     float* s_lb = reinterpret_cast<float*>(smem + SH::CLB_OFF);
     unsigned long long* s_ck = reinterpret_cast<unsigned long long*>(smem + SH::CAND_OFF);
-    int* s_cs = reinterpret_cast<int*>(smem + SH::CAND_OFF + NWC * 8);
+    int* s_cs = reinterpret_cast<int*>(smem + SH::CAND_OFF + NWC * 16 * 8);
     uint64_t* s_full = reinterpret_cast<uint64_t*>(smem + SH::BAR_OFF);
     uint64_t* s_empty = s_full + ST;
     uint64_t* epi_full = s_empty + ST;    // the four consumer warps posted a unit's partial states
@@ -708,12 +709,12 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                 }
                 const float mn0 = fmaxf(m_run[0], t0), mn1 = fmaxf(m_run[1], t1);
                 const float mu0 = (mn0 == -INFINITY) ? 0.f : mn0, mu1 = (mn1 == -INFINITY) ? 0.f : mn1;
-                const float al0 = exp2f((m_run[0] - mu0) * kLog2e), al1 = exp2f((m_run[1] - mu1) * kLog2e);
+                const float al0 = ex2_fast((m_run[0] - mu0) * kLog2e), al1 = ex2_fast((m_run[1] - mu1) * kLog2e);
                 float pr[4];
-                pr[0] = exp2f((x[0] - mu0) * kLog2e);
-                pr[1] = exp2f((x[1] - mu1) * kLog2e);
-                pr[2] = exp2f((x[2] - mu0) * kLog2e);
-                pr[3] = exp2f((x[3] - mu1) * kLog2e);
+                pr[0] = ex2_fast((x[0] - mu0) * kLog2e);
+                pr[1] = ex2_fast((x[1] - mu1) * kLog2e);
+                pr[2] = ex2_fast((x[2] - mu0) * kLog2e);
+                pr[3] = ex2_fast((x[3] - mu1) * kLog2e);
                 l_run[0] = fmaf(l_run[0], al0, pr[0] + pr[2]);   // this lane's slots; summed over lanes at the end
                 l_run[1] = fmaf(l_run[1], al1, pr[1] + pr[3]);
                 m_run[0] = mn0;
@@ -760,17 +761,6 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                 l_run[0] += __shfl_xor_sync(kFull, l_run[0], o2);
                 l_run[1] += __shfl_xor_sync(kFull, l_run[1], o2);
             }
-            if (want_cand) {
-#pragma unroll
-                for (int o2 = 8; o2 >= 1; o2 >>= 1) {
-                    const unsigned long long k2 = __shfl_xor_sync(kFull, cand_key, o2);
-                    const int s2 = __shfl_xor_sync(kFull, cand_slot, o2);
-                    if (k2 < cand_key || (k2 == cand_key && s2 < cand_slot)) {
-                        cand_key = k2;
-                        cand_slot = s2;
-                    }
-                }
-            }
             // the buffer holds the previous unit until the epilogue warp has read it
             if (units_posted > 0 &&
                 !__all_sync(kFull, mbar_wait(epi_empty, (unsigned)(units_posted - 1) & 1u, p.wait_ns))) {
@@ -785,7 +775,7 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
             for (int jh = 0; jh < 2; ++jh) {
                 const int h = 2 * cq + jh;
                 if (h < G) {
-                    float* dst = s_o + (warp * G + h) * D + r;
+                    float* dst = s_o + (warp * G + h) * SH::EPI_LD + r;
 #pragma unroll
                     for (int j = 0; j < D / 16; ++j) {
                         dst[16 * j] = acc[j][jh];
@@ -797,9 +787,11 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                     }
                 }
             }
+            if (lane < 16) {   // each slot lane's best candidate; the epilogue warp reduces the 64
+                s_ck[warp * 16 + lane] = cand_key;
+                s_cs[warp * 16 + lane] = cand_slot;
+            }
             if (lane == 0) {
-                s_ck[warp] = cand_key;
-                s_cs[warp] = cand_slot;
                 if (warp == 0) {
                     s_epi[0] = ub;
                     s_epi[1] = ug;
@@ -882,7 +874,7 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
 #pragma unroll
                 for (int w = 0; w < NWC; ++w) {
                     const float f = __shfl_sync(kFull, fsh, w * G + hh);
-                    const float4 x = *reinterpret_cast<const float4*>(s_o + (w * G + hh) * D + e);
+                    const float4 x = *reinterpret_cast<const float4*>(s_o + (w * G + hh) * SH::EPI_LD + e);
                     out.x = fmaf(f, x.x, out.x);
                     out.y = fmaf(f, x.y, out.y);
                     out.z = fmaf(f, x.z, out.z);
@@ -902,19 +894,28 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                     }
                 }
             }
-            if (want_cand && lane == 0) {
-                unsigned long long bk = s_ck[0];
-                int bs = s_cs[0];
+            if (want_cand) {   // the best of the consumer lanes' 64 candidates (key, then slot)
+                unsigned long long bk = s_ck[lane];
+                int bs = s_cs[lane];
+                if (s_ck[lane + 32] < bk || (s_ck[lane + 32] == bk && s_cs[lane + 32] < bs)) {
+                    bk = s_ck[lane + 32];
+                    bs = s_cs[lane + 32];
+                }
 #pragma unroll
-                for (int w = 1; w < NWC; ++w)
-                    if (s_ck[w] < bk || (s_ck[w] == bk && s_cs[w] < bs)) {
-                        bk = s_ck[w];
-                        bs = s_cs[w];
+                for (int o2 = 16; o2 >= 1; o2 >>= 1) {
+                    const unsigned long long k2 = __shfl_xor_sync(kFull, bk, o2);
+                    const int s2 = __shfl_xor_sync(kFull, bs, o2);
+                    if (k2 < bk || (k2 == bk && s2 < bs)) {
+                        bk = k2;
+                        bs = s2;
                     }
-                EvictCand* c = p.cand + ((size_t)ub * p.Hkv + ug) * p.S + usplit;
-                c->key = bk;
-                c->slot = (bk == ~0ull) ? -1 : bs;
-                c->t = ut + 1;
+                }
+                if (lane == 0) {
+                    EvictCand* c = p.cand + ((size_t)ub * p.Hkv + ug) * p.S + usplit;
+                    c->key = bk;
+                    c->slot = (bk == ~0ull) ? -1 : bs;
+                    c->t = ut + 1;
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(epi_empty);
