@@ -21,20 +21,26 @@
 //    path, which set the pace of short units.
 //  - Four consumer warps each own 16 slots of a tile. Both products run on
 //    the tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate) with the
-//    G query heads as the M rows (padded to 16):
-//      S = Q . K^T       A = q rows (registers), B = K via ldmatrix
-//      O += P . V        A = P in the accumulator layout of S (no shuffles),
-//                        B = V via ldmatrix.trans; P is split into a bf16
-//                        high part and a bf16 residual, two mma each, which
-//                        keeps ~16 bits of P (a single bf16 P would cost
-//                        ~1e-3 relative error in o).
+//    G query heads in the N dimension (8 columns, heads >= G zero), so that
+//    the 16 slots fill the M rows:
+//      S^T = K . Q^T     A = K via ldmatrix, B = q columns (registers)
+//      O^T += V^T . P^T  A = V^T via ldmatrix.trans, B = P^T: the accumulator
+//                        of S^T with each 8x8 block transposed in registers
+//                        (movmatrix); P is split into a bf16 high part and a
+//                        bf16 residual, two mma each, which keeps ~16 bits of
+//                        P (a single bf16 P would cost ~1e-3 relative error
+//                        in o).
 //    Online softmax per warp and head (maxima in natural units, exp2 of
 //    scaled differences), O rescaled only when a maximum moved.
 //  - At the end of a unit each consumer warp posts its unscaled O, its
-//    (m, l) per row and its eviction candidate to shared memory (mbarrier
-//    epi_full) and goes on with the next unit; one epilogue warp combines the
-//    four states, writes the split's state and frees the buffer (epi_empty).
-//    The epilogue of one unit thus overlaps the next unit's tiles.
+//    (m, l) per head and its lanes' eviction candidates to shared memory
+//    (mbarrier epi_full) and goes on with the next unit; one epilogue warp
+//    combines the four states, reduces the candidates, writes the split's
+//    state and frees the buffer (epi_empty). The epilogue of one unit thus
+//    overlaps the next unit's tiles.
+//  - The fused decode step (INS): the producer also takes each row's victim
+//    from the previous step's records and the consumer warp owning the
+//    victim's slot swaps the new token into the staged tile and the cache.
 // Every wait is bounded (wait_ns, 1 s by default); on a timeout the CTA
 // records KVB_DERR_TIMEOUT, stops, drains the copies it issued (bounded) and
 // writes the empty state for every unit it owns.
