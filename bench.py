@@ -67,15 +67,15 @@ WORKLOADS = ("1", "2", "3", "3p", "4", "5", "5p")
 # unchanged since the counters were taken.
 MEASURED_TRAFFIC = {
     # the fused decode step (decode_attn_tc_kernel with the insertion) at the Qwen3-8B-shaped layer,
-    # one split: 545,752,576 read + 3,388,416 written
+    # one split: 545,725,440 read + 3,290,624 written
     # (bench.py --profile c2 under ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum)
-    ("bebded481a40d706", "2", 1): 549140992,
-    # the long-context fused step (136,461,824 + 5,333,248) and its 64-way merge (4,242,688 + 0)
+    ("da634b452e10e999", "2", 1): 549016064,
+    # the long-context fused step (136,462,848 + 4,453,632) and its 64-way merge (4,242,688 + 0)
     # (bench.py --profile c3, the same metrics over both launches)
-    ("bebded481a40d706", "3", 64): 146037760,
-    # the lookup over the prepared memory (102,807,552 + 3,361,792) and its merge (7,000,576 + 0)
+    ("da634b452e10e999", "3", 64): 145159168,
+    # the lookup over the prepared memory (102,808,320 + 3,240,192) and its merge (6,999,040 + 0)
     # (bench.py --profile c4, the same metrics over both launches)
-    ("efd6765f5e1aeb11", "4", 4): 113169920,
+    ("efd6765f5e1aeb11", "4", 4): 113047552,
 }
 
 
