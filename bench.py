@@ -667,8 +667,8 @@ class MementoBench:
     flush_l2 = True
     # the attention's fixed split length (a multiple of the 64-slot page). Measured on this
     # workload: 256 -> 115 us, 512 -> 90.5 us, 768 -> 86.1 us, 1024 -> 86.7 us, 1536 -> 92.9 us per
-    # step; 1280 -> 125 us, where the grid (287 CTAs) is 7 modulo the 14 splits per row, so each CTA
-    # sees only two split indices and the CTAs holding the first splits of the rows do most of the work
+    # step (1280: 125 us on a grid sharing a factor 7 with the 14 splits per row, 88.1 us since the
+    # library takes a grid coprime with the split count)
     SPLIT_LEN = 768
 
     def __init__(self, splits: int = 0, seed=None, paged: bool = False):
