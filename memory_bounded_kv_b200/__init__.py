@@ -177,23 +177,25 @@ def kvb_decode_step(q, k, v, log_beta, pos, len, t, o, lse, k_new, v_new, log_be
     """
     if cand_out is None or cand_in is None:
         raise ValueError("cand_in and cand_out are required")
-    a = _attn_args(q, k, v, log_beta, pos, len, t, o, lse, scale, num_splits, split_len, o_part, lse_part,
-                   cand_out)
+    if q.dim() != 3 or k.dim() != 4:
+        raise ValueError("q must be [B, Hq, d] and k, v [B, Hkv, cap, d]")
     B, Hkv, d = int(q.shape[0]), int(k.shape[1]), int(q.shape[2])
-    for name, x in (("k_new", k_new), ("v_new", v_new)):
-        _need(x, torch.bfloat16, name); _contig(x, name)
-        if tuple(x.shape) != (B, Hkv, d):
-            raise ValueError(f"{name} must be [B, Hkv, d]")
+    # shapes first (they need no device), then the attention's checks, then dtypes and devices
+    _shape(k_new, (B, Hkv, d), "k_new")
+    _shape(v_new, (B, Hkv, d), "v_new")
     if (log_beta is None) != (log_beta_new is None):
         raise ValueError("log_beta_new is needed exactly when log_beta is given")
+    _shape(log_beta_new, (B, Hkv), "log_beta_new")
+    if victim is not None and victim.numel() < B * Hkv:
+        raise ValueError("victim must hold B * Hkv entries")
+    a = _attn_args(q, k, v, log_beta, pos, len, t, o, lse, scale, num_splits, split_len, o_part, lse_part,
+                   cand_out)
+    for name, x in (("k_new", k_new), ("v_new", v_new)):
+        _need(x, torch.bfloat16, name); _contig(x, name)
     if log_beta_new is not None:
         _need(log_beta_new, torch.float32, "log_beta_new"); _contig(log_beta_new, "log_beta_new")
-        if tuple(log_beta_new.shape) != (B, Hkv):
-            raise ValueError("log_beta_new must be [B, Hkv]")
     if victim is not None:
         _need(victim, torch.int32, "victim"); _contig(victim, "victim")
-        if victim.numel() < B * Hkv:
-            raise ValueError("victim must hold B * Hkv entries")
     cin = _cand_ptr(cand_in, B * Hkv * int(num_splits))
     _check(_lib.lib().kvb_decode_step(ctypes.byref(a), k_new.data_ptr(), v_new.data_ptr(),
                                       None if log_beta_new is None else log_beta_new.data_ptr(), int(M), cin,

@@ -65,3 +65,33 @@ def test_evict_insert_and_compaction_check_shapes():
     with pytest.raises(ValueError, match="rm_len"):
         kvb.kvb_compact_blocks(a["k"], a["v"], a["pos"], None, a["len"], torch.zeros(B, dtype=torch.int32),
                                torch.zeros(B - 1, dtype=torch.int32))
+
+
+def test_decode_step_checks_the_new_rows_before_any_launch():
+    a = decode_args()
+    bf = torch.bfloat16
+    kn, vn = torch.zeros(B, Hkv, d, dtype=bf), torch.zeros(B, Hkv, d, dtype=bf)
+    lbn = torch.zeros(B, Hkv)
+    cand = torch.zeros(B * Hkv * 2, dtype=torch.int64)
+
+    def step(**over):
+        x = dict(k_new=kn, v_new=vn, log_beta_new=lbn, cand_in=cand, cand_out=cand, victim=None)
+        x.update(over)
+        kvb.kvb_decode_step(a["q"], a["k"], a["v"], a["log_beta"], a["pos"], a["len"], a["t"], a["o"], a["lse"],
+                            x["k_new"], x["v_new"], x["log_beta_new"], cap, x["cand_in"], x["cand_out"],
+                            victim=x["victim"])
+
+    with pytest.raises(TypeError, match="CUDA"):   # well shaped: the device check refuses
+        step()
+    with pytest.raises(ValueError, match="k_new"):
+        step(k_new=kn[:1])
+    with pytest.raises(ValueError, match="v_new"):
+        step(v_new=torch.zeros(B, Hkv, d - 8, dtype=bf))
+    with pytest.raises(ValueError, match="log_beta_new"):
+        step(log_beta_new=torch.zeros(B, Hkv + 1))
+    with pytest.raises(ValueError, match="log_beta_new"):   # a retention cache needs the new log beta
+        step(log_beta_new=None)
+    with pytest.raises(ValueError, match="victim"):
+        step(victim=torch.zeros(B * Hkv - 1, dtype=torch.int32))
+    with pytest.raises(ValueError, match="cand"):
+        step(cand_in=None)
