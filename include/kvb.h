@@ -60,7 +60,7 @@ enum kvb_device_error {
     KVB_DERR_RANGE = 1u << 2,     /* compaction range outside [0, len) */
     KVB_DERR_TIMEOUT = 1u << 3,   /* a bounded wait on a copy gave up */
     KVB_DERR_PAGES = 1u << 4,     /* a paged cache needed a page and its free stack was empty */
-    KVB_DERR_STEP = 1u << 5       /* kvb_decode_step: a row not full, or records not scored for t */
+    KVB_DERR_STEP = 1u << 5       /* kvb_decode_step: a row below its budget (len != M) */
 };
 
 /* ------------------------------------------------------------------------
@@ -189,11 +189,14 @@ kvb_status kvb_decode_attn(const kvb_attn_args* args, kvb_stream stream);
  *   (callers alternate two), 16-byte aligned.
  * - victim [B, Hkv] int32, may be NULL: the slot each row's new token took,
  *   -1 for an inactive row (t < 0).
- * - Rows with t < 0 are inactive (nothing inserted, empty state). A row that
- *   is not full (len != M), or whose records were not all scored for t[b], or
- *   name no slot, is not changed: it gets the empty state, victim -1, and the
- *   device error word KVB_DERR_STEP (use kvb_evict_insert + kvb_decode_attn
- *   for such a step). Needs pos and t; no batch stride 0 (kv or meta).
+ * - Rows with t < 0 are inactive (nothing inserted, empty state). When a row's
+ *   records were not all scored for t[b] (a skipped position) or name no
+ *   slot, the victim comes from a scan of the row's slots, as in
+ *   kvb_evict_insert (slower: every CTA reading the row scans it). A row that
+ *   is not full (len != M) is not changed: it gets the empty state, victim
+ *   -1, and the device error word KVB_DERR_STEP (use kvb_evict_insert +
+ *   kvb_decode_attn for such a step). Needs pos and t; no batch stride 0
+ *   (kv or meta).
  * ---------------------------------------------------------------------- */
 kvb_status kvb_decode_step(const kvb_attn_args* args, const uint16_t* k_new, const uint16_t* v_new,
                            const float* log_beta_new, int32_t M, const kvb_evict_cand* cand_in, int32_t* victim,

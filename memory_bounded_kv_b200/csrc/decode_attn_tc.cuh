@@ -296,8 +296,9 @@ __device__ __forceinline__ RowRecords load_row_records(const DecodeTcParams& p, 
 }
 
 // Warp-collective (every lane of the producer warp). Returns -1 for an inactive row (t < 0:
-// nothing is inserted) and -2 for a row the fused step cannot update: not full (len != M), or a
-// record scored for another position, or no record naming a slot.
+// nothing is inserted), -2 for a row the fused step cannot update (not full: len != M) and -3
+// when the records cannot name the victim (one scored for another position, or none naming a
+// slot): then row_scan_victim finds it.
 __device__ __forceinline__ int row_victim(const DecodeTcParams& p, const RowRecords& x, int b, int g, int tb, int n,
                                           int lane) {
     unsigned long long best = ~0ull;
@@ -324,7 +325,47 @@ __device__ __forceinline__ int row_victim(const DecodeTcParams& p, const RowReco
     }
     stale = __any_sync(kFull, stale);
     if (tb < 0) return -1;
-    if (n != p.M || stale || best == ~0ull || best_slot >= n) return -2;
+    if (n != p.M) return -2;
+    if (stale || best == ~0ull || best_slot >= n) return -3;
+    return best_slot;
+}
+
+// The victim of a full row from its slots, as kvb_evict_insert's scan: the smallest key
+// (order key of the score (t - pos) log beta, one float32 product) << 32 | the order key of pos.
+// Warp-collective; every unit of the row repeats it, which only happens when the records were not
+// left for this position.
+__device__ __noinline__ int row_scan_victim(const DecodeTcParams& p, int b, int g, int tb, int n, int lane) {
+    const size_t base = (size_t)b * p.m_sb + (size_t)g * p.m_sh;
+    const int* ps = p.pos + base;
+    const float* lb = p.lb != nullptr ? p.lb + base : nullptr;
+    unsigned long long best = ~0ull;
+    int best_slot = 0x7fffffff;
+    for (int s0 = lane; s0 < n; s0 += 32 * 4) {
+        int pv[4];
+        float lv[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {   // four independent loads of each kind in flight
+            const int s = s0 + 32 * k;
+            pv[k] = s < n ? ps[s] : 0;
+            lv[k] = (lb != nullptr && s < n) ? lb[s] : 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int s = s0 + 32 * k;
+            if (s < n) {
+                const float sc = lb != nullptr ? __fmul_rn(__int2float_rn(tb - pv[k]), lv[k]) : 0.f;
+                const unsigned long long key =
+                    ((unsigned long long)float_order_key(sc) << 32) | (unsigned)(pv[k] ^ 0x80000000);
+                argmin_merge(best, best_slot, key, s);
+            }
+        }
+    }
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) {
+        const unsigned long long k2 = __shfl_xor_sync(kFull, best, m);
+        const int s2 = __shfl_xor_sync(kFull, best_slot, m);
+        argmin_merge(best, best_slot, k2, s2);
+    }
     return best_slot;
 }
 
@@ -407,6 +448,7 @@ __global__ void __launch_bounds__(TcShape<D, G>::NT, 2)
                 next_rec = load_row_records(p, end ? p.units : u + u_step, lane);
                 if (!end) {
                     victim = row_victim(p, cur, ui.b, ui.g, raw.t, raw.len, lane);
+                    if (victim == -3) victim = row_scan_victim(p, ui.b, ui.g, raw.t, raw.len, lane);
                     if (ui.split == 0 && lane == 0) {
                         if (victim == -2) raise_error(KVB_DERR_STEP);
                         if (p.victim != nullptr) p.victim[ui.b * p.Hkv + ui.g] = max(victim, -1);

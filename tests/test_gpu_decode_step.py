@@ -1,7 +1,8 @@
 """GPU parity of kvb_decode_step (budget enforcement, insertion and attention in one launch)
 against the oracle's evict_insert followed by decode_attn: victims, lengths and every cached byte
-exact after each step, outputs and split states within the stated tolerances; plus the rows the
-fused step refuses (not full, records scored for another position) and inactive rows."""
+exact after each step, outputs and split states within the stated tolerances; plus records
+scored for another position (the victim then comes from a scan), rows the fused step refuses (not
+full) and inactive rows."""
 import numpy as np
 import pytest
 import torch
@@ -80,10 +81,11 @@ def test_decode_step_matches_evict_insert_then_attention(oracle, d, G, S, with_b
     assert kvb.kvb_get_error() == 0
 
 
-def test_decode_step_refuses_rows_it_cannot_update(oracle):
-    """A row below its budget, and records scored for another position, leave the row unchanged
-    with the empty state and KVB_DERR_STEP; an inactive row (t < 0) is empty and unchanged
-    without an error; the other rows step exactly as evict_insert + decode_attn."""
+def test_decode_step_stale_records_scan_and_rows_below_budget_are_refused(oracle):
+    """Records scored for another position (a skipped position) make the step find the victim by
+    scanning the row's slots, as kvb_evict_insert does; a row below its budget is left unchanged
+    with the empty state and KVB_DERR_STEP; an inactive row (t < 0) is empty and unchanged without
+    an error. Every other row steps exactly as evict_insert + decode_attn."""
     B, Hkv, G, d, cap, M, S = 4, 2, 4, 128, 256, 256, 4
     Hq = Hkv * G
     g = rng(92, 0)
@@ -110,21 +112,20 @@ def test_decode_step_refuses_rows_it_cannot_update(oracle):
     kvb.kvb_decode_step(dev(q), gc.k, gc.v, gc.log_beta, gc.pos, gc.len, dev(t), o, lse, dev(kn), dev(vn),
                         dev(lbn), M, cand[0], cand[1], victim=victim, num_splits=S, o_part=op, lse_part=lp)
     bits = kvb.kvb_get_error()
-    assert bits & _lib.DERR_STEP, bits
+    assert bits == _lib.DERR_STEP, bits
     after = gc.to_host()
     vic = host(victim)
     lse_h, o_h = host(lse), host(o)
-    refused = [(1, 0), (1, 1), (2, 1)]
-    for b, h in refused + [(3, 0), (3, 1)]:
+    for b, h in [(2, 1), (3, 0), (3, 1)]:   # below the budget; inactive
         assert vic[b, h] == -1, (b, h)
         for key in ("k", "v", "pos", "log_beta"):
             np.testing.assert_array_equal(after[key][b, h], before[key][b, h], err_msg=f"{key} {b} {h}")
         assert np.all(lse_h[b, h * G:(h + 1) * G] == -np.inf) and not o_h[b, h * G:(h + 1) * G].any()
-    # the rows that stepped: sequence 0 (both heads) and sequence 2, head 0
+    # the rows that stepped, sequence 1 through the scan
     ref = {key: (None if val is None else val.copy()) for key, val in c.items()}
-    vic_ref = oracle.evict_insert(ref, kn, vn, lbn, np.where(t < 0, -1, t).astype(np.int32), M)
+    vic_ref = oracle.evict_insert(ref, kn, vn, lbn, t, M)
     o_ref, l_ref = oracle.decode_attn(q, ref["k"], ref["v"], ref["log_beta"], ref["pos"], ref["len"], t)
-    for b, h in [(0, 0), (0, 1), (2, 0)]:
+    for b, h in [(0, 0), (0, 1), (1, 0), (1, 1), (2, 0)]:
         assert vic[b, h] == vic_ref[b, h], (b, h)
         for key in ("k", "v", "pos", "log_beta"):
             np.testing.assert_array_equal(after[key][b, h], ref[key][b, h], err_msg=f"{key} {b} {h}")
