@@ -67,12 +67,12 @@ WORKLOADS = ("1", "2", "3", "3p", "4", "5", "5p")
 # unchanged since the counters were taken.
 MEASURED_TRAFFIC = {
     # the fused decode step (decode_attn_tc_kernel with the insertion) at the Qwen3-8B-shaped layer,
-    # one split: 545,725,440 read + 3,290,624 written
+    # one split: 545,730,816 read + 3,399,424 written
     # (bench.py --profile c2 under ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum)
-    ("da634b452e10e999", "2", 1): 549016064,
-    # the long-context fused step (136,462,848 + 4,453,632) and its 64-way merge (4,242,688 + 0)
+    ("2a67484ce58e6b51", "2", 1): 549130240,
+    # the long-context fused step (136,465,408 + 3,846,144) and its 64-way merge (4,247,552 + 0)
     # (bench.py --profile c3, the same metrics over both launches)
-    ("da634b452e10e999", "3", 64): 145159168,
+    ("2a67484ce58e6b51", "3", 64): 144559104,
     # the lookup over the prepared memory (102,808,320 + 3,240,192) and its merge (6,999,040 + 0)
     # (bench.py --profile c4, the same metrics over both launches)
     ("efd6765f5e1aeb11", "4", 4): 113047552,
