@@ -23,7 +23,7 @@ def _nvcc() -> str:
 
 def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh")) +
-                  [os.path.join(ROOT, "include", "kvb.h")])
+                  glob.glob(os.path.join(CSRC, "*.h")) + [os.path.join(ROOT, "include", "kvb.h")])
 
 
 def stale() -> bool:

@@ -12,6 +12,7 @@
 #include <utility>
 
 #include "../../include/kvb.h"
+#include "schedule.h"
 #include "asm_lookup.cuh"
 #include "asm_planes.cuh"
 #include "asm_hier.cuh"
@@ -134,24 +135,6 @@ int resident_ctas(Kern kern, int threads, size_t smem) {
     return n;
 }
 
-// Grid of the round-robin attention (CTA c takes units c, c + grid, ...): as many CTAs as keep every
-// CTA's unit count equal to the busiest one's (the makespan in units is unchanged and no CTA idles
-// while the others finish). With fixed-length splits a row's first splits hold its slots and its
-// last ones are empty, and CTA c meets only the split indices congruent to c modulo gcd(grid, S):
-// then the grid is lowered to the nearest count coprime with S, if that adds at most one unit to
-// the busiest CTA's count and it had at least four (measured on the memento workload: splits of
-// 1280 slots, 14 per row, on 287 CTAs, 7 modulo 14, took 125 us per step against 86 us at 768).
-int rr_grid(int units, int slots, int S, bool fixed_splits) {
-    const int per_cta = (units + slots - 1) / slots;
-    const int grid = (units + per_cta - 1) / per_cta;
-    if (!fixed_splits || S < 2 || per_cta < 4 || std::gcd(grid, S) == 1) return grid;
-    for (int g = grid - 1; g > 0; --g) {
-        if ((units + g - 1) / g > per_cta + 1) break;
-        if (std::gcd(g, S) == 1) return g;
-    }
-    return grid;
-}
-
 // Launch with programmatic stream serialization: the kernel may start while the
 // previous kernel in the stream drains; its first instruction waits for that
 // kernel's completion (griddepcontrol.wait), so only the launch latency overlaps.
@@ -196,7 +179,7 @@ kvb_status launch_decode_tc(const kvb::DecodeTcParams& p, const kvb_attn_args* a
         return KVB_EINVAL;
     const int slots = resident_ctas(kern, SH::NT, smem);
     if (slots <= 0) return KVB_ECUDA;
-    const int grid = rr_grid(p.units, slots, p.S, p.split_len > 0);
+    const int grid = kvb::rr_grid(p.units, slots, p.S, p.split_len > 0);
     if (launch_pdl(kern, dim3(grid), dim3(SH::NT), smem, st, p, mk, mv) != KVB_OK) return KVB_ECUDA;
     if (p.S > 1)
         return launch_merge<D>(p.o_part, p.lse_part, a->B * a->Hq, p.S, p.o, p.o_bf16, p.lse, st);
@@ -286,7 +269,7 @@ kvb_status launch_decode_paged(const kvb::DecodeTcParams& p, const kvb_paged_cac
         return KVB_EINVAL;
     const int slots = resident_ctas(kern, SH::NT, smem);
     if (slots <= 0) return KVB_ECUDA;
-    const int grid = rr_grid(p.units, slots, p.S, p.split_len > 0);
+    const int grid = kvb::rr_grid(p.units, slots, p.S, p.split_len > 0);
     if (launch_pdl(kern, dim3(grid), dim3(SH::NT), smem, st, p, mk, mv) != KVB_OK) return KVB_ECUDA;
     if (p.S > 1) return launch_merge<D>(p.o_part, p.lse_part, c->B * Hq, p.S, p.o, p.o_bf16, p.lse, st);
     return KVB_OK;
